@@ -1,0 +1,169 @@
+"""Byte layout of one 128-token KV page -- CPU oracle (test infrastructure only).
+
+A page holds the K (or V) rows of 128 consecutive tokens of one (layer, KV head)
+(KVMem reproduction, lcz.me/topic/1972, test command: 128-token blocks).  The
+pages fix only the bits per element; the arrangement below is this library's own
+storage spec, written so that one 16-byte load per thread feeds tensor-core
+fragments directly.  Bytes per page equal the AoS block sizes the pages print:
+K Q8_0 = 128 x 8 x 34 = 34,816; V Q4_0 = 128 x 8 x 18 = 18,432; V Q8_0 = 34,816.
+
+Notation: tok in [0,128) is the token slot inside the page, dim in [0,256) the
+channel, b = dim // 32 the block, d[tok][b] the fp16 block scale.  Tokens are
+grouped in sixteens: G = tok // 16.
+
+K page, Q8_0 (34,816 bytes)
+  codes, bytes [0, 32768): byte at
+      ((((G*4 + P)*2 + H)*8 + R)*4 + T)*16 + j          (P<4, H<2, R<8, T<4, j<16)
+  holds the int8 code of token 16G + 8H + R, channel 64P + 32*(j // 8) + 8T + (j % 8).
+  scales, bytes [32768, 34816): fp16 at 32768 + 2*((((G*8 + R)*2 + H)*8) + b)
+  holds d[16G + 8H + R][b].
+
+V page, Q4_0 (18,432 bytes)
+  nibbles, bytes [0, 16384): byte at
+      ((((G*4 + C)*8 + R)*4 + T)*16 + 4*w + y            (C<4, R<8, T<4, w<4, y<4)
+  belongs to block b = 2C + w // 2 and token 16G + 2T + 8*(w % 2) + y // 2; its
+  low nibble is channel 32b + 16*(y % 2) + R and its high nibble that channel + 8.
+  A nibble stores q in [0, 15]; the value is (q - 8) * d.
+  scales, bytes [16384, 18432): fp16 at 16384 + 2*((((G*4 + T)*8 + b)*4) + k)
+  holds d[16G + 2T + (k % 2) + 8*(k // 2)][b]                (k < 4).
+
+V page, Q8_0 (34,816 bytes)
+  codes, bytes [0, 32768): byte at
+      ((((G*8 + b)*8 + R)*4 + T)*16 + 4*w + y            (b<8, R<8, T<4, w<4, y<4)
+  holds the int8 code of token 16G + 2T + 8*(w % 2) + y % 2, channel
+  32b + 16*(w // 2) + 8*(y // 2) + R.
+  scales, bytes [32768, 34816): same arrangement as the Q4_0 V scales.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+PAGE_TOKENS = 128
+HEAD_DIM = 256
+N_BLOCKS = HEAD_DIM // 32
+
+K_Q8_BYTES = 34816
+V_Q4_BYTES = 18432
+V_Q8_BYTES = 34816
+
+
+def page_bytes(role: str, fmt: str) -> int:
+    if role == "k" and fmt == "q8_0":
+        return K_Q8_BYTES
+    if role == "v" and fmt == "q4_0":
+        return V_Q4_BYTES
+    if role == "v" and fmt == "q8_0":
+        return V_Q8_BYTES
+    raise ValueError(f"unsupported page kind {role}/{fmt}")
+
+
+def _k_code_map():
+    G, P, H, R, T, j = np.meshgrid(np.arange(8), np.arange(4), np.arange(2), np.arange(8),
+                                   np.arange(4), np.arange(16), indexing="ij")
+    off = ((((G * 4 + P) * 2 + H) * 8 + R) * 4 + T) * 16 + j
+    tok = 16 * G + 8 * H + R
+    dim = 64 * P + 32 * (j // 8) + 8 * T + (j % 8)
+    return off.ravel(), tok.ravel(), dim.ravel()
+
+
+def _k_scale_map():
+    G, R, H, b = np.meshgrid(np.arange(8), np.arange(8), np.arange(2), np.arange(8), indexing="ij")
+    idx = ((G * 8 + R) * 2 + H) * 8 + b
+    return idx.ravel(), (16 * G + 8 * H + R).ravel(), b.ravel()
+
+
+def _v_scale_map():
+    G, T, b, k = np.meshgrid(np.arange(8), np.arange(4), np.arange(8), np.arange(4), indexing="ij")
+    idx = ((G * 4 + T) * 8 + b) * 4 + k
+    tok = 16 * G + 2 * T + (k % 2) + 8 * (k // 2)
+    return idx.ravel(), tok.ravel(), b.ravel()
+
+
+def _v4_nibble_map():
+    G, C, R, T, w, y = np.meshgrid(np.arange(8), np.arange(4), np.arange(8), np.arange(4),
+                                   np.arange(4), np.arange(4), indexing="ij")
+    off = ((((G * 4 + C) * 8 + R) * 4 + T) * 16) + 4 * w + y
+    b = 2 * C + w // 2
+    tok = 16 * G + 2 * T + 8 * (w % 2) + y // 2
+    lo = 32 * b + 16 * (y % 2) + R
+    return off.ravel(), tok.ravel(), lo.ravel(), (lo + 8).ravel()
+
+
+def _v8_code_map():
+    G, b, R, T, w, y = np.meshgrid(np.arange(8), np.arange(8), np.arange(8), np.arange(4),
+                                   np.arange(4), np.arange(4), indexing="ij")
+    off = ((((G * 8 + b) * 8 + R) * 4 + T) * 16) + 4 * w + y
+    tok = 16 * G + 2 * T + 8 * (w % 2) + y % 2
+    dim = 32 * b + 16 * (w // 2) + 8 * (y // 2) + R
+    return off.ravel(), tok.ravel(), dim.ravel()
+
+
+_K_CODES = _k_code_map()
+_K_SCALES = _k_scale_map()
+_V_SCALES = _v_scale_map()
+_V4_NIBBLES = _v4_nibble_map()
+_V8_CODES = _v8_code_map()
+
+
+def _flat_codes(codes: np.ndarray) -> np.ndarray:
+    """[128][8][32] block codes -> [128][256] channel codes."""
+    return np.asarray(codes).reshape(PAGE_TOKENS, HEAD_DIM)
+
+
+def encode_page(role: str, fmt: str, codes: np.ndarray, d: np.ndarray) -> np.ndarray:
+    """Encode one page.  codes: [128][8][32] (int8 for Q8_0, 0..15 for Q4_0);
+    d: [128][8] float16.  Returns uint8[page_bytes]."""
+    n = page_bytes(role, fmt)
+    out = np.zeros(n, dtype=np.uint8)
+    c = _flat_codes(codes)
+    d16 = np.asarray(d, dtype=np.float16).view(np.uint16)
+    if role == "k":
+        off, tok, dim = _K_CODES
+        out[off] = c[tok, dim].astype(np.int8).view(np.uint8)
+        idx, tok, b = _K_SCALES
+        scale_base = 32768
+    elif fmt == "q4_0":
+        off, tok, lo, hi = _V4_NIBBLES
+        c8 = c.astype(np.uint8)
+        if np.any(c8 > 15):
+            raise ValueError("Q4_0 codes must be in [0, 15]")
+        out[off] = c8[tok, lo] | (c8[tok, hi] << 4)
+        idx, tok, b = _V_SCALES
+        scale_base = 16384
+    else:
+        off, tok, dim = _V8_CODES
+        out[off] = c[tok, dim].astype(np.int8).view(np.uint8)
+        idx, tok, b = _V_SCALES
+        scale_base = 32768
+    sv = d16[tok, b]
+    out[scale_base + 2 * idx] = (sv & 0xFF).astype(np.uint8)
+    out[scale_base + 2 * idx + 1] = (sv >> 8).astype(np.uint8)
+    return out
+
+
+def decode_page(role: str, fmt: str, page: np.ndarray):
+    """Inverse of encode_page: uint8[page_bytes] -> (codes [128][8][32], d [128][8] f16)."""
+    page = np.asarray(page, dtype=np.uint8)
+    if page.size != page_bytes(role, fmt):
+        raise ValueError("wrong page size")
+    c = np.zeros((PAGE_TOKENS, HEAD_DIM), dtype=np.int16)
+    if role == "k":
+        off, tok, dim = _K_CODES
+        c[tok, dim] = page[off].view(np.int8)
+        idx, tok, b = _K_SCALES
+        scale_base = 32768
+    elif fmt == "q4_0":
+        off, tok, lo, hi = _V4_NIBBLES
+        c[tok, lo] = page[off] & 0xF
+        c[tok, hi] = page[off] >> 4
+        idx, tok, b = _V_SCALES
+        scale_base = 16384
+    else:
+        off, tok, dim = _V8_CODES
+        c[tok, dim] = page[off].view(np.int8)
+        idx, tok, b = _V_SCALES
+        scale_base = 32768
+    d16 = np.zeros((PAGE_TOKENS, N_BLOCKS), dtype=np.uint16)
+    d16[tok, b] = page[scale_base + 2 * idx].astype(np.uint16) | (page[scale_base + 2 * idx + 1].astype(np.uint16) << 8)
+    dt = np.int8 if fmt == "q8_0" else np.uint8
+    return c.astype(dt).reshape(PAGE_TOKENS, N_BLOCKS, 32), d16.view(np.float16)

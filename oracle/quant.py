@@ -1,0 +1,99 @@
+"""Q8_0 and Q4_0 block quantisation -- CPU oracle (test infrastructure only).
+
+Both formats split a row into blocks of 32 elements and store one fp16 scale
+``d`` per block (Vulkan speculative-decoding report, lcz.me/topic/1398, section
+"pitfalls": legacy block quants only; q8_0 = 8.5 bits per element, i.e. 32 int8 +
+fp16 = 34 bytes per block; q4_0 K+V = 18 KiB per token, i.e. 16 bytes of nibbles
++ fp16 = 18 bytes per block).
+
+The pages do not spell out the encoders.  The readings used here:
+
+* Q8_0: ``d = amax / 127`` in fp32, ``q = round_half_away(x * (1/d))`` with the
+  reciprocal and the product each rounded to fp32, clamped to [-127, 127]; the
+  stored scale is fp16(d) (round to nearest even).  ``amax == 0`` gives d = 0 and
+  q = 0.  Value = q * d_fp16.
+* Q4_0: value = (q - 8) * d with q in [0, 15].  ``m`` = the signed element of
+  largest magnitude (first one on ties), ``d = m / -8`` in fp32, ``q =
+  min(15, floor(x * (1/d) + 8.5))`` with the product and the sum each rounded to
+  fp32; the element m maps to q = 0.  ``m == 0`` gives d = 0 and q = 8.
+
+Every rounding that decides an integer code is done in fp32, exactly as an IEEE
+fp32 unit would do it, so a GPU encoder can match the codes bit for bit.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+QK = 32  # elements per block
+
+F32 = np.float32
+
+
+def _blocks(x: np.ndarray) -> np.ndarray:
+    x = np.asarray(x, dtype=F32)
+    if x.shape[-1] % QK:
+        raise ValueError("last axis must be a multiple of 32")
+    return x.reshape(x.shape[:-1] + (x.shape[-1] // QK, QK))
+
+
+def _recip_f32(d: np.ndarray) -> np.ndarray:
+    """1/d rounded to fp32, and 0 where d == 0."""
+    out = np.zeros_like(d, dtype=F32)
+    nz = d != 0
+    out[nz] = F32(1.0) / d[nz]
+    return out
+
+
+def round_half_away(y: np.ndarray) -> np.ndarray:
+    """Round fp32 values to the nearest integer, halves away from zero (exact)."""
+    y64 = np.asarray(y, dtype=np.float64)  # exact widening
+    return np.sign(y64) * np.floor(np.abs(y64) + 0.5)
+
+
+def q8_0_quantize(x: np.ndarray):
+    """x: fp32 [..., 32n] -> (qs int8 [..., n, 32], d float16 [..., n])."""
+    xb = _blocks(x)
+    amax = np.max(np.abs(xb), axis=-1)
+    d32 = (amax / F32(127.0)).astype(F32)
+    inv = _recip_f32(d32)
+    y = (xb * inv[..., None]).astype(F32)
+    q = np.clip(round_half_away(y), -127, 127)
+    return q.astype(np.int8), d32.astype(np.float16)
+
+
+def q8_0_dequantize(qs: np.ndarray, d: np.ndarray) -> np.ndarray:
+    """(qs [..., n, 32], d [..., n]) -> float64 [..., 32n], value = q * d."""
+    v = qs.astype(np.float64) * d.astype(np.float64)[..., None]
+    return v.reshape(v.shape[:-2] + (-1,))
+
+
+def q4_0_quantize(x: np.ndarray):
+    """x: fp32 [..., 32n] -> (q uint8 in [0,15] [..., n, 32], d float16 [..., n])."""
+    xb = _blocks(x)
+    idx = np.argmax(np.abs(xb), axis=-1)
+    m = np.take_along_axis(xb, idx[..., None], axis=-1)[..., 0]
+    d32 = (m / F32(-8.0)).astype(F32)
+    inv = _recip_f32(d32)
+    y = (xb * inv[..., None]).astype(F32)
+    z = (y + F32(8.5)).astype(F32)
+    q = np.minimum(15, np.floor(z.astype(np.float64)))
+    return q.astype(np.uint8), d32.astype(np.float16)
+
+
+def q4_0_dequantize(q: np.ndarray, d: np.ndarray) -> np.ndarray:
+    """(q [..., n, 32], d [..., n]) -> float64 [..., 32n], value = (q - 8) * d."""
+    v = (q.astype(np.float64) - 8.0) * d.astype(np.float64)[..., None]
+    return v.reshape(v.shape[:-2] + (-1,))
+
+
+def quantize(x: np.ndarray, fmt: str):
+    return {"q8_0": q8_0_quantize, "q4_0": q4_0_quantize}[fmt](x)
+
+
+def dequantize(codes: np.ndarray, d: np.ndarray, fmt: str) -> np.ndarray:
+    return {"q8_0": q8_0_dequantize, "q4_0": q4_0_dequantize}[fmt](codes, d)
+
+
+def block_bytes(fmt: str) -> int:
+    """Bytes of one 32-element block: fp16 scale + codes."""
+    return {"q8_0": 2 + 32, "q4_0": 2 + 16}[fmt]

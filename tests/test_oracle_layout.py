@@ -1,0 +1,85 @@
+"""Pins for the oracle's page byte layout (CPU only).
+
+The layout is this library's own storage spec; the pins are its size (equal to
+the pages' block sizes), that encoding is a bijection, and spot values of the
+documented offset formulas.
+"""
+import numpy as np
+import pytest
+
+from oracle import layout, quant
+from synth import normal_f32, np_rng
+
+
+def _page(fmt, seed):
+    x = normal_f32(np_rng(seed), (128, 256))
+    return quant.quantize(x, fmt)
+
+
+@pytest.mark.parametrize("role,fmt", [("k", "q8_0"), ("v", "q4_0"), ("v", "q8_0")])
+def test_round_trip(role, fmt):
+    codes, d = _page(fmt, 11)
+    page = layout.encode_page(role, fmt, codes, d)
+    assert page.size == layout.page_bytes(role, fmt) == 128 * 8 * quant.block_bytes(fmt)
+    c2, d2 = layout.decode_page(role, fmt, page)
+    assert np.array_equal(c2, codes) and np.array_equal(d2.view(np.uint16), d.view(np.uint16))
+
+
+def _one_hot(fmt, tok, dim, code):
+    codes = np.zeros((128, 8, 32), dtype=np.int8 if fmt == "q8_0" else np.uint8)
+    if fmt == "q4_0":
+        codes[:] = 0
+    codes[tok, dim // 32, dim % 32] = code
+    return codes, np.zeros((128, 8), np.float16)
+
+
+@pytest.mark.parametrize("tok,dim,off", [
+    (0, 0, 0), (1, 0, 64), (8, 0, 512), (0, 8, 16), (0, 32, 8), (0, 64, 1024),
+    (16, 0, 4096), (5, 200, 3 * 1024 + 5 * 64 + 1 * 16),
+])
+def test_k_code_offsets(tok, dim, off):
+    codes, d = _one_hot("q8_0", tok, dim, 7)
+    page = layout.encode_page("k", "q8_0", codes, d)
+    assert np.flatnonzero(page).tolist() == [off]
+
+
+def test_k_scale_offsets():
+    codes = np.zeros((128, 8, 32), np.int8)
+    d = np.zeros((128, 8), np.float16)
+    d[9, 3] = 1.0          # G=0, R=1, H=1, b=3 -> index ((0*8+1)*2+1)*8+3 = 27
+    page = layout.encode_page("k", "q8_0", codes, d)
+    nz = np.flatnonzero(page)
+    assert nz.tolist() == [32768 + 2 * 27 + 1]     # 1.0 = 0x3C00: only the high byte is set
+
+
+@pytest.mark.parametrize("tok,dim,off,shift", [
+    (0, 0, 0, 0), (0, 8, 0, 4), (0, 16, 1, 0), (0, 24, 1, 4), (1, 0, 2, 0),
+    (8, 0, 4, 0), (2, 0, 16, 0), (0, 1, 64, 0), (0, 32, 8, 0), (0, 64, 512, 0), (16, 0, 2048, 0),
+])
+def test_v_q4_nibble_offsets(tok, dim, off, shift):
+    codes = np.zeros((128, 8, 32), np.uint8)
+    codes[tok, dim // 32, dim % 32] = 5
+    page = layout.encode_page("v", "q4_0", codes, np.zeros((128, 8), np.float16))
+    assert np.flatnonzero(page).tolist() == [off]
+    assert page[off] == 5 << shift
+
+
+@pytest.mark.parametrize("tok,dim,off", [
+    (0, 0, 0), (1, 0, 1), (0, 8, 2), (8, 0, 4), (0, 16, 8), (2, 0, 16), (0, 1, 64), (0, 32, 512),
+    (16, 0, 4096),
+])
+def test_v_q8_code_offsets(tok, dim, off):
+    codes, d = _one_hot("q8_0", tok, dim, 9)
+    page = layout.encode_page("v", "q8_0", codes, d)
+    assert np.flatnonzero(page).tolist() == [off]
+
+
+def test_v_scale_offsets():
+    d = np.zeros((128, 8), np.float16)
+    d[10, 2] = 1.0        # tok 10 = 2T + k%2 + 8*(k//2) with T=1, k=2 -> index ((0*4+1)*8+2)*4+2 = 42
+    for fmt, base in (("q4_0", 16384), ("q8_0", 32768)):
+        codes = np.zeros((128, 8, 32), np.int8 if fmt == "q8_0" else np.uint8)
+        if fmt == "q4_0":
+            codes[:] = 0
+        page = layout.encode_page("v", fmt, codes, d)
+        assert np.flatnonzero(page).tolist() == [base + 2 * 42 + 1]

@@ -1,0 +1,132 @@
+"""Pins for the oracle's Q8_0 / Q4_0 quantisers (CPU only).
+
+Closed-form error bounds, exact round trips of representable blocks, the
+rounding rule at exact halves, the zero block and the scale's fp16 rounding.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import quant
+from synth import normal_f32, np_rng
+
+
+def _x(seed, n_blocks=64, outliers=False):
+    x = normal_f32(np_rng(seed), (n_blocks * 32,))
+    if outliers:
+        x[::37] *= 8.0
+    return x
+
+
+@pytest.mark.parametrize("outliers", [False, True])
+def test_q8_0_error_bound(outliers):
+    x = _x(1, 256, outliers).reshape(-1, 32)
+    qs, d = quant.q8_0_quantize(x)
+    xh = quant.q8_0_dequantize(qs, d).reshape(-1, 32)
+    d32 = (np.max(np.abs(x), axis=1) / np.float32(127)).astype(np.float32).astype(np.float64)
+    d16 = d.astype(np.float64).reshape(-1)
+    bound = d32 * (0.5 + 2.0 ** -16) + 127 * np.abs(d32 - d16)
+    assert np.all(np.abs(x - xh) <= bound[:, None] + 1e-300)
+
+
+def test_q8_0_codes_are_nearest_away_from_zero():
+    x = _x(2, 128).reshape(-1, 32)
+    qs = quant.q8_0_quantize(x)[0].reshape(-1, 32)
+    d32 = (np.max(np.abs(x), axis=1) / np.float32(127)).astype(np.float32)
+    for i in range(x.shape[0]):
+        for j in range(32):
+            exact = Fraction(float(x[i, j])) / Fraction(float(d32[i]))
+            k = int(np.floor(abs(exact) + Fraction(1, 2))) * (1 if exact >= 0 else -1)
+            if abs(abs(exact - int(exact)) - Fraction(1, 2)) > Fraction(1, 10 ** 4):
+                assert qs[i, j] == k
+
+
+def test_q8_0_halves_round_away_from_zero():
+    # amax = 15.875 -> d = 0.125 exactly, 1/d = 8 exactly, so x*8 hits exact halves.
+    x = np.zeros(32, np.float32)
+    x[0] = 15.875
+    x[1:5] = [0.0625, 0.3125, -0.3125, -0.0625]   # 0.5, 2.5, -2.5, -0.5
+    qs, d = quant.q8_0_quantize(x)
+    assert float(d[0]) == 0.125
+    assert list(qs[0, :5]) == [127, 1, 3, -3, -1]
+
+
+def test_q8_0_round_trip_of_representable_block():
+    rng = np_rng(3)
+    q = rng.integers(-127, 128, size=(16, 32)).astype(np.int8)
+    q[:, 5] = 127
+    d = np.float16(2.0 ** -4)
+    x = (q.astype(np.float32) * np.float32(d))
+    qs, dd = quant.q8_0_quantize(x)
+    assert np.array_equal(qs.reshape(q.shape), q) and np.all(dd == d)
+
+
+def test_q8_0_zero_block_and_extremes():
+    x = np.zeros(64, np.float32)
+    x[40] = -3.0
+    qs, d = quant.q8_0_quantize(x)
+    assert d[0] == 0 and np.all(qs[0] == 0)
+    assert qs[1, 8] == -127
+
+
+def test_scale_rounds_to_nearest_even_fp16():
+    # d = amax/127 = 1 + 2^-11 exactly: halfway between fp16 1.0 and 1.0 + 2^-10.
+    x = np.zeros(32, np.float32)
+    x[0] = np.float32(127.06201171875)
+    _, d = quant.q8_0_quantize(x)
+    assert float(d[0]) == 1.0
+
+
+@pytest.mark.parametrize("outliers", [False, True])
+def test_q4_0_error_bound(outliers):
+    x = _x(4, 256, outliers).reshape(-1, 32)
+    q, d = quant.q4_0_quantize(x)
+    assert q.max() <= 15
+    xh = quant.q4_0_dequantize(q, d).reshape(-1, 32)
+    idx = np.argmax(np.abs(x), axis=1)
+    m = x[np.arange(x.shape[0]), idx].astype(np.float64)
+    d32 = np.abs(m) / 8.0
+    d16 = np.abs(d.astype(np.float64).reshape(-1))
+    y = x / (-m[:, None] / 8.0)
+    clamped = y >= 7.5 - 1e-6
+    tol = np.where(clamped, 1.0, 0.5) + 2.0 ** -18
+    bound = d32[:, None] * tol + 8 * np.abs(d32 - d16)[:, None]
+    assert np.all(np.abs(x - xh) <= bound)
+
+
+def test_q4_0_largest_element_maps_to_code_zero():
+    x = _x(5, 64).reshape(-1, 32)
+    q, d = quant.q4_0_quantize(x)
+    q, d = q.reshape(-1, 32), d.reshape(-1)
+    idx = np.argmax(np.abs(x), axis=1)
+    assert np.all(q[np.arange(x.shape[0]), idx] == 0)
+    m = x[np.arange(x.shape[0]), idx]
+    assert np.allclose(-8.0 * d.astype(np.float64), m, rtol=2.0 ** -11)
+
+
+def test_q4_0_round_trip_and_halves():
+    rng = np_rng(6)
+    d = 0.25
+    q = rng.integers(0, 16, size=(8, 32)).astype(np.uint8)
+    q[:, 3] = 0                               # value -8d: the largest magnitude
+    x = ((q.astype(np.float32) - 8) * np.float32(d))
+    qq, dd = quant.q4_0_quantize(x)
+    assert np.array_equal(qq.reshape(q.shape), q) and np.all(dd.astype(np.float64) == d)
+    # exact halves: y = -0.5 -> code 8, y = +0.5 -> code 9, y = 7.5 -> clamp 15
+    x = np.zeros(32, np.float32)
+    x[0] = -8 * d
+    x[1:4] = [-0.5 * d, 0.5 * d, 7.5 * d]
+    qq, _ = quant.q4_0_quantize(x)
+    assert list(qq[0, :4]) == [0, 8, 9, 15]
+
+
+def test_q4_0_zero_block():
+    q, d = quant.q4_0_quantize(np.zeros(32, np.float32))
+    assert d[0] == 0 and np.all(q == 8)
+    assert np.all(quant.q4_0_dequantize(q, d) == 0)
+
+
+def test_block_bytes_match_bits_per_element():
+    assert quant.block_bytes("q8_0") * 8 / 32 == 8.5
+    assert quant.block_bytes("q4_0") * 8 / 32 == 4.5
