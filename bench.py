@@ -1,0 +1,521 @@
+#!/usr/bin/env python
+"""Benchmark of quantized paged-KV attention on B200.
+
+Headline (one JSON line on rank 0): decode at 131,072 context -- 16 layers x 4 KV heads x
+head_dim 256, 24 query heads, 1 query token, Q8_0 K / Q4_0 V pages in a seeded shuffled page
+table.  One step = for every layer: quantize-append the new token's K/V, then split-KV decode
+(with the fused LSE merge).  value = algorithmic KV bytes read per step (416 B per token, KV
+head and layer) / device time per step, in GB/s.  The other workloads (Q8_0/Q8_0 decode,
+MTP verify at 262K with block selection, ...) are measured in the same run and reported under
+"extra".
+
+--impl reference times the CPU oracle (float64 NumPy) on the host cores on the same workload
+and metric, each step a bounded sample of it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from synth import WORKLOADS, derived_seed, np_rng, page_permutation, plant_needles_torch, torch_normal  # noqa: E402
+
+METRIC = "quantized paged KV attention: decode HBM GB/s & prefill TFLOP/s vs roofline"
+BYTES_PER_TOKEN_HEAD = {"q4_0": 34816 // 128 + 18432 // 128, "q8_0": 34816 // 128 + 34816 // 128}  # 416 / 544
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true", help="only the headline workload")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extra-steps", type=int, default=100)
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------- plumbing
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_init(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- caches
+class DecodeCache:
+    """All layers of one workload in device page pools, filled through quantize-append."""
+
+    def __init__(self, kv, w, n_blocks_per_unit, tokens, device, with_needles=False, q_for_needles=None):
+        import torch
+
+        self.kv, self.w = kv, w
+        L, H = w.layers, w.kv_heads
+        self.L, self.H, self.nb = L, H, n_blocks_per_unit
+        n_phys = L * H * n_blocks_per_unit
+        kb = kv.kvattn_page_bytes(kv.ROLE_K, kv.FMT_Q8_0)
+        vb = kv.kvattn_page_bytes(kv.ROLE_V, kv.FMT[w.v_fmt])
+        self.k_pool = torch.empty((n_phys, kb), dtype=torch.uint8, device=device)
+        self.v_pool = torch.empty((n_phys, vb), dtype=torch.uint8, device=device)
+        self.k_pool.zero_()
+        self.v_pool.zero_()
+        rng = np_rng(w.seed, 1)
+        perm = page_permutation(rng, n_phys).reshape(L, H, n_blocks_per_unit)
+        self.page_table = torch.from_numpy(perm).to(device)        # [L][H][nb]
+        self.desc = kv.make_desc(H, w.q_heads, self.k_pool, self.v_pool, n_phys, v_fmt=w.v_fmt)
+        self.needles = {}
+        for l in range(L):
+            k = torch_normal(derived_seed(w.seed, 10, l), (tokens, H, 256), device)
+            v = torch_normal(derived_seed(w.seed, 11, l), (tokens, H, 256), device)
+            if w.outlier_frac:
+                n_out = int(round(w.outlier_frac * 256))
+                for h in range(H):
+                    ch = torch.from_numpy(np_rng(w.seed, 12, l, h).choice(256, n_out, replace=False)).to(device)
+                    k[:, h, ch] *= 8.0
+                    v[:, h, ch] *= 8.0
+            if with_needles:
+                n_full = tokens // 128
+                for h in range(H):
+                    blocks = np.sort(np_rng(w.seed, 13, l, h).choice(n_full - w.recent_blocks, w.needles, replace=False))
+                    self.needles[(l, h)] = blocks
+                    direction = q_for_needles[l, -1, h * w.group:(h + 1) * w.group].to(torch.float64).sum(0)
+                    kh = k[:, h].contiguous()
+                    plant_needles_torch(kh, blocks, direction, derived_seed(w.seed, 14, l, h))
+                    k[:, h] = kh
+            kv.kvattn_quantize_append(self.desc, k, v, tokens, 0, self.page_table[l], n_blocks_per_unit)
+            del k, v
+        torch.cuda.synchronize()
+
+
+def event_pair():
+    import torch
+
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+# --------------------------------------------------------------------------- decode workloads
+class DecodeBench:
+    def __init__(self, kv, wname, device):
+        import torch
+
+        w = WORKLOADS[wname]
+        self.kv, self.w, self.device = kv, w, device
+        self.ctx = w.context
+        self.nb = (self.ctx + 127) // 128
+        self.cache = DecodeCache(kv, w, self.nb, self.ctx, device)
+        L, Hq, H = w.layers, w.q_heads, w.kv_heads
+        self.q = torch_normal(derived_seed(w.seed, 20), (L, 1, Hq, 256), device)
+        self.k_new = torch_normal(derived_seed(w.seed, 21), (L, 1, H, 256), device)
+        self.v_new = torch_normal(derived_seed(w.seed, 22), (L, 1, H, 256), device)
+        self.pos = self.ctx - 1                                   # the new token takes the last slot
+        self.q_pos = torch.tensor([self.pos], dtype=torch.int32, device=device)
+        self.out = torch.empty((L, 1, Hq, 256), device=device)
+        self.lse = torch.empty((L, 1, Hq), device=device)
+        self.ws_bytes = kv.kvattn_decode_workspace_size(self.cache.desc, 1, self.nb)
+        self.ws = torch.zeros((L, max(self.ws_bytes, 256)), dtype=torch.uint8, device=device)
+        self.bytes_per_layer = self.ctx * H * BYTES_PER_TOKEN_HEAD[w.v_fmt]
+        self.bytes_per_step = self.bytes_per_layer * L
+        self.launches_per_step = 2 * L
+
+    def layer(self, l, timed=None):
+        kv, c = self.kv, self.cache
+        kv.kvattn_quantize_append(c.desc, self.k_new[l], self.v_new[l], 1, self.pos, c.page_table[l], self.nb)
+        if timed is not None:
+            timed[0].record()
+        kv.kvattn_decode(c.desc, self.q[l], 1, self.q_pos, c.page_table[l], None, None, self.nb, self.out[l],
+                         self.lse[l], self.ws[l], self.ws_bytes)
+        if timed is not None:
+            timed[1].record()
+
+    def step(self):
+        for l in range(self.w.layers):
+            self.layer(l)
+
+
+class VerifyBench:
+    """MTP verify at 262,144 context: per layer, select 256 + 128 recent blocks (+ the tail
+    page) with the block summaries, append the 4 verify tokens, decode n_q = 4 over the
+    selected pages."""
+
+    def __init__(self, kv, device):
+        import torch
+
+        w = WORKLOADS["verify262k"]
+        self.kv, self.w = kv, w
+        L, H, Hq, g = w.layers, w.kv_heads, w.q_heads, w.group
+        self.n_full = w.context // 128
+        self.nb = self.n_full + 1                                 # + the tail page of the new tokens
+        self.q = torch_normal(derived_seed(w.seed, 20), (L, w.n_q, Hq, 256), device)
+        self.cache = DecodeCache(kv, w, self.nb, w.context, device, with_needles=True, q_for_needles=self.q)
+        c = self.cache
+        self.summ = torch.zeros((L * H, self.nb, 256), device=device)
+        kv.kvattn_block_summaries(c.desc, c.page_table.view(L * H, self.nb), L * H, self.nb, 0, self.n_full, self.summ)
+        # retrieval query rows: the last verify token's query heads, grouped per KV head
+        self.q_group = self.q[:, -1].reshape(L, H, g, 256).contiguous()
+        self.cap = w.budget_blocks + w.recent_blocks + 1
+        self.sel_l = torch.zeros((L, H, self.cap), dtype=torch.int32, device=device)
+        self.sel_p = torch.zeros((L, H, self.cap), dtype=torch.int32, device=device)
+        self.n_sel = torch.zeros((L, H), dtype=torch.int32, device=device)
+        self.sws_bytes = kv.kvattn_select_workspace_size(H, self.nb)
+        self.sws = torch.zeros(self.sws_bytes, dtype=torch.uint8, device=device)
+        self.k_new = torch_normal(derived_seed(w.seed, 21), (L, w.n_q, H, 256), device)
+        self.v_new = torch_normal(derived_seed(w.seed, 22), (L, w.n_q, H, 256), device)
+        self.pos0 = w.context
+        self.q_pos = torch.arange(self.pos0, self.pos0 + w.n_q, dtype=torch.int32, device=device)
+        self.out = torch.empty((L, w.n_q, Hq, 256), device=device)
+        self.lse = torch.empty((L, w.n_q, Hq), device=device)
+        self.ws_bytes = kv.kvattn_decode_workspace_size(c.desc, w.n_q, self.cap)
+        self.ws = torch.zeros((L, max(self.ws_bytes, 256)), dtype=torch.uint8, device=device)
+        tokens = (w.budget_blocks + w.recent_blocks) * 128 + w.n_q
+        self.bytes_per_layer = tokens * H * BYTES_PER_TOKEN_HEAD[w.v_fmt]
+        self.bytes_per_step = self.bytes_per_layer * L
+        self.select_bytes_per_layer = H * (self.n_full - w.recent_blocks) * 256 * 4
+        self.launches_per_step = 4 * L
+
+    def layer(self, l, timed=None):
+        kv, c, w = self.kv, self.cache, self.w
+        kv.kvattn_select_blocks(self.summ[l * w.kv_heads:(l + 1) * w.kv_heads], self.q_group[l], w.kv_heads, w.group,
+                                self.nb, self.n_full, self.nb, w.budget_blocks, w.recent_blocks, c.page_table[l],
+                                self.sel_l[l], self.sel_p[l], self.n_sel[l], self.cap, self.sws, self.sws_bytes)
+        kv.kvattn_quantize_append(c.desc, self.k_new[l], self.v_new[l], w.n_q, self.pos0, c.page_table[l], self.nb)
+        if timed is not None:
+            timed[0].record()
+        kv.kvattn_decode(c.desc, self.q[l], w.n_q, self.q_pos, self.sel_p[l], self.sel_l[l], self.n_sel[l], self.cap,
+                         self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
+        if timed is not None:
+            timed[1].record()
+
+    def step(self):
+        for l in range(self.w.layers):
+            self.layer(l)
+
+
+def time_steps(bench, steps, warmup, world):
+    import torch
+
+    for _ in range(warmup):
+        bench.step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = event_pair()
+    e0.record()
+    for _ in range(steps):
+        bench.step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1) / steps
+    return max_over_ranks(ms, world)
+
+
+def time_kernel(bench, steps):
+    """Average device duration of the decode launches (events on the launching stream)."""
+    import torch
+
+    pairs = []
+    for _ in range(steps):
+        for l in range(bench.w.layers):
+            p = event_pair()
+            bench.layer(l, timed=p)
+            pairs.append(p)
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in pairs)
+
+
+def time_e2e(bench, steps, warmup):
+    """Same step with the per-step inputs in pinned host memory: H2D copies of q and the new
+    K/V and a D2H copy of the outputs are inside the timed region."""
+    import torch
+
+    hq = bench.q.cpu().pin_memory()
+    hk = bench.k_new.cpu().pin_memory()
+    hv = bench.v_new.cpu().pin_memory()
+    ho = torch.empty(bench.out.shape, dtype=torch.float32).pin_memory()
+    hl = torch.empty(bench.lse.shape, dtype=torch.float32).pin_memory()
+
+    def one():
+        bench.q.copy_(hq, non_blocking=True)
+        bench.k_new.copy_(hk, non_blocking=True)
+        bench.v_new.copy_(hv, non_blocking=True)
+        bench.step()
+        ho.copy_(bench.out, non_blocking=True)
+        hl.copy_(bench.lse, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = event_pair()
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    h2d = (hq.numel() + hk.numel() + hv.numel()) * 4
+    d2h = (ho.numel() + hl.numel()) * 4
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+# --------------------------------------------------------------------------- CPU oracle
+_ORACLE_INPUTS = {}
+
+
+def _oracle_inputs(wname, n_tokens):
+    """Seeded codes for one (layer, KV head) unit, quantised by the oracle (untimed setup)."""
+    from oracle import quant as oq
+
+    key = (wname, n_tokens)
+    if key not in _ORACLE_INPUTS:
+        w = WORKLOADS[wname]
+        rng = np_rng(w.seed, 99)
+        k = rng.standard_normal((n_tokens, 256), dtype=np.float32)
+        v = rng.standard_normal((n_tokens, 256), dtype=np.float32)
+        q = rng.standard_normal((w.group, 256), dtype=np.float32)
+        _ORACLE_INPUTS.clear()
+        _ORACLE_INPUTS[key] = (q, oq.q8_0_quantize(k), oq.quantize(v, w.v_fmt))
+    return _ORACLE_INPUTS[key]
+
+
+def oracle_decode_sample(wname, n_tokens, reps_min_s=8.0, max_reps=3):
+    """Times the oracle (dequantise + float64 attention) on one (layer, KV head) unit and
+    the last n_tokens of the workload's context.  Returns (GB/s, seconds, threads, sample)."""
+    from oracle import attention as oatt
+    from oracle import quant as oq
+
+    w = WORKLOADS[wname]
+    q, (kc, kd), (vc, vd) = _oracle_inputs(wname, n_tokens)
+    pos = np.arange(w.context - n_tokens, w.context)
+    t_total, reps = 0.0, 0
+    while reps < max_reps and (reps == 0 or t_total < reps_min_s):
+        t0 = time.perf_counter()
+        kh = oq.q8_0_dequantize(kc, kd)
+        vh = oq.dequantize(vc, vd, w.v_fmt)
+        oatt.attend(q, kh, vh, pos, np.full(w.group, w.context - 1), 1.0 / 16)
+        t_total += time.perf_counter() - t0
+        reps += 1
+    secs = t_total / reps
+    gbs = n_tokens * BYTES_PER_TOKEN_HEAD[w.v_fmt] / secs / 1e9
+    threads = len(os.sched_getaffinity(0))
+    sample = f"1 of {w.layers * w.kv_heads} (layer, KV head) units, {n_tokens} of {w.context} tokens, {w.group} query heads"
+    return gbs, secs, threads, sample
+
+
+def reference_arm(args, world, rank):
+    if world > 1 and rank != 0:
+        return
+    w = WORKLOADS["decode131k"]
+    # size the per-step sample so that warmup + steps take about two minutes
+    probe_tokens = 8192
+    gbs, secs, threads, _ = oracle_decode_sample("decode131k", probe_tokens, 0.0, 1)
+    budget_s = 120.0 / max(1, args.steps + args.warmup)
+    n_tok = int(max(1024, min(w.context, probe_tokens * budget_s / max(secs, 1e-6))) // 128 * 128)
+    times = []
+    for i in range(args.warmup + args.steps):
+        g, s, threads, sample = oracle_decode_sample("decode131k", n_tok, 0.0, 1)
+        if i >= args.warmup:
+            times.append(s)
+    secs = statistics.mean(times)
+    value = n_tok * BYTES_PER_TOKEN_HEAD[w.v_fmt] / secs / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "decode131k", "layers": w.layers, "kv_heads": w.kv_heads, "q_heads": w.q_heads,
+                   "context": w.context, "n_q": 1, "k_fmt": w.k_fmt, "v_fmt": w.v_fmt},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- main
+def main():
+    args = parse_args()
+    world, rank, local = dist_init(args)
+    if args.impl == "reference":
+        reference_arm(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return
+
+    import torch
+
+    from quantized_paged_kv_q4_b200 import build, kvattn
+
+    build.build()
+    torch.cuda.set_device(local)
+    kvattn.kvattn_init(local)
+    device = torch.device("cuda", local)
+    hbm, bf16, bf16_sus, peak_kind = peaks()
+
+    # ---------------- headline: decode at 131K ----------------
+    b = DecodeBench(kvattn, "decode131k", device)
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms = time_steps(b, args.steps, args.warmup, world)
+    clk = clocks.stop()
+    kern_ms = time_kernel(b, max(3, min(args.steps, 50)))
+    e2e_ms, h2d, d2h = time_e2e(b, max(3, min(args.steps, 200)), 3)
+    assert kvattn.kvattn_device_error() == 0
+    value = b.bytes_per_step * world / (ms * 1e-3) / 1e9
+    achieved = b.bytes_per_layer / (kern_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "s8/f16 MMA, f32 accumulate", "data": "synthetic",
+        "config": {"workload": "decode131k", "layers": b.w.layers, "kv_heads": b.w.kv_heads,
+                   "q_heads": b.w.q_heads, "context": b.ctx, "n_q": 1, "k_fmt": "q8_0", "v_fmt": "q4_0",
+                   "outliers": "1% of channels x8", "parallelism": f"{world} independent decodes (one per GPU)",
+                   "l2": "inputs larger than L2 (218 MB of KV per layer launch, 3.49 GB per step)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": None, "kernel": "decode_kernel<1,false,false>",
+                     "peak_kind": f"{peak_kind} copy bandwidth (hbm_gbs)",
+                     "algorithmic_bytes_per_launch": b.bytes_per_layer, "avg_launch_ms": kern_ms},
+        "e2e": {"value": b.bytes_per_step * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": b.launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    del b
+    torch.cuda.empty_cache()
+
+    # ---------------- the other workloads ----------------
+    extra = {}
+    if not args.no_extra:
+        try:
+            b2 = DecodeBench(kvattn, "decode131k_q8q8", device)
+            ms2 = time_steps(b2, args.extra_steps, 5, world)
+            k2 = time_kernel(b2, 10)
+            extra["decode131k_q8q8"] = {"GB/s": b2.bytes_per_step / (ms2 * 1e-3) / 1e9, "ms_per_step": ms2,
+                                        "kernel_GB/s": b2.bytes_per_layer / (k2 * 1e-3) / 1e9,
+                                        "kernel_frac_hbm": b2.bytes_per_layer / (k2 * 1e-3) / 1e9 / hbm}
+            del b2
+            torch.cuda.empty_cache()
+            b3 = VerifyBench(kvattn, device)
+            ms3 = time_steps(b3, args.extra_steps, 5, world)
+            k3 = time_kernel(b3, 10)
+            extra["verify262k"] = {"GB/s": b3.bytes_per_step / (ms3 * 1e-3) / 1e9, "ms_per_step": ms3,
+                                   "decode_kernel_GB/s": b3.bytes_per_layer / (k3 * 1e-3) / 1e9,
+                                   "decode_kernel_frac_hbm": b3.bytes_per_layer / (k3 * 1e-3) / 1e9 / hbm,
+                                   "selected_tokens_per_unit": (b3.w.budget_blocks + b3.w.recent_blocks) * 128 + 4}
+            del b3
+            torch.cuda.empty_cache()
+        except Exception as exc:  # report, do not hide
+            extra["error"] = repr(exc)
+        assert kvattn.kvattn_device_error() == 0
+    line["extra"] = extra
+
+    if rank == 0 and not args.no_cpu_baseline:
+        gbs, secs, threads, sample = oracle_decode_sample("decode131k", 32768)
+        line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample,
+                                "seconds_per_sample": secs}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        barrier(world)
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

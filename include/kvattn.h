@@ -1,0 +1,241 @@
+/*
+ * kvattn -- attention over a block-quantized, paged KV cache on NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libkvattn.so.  Plain pointers and sizes only.  Every entry point returns an
+ * int status (0 = KVATTN_OK, negative = error, see kvattn_status); none throws, none
+ * allocates device memory.  All GPU work is asynchronous on the caller's stream; buffers
+ * must stay valid until that work completes.  The caller owns every buffer.
+ *
+ * Sources (page title, section):
+ *  [KVMEM]  KVMem reproduction on one 7900 XTX (lcz.me/topic/1972): test command (128-token
+ *           blocks, 32,768-token budget, 16,384-token generation reserve), recall section
+ *           (blocks kept on the GPU are chosen by a retrieval query).
+ *  [STREAM] Adaptive KV Streaming + RDNA 4 announcement (wqu.guru): full KV history in
+ *           host RAM, bounded working sets streamed over PCIe alongside compute; method list
+ *           (paged decode attention extended to verify batches; chunked prefill across
+ *           streamed pages merged by online log-sum-exp; layer L+1 transfers overlapped
+ *           with layer L compute).
+ *  [GUIDE]  Adaptive KV Streaming six-step validation guide (alphalab.site): streaming needs
+ *           flash attention with Q8_0 K / Q4_0 V.
+ *  [VULKAN] Vulkan speculative-decoding report, 7900 XTX (lcz.me/topic/1398): model structure
+ *           (16 layers x 4 KV heads x 256 = 16,384 elements per token), pitfalls (q4_0 =
+ *           18 bytes per 32 elements; only legacy block quants are valid KV formats) and
+ *           configs (q8_0 = 8.5 bits per element).
+ *
+ * Data formats (fixed by this library; the pages fix only the bits per element):
+ *  - head_dim = 256, page = 128 tokens of one (layer, KV head).
+ *  - Q8_0: blocks of 32 int8 codes + one fp16 scale d; value = q * d.
+ *    Q4_0: blocks of 32 4-bit codes q in [0,15] + fp16 d; value = (q - 8) * d.
+ *  - K pages are Q8_0 (34,816 B); V pages are Q4_0 (18,432 B) or Q8_0 (34,816 B).  Inside a
+ *    page, codes come first and fp16 scales after them, both in tensor-core fragment order
+ *    (tok = slot in page, c = channel, b = c/32, G = tok/16):
+ *      K Q8_0 code  (tok = 16G+8H+R, c = 64P+32(j/8)+8T+j%8) at ((((G*4+P)*2+H)*8+R)*4+T)*16+j
+ *      K scale      d[16G+8H+R][b] at 32768 + 2*(((G*8+R)*2+H)*8+b)
+ *      V Q4_0 byte  ((((G*4+C)*8+R)*4+T)*16 + 4w + y: block b = 2C+w/2, token
+ *                   16G+2T+8(w%2)+y/2; low nibble c = 32b+16(y%2)+R, high nibble c+8
+ *      V Q8_0 code  (tok = 16G+2T+8(w%2)+y%2, c = 32b+16(w/2)+8(y/2)+R) at
+ *                   ((((G*8+b)*8+R)*4+T)*16 + 4w + y
+ *      V scale      d[16G+2T+k%2+8(k/2)][b] at S + 2*(((G*4+T)*8+b)*4+k), S = 16384 (Q4_0)
+ *                   or 32768 (Q8_0)
+ *    kvattn_quantize_append is the supported writer.
+ *  - Pages live in caller-owned pools: page p's K bytes start at k_pool + p * k_page_stride
+ *    and its V bytes at v_pool + p * v_page_stride.  Pool bases and strides are multiples
+ *    of 16 bytes.  K and V of one page may be interleaved in one allocation by choosing
+ *    v_pool = k_pool + 34816 and equal strides.
+ *  - A page list names, per KV head, the physical pages to attend over and (optionally)
+ *    their logical block indices; key positions are logical * 128 + slot.
+ *
+ * Device-side checks: every page id read on the device is checked against [0, n_pages);
+ * a bad id skips the page and records KVATTN_ERR_BAD_PAGE in a per-device error word that
+ * kvattn_device_error() returns and clears.  Bounded waits inside kernels record
+ * KVATTN_ERR_TIMEOUT there instead of spinning forever.
+ */
+#ifndef KVATTN_H
+#define KVATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define KVATTN_API __attribute__((visibility("default")))
+#else
+#define KVATTN_API
+#endif
+
+/* cudaStream_t / cudaEvent_t, passed opaquely (0 = the legacy default stream). */
+typedef void* kvattn_stream_t;
+typedef void* kvattn_event_t;
+
+enum kvattn_status {
+  KVATTN_OK = 0,
+  KVATTN_ERR_INVALID_ARG = -1,        /* null pointer, bad size or alignment, bad range     */
+  KVATTN_ERR_UNSUPPORTED_ARCH = -2,   /* device is not compute capability 10.0 (sm_100)     */
+  KVATTN_ERR_UNSUPPORTED_FORMAT = -3, /* format / head_dim / page size this build lacks     */
+  KVATTN_ERR_BAD_PAGE = -4,           /* a page id outside [0, n_pages) (device-side check) */
+  KVATTN_ERR_WORKSPACE_TOO_SMALL = -5,
+  KVATTN_ERR_CUDA = -6,               /* a CUDA runtime call failed; see kvattn_last_cuda_error */
+  KVATTN_ERR_TIMEOUT = -7,            /* a bounded wait expired                             */
+  KVATTN_ERR_UNSUPPORTED_SHAPE = -8,  /* e.g. more query rows per KV head than supported    */
+  KVATTN_ERR_NOT_INITIALIZED = -9     /* kvattn_init was not called for the current device  */
+};
+
+enum kvattn_format { KVATTN_FMT_Q4_0 = 4, KVATTN_FMT_Q8_0 = 8 };
+enum kvattn_role { KVATTN_ROLE_K = 0, KVATTN_ROLE_V = 1 };
+
+typedef struct kvattn_kv_desc {
+  int32_t n_kv_heads;     /* H_kv >= 1                                                  */
+  int32_t n_q_heads;      /* H_q, a multiple of H_kv; the GQA group is H_q / H_kv       */
+  int32_t head_dim;       /* must be 256                                                */
+  int32_t page_tokens;    /* must be 128                                                */
+  int32_t k_fmt;          /* KVATTN_FMT_Q8_0                                            */
+  int32_t v_fmt;          /* KVATTN_FMT_Q4_0 or KVATTN_FMT_Q8_0                         */
+  void* k_pool;           /* device memory, 16-byte aligned                              */
+  void* v_pool;           /* device memory, 16-byte aligned                              */
+  int64_t k_page_stride;  /* bytes between consecutive K pages (>= K page bytes, %16==0) */
+  int64_t v_page_stride;  /* bytes between consecutive V pages (>= V page bytes, %16==0) */
+  int64_t n_pages;        /* physical pages addressable in both pools                   */
+} kvattn_kv_desc;
+
+/* ---- setup and status ------------------------------------------------------------- */
+
+/* Checks that `device` is an sm_100 part and prepares the kernels for it (sets it current).
+ * Returns KVATTN_ERR_UNSUPPORTED_ARCH on any other device.  Call once per device before any
+ * other GPU entry point on it.  Not stream-ordered; do not call during stream capture. */
+KVATTN_API int kvattn_init(int device);
+
+/* Static, human-readable name of a status code. */
+KVATTN_API const char* kvattn_status_string(int status);
+
+/* The last cudaError_t seen by the library on this thread (0 if none). */
+KVATTN_API int kvattn_last_cuda_error(void);
+
+/* Synchronises `stream`, then returns and clears the current device's error word
+ * (KVATTN_OK, KVATTN_ERR_BAD_PAGE or KVATTN_ERR_TIMEOUT). */
+KVATTN_API int kvattn_device_error(kvattn_stream_t stream);
+
+/* Bytes of one page of the given role and format (0 if the pair is unsupported). */
+KVATTN_API int64_t kvattn_page_bytes(int role, int fmt);
+
+/* ---- cache write path ----------------------------------------------------------------
+ * Quantizes n_tok new tokens and writes them into their pages (the Q8_0 / Q4_0 encoders of
+ * [VULKAN] pitfalls).  Q8_0: d = amax/127, q = round-half-away(x * fp32(1/d)), clamped to
+ * +-127.  Q4_0: m = the element of largest magnitude, d = m/-8, q = min(15, floor(x * fp32(1/d)
+ * + 8.5)).  Every step that decides a code is rounded to fp32; scales are stored as fp16.
+ *   k, v        device fp32 [n_tok][H_kv][256]
+ *   pos0        position of the first token; token i goes to logical block (pos0+i)/128,
+ *               slot (pos0+i)%128
+ *   page_table  device int32 [H_kv][n_blocks]: logical block -> physical page
+ * Other slots of the touched pages are left unchanged.  Returns INVALID_ARG if a touched
+ * block is >= n_blocks. */
+KVATTN_API int kvattn_quantize_append(const kvattn_kv_desc* desc, const float* k, const float* v,
+                                      int n_tok, int32_t pos0, const int32_t* page_table,
+                                      int n_blocks, kvattn_stream_t stream);
+
+/* ---- split-KV flash decode / MTP verify ---------------------------------------------
+ * Attention of n_q query tokens (1 = decode, up to 4 = MTP verify batch; [STREAM] method
+ * list) of every query head over the pages listed for its KV head.  Query token i sits at
+ * position q_pos[i]; it sees keys with position <= q_pos[i] (causal among the new tokens).
+ *   q            device fp32 [n_q][H_q][256]
+ *   q_pos        device int32 [n_q]
+ *   page_list    device int32 [H_kv][max_pages]: physical page ids, any order
+ *   page_logical device int32 [H_kv][max_pages] logical block of each listed page, or NULL
+ *                (then page_list[h][i] holds logical block i)
+ *   n_pages      device int32 [H_kv] pages used per head (<= max_pages), or NULL (= max_pages)
+ *   out          device fp32 [n_q][H_q][256]: softmax(q.k/16) v
+ *   lse          device fp32 [n_q][H_q]: natural-log log-sum-exp of the scaled scores
+ *                (-inf and out = 0 for a row that sees no key)
+ *   ws, ws_bytes device workspace of at least kvattn_decode_workspace_size() bytes; its
+ *                first 256 bytes must be zero before the first use and are left zero.
+ * Supports group * n_q <= 24 query rows per KV head.  The split count depends only on the
+ * arguments and the device, so results are deterministic. */
+KVATTN_API size_t kvattn_decode_workspace_size(const kvattn_kv_desc* desc, int n_q, int max_pages);
+KVATTN_API int kvattn_decode(const kvattn_kv_desc* desc, const float* q, int n_q, const int32_t* q_pos,
+                             const int32_t* page_list, const int32_t* page_logical,
+                             const int32_t* n_pages, int max_pages, float* out, float* lse,
+                             void* ws, size_t ws_bytes, kvattn_stream_t stream);
+
+/* ---- log-sum-exp merge ([STREAM] method list: online LSE accumulation) -------------
+ * out = sum_p exp(lse_p - lse) * o_p with lse = ln sum_p exp(lse_p), skipping -inf parts.
+ *   o_parts   device fp32 [n_parts][rows][dim];  lse_parts device fp32 [n_parts][rows]
+ *   out       device fp32 [rows][dim];           lse       device fp32 [rows]
+ * dim must be a multiple of 4. */
+KVATTN_API int kvattn_merge_lse(const float* o_parts, const float* lse_parts, int n_parts, int rows,
+                                int dim, float* out, float* lse, kvattn_stream_t stream);
+
+/* ---- KVMem block summaries and selection ([KVMEM]) ---------------------------------
+ * Summary of a full 128-token block = mean dequantized key per channel, rounded once to
+ * fp32 (the per-block sum is exact in fp64 for scales within 2^28 of each other).
+ *   page_table  device int32 [n_units][n_blocks] (a unit is one (layer, KV head))
+ *   summaries   device fp32 [n_units][n_blocks][256]; blocks [block_begin, block_end) of
+ *               every unit are written, others untouched. */
+KVATTN_API int kvattn_block_summaries(const kvattn_kv_desc* desc, const int32_t* page_table,
+                                      int n_units, int n_blocks, int block_begin, int block_end,
+                                      float* summaries, kvattn_stream_t stream);
+
+/* Per unit: score[b] = sum_{j<group, c<256} q_group[j][c] * summary[b][c] in fp64 for the
+ * candidate blocks b < n_full - recent; keep the `budget` best (ties: lower b first), add the
+ * recent window [n_full - recent, n_full) and the partial tail [n_full, n_total); write them
+ * in ascending order.
+ *   summaries   device fp32 [n_units][n_blocks][256]   (n_blocks >= n_total)
+ *   q_group     device fp32 [n_units][group][256]       (the retrieval query rows)
+ *   page_table  device int32 [n_units][n_blocks]
+ *   sel_logical device int32 [n_units][cap], sel_phys device int32 [n_units][cap],
+ *   n_sel       device int32 [n_units]; cap >= min(budget, candidates) + recent + tail.
+ *   ws          device workspace of kvattn_select_workspace_size(n_units, n_blocks) bytes.
+ * Candidates per unit <= 16384. */
+KVATTN_API size_t kvattn_select_workspace_size(int n_units, int n_blocks);
+KVATTN_API int kvattn_select_blocks(const float* summaries, const float* q_group, int n_units,
+                                    int group, int n_blocks, int n_full, int n_total, int budget,
+                                    int recent, const int32_t* page_table, int32_t* sel_logical,
+                                    int32_t* sel_phys, int32_t* n_sel, int cap, void* ws,
+                                    size_t ws_bytes, kvattn_stream_t stream);
+
+/* ---- chunked prefill on tcgen05 ([STREAM] method list) -----------------------------
+ * Attention of n_q bf16 query tokens (positions q_pos[i], device int32 [n_q]) over the
+ * listed pages, causal.  K/V pages are dequantized to bf16 in shared memory; QK^T and PV
+ * run on tcgen05 tensor cores with fp32 accumulation in tensor memory.  The keys are taken
+ * in splits of kv_split_tokens (a multiple of 128); partial results are merged by
+ * log-sum-exp.
+ *   q      device bf16 bits [n_q][H_q][256];  out device fp32 [n_q][H_q][256];
+ *   lse    device fp32 [n_q][H_q];  page arguments as for kvattn_decode.
+ *   ws     device workspace of kvattn_prefill_workspace_size() bytes (first 256 zero). */
+KVATTN_API size_t kvattn_prefill_workspace_size(const kvattn_kv_desc* desc, int n_q, int max_pages,
+                                                int kv_split_tokens);
+KVATTN_API int kvattn_prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* q, int n_q,
+                                    const int32_t* q_pos, const int32_t* page_list,
+                                    const int32_t* page_logical, const int32_t* n_pages,
+                                    int max_pages, int kv_split_tokens, float* out, float* lse,
+                                    void* ws, size_t ws_bytes, kvattn_stream_t stream);
+
+/* ---- host page streaming ([STREAM]: full history in pinned host RAM, working set over
+ * PCIe; layer L+1 prefetched while layer L computes) ----------------------------------
+ * Copies n pages from a pinned host pool to device slots with cudaMemcpyAsync on
+ * copy_stream, merging runs where both the host page id and the device slot increase by
+ * one.  Page i: host_pool + host_ids[i]*host_stride -> dev_pool + dev_slots[i]*dev_stride,
+ * page_bytes bytes.  host_ids and dev_slots are HOST arrays.  If `done` is non-null it is
+ * recorded on copy_stream after the last copy.  Returns the number of copies issued through
+ * *n_copies when non-null. */
+KVATTN_API int kvattn_stream_pages(const void* host_pool, int64_t host_stride, void* dev_pool,
+                                   int64_t dev_stride, int64_t page_bytes, const int32_t* host_ids,
+                                   const int32_t* dev_slots, int n, kvattn_stream_t copy_stream,
+                                   kvattn_event_t done, int* n_copies);
+
+/* The copy plan of kvattn_stream_pages, computed on the host without touching the GPU:
+ * splits the n (host id, device slot) pairs into maximal runs in which both increase by one.
+ * Writes up to max_runs (first index, length) pairs into run_first / run_len (HOST arrays,
+ * may be NULL when max_runs is 0) and returns the number of runs (or a negative status). */
+KVATTN_API int kvattn_stream_plan(const int32_t* host_ids, const int32_t* dev_slots, int n, int32_t* run_first,
+                                  int32_t* run_len, int max_runs);
+
+/* Polls `event` until it completes or timeout_ms elapses (KVATTN_ERR_TIMEOUT). */
+KVATTN_API int kvattn_stream_wait(kvattn_event_t event, int timeout_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVATTN_H */

@@ -1,0 +1,592 @@
+// Split-KV flash decode over Q8_0 K / Q4_0 (or Q8_0) V pages, for one query token or an
+// MTP verify batch of up to 4 (Adaptive KV Streaming + RDNA 4 announcement, wqu.guru,
+// method list: "paged decode attention extended to verify batches").
+//
+// Grid: (split, KV head).  One CTA per SM: warp 8 streams whole pages into a shared-memory
+// ring with bulk async copies (TMA engine, one 34,816 B K copy and one V copy per page);
+// warps 0-7 consume them.  All query rows of the KV head's group (group x n_q <= 24) are
+// packed into the N dimension of legacy tensor-core MMAs so every KV byte is read once per
+// group:
+//   QK^T: int8 MMA (m16n8k32), A = raw Q8_0 key codes straight from the page (16 tokens on
+//         M), B = the query split exactly into two int8 levels (q ~ s (a + b/254)); each
+//         32-channel block gets a fresh int32 accumulator that is scaled by the key's fp16
+//         block scale, so the dot product itself is exact integer arithmetic.
+//   PV:   f16 MMA (m16n8k16), A = V^T decoded in registers from nibbles (value q - 8, exact
+//         in f16), B = P^T (probabilities, transposed in registers with movmatrix) times the
+//         V block scale.
+// The online softmax keeps a per-row running maximum and rescales the accumulators only
+// when the maximum grows by more than 2^8 (p stays <= 256, safe in f16).  Warps merge their
+// partial states in shared memory; CTAs write (o, lse) partials and the last CTA of each KV
+// head merges them (log-sum-exp merge, the same arithmetic as kvattn_merge_lse).
+#include "decode.cuh"
+
+namespace kvattn {
+
+
+template <int NT, bool PAIR, bool VQ8>
+struct DecodeCfg {
+  static constexpr int kConsumerWarps = 8;
+  static constexpr int kThreads = kConsumerWarps * 32;  // lane 0 of warp 0 also issues the copies
+  static constexpr int kNB = PAIR ? 4 : 8;      // 32-channel blocks per warp
+  static constexpr int kTilesPerWarp = PAIR ? 2 : 1;
+  static constexpr int kVBytes = VQ8 ? kV8PageBytes : kV4PageBytes;
+  static constexpr int kStageBytes = kKPageBytes + kVBytes;
+  static constexpr int kStages = PAIR ? (VQ8 ? 2 : 3) : (VQ8 ? 3 : 4);
+  static constexpr int kUnits = PAIR ? 4 : 8;   // independent softmax streams per CTA
+  static constexpr int kRowsPad = NT * 8;
+  static constexpr int kXBytes = PAIR ? 4 * 2 * 2 * NT * 32 * 16 : 0;  // pair S exchange
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static constexpr int kMergeBytes = kUnits * kRowsPad * (kHeadDim + 2) * 4;
+  static_assert(kMergeBytes <= kRingBytes, "merge buffer must fit in the ring");
+  static constexpr int kBarOffset = kRingBytes + kXBytes;
+  static constexpr int kSmemBytes = kBarOffset + 256;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+constexpr uint32_t kHalf2Magic = 0x64006400u;  // f16 1024.0 in both halves
+constexpr uint32_t kHalf2_1032 = 0x64086408u;  // 1024 + 8
+constexpr uint32_t kHalf2_1152 = 0x64806480u;  // 1024 + 128
+constexpr uint32_t kHalf2_1_16 = 0x2C002C00u;  // 1/16
+constexpr uint32_t kHalf2_m72 = 0xD480D480u;   // -(64 + 8)
+
+template <int NT, bool PAIR, bool VQ8>
+__global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_kernel(const DecodeParams p) {
+  using C = DecodeCfg<NT, PAIR, VQ8>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* xbar = empty + C::kStages;  // [4] pair exchange barriers (PAIR only)
+  int* st_logical = reinterpret_cast<int*>(xbar + 4);
+  int* st_valid = st_logical + C::kStages;
+  int* s_flags = st_valid + C::kStages;  // [0] abort, [1] last-CTA flag
+
+  const int h = blockIdx.y;
+  const int split = blockIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int n_rows = p.group * p.n_q;
+
+  int np = p.max_pages;
+  if (p.n_pages_arr) np = min(max(p.n_pages_arr[h], 0), p.max_pages);
+  const int first = static_cast<int>(static_cast<long long>(split) * np / p.n_splits);
+  const int last = static_cast<int>(static_cast<long long>(split + 1) * np / p.n_splits);
+  const int count = last - first;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], C::kConsumerWarps);
+    }
+    for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 2);
+    s_flags[0] = 0;
+    s_flags[1] = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  // per-warp softmax state (consumers)
+  float m_run[NT][2], l_run[NT][2];
+  float oacc[2 * C::kNB][NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      m_run[nt][c] = -INFINITY;
+      l_run[nt][c] = 0.f;
+    }
+#pragma unroll
+  for (int i = 0; i < 2 * C::kNB; ++i)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) oacc[i][nt][e] = 0.f;
+
+  const int half = PAIR ? (warp & 1) : 0;
+  const int blk0 = PAIR ? 4 * half : 0;
+
+  // Page copies are issued by lane 0 of warp 0, at most kStages pages ahead of its own
+  // consumption.  A stage is refilled only after all eight warps released its previous page
+  // (empty barrier); refills are attempted without blocking, except for the page warp 0 is
+  // about to consume, so no warp ever waits on a slower one except through that page.
+  const int32_t* plist = p.page_list + static_cast<long long>(h) * p.max_pages;
+  const int32_t* plog = p.page_logical ? p.page_logical + static_cast<long long>(h) * p.max_pages : nullptr;
+  int next = 0;  // next page to issue (meaningful in lane 0 of warp 0 only)
+  auto issue_upto = [&](int i) -> bool {
+    while (next < count && next < i + C::kStages) {
+      const int s = next % C::kStages;
+      const int prev = next - C::kStages;
+      if (prev >= 0) {
+        const uint32_t ppar = (prev / C::kStages) & 1;
+        if (next == i) {
+          if (!mbar_wait(&empty[s], ppar)) return false;
+        } else if (!mbar_try_wait(&empty[s], ppar)) {
+          break;
+        }
+      }
+      const int idx = first + next;
+      const int page = plist[idx];
+      st_logical[s] = plog ? plog[idx] : idx;
+      if (page < 0 || page >= p.n_pages) {
+        record_error(KVATTN_ERR_BAD_PAGE);
+        st_valid[s] = 0;
+        mbar_arrive(&full[s]);
+      } else {
+        st_valid[s] = 1;
+        uint8_t* stage = smem + s * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+        bulk_g2s(stage, p.k_pool + static_cast<int64_t>(page) * p.k_stride, kKPageBytes, &full[s]);
+        bulk_g2s(stage + kKPageBytes, p.v_pool + static_cast<int64_t>(page) * p.v_stride, C::kVBytes, &full[s]);
+      }
+      ++next;
+    }
+    return true;
+  };
+  const bool issuer = (warp == 0 && lane == 0);
+  if (issuer) issue_upto(0);
+
+  {
+    // ------------------------------------------------------------------ consumers
+    // query rows of this KV head: r = qi * group + j  ->  q[qi][h * group + j][:]
+    // B fragments: level a and level b, per block and n-tile: two regs each.
+    uint32_t qf[C::kNB][NT][2][2];
+    float crow[NT][2];
+    int qpos_row[NT][2];
+    int qpos_min = INT_MAX;
+    for (int i = 0; i < p.n_q; ++i) qpos_min = min(qpos_min, p.q_pos[i]);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int r = nt * 8 + g;
+      float x[kBlocks][8];
+      if (r < n_rows) {
+        const int qi = r / p.group, j = r % p.group;
+        const float* qr = p.q + (static_cast<long long>(qi) * p.n_qh + h * p.group + j) * kHeadDim;
+#pragma unroll
+        for (int b = 0; b < kBlocks; ++b) {
+          const float4 u = *reinterpret_cast<const float4*>(qr + 32 * b + 8 * t);
+          const float4 w = *reinterpret_cast<const float4*>(qr + 32 * b + 8 * t + 4);
+          x[b][0] = u.x; x[b][1] = u.y; x[b][2] = u.z; x[b][3] = u.w;
+          x[b][4] = w.x; x[b][5] = w.y; x[b][6] = w.z; x[b][7] = w.w;
+        }
+      } else {
+#pragma unroll
+        for (int b = 0; b < kBlocks; ++b)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[b][e] = 0.f;
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int b = 0; b < kBlocks; ++b)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[b][e]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      const float sq = amax / 127.f;
+      const float inv = amax > 0.f ? 127.f / amax : 0.f;
+#pragma unroll
+      for (int bl = 0; bl < C::kNB; ++bl) {
+        uint32_t la[2] = {0u, 0u}, lb[2] = {0u, 0u};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          // blk0 is 0 or 4: select with constant indices (no local-memory array)
+          const float xv = (PAIR && half) ? x[(4 + bl) % kBlocks][e] : x[bl][e];
+          const float a = fminf(fmaxf(rintf(xv * inv), -127.f), 127.f);
+          const float res = xv - a * sq;
+          const float bb = fminf(fmaxf(rintf(res * inv * 254.f), -127.f), 127.f);
+          la[e >> 2] |= (static_cast<uint32_t>(static_cast<int>(a)) & 0xFFu) << (8 * (e & 3));
+          lb[e >> 2] |= (static_cast<uint32_t>(static_cast<int>(bb)) & 0xFFu) << (8 * (e & 3));
+        }
+        qf[bl][nt][0][0] = la[0];
+        qf[bl][nt][0][1] = la[1];
+        qf[bl][nt][1][0] = lb[0];
+        qf[bl][nt][1][1] = lb[1];
+      }
+      // score factor of this lane's row, then fetch those of rows 2t, 2t+1
+      const float cr = sq * (1.0f / 254.0f) * (1.0f / 16.0f) * 1.4426950408889634f;
+      crow[nt][0] = __shfl_sync(0xffffffffu, cr, (2 * t) * 4);
+      crow[nt][1] = __shfl_sync(0xffffffffu, cr, (2 * t + 1) * 4);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int rr = nt * 8 + 2 * t + c;
+        qpos_row[nt][c] = rr < n_rows ? p.q_pos[rr / p.group] : INT_MAX;
+      }
+    }
+
+    const int pair = PAIR ? (warp >> 1) : 0;
+    float* xbuf = reinterpret_cast<float*>(smem + C::kRingBytes);
+    int xpar = 0;
+    uint32_t xphase = 0;
+    bool aborted = false;
+
+    for (int i = 0; i < count; ++i) {
+      const int s = i % C::kStages;
+      const uint32_t par = (i / C::kStages) & 1;
+      if (warp == 0) {
+        int ok = 1;
+        if (lane == 0) ok = issue_upto(i) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          s_flags[0] = 1;
+          break;
+        }
+      }
+      if (!mbar_wait(&full[s], par)) {
+        s_flags[0] = 1;
+        break;
+      }
+      if (st_valid[s]) {
+        const uint32_t kb = smem_u32(smem + s * C::kStageBytes);
+        const uint32_t vb = kb + kKPageBytes;
+        const int logical = st_logical[s];
+        const bool need_mask = static_cast<long long>(logical) * kPageTokens + (kPageTokens - 1) > qpos_min;
+#pragma unroll
+        for (int tt = 0; tt < C::kTilesPerWarp; ++tt) {
+          const int G = PAIR ? (2 * pair + tt) : warp;
+          // ---------------- S = K Q^T over this warp's channel blocks ----------------
+          float sacc[NT][4];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+          // key scales for rows g (H=0) and g+8 (H=1), blocks blk0..blk0+kNB-1
+          float dk[2][C::kNB];
+#pragma unroll
+          for (int H = 0; H < 2; ++H) {
+            const uint32_t a = kb + kKScaleOffset + (((G * 8 + g) * 2 + H) * 8 + blk0) * 2;
+            if constexpr (C::kNB == 8) {
+              const uint4 v = lds128(a);
+              const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                dk[H][2 * e] = half_lo(w[e]);
+                dk[H][2 * e + 1] = half_hi(w[e]);
+              }
+            } else {
+              uint32_t w0, w1;
+              asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(a));
+              dk[H][0] = half_lo(w0);
+              dk[H][1] = half_hi(w0);
+              dk[H][2] = half_lo(w1);
+              dk[H][3] = half_hi(w1);
+            }
+          }
+#pragma unroll
+          for (int pp = 0; pp < C::kNB / 2; ++pp) {
+            const int P = blk0 / 2 + pp;
+            const uint4 ka = lds128(kb + ((((G * 4 + P) * 2 + 0) * 8 + g) * 4 + t) * 16);
+            const uint4 kc = lds128(kb + ((((G * 4 + P) * 2 + 1) * 8 + g) * 4 + t) * 16);
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int bl = 2 * pp + e;
+              const uint32_t a0 = e ? ka.z : ka.x, a2 = e ? ka.w : ka.y;
+              const uint32_t a1 = e ? kc.z : kc.x, a3 = e ? kc.w : kc.y;
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                const int zero[4] = {0, 0, 0, 0};
+                int ca[4], cb[4];
+                mma_s8(ca, a0, a1, a2, a3, qf[bl][nt][0][0], qf[bl][nt][0][1], zero);
+                mma_s8(cb, a0, a1, a2, a3, qf[bl][nt][1][0], qf[bl][nt][1][1], zero);
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2) {
+                  const float v = __int2float_rn(254 * ca[e2] + cb[e2]);
+                  sacc[nt][e2] = fmaf(dk[e2 >> 1][bl], v, sacc[nt][e2]);
+                }
+              }
+            }
+          }
+          if constexpr (PAIR) {
+            // exchange partial scores with the partner warp (other channel half)
+            float* mine = xbuf + ((((pair * 2 + half) * 2 + xpar) * NT) * 32) * 4;
+            float* theirs = xbuf + ((((pair * 2 + (half ^ 1)) * 2 + xpar) * NT) * 32) * 4;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+              *reinterpret_cast<float4*>(mine + (nt * 32 + lane) * 4) =
+                  make_float4(sacc[nt][0], sacc[nt][1], sacc[nt][2], sacc[nt][3]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xbar[pair]);
+            if (!mbar_wait(&xbar[pair], xphase)) {
+              s_flags[0] = 1;
+              aborted = true;
+              break;
+            }
+            xphase ^= 1;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              const float4 o = *reinterpret_cast<const float4*>(theirs + (nt * 32 + lane) * 4);
+              // same operands in both warps, so both get bit-identical sums
+              if (half == 0) {
+                sacc[nt][0] += o.x; sacc[nt][1] += o.y; sacc[nt][2] += o.z; sacc[nt][3] += o.w;
+              } else {
+                sacc[nt][0] = o.x + sacc[nt][0]; sacc[nt][1] = o.y + sacc[nt][1];
+                sacc[nt][2] = o.z + sacc[nt][2]; sacc[nt][3] = o.w + sacc[nt][3];
+              }
+            }
+            xpar ^= 1;
+          }
+          // ---------------- online softmax (base 2) ----------------
+          const int key0 = logical * kPageTokens + 16 * G + g;  // rows e<2: token g, e>=2: g+8
+          uint32_t pb[NT][2];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            float sv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              sv[e] = sacc[nt][e] * crow[nt][e & 1];
+              if (need_mask && key0 + 8 * (e >> 1) > qpos_row[nt][e & 1]) sv[e] = -INFINITY;
+            }
+            float pr[4];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              float mx = fmaxf(sv[c], sv[c + 2]);
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+              if (mx > m_run[nt][c] + 8.f) {
+                const float alpha = fast_exp2(m_run[nt][c] - mx);
+                l_run[nt][c] *= alpha;
+#pragma unroll
+                for (int mt = 0; mt < 2 * C::kNB; ++mt) {
+                  oacc[mt][nt][c] *= alpha;
+                  oacc[mt][nt][c + 2] *= alpha;
+                }
+                m_run[nt][c] = mx;
+              }
+              const float mu = m_run[nt][c] == -INFINITY ? 0.f : m_run[nt][c];
+              pr[c] = fast_exp2(sv[c] - mu);
+              pr[c + 2] = fast_exp2(sv[c + 2] - mu);
+              l_run[nt][c] += pr[c] + pr[c + 2];
+            }
+            pb[nt][0] = movmatrix_t(pack_half2(pr[0], pr[1]));
+            pb[nt][1] = movmatrix_t(pack_half2(pr[2], pr[3]));
+          }
+          // ---------------- O^T += V^T P^T ----------------
+          if constexpr (!VQ8) {
+#pragma unroll
+            for (int cc = 0; cc < C::kNB / 2; ++cc) {
+              const int Cc = blk0 / 2 + cc;
+              const uint4 vw = lds128(vb + ((((G * 4 + Cc) * 8 + g) * 4 + t) * 16));
+              const uint4 dv = lds128(vb + kV4ScaleOffset + (((G * 4 + t) * 8 + 2 * Cc) * 4) * 2);
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int bl = 2 * cc + e;
+                const uint32_t W0 = e ? vw.z : vw.x, W1 = e ? vw.w : vw.y;
+                const uint32_t d0 = e ? dv.z : dv.x, d1 = e ? dv.w : dv.y;
+                const uint32_t W0s = W0 >> 8, W1s = W1 >> 8;
+                const uint32_t a00 = hsub2(and_or(W0, 0x000F000Fu, kHalf2Magic), kHalf2_1032);
+                const uint32_t a01 = hfma2(and_or(W0, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kHalf2_m72);
+                const uint32_t a02 = hsub2(and_or(W1, 0x000F000Fu, kHalf2Magic), kHalf2_1032);
+                const uint32_t a03 = hfma2(and_or(W1, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kHalf2_m72);
+                const uint32_t a10 = hsub2(and_or(W0s, 0x000F000Fu, kHalf2Magic), kHalf2_1032);
+                const uint32_t a11 = hfma2(and_or(W0s, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kHalf2_m72);
+                const uint32_t a12 = hsub2(and_or(W1s, 0x000F000Fu, kHalf2Magic), kHalf2_1032);
+                const uint32_t a13 = hfma2(and_or(W1s, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kHalf2_m72);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                  const uint32_t b0 = hmul2(pb[nt][0], d0), b1 = hmul2(pb[nt][1], d1);
+                  mma_f16(oacc[2 * bl][nt], a00, a01, a02, a03, b0, b1);
+                  mma_f16(oacc[2 * bl + 1][nt], a10, a11, a12, a13, b0, b1);
+                }
+              }
+            }
+          } else {
+#pragma unroll
+            for (int bl = 0; bl < C::kNB; ++bl) {
+              const int b = blk0 + bl;
+              const uint4 vw = lds128(vb + ((((G * 8 + b) * 8 + g) * 4 + t) * 16));
+              uint32_t d0, d1;
+              asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
+                           : "=r"(d0), "=r"(d1)
+                           : "r"(vb + kV8ScaleOffset + (((G * 4 + t) * 8 + b) * 4) * 2));
+              const uint32_t w[4] = {vw.x ^ 0x80808080u, vw.y ^ 0x80808080u, vw.z ^ 0x80808080u,
+                                     vw.w ^ 0x80808080u};
+              uint32_t a[4][2];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                a[q][0] = hsub2(prmt(w[q], kHalf2Magic, 0x4140u), kHalf2_1152);
+                a[q][1] = hsub2(prmt(w[q], kHalf2Magic, 0x4342u), kHalf2_1152);
+              }
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                const uint32_t b0 = hmul2(pb[nt][0], d0), b1 = hmul2(pb[nt][1], d1);
+                mma_f16(oacc[2 * bl][nt], a[0][0], a[0][1], a[1][0], a[1][1], b0, b1);
+                mma_f16(oacc[2 * bl + 1][nt], a[2][0], a[2][1], a[3][0], a[3][1], b0, b1);
+              }
+            }
+          }
+        }
+      }
+      if (aborted) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    // reduce the per-thread partial sums over the 8 token lanes
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float l = l_run[nt][c];
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        l_run[nt][c] = l;
+      }
+  }
+
+  __syncthreads();
+  if (s_flags[0]) {
+    // A bounded wait expired: wait (bounded) for the copies still in flight, then leave.
+    if (issuer) {
+      for (int pg = next - C::kStages < 0 ? 0 : next - C::kStages; pg < next; ++pg) {
+        const unsigned long long t0 = global_timer_ns();
+        while (!mbar_try_wait(&full[pg % C::kStages], (pg / C::kStages) & 1)) {
+          if (global_timer_ns() - t0 > kWaitTimeoutNs) break;
+        }
+      }
+    }
+    return;
+  }
+
+  // ---------------- merge the CTA's softmax streams in shared memory ----------------
+  // layout: ms[unit][row], ls[unit][row], os[unit][row][256]  (all fp32)
+  float* ms = reinterpret_cast<float*>(smem);
+  float* ls = ms + C::kUnits * C::kRowsPad;
+  float* os = ls + C::kUnits * C::kRowsPad;
+  {
+    const int unit = PAIR ? (warp >> 1) : warp;
+    if (g == 0 && half == 0) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          ms[unit * C::kRowsPad + nt * 8 + 2 * t + c] = m_run[nt][c];
+          ls[unit * C::kRowsPad + nt * 8 + 2 * t + c] = l_run[nt][c];
+        }
+    }
+#pragma unroll
+    for (int mt = 0; mt < 2 * C::kNB; ++mt) {
+      const int b = blk0 + (mt >> 1), hb = mt & 1;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int row = nt * 8 + 2 * t + (e & 1);
+          const int dim = 32 * b + 16 * hb + g + 8 * (e >> 1);
+          os[(unit * C::kRowsPad + row) * kHeadDim + dim] = oacc[mt][nt][e];
+        }
+    }
+  }
+  __syncthreads();
+
+  const bool direct = p.n_splits == 1;
+  float* part_o = p.part_o + (static_cast<long long>(h) * p.n_splits + split) * C::kRowsPad * kHeadDim;
+  float* part_l = p.part_lse + (static_cast<long long>(h) * p.n_splits + split) * C::kRowsPad;
+  for (int idx = threadIdx.x; idx < n_rows * (kHeadDim / 4); idx += C::kThreads) {
+    const int row = idx / (kHeadDim / 4);
+    const int d4 = (idx % (kHeadDim / 4)) * 4;
+    float M = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < C::kUnits; ++u) M = fmaxf(M, ms[u * C::kRowsPad + row]);
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int u = 0; u < C::kUnits; ++u) {
+        const float w = fast_exp2(ms[u * C::kRowsPad + row] - M);
+        L += w * ls[u * C::kRowsPad + row];
+        const float4 o = *reinterpret_cast<const float4*>(os + (u * C::kRowsPad + row) * kHeadDim + d4);
+        acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
+      }
+    }
+    const float invL = L > 0.f ? 1.f / L : 0.f;
+    acc.x *= invL; acc.y *= invL; acc.z *= invL; acc.w *= invL;
+    const float lse2 = L > 0.f ? M + log2f(L) : -INFINITY;
+    if (direct) {
+      const int qi = row / p.group, j = row % p.group;
+      const long long orow = static_cast<long long>(qi) * p.n_qh + h * p.group + j;
+      *reinterpret_cast<float4*>(p.out + orow * kHeadDim + d4) = acc;
+      if (d4 == 0) p.lse[orow] = lse2 * 0.69314718055994531f;
+    } else {
+      *reinterpret_cast<float4*>(part_o + row * kHeadDim + d4) = acc;
+      if (d4 == 0) part_l[row] = lse2;
+    }
+  }
+  if (direct) return;
+
+  // ---------------- last CTA of this KV head merges the splits ----------------
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int prev = atomicAdd(&p.counters[h], 1);
+    s_flags[1] = (prev == p.n_splits - 1);
+  }
+  __syncthreads();
+  if (!s_flags[1]) return;
+  __threadfence();
+  const float* po = p.part_o + static_cast<long long>(h) * p.n_splits * C::kRowsPad * kHeadDim;
+  const float* pl = p.part_lse + static_cast<long long>(h) * p.n_splits * C::kRowsPad;
+  // per-row maxima and normalisers of the split lse values
+  float* rowM = reinterpret_cast<float*>(smem);
+  float* rowL = rowM + C::kRowsPad;
+  for (int row = threadIdx.x; row < n_rows; row += C::kThreads) {
+    float M = -INFINITY;
+    for (int s2 = 0; s2 < p.n_splits; ++s2) M = fmaxf(M, __ldcg(pl + s2 * C::kRowsPad + row));
+    float L = 0.f;
+    if (M != -INFINITY)
+      for (int s2 = 0; s2 < p.n_splits; ++s2) L += fast_exp2(__ldcg(pl + s2 * C::kRowsPad + row) - M);
+    rowM[row] = M;
+    rowL[row] = L;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < n_rows * (kHeadDim / 4); idx += C::kThreads) {
+    const int row = idx / (kHeadDim / 4);
+    const int d4 = (idx % (kHeadDim / 4)) * 4;
+    const float M = rowM[row], L = rowL[row];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+      const float invL = 1.f / L;
+#pragma unroll 8
+      for (int s2 = 0; s2 < p.n_splits; ++s2) {
+        const float w = fast_exp2(__ldcg(pl + s2 * C::kRowsPad + row) - M) * invL;
+        const float4 o = __ldcg(reinterpret_cast<const float4*>(po + (s2 * C::kRowsPad + row) * kHeadDim + d4));
+        acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
+      }
+    }
+    const int qi = row / p.group, j = row % p.group;
+    const long long orow = static_cast<long long>(qi) * p.n_qh + h * p.group + j;
+    *reinterpret_cast<float4*>(p.out + orow * kHeadDim + d4) = acc;
+    if (d4 == 0) p.lse[orow] = M != -INFINITY ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+  }
+  if (threadIdx.x == 0) p.counters[h] = 0;  // ready for the next launch
+}
+
+// ---------------------------------------------------------------------------------------
+template <int NT, bool PAIR, bool VQ8>
+static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream_t stream) {
+  using C = DecodeCfg<NT, PAIR, VQ8>;
+  dim3 grid(prm.n_splits, n_kv);
+  decode_kernel<NT, PAIR, VQ8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(prm);
+  return cudaGetLastError();
+}
+
+int decode_rows_pad(int rows) { return ((rows + 7) / 8) * 8; }
+
+cudaError_t prepare_decode_kernels() {
+  cudaError_t e;
+#define KV_SET(NT, PAIR, VQ8)                                                                   \
+  e = cudaFuncSetAttribute(decode_kernel<NT, PAIR, VQ8>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                           DecodeCfg<NT, PAIR, VQ8>::kSmemBytes);                               \
+  if (e != cudaSuccess) return e;
+  KV_SET(1, false, false) KV_SET(1, false, true) KV_SET(2, true, false) KV_SET(2, true, true)
+  KV_SET(3, true, false) KV_SET(3, true, true)
+#undef KV_SET
+  return cudaSuccess;
+}
+
+cudaError_t launch_decode(const DecodeParams& prm, int n_kv, bool vq8, cudaStream_t stream) {
+  const int nt = decode_rows_pad(prm.group * prm.n_q) / 8;
+  if (nt == 1) return vq8 ? launch_decode_t<1, false, true>(prm, n_kv, stream) : launch_decode_t<1, false, false>(prm, n_kv, stream);
+  if (nt == 2) return vq8 ? launch_decode_t<2, true, true>(prm, n_kv, stream) : launch_decode_t<2, true, false>(prm, n_kv, stream);
+  return vq8 ? launch_decode_t<3, true, true>(prm, n_kv, stream) : launch_decode_t<3, true, false>(prm, n_kv, stream);
+}
+
+}  // namespace kvattn

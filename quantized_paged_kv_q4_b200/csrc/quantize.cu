@@ -1,0 +1,170 @@
+// Q8_0 / Q4_0 encoders that append new tokens into their KV pages.
+//
+// Formats (Vulkan speculative-decoding report, lcz.me/topic/1398, "pitfalls" and
+// "configs"): 32-element blocks with one fp16 scale; Q8_0 stores int8 codes (8.5 bits per
+// element), Q4_0 stores 4-bit codes q with value (q - 8) * d (18 bytes per block).
+// Encoder readings (the pages do not spell them out):
+//   Q8_0: d = amax / 127, q = round-half-away(x * fp32(1/d)), |q| <= 127.
+//   Q4_0: m = the signed element of largest magnitude (first on ties), d = m / -8,
+//         q = min(15, floor(fp32(fp32(x * fp32(1/d)) + 8.5))).
+// Every operation that decides a code is an IEEE fp32 operation with round-to-nearest
+// (no FMA contraction), so the codes equal those of any correct fp32 implementation.
+//
+// One warp encodes one (token, KV head) row: lane l owns channels [8l, 8l+8), four lanes
+// form one 32-element block.
+#include "common.cuh"
+
+namespace kvattn {
+
+__device__ __forceinline__ int q8_code(float x, float inv) {
+  const float y = __fmul_rn(x, inv);
+  float r = roundf(y);  // halves away from zero
+  r = fminf(fmaxf(r, -127.f), 127.f);
+  return static_cast<int>(r);
+}
+
+__device__ __forceinline__ int q4_code(float x, float inv) {
+  const float y = __fmul_rn(x, inv);
+  const float z = __fadd_rn(y, 8.5f);
+  return min(15, __float2int_rz(z));  // z > 0, so truncation is floor
+}
+
+// Q8_0 block scale of this lane's block: returns d (fp32) and writes 1/d to *inv.
+__device__ __forceinline__ float q8_scale(const float (&x)[8], float* inv) {
+  float a = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(x[e]));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+  const float d = __fdiv_rn(a, 127.f);
+  *inv = d != 0.f ? __frcp_rn(d) : 0.f;
+  return d;
+}
+
+__global__ void __launch_bounds__(256) quantize_append_kernel(const float* __restrict__ k,
+                                                              const float* __restrict__ v, int n_tok,
+                                                              int n_kv, int32_t pos0,
+                                                              const int32_t* __restrict__ page_table,
+                                                              int n_blocks, uint8_t* k_pool, int64_t k_stride,
+                                                              uint8_t* v_pool, int64_t v_stride, int64_t n_pages,
+                                                              int v_q8) {
+  const int lane = threadIdx.x & 31;
+  const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (row >= static_cast<long long>(n_tok) * n_kv) return;
+  const int i = static_cast<int>(row / n_kv);
+  const int h = static_cast<int>(row % n_kv);
+  const int32_t pos = pos0 + i;
+  const int blk = pos / kPageTokens;
+  const int tok = pos % kPageTokens;
+  const int page = page_table[static_cast<long long>(h) * n_blocks + blk];
+  if (page < 0 || page >= n_pages) {
+    if (lane == 0) record_error(KVATTN_ERR_BAD_PAGE);
+    return;
+  }
+  const int G = tok >> 4, tl = tok & 15, H = tl >> 3, R = tok & 7;
+  const int b = lane >> 2;  // this lane's block
+
+  // ---------------- K: Q8_0 ----------------
+  {
+    const float4* src = reinterpret_cast<const float4*>(k + row * kHeadDim + lane * 8);
+    const float4 x0 = src[0], x1 = src[1];
+    const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    float inv;
+    const float d = q8_scale(x, &inv);
+    uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w0 |= (static_cast<uint32_t>(q8_code(x[e], inv)) & 0xFFu) << (8 * e);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w1 |= (static_cast<uint32_t>(q8_code(x[4 + e], inv)) & 0xFFu) << (8 * e);
+    uint8_t* pg = k_pool + static_cast<int64_t>(page) * k_stride;
+    const int P = lane >> 3, T = lane & 3, jhi = (lane & 7) >> 2;
+    const int off = ((((G * 4 + P) * 2 + H) * 8 + R) * 4 + T) * 16 + 8 * jhi;
+    *reinterpret_cast<uint2*>(pg + off) = make_uint2(w0, w1);
+    if ((lane & 3) == 0) {
+      const int so = kKScaleOffset + 2 * (((G * 8 + R) * 2 + H) * 8 + b);
+      *reinterpret_cast<__half*>(pg + so) = __float2half_rn(d);
+    }
+  }
+
+  // ---------------- V: Q4_0 or Q8_0 ----------------
+  {
+    const float4* src = reinterpret_cast<const float4*>(v + row * kHeadDim + lane * 8);
+    const float4 x0 = src[0], x1 = src[1];
+    const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    uint8_t* pg = v_pool + static_cast<int64_t>(page) * v_stride;
+    const int T = (tl & 7) >> 1, wlo = tl >> 3, ylo = tl & 1;
+    const int k_slot = ylo + 2 * wlo;
+    const int cl = lane & 3;  // which 8-channel group of the block
+    float d;
+    int codes[8];
+    if (!v_q8) {
+      // signed element of largest magnitude, first index on ties
+      float best = x[0];
+      int bidx = lane * 8;
+#pragma unroll
+      for (int e = 1; e < 8; ++e)
+        if (fabsf(x[e]) > fabsf(best)) {
+          best = x[e];
+          bidx = lane * 8 + e;
+        }
+#pragma unroll
+      for (int s = 1; s <= 2; s <<= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, best, s);
+        const int oi = __shfl_xor_sync(0xffffffffu, bidx, s);
+        if (fabsf(ob) > fabsf(best) || (fabsf(ob) == fabsf(best) && oi < bidx)) {
+          best = ob;
+          bidx = oi;
+        }
+      }
+      d = __fdiv_rn(best, -8.f);
+      const float inv = d != 0.f ? __frcp_rn(d) : 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) codes[e] = q4_code(x[e], inv);
+      // lanes cl = 0,1 share bytes (lo, hi nibble) with y%2 = 0; lanes 2,3 with y%2 = 1
+      int other[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) other[e] = __shfl_xor_sync(0xffffffffu, codes[e], 1);
+      if ((cl & 1) == 0) {
+        const int C = b >> 1, w = 2 * (b & 1) + wlo, y = 2 * ylo + (cl >> 1);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int off = ((((G * 4 + C) * 8 + e) * 4 + T) * 16) + 4 * w + y;
+          pg[off] = static_cast<uint8_t>(codes[e] | (other[e] << 4));
+        }
+      }
+      if (cl == 0) {
+        const int so = kV4ScaleOffset + 2 * (((G * 4 + T) * 8 + b) * 4 + k_slot);
+        *reinterpret_cast<__half*>(pg + so) = __float2half_rn(d);
+      }
+    } else {
+      float inv;
+      d = q8_scale(x, &inv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) codes[e] = q8_code(x[e], inv);
+      const int w = 2 * (cl >> 1) + wlo, y = 2 * (cl & 1) + ylo;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int off = ((((G * 8 + b) * 8 + e) * 4 + T) * 16) + 4 * w + y;
+        pg[off] = static_cast<uint8_t>(codes[e] & 0xFF);
+      }
+      if (cl == 0) {
+        const int so = kV8ScaleOffset + 2 * (((G * 4 + T) * 8 + b) * 4 + k_slot);
+        *reinterpret_cast<__half*>(pg + so) = __float2half_rn(d);
+      }
+    }
+  }
+}
+
+cudaError_t launch_quantize_append(const kvattn_kv_desc& desc, const float* k, const float* v, int n_tok,
+                                   int32_t pos0, const int32_t* page_table, int n_blocks, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(n_tok) * desc.n_kv_heads;
+  const int warps_per_block = 8;
+  const long long grid = (rows + warps_per_block - 1) / warps_per_block;
+  quantize_append_kernel<<<static_cast<unsigned>(grid), 32 * warps_per_block, 0, stream>>>(
+      k, v, n_tok, desc.n_kv_heads, pos0, page_table, n_blocks, static_cast<uint8_t*>(desc.k_pool),
+      desc.k_page_stride, static_cast<uint8_t*>(desc.v_pool), desc.v_page_stride, desc.n_pages,
+      desc.v_fmt == KVATTN_FMT_Q8_0);
+  return cudaGetLastError();
+}
+
+}  // namespace kvattn

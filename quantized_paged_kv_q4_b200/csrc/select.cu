@@ -1,0 +1,222 @@
+// KVMem-style block summaries and top-k block selection (KVMem reproduction on one
+// 7900 XTX, lcz.me/topic/1972: 128-token blocks; a retrieval query chooses which blocks
+// fill a 32,768-token GPU budget, and a 16,384-token recent reserve is always kept).
+//
+// Readings (the pages do not define the ranking):
+//   summary[b][c] = mean over the block's 128 tokens of the dequantized key, rounded once
+//                   to fp32.  Computed exactly: each fp16 scale is split into an 11-bit
+//                   integer significand and an exponent, every code x significand product is
+//                   shifted onto a common 2^-24 grid and summed in int64 (< 2^54, no
+//                   overflow), then converted to fp32 with one rounding.
+//   score[b]      = sum_c (sum_j q[j][c]) * summary[b][c] in fp64.
+//   selection     = the `budget` highest scores among blocks older than the recent window
+//                   (ties: lower block index), plus the recent window and partial tail
+//                   blocks, written in ascending order.
+#include "common.cuh"
+
+namespace kvattn {
+
+// ---------------------------------------------------------------- summaries
+__global__ void __launch_bounds__(256) block_summary_kernel(const uint8_t* __restrict__ k_pool, int64_t k_stride,
+                                                            int64_t n_pages, const int32_t* __restrict__ page_table,
+                                                            int n_blocks, int block_begin, int n_range,
+                                                            float* __restrict__ summaries) {
+  __shared__ __align__(16) uint8_t page[kKPageBytes];
+  const int unit = blockIdx.y;
+  const int b = block_begin + blockIdx.x;
+  const int pg = page_table[static_cast<long long>(unit) * n_blocks + b];
+  if (pg < 0 || pg >= n_pages) {
+    if (threadIdx.x == 0) record_error(KVATTN_ERR_BAD_PAGE);
+    return;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(k_pool + static_cast<int64_t>(pg) * k_stride);
+  uint4* dst = reinterpret_cast<uint4*>(page);
+  for (int i = threadIdx.x; i < kKPageBytes / 16; i += blockDim.x) dst[i] = src[i];
+  __syncthreads();
+  const int c = threadIdx.x;  // channel
+  const int blk = c >> 5;
+  const int P = c >> 6, cc = c & 63, T = (cc & 31) >> 3, j = 8 * (cc >> 5) + (cc & 7);
+  long long acc = 0;
+  for (int tok = 0; tok < kPageTokens; ++tok) {
+    const int G = tok >> 4, H = (tok & 15) >> 3, R = tok & 7;
+    const int q = static_cast<int8_t>(page[((((G * 4 + P) * 2 + H) * 8 + R) * 4 + T) * 16 + j]);
+    const uint16_t hb = *reinterpret_cast<const uint16_t*>(page + kKScaleOffset + 2 * (((G * 8 + R) * 2 + H) * 8 + blk));
+    const int e = (hb >> 10) & 31;
+    const int mant = hb & 1023;
+    const int m = e ? (1024 | mant) : mant;
+    const int eff = e ? e : 1;
+    const long long term = static_cast<long long>(q * m) * (1ll << (eff - 1));
+    acc += (hb & 0x8000) ? -term : term;
+  }
+  // value = acc * 2^-24 / 128
+  const float r = __ll2float_rn(acc) * 4.656612873077392578125e-10f;  // 2^-31
+  summaries[(static_cast<long long>(unit) * n_blocks + b) * kHeadDim + c] = r;
+}
+
+// ---------------------------------------------------------------- scores
+__global__ void __launch_bounds__(256) block_score_kernel(const float* __restrict__ summaries,
+                                                          const float* __restrict__ q_group, int group, int n_blocks,
+                                                          int n_cand, double* __restrict__ scores) {
+  const int unit = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (b >= n_cand) return;
+  const float* qg = q_group + static_cast<long long>(unit) * group * kHeadDim;
+  const float* sm = summaries + (static_cast<long long>(unit) * n_blocks + b) * kHeadDim;
+  double acc = 0.0;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int c0 = lane * 4 + 128 * k;
+    const float4 sv = *reinterpret_cast<const float4*>(sm + c0);
+    double u[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int j = 0; j < group; ++j) {
+      const float4 qv = *reinterpret_cast<const float4*>(qg + j * kHeadDim + c0);
+      u[0] += qv.x; u[1] += qv.y; u[2] += qv.z; u[3] += qv.w;
+    }
+    acc = fma(u[0], static_cast<double>(sv.x), acc);
+    acc = fma(u[1], static_cast<double>(sv.y), acc);
+    acc = fma(u[2], static_cast<double>(sv.z), acc);
+    acc = fma(u[3], static_cast<double>(sv.w), acc);
+  }
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (lane == 0) scores[static_cast<long long>(unit) * n_blocks + b] = acc;
+}
+
+// ---------------------------------------------------------------- top-k + compaction
+__device__ __forceinline__ unsigned long long order_key(double x) {
+  unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(x));
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+constexpr int kSelThreads = 1024;
+constexpr int kMaxCand = 16384;
+constexpr int kMaxTotal = 65536;
+
+__global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const double* __restrict__ scores, int n_blocks,
+                                                                 int n_cand, int n_total, int budget,
+                                                                 const int32_t* __restrict__ page_table,
+                                                                 int32_t* __restrict__ sel_logical,
+                                                                 int32_t* __restrict__ sel_phys,
+                                                                 int32_t* __restrict__ n_sel, int cap) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int unit = blockIdx.x;
+  int npad = 1;
+  while (npad < n_cand) npad <<= 1;
+  unsigned long long* key = reinterpret_cast<unsigned long long*>(sm);
+  int* idx = reinterpret_cast<int*>(key + npad);
+  int* counts = idx + npad;                                   // [kSelThreads + 1]
+  uint32_t* bits = reinterpret_cast<uint32_t*>(counts + kSelThreads + 1);  // [n_total / 32]
+  const double* sc = scores + static_cast<long long>(unit) * n_blocks;
+  for (int i = threadIdx.x; i < npad; i += kSelThreads) {
+    if (i < n_cand) {
+      key[i] = order_key(sc[i]);
+      idx[i] = i;
+    } else {
+      key[i] = 0ull;
+      idx[i] = INT_MAX;
+    }
+  }
+  __syncthreads();
+  // bitonic sort: descending key, ascending index
+  for (int k = 2; k <= npad; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < npad; i += kSelThreads) {
+        const int l = i ^ j;
+        if (l > i) {
+          const unsigned long long ki = key[i], kl = key[l];
+          const int ii = idx[i], il = idx[l];
+          const bool i_first = ki > kl || (ki == kl && ii < il);  // i precedes l in the target order
+          const bool up = (i & k) == 0;
+          if (up != i_first) {
+            key[i] = kl; key[l] = ki;
+            idx[i] = il; idx[l] = ii;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // mark the chosen candidates in a bitmap over [0, n_total)
+  const int take = min(budget, n_cand);
+  const int* chosen = idx;
+  const int words = (n_total + 31) / 32;
+  for (int w = threadIdx.x; w < words; w += kSelThreads) bits[w] = 0u;
+  __syncthreads();
+  for (int i = threadIdx.x; i < take; i += kSelThreads) atomicOr(&bits[chosen[i] >> 5], 1u << (chosen[i] & 31));
+  for (int b = n_cand + threadIdx.x; b < n_total; b += kSelThreads) atomicOr(&bits[b >> 5], 1u << (b & 31));
+  __syncthreads();
+  // each thread owns a contiguous range of words; exclusive scan of their popcounts
+  const int per = (words + kSelThreads - 1) / kSelThreads;
+  const int w0 = threadIdx.x * per, w1 = min(words, w0 + per);
+  int cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
+  counts[threadIdx.x] = cnt;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int i = 0; i < kSelThreads; ++i) {
+      const int c = counts[i];
+      counts[i] = run;
+      run += c;
+    }
+    counts[kSelThreads] = run;
+  }
+  __syncthreads();
+  int pos = counts[threadIdx.x];
+  const int total = counts[kSelThreads];
+  int32_t* out_l = sel_logical + static_cast<long long>(unit) * cap;
+  int32_t* out_p = sel_phys + static_cast<long long>(unit) * cap;
+  const int32_t* pt = page_table + static_cast<long long>(unit) * n_blocks;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t m = bits[w];
+    while (m) {
+      const int bit = __ffs(m) - 1;
+      m &= m - 1;
+      const int b = w * 32 + bit;
+      if (pos < cap) {
+        out_l[pos] = b;
+        out_p[pos] = pt[b];
+      }
+      ++pos;
+    }
+  }
+  if (threadIdx.x == 0) n_sel[unit] = min(total, cap);
+}
+
+cudaError_t launch_block_summaries(const kvattn_kv_desc& d, const int32_t* page_table, int n_units, int n_blocks,
+                                   int block_begin, int block_end, float* summaries, cudaStream_t stream) {
+  const int n = block_end - block_begin;
+  if (n <= 0 || n_units <= 0) return cudaSuccess;
+  dim3 grid(n, n_units);
+  block_summary_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(d.k_pool), d.k_page_stride, d.n_pages,
+                                                 page_table, n_blocks, block_begin, n, summaries);
+  return cudaGetLastError();
+}
+
+size_t select_smem_bytes(int n_cand, int n_total) {
+  int npad = 1;
+  while (npad < n_cand) npad <<= 1;
+  return static_cast<size_t>(npad) * 12 + (kSelThreads + 1) * 4 + static_cast<size_t>((n_total + 31) / 32) * 4;
+}
+
+cudaError_t prepare_select_kernels() {
+  return cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(select_smem_bytes(kMaxCand, kMaxTotal)));
+}
+
+cudaError_t launch_select(const float* summaries, const float* q_group, int n_units, int group, int n_blocks,
+                          int n_cand, int n_total, int budget, const int32_t* page_table, int32_t* sel_logical,
+                          int32_t* sel_phys, int32_t* n_sel, int cap, double* scores, cudaStream_t stream) {
+  if (n_cand > 0) {
+    dim3 grid((n_cand + 7) / 8, n_units);
+    block_score_kernel<<<grid, 256, 0, stream>>>(summaries, q_group, group, n_blocks, n_cand, scores);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  select_topk_kernel<<<n_units, kSelThreads, select_smem_bytes(max(n_cand, 1), n_total), stream>>>(
+      scores, n_blocks, n_cand, n_total, budget, page_table, sel_logical, sel_phys, n_sel, cap);
+  return cudaGetLastError();
+}
+
+}  // namespace kvattn

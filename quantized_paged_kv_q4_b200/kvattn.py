@@ -1,0 +1,241 @@
+"""Thin ctypes binding of libkvattn (include/kvattn.h).
+
+Argument marshalling only: every computation runs in the CUDA library.  Pointer arguments
+accept torch tensors (their data_ptr), plain integers (raw addresses) or None; stream
+arguments accept torch.cuda.Stream objects, raw handles or None (the current torch
+stream).  A nonzero status raises KVAttnError.  If libkvattn.so is missing the import of
+any entry point fails loudly: there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_int, c_int32, c_int64, c_size_t, c_uint16, c_void_p
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkvattn.so")
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED_ARCH = -2
+ERR_UNSUPPORTED_FORMAT = -3
+ERR_BAD_PAGE = -4
+ERR_WORKSPACE_TOO_SMALL = -5
+ERR_CUDA = -6
+ERR_TIMEOUT = -7
+ERR_UNSUPPORTED_SHAPE = -8
+ERR_NOT_INITIALIZED = -9
+
+FMT_Q4_0 = 4
+FMT_Q8_0 = 8
+ROLE_K = 0
+ROLE_V = 1
+FMT = {"q4_0": FMT_Q4_0, "q8_0": FMT_Q8_0}
+
+
+class KVAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+class kvattn_kv_desc(ctypes.Structure):
+    _fields_ = [
+        ("n_kv_heads", c_int32), ("n_q_heads", c_int32), ("head_dim", c_int32), ("page_tokens", c_int32),
+        ("k_fmt", c_int32), ("v_fmt", c_int32), ("k_pool", c_void_p), ("v_pool", c_void_p),
+        ("k_page_stride", c_int64), ("v_page_stride", c_int64), ("n_pages", c_int64),
+    ]
+
+
+_SIGS = {
+    "kvattn_init": (c_int, [c_int]),
+    "kvattn_status_string": (ctypes.c_char_p, [c_int]),
+    "kvattn_last_cuda_error": (c_int, []),
+    "kvattn_device_error": (c_int, [c_void_p]),
+    "kvattn_page_bytes": (c_int64, [c_int, c_int]),
+    "kvattn_quantize_append": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_void_p, c_int, c_int32, c_void_p, c_int,
+                                       c_void_p]),
+    "kvattn_decode_workspace_size": (c_size_t, [POINTER(kvattn_kv_desc), c_int, c_int]),
+    "kvattn_decode": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                              c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "kvattn_merge_lse": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+    "kvattn_block_summaries": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_int, c_int, c_int, c_int, c_void_p,
+                                       c_void_p]),
+    "kvattn_select_workspace_size": (c_size_t, [c_int, c_int]),
+    "kvattn_select_blocks": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p,
+                                     c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
+    "kvattn_prefill_workspace_size": (c_size_t, [POINTER(kvattn_kv_desc), c_int, c_int, c_int]),
+    "kvattn_prefill_chunk": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                     c_int, c_int, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "kvattn_stream_pages": (c_int, [c_void_p, c_int64, c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_int,
+                                    c_void_p, c_void_p, POINTER(c_int)]),
+    "kvattn_stream_plan": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int]),
+    "kvattn_stream_wait": (c_int, [c_void_p, c_int]),
+}
+
+_lib = None
+
+
+def lib():
+    """The loaded libkvattn.so (raises if it was never built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with quantized_paged_kv_q4_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _p(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _s(stream):
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, what: str) -> int:
+    if status != OK:
+        raise KVAttnError(status, what)
+    return status
+
+
+def status_string(status: int) -> str:
+    return lib().kvattn_status_string(status).decode()
+
+
+def make_desc(n_kv_heads, n_q_heads, k_pool, v_pool, n_pages, v_fmt="q4_0", k_page_stride=None,
+              v_page_stride=None, head_dim=256, page_tokens=128, k_fmt="q8_0") -> kvattn_kv_desc:
+    kf, vf = FMT[k_fmt] if isinstance(k_fmt, str) else k_fmt, FMT[v_fmt] if isinstance(v_fmt, str) else v_fmt
+    return kvattn_kv_desc(n_kv_heads, n_q_heads, head_dim, page_tokens, kf, vf, _p(k_pool), _p(v_pool),
+                          k_page_stride or kvattn_page_bytes(ROLE_K, kf), v_page_stride or kvattn_page_bytes(ROLE_V, vf),
+                          n_pages)
+
+
+# ---------------------------------------------------------------- entry points
+def kvattn_init(device: int = 0) -> None:
+    _check(lib().kvattn_init(device), "kvattn_init")
+
+
+def kvattn_last_cuda_error() -> int:
+    return lib().kvattn_last_cuda_error()
+
+
+def kvattn_device_error(stream=None) -> int:
+    """Returns (and clears) the device error word; does not raise for BAD_PAGE/TIMEOUT."""
+    st = lib().kvattn_device_error(_s(stream))
+    if st in (ERR_CUDA, ERR_NOT_INITIALIZED):
+        raise KVAttnError(st, "kvattn_device_error")
+    return st
+
+
+def kvattn_page_bytes(role: int, fmt: int) -> int:
+    return lib().kvattn_page_bytes(role, fmt)
+
+
+def kvattn_quantize_append(desc, k, v, n_tok, pos0, page_table, n_blocks, stream=None) -> None:
+    _check(lib().kvattn_quantize_append(ctypes.byref(desc), _p(k), _p(v), n_tok, pos0, _p(page_table), n_blocks,
+                                        _s(stream)), "kvattn_quantize_append")
+
+
+def kvattn_decode_workspace_size(desc, n_q, max_pages) -> int:
+    return lib().kvattn_decode_workspace_size(ctypes.byref(desc), n_q, max_pages)
+
+
+def kvattn_decode(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pages, out, lse, ws, ws_bytes,
+                  stream=None) -> None:
+    _check(lib().kvattn_decode(ctypes.byref(desc), _p(q), n_q, _p(q_pos), _p(page_list), _p(page_logical),
+                               _p(n_pages), max_pages, _p(out), _p(lse), _p(ws), ws_bytes, _s(stream)),
+           "kvattn_decode")
+
+
+def kvattn_merge_lse(o_parts, lse_parts, n_parts, rows, dim, out, lse, stream=None) -> None:
+    _check(lib().kvattn_merge_lse(_p(o_parts), _p(lse_parts), n_parts, rows, dim, _p(out), _p(lse), _s(stream)),
+           "kvattn_merge_lse")
+
+
+def kvattn_block_summaries(desc, page_table, n_units, n_blocks, block_begin, block_end, summaries,
+                           stream=None) -> None:
+    _check(lib().kvattn_block_summaries(ctypes.byref(desc), _p(page_table), n_units, n_blocks, block_begin,
+                                        block_end, _p(summaries), _s(stream)), "kvattn_block_summaries")
+
+
+def kvattn_select_workspace_size(n_units, n_blocks) -> int:
+    return lib().kvattn_select_workspace_size(n_units, n_blocks)
+
+
+def kvattn_select_blocks(summaries, q_group, n_units, group, n_blocks, n_full, n_total, budget, recent, page_table,
+                         sel_logical, sel_phys, n_sel, cap, ws, ws_bytes, stream=None) -> None:
+    _check(lib().kvattn_select_blocks(_p(summaries), _p(q_group), n_units, group, n_blocks, n_full, n_total, budget,
+                                      recent, _p(page_table), _p(sel_logical), _p(sel_phys), _p(n_sel), cap, _p(ws),
+                                      ws_bytes, _s(stream)), "kvattn_select_blocks")
+
+
+def kvattn_prefill_workspace_size(desc, n_q, max_pages, kv_split_tokens) -> int:
+    return lib().kvattn_prefill_workspace_size(ctypes.byref(desc), n_q, max_pages, kv_split_tokens)
+
+
+def kvattn_prefill_chunk(desc, q_bf16, n_q, q_pos, page_list, page_logical, n_pages, max_pages, kv_split_tokens, out,
+                         lse, ws, ws_bytes, stream=None) -> None:
+    _check(lib().kvattn_prefill_chunk(ctypes.byref(desc), _p(q_bf16), n_q, _p(q_pos), _p(page_list),
+                                      _p(page_logical), _p(n_pages), max_pages, kv_split_tokens, _p(out), _p(lse),
+                                      _p(ws), ws_bytes, _s(stream)), "kvattn_prefill_chunk")
+
+
+def _host_i32(a):
+    import numpy as np
+
+    arr = np.ascontiguousarray(a, dtype=np.int32)
+    return arr, arr.ctypes.data
+
+
+def kvattn_stream_plan(host_ids, dev_slots):
+    """Returns the list of (first index, length) copy runs kvattn_stream_pages would issue."""
+    import numpy as np
+
+    h, hp = _host_i32(host_ids)
+    d, dp = _host_i32(dev_slots)
+    n = int(h.size)
+    first = np.zeros(max(n, 1), np.int32)
+    length = np.zeros(max(n, 1), np.int32)
+    runs = lib().kvattn_stream_plan(hp, dp, n, first.ctypes.data, length.ctypes.data, n)
+    if runs < 0:
+        raise KVAttnError(runs, "kvattn_stream_plan")
+    return list(zip(first[:runs].tolist(), length[:runs].tolist()))
+
+
+def kvattn_stream_pages(host_pool, host_stride, dev_pool, dev_stride, page_bytes, host_ids, dev_slots,
+                        copy_stream=None, done=None) -> int:
+    """host_ids / dev_slots are host sequences; returns the number of copies issued."""
+    h, hp = _host_i32(host_ids)
+    d, dp = _host_i32(dev_slots)
+    n_copies = c_int(0)
+    ev = None if done is None else (done if isinstance(done, int) else done.cuda_event)
+    _check(lib().kvattn_stream_pages(_p(host_pool), host_stride, _p(dev_pool), dev_stride, page_bytes, hp, dp,
+                                     int(h.size), _s(copy_stream), ev, ctypes.byref(n_copies)),
+           "kvattn_stream_pages")
+    return n_copies.value
+
+
+def kvattn_stream_wait(event, timeout_ms: int) -> int:
+    """Returns OK or ERR_TIMEOUT; raises on other errors."""
+    ev = event if isinstance(event, int) else event.cuda_event
+    st = lib().kvattn_stream_wait(ev, timeout_ms)
+    if st not in (OK, ERR_TIMEOUT):
+        raise KVAttnError(st, "kvattn_stream_wait")
+    return st

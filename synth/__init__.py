@@ -167,3 +167,23 @@ WORKLOADS = {
     "stream524k": Workload("stream524k", layers=16, kv_heads=4, q_heads=24, context=524288, n_q=1,
                            budget_blocks=256, recent_blocks=0, steps=512, seed=5005),
 }
+
+
+def plant_needles_torch(k, blocks, direction, seed: int, cosine: float = 0.9, page_tokens: int = PAGE_TOKENS):
+    """Device version of plant_needles for multi-GB caches.
+
+    k: torch fp32 [T][D] view of one (layer, KV head) (modified in place); blocks: iterable of
+    block indices; direction: torch [D].  Random orthogonal parts come from torch_normal(seed)."""
+    import torch
+
+    u = direction.to(torch.float64)
+    u = u / torch.linalg.norm(u)
+    s = math.sqrt(1.0 - cosine * cosine)
+    idx = torch.as_tensor([int(b) for b in blocks], device=k.device, dtype=torch.int64)
+    rows = (idx[:, None] * page_tokens + torch.arange(page_tokens, device=k.device)[None, :]).reshape(-1)
+    kb = k[rows].to(torch.float64)
+    norms = torch.linalg.norm(kb, dim=1, keepdim=True)
+    w = torch_normal(seed, kb.shape, k.device, torch.float64)
+    w = w - (w @ u)[:, None] * u[None, :]
+    w = w / torch.linalg.norm(w, dim=1, keepdim=True)
+    k[rows] = (norms * (cosine * u[None, :] + s * w)).to(torch.float32)

@@ -1,0 +1,111 @@
+"""Shared helpers of the GPU parity tests: cache construction through the CUDA library and
+the oracle's view of the same seeded inputs.  Imported by tests only."""
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import attention as oatt
+from oracle import layout as olay
+from oracle import quant as oq
+
+ATOL = 2e-3      # max abs error on fp32 outputs (the target's tolerance)
+RTOL_GATE = 2e-3  # internal gate on ||o_gpu - o_ref|| / ||o_ref||
+
+
+def torch_mod():
+    import torch
+
+    return torch
+
+
+def lib():
+    from quantized_paged_kv_q4_b200 import kvattn
+
+    return kvattn
+
+
+class GpuCache:
+    """Device page pools for one layer (H_kv units) filled through kvattn_quantize_append."""
+
+    def __init__(self, H_kv, H_q, n_blocks, v_fmt="q4_0", n_phys=None, perm=None, device="cuda"):
+        torch = torch_mod()
+        kv = lib()
+        self.H_kv, self.H_q, self.n_blocks, self.v_fmt = H_kv, H_q, n_blocks, v_fmt
+        self.n_phys = n_phys or H_kv * n_blocks
+        kb = olay.page_bytes("k", "q8_0")
+        vb = olay.page_bytes("v", v_fmt)
+        self.k_pool = torch.zeros((self.n_phys, kb), dtype=torch.uint8, device=device)
+        self.v_pool = torch.zeros((self.n_phys, vb), dtype=torch.uint8, device=device)
+        if perm is None:
+            perm = np.arange(self.n_phys, dtype=np.int32)
+        self.page_table_np = np.asarray(perm[: H_kv * n_blocks], dtype=np.int32).reshape(H_kv, n_blocks)
+        self.page_table = torch.from_numpy(self.page_table_np.copy()).to(device)
+        self.desc = kv.make_desc(H_kv, H_q, self.k_pool, self.v_pool, self.n_phys, v_fmt=v_fmt)
+
+    def append(self, k, v, pos0):
+        """k, v: fp32 arrays [n][H_kv][256] (numpy or torch)."""
+        torch = torch_mod()
+        kt = torch.as_tensor(np.ascontiguousarray(k) if isinstance(k, np.ndarray) else k).to("cuda").contiguous()
+        vt = torch.as_tensor(np.ascontiguousarray(v) if isinstance(v, np.ndarray) else v).to("cuda").contiguous()
+        lib().kvattn_quantize_append(self.desc, kt, vt, kt.shape[0], pos0, self.page_table, self.n_blocks)
+
+
+class OracleCache:
+    """The oracle's quantised view of one layer: codes and scales per unit and token."""
+
+    def __init__(self, k, v, v_fmt="q4_0"):
+        # k, v: fp32 [T][H_kv][256]
+        self.v_fmt = v_fmt
+        self.kc, self.kd = oq.q8_0_quantize(np.asarray(k, np.float32))          # [T][H][8][32], [T][H][8]
+        self.vc, self.vd = oq.quantize(np.asarray(v, np.float32), v_fmt)
+        self.T = k.shape[0]
+
+    def khat(self, h):
+        return oq.q8_0_dequantize(self.kc[:, h], self.kd[:, h])
+
+    def vhat(self, h):
+        return oq.dequantize(self.vc[:, h], self.vd[:, h], self.v_fmt)
+
+    def page_bytes(self, h, blk, role):
+        """Expected bytes of logical block `blk` of unit h (tokens beyond T stay zero codes)."""
+        a, b = blk * 128, min((blk + 1) * 128, self.T)
+        if role == "k":
+            codes = np.zeros((128, 8, 32), np.int8)
+            d = np.zeros((128, 8), np.float16)
+            codes[: b - a] = self.kc[a:b, h]
+            d[: b - a] = self.kd[a:b, h]
+            return olay.encode_page("k", "q8_0", codes, d)
+        codes = np.zeros((128, 8, 32), np.int8 if self.v_fmt == "q8_0" else np.uint8)
+        d = np.zeros((128, 8), np.float16)
+        codes[: b - a] = self.vc[a:b, h]
+        d[: b - a] = self.vd[a:b, h]
+        return olay.encode_page("v", self.v_fmt, codes, d)
+
+    def attend(self, q, q_pos, h, group, key_idx=None):
+        """q: [n_q][H_q][256]; returns (o [n_q][group][256], lse [n_q][group]) for KV head h."""
+        n_q = q.shape[0]
+        rows = np.concatenate([q[i, h * group:(h + 1) * group] for i in range(n_q)], 0)
+        qp = np.repeat(np.asarray(q_pos), group)
+        kh, vh = self.khat(h), self.vhat(h)
+        pos = np.arange(self.T)
+        if key_idx is not None:
+            kh, vh, pos = kh[key_idx], vh[key_idx], pos[key_idx]
+        o, l = oatt.attend(rows, kh, vh, pos, qp, 1.0 / 16.0)
+        return o.reshape(n_q, group, -1), l.reshape(n_q, group)
+
+
+def compare(o_gpu, lse_gpu, o_ref, lse_ref):
+    """Asserts the tolerance; returns (max_abs, rel, lse_abs)."""
+    o_gpu = np.asarray(o_gpu, np.float64)
+    o_ref = np.asarray(o_ref, np.float64)
+    err = np.abs(o_gpu - o_ref)
+    max_abs = float(err.max()) if err.size else 0.0
+    rel = float(np.linalg.norm(o_gpu - o_ref) / max(np.linalg.norm(o_ref), 1e-30))
+    lg, lr = np.asarray(lse_gpu, np.float64), np.asarray(lse_ref, np.float64)
+    both_inf = np.isneginf(lg) & np.isneginf(lr)
+    assert np.array_equal(np.isneginf(lg), np.isneginf(lr)), "masked rows differ"
+    lse_abs = float(np.abs(np.where(both_inf, 0, lg - lr)).max()) if lg.size else 0.0
+    assert max_abs <= ATOL, f"max abs error {max_abs}"
+    assert rel <= RTOL_GATE, f"relative error {rel}"
+    assert lse_abs <= ATOL, f"lse error {lse_abs}"
+    return max_abs, rel, lse_abs

@@ -1,0 +1,139 @@
+"""GPU: split-KV decode / MTP verify against the oracle (max abs 2e-3, relative gate)."""
+import numpy as np
+import pytest
+import torch
+
+from helpers_kv import GpuCache, OracleCache, compare
+from synth import normal_f32, np_rng, page_permutation
+
+pytestmark = pytest.mark.gpu
+
+
+def _layer(seed, H, T, v_fmt, n_blocks=None, spare=0, outliers=True):
+    rng = np_rng(seed)
+    k = normal_f32(rng, (T, H, 256))
+    v = normal_f32(rng, (T, H, 256))
+    if outliers:
+        for h in range(H):
+            ch = rng.choice(256, 3, replace=False)
+            k[:, h, ch] *= 8
+            v[:, h, ch] *= 8
+    n_blocks = n_blocks or (T + 127) // 128
+    n_phys = H * n_blocks + spare
+    cache = GpuCache(H, 0, n_blocks, v_fmt, n_phys=n_phys, perm=page_permutation(rng, n_phys))
+    return rng, k, v, cache
+
+
+def _run_decode(kv, cache, H_q, q, q_pos, page_list, page_logical=None, n_pages=None, max_pages=None):
+    cache.desc.n_q_heads = H_q
+    n_q = q.shape[0]
+    max_pages = page_list.shape[1] if max_pages is None else max_pages
+    qd = torch.from_numpy(np.ascontiguousarray(q)).cuda()
+    qp = torch.tensor(q_pos, dtype=torch.int32, device="cuda")
+    out = torch.full((n_q, H_q, 256), float("nan"), device="cuda")
+    lse = torch.full((n_q, H_q), float("nan"), device="cuda")
+    wsb = kv.kvattn_decode_workspace_size(cache.desc, n_q, max_pages)
+    ws = torch.zeros(max(wsb, 256), dtype=torch.uint8, device="cuda")
+    pl = torch.as_tensor(page_list, dtype=torch.int32).cuda() if page_list is not None else None
+    lg = torch.as_tensor(page_logical, dtype=torch.int32).cuda() if page_logical is not None else None
+    npg = torch.as_tensor(n_pages, dtype=torch.int32).cuda() if n_pages is not None else None
+    kv.kvattn_decode(cache.desc, qd, n_q, qp, pl, lg, npg, max_pages, out, lse, ws, wsb)
+    torch.cuda.synchronize()
+    return out.cpu().numpy(), lse.cpu().numpy(), (qd, qp, pl, lg, npg, out, lse, ws, wsb)
+
+
+@pytest.mark.parametrize("v_fmt", ["q4_0", "q8_0"])
+@pytest.mark.parametrize("n_q", [1, 2, 3, 4])
+def test_decode_matches_oracle(kv_gpu, v_fmt, n_q):
+    H, H_q, T = 4, 24, 37 * 128 + 77          # ragged tail page
+    rng, k, v, cache = _layer(600 + n_q, H, T, v_fmt, spare=5)
+    cache.append(k, v, 0)
+    q = normal_f32(rng, (n_q, H_q, 256))
+    q_pos = [T - n_q + i for i in range(n_q)]
+    out, lse, keep = _run_decode(kv_gpu, cache, H_q, q, q_pos, cache.page_table_np)
+    oc = OracleCache(k, v, v_fmt)
+    for h in range(H):
+        o_ref, l_ref = oc.attend(q, q_pos, h, 6)
+        compare(out[:, 6 * h:6 * h + 6], lse[:, 6 * h:6 * h + 6], o_ref, l_ref)
+    # a second launch reuses the workspace (split counters are left at zero) bit-identically
+    qd, qp, pl, lg, npg, o2, l2, ws, wsb = keep
+    kv_gpu.kvattn_decode(cache.desc, qd, n_q, qp, pl, lg, npg, pl.shape[1], o2, l2, ws, wsb)
+    torch.cuda.synchronize()
+    assert np.array_equal(o2.cpu().numpy(), out) and np.array_equal(l2.cpu().numpy(), lse)
+
+
+def test_tiny_workload(kv_gpu):
+    # 1 layer, 1 KV head, 6 query heads, 4,096 tokens in 32 shuffled pages, 1 query token
+    rng, k, v, cache = _layer(1001, 1, 4096, "q4_0", outliers=False)
+    cache.append(k, v, 0)
+    q = normal_f32(rng, (1, 6, 256))
+    out, lse, _ = _run_decode(kv_gpu, cache, 6, q, [4095], cache.page_table_np)
+    o_ref, l_ref = OracleCache(k, v, "q4_0").attend(q, [4095], 0, 6)
+    compare(out, lse, o_ref, l_ref)
+
+
+def test_page_subsets_in_any_order(kv_gpu):
+    H, H_q, T = 4, 24, 20 * 128
+    rng, k, v, cache = _layer(700, H, T, "q4_0")
+    cache.append(k, v, 0)
+    q = normal_f32(rng, (1, H_q, 256))
+    max_pages = 12
+    counts = [12, 7, 1, 0]
+    plist = np.zeros((H, max_pages), np.int32)
+    plog = np.zeros((H, max_pages), np.int32)
+    chosen = []
+    for h in range(H):
+        blocks = rng.choice(20, counts[h], replace=False)
+        chosen.append(blocks)
+        plog[h, :counts[h]] = blocks
+        plist[h, :counts[h]] = cache.page_table_np[h, blocks]
+        plist[h, counts[h]:] = 10 ** 6            # never read: beyond n_pages[h]
+    out, lse, _ = _run_decode(kv_gpu, cache, H_q, q, [T - 1], plist, plog, counts, max_pages)
+    oc = OracleCache(k, v, "q4_0")
+    for h in range(H):
+        keys = (chosen[h][:, None] * 128 + np.arange(128)[None, :]).ravel()
+        o_ref, l_ref = oc.attend(q, [T - 1], h, 6, key_idx=keys)
+        compare(out[:, 6 * h:6 * h + 6], lse[:, 6 * h:6 * h + 6], o_ref, l_ref)
+    assert np.all(out[:, 18:] == 0) and np.all(np.isneginf(lse[:, 18:]))
+
+
+def test_causal_and_fully_masked_rows(kv_gpu):
+    H, H_q, T = 2, 12, 9 * 128
+    rng, k, v, cache = _layer(710, H, T, "q4_0")
+    cache.append(k, v, 0)
+    q = normal_f32(rng, (4, H_q, 256))
+    q_pos = [3 * 128 + 5, 0, -1, T - 1]        # early, first key only, nothing visible, everything
+    out, lse, _ = _run_decode(kv_gpu, cache, H_q, q, q_pos, cache.page_table_np)
+    oc = OracleCache(k, v, "q4_0")
+    for h in range(H):
+        o_ref, l_ref = oc.attend(q, q_pos, h, 6)
+        compare(out[:, 6 * h:6 * h + 6], lse[:, 6 * h:6 * h + 6], o_ref, l_ref)
+    assert np.all(out[2] == 0) and np.all(np.isneginf(lse[2]))
+
+
+def test_single_short_page_and_empty_list(kv_gpu):
+    rng, k, v, cache = _layer(720, 1, 5, "q4_0", n_blocks=1)
+    cache.append(k, v, 0)
+    q = normal_f32(rng, (1, 6, 256))
+    out, lse, _ = _run_decode(kv_gpu, cache, 6, q, [4], cache.page_table_np)
+    o_ref, l_ref = OracleCache(k, v, "q4_0").attend(q, [4], 0, 6)
+    compare(out, lse, o_ref, l_ref)
+    out, lse, _ = _run_decode(kv_gpu, cache, 6, q, [4], np.zeros((1, 1), np.int32), n_pages=[0], max_pages=1)
+    assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+def test_bad_page_id_is_reported(kv_gpu):
+    rng, k, v, cache = _layer(730, 1, 256, "q4_0")
+    cache.append(k, v, 0)
+    q = normal_f32(rng, (1, 6, 256))
+    plist = cache.page_table_np.copy()
+    plist[0, 1] = 12345
+    _run_decode(kv_gpu, cache, 6, q, [255], plist)
+    assert kv_gpu.kvattn_device_error() == kv_gpu.ERR_BAD_PAGE
+
+
+def test_rejects_unsupported_shapes(kv_gpu):
+    rng, k, v, cache = _layer(740, 1, 128, "q4_0")
+    with pytest.raises(kv_gpu.KVAttnError) as e:
+        _run_decode(kv_gpu, cache, 6, normal_f32(rng, (5, 6, 256)), [127] * 5, cache.page_table_np)
+    assert e.value.status == kv_gpu.ERR_UNSUPPORTED_SHAPE
