@@ -43,6 +43,8 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="only the headline workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extra-steps", type=int, default=100)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling only: override the layer count of the headline workload")
     return ap.parse_args()
 
 
@@ -192,10 +194,14 @@ def event_pair():
 
 # --------------------------------------------------------------------------- decode workloads
 class DecodeBench:
-    def __init__(self, kv, wname, device):
+    def __init__(self, kv, wname, device, layers=0):
+        import dataclasses
+
         import torch
 
         w = WORKLOADS[wname]
+        if layers:
+            w = dataclasses.replace(w, layers=layers)
         self.kv, self.w, self.device = kv, w, device
         self.ctx = w.context
         self.nb = (self.ctx + 127) // 128
@@ -448,7 +454,7 @@ def main():
     hbm, bf16, bf16_sus, peak_kind = peaks()
 
     # ---------------- headline: decode at 131K ----------------
-    b = DecodeBench(kvattn, "decode131k", device)
+    b = DecodeBench(kvattn, "decode131k", device, layers=args.layers)
     clocks = ClockSampler(local)
     clocks.start()
     ms = time_steps(b, args.steps, args.warmup, world)
@@ -475,6 +481,8 @@ def main():
         "gpu_launches": b.launches_per_step * args.steps,
         "clocks": clk,
     }
+    if args.layers:
+        line["profiling_run"] = f"layers overridden to {args.layers}: not a bench value"
     del b
     torch.cuda.empty_cache()
 

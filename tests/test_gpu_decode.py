@@ -20,7 +20,7 @@ def _layer(seed, H, T, v_fmt, n_blocks=None, spare=0, outliers=True):
             v[:, h, ch] *= 8
     n_blocks = n_blocks or (T + 127) // 128
     n_phys = H * n_blocks + spare
-    cache = GpuCache(H, 0, n_blocks, v_fmt, n_phys=n_phys, perm=page_permutation(rng, n_phys))
+    cache = GpuCache(H, 6 * H, n_blocks, v_fmt, n_phys=n_phys, perm=page_permutation(rng, n_phys))
     return rng, k, v, cache
 
 

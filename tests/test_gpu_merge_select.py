@@ -26,7 +26,8 @@ def test_merge_lse(kv_gpu, n_parts, rows, dim):
     lg = lse.cpu().numpy()
     assert np.array_equal(np.isneginf(lg), np.isneginf(l_ref))
     fin = np.isfinite(l_ref)
-    assert np.abs(lg[fin] - l_ref[fin]).max() <= 1e-5
+    if fin.any():
+        assert np.abs(lg[fin] - l_ref[fin]).max() <= 1e-5
     assert np.all(out.cpu().numpy()[0] == 0)
 
 
