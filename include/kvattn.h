@@ -148,8 +148,10 @@ KVATTN_API int kvattn_quantize_append(const kvattn_kv_desc* desc, const float* k
  *   out          device fp32 [n_q][H_q][256]: softmax(q.k/16) v
  *   lse          device fp32 [n_q][H_q]: natural-log log-sum-exp of the scaled scores
  *                (-inf and out = 0 for a row that sees no key)
- *   ws, ws_bytes device workspace of at least kvattn_decode_workspace_size() bytes; its
- *                first 256 bytes must be zero before the first use and are left zero.
+ *   ws, ws_bytes device workspace of at least kvattn_decode_workspace_size() bytes (256-byte
+ *                aligned; may be NULL when that size is 0).  The keys of each KV head are
+ *                split across CTAs; per-split (o, lse) partials go to the workspace and a
+ *                second grid, launched behind the first, merges them.
  * Supports group * n_q <= 24 query rows per KV head.  The split count depends only on the
  * arguments and the device, so results are deterministic. */
 KVATTN_API size_t kvattn_decode_workspace_size(const kvattn_kv_desc* desc, int n_q, int max_pages);
@@ -202,7 +204,7 @@ KVATTN_API int kvattn_select_blocks(const float* summaries, const float* q_group
  * log-sum-exp.
  *   q      device bf16 bits [n_q][H_q][256];  out device fp32 [n_q][H_q][256];
  *   lse    device fp32 [n_q][H_q];  page arguments as for kvattn_decode.
- *   ws     device workspace of kvattn_prefill_workspace_size() bytes (first 256 zero). */
+ *   ws     device workspace of kvattn_prefill_workspace_size() bytes. */
 KVATTN_API size_t kvattn_prefill_workspace_size(const kvattn_kv_desc* desc, int n_q, int max_pages,
                                                 int kv_split_tokens);
 KVATTN_API int kvattn_prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* q, int n_q,

@@ -90,7 +90,7 @@ DecodePlan plan_decode(const kvattn_kv_desc* d, int n_q, int max_pages) {
   if (s < 1) s = 1;
   if (s > max_pages) s = max_pages < 1 ? 1 : max_pages;
   p.n_splits = s;
-  p.lse_off = 256;
+  p.lse_off = 0;
   p.o_off = round_up(p.lse_off + sizeof(float) * d->n_kv_heads * s * p.rows_pad, 256);
   p.bytes = s > 1 ? p.o_off + sizeof(float) * static_cast<size_t>(d->n_kv_heads) * s * p.rows_pad * kHeadDim : 0;
   return p;
@@ -202,7 +202,6 @@ KVATTN_API int kvattn_decode(const kvattn_kv_desc* desc, const float* q, int n_q
   prm.out = out;
   prm.lse = lse;
   uint8_t* w = static_cast<uint8_t*>(ws);
-  prm.counters = plan.bytes ? reinterpret_cast<int*>(w) : nullptr;
   prm.part_lse = plan.bytes ? reinterpret_cast<float*>(w + plan.lse_off) : nullptr;
   prm.part_o = plan.bytes ? reinterpret_cast<float*>(w + plan.o_off) : nullptr;
   prm.n_q = n_q;

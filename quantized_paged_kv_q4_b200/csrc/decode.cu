@@ -7,17 +7,16 @@
 // warps 0-7 consume them.  All query rows of the KV head's group (group x n_q <= 24) are
 // packed into the N dimension of legacy tensor-core MMAs so every KV byte is read once per
 // group:
-//   QK^T: int8 MMA (m16n8k32), A = raw Q8_0 key codes straight from the page (16 tokens on
-//         M), B = the query split exactly into two int8 levels (q ~ s (a + b/254)); each
-//         32-channel block gets a fresh int32 accumulator that is scaled by the key's fp16
-//         block scale, so the dot product itself is exact integer arithmetic.
+//   QK^T: f16 MMA (m16n8k16), A = Q8_0 key codes dequantized in registers (int8 -> f16 by
+//         byte permutes, exact; times the fp16 block scale, one f16 rounding), 16 tokens on
+//         M; B = the query row divided by its largest magnitude, in f16.
 //   PV:   f16 MMA (m16n8k16), A = V^T decoded in registers from nibbles (value q - 8, exact
 //         in f16), B = P^T (probabilities, transposed in registers with movmatrix) times the
 //         V block scale.
 // The online softmax keeps a per-row running maximum and rescales the accumulators only
 // when the maximum grows by more than 2^8 (p stays <= 256, safe in f16).  Warps merge their
-// partial states in shared memory; CTAs write (o, lse) partials and the last CTA of each KV
-// head merges them (log-sum-exp merge, the same arithmetic as kvattn_merge_lse).
+// partial states in shared memory; CTAs write (o, lse) partials that a small follow-up grid
+// (programmatic dependent launch) merges by log-sum-exp, the arithmetic of kvattn_merge_lse.
 #include "decode.cuh"
 
 namespace kvattn {
@@ -44,6 +43,7 @@ struct DecodeCfg {
 };
 
 constexpr uint32_t kHalf2Magic = 0x64006400u;  // f16 1024.0 in both halves
+constexpr uint32_t kByte64x4 = 0x64646464u;    // high byte of f16 1024.0, for byte permutes
 constexpr uint32_t kHalf2_1032 = 0x64086408u;  // 1024 + 8
 constexpr uint32_t kHalf2_1152 = 0x64806480u;  // 1024 + 128
 constexpr uint32_t kHalf2_1_16 = 0x2C002C00u;  // 1/16
@@ -58,8 +58,10 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
   uint64_t* xbar = empty + C::kStages;  // [4] pair exchange barriers (PAIR only)
   int* st_logical = reinterpret_cast<int*>(xbar + 4);
   int* st_valid = st_logical + C::kStages;
-  int* s_flags = st_valid + C::kStages;  // [0] abort, [1] last-CTA flag
+  int* s_flags = st_valid + C::kStages;  // [0] abort
 
+  // the LSE-merge grid that follows may start launching now; it waits for this grid's data
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int h = blockIdx.y;
   const int split = blockIdx.x;
   const int warp = threadIdx.x >> 5;
@@ -80,7 +82,6 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
     }
     for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 2);
     s_flags[0] = 0;
-    s_flags[1] = 0;
     fence_barrier_init();
   }
   __syncthreads();
@@ -148,8 +149,10 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
   {
     // ------------------------------------------------------------------ consumers
     // query rows of this KV head: r = qi * group + j  ->  q[qi][h * group + j][:]
-    // B fragments: level a and level b, per block and n-tile: two regs each.
-    uint32_t qf[C::kNB][NT][2][2];
+    // B fragments: the query row divided by its largest magnitude, in f16, per block, k-step
+    // and n-tile (two regs each); crow[nt][c] = amax / 16 * log2(e) turns a dot product with
+    // the normalised row into a base-2 softmax score.
+    uint32_t qf[C::kNB][2][NT][2];
     float crow[NT][2];
     int qpos_row[NT][2];
     int qpos_min = INT_MAX;
@@ -181,28 +184,19 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
         for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[b][e]));
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-      const float sq = amax / 127.f;
-      const float inv = amax > 0.f ? 127.f / amax : 0.f;
+      const float inv = amax > 0.f ? 1.f / amax : 0.f;
 #pragma unroll
       for (int bl = 0; bl < C::kNB; ++bl) {
-        uint32_t la[2] = {0u, 0u}, lb[2] = {0u, 0u};
+        float xv[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          // blk0 is 0 or 4: select with constant indices (no local-memory array)
-          const float xv = (PAIR && half) ? x[(4 + bl) % kBlocks][e] : x[bl][e];
-          const float a = fminf(fmaxf(rintf(xv * inv), -127.f), 127.f);
-          const float res = xv - a * sq;
-          const float bb = fminf(fmaxf(rintf(res * inv * 254.f), -127.f), 127.f);
-          la[e >> 2] |= (static_cast<uint32_t>(static_cast<int>(a)) & 0xFFu) << (8 * (e & 3));
-          lb[e >> 2] |= (static_cast<uint32_t>(static_cast<int>(bb)) & 0xFFu) << (8 * (e & 3));
-        }
-        qf[bl][nt][0][0] = la[0];
-        qf[bl][nt][0][1] = la[1];
-        qf[bl][nt][1][0] = lb[0];
-        qf[bl][nt][1][1] = lb[1];
+        for (int e = 0; e < 8; ++e) xv[e] = ((PAIR && half) ? x[(4 + bl) % kBlocks][e] : x[bl][e]) * inv;
+        // k-step 0 of the block: channels 8t+0..3, k-step 1: 8t+4..7 (k = 2t, 2t+1 | 2t+8, 2t+9)
+        qf[bl][0][nt][0] = pack_half2(xv[0], xv[1]);
+        qf[bl][0][nt][1] = pack_half2(xv[2], xv[3]);
+        qf[bl][1][nt][0] = pack_half2(xv[4], xv[5]);
+        qf[bl][1][nt][1] = pack_half2(xv[6], xv[7]);
       }
-      // score factor of this lane's row, then fetch those of rows 2t, 2t+1
-      const float cr = sq * (1.0f / 254.0f) * (1.0f / 16.0f) * 1.4426950408889634f;
+      const float cr = amax * (1.0f / 16.0f) * 1.4426950408889634f;
       crow[nt][0] = __shfl_sync(0xffffffffu, cr, (2 * t) * 4);
       crow[nt][1] = __shfl_sync(0xffffffffu, cr, (2 * t + 1) * 4);
 #pragma unroll
@@ -248,26 +242,23 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
           for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-          // key scales for rows g (H=0) and g+8 (H=1), blocks blk0..blk0+kNB-1
-          float dk[2][C::kNB];
+          // key scales of rows g (H=0) and g+8 (H=1) for this warp's blocks, as f16 pairs
+          uint32_t dk2[2][C::kNB];
 #pragma unroll
           for (int H = 0; H < 2; ++H) {
             const uint32_t a = kb + kKScaleOffset + (((G * 8 + g) * 2 + H) * 8 + blk0) * 2;
+            uint32_t w[4];
             if constexpr (C::kNB == 8) {
               const uint4 v = lds128(a);
-              const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                dk[H][2 * e] = half_lo(w[e]);
-                dk[H][2 * e + 1] = half_hi(w[e]);
-              }
+              w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
             } else {
-              uint32_t w0, w1;
-              asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(a));
-              dk[H][0] = half_lo(w0);
-              dk[H][1] = half_hi(w0);
-              dk[H][2] = half_lo(w1);
-              dk[H][3] = half_hi(w1);
+              asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(a));
+              w[2] = w[3] = 0u;
+            }
+#pragma unroll
+            for (int e = 0; e < C::kNB / 2; ++e) {
+              dk2[H][2 * e] = prmt(w[e], 0u, 0x1010u);
+              dk2[H][2 * e + 1] = prmt(w[e], 0u, 0x3232u);
             }
           }
 #pragma unroll
@@ -275,22 +266,20 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
             const int P = blk0 / 2 + pp;
             const uint4 ka = lds128(kb + ((((G * 4 + P) * 2 + 0) * 8 + g) * 4 + t) * 16);
             const uint4 kc = lds128(kb + ((((G * 4 + P) * 2 + 1) * 8 + g) * 4 + t) * 16);
+            const uint32_t wg[4] = {ka.x ^ 0x80808080u, ka.y ^ 0x80808080u, ka.z ^ 0x80808080u, ka.w ^ 0x80808080u};
+            const uint32_t w8[4] = {kc.x ^ 0x80808080u, kc.y ^ 0x80808080u, kc.z ^ 0x80808080u, kc.w ^ 0x80808080u};
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int bl = 2 * pp + e;
-              const uint32_t a0 = e ? ka.z : ka.x, a2 = e ? ka.w : ka.y;
-              const uint32_t a1 = e ? kc.z : kc.x, a3 = e ? kc.w : kc.y;
 #pragma unroll
-              for (int nt = 0; nt < NT; ++nt) {
-                const int zero[4] = {0, 0, 0, 0};
-                int ca[4], cb[4];
-                mma_s8(ca, a0, a1, a2, a3, qf[bl][nt][0][0], qf[bl][nt][0][1], zero);
-                mma_s8(cb, a0, a1, a2, a3, qf[bl][nt][1][0], qf[bl][nt][1][1], zero);
+              for (int ks = 0; ks < 2; ++ks) {
+                // exact int8 -> f16 (1024 + u - 1152), then the block scale (one f16 rounding)
+                const uint32_t A0 = hmul2(hsub2(prmt(wg[2 * e + ks], kByte64x4, 0x4140u), kHalf2_1152), dk2[0][bl]);
+                const uint32_t A2 = hmul2(hsub2(prmt(wg[2 * e + ks], kByte64x4, 0x4342u), kHalf2_1152), dk2[0][bl]);
+                const uint32_t A1 = hmul2(hsub2(prmt(w8[2 * e + ks], kByte64x4, 0x4140u), kHalf2_1152), dk2[1][bl]);
+                const uint32_t A3 = hmul2(hsub2(prmt(w8[2 * e + ks], kByte64x4, 0x4342u), kHalf2_1152), dk2[1][bl]);
 #pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2) {
-                  const float v = __int2float_rn(254 * ca[e2] + cb[e2]);
-                  sacc[nt][e2] = fmaf(dk[e2 >> 1][bl], v, sacc[nt][e2]);
-                }
+                for (int nt = 0; nt < NT; ++nt) mma_f16(sacc[nt], A0, A1, A2, A3, qf[bl][ks][nt][0], qf[bl][ks][nt][1]);
               }
             }
           }
@@ -402,8 +391,8 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
               uint32_t a[4][2];
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                a[q][0] = hsub2(prmt(w[q], kHalf2Magic, 0x4140u), kHalf2_1152);
-                a[q][1] = hsub2(prmt(w[q], kHalf2Magic, 0x4342u), kHalf2_1152);
+                a[q][0] = hsub2(prmt(w[q], kByte64x4, 0x4140u), kHalf2_1152);
+                a[q][1] = hsub2(prmt(w[q], kByte64x4, 0x4342u), kHalf2_1152);
               }
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt) {
@@ -510,53 +499,39 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
       if (d4 == 0) part_l[row] = lse2;
     }
   }
-  if (direct) return;
+}
 
-  // ---------------- last CTA of this KV head merges the splits ----------------
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int prev = atomicAdd(&p.counters[h], 1);
-    s_flags[1] = (prev == p.n_splits - 1);
-  }
-  __syncthreads();
-  if (!s_flags[1]) return;
-  __threadfence();
-  const float* po = p.part_o + static_cast<long long>(h) * p.n_splits * C::kRowsPad * kHeadDim;
-  const float* pl = p.part_lse + static_cast<long long>(h) * p.n_splits * C::kRowsPad;
-  // per-row maxima and normalisers of the split lse values
-  float* rowM = reinterpret_cast<float*>(smem);
-  float* rowL = rowM + C::kRowsPad;
-  for (int row = threadIdx.x; row < n_rows; row += C::kThreads) {
-    float M = -INFINITY;
-    for (int s2 = 0; s2 < p.n_splits; ++s2) M = fmaxf(M, __ldcg(pl + s2 * C::kRowsPad + row));
-    float L = 0.f;
-    if (M != -INFINITY)
-      for (int s2 = 0; s2 < p.n_splits; ++s2) L += fast_exp2(__ldcg(pl + s2 * C::kRowsPad + row) - M);
-    rowM[row] = M;
-    rowL[row] = L;
-  }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < n_rows * (kHeadDim / 4); idx += C::kThreads) {
-    const int row = idx / (kHeadDim / 4);
-    const int d4 = (idx % (kHeadDim / 4)) * 4;
-    const float M = rowM[row], L = rowL[row];
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (M != -INFINITY) {
-      const float invL = 1.f / L;
-#pragma unroll 8
-      for (int s2 = 0; s2 < p.n_splits; ++s2) {
-        const float w = fast_exp2(__ldcg(pl + s2 * C::kRowsPad + row) - M) * invL;
-        const float4 o = __ldcg(reinterpret_cast<const float4*>(po + (s2 * C::kRowsPad + row) * kHeadDim + d4));
-        acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
-      }
+// Log-sum-exp merge of the per-split partials of kvattn_decode, launched right behind the
+// decode grid with programmatic dependent launch: its CTAs start while the decode grid
+// drains and wait (griddepcontrol.wait) until all partials are written.  One CTA per
+// (query row, KV head); each thread owns four channels.
+__global__ void __launch_bounds__(64) decode_merge_kernel(const float* __restrict__ part_o,
+                                                          const float* __restrict__ part_lse, int n_splits,
+                                                          int rows_pad, int group, int n_qh, float* __restrict__ out,
+                                                          float* __restrict__ lse) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int row = blockIdx.x, h = blockIdx.y;
+  const float* pl = part_lse + static_cast<long long>(h) * n_splits * rows_pad + row;
+  const float* po = part_o + (static_cast<long long>(h) * n_splits * rows_pad + row) * kHeadDim + threadIdx.x * 4;
+  float M = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, pl[s * rows_pad]);
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (M != -INFINITY) {
+#pragma unroll 4
+    for (int s = 0; s < n_splits; ++s) {
+      const float w = fast_exp2(pl[s * rows_pad] - M);
+      L += w;
+      const float4 o = *reinterpret_cast<const float4*>(po + static_cast<long long>(s) * rows_pad * kHeadDim);
+      acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
     }
-    const int qi = row / p.group, j = row % p.group;
-    const long long orow = static_cast<long long>(qi) * p.n_qh + h * p.group + j;
-    *reinterpret_cast<float4*>(p.out + orow * kHeadDim + d4) = acc;
-    if (d4 == 0) p.lse[orow] = M != -INFINITY ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    const float inv = 1.f / L;
+    acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
   }
-  if (threadIdx.x == 0) p.counters[h] = 0;  // ready for the next launch
+  const int qi = row / group, j = row % group;
+  const long long orow = static_cast<long long>(qi) * n_qh + h * group + j;
+  *reinterpret_cast<float4*>(out + orow * kHeadDim + threadIdx.x * 4) = acc;
+  if (threadIdx.x == 0) lse[orow] = M != -INFINITY ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -565,7 +540,20 @@ static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream
   using C = DecodeCfg<NT, PAIR, VQ8>;
   dim3 grid(prm.n_splits, n_kv);
   decode_kernel<NT, PAIR, VQ8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(prm);
-  return cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || prm.n_splits == 1) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(prm.group * prm.n_q, n_kv);
+  cfg.blockDim = dim3(kHeadDim / 4);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_merge_kernel, static_cast<const float*>(prm.part_o),
+                            static_cast<const float*>(prm.part_lse), prm.n_splits, C::kRowsPad, prm.group, prm.n_qh,
+                            prm.out, prm.lse);
 }
 
 int decode_rows_pad(int rows) { return ((rows + 7) / 8) * 8; }

@@ -18,7 +18,6 @@ struct DecodeParams {
   float* lse;  // [n_q][H_q]
   float* part_o;    // [H_kv][n_splits][rows_pad][256]
   float* part_lse;  // [H_kv][n_splits][rows_pad]   (log2 units)
-  int* counters;    // [H_kv]
   int n_q, group, n_qh, max_pages, n_splits;
 };
 
