@@ -43,6 +43,7 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="only the headline workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extra-steps", type=int, default=100)
+    ap.add_argument("--prefill-layers", type=int, default=0, help="layers of the prefill workload (0 = 16)")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling only: override the layer count of the headline workload")
     return ap.parse_args()
@@ -293,6 +294,56 @@ class VerifyBench:
             self.layer(l)
 
 
+class PrefillBench:
+    """Chunked prefill: a 2,048-token bf16 chunk (4 ubatches of 512) over 524,288 prior tokens,
+    16 layers x 4 KV heads, 4,096-token KV splits.  One step = for every layer: append the
+    chunk's K/V, then the four ubatch prefill calls."""
+
+    def __init__(self, kv, device, layers=0):
+        import dataclasses
+
+        import torch
+
+        w = WORKLOADS["prefill524k"]
+        if layers:
+            w = dataclasses.replace(w, layers=layers)
+        self.kv, self.w = kv, w
+        L, H, Hq = w.layers, w.kv_heads, w.q_heads
+        self.total = w.context + w.n_q
+        self.nb = (self.total + 127) // 128
+        self.cache = DecodeCache(kv, w, self.nb, w.context, device)
+        self.k_new = torch_normal(derived_seed(w.seed, 21), (L, w.n_q, H, 256), device)
+        self.v_new = torch_normal(derived_seed(w.seed, 22), (L, w.n_q, H, 256), device)
+        self.q = torch_normal(derived_seed(w.seed, 20), (L, w.n_q, Hq, 256), device).to(torch.bfloat16)
+        self.q_bits = self.q.view(torch.int16)
+        self.q_pos = torch.arange(w.context, self.total, dtype=torch.int32, device=device)
+        self.out = torch.empty((L, w.n_q, Hq, 256), device=device)
+        self.lse = torch.empty((L, w.n_q, Hq), device=device)
+        self.ws_bytes = kv.kvattn_prefill_workspace_size(self.cache.desc, w.ubatch, self.nb, w.kv_split_tokens)
+        self.ws = torch.zeros(max(self.ws_bytes, 256), dtype=torch.uint8, device=device)
+        g = w.group
+        self.flops_per_layer = 4.0 * Hq * 256 * (w.n_q * w.context + w.n_q * (w.n_q + 1) / 2)
+        self.flops_per_step = self.flops_per_layer * L
+        self.launches_per_step = L * (1 + 2 * (w.n_q // w.ubatch))
+
+    def layer(self, l, timed=None):
+        kv, c, w = self.kv, self.cache, self.w
+        kv.kvattn_quantize_append(c.desc, self.k_new[l], self.v_new[l], w.n_q, w.context, c.page_table[l], self.nb)
+        if timed is not None:
+            timed[0].record()
+        for u in range(w.n_q // w.ubatch):
+            a, b = u * w.ubatch, (u + 1) * w.ubatch
+            kv.kvattn_prefill_chunk(c.desc, self.q_bits[l, a:b], w.ubatch, self.q_pos[a:b], c.page_table[l], None,
+                                    None, self.nb, w.kv_split_tokens, self.out[l, a:b], self.lse[l, a:b], self.ws,
+                                    self.ws_bytes)
+        if timed is not None:
+            timed[1].record()
+
+    def step(self):
+        for l in range(self.w.layers):
+            self.layer(l)
+
+
 def time_steps(bench, steps, warmup, world):
     import torch
 
@@ -506,6 +557,16 @@ def main():
                                    "decode_kernel_frac_hbm": b3.bytes_per_layer / (k3 * 1e-3) / 1e9 / hbm,
                                    "selected_tokens_per_unit": (b3.w.budget_blocks + b3.w.recent_blocks) * 128 + 4}
             del b3
+            torch.cuda.empty_cache()
+            b4 = PrefillBench(kvattn, device, layers=args.prefill_layers)
+            ms4 = time_steps(b4, max(1, args.extra_steps // 50), 1, world)
+            k4 = time_kernel(b4, 1)
+            tf = b4.flops_per_layer / (k4 * 1e-3) / 1e12
+            extra["prefill524k"] = {"TFLOP/s": b4.flops_per_step / (ms4 * 1e-3) / 1e12, "ms_per_step": ms4,
+                                    "layers": b4.w.layers, "kernel_TFLOP/s": tf, "kernel_frac_bf16": tf / bf16,
+                                    "flop_per_layer": b4.flops_per_layer,
+                                    "peak": f"{peak_kind} dense bf16 (f16 operands run at the same rate)"}
+            del b4
             torch.cuda.empty_cache()
         except Exception as exc:  # report, do not hide
             extra["error"] = repr(exc)

@@ -12,6 +12,7 @@ cudaError_t launch_quantize_append(const kvattn_kv_desc&, const float*, const fl
                                    int, cudaStream_t);
 cudaError_t prepare_select_kernels();
 cudaError_t prepare_prefill_kernels();
+struct PrefillParams;
 cudaError_t launch_merge_lse(const float*, const float*, int, int, int, float*, float*, int, cudaStream_t);
 cudaError_t launch_block_summaries(const kvattn_kv_desc&, const int32_t*, int, int, int, int, float*, cudaStream_t);
 cudaError_t launch_select(const float*, const float*, int, int, int, int, int, int, const int32_t*, int32_t*,
@@ -347,17 +348,60 @@ extern "C" {
 
 KVATTN_API size_t kvattn_prefill_workspace_size(const kvattn_kv_desc* desc, int n_q, int max_pages,
                                                 int kv_split_tokens) {
-  (void)desc; (void)n_q; (void)max_pages; (void)kv_split_tokens;
-  return 0;
+  if (validate_desc(desc) || n_q < 1 || max_pages < 0 || kv_split_tokens < kPageTokens ||
+      kv_split_tokens % kPageTokens)
+    return 0;
+  return plan_prefill(desc->n_kv_heads, desc->n_q_heads / desc->n_kv_heads, n_q, max_pages, kv_split_tokens).bytes;
 }
 
 KVATTN_API int kvattn_prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* q, int n_q, const int32_t* q_pos,
                                     const int32_t* page_list, const int32_t* page_logical, const int32_t* n_pages,
                                     int max_pages, int kv_split_tokens, float* out, float* lse, void* ws,
                                     size_t ws_bytes, kvattn_stream_t stream) {
-  (void)desc; (void)q; (void)n_q; (void)q_pos; (void)page_list; (void)page_logical; (void)n_pages;
-  (void)max_pages; (void)kv_split_tokens; (void)out; (void)lse; (void)ws; (void)ws_bytes; (void)stream;
-  return KVATTN_ERR_UNSUPPORTED_SHAPE;
+  int st = validate_desc(desc);
+  if (st) return st;
+  if (desc->v_fmt != KVATTN_FMT_Q4_0) return KVATTN_ERR_UNSUPPORTED_FORMAT;
+  if (n_q < 1 || max_pages < 0 || !q || !q_pos || !out || !lse || (max_pages > 0 && !page_list))
+    return KVATTN_ERR_INVALID_ARG;
+  if (kv_split_tokens < kPageTokens || kv_split_tokens % kPageTokens || kv_split_tokens > 65536)
+    return KVATTN_ERR_INVALID_ARG;
+  if (!aligned16(q)) return KVATTN_ERR_INVALID_ARG;
+  const int group = desc->n_q_heads / desc->n_kv_heads;
+  const long long rows = static_cast<long long>(n_q) * group;
+  if (rows > (1ll << 24)) return KVATTN_ERR_UNSUPPORTED_SHAPE;
+  const PrefillPlan plan = plan_prefill(desc->n_kv_heads, group, n_q, max_pages, kv_split_tokens);
+  if (plan.n_ks > 65535 || plan.n_mt > (1 << 30)) return KVATTN_ERR_UNSUPPORTED_SHAPE;
+  if (plan.bytes) {
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return KVATTN_ERR_INVALID_ARG;
+    if (ws_bytes < plan.bytes) return KVATTN_ERR_WORKSPACE_TOO_SMALL;
+  }
+  int dev;
+  if ((st = current_device_checked(&dev))) return st;
+  PrefillParams prm{};
+  prm.k_pool = static_cast<const uint8_t*>(desc->k_pool);
+  prm.v_pool = static_cast<const uint8_t*>(desc->v_pool);
+  prm.k_stride = desc->k_page_stride;
+  prm.v_stride = desc->v_page_stride;
+  prm.n_pages = desc->n_pages;
+  prm.q = q;
+  prm.q_pos = q_pos;
+  prm.page_list = page_list;
+  prm.page_logical = page_logical;
+  prm.n_pages_arr = n_pages;
+  prm.out = out;
+  prm.lse = lse;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  prm.part_lse = plan.bytes ? reinterpret_cast<float*>(w + plan.lse_off) : nullptr;
+  prm.part_o = plan.bytes ? reinterpret_cast<float*>(w + plan.o_off) : nullptr;
+  prm.n_q = n_q;
+  prm.group = group;
+  prm.n_qh = desc->n_q_heads;
+  prm.max_pages = max_pages;
+  prm.pages_per_split = plan.pps;
+  prm.n_ks = plan.n_ks;
+  prm.rows_pad = plan.rows_pad;
+  cudaError_t e = launch_prefill(prm, desc->n_kv_heads, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVATTN_OK : cuda_fail(e);
 }
 
 }  // extern "C"

@@ -54,9 +54,10 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
   using C = DecodeCfg<NT, PAIR, VQ8>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
-  uint64_t* empty = full + C::kStages;
-  uint64_t* xbar = empty + C::kStages;  // [4] pair exchange barriers (PAIR only)
-  int* st_logical = reinterpret_cast<int*>(xbar + 4);
+  uint64_t* xbar = full + C::kStages;   // [4] pair exchange barriers (PAIR only)
+  int* rel_cnt = reinterpret_cast<int*>(xbar + 4);  // [kStages] warps done with the stage
+  int* s_issued = rel_cnt + C::kStages;              // pages issued so far
+  int* st_logical = s_issued + 1;
   int* st_valid = st_logical + C::kStages;
   int* s_flags = st_valid + C::kStages;  // [0] abort
 
@@ -78,8 +79,9 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], C::kConsumerWarps);
+      rel_cnt[s] = 0;
     }
+    *s_issued = 0;
     for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 2);
     s_flags[0] = 0;
     fence_barrier_init();
@@ -106,45 +108,32 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
   const int half = PAIR ? (warp & 1) : 0;
   const int blk0 = PAIR ? 4 * half : 0;
 
-  // Page copies are issued by lane 0 of warp 0, at most kStages pages ahead of its own
-  // consumption.  A stage is refilled only after all eight warps released its previous page
-  // (empty barrier); refills are attempted without blocking, except for the page warp 0 is
-  // about to consume, so no warp ever waits on a slower one except through that page.
+  // Page copies: the first kStages pages are issued up front by lane 0 of warp 0; after
+  // that, the warp that is the last of the eight to finish with a stage refills it at
+  // once with the page kStages further on, so kStages - 1 pages stay in flight while one
+  // is being consumed.  Pages are issued in increasing order.
   const int32_t* plist = p.page_list + static_cast<long long>(h) * p.max_pages;
   const int32_t* plog = p.page_logical ? p.page_logical + static_cast<long long>(h) * p.max_pages : nullptr;
-  int next = 0;  // next page to issue (meaningful in lane 0 of warp 0 only)
-  auto issue_upto = [&](int i) -> bool {
-    while (next < count && next < i + C::kStages) {
-      const int s = next % C::kStages;
-      const int prev = next - C::kStages;
-      if (prev >= 0) {
-        const uint32_t ppar = (prev / C::kStages) & 1;
-        if (next == i) {
-          if (!mbar_wait(&empty[s], ppar)) return false;
-        } else if (!mbar_try_wait(&empty[s], ppar)) {
-          break;
-        }
-      }
-      const int idx = first + next;
-      const int page = plist[idx];
-      st_logical[s] = plog ? plog[idx] : idx;
-      if (page < 0 || page >= p.n_pages) {
-        record_error(KVATTN_ERR_BAD_PAGE);
-        st_valid[s] = 0;
-        mbar_arrive(&full[s]);
-      } else {
-        st_valid[s] = 1;
-        uint8_t* stage = smem + s * C::kStageBytes;
-        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-        bulk_g2s(stage, p.k_pool + static_cast<int64_t>(page) * p.k_stride, kKPageBytes, &full[s]);
-        bulk_g2s(stage + kKPageBytes, p.v_pool + static_cast<int64_t>(page) * p.v_stride, C::kVBytes, &full[s]);
-      }
-      ++next;
+  auto issue = [&](int i) {
+    const int s = i % C::kStages;
+    const int idx = first + i;
+    const int page = plist[idx];
+    st_logical[s] = plog ? plog[idx] : idx;
+    if (page < 0 || page >= p.n_pages) {
+      record_error(KVATTN_ERR_BAD_PAGE);
+      st_valid[s] = 0;
+      mbar_arrive(&full[s]);
+    } else {
+      st_valid[s] = 1;
+      uint8_t* stage = smem + s * C::kStageBytes;
+      mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+      bulk_g2s(stage, p.k_pool + static_cast<int64_t>(page) * p.k_stride, kKPageBytes, &full[s]);
+      bulk_g2s(stage + kKPageBytes, p.v_pool + static_cast<int64_t>(page) * p.v_stride, C::kVBytes, &full[s]);
     }
-    return true;
+    *reinterpret_cast<volatile int*>(s_issued) = i + 1;
   };
-  const bool issuer = (warp == 0 && lane == 0);
-  if (issuer) issue_upto(0);
+  if (warp == 0 && lane == 0)
+    for (int i = 0; i < count && i < C::kStages; ++i) issue(i);
 
   {
     // ------------------------------------------------------------------ consumers
@@ -215,15 +204,6 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
     for (int i = 0; i < count; ++i) {
       const int s = i % C::kStages;
       const uint32_t par = (i / C::kStages) & 1;
-      if (warp == 0) {
-        int ok = 1;
-        if (lane == 0) ok = issue_upto(i) ? 1 : 0;
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) {
-          s_flags[0] = 1;
-          break;
-        }
-      }
       if (!mbar_wait(&full[s], par)) {
         s_flags[0] = 1;
         break;
@@ -406,7 +386,12 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
       }
       if (aborted) break;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      if (lane == 0) {
+        if (atomicAdd(&rel_cnt[s], 1) == C::kConsumerWarps - 1) {
+          rel_cnt[s] = 0;
+          if (i + C::kStages < count) issue(i + C::kStages);
+        }
+      }
     }
     // reduce the per-thread partial sums over the 8 token lanes
 #pragma unroll
@@ -424,7 +409,8 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
   __syncthreads();
   if (s_flags[0]) {
     // A bounded wait expired: wait (bounded) for the copies still in flight, then leave.
-    if (issuer) {
+    if (threadIdx.x == 0) {
+      const int next = *reinterpret_cast<volatile int*>(s_issued);
       for (int pg = next - C::kStages < 0 ? 0 : next - C::kStages; pg < next; ++pg) {
         const unsigned long long t0 = global_timer_ns();
         while (!mbar_try_wait(&full[pg % C::kStages], (pg / C::kStages) & 1)) {

@@ -117,7 +117,7 @@ def test_single_short_page_and_empty_list(kv_gpu):
     q = normal_f32(rng, (1, 6, 256))
     out, lse, _ = _run_decode(kv_gpu, cache, 6, q, [4], cache.page_table_np)
     o_ref, l_ref = OracleCache(k, v, "q4_0").attend(q, [4], 0, 6)
-    compare(out, lse, o_ref, l_ref)
+    compare(out, lse, o_ref, l_ref, magnitude_scaled=True)   # 5 keys: outputs of size ~1-10
     out, lse, _ = _run_decode(kv_gpu, cache, 6, q, [4], np.zeros((1, 1), np.int32), n_pages=[0], max_pages=1)
     assert np.all(out == 0) and np.all(np.isneginf(lse))
 
