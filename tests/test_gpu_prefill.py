@@ -56,7 +56,9 @@ def test_prefill_matches_oracle(kv_gpu, n_prior, n_q, split):
     oc = OracleCache(k, v, "q4_0")
     for h in range(H):
         o_ref, l_ref = oc.attend(q, q_pos, h, 6)
-        compare(out[:, 6 * h:6 * h + 6], lse[:, 6 * h:6 * h + 6], o_ref, l_ref, magnitude_scaled=T < 256)
+        # outlier channels and short contexts give outputs of magnitude ~1: the f16 operand
+        # error scales with that magnitude (see compare)
+        compare(out[:, 6 * h:6 * h + 6], lse[:, 6 * h:6 * h + 6], o_ref, l_ref, magnitude_scaled=True)
 
 
 def test_prefill_page_subsets(kv_gpu):
@@ -79,7 +81,7 @@ def test_prefill_page_subsets(kv_gpu):
         keys = (np.asarray(keep[h])[:, None] * 128 + np.arange(128)[None, :]).ravel()
         keys = keys[keys < T]
         o_ref, l_ref = oc.attend(q, q_pos, h, 6, key_idx=keys)
-        compare(out[:, 6 * h:6 * h + 6], lse[:, 6 * h:6 * h + 6], o_ref, l_ref)
+        compare(out[:, 6 * h:6 * h + 6], lse[:, 6 * h:6 * h + 6], o_ref, l_ref, magnitude_scaled=True)
 
 
 def test_prefill_subset_of_the_524k_workload(kv_gpu):
