@@ -160,6 +160,21 @@ KVATTN_API int kvattn_decode(const kvattn_kv_desc* desc, const float* q, int n_q
                              const int32_t* n_pages, int max_pages, float* out, float* lse,
                              void* ws, size_t ws_bytes, kvattn_stream_t stream);
 
+/* Same computation and arguments as kvattn_decode, for callers that cannot allocate device
+ * memory (for example code hosted by a framework whose memory pool owns the device memory
+ * and forbids cudaMalloc, or loops that must never enter the allocator).  It has no
+ * counterpart on the source pages.  The per-split scratch is a 4 MiB file-scope device array
+ * (every GPU that loads the library holds it until exit); plans larger than that return
+ * KVATTN_ERR_WORKSPACE_TOO_SMALL.  The first call on a device looks up the array's device
+ * address (with that device current) and should come before any stream capture.  All calls
+ * on a device share that device's array, which keeps the last call's contents: calls on one
+ * device whose GPU work overlaps (for example on two streams) race, so order them on one
+ * stream.  Calls no allocating routine. */
+KVATTN_API int kvattn_decode_noalloc(const kvattn_kv_desc* desc, const float* q, int n_q, const int32_t* q_pos,
+                                     const int32_t* page_list, const int32_t* page_logical,
+                                     const int32_t* n_pages, int max_pages, float* out, float* lse,
+                                     kvattn_stream_t stream);
+
 /* ---- log-sum-exp merge ([STREAM] method list: online LSE accumulation) -------------
  * out = sum_p exp(lse_p - lse) * o_p with lse = ln sum_p exp(lse_p), skipping -inf parts.
  *   o_parts   device fp32 [n_parts][rows][dim];  lse_parts device fp32 [n_parts][rows]

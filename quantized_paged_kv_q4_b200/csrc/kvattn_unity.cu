@@ -6,3 +6,4 @@
 #include "select.cu"
 #include "prefill.cu"
 #include "api.cu"
+#include "noalloc.cu"

@@ -58,6 +58,8 @@ _SIGS = {
     "kvattn_decode_workspace_size": (c_size_t, [POINTER(kvattn_kv_desc), c_int, c_int]),
     "kvattn_decode": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                               c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "kvattn_decode_noalloc": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_int, c_void_p, c_void_p, c_void_p,
+                                      c_void_p, c_int, c_void_p, c_void_p, c_void_p]),
     "kvattn_merge_lse": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
     "kvattn_block_summaries": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_int, c_int, c_int, c_int, c_void_p,
                                        c_void_p]),
@@ -162,6 +164,14 @@ def kvattn_decode(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pag
     _check(lib().kvattn_decode(ctypes.byref(desc), _p(q), n_q, _p(q_pos), _p(page_list), _p(page_logical),
                                _p(n_pages), max_pages, _p(out), _p(lse), _p(ws), ws_bytes, _s(stream)),
            "kvattn_decode")
+
+
+def kvattn_decode_noalloc(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pages, out, lse,
+                          stream=None) -> None:
+    """kvattn_decode without a caller workspace (scratch in a fixed device array of the library)."""
+    _check(lib().kvattn_decode_noalloc(ctypes.byref(desc), _p(q), n_q, _p(q_pos), _p(page_list), _p(page_logical),
+                                       _p(n_pages), max_pages, _p(out), _p(lse), _s(stream)),
+           "kvattn_decode_noalloc")
 
 
 def kvattn_merge_lse(o_parts, lse_parts, n_parts, rows, dim, out, lse, stream=None) -> None:
