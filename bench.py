@@ -44,6 +44,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extra-steps", type=int, default=100)
     ap.add_argument("--prefill-layers", type=int, default=0, help="layers of the prefill workload (0 = 16)")
+    ap.add_argument("--profile", choices=["none", "decode", "prefill", "verify"], default="none",
+                    help="profiling only: run just this workload's steps (no JSON bench line)")
+    ap.add_argument("--context", type=int, default=0, help="profiling only: prior-context override")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling only: override the layer count of the headline workload")
     return ap.parse_args()
@@ -299,7 +302,7 @@ class PrefillBench:
     16 layers x 4 KV heads, 4,096-token KV splits.  One step = for every layer: append the
     chunk's K/V, then the four ubatch prefill calls."""
 
-    def __init__(self, kv, device, layers=0):
+    def __init__(self, kv, device, layers=0, context=0):
         import dataclasses
 
         import torch
@@ -307,6 +310,8 @@ class PrefillBench:
         w = WORKLOADS["prefill524k"]
         if layers:
             w = dataclasses.replace(w, layers=layers)
+        if context:
+            w = dataclasses.replace(w, context=context)
         self.kv, self.w = kv, w
         L, H, Hq = w.layers, w.kv_heads, w.q_heads
         self.total = w.context + w.n_q
@@ -503,6 +508,21 @@ def main():
     kvattn.kvattn_init(local)
     device = torch.device("cuda", local)
     hbm, bf16, bf16_sus, peak_kind = peaks()
+
+    if args.profile != "none":
+        # a short run of one workload for ncu captures; prints no bench line
+        if args.profile == "decode":
+            b = DecodeBench(kvattn, "decode131k", device, layers=args.layers or 2)
+        elif args.profile == "verify":
+            b = VerifyBench(kvattn, device)
+        else:
+            b = PrefillBench(kvattn, device, layers=args.layers or 1, context=args.context)
+        for _ in range(args.warmup + args.steps):
+            b.step()
+        torch.cuda.synchronize()
+        assert kvattn.kvattn_device_error() == 0
+        print(json.dumps({"profiling_run": args.profile, "steps": args.steps, "warmup": args.warmup}))
+        return
 
     # ---------------- headline: decode at 131K ----------------
     b = DecodeBench(kvattn, "decode131k", device, layers=args.layers)

@@ -14,7 +14,8 @@
 //         in f16), B = P^T (probabilities, transposed in registers with movmatrix) times the
 //         V block scale.
 // The online softmax keeps a per-row running maximum and rescales the accumulators only
-// when the maximum grows by more than 2^8 (p stays <= 256, safe in f16).  Warps merge their
+// when the maximum grows by more than 2^8 (p stays <= 256, safe in f16); the exact
+// cross-lane maximum is only computed when a warp vote says some score crossed that bound.  Warps merge their
 // partial states in shared memory; CTAs write (o, lse) partials that a small follow-up grid
 // (programmatic dependent launch) merges by log-sum-exp, the arithmetic of kvattn_merge_lse.
 #include "decode.cuh"
@@ -293,36 +294,56 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
             xpar ^= 1;
           }
           // ---------------- online softmax (base 2) ----------------
+          // The running maximum m_run of a row is shared by the 8 lanes that hold the row.
+          // It only has to bound the scores to within 2^8 (p <= 256 in f16), so the exact
+          // cross-lane maximum is computed only when some lane sees a score above
+          // m_run + 8: one warp vote per tile instead of three shuffles per row.
           const int key0 = logical * kPageTokens + 16 * G + g;  // rows e<2: token g, e>=2: g+8
+          float sv[NT][4], lm[NT][2];
+          bool need = false;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              sv[nt][e] = sacc[nt][e] * crow[nt][e & 1];
+              if (need_mask && key0 + 8 * (e >> 1) > qpos_row[nt][e & 1]) sv[nt][e] = -INFINITY;
+            }
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              lm[nt][c] = fmaxf(sv[nt][c], sv[nt][c + 2]);
+              need |= lm[nt][c] > m_run[nt][c] + 8.f;
+            }
+          }
+          if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int c = 0; c < 2; ++c) {
+                float mx = lm[nt][c];
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                if (mx > m_run[nt][c] + 8.f) {
+                  const float alpha = fast_exp2(m_run[nt][c] - mx);  // 0 when m_run = -inf
+                  l_run[nt][c] *= alpha;
+#pragma unroll
+                  for (int mt = 0; mt < 2 * C::kNB; ++mt) {
+                    oacc[mt][nt][c] *= alpha;
+                    oacc[mt][nt][c + 2] *= alpha;
+                  }
+                  m_run[nt][c] = mx;
+                }
+              }
+          }
           uint32_t pb[NT][2];
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            float sv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              sv[e] = sacc[nt][e] * crow[nt][e & 1];
-              if (need_mask && key0 + 8 * (e >> 1) > qpos_row[nt][e & 1]) sv[e] = -INFINITY;
-            }
             float pr[4];
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-              float mx = fmaxf(sv[c], sv[c + 2]);
-              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-              if (mx > m_run[nt][c] + 8.f) {
-                const float alpha = fast_exp2(m_run[nt][c] - mx);
-                l_run[nt][c] *= alpha;
-#pragma unroll
-                for (int mt = 0; mt < 2 * C::kNB; ++mt) {
-                  oacc[mt][nt][c] *= alpha;
-                  oacc[mt][nt][c + 2] *= alpha;
-                }
-                m_run[nt][c] = mx;
-              }
               const float mu = m_run[nt][c] == -INFINITY ? 0.f : m_run[nt][c];
-              pr[c] = fast_exp2(sv[c] - mu);
-              pr[c + 2] = fast_exp2(sv[c + 2] - mu);
+              pr[c] = fast_exp2(sv[nt][c] - mu);
+              pr[c + 2] = fast_exp2(sv[nt][c + 2] - mu);
               l_run[nt][c] += pr[c] + pr[c + 2];
             }
             pb[nt][0] = movmatrix_t(pack_half2(pr[0], pr[1]));
@@ -487,37 +508,81 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
   }
 }
 
-// Log-sum-exp merge of the per-split partials of kvattn_decode, launched right behind the
-// decode grid with programmatic dependent launch: its CTAs start while the decode grid
-// drains and wait (griddepcontrol.wait) until all partials are written.  One CTA per
-// (query row, KV head); each thread owns four channels.
-__global__ void __launch_bounds__(64) decode_merge_kernel(const float* __restrict__ part_o,
-                                                          const float* __restrict__ part_lse, int n_splits,
-                                                          int rows_pad, int group, int n_qh, float* __restrict__ out,
-                                                          float* __restrict__ lse) {
+// Log-sum-exp merge of the per-split partials of kvattn_decode (and kvattn_prefill_chunk),
+// launched right behind the producing grid with programmatic dependent launch: its CTAs
+// start while that grid drains and wait (griddepcontrol.wait) until all partials are
+// written.  One CTA per (query row, KV head), 256 threads: the split log-sum-exps are
+// reduced cooperatively, then four groups of 64 threads (four channels each) accumulate
+// interleaved splits with independent loads and are summed through shared memory.
+constexpr int kMergeThreads = 256;
+constexpr int kMergeGroups = kMergeThreads / (kHeadDim / 4);
+
+__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const float* __restrict__ part_o,
+                                                                     const float* __restrict__ part_lse, int n_splits,
+                                                                     int rows_pad, int group, int n_qh,
+                                                                     float* __restrict__ out, float* __restrict__ lse) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ float red_m[kMergeThreads / 32], red_l[kMergeThreads / 32];
+  __shared__ float4 red_o[kMergeGroups - 1][kHeadDim / 4];
   const int row = blockIdx.x, h = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const float* pl = part_lse + static_cast<long long>(h) * n_splits * rows_pad + row;
-  const float* po = part_o + (static_cast<long long>(h) * n_splits * rows_pad + row) * kHeadDim + threadIdx.x * 4;
+  // (max, sum of exp2) over this thread's splits, then over the block
+  float m = -INFINITY, l = 0.f;
+  for (int sp = tid; sp < n_splits; sp += kMergeThreads) {
+    const float v = pl[static_cast<long long>(sp) * rows_pad];
+    if (v > m) {
+      l = (m == -INFINITY ? 0.f : l * fast_exp2(m - v)) + 1.f;
+      m = v;
+    } else if (v != -INFINITY) {
+      l += fast_exp2(v - m);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), l2 = __shfl_xor_sync(0xffffffffu, l, o);
+    const float mm = fmaxf(m, m2);
+    l = (mm == -INFINITY) ? 0.f : l * fast_exp2(m - mm) + l2 * fast_exp2(m2 - mm);
+    m = mm;
+  }
+  if (lane == 0) {
+    red_m[wid] = m;
+    red_l[wid] = l;
+  }
+  __syncthreads();
   float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, pl[s * rows_pad]);
+#pragma unroll
+  for (int w = 0; w < kMergeThreads / 32; ++w) M = fmaxf(M, red_m[w]);
   float L = 0.f;
+  if (M != -INFINITY)
+#pragma unroll
+    for (int w = 0; w < kMergeThreads / 32; ++w) L += red_l[w] * fast_exp2(red_m[w] - M);
+  // weighted sum of the partial outputs
+  const int grp = tid / (kHeadDim / 4), d4 = tid % (kHeadDim / 4);
+  const float* po = part_o + (static_cast<long long>(h) * n_splits * rows_pad + row) * kHeadDim + d4 * 4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (M != -INFINITY) {
-#pragma unroll 4
-    for (int s = 0; s < n_splits; ++s) {
-      const float w = fast_exp2(pl[s * rows_pad] - M);
-      L += w;
-      const float4 o = *reinterpret_cast<const float4*>(po + static_cast<long long>(s) * rows_pad * kHeadDim);
+    const float inv = 1.f / L;
+#pragma unroll 8
+    for (int sp = grp; sp < n_splits; sp += kMergeGroups) {
+      const float w = fast_exp2(pl[static_cast<long long>(sp) * rows_pad] - M) * inv;
+      const float4 o = *reinterpret_cast<const float4*>(po + static_cast<long long>(sp) * rows_pad * kHeadDim);
       acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
     }
-    const float inv = 1.f / L;
-    acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
   }
-  const int qi = row / group, j = row % group;
-  const long long orow = static_cast<long long>(qi) * n_qh + h * group + j;
-  *reinterpret_cast<float4*>(out + orow * kHeadDim + threadIdx.x * 4) = acc;
-  if (threadIdx.x == 0) lse[orow] = M != -INFINITY ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+  if (grp > 0) red_o[grp - 1][d4] = acc;
+  __syncthreads();
+  if (grp == 0) {
+#pragma unroll
+    for (int gq = 0; gq < kMergeGroups - 1; ++gq) {
+      const float4 o = red_o[gq][d4];
+      acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+    }
+    const int qi = row / group, j = row % group;
+    const long long orow = static_cast<long long>(qi) * n_qh + h * group + j;
+    *reinterpret_cast<float4*>(out + orow * kHeadDim + d4 * 4) = acc;
+    if (tid == 0) lse[orow] = M != -INFINITY ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+  }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -530,7 +595,7 @@ static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream
   if (e != cudaSuccess || prm.n_splits == 1) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(prm.group * prm.n_q, n_kv);
-  cfg.blockDim = dim3(kHeadDim / 4);
+  cfg.blockDim = dim3(kMergeThreads);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

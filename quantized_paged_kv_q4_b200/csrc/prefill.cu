@@ -483,9 +483,6 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
   }
 }
 
-__global__ void __launch_bounds__(64) decode_merge_kernel(const float* __restrict__, const float* __restrict__, int,
-                                                          int, int, int, float* __restrict__, float* __restrict__);
-
 cudaError_t prepare_prefill_kernels() {
   return cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::kSmemBytes);
 }
@@ -517,7 +514,7 @@ cudaError_t launch_prefill(const PrefillParams& prm0, int n_kv, cudaStream_t str
   if (e != cudaSuccess || prm.n_ks == 1) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rows, n_kv);
-  cfg.blockDim = dim3(kHeadDim / 4);
+  cfg.blockDim = dim3(kMergeThreads);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
