@@ -351,7 +351,9 @@ KVATTN_API size_t kvattn_prefill_workspace_size(const kvattn_kv_desc* desc, int 
   if (validate_desc(desc) || n_q < 1 || max_pages < 0 || kv_split_tokens < kPageTokens ||
       kv_split_tokens % kPageTokens)
     return 0;
-  return plan_prefill(desc->n_kv_heads, desc->n_q_heads / desc->n_kv_heads, n_q, max_pages, kv_split_tokens).bytes;
+  return plan_prefill(desc->n_kv_heads, desc->n_q_heads / desc->n_kv_heads, n_q, max_pages, kv_split_tokens,
+                      sm_count_for_planning())
+      .bytes;
 }
 
 KVATTN_API int kvattn_prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* q, int n_q, const int32_t* q_pos,
@@ -369,7 +371,8 @@ KVATTN_API int kvattn_prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* 
   const int group = desc->n_q_heads / desc->n_kv_heads;
   const long long rows = static_cast<long long>(n_q) * group;
   if (rows > (1ll << 24)) return KVATTN_ERR_UNSUPPORTED_SHAPE;
-  const PrefillPlan plan = plan_prefill(desc->n_kv_heads, group, n_q, max_pages, kv_split_tokens);
+  const PrefillPlan plan =
+      plan_prefill(desc->n_kv_heads, group, n_q, max_pages, kv_split_tokens, sm_count_for_planning());
   if (plan.n_ks > 65535 || plan.n_mt > (1 << 30)) return KVATTN_ERR_UNSUPPORTED_SHAPE;
   if (plan.bytes) {
     if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return KVATTN_ERR_INVALID_ARG;

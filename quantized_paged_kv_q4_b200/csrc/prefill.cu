@@ -5,19 +5,22 @@
 //
 // Work unit (one CTA): a KV head h, an M-tile of 128 query rows of that head's group
 // (row r = token t * group + j: all query heads of a group share the K/V tiles, so each
-// dequantized tile serves 128 rows), and one KV split of kv_split_tokens keys.  The split
-// is walked in 64-key tiles (half pages):
+// dequantized tile serves 128 rows), and one KV split of kv_split_tokens keys, walked in
+// 64-key tiles (half pages).  Roles:
 //
-//   dequant warps (8)   raw Q8_0 K / Q4_0 V from global -> f16 in shared memory, block
-//                       scales folded in (one f16 rounding):  K^ [64 keys][256] and
-//                       V^T [256 dims][64 keys], both K-major, 128-byte swizzle
-//   MMA warp (1 thread) S = Q K^T      (M = 128 rows, N = 64 keys, K = 256)  -> TMEM
-//                       O^T += V^T P^T (M = 128 dims x 2, N = 128 rows, K = 64 keys) -> TMEM
-//   softmax warps (4)   thread = query row: S from TMEM, causal mask, running max (the
-//                       accumulators are rescaled only when the max grows by > 2^8),
-//                       P = exp2(S - m) as f16 into shared memory
+//   producer (1 thread)   bulk async copies (TMA engine) of a tile's raw Q8_0 K / Q4_0 V
+//                         bytes (26 KB) into a two-stage shared-memory ring
+//   dequant warps (8)     raw -> f16 with the block scales folded in (one f16 rounding):
+//                         K^ [64 keys][256] and V^T [256 dims][64 keys], K-major, 128-byte
+//                         swizzle, double-buffered
+//   MMA issuer (1 thread) S = Q K^T  (M = 128 rows, N = 64 keys, K = 256; Q from tensor memory)
+//                         O += P V   (M = 128 rows, N = 256 dims, K = 64 keys; P from tensor
+//                         memory), both accumulated in tensor memory
+//   softmax warps (4)     thread = query row = TMEM lane: S -> causal mask -> running max
+//                         (the row of O is rescaled only when its max grows by more than
+//                         2^8) -> P = exp2(S - m) as f16 into tensor memory, over S
 //
-// Q (bf16) is converted to f16 and pre-scaled by log2(e)/16 so S is a base-2 score.  The
+// Q (bf16) is converted to f16 and pre-scaled by log2(e)/16, so S is a base-2 score.  The
 // CTA writes a normalised partial (o, lse) per row; a second grid merges the splits.
 #include "decode.cuh"
 #include "tcgen05.cuh"
@@ -43,24 +46,28 @@ struct PrefillParams {
 namespace pf {
 constexpr int kRows = 128;
 constexpr int kKeys = 64;
-constexpr int kSoftmaxWarps = 4;   // warps 0-3: TMEM lane quarters 0-3
+constexpr int kSoftmaxWarps = 4;  // warps 0-3: TMEM lane quarters 0-3
 constexpr int kMmaWarp = 4;
-constexpr int kDequantWarps = 8;   // warps 5-12
-constexpr int kThreads = (kSoftmaxWarps + 1 + kDequantWarps) * 32;
-constexpr int kDq0 = (kSoftmaxWarps + 1) * 32;  // first dequant thread
+constexpr int kLoadWarp = 5;
+constexpr int kDequantWarps = 8;  // warps 6-13
+constexpr int kThreads = (kSoftmaxWarps + 2 + kDequantWarps) * 32;
+constexpr int kDq0 = (kSoftmaxWarps + 2) * 32;  // first dequant thread
+// raw bytes of one 64-key tile, as copied from the page
+constexpr int kRawKc = 16384, kRawKs = 1024, kRawVc = 8192, kRawVs = 1024;
+constexpr int kRawBytes = kRawKc + kRawKs + kRawVc + kRawVs;  // 26,624
 // shared memory map (bytes)
-constexpr int kQOff = 0;                        // 4 atoms x [128 rows][128 B]
-constexpr int kKOff = 65536;                    // 2 buffers x 4 atoms x [64 keys][128 B]
-constexpr int kVOff = kKOff + 2 * 32768;        // 2 buffers x [256 dims][128 B]
-constexpr int kPOff = kVOff + 2 * 32768;        // 2 buffers x [128 rows][128 B]
-constexpr int kMiscOff = kPOff + 2 * 16384;     // barriers, TMEM base, row stats
-constexpr int kSmemBytes = kMiscOff + 3072;   // = 227 KB, the per-CTA maximum
+constexpr int kKOff = 0;                     // 2 buffers x 4 atoms x [64 keys][128 B]
+constexpr int kVOff = kKOff + 2 * 32768;     // 2 buffers x [256 dims][128 B]
+constexpr int kRawOff = kVOff + 2 * 32768;   // 2 stages of raw tile bytes
+constexpr int kMiscOff = kRawOff + 2 * kRawBytes;
+constexpr int kSmemBytes = kMiscOff + 1024;
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSCol0 = 0;     // S buffers: [0,64), [64,128)
-constexpr uint32_t kOCol0 = 128;   // O^T dims 0-127: [128,256); dims 128-255: [256,384)
+constexpr uint32_t kSCol0 = 0;    // S buffers [0,64), [64,128); P (f16 pairs) over their first 32
+constexpr uint32_t kOCol0 = 128;  // O [row][256 dims]: [128, 384)
+constexpr uint32_t kQCol0 = 384;  // Q [row][256 dims] as f16 pairs: [384, 512)
 constexpr uint32_t kIdescQK = tc::idesc_f16(128, kKeys, 0, 0);
-constexpr uint32_t kIdescPV = tc::idesc_f16(128, kRows, 0, 0);
+constexpr uint32_t kIdescPV = tc::idesc_f16(128, 256, 0, 0);
 }  // namespace pf
 
 struct PfTile {
@@ -90,23 +97,37 @@ __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {
   return row * 128 + ((chunk ^ (row & 7)) << 4);
 }
 
+// Tensor-memory address of this warp's lane quarter.
+__device__ __forceinline__ uint32_t tmem_lane(uint32_t tmem, int warp) {
+  return tmem + ((static_cast<uint32_t>(warp & 3) * 32) << 16);
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]; issued by one thread.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pf::kMiscOff);
-  uint64_t* kready = bars + 0;   // [2] dequant -> MMA
-  uint64_t* vready = bars + 2;   // [2]
-  uint64_t* kfree = bars + 4;    // [2] MMA (QK done) -> dequant
-  uint64_t* vfree = bars + 6;    // [2] MMA (PV done) -> dequant, softmax
-  uint64_t* sready = bars + 8;   // [2] MMA -> softmax
-  uint64_t* pready = bars + 10;  // [2] softmax -> MMA
-  uint64_t* ofinal = bars + 12;  // MMA -> softmax (epilogue)
-  uint64_t* wgbar = bars + 13;   // softmax warpgroup rendezvous
-  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* rawfull = bars + 0;   // [2] producer (tx bytes) -> dequant
+  uint64_t* rawempty = bars + 2;  // [2] dequant -> producer
+  uint64_t* kready = bars + 4;    // [2] dequant -> MMA
+  uint64_t* vready = bars + 6;    // [2]
+  uint64_t* kfree = bars + 8;     // [2] MMA (QK done) -> dequant
+  uint64_t* vfree = bars + 10;    // [2] MMA (PV done) -> dequant, softmax
+  uint64_t* sready = bars + 12;   // [2] MMA -> softmax
+  uint64_t* pready = bars + 14;   // [2] softmax -> MMA
+  uint64_t* ofinal = bars + 16;   // MMA -> softmax (epilogue)
+  uint64_t* qready = bars + 17;   // softmax (Q in TMEM) -> MMA
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bars + 18);
   int* s_abort = reinterpret_cast<int*>(tmem_base_s + 1);
-  int* s_any = s_abort + 1;                              // [2][4] per tile parity and softmax warp
-  float* s_alpha = reinterpret_cast<float*>(s_any + 8);  // [2][128]
-  float* s_l = s_alpha + 2 * pf::kRows;                  // [128]
-  float* s_m = s_l + pf::kRows;                          // [128] (ends before kMiscOff + 2232)
 
   const int mt = blockIdx.x, ks = blockIdx.y, h = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -124,6 +145,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < 2; ++b) {
+      mbar_init(&rawfull[b], 1);
+      mbar_init(&rawempty[b], pf::kDequantWarps);
       mbar_init(&kready[b], pf::kDequantWarps);
       mbar_init(&vready[b], pf::kDequantWarps);
       mbar_init(&kfree[b], 1);
@@ -132,7 +155,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       mbar_init(&pready[b], pf::kSoftmaxWarps);
     }
     mbar_init(ofinal, 1);
-    mbar_init(wgbar, pf::kSoftmaxWarps);
+    mbar_init(qready, pf::kSoftmaxWarps);
     *s_abort = 0;
     if (smem_u32(smem) & 1023) record_error(KVATTN_ERR_INVALID_ARG);
     fence_barrier_init();
@@ -141,49 +164,44 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     tc::tmem_alloc(tmem_base_s, pf::kTmemCols);
     tc::tmem_relinquish();
   }
-  // ---- Q tile: bf16 -> f16 * log2(e)/16, swizzled K-major (dequant warps) ----
-  if (threadIdx.x >= pf::kDq0) {
-    const int d = threadIdx.x - pf::kDq0;  // 0..255
-    const int r = d >> 1, hq = d & 1;       // row, which 128 channels
-    const int R = row0 + r;
-    const uint16_t* src = nullptr;
-    if (R < n_rows) {
-      const int t = R / p.group, j = R % p.group;
-      src = p.q + (static_cast<long long>(t) * p.n_qh + h * p.group + j) * kHeadDim + hq * 128;
-    }
-    const float sc = 1.4426950408889634f / 16.0f;
-#pragma unroll 4
-    for (int c = 0; c < 16; ++c) {  // 16 chunks of 8 channels
-      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-      if (src) raw = *reinterpret_cast<const uint4*>(src + c * 8);
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-      uint32_t o[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float lo = __uint_as_float(w[e] << 16) * sc;
-        const float hi = __uint_as_float(w[e] & 0xFFFF0000u) * sc;
-        o[e] = pack_half2(lo, hi);
-      }
-      const int chan = hq * 128 + c * 8;
-      const int atom = chan >> 6, chunk = (chan & 63) >> 3;
-      uint4* dst = reinterpret_cast<uint4*>(smem + pf::kQOff + atom * 16384 + swz(r, chunk));
-      *dst = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-    tc::fence_proxy_async_smem();
-  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_base_s;
 
-  if (warp == pf::kMmaWarp) {
+  if (warp == pf::kLoadWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int j = 0;
+      for (int i = 0; i < n_cand; ++i) {
+        PfTile tl;
+        if (!pf_tile(p, h, ks, i, np, max_qpos, &tl)) continue;
+        const int r = j & 1;
+        if (j >= 2 && !mbar_wait(&rawempty[r], ((j - 2) >> 1) & 1)) {
+          *s_abort = 1;
+          break;
+        }
+        uint8_t* st = smem + pf::kRawOff + r * pf::kRawBytes;
+        const uint8_t* kp = p.k_pool + static_cast<int64_t>(tl.page) * p.k_stride;
+        const uint8_t* vp = p.v_pool + static_cast<int64_t>(tl.page) * p.v_stride;
+        mbar_arrive_expect_tx(&rawfull[r], pf::kRawBytes);
+        bulk_g2s(st, kp + tl.half * pf::kRawKc, pf::kRawKc, &rawfull[r]);
+        bulk_g2s(st + pf::kRawKc, kp + kKScaleOffset + tl.half * pf::kRawKs, pf::kRawKs, &rawfull[r]);
+        bulk_g2s(st + pf::kRawKc + pf::kRawKs, vp + tl.half * pf::kRawVc, pf::kRawVc, &rawfull[r]);
+        bulk_g2s(st + pf::kRawKc + pf::kRawKs + pf::kRawVc, vp + kV4ScaleOffset + tl.half * pf::kRawVs, pf::kRawVs,
+                 &rawfull[r]);
+        ++j;
+      }
+      // every copy issued must land before the CTA may exit
+      for (int jj = j - 2 < 0 ? 0 : j - 2; jj < j; ++jj) mbar_wait(&rawfull[jj & 1], (jj >> 1) & 1);
+    }
+  } else if (warp == pf::kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t q_base = smem_u32(smem + pf::kQOff);
       const uint32_t k_base = smem_u32(smem + pf::kKOff);
       const uint32_t v_base = smem_u32(smem + pf::kVOff);
-      const uint32_t p_base = smem_u32(smem + pf::kPOff);
-      int j = 0;  // valid tiles issued (QK)
+      int j = 0;
+      bool ok = mbar_wait(qready, 0);
       auto issue_pv = [&](int jj) -> bool {
         const int b = jj & 1;
         const uint32_t par = (jj >> 1) & 1;
@@ -191,32 +209,27 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         tc::fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
-#pragma unroll
-          for (int a = 0; a < 2; ++a) {
-            const uint64_t ad = tc::sw128_desc(v_base + b * 32768 + a * 16384 + kk * 32, 1024, 16);
-            const uint64_t bd = tc::sw128_desc(p_base + b * 16384 + kk * 32, 1024, 16);
-            tc::mma_f16_ss(tmem + pf::kOCol0 + a * 128, ad, bd, pf::kIdescPV, (jj > 0 || kk > 0) ? 1u : 0u);
-          }
+          const uint64_t bd = tc::sw128_desc(v_base + b * 32768 + kk * 32, 1024, 16);
+          mma_f16_ts(tmem + pf::kOCol0, tmem + pf::kSCol0 + b * pf::kKeys + kk * 8, bd, pf::kIdescPV,
+                     (jj > 0 || kk > 0) ? 1u : 0u);
         }
         tc::commit(&vfree[b]);
         return true;
       };
-      bool ok = true;
       for (int i = 0; i < n_cand && ok; ++i) {
         PfTile tl;
         if (!pf_tile(p, h, ks, i, np, max_qpos, &tl)) continue;
         const int b = j & 1;
-        const uint32_t par = (j >> 1) & 1;
-        if (!mbar_wait(&kready[b], par)) {
+        if (!mbar_wait(&kready[b], (j >> 1) & 1)) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-          const uint64_t ad = tc::sw128_desc(q_base + (kk >> 2) * 16384 + (kk & 3) * 32, 1024, 16);
           const uint64_t bd = tc::sw128_desc(k_base + b * 32768 + (kk >> 2) * 8192 + (kk & 3) * 32, 1024, 16);
-          tc::mma_f16_ss(tmem + pf::kSCol0 + b * pf::kKeys, ad, bd, pf::kIdescQK, kk > 0 ? 1u : 0u);
+          mma_f16_ts(tmem + pf::kSCol0 + b * pf::kKeys, tmem + pf::kQCol0 + kk * 8, bd, pf::kIdescQK,
+                     kk > 0 ? 1u : 0u);
         }
         tc::commit(&sready[b]);
         tc::commit(&kfree[b]);
@@ -225,7 +238,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       }
       if (ok && j >= 1) ok = issue_pv(j - 1);
       if (!ok) *s_abort = 1;
-      tc::commit(ofinal);  // arrives when every MMA above has completed
+      tc::commit(ofinal);    // arrives when every MMA above has completed
       mbar_wait(ofinal, 0);  // no MMA may still run when the tensor memory is freed
     }
   } else if (warp < pf::kSoftmaxWarps) {
@@ -233,42 +246,62 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     const int r = threadIdx.x;  // 0..127 == TMEM lane
     const int R = row0 + r;
     const int qpos = R < n_rows ? p.q_pos[R / p.group] : INT_MAX;
-    const uint32_t lane_base = tmem + ((static_cast<uint32_t>(warp) * 32) << 16);
+    const uint32_t lane_base = tmem_lane(tmem, warp);
+    // ---- Q row: bf16 -> f16 * log2(e)/16 into tensor memory (A operand of S = Q K^T) ----
+    {
+      const uint16_t* src = nullptr;
+      if (R < n_rows) {
+        const int t = R / p.group, jq = R % p.group;
+        src = p.q + (static_cast<long long>(t) * p.n_qh + h * p.group + jq) * kHeadDim;
+      }
+      const float sc = 1.4426950408889634f / 16.0f;
+      for (int c0 = 0; c0 < 4; ++c0) {  // 64 channels = 32 columns at a time
+        uint32_t w[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+          if (src) raw = *reinterpret_cast<const uint4*>(src + c0 * 64 + c * 8);
+          const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w[c * 4 + e] = pack_half2(__uint_as_float(in[e] << 16) * sc, __uint_as_float(in[e] & 0xFFFF0000u) * sc);
+        }
+        tc::st32(lane_base + pf::kQCol0 + c0 * 32, w);
+      }
+      tc::wait_st();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qready);
+    }
     float m_ref = -INFINITY, l_sum = 0.f;
-    uint32_t wg_phase = 0;
     int j = 0;
     bool ok = true;
     for (int i = 0; i < n_cand && ok; ++i) {
       PfTile tl;
       if (!pf_tile(p, h, ks, i, np, max_qpos, &tl)) continue;
       const int b = j & 1;
-      const uint32_t par = (j >> 1) & 1;
-      if (!mbar_wait(&sready[b], par)) {
+      if (!mbar_wait(&sready[b], (j >> 1) & 1)) {
         ok = false;
         break;
       }
       tc::fence_after_sync();
-      float s[pf::kKeys];
-      {
-        uint32_t v[32];
-        tc::ld32(lane_base + pf::kSCol0 + b * pf::kKeys, v);
-        tc::wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(v[c]);
-        tc::ld32(lane_base + pf::kSCol0 + b * pf::kKeys + 32, v);
-        tc::wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) s[32 + c] = __uint_as_float(v[c]);
-      }
+      // two passes over the 64 scores (32 columns at a time) keep register pressure low:
+      // the maximum first, then P; the second pass reads S from tensor memory again
       const int key0 = tl.logical * kPageTokens + tl.half * pf::kKeys;
-      if (key0 + pf::kKeys - 1 > qpos) {
-#pragma unroll
-        for (int c = 0; c < pf::kKeys; ++c)
-          if (key0 + c > qpos) s[c] = -INFINITY;
-      }
+      const bool masked = key0 + pf::kKeys - 1 > qpos;
+      const uint32_t scol = lane_base + pf::kSCol0 + b * pf::kKeys;
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < pf::kKeys; ++c) mx = fmaxf(mx, s[c]);
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t v[32];
+        tc::ld32(scol + 32 * hh, v);
+        tc::wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float x = (masked && key0 + 32 * hh + c > qpos) ? -INFINITY : __uint_as_float(v[c]);
+          mx = fmaxf(mx, x);
+        }
+      }
       float alpha = 1.f;
       bool resc = false;
       if (mx > m_ref + 8.f) {
@@ -277,146 +310,150 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         l_sum *= alpha;
         m_ref = mx;
       }
-      // rescale O^T columns of the rows whose maximum jumped (rare)
-      // (double-buffered by tile parity: a warp can run at most one rendezvous ahead)
-      int* any_b = s_any + 4 * b;
-      float* alpha_b = s_alpha + pf::kRows * b;
-      const unsigned any = __ballot_sync(0xffffffffu, resc);
-      if (lane == 0) any_b[warp] = any != 0;
-      alpha_b[r] = resc ? alpha : 1.f;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(wgbar);
-      if (!mbar_wait(wgbar, wg_phase)) {
-        ok = false;
-        break;
-      }
-      wg_phase ^= 1;
-      if (any_b[0] | any_b[1] | any_b[2] | any_b[3]) {
-        // O^T must hold the previous tile's PV before it is rescaled
+      if (__any_sync(0xffffffffu, resc)) {
+        // this warp's rows of O hold the previous tile's PV only once it completed
         if (!mbar_wait(&vfree[(j - 1) & 1], ((j - 1) >> 1) & 1)) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
-        for (int a = 0; a < 2; ++a) {
-          for (int c0 = 0; c0 < pf::kRows; c0 += 32) {
-            uint32_t v[32];
-            tc::ld32(lane_base + pf::kOCol0 + a * 128 + c0, v);
-            tc::wait_ld();
+        const float f = resc ? alpha : 1.f;
+        for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
+          uint32_t v[32];
+          tc::ld32(lane_base + pf::kOCol0 + c0, v);
+          tc::wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) * alpha_b[c0 + c]);
-            tc::st32(lane_base + pf::kOCol0 + a * 128 + c0, v);
-          }
+          for (int c = 0; c < 32; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) * f);
+          tc::st32(lane_base + pf::kOCol0 + c0, v);
         }
         tc::wait_st();
       }
       const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-      // P buffer b was last read by the PV of tile j-2
-      if (j >= 2 && !mbar_wait(&vfree[b], ((j - 2) >> 1) & 1)) {
-        ok = false;
-        break;
-      }
-      uint8_t* prow = smem + pf::kPOff + b * 16384;
 #pragma unroll
-      for (int c8 = 0; c8 < pf::kKeys / 8; ++c8) {
-        uint32_t w[4];
+      for (int hh = 0; hh < 2; ++hh) {  // P as f16 pairs over the first 32 columns of S
+        uint32_t v[32];
+        tc::ld32(scol + 32 * hh, v);
+        tc::wait_ld();
+        uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = fast_exp2(s[c8 * 8 + 2 * e] - mu);
-          const float p1 = fast_exp2(s[c8 * 8 + 2 * e + 1] - mu);
+        for (int c = 0; c < 16; ++c) {
+          const float s0 = (masked && key0 + 32 * hh + 2 * c > qpos) ? -INFINITY : __uint_as_float(v[2 * c]);
+          const float s1 = (masked && key0 + 32 * hh + 2 * c + 1 > qpos) ? -INFINITY : __uint_as_float(v[2 * c + 1]);
+          const float p0 = fast_exp2(s0 - mu), p1 = fast_exp2(s1 - mu);
           l_sum += p0 + p1;
-          w[e] = pack_half2(p0, p1);
+          w[c] = pack_half2(p0, p1);
         }
-        *reinterpret_cast<uint4*>(prow + swz(r, c8)) = make_uint4(w[0], w[1], w[2], w[3]);
+        // the first half's P lands in columns 0-15, which the second half no longer reads
+        tc::st16(scol + 16 * hh, w);
       }
-      tc::fence_proxy_async_smem();
+      tc::wait_st();
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&pready[b]);
       ++j;
     }
-    if (!ok) *s_abort = 1;
-    // ---- epilogue: normalised partial (o, lse) of every row of the tile ----
-    s_l[r] = l_sum;
-    s_m[r] = m_ref;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(wgbar);
-    const bool ok2 = mbar_wait(wgbar, wg_phase);
-    wg_phase ^= 1;
+    // ---- epilogue: normalised partial (o, lse) of this row ----
     bool have = false;
-    if (ok && ok2 && j > 0) {
+    if (ok && j > 0) {
       have = mbar_wait(ofinal, 0);
       ok = have;
     }
-    if (!ok || !ok2) *s_abort = 1;
+    if (!ok) *s_abort = 1;
     tc::fence_after_sync();
     const bool direct = p.n_ks == 1;
-    for (int a = 0; a < 2; ++a) {
-      const int dim = a * 128 + r;
-      for (int c0 = 0; c0 < pf::kRows; c0 += 32) {
-        uint32_t v[32];
-        if (have) {
-          tc::ld32(lane_base + pf::kOCol0 + a * 128 + c0, v);
-          tc::wait_ld();
-        }
-#pragma unroll 4
-        for (int c = 0; c < 32; ++c) {
-          const int rr = c0 + c, RR = row0 + rr;
-          if (RR >= n_rows) break;
-          const float lr = s_l[rr];
-          const float o = (have && lr > 0.f) ? __uint_as_float(v[c]) / lr : 0.f;
-          if (direct) {
-            const int t = RR / p.group, jj = RR % p.group;
-            p.out[(static_cast<long long>(t) * p.n_qh + h * p.group + jj) * kHeadDim + dim] = o;
-          } else {
-            p.part_o[((static_cast<long long>(h) * p.n_ks + ks) * p.rows_pad + RR) * kHeadDim + dim] = o;
-          }
-        }
+    float* dst = nullptr;
+    if (R < n_rows) {
+      if (direct) {
+        const int t = R / p.group, jq = R % p.group;
+        dst = p.out + (static_cast<long long>(t) * p.n_qh + h * p.group + jq) * kHeadDim;
+      } else {
+        dst = p.part_o + ((static_cast<long long>(h) * p.n_ks + ks) * p.rows_pad + R) * kHeadDim;
+      }
+    }
+    const float inv = (have && l_sum > 0.f) ? 1.f / l_sum : 0.f;
+    const bool warp_have = __any_sync(0xffffffffu, have);
+    for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
+      uint32_t v[32];
+      if (warp_have) {  // the load is warp-collective
+        tc::ld32(lane_base + pf::kOCol0 + c0, v);
+        tc::wait_ld();
+      }
+      if (!have) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) v[c] = 0u;
+      }
+      if (dst) {
+#pragma unroll
+        for (int c = 0; c < 32; c += 4)
+          *reinterpret_cast<float4*>(dst + c0 + c) =
+              make_float4(__uint_as_float(v[c]) * inv, __uint_as_float(v[c + 1]) * inv,
+                          __uint_as_float(v[c + 2]) * inv, __uint_as_float(v[c + 3]) * inv);
       }
     }
     if (R < n_rows) {
       const float l2 = (have && l_sum > 0.f) ? m_ref + log2f(l_sum) : -INFINITY;
       if (direct) {
-        const int t = R / p.group, jj = R % p.group;
-        p.lse[static_cast<long long>(t) * p.n_qh + h * p.group + jj] = l2 * 0.69314718055994531f;
+        const int t = R / p.group, jq = R % p.group;
+        p.lse[static_cast<long long>(t) * p.n_qh + h * p.group + jq] = l2 * 0.69314718055994531f;
       } else {
         p.part_lse[(static_cast<long long>(h) * p.n_ks + ks) * p.rows_pad + R] = l2;
       }
     }
-  } else if (warp > pf::kMmaWarp) {
+  } else if (warp >= pf::kDq0 / 32) {
     // ------------------------------------------------------------ dequant (256 threads)
     const int d = threadIdx.x - pf::kDq0;
-    // K task: key n of the tile, channel quarter P (blocks 2P, 2P+1)
-    const int kn = d >> 2, kP = d & 3;
-    // V task: 16-key group G', block pair C, row R (channels R + 8k of both blocks), half h8
-    const int vG = d >> 6, vC = (d >> 4) & 3, vR = (d >> 1) & 7, vh = d & 1;
+    // K task: channel quarter kP (blocks 2kP, 2kP+1) of key kn; 8 consecutive threads take
+    // 8 consecutive keys, so their swizzled 16-byte stores hit 8 different bank groups.
+    const int kP = d >> 6, kn = d & 63;
+    const int kG = kn >> 4, kH = (kn >> 3) & 1, kR = kn & 7;
+    // V task: token group vG (16 keys), block pair vC, channel row vR (channels vR + 8k of
+    // both blocks), key half vh (keys 8vh..8vh+7 of the group)
+    const int vR = d & 7, vh = (d >> 3) & 1, vC = (d >> 4) & 3, vG = d >> 6;
+    // 16-byte chunks are read in an order rotated by (row / 2): 8 threads at a 64-byte
+    // stride then touch 8 different bank groups
+    const int rotK = kR >> 1, rotV = vR >> 1;
     int j = 0;
     bool ok = true;
     for (int i = 0; i < n_cand && ok; ++i) {
       PfTile tl;
       if (!pf_tile(p, h, ks, i, np, max_qpos, &tl)) continue;
-      const int b = j & 1;
-      const uint8_t* kp = p.k_pool + static_cast<int64_t>(tl.page) * p.k_stride;
-      const uint8_t* vp = p.v_pool + static_cast<int64_t>(tl.page) * p.v_stride;
-      // ---------------- K^ ----------------
-      {
-        const int tok = tl.half * pf::kKeys + kn;
-        const int G = tok >> 4, H = (tok >> 3) & 1, R = tok & 7;
-        const uint4* src = reinterpret_cast<const uint4*>(kp + ((((G * 4 + kP) * 2 + H) * 8 + R) * 4) * 16);
-        uint4 raw[4];
+      const int b = j & 1, r = j & 1;
+      if (!mbar_wait(&rawfull[r], (j >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      const uint32_t stu = smem_u32(smem + pf::kRawOff + r * pf::kRawBytes);
+      // ---------------- raw K, V -> registers; the stage is then released ----------------
+      uint4 kraw[4];
+      const uint32_t kbase = stu + ((((kG * 4 + kP) * 2 + kH) * 8 + kR) * 4) * 16;
 #pragma unroll
-        for (int T = 0; T < 4; ++T) raw[T] = src[T];
-        const uint32_t dkw = *reinterpret_cast<const uint32_t*>(kp + kKScaleOffset + 2 * (((G * 8 + R) * 2 + H) * 8 + 2 * kP));
+      for (int ii = 0; ii < 4; ++ii) kraw[ii] = lds128(kbase + (((ii + rotK) & 3) << 4));
+      uint32_t dkw;
+      asm volatile("ld.shared.u32 %0, [%1];"
+                   : "=r"(dkw)
+                   : "r"(stu + pf::kRawKc + ((kG * 8 + kR) * 2 + kH) * 16 + 4 * kP));
+      uint4 vraw[4], dvr[4];
+      const uint32_t vbase = stu + pf::kRawKc + pf::kRawKs + ((((vG * 4 + vC) * 8 + vR) * 4) * 16);
+#pragma unroll
+      for (int ii = 0; ii < 4; ++ii) vraw[ii] = lds128(vbase + (((ii + rotV) & 3) << 4));
+#pragma unroll
+      for (int T = 0; T < 4; ++T)
+        dvr[T] = lds128(stu + pf::kRawKc + pf::kRawKs + pf::kRawVc + ((vG * 4 + T) * 8 + 2 * vC) * 8);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rawempty[r]);
+      // ---------------- K^ ----------------
+      if (j >= 2 && !mbar_wait(&kfree[b], ((j - 2) >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      {
         const uint32_t dlo = prmt(dkw, 0u, 0x1010u), dhi = prmt(dkw, 0u, 0x3232u);
-        if (j >= 2 && !mbar_wait(&kfree[b], ((j - 2) >> 1) & 1)) {
-          ok = false;
-          break;
-        }
         uint8_t* katom = smem + pf::kKOff + b * 32768 + kP * 8192;
 #pragma unroll
-        for (int T = 0; T < 4; ++T) {
-          const uint32_t w[4] = {raw[T].x ^ 0x80808080u, raw[T].y ^ 0x80808080u, raw[T].z ^ 0x80808080u,
-                                 raw[T].w ^ 0x80808080u};
+        for (int ii = 0; ii < 4; ++ii) {
+          const int T = (ii + rotK) & 3;
+          const uint32_t w[4] = {kraw[ii].x ^ 0x80808080u, kraw[ii].y ^ 0x80808080u, kraw[ii].z ^ 0x80808080u,
+                                 kraw[ii].w ^ 0x80808080u};
           uint32_t o[8];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -427,37 +464,40 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
           *reinterpret_cast<uint4*>(katom + swz(kn, T)) = make_uint4(o[0], o[1], o[2], o[3]);
           *reinterpret_cast<uint4*>(katom + swz(kn, 4 + T)) = make_uint4(o[4], o[5], o[6], o[7]);
         }
-        tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&kready[b]);
       }
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&kready[b]);
       // ---------------- V^T ----------------
+      if (j >= 2 && !mbar_wait(&vfree[b], ((j - 2) >> 1) & 1)) {
+        ok = false;
+        break;
+      }
       {
-        const int G = tl.half * 4 + vG;  // 16-token group inside the page
-        const uint4* src = reinterpret_cast<const uint4*>(vp + ((((G * 4 + vC) * 8 + vR) * 4) * 16));
-        uint4 raw[4], dvr[4];
-#pragma unroll
-        for (int T = 0; T < 4; ++T) {
-          raw[T] = src[T];
-          dvr[T] = *reinterpret_cast<const uint4*>(vp + kV4ScaleOffset + 2 * (((G * 4 + T) * 8 + 2 * vC) * 4));
-        }
-        if (j >= 2 && !mbar_wait(&vfree[b], ((j - 2) >> 1) & 1)) {
-          ok = false;
-          break;
-        }
         uint8_t* vt = smem + pf::kVOff + b * 32768;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {  // block 2C + e
           uint32_t o[4][4];            // [k][T]
 #pragma unroll
-          for (int T = 0; T < 4; ++T) {
-            const uint32_t W = e ? (vh ? raw[T].w : raw[T].z) : (vh ? raw[T].y : raw[T].x);
-            const uint32_t dv = e ? (vh ? dvr[T].w : dvr[T].z) : (vh ? dvr[T].y : dvr[T].x);
+          for (int ii = 0; ii < 4; ++ii) {
+            const uint32_t W = e ? (vh ? vraw[ii].w : vraw[ii].z) : (vh ? vraw[ii].y : vraw[ii].x);
             const uint32_t Ws = W >> 8;
-            o[0][T] = hmul2(hsub2(and_or(W, 0x000F000Fu, 0x64006400u), 0x64086408u), dv);
-            o[1][T] = hmul2(hfma2(and_or(W, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u), dv);
-            o[2][T] = hmul2(hsub2(and_or(Ws, 0x000F000Fu, 0x64006400u), 0x64086408u), dv);
-            o[3][T] = hmul2(hfma2(and_or(Ws, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u), dv);
+            const uint32_t v0 = hsub2(and_or(W, 0x000F000Fu, 0x64006400u), 0x64086408u);
+            const uint32_t v1 = hfma2(and_or(W, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
+            const uint32_t v2 = hsub2(and_or(Ws, 0x000F000Fu, 0x64006400u), 0x64086408u);
+            const uint32_t v3 = hfma2(and_or(Ws, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
+            // chunk ii holds token pair T = (ii + rotV) & 3; scale by that pair's fp16 scales
+            // (select with constant register indices)
+#pragma unroll
+            for (int T = 0; T < 4; ++T) {
+              if (T == ((ii + rotV) & 3)) {
+                const uint32_t dv = e ? (vh ? dvr[T].w : dvr[T].z) : (vh ? dvr[T].y : dvr[T].x);
+                o[0][T] = hmul2(v0, dv);
+                o[1][T] = hmul2(v1, dv);
+                o[2][T] = hmul2(v2, dv);
+                o[3][T] = hmul2(v3, dv);
+              }
+            }
           }
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -465,10 +505,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
             *reinterpret_cast<uint4*>(vt + swz(dim, 2 * vG + vh)) = make_uint4(o[k][0], o[k][1], o[k][2], o[k][3]);
           }
         }
-        tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&vready[b]);
       }
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&vready[b]);
       ++j;
     }
     if (!ok) *s_abort = 1;
@@ -476,7 +516,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
 
   tc::fence_before_sync();
   __syncthreads();
-  if (*s_abort) record_error(KVATTN_ERR_TIMEOUT);
+  if (*s_abort && threadIdx.x == 0) record_error(KVATTN_ERR_TIMEOUT);
   if (warp == pf::kMmaWarp) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, pf::kTmemCols);
@@ -492,12 +532,18 @@ struct PrefillPlan {
   size_t lse_off, o_off, bytes;
 };
 
-PrefillPlan plan_prefill(int n_kv, int group, int n_q, int max_pages, int kv_split_tokens) {
+// A CTA walks `spc` consecutive KV splits, merging them online in tensor memory, as long as
+// the grid keeps at least ~16 waves of CTAs: fewer partials to write and merge.
+PrefillPlan plan_prefill(int n_kv, int group, int n_q, int max_pages, int kv_split_tokens, int sm_count) {
   PrefillPlan pl{};
   const int rows = n_q * group;
   pl.n_mt = (rows + pf::kRows - 1) / pf::kRows;
   pl.rows_pad = pl.n_mt * pf::kRows;
-  pl.pps = kv_split_tokens / kPageTokens;
+  const int base = kv_split_tokens / kPageTokens;
+  const long long splits0 = max_pages > 0 ? (max_pages + base - 1) / base : 1;
+  long long spc = static_cast<long long>(n_kv) * pl.n_mt * splits0 / (static_cast<long long>(sm_count) * 16);
+  spc = spc < 1 ? 1 : (spc > splits0 ? splits0 : spc);
+  pl.pps = static_cast<int>(base * spc);
   pl.n_ks = max_pages > 0 ? (max_pages + pl.pps - 1) / pl.pps : 1;
   pl.lse_off = 0;
   pl.o_off = ((sizeof(float) * static_cast<size_t>(n_kv) * pl.n_ks * pl.rows_pad + 255) / 256) * 256;
