@@ -44,7 +44,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extra-steps", type=int, default=100)
     ap.add_argument("--prefill-layers", type=int, default=0, help="layers of the prefill workload (0 = 16)")
-    ap.add_argument("--profile", choices=["none", "decode", "prefill", "verify"], default="none",
+    ap.add_argument("--profile", choices=["none", "decode", "prefill", "verify", "stream"], default="none",
                     help="profiling only: run just this workload's steps (no JSON bench line)")
     ap.add_argument("--context", type=int, default=0, help="profiling only: prior-context override")
     ap.add_argument("--layers", type=int, default=0,
@@ -349,6 +349,221 @@ class PrefillBench:
             self.layer(l)
 
 
+class StreamBench:
+    """Host-streamed decode: the full 524,288-token cache of 16 layers x 4 KV heads sits in
+    pinned host RAM (K|V interleaved per page); per layer the retrieval query selects 256
+    blocks per KV head, a copy kernel brings those pages into device slots on a side stream
+    (layer L+1 while layer L decodes; the tail page stays resident), the new token is
+    quantize-appended into the tail page and written back to host RAM, and decode attends over
+    the 256 + 1 pages."""
+
+    PAGE = 34816 + 18432
+
+    def __init__(self, kv, device, layers=0, context=0):
+        import dataclasses
+
+        import torch
+
+        w = WORKLOADS["stream524k"]
+        if layers:
+            w = dataclasses.replace(w, layers=layers)
+        if context:
+            w = dataclasses.replace(w, context=context)
+        self.kv, self.w, self.device = kv, w, device
+        L, H, Hq, g = w.layers, w.kv_heads, w.q_heads, w.group
+        self.n_full = w.context // 128
+        self.nb = self.n_full + 1
+        self.budget = w.budget_blocks
+        self.cap = self.budget + 1
+        P = self.PAGE
+        # ---- build: per layer on the device, then into pinned host RAM ----
+        self.host = torch.empty((L * H * self.nb, P), dtype=torch.uint8).pin_memory()
+        self.summ = torch.zeros((L * H, self.nb, 256), device=device)
+        tmp = torch.zeros((H * self.nb, P), dtype=torch.uint8, device=device)
+        tdesc = kv.make_desc(H, Hq, tmp, tmp.data_ptr() + 34816, H * self.nb, k_page_stride=P, v_page_stride=P)
+        ttab = torch.arange(H * self.nb, dtype=torch.int32, device=device).view(H, self.nb)
+        for l in range(L):
+            k = torch_normal(derived_seed(w.seed, 10, l), (w.context, H, 256), device)
+            v = torch_normal(derived_seed(w.seed, 11, l), (w.context, H, 256), device)
+            tmp.zero_()
+            kv.kvattn_quantize_append(tdesc, k, v, w.context, 0, ttab, self.nb)
+            del k, v
+            kv.kvattn_block_summaries(tdesc, ttab, H, self.nb, 0, self.n_full, self.summ[l * H:(l + 1) * H])
+            self.host[l * H * self.nb:(l + 1) * H * self.nb].copy_(tmp)
+        del tmp
+        torch.cuda.synchronize()
+        # host page ids per (layer, head, block)
+        self.host_table = torch.arange(L * H * self.nb, dtype=torch.int32, device=device).view(L, H, self.nb)
+        # ---- device slots: 2 buffers x H x budget streamed pages + L x H resident tail pages ----
+        self.n_stream_slots = 2 * H * self.budget
+        self.n_slots = self.n_stream_slots + L * H
+        self.slots = torch.zeros((self.n_slots, P), dtype=torch.uint8, device=device)
+        for l in range(L):
+            for h in range(H):
+                self.slots[self.n_stream_slots + l * H + h].copy_(self.host[(l * H + h) * self.nb + self.n_full])
+        self.desc = kv.make_desc(H, Hq, self.slots, self.slots.data_ptr() + 34816, self.n_slots, k_page_stride=P,
+                                 v_page_stride=P)
+        # per buffer: gather destinations (-1 for the tail entry) and the decode page lists
+        self.dst = []
+        self.plist = []
+        for b in range(2):
+            base = b * H * self.budget
+            self.dst.append(torch.tensor([[base + h * self.budget + i if i < self.budget else -1 for i in range(self.cap)]
+                                          for h in range(H)], dtype=torch.int32, device=device))
+        for l in range(L):
+            b = l % 2
+            base = b * H * self.budget
+            self.plist.append(torch.tensor([[base + h * self.budget + i if i < self.budget
+                                             else self.n_stream_slots + l * H + h for i in range(self.cap)]
+                                            for h in range(H)], dtype=torch.int32, device=device))
+        # tail page table for the append: logical block n_full -> the layer's tail slot
+        self.tail_tab = torch.full((L, H, self.nb), 0, dtype=torch.int32, device=device)
+        for l in range(L):
+            for h in range(H):
+                self.tail_tab[l, h, :] = self.n_stream_slots + l * H + h
+        self.tail_host = torch.tensor([[(l * H + h) * self.nb + self.n_full for h in range(H)] for l in range(L)],
+                                      dtype=torch.int32, device=device)
+        self.tail_slot = torch.tensor([[self.n_stream_slots + l * H + h for h in range(H)] for l in range(L)],
+                                      dtype=torch.int32, device=device)
+        # selection outputs and workspaces
+        self.sel_l = torch.zeros((L, H, self.cap), dtype=torch.int32, device=device)
+        self.sel_p = torch.zeros((L, H, self.cap), dtype=torch.int32, device=device)
+        self.n_sel = torch.zeros((L, H), dtype=torch.int32, device=device)
+        self.sws_bytes = kv.kvattn_select_workspace_size(H, self.nb)
+        self.sws = torch.zeros((L, self.sws_bytes), dtype=torch.uint8, device=device)
+        self.ws_bytes = kv.kvattn_decode_workspace_size(self.desc, 1, self.cap)
+        self.ws = torch.zeros((L, max(self.ws_bytes, 256)), dtype=torch.uint8, device=device)
+        # per-step inputs
+        self.q = torch_normal(derived_seed(w.seed, 20), (L, 1, Hq, 256), device)
+        self.q_group = self.q[:, 0].reshape(L, H, g, 256).contiguous()
+        self.k_new = torch_normal(derived_seed(w.seed, 21), (L, 1, H, 256), device)
+        self.v_new = torch_normal(derived_seed(w.seed, 22), (L, 1, H, 256), device)
+        self.pos = w.context
+        self.q_pos = torch.tensor([self.pos], dtype=torch.int32, device=device)
+        self.out = torch.empty((L, 1, Hq, 256), device=device)
+        self.lse = torch.empty((L, 1, Hq), device=device)
+        self.copy_stream = torch.cuda.Stream(device=device)
+        self.ev_sel = [torch.cuda.Event() for _ in range(L)]
+        self.ev_copy = [torch.cuda.Event() for _ in range(L)]
+        self.ev_dec = [torch.cuda.Event() for _ in range(L)]
+        self.copy_bytes_per_step = L * H * self.budget * P
+        tokens = self.budget * 128 + 1
+        self.attn_bytes_per_step = L * H * tokens * BYTES_PER_TOKEN_HEAD["q4_0"]
+        self.launches_per_step = 5 * L
+        self.gather_ctas = 16
+
+    def _select(self, l):
+        w = self.w
+        self.kv.kvattn_select_blocks(self.summ[l * w.kv_heads:(l + 1) * w.kv_heads], self.q_group[l], w.kv_heads,
+                                     w.group, self.nb, self.n_full, self.nb, self.budget, 0, self.host_table[l],
+                                     self.sel_l[l], self.sel_p[l], self.n_sel[l], self.cap, self.sws[l],
+                                     self.sws_bytes)
+
+    def _gather(self, l, stream):
+        H = self.w.kv_heads
+        self.kv.kvattn_gather_pages(self.host, self.PAGE, self.host.shape[0], self.slots, self.PAGE, self.n_slots,
+                                    self.PAGE, self.sel_p[l], self.dst[l % 2], H * self.cap, self.gather_ctas,
+                                    stream)
+
+    def _attend(self, l, timed=None):
+        kv, w = self.kv, self.w
+        kv.kvattn_quantize_append(self.desc, self.k_new[l], self.v_new[l], 1, self.pos, self.tail_tab[l], self.nb)
+        if timed is not None:
+            timed[0].record()
+        kv.kvattn_decode(self.desc, self.q[l], 1, self.q_pos, self.plist[l], self.sel_l[l], self.n_sel[l], self.cap,
+                         self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
+        if timed is not None:
+            timed[1].record()
+        kv.kvattn_scatter_pages(self.host, self.PAGE, self.host.shape[0], self.slots, self.PAGE, self.n_slots,
+                                self.PAGE, self.tail_host[l], self.tail_slot[l], w.kv_heads, 4)
+
+    def step(self, stream_pages=True, timed=None):
+        import torch
+
+        L = self.w.layers
+        main = torch.cuda.current_stream()
+        cs = self.copy_stream
+        self._select(0)
+        self.ev_sel[0].record(main)
+        if stream_pages:
+            cs.wait_event(self.ev_sel[0])
+            self._gather(0, cs)
+            self.ev_copy[0].record(cs)
+        for l in range(L):
+            if l + 1 < L:
+                self._select(l + 1)
+                self.ev_sel[l + 1].record(main)
+                if stream_pages:
+                    cs.wait_event(self.ev_sel[l + 1])
+                    if l >= 1:
+                        cs.wait_event(self.ev_dec[l - 1])  # buffer (l+1)%2 was read by layer l-1
+                    self._gather(l + 1, cs)
+                    self.ev_copy[l + 1].record(cs)
+            if stream_pages:
+                main.wait_event(self.ev_copy[l])
+            self._attend(l, timed[l] if timed is not None else None)
+            self.ev_dec[l].record(main)
+
+    def copies_only(self):
+        import torch
+
+        cs = torch.cuda.current_stream()
+        for l in range(self.w.layers):
+            self._gather(l, cs)
+
+
+def time_stream(b, steps, warmup):
+    """T_stream (pipelined), T_resident (no page copies), T_copy (copies alone), decode time."""
+    import torch
+
+    def timed(fn, n, w_):
+        for _ in range(w_):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = event_pair()
+        e0.record()
+        for _ in range(n):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    t_stream = timed(lambda: b.step(True), steps, warmup)
+    t_res = timed(lambda: b.step(False), steps, warmup)
+    t_copy = timed(b.copies_only, steps, warmup)
+    pairs = [event_pair() for _ in range(b.w.layers)]
+    b.step(True, timed=pairs)
+    torch.cuda.synchronize()
+    t_dec = sum(a.elapsed_time(c) for a, c in pairs)
+    return t_stream, t_res, t_copy, t_dec
+
+
+def time_memcpy_route(b):
+    """The same step's page copies through kvattn_stream_pages (one cudaMemcpyAsync per run of
+    consecutive pages, page ids on the host): device time of the copies and host enqueue time."""
+    import torch
+
+    L, H = b.w.layers, b.w.kv_heads
+    for l in range(L):
+        b._select(l)
+    sel = b.sel_p.cpu().numpy()
+    cs = b.copy_stream
+    e0, e1 = event_pair()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    e0.record(cs)
+    n_copies = 0
+    for l in range(L):
+        base = (l % 2) * H * b.budget
+        hid = sel[l, :, :b.budget].reshape(-1)
+        slots = base + np.arange(H * b.budget, dtype=np.int32)
+        n_copies += b.kv.kvattn_stream_pages(b.host, b.PAGE, b.slots, b.PAGE, b.PAGE, hid, slots, copy_stream=cs)
+    e1.record(cs)
+    t_enq = time.perf_counter() - t0
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1), t_enq * 1e3, n_copies
+
+
 def time_steps(bench, steps, warmup, world):
     import torch
 
@@ -515,6 +730,8 @@ def main():
             b = DecodeBench(kvattn, "decode131k", device, layers=args.layers or 2)
         elif args.profile == "verify":
             b = VerifyBench(kvattn, device)
+        elif args.profile == "stream":
+            b = StreamBench(kvattn, device, layers=args.layers or 2, context=args.context)
         else:
             b = PrefillBench(kvattn, device, layers=args.layers or 1, context=args.context)
         for _ in range(args.warmup + args.steps):
@@ -587,6 +804,20 @@ def main():
                                     "flop_per_layer": b4.flops_per_layer,
                                     "peak": f"{peak_kind} dense bf16 (f16 operands run at the same rate)"}
             del b4
+            torch.cuda.empty_cache()
+            b5 = StreamBench(kvattn, device)
+            ts, tr, tcp, td = time_stream(b5, max(3, args.extra_steps // 5), 2)
+            tm, tenq, ncp = time_memcpy_route(b5)
+            extra["stream524k"] = {
+                "ms_per_step": ts, "ms_per_step_resident": tr, "ms_copies_only": tcp, "ms_decode": td,
+                "pcie_GB/s": b5.copy_bytes_per_step / (tcp * 1e-3) / 1e9,
+                "hbm_GB/s_decode": b5.attn_bytes_per_step / (td * 1e-3) / 1e9,
+                "hidden_copy_fraction": max(0.0, 1.0 - (ts - tr) / tcp) if tcp > 0 else None,
+                "copy_bytes_per_step": b5.copy_bytes_per_step,
+                "memcpy_route": {"ms_device": tm, "ms_host_enqueue": tenq, "copies": ncp,
+                                 "pcie_GB/s": b5.copy_bytes_per_step / (max(tm, tenq) * 1e-3) / 1e9},
+                "host_pool_GB": b5.host.numel() / 1e9}
+            del b5
             torch.cuda.empty_cache()
         except Exception as exc:  # report, do not hide
             extra["error"] = repr(exc)

@@ -248,6 +248,28 @@ KVATTN_API int kvattn_stream_pages(const void* host_pool, int64_t host_stride, v
 KVATTN_API int kvattn_stream_plan(const int32_t* host_ids, const int32_t* dev_slots, int n, int32_t* run_first,
                                   int32_t* run_len, int max_runs);
 
+/* Moves pages between a pinned host pool and device slots with a copy kernel that reads (or
+ * writes) the device-mapped host memory directly over PCIe.  The page lists live in device
+ * memory, so a selection computed on the GPU (kvattn_select_blocks) drives the copy with no
+ * host round trip; with n_ctas small the copy shares the GPU with attention running on
+ * another stream.
+ *   host_pool   pinned host memory (cudaHostAlloc or registered; mapped into the device
+ *               address space), n_host_pages pages of host_stride bytes.  Checked on the host:
+ *               anything else (e.g. pageable memory) returns KVATTN_ERR_INVALID_ARG.
+ *   dev_pool    device memory, n_slots slots of dev_stride bytes
+ *   host_ids    device int32 [n]: host page of entry i;  dev_slots device int32 [n]: its slot;
+ *               entries with a negative slot are skipped; ids out of range are skipped and
+ *               set KVATTN_ERR_BAD_PAGE in the device error word
+ *   page_bytes  bytes per page, a multiple of 16 (strides and pointers 16-byte aligned)
+ *   n_ctas      CTAs of the copy kernel (0 = 32)
+ * kvattn_gather_pages copies host -> device, kvattn_scatter_pages device -> host. */
+KVATTN_API int kvattn_gather_pages(const void* host_pool, int64_t host_stride, int64_t n_host_pages, void* dev_pool,
+                                   int64_t dev_stride, int64_t n_slots, int64_t page_bytes, const int32_t* host_ids,
+                                   const int32_t* dev_slots, int n, int n_ctas, kvattn_stream_t stream);
+KVATTN_API int kvattn_scatter_pages(void* host_pool, int64_t host_stride, int64_t n_host_pages, const void* dev_pool,
+                                    int64_t dev_stride, int64_t n_slots, int64_t page_bytes, const int32_t* host_ids,
+                                    const int32_t* dev_slots, int n, int n_ctas, kvattn_stream_t stream);
+
 /* Polls `event` until it completes or timeout_ms elapses (KVATTN_ERR_TIMEOUT). */
 KVATTN_API int kvattn_stream_wait(kvattn_event_t event, int timeout_ms);
 

@@ -17,6 +17,8 @@ cudaError_t launch_merge_lse(const float*, const float*, int, int, int, float*, 
 cudaError_t launch_block_summaries(const kvattn_kv_desc&, const int32_t*, int, int, int, int, float*, cudaStream_t);
 cudaError_t launch_select(const float*, const float*, int, int, int, int, int, int, const int32_t*, int32_t*,
                           int32_t*, int32_t*, int, double*, cudaStream_t);
+cudaError_t launch_page_copy(const void*, int64_t, int64_t, void*, int64_t, int64_t, int64_t, const int32_t*,
+                             const int32_t*, int, int, int, cudaStream_t);
 
 }  // namespace kvattn
 
@@ -326,6 +328,67 @@ KVATTN_API int kvattn_stream_pages(const void* host_pool, int64_t host_stride, v
   }
   if (n_copies) *n_copies = copies;
   return KVATTN_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Device address of a pinned, device-mapped host range; INVALID_ARG for anything else
+// (pageable memory would fault the copy kernel, so it is refused here on the host).
+int mapped_host_range(const void* host, int64_t bytes, void** dev) {
+  if (!host || bytes <= 0 || !aligned16(host)) return KVATTN_ERR_INVALID_ARG;
+  cudaPointerAttributes a{}, b{};
+  if (cudaPointerGetAttributes(&a, host) != cudaSuccess) {
+    cudaGetLastError();
+    return KVATTN_ERR_INVALID_ARG;
+  }
+  const void* last = static_cast<const uint8_t*>(host) + (bytes - 1);
+  if (cudaPointerGetAttributes(&b, last) != cudaSuccess) {
+    cudaGetLastError();
+    return KVATTN_ERR_INVALID_ARG;
+  }
+  if (a.type != cudaMemoryTypeHost || b.type != cudaMemoryTypeHost || !a.devicePointer || !b.devicePointer)
+    return KVATTN_ERR_INVALID_ARG;
+  if (static_cast<const uint8_t*>(b.devicePointer) - static_cast<const uint8_t*>(a.devicePointer) != bytes - 1)
+    return KVATTN_ERR_INVALID_ARG;
+  *dev = a.devicePointer;
+  return KVATTN_OK;
+}
+
+int page_copy_common(const void* host_pool, int64_t host_stride, int64_t n_host_pages, void* dev_pool,
+                     int64_t dev_stride, int64_t n_slots, int64_t page_bytes, const int32_t* host_ids,
+                     const int32_t* dev_slots, int n, int n_ctas, int to_device, kvattn_stream_t stream) {
+  if (n < 0 || n_ctas < 0 || page_bytes <= 0 || (page_bytes & 15) || host_stride < page_bytes ||
+      dev_stride < page_bytes || (host_stride & 15) || (dev_stride & 15) || n_host_pages < 1 || n_slots < 1)
+    return KVATTN_ERR_INVALID_ARG;
+  if (n == 0) return KVATTN_OK;
+  if (!dev_pool || !aligned16(dev_pool) || !host_ids || !dev_slots) return KVATTN_ERR_INVALID_ARG;
+  int dev, st;
+  if ((st = current_device_checked(&dev))) return st;
+  void* hdev = nullptr;
+  if ((st = mapped_host_range(host_pool, (n_host_pages - 1) * host_stride + page_bytes, &hdev))) return st;
+  cudaError_t e = launch_page_copy(hdev, host_stride, n_host_pages, dev_pool, dev_stride, n_slots, page_bytes,
+                                   host_ids, dev_slots, n, n_ctas, to_device, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVATTN_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+KVATTN_API int kvattn_gather_pages(const void* host_pool, int64_t host_stride, int64_t n_host_pages, void* dev_pool,
+                                   int64_t dev_stride, int64_t n_slots, int64_t page_bytes, const int32_t* host_ids,
+                                   const int32_t* dev_slots, int n, int n_ctas, kvattn_stream_t stream) {
+  return page_copy_common(host_pool, host_stride, n_host_pages, dev_pool, dev_stride, n_slots, page_bytes, host_ids,
+                          dev_slots, n, n_ctas, 1, stream);
+}
+
+KVATTN_API int kvattn_scatter_pages(void* host_pool, int64_t host_stride, int64_t n_host_pages, const void* dev_pool,
+                                    int64_t dev_stride, int64_t n_slots, int64_t page_bytes, const int32_t* host_ids,
+                                    const int32_t* dev_slots, int n, int n_ctas, kvattn_stream_t stream) {
+  return page_copy_common(host_pool, host_stride, n_host_pages, const_cast<void*>(dev_pool), dev_stride, n_slots,
+                          page_bytes, host_ids, dev_slots, n, n_ctas, 0, stream);
 }
 
 KVATTN_API int kvattn_stream_wait(kvattn_event_t event, int timeout_ms) {

@@ -5,5 +5,6 @@
 #include "merge.cu"
 #include "select.cu"
 #include "prefill.cu"
+#include "stream.cu"
 #include "api.cu"
 #include "noalloc.cu"

@@ -71,6 +71,10 @@ _SIGS = {
                                      c_int, c_int, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "kvattn_stream_pages": (c_int, [c_void_p, c_int64, c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_int,
                                     c_void_p, c_void_p, POINTER(c_int)]),
+    "kvattn_gather_pages": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_int64, c_int64, c_int64, c_void_p,
+                                    c_void_p, c_int, c_int, c_void_p]),
+    "kvattn_scatter_pages": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_int64, c_int64, c_int64, c_void_p,
+                                     c_void_p, c_int, c_int, c_void_p]),
     "kvattn_stream_plan": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int]),
     "kvattn_stream_wait": (c_int, [c_void_p, c_int]),
 }
@@ -207,6 +211,22 @@ def kvattn_prefill_chunk(desc, q_bf16, n_q, q_pos, page_list, page_logical, n_pa
                                       _p(ws), ws_bytes, _s(stream)), "kvattn_prefill_chunk")
 
 
+def kvattn_gather_pages(host_pool, host_stride, n_host_pages, dev_pool, dev_stride, n_slots, page_bytes, host_ids,
+                        dev_slots, n, n_ctas=0, stream=None) -> None:
+    """Host (pinned, mapped) -> device page copy driven by device-side page lists."""
+    _check(lib().kvattn_gather_pages(_p(host_pool), host_stride, n_host_pages, _p(dev_pool), dev_stride, n_slots,
+                                     page_bytes, _p(host_ids), _p(dev_slots), n, n_ctas, _s(stream)),
+           "kvattn_gather_pages")
+
+
+def kvattn_scatter_pages(host_pool, host_stride, n_host_pages, dev_pool, dev_stride, n_slots, page_bytes, host_ids,
+                         dev_slots, n, n_ctas=0, stream=None) -> None:
+    """Device -> host (pinned, mapped) page copy driven by device-side page lists."""
+    _check(lib().kvattn_scatter_pages(_p(host_pool), host_stride, n_host_pages, _p(dev_pool), dev_stride, n_slots,
+                                      page_bytes, _p(host_ids), _p(dev_slots), n, n_ctas, _s(stream)),
+           "kvattn_scatter_pages")
+
+
 def _host_i32(a):
     import numpy as np
 
@@ -229,13 +249,25 @@ def kvattn_stream_plan(host_ids, dev_slots):
     return list(zip(first[:runs].tolist(), length[:runs].tolist()))
 
 
+def _event_handle(event, stream=None):
+    """The cudaEvent_t of a torch.cuda.Event (created on first record, so an unused one is
+    recorded on `stream` once to bring it into existence) or a raw handle passed as int."""
+    if isinstance(event, int):
+        return event
+    if event.cuda_event == 0:
+        import torch
+
+        event.record(stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.current_stream())
+    return event.cuda_event
+
+
 def kvattn_stream_pages(host_pool, host_stride, dev_pool, dev_stride, page_bytes, host_ids, dev_slots,
                         copy_stream=None, done=None) -> int:
     """host_ids / dev_slots are host sequences; returns the number of copies issued."""
     h, hp = _host_i32(host_ids)
     d, dp = _host_i32(dev_slots)
     n_copies = c_int(0)
-    ev = None if done is None else (done if isinstance(done, int) else done.cuda_event)
+    ev = None if done is None else _event_handle(done, copy_stream)
     _check(lib().kvattn_stream_pages(_p(host_pool), host_stride, _p(dev_pool), dev_stride, page_bytes, hp, dp,
                                      int(h.size), _s(copy_stream), ev, ctypes.byref(n_copies)),
            "kvattn_stream_pages")
@@ -244,8 +276,7 @@ def kvattn_stream_pages(host_pool, host_stride, dev_pool, dev_stride, page_bytes
 
 def kvattn_stream_wait(event, timeout_ms: int) -> int:
     """Returns OK or ERR_TIMEOUT; raises on other errors."""
-    ev = event if isinstance(event, int) else event.cuda_event
-    st = lib().kvattn_stream_wait(ev, timeout_ms)
+    st = lib().kvattn_stream_wait(_event_handle(event), timeout_ms)
     if st not in (OK, ERR_TIMEOUT):
         raise KVAttnError(st, "kvattn_stream_wait")
     return st
