@@ -28,7 +28,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from synth import WORKLOADS, derived_seed, np_rng, page_permutation, plant_needles_torch, torch_normal  # noqa: E402
+from synth import WORKLOADS, derived_seed, np_rng, page_permutation, torch_normal, workload_layer_kv  # noqa: E402
 
 METRIC = "quantized paged KV attention: decode HBM GB/s & prefill TFLOP/s vs roofline"
 BYTES_PER_TOKEN_HEAD = {"q4_0": 34816 // 128 + 18432 // 128, "q8_0": 34816 // 128 + 34816 // 128}  # 416 / 544
@@ -168,23 +168,9 @@ class DecodeCache:
         self.desc = kv.make_desc(H, w.q_heads, self.k_pool, self.v_pool, n_phys, v_fmt=w.v_fmt)
         self.needles = {}
         for l in range(L):
-            k = torch_normal(derived_seed(w.seed, 10, l), (tokens, H, 256), device)
-            v = torch_normal(derived_seed(w.seed, 11, l), (tokens, H, 256), device)
-            if w.outlier_frac:
-                n_out = int(round(w.outlier_frac * 256))
-                for h in range(H):
-                    ch = torch.from_numpy(np_rng(w.seed, 12, l, h).choice(256, n_out, replace=False)).to(device)
-                    k[:, h, ch] *= 8.0
-                    v[:, h, ch] *= 8.0
-            if with_needles:
-                n_full = tokens // 128
-                for h in range(H):
-                    blocks = np.sort(np_rng(w.seed, 13, l, h).choice(n_full - w.recent_blocks, w.needles, replace=False))
-                    self.needles[(l, h)] = blocks
-                    direction = q_for_needles[l, -1, h * w.group:(h + 1) * w.group].to(torch.float64).sum(0)
-                    kh = k[:, h].contiguous()
-                    plant_needles_torch(kh, blocks, direction, derived_seed(w.seed, 14, l, h))
-                    k[:, h] = kh
+            k, v, nd = workload_layer_kv(w, l, tokens, device, q_for_needles[l] if with_needles else None)
+            for h, blocks in nd.items():
+                self.needles[(l, h)] = blocks
             kv.kvattn_quantize_append(self.desc, k, v, tokens, 0, self.page_table[l], n_blocks_per_unit)
             del k, v
         torch.cuda.synchronize()
@@ -244,10 +230,14 @@ class VerifyBench:
     page) with the block summaries, append the 4 verify tokens, decode n_q = 4 over the
     selected pages."""
 
-    def __init__(self, kv, device):
+    def __init__(self, kv, device, layers=0):
+        import dataclasses
+
         import torch
 
         w = WORKLOADS["verify262k"]
+        if layers:
+            w = dataclasses.replace(w, layers=layers)
         self.kv, self.w = kv, w
         L, H, Hq, g = w.layers, w.kv_heads, w.q_heads, w.group
         self.n_full = w.context // 128
@@ -383,8 +373,7 @@ class StreamBench:
         tdesc = kv.make_desc(H, Hq, tmp, tmp.data_ptr() + 34816, H * self.nb, k_page_stride=P, v_page_stride=P)
         ttab = torch.arange(H * self.nb, dtype=torch.int32, device=device).view(H, self.nb)
         for l in range(L):
-            k = torch_normal(derived_seed(w.seed, 10, l), (w.context, H, 256), device)
-            v = torch_normal(derived_seed(w.seed, 11, l), (w.context, H, 256), device)
+            k, v, _ = workload_layer_kv(w, l, w.context, device)
             tmp.zero_()
             kv.kvattn_quantize_append(tdesc, k, v, w.context, 0, ttab, self.nb)
             del k, v
@@ -650,9 +639,24 @@ def _oracle_inputs(wname, n_tokens):
     return _ORACLE_INPUTS[key]
 
 
-def oracle_decode_sample(wname, n_tokens, reps_min_s=8.0, max_reps=3):
+def _blas_threads():
+    """Threads the oracle can use: numpy's BLAS pool runs the contractions; the elementwise
+    steps run on one thread."""
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_decode_sample(wname, n_tokens, reps_min_s=10.0, max_reps=200):
     """Times the oracle (dequantise + float64 attention) on one (layer, KV head) unit and
-    the last n_tokens of the workload's context.  Returns (GB/s, seconds, threads, sample)."""
+    the last n_tokens of the workload's context, repeated until reps_min_s seconds of CPU
+    work have been timed.  Returns (GB/s, seconds per repetition, threads, sample)."""
     from oracle import attention as oatt
     from oracle import quant as oq
 
@@ -669,8 +673,9 @@ def oracle_decode_sample(wname, n_tokens, reps_min_s=8.0, max_reps=3):
         reps += 1
     secs = t_total / reps
     gbs = n_tokens * BYTES_PER_TOKEN_HEAD[w.v_fmt] / secs / 1e9
-    threads = len(os.sched_getaffinity(0))
-    sample = f"1 of {w.layers * w.kv_heads} (layer, KV head) units, {n_tokens} of {w.context} tokens, {w.group} query heads"
+    threads = _blas_threads()
+    sample = (f"1 of {w.layers * w.kv_heads} (layer, KV head) units, {n_tokens} of {w.context} tokens, "
+              f"{w.group} query heads, timed {reps} times ({t_total:.1f} s of CPU work)")
     return gbs, secs, threads, sample
 
 
@@ -825,7 +830,7 @@ def main():
     line["extra"] = extra
 
     if rank == 0 and not args.no_cpu_baseline:
-        gbs, secs, threads, sample = oracle_decode_sample("decode131k", 32768)
+        gbs, secs, threads, sample = oracle_decode_sample("decode131k", 131072)
         line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample,
                                 "seconds_per_sample": secs}
     if rank == 0:

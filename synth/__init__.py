@@ -187,3 +187,35 @@ def plant_needles_torch(k, blocks, direction, seed: int, cosine: float = 0.9, pa
     w = w - (w @ u)[:, None] * u[None, :]
     w = w / torch.linalg.norm(w, dim=1, keepdim=True)
     k[rows] = (norms * (cosine * u[None, :] + s * w)).to(torch.float32)
+
+
+def workload_layer_kv(w: Workload, layer: int, tokens: int, device, q=None):
+    """K and V of one layer of a workload, fp32 torch [tokens][kv_heads][D] on `device`.
+
+    Draws come from torch_normal with per-layer seeds; the workload's outlier channels are
+    scaled x8 in K and V; with needles, every KV head gets w.needles seeded older blocks
+    planted towards the summed last-token query of its group (q: [n_q][q_heads][D] of this
+    layer).  Returns (k, v, needles) with needles {kv_head: sorted block indices}."""
+    import torch
+
+    H = w.kv_heads
+    k = torch_normal(derived_seed(w.seed, 10, layer), (tokens, H, HEAD_DIM), device)
+    v = torch_normal(derived_seed(w.seed, 11, layer), (tokens, H, HEAD_DIM), device)
+    if w.outlier_frac:
+        n_out = int(round(w.outlier_frac * HEAD_DIM))
+        for h in range(H):
+            ch = torch.from_numpy(np_rng(w.seed, 12, layer, h).choice(HEAD_DIM, n_out, replace=False)).to(device)
+            k[:, h, ch] *= 8.0
+            v[:, h, ch] *= 8.0
+    needles = {}
+    if w.needles:
+        n_full = tokens // PAGE_TOKENS
+        g = w.group
+        for h in range(H):
+            blocks = np.sort(np_rng(w.seed, 13, layer, h).choice(n_full - w.recent_blocks, w.needles, replace=False))
+            needles[h] = blocks
+            direction = q[-1, h * g:(h + 1) * g].to(torch.float64).sum(0)
+            kh = k[:, h].contiguous()
+            plant_needles_torch(kh, blocks, direction, derived_seed(w.seed, 14, layer, h))
+            k[:, h] = kh
+    return k, v, needles

@@ -1,0 +1,144 @@
+"""GPU parity at the benchmark's full sizes, in the launch configuration the benchmark times.
+
+Each test builds one layer of a benchmark workload through the benchmark's own classes (same
+context length, head counts, page table, split plan and launch sequence as every timed
+layer), runs that layer once, and checks outputs against the oracle:
+
+* decode, 131,072 tokens (Q8_0 K with Q4_0 or Q8_0 V): every output row of the layer, plus
+  page bytes of sampled blocks bit-exact;
+* MTP verify, 262,144 tokens + 4: the selection bit-exact (needles included) and the 4 x 24
+  rows over the selected blocks, for two sampled KV heads;
+* chunked prefill, 524,288 prior tokens + the 2,048-token chunk: 64 seeded (token, query head)
+  rows over the full context;
+* the streamed 524,288-token working set: selection and decode rows of two KV heads.
+
+The oracle's inputs are the same seeded draws (made on the device by torch's generator and
+copied to the host) with the oracle's own quantisation; nothing the CUDA library computes
+reaches the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import bench
+from helpers_kv import OracleCache, compare
+from oracle import attention as oatt
+from oracle import select as osel
+from synth import np_rng, workload_layer_kv
+
+pytestmark = [pytest.mark.gpu]
+
+DEV = "cuda"
+
+
+def _head(x, h):
+    return x[:, h].contiguous().cpu().numpy()
+
+
+def _oracle_unit(k, v, h, v_fmt, k_tail=None, v_tail=None):
+    """OracleCache of KV head h: the workload's draws, then the appended tokens."""
+    kh, vh = _head(k, h), _head(v, h)
+    if k_tail is not None:
+        kh = np.concatenate([kh, k_tail[:, h].cpu().numpy()], 0)
+        vh = np.concatenate([vh, v_tail[:, h].cpu().numpy()], 0)
+    return OracleCache(kh[:, None], vh[:, None], v_fmt)
+
+
+@pytest.mark.parametrize("wname", ["decode131k", "decode131k_q8q8"])
+def test_decode_full_context(kv_gpu, wname):
+    b = bench.DecodeBench(kv_gpu, wname, torch.device(DEV), layers=1)
+    b.layer(0)
+    torch.cuda.synchronize()
+    assert kv_gpu.kvattn_device_error() == 0
+    w, ctx, g = b.w, b.ctx, b.w.group
+    out, lse = b.out[0].cpu().numpy(), b.lse[0].cpu().numpy()
+    k, v, _ = workload_layer_kv(w, 0, ctx, DEV)
+    # the step's new token overwrites the last position
+    k[ctx - 1] = b.k_new[0, 0]
+    v[ctx - 1] = b.v_new[0, 0]
+    q = b.q[0].cpu().numpy()
+    pt = b.cache.page_table[0].cpu().numpy()
+    rng = np_rng(7100)
+    for h in range(w.kv_heads):
+        oc = _oracle_unit(k, v, h, w.v_fmt)
+        for blk in [0, b.nb - 1] + rng.choice(b.nb, 4, replace=False).tolist():
+            phys = int(pt[h, blk])
+            assert np.array_equal(b.cache.k_pool[phys].cpu().numpy(), oc.page_bytes(0, blk, "k"))
+            assert np.array_equal(b.cache.v_pool[phys].cpu().numpy(), oc.page_bytes(0, blk, "v"))
+        o_ref, l_ref = oc.attend(q[:, h * g:(h + 1) * g], [ctx - 1], 0, g)
+        compare(out[:, h * g:(h + 1) * g], lse[:, h * g:(h + 1) * g], o_ref, l_ref)
+
+
+def _selected_keys(sel, T):
+    keys = (np.asarray(sel)[:, None] * 128 + np.arange(128)[None, :]).ravel()
+    return keys[keys < T]
+
+
+def test_verify_full_context(kv_gpu):
+    b = bench.VerifyBench(kv_gpu, torch.device(DEV), layers=1)
+    b.layer(0)
+    torch.cuda.synchronize()
+    assert kv_gpu.kvattn_device_error() == 0
+    w, g = b.w, b.w.group
+    ctx = w.context
+    k, v, needles = workload_layer_kv(w, 0, ctx, DEV, b.q[0])
+    q = b.q[0].cpu().numpy()
+    out, lse = b.out[0].cpu().numpy(), b.lse[0].cpu().numpy()
+    sel_l, n_sel = b.sel_l[0].cpu().numpy(), b.n_sel[0].cpu().numpy()
+    for h in (0, w.kv_heads - 1):
+        oc = _oracle_unit(k, v, h, w.v_fmt, b.k_new[0], b.v_new[0])
+        T = ctx + w.n_q
+        kc = oc.kc[: b.n_full * 128, 0].reshape(b.n_full, 128, 8, 32)
+        kd = oc.kd[: b.n_full * 128, 0].reshape(b.n_full, 128, 8)
+        sc = osel.block_scores(osel.block_summaries(kc, kd), q[-1, h * g:(h + 1) * g])
+        ref_sel, gap = osel.select_blocks(sc, b.n_full, b.nb, w.budget_blocks, w.recent_blocks)
+        assert gap > 1e-9 * np.abs(sc).max()
+        assert sel_l[h, : n_sel[h]].tolist() == ref_sel.tolist()
+        assert set(needles[h].tolist()) <= set(ref_sel.tolist())
+        o_ref, l_ref = oc.attend(q[:, h * g:(h + 1) * g], list(range(ctx, T)), 0, g,
+                                 key_idx=_selected_keys(ref_sel, T))
+        compare(out[:, h * g:(h + 1) * g], lse[:, h * g:(h + 1) * g], o_ref, l_ref)
+
+
+def test_prefill_full_context_sampled_rows(kv_gpu):
+    b = bench.PrefillBench(kv_gpu, torch.device(DEV), layers=1)
+    b.layer(0)
+    torch.cuda.synchronize()
+    assert kv_gpu.kvattn_device_error() == 0
+    w, g = b.w, b.w.group
+    ctx, T = w.context, b.total
+    rng = np_rng(7200)
+    heads = np.sort(rng.choice(w.kv_heads, 2, replace=False))
+    k, v, _ = workload_layer_kv(w, 0, ctx, DEV)
+    q = b.q[0].float().cpu().numpy()                   # bf16 values, exact in fp32
+    out, lse = b.out[0].cpu().numpy(), b.lse[0].cpu().numpy()
+    for h in heads:
+        oc = _oracle_unit(k, v, int(h), w.v_fmt, b.k_new[0], b.v_new[0])
+        t = np.sort(rng.choice(w.n_q, 32, replace=False))
+        j = h * g + rng.integers(0, g, 32)
+        rows = q[t, j]
+        o_ref, l_ref = oatt.attend(rows, oc.khat(0), oc.vhat(0), np.arange(T), ctx + t, 1.0 / 16.0)
+        compare(out[t, j], lse[t, j], o_ref, l_ref)
+
+
+def test_stream_full_context(kv_gpu):
+    b = bench.StreamBench(kv_gpu, torch.device(DEV), layers=1)
+    b.step(True)
+    torch.cuda.synchronize()
+    assert kv_gpu.kvattn_device_error() == 0
+    w, g = b.w, b.w.group
+    ctx = w.context
+    T = ctx + 1
+    k, v, _ = workload_layer_kv(w, 0, ctx, DEV)
+    q = b.q[0].cpu().numpy()
+    out, lse = b.out[0].cpu().numpy(), b.lse[0].cpu().numpy()
+    sel_l, n_sel = b.sel_l[0].cpu().numpy(), b.n_sel[0].cpu().numpy()
+    for h in (1, 2):
+        oc = _oracle_unit(k, v, h, w.v_fmt, b.k_new[0], b.v_new[0])
+        kc = oc.kc[: b.n_full * 128, 0].reshape(b.n_full, 128, 8, 32)
+        kd = oc.kd[: b.n_full * 128, 0].reshape(b.n_full, 128, 8)
+        sc = osel.block_scores(osel.block_summaries(kc, kd), q[0, h * g:(h + 1) * g])
+        ref_sel, gap = osel.select_blocks(sc, b.n_full, b.nb, w.budget_blocks, 0)
+        assert gap > 1e-9 * np.abs(sc).max()
+        assert sel_l[h, : n_sel[h]].tolist() == ref_sel.tolist()
+        o_ref, l_ref = oc.attend(q[:, h * g:(h + 1) * g], [ctx], 0, g, key_idx=_selected_keys(ref_sel, T))
+        compare(out[:, h * g:(h + 1) * g], lse[:, h * g:(h + 1) * g], o_ref, l_ref)
