@@ -213,10 +213,12 @@ KVATTN_API int kvattn_select_blocks(const float* summaries, const float* q_group
 
 /* ---- chunked prefill on tcgen05 ([STREAM] method list) -----------------------------
  * Attention of n_q bf16 query tokens (positions q_pos[i], device int32 [n_q]) over the
- * listed pages, causal.  K/V pages are dequantized to bf16 in shared memory; QK^T and PV
- * run on tcgen05 tensor cores with fp32 accumulation in tensor memory.  The keys are taken
- * in splits of kv_split_tokens (a multiple of 128); partial results are merged by
- * log-sum-exp.
+ * listed pages, causal.  K/V tiles are dequantized to f16 (block scales folded in) in
+ * shared memory and Q is rounded to f16 after scaling by log2(e)/16; QK^T and PV run on
+ * tcgen05 tensor cores with fp32 accumulation in tensor memory.  The keys are taken in
+ * splits of kv_split_tokens (a multiple of 128, at most 65,536; a CTA may walk several
+ * consecutive splits); partial results are merged by log-sum-exp.  A page id outside
+ * [0, n_pages) skips its page and records KVATTN_ERR_BAD_PAGE.
  *   q      device bf16 bits [n_q][H_q][256];  out device fp32 [n_q][H_q][256];
  *   lse    device fp32 [n_q][H_q];  page arguments as for kvattn_decode.
  *   ws     device workspace of kvattn_prefill_workspace_size() bytes. */

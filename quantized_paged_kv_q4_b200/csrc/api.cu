@@ -412,7 +412,7 @@ extern "C" {
 KVATTN_API size_t kvattn_prefill_workspace_size(const kvattn_kv_desc* desc, int n_q, int max_pages,
                                                 int kv_split_tokens) {
   if (validate_desc(desc) || n_q < 1 || max_pages < 0 || kv_split_tokens < kPageTokens ||
-      kv_split_tokens % kPageTokens)
+      kv_split_tokens % kPageTokens || kv_split_tokens > 65536)
     return 0;
   return plan_prefill(desc->n_kv_heads, desc->n_q_heads / desc->n_kv_heads, n_q, max_pages, kv_split_tokens,
                       sm_count_for_planning())

@@ -55,12 +55,17 @@ constexpr int kDq0 = (kSoftmaxWarps + 2) * 32;  // first dequant thread
 // raw bytes of one 64-key tile, as copied from the page
 constexpr int kRawKc = 16384, kRawKs = 1024, kRawVc = 8192, kRawVs = 1024;
 constexpr int kRawBytes = kRawKc + kRawKs + kRawVc + kRawVs;  // 26,624
+constexpr int kRawStages = 3;
+// a CTA walks at most this many 64-key tiles (the host plan keeps pages per CTA <= 512)
+constexpr int kMaxTiles = 1024;
 // shared memory map (bytes)
-constexpr int kKOff = 0;                     // 2 buffers x 4 atoms x [64 keys][128 B]
-constexpr int kVOff = kKOff + 2 * 32768;     // 2 buffers x [256 dims][128 B]
-constexpr int kRawOff = kVOff + 2 * 32768;   // 2 stages of raw tile bytes
-constexpr int kMiscOff = kRawOff + 2 * kRawBytes;
+constexpr int kKOff = 0;                                  // 2 buffers x 4 atoms x [64 keys][128 B]
+constexpr int kVOff = kKOff + 2 * 32768;                  // 2 buffers x [256 dims][128 B]
+constexpr int kRawOff = kVOff + 2 * 32768;                // kRawStages stages of raw tile bytes
+constexpr int kTileOff = kRawOff + kRawStages * kRawBytes;  // int2 [kMaxTiles]: page, 2*logical+half
+constexpr int kMiscOff = kTileOff + 8 * kMaxTiles;
 constexpr int kSmemBytes = kMiscOff + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol0 = 0;    // S buffers [0,64), [64,128); P (f16 pairs) over their first 32
@@ -70,27 +75,22 @@ constexpr uint32_t kIdescQK = tc::idesc_f16(128, kKeys, 0, 0);
 constexpr uint32_t kIdescPV = tc::idesc_f16(128, 256, 0, 0);
 }  // namespace pf
 
-struct PfTile {
-  int page, logical, half;
-};
-
-// The CTA's i-th candidate tile (2 per listed page); false if the tile holds no key that
-// any row of the M-tile may see, or its page id is invalid.  Every role evaluates the same
-// predicate, so all agree on the tile sequence.
-__device__ __forceinline__ bool pf_tile(const PrefillParams& p, int h, int ks, int i, int np, int max_qpos,
-                                        PfTile* tile) {
+// The CTA's i-th candidate tile (2 per listed page): 1 if it holds a key that some row of
+// the M-tile may see (*page, *lh = 2 * logical block + half), 0 if not, -1 if its page id is
+// out of range.
+__device__ __forceinline__ int pf_candidate(const PrefillParams& p, int h, int ks, int i, int np, int max_qpos,
+                                            int* page_out, int* lh_out) {
   const int idx = ks * p.pages_per_split + (i >> 1);
-  if (idx >= np) return false;
+  if (idx >= np) return 0;
   const long long li = static_cast<long long>(h) * p.max_pages + idx;
   const int page = p.page_list[li];
   const int logical = p.page_logical ? p.page_logical[li] : idx;
   const int half = i & 1;
-  if (static_cast<long long>(logical) * kPageTokens + half * pf::kKeys > max_qpos) return false;
-  if (page < 0 || page >= p.n_pages) return false;
-  tile->page = page;
-  tile->logical = logical;
-  tile->half = half;
-  return true;
+  if (static_cast<long long>(logical) * kPageTokens + half * pf::kKeys > max_qpos) return 0;
+  if (page < 0 || page >= p.n_pages) return -1;
+  *page_out = page;
+  *lh_out = 2 * logical + half;
+  return 1;
 }
 
 __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t chunk) {
@@ -116,18 +116,20 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pf::kMiscOff);
-  uint64_t* rawfull = bars + 0;   // [2] producer (tx bytes) -> dequant
-  uint64_t* rawempty = bars + 2;  // [2] dequant -> producer
-  uint64_t* kready = bars + 4;    // [2] dequant -> MMA
-  uint64_t* vready = bars + 6;    // [2]
-  uint64_t* kfree = bars + 8;     // [2] MMA (QK done) -> dequant
-  uint64_t* vfree = bars + 10;    // [2] MMA (PV done) -> dequant, softmax
-  uint64_t* sready = bars + 12;   // [2] MMA -> softmax
-  uint64_t* pready = bars + 14;   // [2] softmax -> MMA
-  uint64_t* ofinal = bars + 16;   // MMA -> softmax (epilogue)
-  uint64_t* qready = bars + 17;   // softmax (Q in TMEM) -> MMA
-  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* rawfull = bars + 0;   // [3] producer (tx bytes) -> dequant
+  uint64_t* rawempty = bars + 3;  // [3] dequant -> producer
+  uint64_t* kready = bars + 6;    // [2] dequant -> MMA
+  uint64_t* vready = bars + 8;    // [2]
+  uint64_t* kfree = bars + 10;    // [2] MMA (QK done) -> dequant
+  uint64_t* vfree = bars + 12;    // [2] MMA (PV done) -> dequant, softmax
+  uint64_t* sready = bars + 14;   // [2] MMA -> softmax
+  uint64_t* pready = bars + 16;   // [2] softmax -> MMA
+  uint64_t* ofinal = bars + 18;   // MMA -> softmax (epilogue)
+  uint64_t* qready = bars + 19;   // softmax (Q in TMEM) -> MMA
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bars + 20);
   int* s_abort = reinterpret_cast<int*>(tmem_base_s + 1);
+  int* s_ntiles = s_abort + 1;
+  const int2* tiles = reinterpret_cast<const int2*>(smem + pf::kTileOff);
 
   const int mt = blockIdx.x, ks = blockIdx.y, h = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -141,12 +143,13 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     const int t0 = row0 / p.group, t1 = min(n_rows - 1, row0 + pf::kRows - 1) / p.group;
     for (int t = t0; t <= t1; ++t) max_qpos = max(max_qpos, p.q_pos[t]);
   }
-  const int n_cand = 2 * p.pages_per_split;
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < pf::kRawStages; ++b) {
       mbar_init(&rawfull[b], 1);
       mbar_init(&rawempty[b], pf::kDequantWarps);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&kready[b], pf::kDequantWarps);
       mbar_init(&vready[b], pf::kDequantWarps);
       mbar_init(&kfree[b], 1);
@@ -160,6 +163,25 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     if (smem_u32(smem) & 1023) record_error(KVATTN_ERR_INVALID_ARG);
     fence_barrier_init();
   }
+  if (warp == 0) {
+    // the CTA's tiles in key order, compacted once: (page, 2 * logical block + half)
+    int2* list = reinterpret_cast<int2*>(smem + pf::kTileOff);
+    int n_cand = 2 * p.pages_per_split;
+    if (n_cand > pf::kMaxTiles) {
+      if (lane == 0) record_error(KVATTN_ERR_INVALID_ARG);
+      n_cand = 0;
+    }
+    int cnt = 0;
+    for (int i0 = 0; i0 < n_cand; i0 += 32) {
+      int page = 0, lh = 0;
+      const int c = i0 + lane < n_cand ? pf_candidate(p, h, ks, i0 + lane, np, max_qpos, &page, &lh) : 0;
+      if (c < 0) record_error(KVATTN_ERR_BAD_PAGE);
+      const unsigned m = __ballot_sync(0xffffffffu, c > 0);
+      if (c > 0) list[cnt + __popc(m & ((1u << lane) - 1u))] = make_int2(page, lh);
+      cnt += __popc(m);
+    }
+    if (lane == 0) *s_ntiles = cnt;
+  }
   if (warp == pf::kMmaWarp) {
     tc::tmem_alloc(tmem_base_s, pf::kTmemCols);
     tc::tmem_relinquish();
@@ -168,32 +190,33 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_base_s;
+  const int n_tiles = *s_ntiles;
 
   if (warp == pf::kLoadWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int j = 0;
-      for (int i = 0; i < n_cand; ++i) {
-        PfTile tl;
-        if (!pf_tile(p, h, ks, i, np, max_qpos, &tl)) continue;
-        const int r = j & 1;
-        if (j >= 2 && !mbar_wait(&rawempty[r], ((j - 2) >> 1) & 1)) {
+      for (; j < n_tiles; ++j) {
+        const int2 tl = tiles[j];
+        const int r = j % pf::kRawStages;
+        if (j >= pf::kRawStages && !mbar_wait(&rawempty[r], ((j / pf::kRawStages) - 1) & 1)) {
           *s_abort = 1;
           break;
         }
+        const int half = tl.y & 1;
         uint8_t* st = smem + pf::kRawOff + r * pf::kRawBytes;
-        const uint8_t* kp = p.k_pool + static_cast<int64_t>(tl.page) * p.k_stride;
-        const uint8_t* vp = p.v_pool + static_cast<int64_t>(tl.page) * p.v_stride;
+        const uint8_t* kp = p.k_pool + static_cast<int64_t>(tl.x) * p.k_stride;
+        const uint8_t* vp = p.v_pool + static_cast<int64_t>(tl.x) * p.v_stride;
         mbar_arrive_expect_tx(&rawfull[r], pf::kRawBytes);
-        bulk_g2s(st, kp + tl.half * pf::kRawKc, pf::kRawKc, &rawfull[r]);
-        bulk_g2s(st + pf::kRawKc, kp + kKScaleOffset + tl.half * pf::kRawKs, pf::kRawKs, &rawfull[r]);
-        bulk_g2s(st + pf::kRawKc + pf::kRawKs, vp + tl.half * pf::kRawVc, pf::kRawVc, &rawfull[r]);
-        bulk_g2s(st + pf::kRawKc + pf::kRawKs + pf::kRawVc, vp + kV4ScaleOffset + tl.half * pf::kRawVs, pf::kRawVs,
+        bulk_g2s(st, kp + half * pf::kRawKc, pf::kRawKc, &rawfull[r]);
+        bulk_g2s(st + pf::kRawKc, kp + kKScaleOffset + half * pf::kRawKs, pf::kRawKs, &rawfull[r]);
+        bulk_g2s(st + pf::kRawKc + pf::kRawKs, vp + half * pf::kRawVc, pf::kRawVc, &rawfull[r]);
+        bulk_g2s(st + pf::kRawKc + pf::kRawKs + pf::kRawVc, vp + kV4ScaleOffset + half * pf::kRawVs, pf::kRawVs,
                  &rawfull[r]);
-        ++j;
       }
       // every copy issued must land before the CTA may exit
-      for (int jj = j - 2 < 0 ? 0 : j - 2; jj < j; ++jj) mbar_wait(&rawfull[jj & 1], (jj >> 1) & 1);
+      for (int jj = j - pf::kRawStages < 0 ? 0 : j - pf::kRawStages; jj < j; ++jj)
+        mbar_wait(&rawfull[jj % pf::kRawStages], (jj / pf::kRawStages) & 1);
     }
   } else if (warp == pf::kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -216,9 +239,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         tc::commit(&vfree[b]);
         return true;
       };
-      for (int i = 0; i < n_cand && ok; ++i) {
-        PfTile tl;
-        if (!pf_tile(p, h, ks, i, np, max_qpos, &tl)) continue;
+      for (; j < n_tiles && ok; ++j) {
         const int b = j & 1;
         if (!mbar_wait(&kready[b], (j >> 1) & 1)) {
           ok = false;
@@ -234,7 +255,6 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         tc::commit(&sready[b]);
         tc::commit(&kfree[b]);
         if (j >= 1) ok = issue_pv(j - 1);
-        ++j;
       }
       if (ok && j >= 1) ok = issue_pv(j - 1);
       if (!ok) *s_abort = 1;
@@ -276,9 +296,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     float m_ref = -INFINITY, l_sum = 0.f;
     int j = 0;
     bool ok = true;
-    for (int i = 0; i < n_cand && ok; ++i) {
-      PfTile tl;
-      if (!pf_tile(p, h, ks, i, np, max_qpos, &tl)) continue;
+    for (; j < n_tiles && ok; ++j) {
+      const int2 tl = tiles[j];
       const int b = j & 1;
       if (!mbar_wait(&sready[b], (j >> 1) & 1)) {
         ok = false;
@@ -287,7 +306,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       tc::fence_after_sync();
       // two passes over the 64 scores (32 columns at a time) keep register pressure low:
       // the maximum first, then P; the second pass reads S from tensor memory again
-      const int key0 = tl.logical * kPageTokens + tl.half * pf::kKeys;
+      const int key0 = tl.y * pf::kKeys;
       const bool masked = key0 + pf::kKeys - 1 > qpos;
       const uint32_t scol = lane_base + pf::kSCol0 + b * pf::kKeys;
       float mx = -INFINITY;
@@ -350,7 +369,6 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&pready[b]);
-      ++j;
     }
     // ---- epilogue: normalised partial (o, lse) of this row ----
     bool have = false;
@@ -414,11 +432,9 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     const int rotK = kR >> 1, rotV = vR >> 1;
     int j = 0;
     bool ok = true;
-    for (int i = 0; i < n_cand && ok; ++i) {
-      PfTile tl;
-      if (!pf_tile(p, h, ks, i, np, max_qpos, &tl)) continue;
-      const int b = j & 1, r = j & 1;
-      if (!mbar_wait(&rawfull[r], (j >> 1) & 1)) {
+    for (; j < n_tiles && ok; ++j) {
+      const int b = j & 1, r = j % pf::kRawStages;
+      if (!mbar_wait(&rawfull[r], (j / pf::kRawStages) & 1)) {
         ok = false;
         break;
       }
@@ -474,30 +490,46 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         break;
       }
       {
+        // This thread's words (key half vh, blocks 2C and 2C+1) of each raw chunk; chunk ii
+        // holds token pair (ii + rotV) & 3.  Two select stages undo the rotation so that
+        // wv[T] is token pair T: an array indexed by the runtime rotation would be placed in
+        // local memory.
+        uint32_t wv[4][2];
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) {
+          wv[ii][0] = vh ? vraw[ii].y : vraw[ii].x;
+          wv[ii][1] = vh ? vraw[ii].w : vraw[ii].z;
+        }
+        {
+          const bool r1 = rotV & 1;
+          uint32_t t[4][2];
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) t[x][e] = r1 ? wv[(x + 3) & 3][e] : wv[x][e];
+          const bool r2 = rotV & 2;
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) wv[x][e] = r2 ? t[(x + 2) & 3][e] : t[x][e];
+        }
         uint8_t* vt = smem + pf::kVOff + b * 32768;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {  // block 2C + e
           uint32_t o[4][4];            // [k][T]
 #pragma unroll
-          for (int ii = 0; ii < 4; ++ii) {
-            const uint32_t W = e ? (vh ? vraw[ii].w : vraw[ii].z) : (vh ? vraw[ii].y : vraw[ii].x);
+          for (int T = 0; T < 4; ++T) {
+            const uint32_t W = wv[T][e];
             const uint32_t Ws = W >> 8;
+            const uint32_t dv = e ? (vh ? dvr[T].w : dvr[T].z) : (vh ? dvr[T].y : dvr[T].x);
             const uint32_t v0 = hsub2(and_or(W, 0x000F000Fu, 0x64006400u), 0x64086408u);
             const uint32_t v1 = hfma2(and_or(W, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
             const uint32_t v2 = hsub2(and_or(Ws, 0x000F000Fu, 0x64006400u), 0x64086408u);
             const uint32_t v3 = hfma2(and_or(Ws, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
-            // chunk ii holds token pair T = (ii + rotV) & 3; scale by that pair's fp16 scales
-            // (select with constant register indices)
-#pragma unroll
-            for (int T = 0; T < 4; ++T) {
-              if (T == ((ii + rotV) & 3)) {
-                const uint32_t dv = e ? (vh ? dvr[T].w : dvr[T].z) : (vh ? dvr[T].y : dvr[T].x);
-                o[0][T] = hmul2(v0, dv);
-                o[1][T] = hmul2(v1, dv);
-                o[2][T] = hmul2(v2, dv);
-                o[3][T] = hmul2(v3, dv);
-              }
-            }
+            o[0][T] = hmul2(v0, dv);
+            o[1][T] = hmul2(v1, dv);
+            o[2][T] = hmul2(v2, dv);
+            o[3][T] = hmul2(v3, dv);
           }
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -509,7 +541,6 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&vready[b]);
-      ++j;
     }
     if (!ok) *s_abort = 1;
   }
@@ -533,7 +564,8 @@ struct PrefillPlan {
 };
 
 // A CTA walks `spc` consecutive KV splits, merging them online in tensor memory, as long as
-// the grid keeps at least ~16 waves of CTAs: fewer partials to write and merge.
+// the grid keeps at least ~16 waves of CTAs and the CTA's tile list fits in shared memory:
+// fewer partials to write and merge.
 PrefillPlan plan_prefill(int n_kv, int group, int n_q, int max_pages, int kv_split_tokens, int sm_count) {
   PrefillPlan pl{};
   const int rows = n_q * group;
@@ -542,7 +574,10 @@ PrefillPlan plan_prefill(int n_kv, int group, int n_q, int max_pages, int kv_spl
   const int base = kv_split_tokens / kPageTokens;
   const long long splits0 = max_pages > 0 ? (max_pages + base - 1) / base : 1;
   long long spc = static_cast<long long>(n_kv) * pl.n_mt * splits0 / (static_cast<long long>(sm_count) * 16);
+  long long spc_max = (pf::kMaxTiles / 2) / base;  // the API keeps kv_split_tokens <= 65,536
+  spc_max = spc_max < 1 ? 1 : spc_max;
   spc = spc < 1 ? 1 : (spc > splits0 ? splits0 : spc);
+  spc = spc > spc_max ? spc_max : spc;
   pl.pps = static_cast<int>(base * spc);
   pl.n_ks = max_pages > 0 ? (max_pages + pl.pps - 1) / pl.pps : 1;
   pl.lse_off = 0;

@@ -96,3 +96,33 @@ def test_prefill_subset_of_the_524k_workload(kv_gpu):
         out, lse = _prefill(kv_gpu, cache, 6, q[rows], q_pos, cache.page_table_np, 4096)
         o_ref, l_ref = oc.attend(q[rows], q_pos, 0, 6)
         compare(out, lse, o_ref, l_ref)
+
+
+def test_prefill_largest_split(kv_gpu):
+    """kv_split_tokens = 65,536 (the largest accepted): 1,024 tiles per CTA, two splits."""
+    H, n_prior, n_q = 1, 70000, 16
+    rng, k, v, q, cache, T = _case(1400, H, n_prior, n_q, outliers=False)
+    q_pos = np.arange(n_prior, T)
+    out, lse = _prefill(kv_gpu, cache, 6, q, q_pos, cache.page_table_np, 65536)
+    o_ref, l_ref = OracleCache(k, v, "q4_0").attend(q, q_pos, 0, 6)
+    compare(out, lse, o_ref, l_ref)
+
+
+def test_prefill_bad_page_id_is_skipped_and_reported(kv_gpu):
+    H, n_prior, n_q = 1, 1000, 24
+    rng, k, v, q, cache, T = _case(1500, H, n_prior, n_q, outliers=False)
+    plist = cache.page_table_np.copy()
+    plist[0, 3] = cache.n_phys + 5
+    q_pos = np.arange(n_prior, T)
+    qb = torch.from_numpy(bf16_bits(q).view(np.int16)).cuda()
+    out = torch.empty((n_q, 6, 256), device="cuda")
+    lse = torch.empty((n_q, 6), device="cuda")
+    wsb = kv_gpu.kvattn_prefill_workspace_size(cache.desc, n_q, plist.shape[1], 256)
+    ws = torch.zeros(max(wsb, 256), dtype=torch.uint8, device="cuda")
+    kv_gpu.kvattn_prefill_chunk(cache.desc, qb, n_q, torch.from_numpy(q_pos.astype(np.int32)).cuda(),
+                                torch.from_numpy(plist).cuda(), None, None, plist.shape[1], 256, out, lse, ws, wsb)
+    assert kv_gpu.kvattn_device_error() == kv_gpu.ERR_BAD_PAGE
+    keys = np.arange(T)
+    keys = keys[(keys < 3 * 128) | (keys >= 4 * 128)]
+    o_ref, l_ref = OracleCache(k, v, "q4_0").attend(q, q_pos, 0, 6, key_idx=keys)
+    compare(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref)
