@@ -113,6 +113,54 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
       : "memory");
 }
 
+// Softmax pieces for one 64-key tile of S (this thread's row, 32 columns per tensor-memory
+// load).  Column c is visible iff c <= lim; kMask = false when every row of the warp sees
+// the whole tile, so the common case carries no per-element test.  Independent partial
+// maxima and sums keep the dependency chains short.
+template <bool kMask>
+__device__ __forceinline__ float pf_row_max(uint32_t scol, int lim) {
+  float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    uint32_t v[32];
+    tc::ld32(scol + 32 * hh, v);
+    tc::wait_ld();
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      float x = __uint_as_float(v[c]);
+      if (kMask && 32 * hh + c > lim) x = -INFINITY;
+      m[c & 3] = fmaxf(m[c & 3], x);
+    }
+  }
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// P = exp2(S - mu) as f16 pairs over the first 32 columns of S; returns the row sum of P.
+template <bool kMask>
+__device__ __forceinline__ float pf_row_p(uint32_t scol, int lim, float mu) {
+  float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    uint32_t v[32];
+    tc::ld32(scol + 32 * hh, v);
+    tc::wait_ld();
+    uint32_t w[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      float s0 = __uint_as_float(v[2 * c]), s1 = __uint_as_float(v[2 * c + 1]);
+      if (kMask && 32 * hh + 2 * c > lim) s0 = -INFINITY;
+      if (kMask && 32 * hh + 2 * c + 1 > lim) s1 = -INFINITY;
+      const float p0 = fast_exp2(s0 - mu), p1 = fast_exp2(s1 - mu);
+      ls[(2 * c) & 3] += p0;
+      ls[(2 * c + 1) & 3] += p1;
+      w[c] = pack_half2(p0, p1);
+    }
+    // the first half's P lands in columns 0-15, which the second half no longer reads
+    tc::st16(scol + 16 * hh, w);
+  }
+  return (ls[0] + ls[1]) + (ls[2] + ls[3]);
+}
+
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pf::kMiscOff);
@@ -306,21 +354,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       tc::fence_after_sync();
       // two passes over the 64 scores (32 columns at a time) keep register pressure low:
       // the maximum first, then P; the second pass reads S from tensor memory again
-      const int key0 = tl.y * pf::kKeys;
-      const bool masked = key0 + pf::kKeys - 1 > qpos;
+      const int lim = qpos - tl.y * pf::kKeys;  // columns beyond lim are in this row's future
+      const bool need_mask = __any_sync(0xffffffffu, lim < pf::kKeys - 1);
       const uint32_t scol = lane_base + pf::kSCol0 + b * pf::kKeys;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t v[32];
-        tc::ld32(scol + 32 * hh, v);
-        tc::wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float x = (masked && key0 + 32 * hh + c > qpos) ? -INFINITY : __uint_as_float(v[c]);
-          mx = fmaxf(mx, x);
-        }
-      }
+      const float mx = need_mask ? pf_row_max<true>(scol, lim) : pf_row_max<false>(scol, lim);
       float alpha = 1.f;
       bool resc = false;
       if (mx > m_ref + 8.f) {
@@ -348,23 +385,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         tc::wait_st();
       }
       const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {  // P as f16 pairs over the first 32 columns of S
-        uint32_t v[32];
-        tc::ld32(scol + 32 * hh, v);
-        tc::wait_ld();
-        uint32_t w[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float s0 = (masked && key0 + 32 * hh + 2 * c > qpos) ? -INFINITY : __uint_as_float(v[2 * c]);
-          const float s1 = (masked && key0 + 32 * hh + 2 * c + 1 > qpos) ? -INFINITY : __uint_as_float(v[2 * c + 1]);
-          const float p0 = fast_exp2(s0 - mu), p1 = fast_exp2(s1 - mu);
-          l_sum += p0 + p1;
-          w[c] = pack_half2(p0, p1);
-        }
-        // the first half's P lands in columns 0-15, which the second half no longer reads
-        tc::st16(scol + 16 * hh, w);
-      }
+      l_sum += need_mask ? pf_row_p<true>(scol, lim, mu) : pf_row_p<false>(scol, lim, mu);
       tc::wait_st();
       tc::fence_before_sync();
       __syncwarp();
