@@ -113,52 +113,48 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
       : "memory");
 }
 
-// Softmax pieces for one 64-key tile of S (this thread's row, 32 columns per tensor-memory
-// load).  Column c is visible iff c <= lim; kMask = false when every row of the warp sees
-// the whole tile, so the common case carries no per-element test.  Independent partial
-// maxima and sums keep the dependency chains short.
-template <bool kMask>
-__device__ __forceinline__ float pf_row_max(uint32_t scol, int lim) {
+// Softmax pieces for one 64-key tile of S: this thread's row, loaded from tensor memory as
+// two 32-column halves.  Independent partial maxima and sums keep dependency chains short;
+// packed f32x2 arithmetic halves the subtractions and additions.
+__device__ __forceinline__ void pf_mask32(uint32_t (&v)[32], int lim, int c0) {
+#pragma unroll
+  for (int c = 0; c < 32; ++c)
+    if (c0 + c > lim) v[c] = 0xFF800000u;  // -inf: the key is in this row's future
+}
+
+__device__ __forceinline__ float pf_max32(const uint32_t (&v)[32]) {
   float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    uint32_t v[32];
-    tc::ld32(scol + 32 * hh, v);
-    tc::wait_ld();
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      float x = __uint_as_float(v[c]);
-      if (kMask && 32 * hh + c > lim) x = -INFINITY;
-      m[c & 3] = fmaxf(m[c & 3], x);
-    }
-  }
+  for (int c = 0; c < 32; ++c) m[c & 3] = fmaxf(m[c & 3], __uint_as_float(v[c]));
   return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
-// P = exp2(S - mu) as f16 pairs over the first 32 columns of S; returns the row sum of P.
-template <bool kMask>
-__device__ __forceinline__ float pf_row_p(uint32_t scol, int lim, float mu) {
-  float ls[4] = {0.f, 0.f, 0.f, 0.f};
+__device__ __forceinline__ uint64_t f32x2_pack(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+
+// P = exp2(S - mu) for 32 columns as 16 f16 pairs; returns the sum of the 32 values of P.
+__device__ __forceinline__ float pf_p32(const uint32_t (&v)[32], uint32_t mu_bits, uint32_t (&w)[16]) {
+  const uint64_t mm = f32x2_pack(mu_bits, mu_bits);
+  uint64_t acc[2] = {0ull, 0ull};  // two f32x2 partial sums (0.0f bit patterns)
 #pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    uint32_t v[32];
-    tc::ld32(scol + 32 * hh, v);
-    tc::wait_ld();
-    uint32_t w[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      float s0 = __uint_as_float(v[2 * c]), s1 = __uint_as_float(v[2 * c + 1]);
-      if (kMask && 32 * hh + 2 * c > lim) s0 = -INFINITY;
-      if (kMask && 32 * hh + 2 * c + 1 > lim) s1 = -INFINITY;
-      const float p0 = fast_exp2(s0 - mu), p1 = fast_exp2(s1 - mu);
-      ls[(2 * c) & 3] += p0;
-      ls[(2 * c + 1) & 3] += p1;
-      w[c] = pack_half2(p0, p1);
-    }
-    // the first half's P lands in columns 0-15, which the second half no longer reads
-    tc::st16(scol + 16 * hh, w);
+  for (int c = 0; c < 16; ++c) {
+    uint64_t x = f32x2_pack(v[2 * c], v[2 * c + 1]);
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(x) : "l"(x), "l"(mm));
+    uint32_t d0, d1;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(d0), "=r"(d1) : "l"(x));
+    const float p0 = fast_exp2(__uint_as_float(d0)), p1 = fast_exp2(__uint_as_float(d1));
+    const uint64_t pp = f32x2_pack(__float_as_uint(p0), __float_as_uint(p1));
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(acc[c & 1]) : "l"(acc[c & 1]), "l"(pp));
+    w[c] = pack_half2(p0, p1);
   }
-  return (ls[0] + ls[1]) + (ls[2] + ls[3]);
+  uint64_t t;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(acc[0]), "l"(acc[1]));
+  uint32_t a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(t));
+  return __uint_as_float(a) + __uint_as_float(b);
 }
 
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillParams p) {
@@ -352,12 +348,18 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         break;
       }
       tc::fence_after_sync();
-      // two passes over the 64 scores (32 columns at a time) keep register pressure low:
-      // the maximum first, then P; the second pass reads S from tensor memory again
+      // the 64 scores in one tensor-memory round trip; P overwrites their first 32 columns
       const int lim = qpos - tl.y * pf::kKeys;  // columns beyond lim are in this row's future
-      const bool need_mask = __any_sync(0xffffffffu, lim < pf::kKeys - 1);
       const uint32_t scol = lane_base + pf::kSCol0 + b * pf::kKeys;
-      const float mx = need_mask ? pf_row_max<true>(scol, lim) : pf_row_max<false>(scol, lim);
+      uint32_t v0[32], v1[32];
+      tc::ld32(scol, v0);
+      tc::ld32(scol + 32, v1);
+      tc::wait_ld();
+      if (__any_sync(0xffffffffu, lim < pf::kKeys - 1)) {  // warp-uniform: only diagonal tiles
+        pf_mask32(v0, lim, 0);
+        pf_mask32(v1, lim, 32);
+      }
+      const float mx = fmaxf(pf_max32(v0), pf_max32(v1));
       float alpha = 1.f;
       bool resc = false;
       if (mx > m_ref + 8.f) {
@@ -366,8 +368,17 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         l_sum *= alpha;
         m_ref = mx;
       }
+      const float mu = m_ref == -INFINITY ? 0.f : m_ref;
+      {
+        uint32_t w[16];
+        l_sum += pf_p32(v0, __float_as_uint(mu), w);
+        tc::st16(scol, w);
+        l_sum += pf_p32(v1, __float_as_uint(mu), w);
+        tc::st16(scol + 16, w);
+      }
       if (__any_sync(0xffffffffu, resc)) {
-        // this warp's rows of O hold the previous tile's PV only once it completed
+        // O is rescaled to the new maximum before PV of this tile accumulates into it; this
+        // warp's rows of O hold the previous tile's PV only once that completed
         if (!mbar_wait(&vfree[(j - 1) & 1], ((j - 1) >> 1) & 1)) {
           ok = false;
           break;
@@ -382,10 +393,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
           for (int c = 0; c < 32; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) * f);
           tc::st32(lane_base + pf::kOCol0 + c0, v);
         }
-        tc::wait_st();
       }
-      const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-      l_sum += need_mask ? pf_row_p<true>(scol, lim, mu) : pf_row_p<false>(scol, lim, mu);
       tc::wait_st();
       tc::fence_before_sync();
       __syncwarp();
