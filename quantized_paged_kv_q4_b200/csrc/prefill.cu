@@ -102,16 +102,6 @@ __device__ __forceinline__ uint32_t tmem_lane(uint32_t tmem, int warp) {
   return tmem + ((static_cast<uint32_t>(warp & 3) * 32) << 16);
 }
 
-// D[tmem] (+)= A[tmem] * B[smem desc]; issued by one thread.
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                           uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 
 // Softmax pieces for one 64-key tile of S: this thread's row, loaded from tensor memory as
 // two 32-column halves.  Independent partial maxima and sums keep dependency chains short;
@@ -264,28 +254,33 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     }
   } else if (warp == pf::kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop (one elected lane issues each instruction); every wait
+    // result is made warp-uniform so the lanes never diverge around elect.sync.
+    {
       const uint32_t k_base = smem_u32(smem + pf::kKOff);
       const uint32_t v_base = smem_u32(smem + pf::kVOff);
+      auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, par));
+      };
       int j = 0;
-      bool ok = mbar_wait(qready, 0);
+      bool ok = wait_all(qready, 0);
       auto issue_pv = [&](int jj) -> bool {
         const int b = jj & 1;
         const uint32_t par = (jj >> 1) & 1;
-        if (!mbar_wait(&pready[b], par) || !mbar_wait(&vready[b], par)) return false;
+        if (!wait_all(&pready[b], par) || !wait_all(&vready[b], par)) return false;
         tc::fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
           const uint64_t bd = tc::sw128_desc(v_base + b * 32768 + kk * 32, 1024, 16);
-          mma_f16_ts(tmem + pf::kOCol0, tmem + pf::kSCol0 + b * pf::kKeys + kk * 8, bd, pf::kIdescPV,
-                     (jj > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_f16_ts_warp(tmem + pf::kOCol0, tmem + pf::kSCol0 + b * pf::kKeys + kk * 8, bd, pf::kIdescPV,
+                              (jj > 0 || kk > 0) ? 1u : 0u);
         }
-        tc::commit(&vfree[b]);
+        tc::commit_warp(&vfree[b]);
         return true;
       };
       for (; j < n_tiles && ok; ++j) {
         const int b = j & 1;
-        if (!mbar_wait(&kready[b], (j >> 1) & 1)) {
+        if (!wait_all(&kready[b], (j >> 1) & 1)) {
           ok = false;
           break;
         }
@@ -293,17 +288,17 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
 #pragma unroll
         for (int kk = 0; kk < kHeadDim / 16; ++kk) {
           const uint64_t bd = tc::sw128_desc(k_base + b * 32768 + (kk >> 2) * 8192 + (kk & 3) * 32, 1024, 16);
-          mma_f16_ts(tmem + pf::kSCol0 + b * pf::kKeys, tmem + pf::kQCol0 + kk * 8, bd, pf::kIdescQK,
-                     kk > 0 ? 1u : 0u);
+          tc::mma_f16_ts_warp(tmem + pf::kSCol0 + b * pf::kKeys, tmem + pf::kQCol0 + kk * 8, bd, pf::kIdescQK,
+                              kk > 0 ? 1u : 0u);
         }
-        tc::commit(&sready[b]);
-        tc::commit(&kfree[b]);
+        tc::commit_warp(&sready[b]);
+        tc::commit_warp(&kfree[b]);
         if (j >= 1) ok = issue_pv(j - 1);
       }
       if (ok && j >= 1) ok = issue_pv(j - 1);
-      if (!ok) *s_abort = 1;
-      tc::commit(ofinal);    // arrives when every MMA above has completed
-      mbar_wait(ofinal, 0);  // no MMA may still run when the tensor memory is freed
+      if (!ok && lane == 0) *s_abort = 1;
+      tc::commit_warp(ofinal);  // arrives when every MMA above has completed
+      wait_all(ofinal, 0);      // no MMA may still run when the tensor memory is freed
     }
   } else if (warp < pf::kSoftmaxWarps) {
     // ------------------------------------------------------------ softmax (thread = row)
