@@ -46,25 +46,30 @@ struct PrefillParams {
 namespace pf {
 constexpr int kRows = 128;
 constexpr int kKeys = 64;
-constexpr int kSoftmaxWarps = 4;  // warps 0-3: TMEM lane quarters 0-3
+constexpr int kPairKeys = kKeys / 2;  // keys of a tile each CTA of a pair dequantizes
+constexpr int kSoftmaxWarps = 4;      // warps 0-3: TMEM lane quarters 0-3
 constexpr int kMmaWarp = 4;
 constexpr int kLoadWarp = 5;
 constexpr int kDequantWarps = 8;  // warps 6-13
 constexpr int kThreads = (kSoftmaxWarps + 2 + kDequantWarps) * 32;
 constexpr int kDq0 = (kSoftmaxWarps + 2) * 32;  // first dequant thread
-// raw bytes of one 64-key tile, as copied from the page
-constexpr int kRawKc = 16384, kRawKs = 1024, kRawVc = 8192, kRawVs = 1024;
-constexpr int kRawBytes = kRawKc + kRawKs + kRawVc + kRawVs;  // 26,624
-constexpr int kRawStages = 3;
-// a CTA walks at most this many 64-key tiles (the host plan keeps pages per CTA <= 512)
-constexpr int kMaxTiles = 1024;
+// raw bytes a CTA copies per 64-key tile: K codes and scales of its 32 keys (contiguous in
+// the page), V codes of its 128 head dimensions for all 64 keys (four 1 KB pieces, one per
+// 16-key group), and all V scales of the tile
+constexpr int kRawKc = 8192, kRawKs = 512, kRawVc = 4096, kRawVs = 1024;
+constexpr int kRawBytes = kRawKc + kRawKs + kRawVc + kRawVs;  // 13,824
+constexpr uint32_t kHalfBytes = 16384;  // K^ or V^T bytes a CTA receives from its peer per tile
+constexpr int kRawStages = 2;
+constexpr int kBufs = 3;  // K^ and V^T buffers: dequant runs up to two tiles ahead of the MMAs
+// a CTA walks at most this many 64-key tiles (the host plan keeps pages per CTA <= 256)
+constexpr int kMaxTiles = 512;
 // shared memory map (bytes)
-constexpr int kKOff = 0;                                  // 2 buffers x 4 atoms x [64 keys][128 B]
-constexpr int kVOff = kKOff + 2 * 32768;                  // 2 buffers x [256 dims][128 B]
-constexpr int kRawOff = kVOff + 2 * 32768;                // kRawStages stages of raw tile bytes
+constexpr int kKOff = 0;                                  // kBufs buffers x 4 atoms x [64 keys][128 B]
+constexpr int kVOff = kKOff + kBufs * 32768;              // kBufs buffers x [256 dims][128 B]
+constexpr int kRawOff = kVOff + kBufs * 32768;            // kRawStages stages of raw tile bytes
 constexpr int kTileOff = kRawOff + kRawStages * kRawBytes;  // int2 [kMaxTiles]: page, 2*logical+half
 constexpr int kMiscOff = kTileOff + 8 * kMaxTiles;
-constexpr int kSmemBytes = kMiscOff + 1024;
+constexpr int kSmemBytes = kMiscOff + 512;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
@@ -74,6 +79,91 @@ constexpr uint32_t kQCol0 = 384;  // Q [row][256 dims] as f16 pairs: [384, 512)
 constexpr uint32_t kIdescQK = tc::idesc_f16(128, kKeys, 0, 0);
 constexpr uint32_t kIdescPV = tc::idesc_f16(128, 256, 0, 0);
 }  // namespace pf
+
+// ---- the CTA pair (a cluster of two): shared-memory addresses in the peer, remote stores
+// and barrier arrivals, cluster-scope waits ----
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of this CTA's shared-memory address `a` in CTA `rank`.
+__device__ __forceinline__ uint32_t map_shared(uint32_t a, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+// Orders this thread's shared-memory writes (its own CTA's and the peer's) before later
+// tensor-core reads of them.
+__device__ __forceinline__ void fence_proxy_async_cluster() {
+  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts128u(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+// Copy engine: `bytes` of this CTA's shared memory at `src` to the peer's shared memory at
+// shared::cluster address `dst`, completing the peer's barrier at `bar` by byte count.
+// Addresses and size are multiples of 16.
+__device__ __forceinline__ void bulk_s2peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "r"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+// Waits until every bulk copy this thread issued has completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Named barrier over `n` threads that also ANDs a flag over them.
+__device__ __forceinline__ bool bar_and(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+// Arrives on the barrier at shared::cluster address `addr` (this CTA's or the peer's).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+// mbar_wait for barriers that the peer CTA (or a multicast commit) also arrives on.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait_cluster(bar, parity, 0u)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  while (!mbar_try_wait_cluster(bar, parity, 1000000u)) {
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      record_error(KVATTN_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
 
 // The CTA's i-th candidate tile (2 per listed page): 1 if it holds a key that some row of
 // the M-tile may see (*page, *lh = 2 * logical block + half), 0 if not, -1 if its page id is
@@ -150,17 +240,18 @@ __device__ __forceinline__ float pf_p32(const uint32_t (&v)[32], uint32_t mu_bit
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pf::kMiscOff);
-  uint64_t* rawfull = bars + 0;   // [3] producer (tx bytes) -> dequant
-  uint64_t* rawempty = bars + 3;  // [3] dequant -> producer
-  uint64_t* kready = bars + 6;    // [2] dequant -> MMA
-  uint64_t* vready = bars + 8;    // [2]
-  uint64_t* kfree = bars + 10;    // [2] MMA (QK done) -> dequant
-  uint64_t* vfree = bars + 12;    // [2] MMA (PV done) -> dequant, softmax
-  uint64_t* sready = bars + 14;   // [2] MMA -> softmax
-  uint64_t* pready = bars + 16;   // [2] softmax -> MMA
-  uint64_t* ofinal = bars + 18;   // MMA -> softmax (epilogue)
-  uint64_t* qready = bars + 19;   // softmax (Q in TMEM) -> MMA
-  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bars + 20);
+  uint64_t* rawfull = bars + 0;    // [2] producer (tx bytes) -> dequant
+  uint64_t* rawempty = bars + 2;   // [2] dequant -> producer
+  uint64_t* kready = bars + 4;     // [3] both halves of K^ in place (local + peer copy) -> MMA
+  uint64_t* vready = bars + 7;     // [3]
+  uint64_t* kfree = bars + 10;     // [3] QK done in both CTAs -> dequant
+  uint64_t* vfreep = bars + 13;    // [3] PV done in both CTAs -> dequant
+  uint64_t* vfree = bars + 16;     // one phase per PV of this CTA -> softmax (rescale of O)
+  uint64_t* sready = bars + 17;    // [2] MMA -> softmax
+  uint64_t* pready = bars + 19;    // [2] softmax -> MMA
+  uint64_t* ofinal = bars + 21;    // MMA -> softmax (epilogue)
+  uint64_t* qready = bars + 22;    // softmax (Q in TMEM) -> MMA
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bars + 23);
   int* s_abort = reinterpret_cast<int*>(tmem_base_s + 1);
   int* s_ntiles = s_abort + 1;
   const int2* tiles = reinterpret_cast<const int2*>(smem + pf::kTileOff);
@@ -172,25 +263,31 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
   int np = p.max_pages;
   if (p.n_pages_arr) np = min(max(p.n_pages_arr[h], 0), p.max_pages);
   // largest query position among this M-tile's rows: keys beyond it are never visible
+  // (over both M-tiles of the pair: the two CTAs walk the same tiles)
   int max_qpos = INT_MIN;
   {
-    const int t0 = row0 / p.group, t1 = min(n_rows - 1, row0 + pf::kRows - 1) / p.group;
+    const int pair_row0 = (mt & ~1) * pf::kRows;
+    const int t0 = pair_row0 / p.group, t1 = min(n_rows - 1, pair_row0 + 2 * pf::kRows - 1) / p.group;
     for (int t = t0; t <= t1; ++t) max_qpos = max(max_qpos, p.q_pos[t]);
   }
+  const uint32_t crank = cluster_rank(), peer = crank ^ 1u;
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < pf::kRawStages; ++b) {
       mbar_init(&rawfull[b], 1);
       mbar_init(&rawempty[b], pf::kDequantWarps);
     }
+    for (int b = 0; b < pf::kBufs; ++b) {
+      mbar_init(&kready[b], 1);  // + the peer's half as transaction bytes
+      mbar_init(&vready[b], 1);
+      mbar_init(&kfree[b], 2);
+      mbar_init(&vfreep[b], 2);
+    }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&kready[b], pf::kDequantWarps);
-      mbar_init(&vready[b], pf::kDequantWarps);
-      mbar_init(&kfree[b], 1);
-      mbar_init(&vfree[b], 1);
       mbar_init(&sready[b], 1);
       mbar_init(&pready[b], pf::kSoftmaxWarps);
     }
+    mbar_init(vfree, 1);
     mbar_init(ofinal, 1);
     mbar_init(qready, pf::kSoftmaxWarps);
     *s_abort = 0;
@@ -222,6 +319,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
   }
   tc::fence_before_sync();
   __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before any remote arrival or store
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_base_s;
   const int n_tiles = *s_ntiles;
@@ -237,14 +335,17 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
           *s_abort = 1;
           break;
         }
-        const int half = tl.y & 1;
+        // K: this CTA's 32 keys of the tile (quarter q of the page); V: its 128 dimensions
+        const int half = tl.y & 1, q = 2 * half + static_cast<int>(crank);
         uint8_t* st = smem + pf::kRawOff + r * pf::kRawBytes;
         const uint8_t* kp = p.k_pool + static_cast<int64_t>(tl.x) * p.k_stride;
         const uint8_t* vp = p.v_pool + static_cast<int64_t>(tl.x) * p.v_stride;
         mbar_arrive_expect_tx(&rawfull[r], pf::kRawBytes);
-        bulk_g2s(st, kp + half * pf::kRawKc, pf::kRawKc, &rawfull[r]);
-        bulk_g2s(st + pf::kRawKc, kp + kKScaleOffset + half * pf::kRawKs, pf::kRawKs, &rawfull[r]);
-        bulk_g2s(st + pf::kRawKc + pf::kRawKs, vp + half * pf::kRawVc, pf::kRawVc, &rawfull[r]);
+        bulk_g2s(st, kp + q * pf::kRawKc, pf::kRawKc, &rawfull[r]);
+        bulk_g2s(st + pf::kRawKc, kp + kKScaleOffset + q * pf::kRawKs, pf::kRawKs, &rawfull[r]);
+        for (int g = 0; g < 4; ++g)
+          bulk_g2s(st + pf::kRawKc + pf::kRawKs + g * 1024, vp + half * 8192 + g * 2048 + crank * 1024, 1024,
+                   &rawfull[r]);
         bulk_g2s(st + pf::kRawKc + pf::kRawKs + pf::kRawVc, vp + kV4ScaleOffset + half * pf::kRawVs, pf::kRawVs,
                  &rawfull[r]);
       }
@@ -254,51 +355,67 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     }
   } else if (warp == pf::kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    // The whole warp runs this loop (one elected lane issues each instruction); every wait
-    // result is made warp-uniform so the lanes never diverge around elect.sync.
+    // The whole warp runs this loop (one elected lane issues each instruction); barrier
+    // checks are made warp-uniform so the lanes never diverge around elect.sync.  Each pass
+    // issues whichever is ready of QK of the next tile (once its K^ is in place and the S
+    // buffer it overwrites was consumed by PV two tiles back) and PV of the oldest tile whose
+    // P is written, so a late K^ does not hold back a ready PV.
     {
       const uint32_t k_base = smem_u32(smem + pf::kKOff);
       const uint32_t v_base = smem_u32(smem + pf::kVOff);
-      auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
-        return __all_sync(0xffffffffu, mbar_wait(bar, par));
+      auto ready_all = [&](uint64_t* bar, uint32_t par) -> bool {
+        return __all_sync(0xffffffffu, mbar_try_wait_cluster(bar, par, 0u));
       };
-      int j = 0;
-      bool ok = wait_all(qready, 0);
-      auto issue_pv = [&](int jj) -> bool {
-        const int b = jj & 1;
-        const uint32_t par = (jj >> 1) & 1;
-        if (!wait_all(&pready[b], par) || !wait_all(&vready[b], par)) return false;
-        tc::fence_after_sync();
+      bool ok = __all_sync(0xffffffffu, mbar_wait(qready, 0));
+      int jq = 0, jp = 0;  // next QK, next PV
+      unsigned long long t_idle = 0;
+      while (ok && jp < n_tiles) {
+        bool did = false;
+        if (jq < n_tiles && jq <= jp + 1 && ready_all(&kready[jq % pf::kBufs], (jq / pf::kBufs) & 1)) {
+          const int b = jq % pf::kBufs, s2 = jq & 1;
+          tc::fence_after_sync();
 #pragma unroll
-        for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
-          const uint64_t bd = tc::sw128_desc(v_base + b * 32768 + kk * 32, 1024, 16);
-          tc::mma_f16_ts_warp(tmem + pf::kOCol0, tmem + pf::kSCol0 + b * pf::kKeys + kk * 8, bd, pf::kIdescPV,
-                              (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc::commit_warp(&vfree[b]);
-        return true;
-      };
-      for (; j < n_tiles && ok; ++j) {
-        const int b = j & 1;
-        if (!wait_all(&kready[b], (j >> 1) & 1)) {
-          ok = false;
-          break;
-        }
-        tc::fence_after_sync();
+          for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+            const uint64_t bd = tc::sw128_desc(k_base + b * 32768 + (kk >> 2) * 8192 + (kk & 3) * 32, 1024, 16);
+            tc::mma_f16_ts_warp(tmem + pf::kSCol0 + s2 * pf::kKeys, tmem + pf::kQCol0 + kk * 8, bd, pf::kIdescQK,
+                                kk > 0 ? 1u : 0u);
+          }
+          tc::commit_warp(&sready[s2]);
+          tc::commit_pair_warp(&kfree[b]);
+          ++jq;
+          did = true;
+        } else if (jp < jq && ready_all(&pready[jp & 1], (jp >> 1) & 1) &&
+                   ready_all(&vready[jp % pf::kBufs], (jp / pf::kBufs) & 1)) {
+          const int b = jp % pf::kBufs, s2 = jp & 1;
+          tc::fence_after_sync();
 #pragma unroll
-        for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-          const uint64_t bd = tc::sw128_desc(k_base + b * 32768 + (kk >> 2) * 8192 + (kk & 3) * 32, 1024, 16);
-          tc::mma_f16_ts_warp(tmem + pf::kSCol0 + b * pf::kKeys, tmem + pf::kQCol0 + kk * 8, bd, pf::kIdescQK,
-                              kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
+            const uint64_t bd = tc::sw128_desc(v_base + b * 32768 + kk * 32, 1024, 16);
+            tc::mma_f16_ts_warp(tmem + pf::kOCol0, tmem + pf::kSCol0 + s2 * pf::kKeys + kk * 8, bd, pf::kIdescPV,
+                                (jp > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc::commit_warp(vfree);
+          tc::commit_pair_warp(&vfreep[b]);
+          ++jp;
+          did = true;
         }
-        tc::commit_warp(&sready[b]);
-        tc::commit_warp(&kfree[b]);
-        if (j >= 1) ok = issue_pv(j - 1);
+        if (did) {
+          t_idle = 0;
+        } else {
+          const unsigned long long now = global_timer_ns();
+          if (t_idle == 0) {
+            t_idle = now;
+          } else if (now - t_idle > kWaitTimeoutNs) {
+            if (lane == 0) record_error(KVATTN_ERR_TIMEOUT);
+            ok = false;
+          }
+          __nanosleep(32);
+        }
+        ok = __all_sync(0xffffffffu, ok);
       }
-      if (ok && j >= 1) ok = issue_pv(j - 1);
       if (!ok && lane == 0) *s_abort = 1;
       tc::commit_warp(ofinal);  // arrives when every MMA above has completed
-      wait_all(ofinal, 0);      // no MMA may still run when the tensor memory is freed
+      __all_sync(0xffffffffu, mbar_wait(ofinal, 0));  // no MMA may still run when TMEM is freed
     }
   } else if (warp < pf::kSoftmaxWarps) {
     // ------------------------------------------------------------ softmax (thread = row)
@@ -374,7 +491,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       if (__any_sync(0xffffffffu, resc)) {
         // O is rescaled to the new maximum before PV of this tile accumulates into it; this
         // warp's rows of O hold the previous tile's PV only once that completed
-        if (!mbar_wait(&vfree[(j - 1) & 1], ((j - 1) >> 1) & 1)) {
+        if (!mbar_wait(vfree, (j - 1) & 1)) {
           ok = false;
           break;
         }
@@ -443,57 +560,67 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     }
   } else if (warp >= pf::kDq0 / 32) {
     // ------------------------------------------------------------ dequant (256 threads)
+    // This CTA dequantizes half of every tile (K^: its 32 keys; V^T: its 128 dimensions) into
+    // its own buffers; one thread then copies that half into the peer's buffers with the
+    // copy engine, which completes the peer's barrier by byte count.
     const int d = threadIdx.x - pf::kDq0;
-    // K task: channel quarter kP (blocks 2kP, 2kP+1) of key kn; 8 consecutive threads take
-    // 8 consecutive keys, so their swizzled 16-byte stores hit 8 different bank groups.
-    const int kP = d >> 6, kn = d & 63;
-    const int kG = kn >> 4, kH = (kn >> 3) & 1, kR = kn & 7;
-    // V task: token group vG (16 keys), block pair vC, channel row vR (channels vR + 8k of
-    // both blocks), key half vh (keys 8vh..8vh+7 of the group)
-    const int vR = d & 7, vh = (d >> 3) & 1, vC = (d >> 4) & 3, vG = d >> 6;
+    // K task: key kl of this CTA's 32, channel quarter kP (blocks 2kP, 2kP+1), raw chunks
+    // 2cp and 2cp+1 of the four; 8 consecutive threads take 8 consecutive keys, so their
+    // swizzled 16-byte stores hit 8 different bank groups.
+    const int kl = d & 31, kP = (d >> 5) & 3, cp = d >> 7;
+    const int kGl = kl >> 4, kH = (kl >> 3) & 1, kR = kl & 7;
+    const int kn = pf::kPairKeys * static_cast<int>(crank) + kl;  // row of K^ (key within the tile)
+    // V task: channel row vR (channels vR + 8k of block 2vC + ve, vC = 2 * rank + vCl), key
+    // half vh of token group vG (16 keys)
+    const int vR = d & 7, vh = (d >> 3) & 1, vCl = (d >> 4) & 1, vG = (d >> 5) & 3, ve = d >> 7;
+    const int vC = 2 * static_cast<int>(crank) + vCl;
     // 16-byte chunks are read in an order rotated by (row / 2): 8 threads at a 64-byte
     // stride then touch 8 different bank groups
     const int rotK = kR >> 1, rotV = vR >> 1;
+    const uint32_t own = smem_u32(smem), other = map_shared(own, peer);
+    const uint32_t kready_peer = map_shared(smem_u32(&kready[0]), peer);
+    const uint32_t vready_peer = map_shared(smem_u32(&vready[0]), peer);
     int j = 0;
     bool ok = true;
     for (; j < n_tiles && ok; ++j) {
-      const int b = j & 1, r = j % pf::kRawStages;
-      if (!mbar_wait(&rawfull[r], (j / pf::kRawStages) & 1)) {
-        ok = false;
-        break;
-      }
-      const uint32_t stu = smem_u32(smem + pf::kRawOff + r * pf::kRawBytes);
+      const int b = j % pf::kBufs, r = j % pf::kRawStages;
+      // every wait result is combined over the 256 dequant threads at the named barriers, so
+      // all of them stop at the same tile when one gives up
+      bool wok = mbar_wait(&rawfull[r], (j / pf::kRawStages) & 1);
+      const uint32_t stu = own + pf::kRawOff + r * pf::kRawBytes;
       // ---------------- raw K, V -> registers; the stage is then released ----------------
-      uint4 kraw[4];
-      const uint32_t kbase = stu + ((((kG * 4 + kP) * 2 + kH) * 8 + kR) * 4) * 16;
+      uint4 kraw[2] = {};
+      uint32_t dkw = 0;
+      uint2 vraw[4] = {}, dvr[4] = {};
+      if (wok) {
+        const uint32_t kbase = stu + ((((kGl * 4 + kP) * 2 + kH) * 8 + kR) * 4) * 16;
 #pragma unroll
-      for (int ii = 0; ii < 4; ++ii) kraw[ii] = lds128(kbase + (((ii + rotK) & 3) << 4));
-      uint32_t dkw;
-      asm volatile("ld.shared.u32 %0, [%1];"
-                   : "=r"(dkw)
-                   : "r"(stu + pf::kRawKc + ((kG * 8 + kR) * 2 + kH) * 16 + 4 * kP));
-      uint4 vraw[4], dvr[4];
-      const uint32_t vbase = stu + pf::kRawKc + pf::kRawKs + ((((vG * 4 + vC) * 8 + vR) * 4) * 16);
+        for (int i = 0; i < 2; ++i) kraw[i] = lds128(kbase + (((2 * cp + i + rotK) & 3) << 4));
+        asm volatile("ld.shared.u32 %0, [%1];"
+                     : "=r"(dkw)
+                     : "r"(stu + pf::kRawKc + ((kGl * 8 + kR) * 2 + kH) * 16 + 4 * kP));
+        // this thread's two words (block 2vC + ve, both key halves) of each raw chunk and of
+        // the scales of each token pair
+        const uint32_t vbase = stu + pf::kRawKc + pf::kRawKs + vG * 1024 + ((vCl * 8 + vR) * 4) * 16 + 8 * ve;
 #pragma unroll
-      for (int ii = 0; ii < 4; ++ii) vraw[ii] = lds128(vbase + (((ii + rotV) & 3) << 4));
+        for (int ii = 0; ii < 4; ++ii) vraw[ii] = lds64(vbase + (((ii + rotV) & 3) << 4));
 #pragma unroll
-      for (int T = 0; T < 4; ++T)
-        dvr[T] = lds128(stu + pf::kRawKc + pf::kRawKs + pf::kRawVc + ((vG * 4 + T) * 8 + 2 * vC) * 8);
+        for (int T = 0; T < 4; ++T)
+          dvr[T] = lds64(stu + pf::kRawKc + pf::kRawKs + pf::kRawVc + ((vG * 4 + T) * 8 + 2 * vC) * 8 + 8 * ve);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&rawempty[r]);
-      // ---------------- K^ ----------------
-      if (j >= 2 && !mbar_wait(&kfree[b], ((j - 2) >> 1) & 1)) {
-        ok = false;
-        break;
-      }
-      {
+      // ---------------- K^ (both CTAs' buffers are free once both QK(j - 3) completed) ----
+      if (wok && j >= pf::kBufs) wok = mbar_wait_cluster(&kfree[b], ((j / pf::kBufs) - 1) & 1);
+      const uint32_t katom0 = pf::kKOff + b * 32768;
+      if (wok) {
         const uint32_t dlo = prmt(dkw, 0u, 0x1010u), dhi = prmt(dkw, 0u, 0x3232u);
-        uint8_t* katom = smem + pf::kKOff + b * 32768 + kP * 8192;
+        const uint32_t katom = katom0 + kP * 8192;
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-          const int T = (ii + rotK) & 3;
-          const uint32_t w[4] = {kraw[ii].x ^ 0x80808080u, kraw[ii].y ^ 0x80808080u, kraw[ii].z ^ 0x80808080u,
-                                 kraw[ii].w ^ 0x80808080u};
+        for (int i = 0; i < 2; ++i) {
+          const int T = (2 * cp + i + rotK) & 3;
+          const uint32_t w[4] = {kraw[i].x ^ 0x80808080u, kraw[i].y ^ 0x80808080u, kraw[i].z ^ 0x80808080u,
+                                 kraw[i].w ^ 0x80808080u};
           uint32_t o[8];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -501,76 +628,80 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
             o[2 * e] = hmul2(hsub2(prmt(w[e], 0x64646464u, 0x4140u), 0x64806480u), sc);
             o[2 * e + 1] = hmul2(hsub2(prmt(w[e], 0x64646464u, 0x4342u), 0x64806480u), sc);
           }
-          *reinterpret_cast<uint4*>(katom + swz(kn, T)) = make_uint4(o[0], o[1], o[2], o[3]);
-          *reinterpret_cast<uint4*>(katom + swz(kn, 4 + T)) = make_uint4(o[4], o[5], o[6], o[7]);
+          sts128u(own + katom + swz(kn, T), o[0], o[1], o[2], o[3]);
+          sts128u(own + katom + swz(kn, 4 + T), o[4], o[5], o[6], o[7]);
         }
+        tc::fence_proxy_async_smem();
       }
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&kready[b]);
-      // ---------------- V^T ----------------
-      if (j >= 2 && !mbar_wait(&vfree[b], ((j - 2) >> 1) & 1)) {
+      if (!bar_and(1, 32 * pf::kDequantWarps, wok)) {
         ok = false;
         break;
       }
-      {
-        // This thread's words (key half vh, blocks 2C and 2C+1) of each raw chunk; chunk ii
-        // holds token pair (ii + rotV) & 3.  Two select stages undo the rotation so that
-        // wv[T] is token pair T: an array indexed by the runtime rotation would be placed in
-        // local memory.
-        uint32_t wv[4][2];
+      if (d == 0) {
+        // this CTA's 32 rows of each of the four K^ atoms -> the peer; the peer's half comes
+        // the other way as transaction bytes on kready
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-          wv[ii][0] = vh ? vraw[ii].y : vraw[ii].x;
-          wv[ii][1] = vh ? vraw[ii].w : vraw[ii].z;
+        for (int a = 0; a < 4; ++a) {
+          const uint32_t off = katom0 + a * 8192 + crank * 4096;
+          bulk_s2peer(other + off, own + off, 4096, kready_peer + 8 * b);
         }
-        {
-          const bool r1 = rotV & 1;
-          uint32_t t[4][2];
-#pragma unroll
-          for (int x = 0; x < 4; ++x)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) t[x][e] = r1 ? wv[(x + 3) & 3][e] : wv[x][e];
-          const bool r2 = rotV & 2;
-#pragma unroll
-          for (int x = 0; x < 4; ++x)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) wv[x][e] = r2 ? t[(x + 2) & 3][e] : t[x][e];
-        }
-        uint8_t* vt = smem + pf::kVOff + b * 32768;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {  // block 2C + e
-          uint32_t o[4][4];            // [k][T]
-#pragma unroll
-          for (int T = 0; T < 4; ++T) {
-            const uint32_t W = wv[T][e];
-            const uint32_t Ws = W >> 8;
-            const uint32_t dv = e ? (vh ? dvr[T].w : dvr[T].z) : (vh ? dvr[T].y : dvr[T].x);
-            const uint32_t v0 = hsub2(and_or(W, 0x000F000Fu, 0x64006400u), 0x64086408u);
-            const uint32_t v1 = hfma2(and_or(W, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
-            const uint32_t v2 = hsub2(and_or(Ws, 0x000F000Fu, 0x64006400u), 0x64086408u);
-            const uint32_t v3 = hfma2(and_or(Ws, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
-            o[0][T] = hmul2(v0, dv);
-            o[1][T] = hmul2(v1, dv);
-            o[2][T] = hmul2(v2, dv);
-            o[3][T] = hmul2(v3, dv);
-          }
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int dim = 32 * (2 * vC + e) + 8 * k + vR;
-            *reinterpret_cast<uint4*>(vt + swz(dim, 2 * vG + vh)) = make_uint4(o[k][0], o[k][1], o[k][2], o[k][3]);
-          }
-        }
+        mbar_arrive_expect_tx(&kready[b], pf::kHalfBytes);
       }
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&vready[b]);
+      // ---------------- V^T: rows 128 * rank .. of the buffer ----------------
+      if (j >= pf::kBufs) wok = mbar_wait_cluster(&vfreep[b], ((j / pf::kBufs) - 1) & 1);
+      const uint32_t vt = pf::kVOff + b * 32768;
+      if (wok) {
+        // chunk ii holds token pair (ii + rotV) & 3: two select stages undo the rotation so
+        // that wv[T] is token pair T (an array indexed by the runtime rotation would be
+        // placed in local memory)
+        uint32_t wv[4], t[4];
+#pragma unroll
+        for (int ii = 0; ii < 4; ++ii) wv[ii] = vh ? vraw[ii].y : vraw[ii].x;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) t[x] = (rotV & 1) ? wv[(x + 3) & 3] : wv[x];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) wv[x] = (rotV & 2) ? t[(x + 2) & 3] : t[x];
+        uint32_t o[4][4];  // [k][T]
+#pragma unroll
+        for (int T = 0; T < 4; ++T) {
+          const uint32_t W = wv[T];
+          const uint32_t Ws = W >> 8;
+          const uint32_t dv = vh ? dvr[T].y : dvr[T].x;
+          const uint32_t v0 = hsub2(and_or(W, 0x000F000Fu, 0x64006400u), 0x64086408u);
+          const uint32_t v1 = hfma2(and_or(W, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
+          const uint32_t v2 = hsub2(and_or(Ws, 0x000F000Fu, 0x64006400u), 0x64086408u);
+          const uint32_t v3 = hfma2(and_or(Ws, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
+          o[0][T] = hmul2(v0, dv);
+          o[1][T] = hmul2(v1, dv);
+          o[2][T] = hmul2(v2, dv);
+          o[3][T] = hmul2(v3, dv);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int dim = 32 * (2 * vC + ve) + 8 * k + vR;
+          sts128u(own + vt + swz(dim, 2 * vG + vh), o[k][0], o[k][1], o[k][2], o[k][3]);
+        }
+        tc::fence_proxy_async_smem();
+      }
+      if (!bar_and(2, 32 * pf::kDequantWarps, wok)) {
+        ok = false;
+        break;
+      }
+      if (d == 0) {
+        const uint32_t off = vt + crank * pf::kHalfBytes;
+        bulk_s2peer(other + off, own + off, pf::kHalfBytes, vready_peer + 8 * b);
+        mbar_arrive_expect_tx(&vready[b], pf::kHalfBytes);
+      }
     }
     if (!ok) *s_abort = 1;
+    // the copies this CTA sent must have landed before either CTA may leave
+    if (d == 0) bulk_wait_all();
   }
 
   tc::fence_before_sync();
   __syncthreads();
+  // the peer stores into and arrives on this CTA's shared memory until it gets here
+  cluster_sync();
   if (*s_abort && threadIdx.x == 0) record_error(KVATTN_ERR_TIMEOUT);
   if (warp == pf::kMmaWarp) {
     tc::fence_after_sync();
@@ -594,15 +725,15 @@ PrefillPlan plan_prefill(int n_kv, int group, int n_q, int max_pages, int kv_spl
   PrefillPlan pl{};
   const int rows = n_q * group;
   pl.n_mt = (rows + pf::kRows - 1) / pf::kRows;
+  pl.n_mt += pl.n_mt & 1;  // M-tiles come in pairs (one cluster of two CTAs per pair)
   pl.rows_pad = pl.n_mt * pf::kRows;
   const int base = kv_split_tokens / kPageTokens;
   const long long splits0 = max_pages > 0 ? (max_pages + base - 1) / base : 1;
   long long spc = static_cast<long long>(n_kv) * pl.n_mt * splits0 / (static_cast<long long>(sm_count) * 16);
-  long long spc_max = (pf::kMaxTiles / 2) / base;  // the API keeps kv_split_tokens <= 65,536
-  spc_max = spc_max < 1 ? 1 : spc_max;
   spc = spc < 1 ? 1 : (spc > splits0 ? splits0 : spc);
-  spc = spc > spc_max ? spc_max : spc;
-  pl.pps = static_cast<int>(base * spc);
+  // pages per CTA: spc splits, at most kMaxTiles / 2 (a large split is then divided)
+  const long long pps = base * spc;
+  pl.pps = static_cast<int>(pps < pf::kMaxTiles / 2 ? pps : pf::kMaxTiles / 2);
   pl.n_ks = max_pages > 0 ? (max_pages + pl.pps - 1) / pl.pps : 1;
   pl.lse_off = 0;
   pl.o_off = ((sizeof(float) * static_cast<size_t>(n_kv) * pl.n_ks * pl.rows_pad + 255) / 256) * 256;
@@ -613,10 +744,22 @@ PrefillPlan plan_prefill(int n_kv, int group, int n_q, int max_pages, int kv_spl
 cudaError_t launch_prefill(const PrefillParams& prm0, int n_kv, cudaStream_t stream) {
   PrefillParams prm = prm0;
   const int rows = prm.n_q * prm.group;
-  dim3 grid((rows + pf::kRows - 1) / pf::kRows, prm.n_ks, n_kv);
-  prefill_kernel<<<grid, pf::kThreads, pf::kSmemBytes, stream>>>(prm);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || prm.n_ks == 1) return e;
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(prm.rows_pad / pf::kRows, prm.n_ks, n_kv);
+    cfg.blockDim = dim3(pf::kThreads);
+    cfg.dynamicSmemBytes = pf::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_kernel, prm);
+    if (e != cudaSuccess || prm.n_ks == 1) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rows, n_kv);
   cfg.blockDim = dim3(kMergeThreads);
