@@ -151,7 +151,10 @@ KVATTN_API int kvattn_quantize_append(const kvattn_kv_desc* desc, const float* k
  *   ws, ws_bytes device workspace of at least kvattn_decode_workspace_size() bytes (256-byte
  *                aligned; may be NULL when that size is 0).  The keys of each KV head are
  *                split across CTAs; per-split (o, lse) partials go to the workspace and a
- *                second grid, launched behind the first, merges them.
+ *                second grid, launched behind the first, merges them.  Calls that share a
+ *                workspace must not overlap on the GPU.
+ * Both grids use programmatic dependent launch: each may start while the kernel before it on
+ * the stream finishes, and waits for that kernel before reading any argument.
  * Supports group * n_q <= 24 query rows per KV head.  The split count depends only on the
  * arguments and the device, so results are deterministic. */
 KVATTN_API size_t kvattn_decode_workspace_size(const kvattn_kv_desc* desc, int n_q, int max_pages);

@@ -71,12 +71,6 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
   const int g = lane >> 2, t = lane & 3;
   const int n_rows = p.group * p.n_q;
 
-  int np = p.max_pages;
-  if (p.n_pages_arr) np = min(max(p.n_pages_arr[h], 0), p.max_pages);
-  const int first = static_cast<int>(static_cast<long long>(split) * np / p.n_splits);
-  const int last = static_cast<int>(static_cast<long long>(split + 1) * np / p.n_splits);
-  const int count = last - first;
-
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -88,6 +82,16 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
     fence_barrier_init();
   }
   __syncthreads();
+  // Launched with programmatic dependent launch: the CTAs become resident and set up while
+  // the previous kernel on the stream (typically the quantize-append of the new token)
+  // drains; every read of the caller's data comes after this wait.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  int np = p.max_pages;
+  if (p.n_pages_arr) np = min(max(p.n_pages_arr[h], 0), p.max_pages);
+  const int first = static_cast<int>(static_cast<long long>(split) * np / p.n_splits);
+  const int last = static_cast<int>(static_cast<long long>(split + 1) * np / p.n_splits);
+  const int count = last - first;
 
   // per-warp softmax state (consumers)
   float m_run[NT][2], l_run[NT][2];
@@ -133,8 +137,12 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
     }
     *reinterpret_cast<volatile int*>(s_issued) = i + 1;
   };
-  if (warp == 0 && lane == 0)
-    for (int i = 0; i < count && i < C::kStages; ++i) issue(i);
+  // the first stages are issued by parallel lanes: their page-table reads overlap
+  if (warp == 0) {
+    if (lane < C::kStages && lane < count) issue(lane);
+    __syncwarp();
+    if (lane == 0) *reinterpret_cast<volatile int*>(s_issued) = count < C::kStages ? count : C::kStages;
+  }
 
   {
     // ------------------------------------------------------------------ consumers
@@ -589,19 +597,23 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const float
 template <int NT, bool PAIR, bool VQ8>
 static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream_t stream) {
   using C = DecodeCfg<NT, PAIR, VQ8>;
-  dim3 grid(prm.n_splits, n_kv);
-  decode_kernel<NT, PAIR, VQ8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(prm);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || prm.n_splits == 1) return e;
+  // programmatic dependent launch: the grid may start while the previous kernel on the
+  // stream drains; the kernel waits for it (griddepcontrol.wait) before reading any input
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(prm.group * prm.n_q, n_kv);
-  cfg.blockDim = dim3(kMergeThreads);
+  cfg.gridDim = dim3(prm.n_splits, n_kv);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<NT, PAIR, VQ8>, prm);
+  if (e != cudaSuccess || prm.n_splits == 1) return e;
+  cfg.gridDim = dim3(prm.group * prm.n_q, n_kv);
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.dynamicSmemBytes = 0;
   return cudaLaunchKernelEx(&cfg, decode_merge_kernel, static_cast<const float*>(prm.part_o),
                             static_cast<const float*>(prm.part_lse), prm.n_splits, C::kRowsPad, prm.group, prm.n_qh,
                             prm.out, prm.lse);

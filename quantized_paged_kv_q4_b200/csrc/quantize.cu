@@ -48,6 +48,9 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
                                                               int n_blocks, uint8_t* k_pool, int64_t k_stride,
                                                               uint8_t* v_pool, int64_t v_stride, int64_t n_pages,
                                                               int v_q8) {
+  // a kernel launched behind this one with programmatic dependent launch (decode) may start
+  // its setup now; it waits for this grid to complete before reading the pages
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= static_cast<long long>(n_tok) * n_kv) return;
