@@ -152,9 +152,16 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
     // the normalised row into a base-2 softmax score.
     uint32_t qf[C::kNB][2][NT][2];
     float crow[NT][2];
+    // query positions of this thread's accumulator rows, loaded first: every global read of
+    // the setup is issued before any of them is used
     int qpos_row[NT][2];
-    int qpos_min = INT_MAX;
-    for (int i = 0; i < p.n_q; ++i) qpos_min = min(qpos_min, p.q_pos[i]);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int rr = nt * 8 + 2 * t + c;
+        qpos_row[nt][c] = rr < n_rows ? p.q_pos[rr / p.group] : INT_MAX;
+      }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int r = nt * 8 + g;
@@ -197,12 +204,13 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
       const float cr = amax * (1.0f / 16.0f) * 1.4426950408889634f;
       crow[nt][0] = __shfl_sync(0xffffffffu, cr, (2 * t) * 4);
       crow[nt][1] = __shfl_sync(0xffffffffu, cr, (2 * t + 1) * 4);
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int rr = nt * 8 + 2 * t + c;
-        qpos_row[nt][c] = rr < n_rows ? p.q_pos[rr / p.group] : INT_MAX;
-      }
     }
+    // the smallest query position over all rows (the four t-lanes of a quad hold all rows)
+    int qpos_min = INT_MAX;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) qpos_min = min(qpos_min, min(qpos_row[nt][0], qpos_row[nt][1]));
+    qpos_min = min(qpos_min, __shfl_xor_sync(0xffffffffu, qpos_min, 1));
+    qpos_min = min(qpos_min, __shfl_xor_sync(0xffffffffu, qpos_min, 2));
 
     const int pair = PAIR ? (warp >> 1) : 0;
     float* xbuf = reinterpret_cast<float*>(smem + C::kRingBytes);
@@ -519,77 +527,79 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
 // Log-sum-exp merge of the per-split partials of kvattn_decode (and kvattn_prefill_chunk),
 // launched right behind the producing grid with programmatic dependent launch: its CTAs
 // start while that grid drains and wait (griddepcontrol.wait) until all partials are
-// written.  One CTA per (query row, KV head), 256 threads: the split log-sum-exps are
-// reduced cooperatively, then four groups of 64 threads (four channels each) accumulate
-// interleaved splits with independent loads and are summed through shared memory.
+// written.  One CTA per (query row, KV head), 256 threads = four groups of 64 (four
+// channels each); group g takes splits g, g + 4, ...  Each thread keeps an online (max, sum,
+// weighted output) over its splits, loading a batch of splits before using any of them, and
+// the four groups are combined once through shared memory.  Arithmetic of kvattn_merge_lse
+// (log2 units).
 constexpr int kMergeThreads = 256;
 constexpr int kMergeGroups = kMergeThreads / (kHeadDim / 4);
+constexpr int kMergeBatch = 8;
 
 __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const float* __restrict__ part_o,
                                                                      const float* __restrict__ part_lse, int n_splits,
                                                                      int rows_pad, int group, int n_qh,
                                                                      float* __restrict__ out, float* __restrict__ lse) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  __shared__ float red_m[kMergeThreads / 32], red_l[kMergeThreads / 32];
-  __shared__ float4 red_o[kMergeGroups - 1][kHeadDim / 4];
+  __shared__ float red_m[kMergeGroups], red_l[kMergeGroups];
+  __shared__ float4 red_o[kMergeGroups][kHeadDim / 4];
   const int row = blockIdx.x, h = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int tid = threadIdx.x, grp = tid / (kHeadDim / 4), d4 = tid % (kHeadDim / 4);
   const float* pl = part_lse + static_cast<long long>(h) * n_splits * rows_pad + row;
-  // (max, sum of exp2) over this thread's splits, then over the block
-  float m = -INFINITY, l = 0.f;
-  for (int sp = tid; sp < n_splits; sp += kMergeThreads) {
-    const float v = pl[static_cast<long long>(sp) * rows_pad];
-    if (v > m) {
-      l = (m == -INFINITY ? 0.f : l * fast_exp2(m - v)) + 1.f;
-      m = v;
-    } else if (v != -INFINITY) {
-      l += fast_exp2(v - m);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), l2 = __shfl_xor_sync(0xffffffffu, l, o);
-    const float mm = fmaxf(m, m2);
-    l = (mm == -INFINITY) ? 0.f : l * fast_exp2(m - mm) + l2 * fast_exp2(m2 - mm);
-    m = mm;
-  }
-  if (lane == 0) {
-    red_m[wid] = m;
-    red_l[wid] = l;
-  }
-  __syncthreads();
-  float M = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < kMergeThreads / 32; ++w) M = fmaxf(M, red_m[w]);
-  float L = 0.f;
-  if (M != -INFINITY)
-#pragma unroll
-    for (int w = 0; w < kMergeThreads / 32; ++w) L += red_l[w] * fast_exp2(red_m[w] - M);
-  // weighted sum of the partial outputs
-  const int grp = tid / (kHeadDim / 4), d4 = tid % (kHeadDim / 4);
   const float* po = part_o + (static_cast<long long>(h) * n_splits * rows_pad + row) * kHeadDim + d4 * 4;
+  float m = -INFINITY, l = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (M != -INFINITY) {
-    const float inv = 1.f / L;
-#pragma unroll 8
-    for (int sp = grp; sp < n_splits; sp += kMergeGroups) {
-      const float w = fast_exp2(pl[static_cast<long long>(sp) * rows_pad] - M) * inv;
-      const float4 o = *reinterpret_cast<const float4*>(po + static_cast<long long>(sp) * rows_pad * kHeadDim);
-      acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
+  for (int sp0 = grp; sp0 < n_splits; sp0 += kMergeGroups * kMergeBatch) {
+    float v[kMergeBatch];
+    float4 o[kMergeBatch];
+#pragma unroll
+    for (int k = 0; k < kMergeBatch; ++k) {
+      const int sp = sp0 + k * kMergeGroups;
+      v[k] = sp < n_splits ? pl[static_cast<long long>(sp) * rows_pad] : -INFINITY;
+      o[k] = sp < n_splits ? *reinterpret_cast<const float4*>(po + static_cast<long long>(sp) * rows_pad * kHeadDim)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < kMergeBatch; ++k) {
+      if (v[k] == -INFINITY) continue;  // a split that saw no key
+      if (v[k] > m) {
+        const float a = fast_exp2(m - v[k]);  // 0 when m = -inf
+        l *= a;
+        acc.x *= a; acc.y *= a; acc.z *= a; acc.w *= a;
+        m = v[k];
+      }
+      const float w = fast_exp2(v[k] - m);
+      l += w;
+      acc.x += w * o[k].x; acc.y += w * o[k].y; acc.z += w * o[k].z; acc.w += w * o[k].w;
     }
   }
-  if (grp > 0) red_o[grp - 1][d4] = acc;
+  if (d4 == 0) {
+    red_m[grp] = m;
+    red_l[grp] = l;
+  }
+  red_o[grp][d4] = acc;
   __syncthreads();
   if (grp == 0) {
+    float M = -INFINITY;
 #pragma unroll
-    for (int gq = 0; gq < kMergeGroups - 1; ++gq) {
-      const float4 o = red_o[gq][d4];
-      acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+    for (int gq = 0; gq < kMergeGroups; ++gq) M = fmaxf(M, red_m[gq]);
+    float L = 0.f;
+    float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int gq = 0; gq < kMergeGroups; ++gq) {
+        const float w = fast_exp2(red_m[gq] - M);  // 0 for a group that saw no key
+        L += w * red_l[gq];
+        const float4 o = red_o[gq][d4];
+        r.x += w * o.x; r.y += w * o.y; r.z += w * o.z; r.w += w * o.w;
+      }
+      const float inv = 1.f / L;
+      r.x *= inv; r.y *= inv; r.z *= inv; r.w *= inv;
     }
     const int qi = row / group, j = row % group;
     const long long orow = static_cast<long long>(qi) * n_qh + h * group + j;
-    *reinterpret_cast<float4*>(out + orow * kHeadDim + d4 * 4) = acc;
-    if (tid == 0) lse[orow] = M != -INFINITY ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    *reinterpret_cast<float4*>(out + orow * kHeadDim + d4 * 4) = r;
+    if (d4 == 0) lse[orow] = M != -INFINITY ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
   }
 }
 
