@@ -529,17 +529,19 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
 // start while that grid drains and wait (griddepcontrol.wait) until all partials are
 // written.  One CTA per (query row, KV head), 256 threads = four groups of 64 (four
 // channels each); group g takes splits g, g + 4, ...  Each thread keeps an online (max, sum,
-// weighted output) over its splits, loading a batch of splits before using any of them, and
+// weighted output) over its splits, loading a batch of up to 16 splits before using any of them, and
 // the four groups are combined once through shared memory.  Arithmetic of kvattn_merge_lse
 // (log2 units).
 constexpr int kMergeThreads = 256;
 constexpr int kMergeGroups = kMergeThreads / (kHeadDim / 4);
-constexpr int kMergeBatch = 8;
-
-__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const float* __restrict__ part_o,
+// kBatch splits are loaded ahead per thread: 16 for decode (a few dozen splits, one round
+// trip), 8 with two CTAs per SM for prefill (tens of thousands of small CTAs).
+template <int kBatch, int kMinBlocks>
+__global__ void __launch_bounds__(kMergeThreads, kMinBlocks) decode_merge_kernel(const float* __restrict__ part_o,
                                                                      const float* __restrict__ part_lse, int n_splits,
                                                                      int rows_pad, int group, int n_qh,
                                                                      float* __restrict__ out, float* __restrict__ lse) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the next kernel may set up
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float red_m[kMergeGroups], red_l[kMergeGroups];
   __shared__ float4 red_o[kMergeGroups][kHeadDim / 4];
@@ -549,18 +551,18 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(const float
   const float* po = part_o + (static_cast<long long>(h) * n_splits * rows_pad + row) * kHeadDim + d4 * 4;
   float m = -INFINITY, l = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int sp0 = grp; sp0 < n_splits; sp0 += kMergeGroups * kMergeBatch) {
-    float v[kMergeBatch];
-    float4 o[kMergeBatch];
+  for (int sp0 = grp; sp0 < n_splits; sp0 += kMergeGroups * kBatch) {
+    float v[kBatch];
+    float4 o[kBatch];
 #pragma unroll
-    for (int k = 0; k < kMergeBatch; ++k) {
+    for (int k = 0; k < kBatch; ++k) {
       const int sp = sp0 + k * kMergeGroups;
       v[k] = sp < n_splits ? pl[static_cast<long long>(sp) * rows_pad] : -INFINITY;
       o[k] = sp < n_splits ? *reinterpret_cast<const float4*>(po + static_cast<long long>(sp) * rows_pad * kHeadDim)
                            : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int k = 0; k < kMergeBatch; ++k) {
+    for (int k = 0; k < kBatch; ++k) {
       if (v[k] == -INFINITY) continue;  // a split that saw no key
       if (v[k] > m) {
         const float a = fast_exp2(m - v[k]);  // 0 when m = -inf
@@ -624,7 +626,7 @@ static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream
   cfg.gridDim = dim3(prm.group * prm.n_q, n_kv);
   cfg.blockDim = dim3(kMergeThreads);
   cfg.dynamicSmemBytes = 0;
-  return cudaLaunchKernelEx(&cfg, decode_merge_kernel, static_cast<const float*>(prm.part_o),
+  return cudaLaunchKernelEx(&cfg, decode_merge_kernel<16, 1>, static_cast<const float*>(prm.part_o),
                             static_cast<const float*>(prm.part_lse), prm.n_splits, C::kRowsPad, prm.group, prm.n_qh,
                             prm.out, prm.lse);
 }

@@ -769,7 +769,7 @@ cudaError_t launch_prefill(const PrefillParams& prm0, int n_kv, cudaStream_t str
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_merge_kernel, static_cast<const float*>(prm.part_o),
+  return cudaLaunchKernelEx(&cfg, decode_merge_kernel<8, 2>, static_cast<const float*>(prm.part_o),
                             static_cast<const float*>(prm.part_lse), prm.n_ks, prm.rows_pad, prm.group, prm.n_qh,
                             prm.out, prm.lse);
 }

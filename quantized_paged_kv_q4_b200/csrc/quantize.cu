@@ -51,6 +51,8 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
   // a kernel launched behind this one with programmatic dependent launch (decode) may start
   // its setup now; it waits for this grid to complete before reading the pages
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // this grid is itself launched that way: wait for the previous kernel before any read
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (row >= static_cast<long long>(n_tok) * n_kv) return;
@@ -59,6 +61,10 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
   const int32_t pos = pos0 + i;
   const int blk = pos / kPageTokens;
   const int tok = pos % kPageTokens;
+  // all global reads are issued before any of them is used
+  const float4* ksrc = reinterpret_cast<const float4*>(k + row * kHeadDim + lane * 8);
+  const float4* vsrc = reinterpret_cast<const float4*>(v + row * kHeadDim + lane * 8);
+  const float4 kx0 = ksrc[0], kx1 = ksrc[1], vx0 = vsrc[0], vx1 = vsrc[1];
   const int page = page_table[static_cast<long long>(h) * n_blocks + blk];
   if (page < 0 || page >= n_pages) {
     if (lane == 0) record_error(KVATTN_ERR_BAD_PAGE);
@@ -69,9 +75,7 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
 
   // ---------------- K: Q8_0 ----------------
   {
-    const float4* src = reinterpret_cast<const float4*>(k + row * kHeadDim + lane * 8);
-    const float4 x0 = src[0], x1 = src[1];
-    const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    const float x[8] = {kx0.x, kx0.y, kx0.z, kx0.w, kx1.x, kx1.y, kx1.z, kx1.w};
     float inv;
     const float d = q8_scale(x, &inv);
     uint32_t w0 = 0, w1 = 0;
@@ -91,9 +95,7 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
 
   // ---------------- V: Q4_0 or Q8_0 ----------------
   {
-    const float4* src = reinterpret_cast<const float4*>(v + row * kHeadDim + lane * 8);
-    const float4 x0 = src[0], x1 = src[1];
-    const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    const float x[8] = {vx0.x, vx0.y, vx0.z, vx0.w, vx1.x, vx1.y, vx1.z, vx1.w};
     uint8_t* pg = v_pool + static_cast<int64_t>(page) * v_stride;
     const int T = (tl & 7) >> 1, wlo = tl >> 3, ylo = tl & 1;
     const int k_slot = ylo + 2 * wlo;
@@ -163,11 +165,21 @@ cudaError_t launch_quantize_append(const kvattn_kv_desc& desc, const float* k, c
   const long long rows = static_cast<long long>(n_tok) * desc.n_kv_heads;
   const int warps_per_block = 8;
   const long long grid = (rows + warps_per_block - 1) / warps_per_block;
-  quantize_append_kernel<<<static_cast<unsigned>(grid), 32 * warps_per_block, 0, stream>>>(
-      k, v, n_tok, desc.n_kv_heads, pos0, page_table, n_blocks, static_cast<uint8_t*>(desc.k_pool),
-      desc.k_page_stride, static_cast<uint8_t*>(desc.v_pool), desc.v_page_stride, desc.n_pages,
-      desc.v_fmt == KVATTN_FMT_Q8_0);
-  return cudaGetLastError();
+  // programmatic dependent launch: the grid may start while the previous kernel finishes;
+  // it waits for it (griddepcontrol.wait) before reading anything
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(32 * warps_per_block);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_append_kernel, k, v, n_tok, desc.n_kv_heads, pos0, page_table, n_blocks,
+                            static_cast<uint8_t*>(desc.k_pool), desc.k_page_stride,
+                            static_cast<uint8_t*>(desc.v_pool), desc.v_page_stride, desc.n_pages,
+                            static_cast<int>(desc.v_fmt == KVATTN_FMT_Q8_0));
 }
 
 }  // namespace kvattn
