@@ -241,7 +241,7 @@ class DecodeBench:
         self.ws = torch.zeros((L, max(self.ws_bytes, 256)), dtype=torch.uint8, device=device)
         self.bytes_per_layer = self.ctx * H * BYTES_PER_TOKEN_HEAD[w.v_fmt]
         self.bytes_per_step = self.bytes_per_layer * L
-        self.launches_per_step = 2 * L
+        self.launches_per_step = 3 * L  # quantize-append, decode, split merge
 
     def layer(self, l, timed=None):
         kv, c = self.kv, self.cache
@@ -300,7 +300,7 @@ class VerifyBench:
         self.bytes_per_layer = tokens * H * BYTES_PER_TOKEN_HEAD[w.v_fmt]
         self.bytes_per_step = self.bytes_per_layer * L
         self.select_bytes_per_layer = H * (self.n_full - w.recent_blocks) * 256 * 4
-        self.launches_per_step = 4 * L
+        self.launches_per_step = 5 * L  # block scores, top-k, quantize-append, decode, split merge
 
     def layer(self, l, timed=None):
         kv, c, w = self.kv, self.cache, self.w

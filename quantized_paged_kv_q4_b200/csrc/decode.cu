@@ -36,7 +36,10 @@ struct DecodeCfg {
   static constexpr int kRowsPad = NT * 8;
   static constexpr int kXBytes = PAIR ? 4 * 2 * 2 * NT * 32 * 16 : 0;  // pair S exchange
   static constexpr int kRingBytes = kStages * kStageBytes;
-  static constexpr int kMergeBytes = kUnits * kRowsPad * (kHeadDim + 2) * 4;
+  // rows of the output merge buffer are padded by 4 floats: the four lanes of an MMA quad
+  // store rows 2t, 2t+1 of the same dims and then fall into different banks
+  static constexpr int kOStride = kHeadDim + 4;
+  static constexpr int kMergeBytes = kUnits * kRowsPad * (kOStride + 2) * 4;
   static_assert(kMergeBytes <= kRingBytes, "merge buffer must fit in the ring");
   static constexpr int kBarOffset = kRingBytes + kXBytes;
   static constexpr int kSmemBytes = kBarOffset + 256;
@@ -459,7 +462,7 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
   }
 
   // ---------------- merge the CTA's softmax streams in shared memory ----------------
-  // layout: ms[unit][row], ls[unit][row], os[unit][row][256]  (all fp32)
+  // layout: ms[unit][row], ls[unit][row], os[unit][row][kOStride]  (all fp32)
   float* ms = reinterpret_cast<float*>(smem);
   float* ls = ms + C::kUnits * C::kRowsPad;
   float* os = ls + C::kUnits * C::kRowsPad;
@@ -483,7 +486,7 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
         for (int e = 0; e < 4; ++e) {
           const int row = nt * 8 + 2 * t + (e & 1);
           const int dim = 32 * b + 16 * hb + g + 8 * (e >> 1);
-          os[(unit * C::kRowsPad + row) * kHeadDim + dim] = oacc[mt][nt][e];
+          os[(unit * C::kRowsPad + row) * C::kOStride + dim] = oacc[mt][nt][e];
         }
     }
   }
@@ -505,7 +508,7 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
       for (int u = 0; u < C::kUnits; ++u) {
         const float w = fast_exp2(ms[u * C::kRowsPad + row] - M);
         L += w * ls[u * C::kRowsPad + row];
-        const float4 o = *reinterpret_cast<const float4*>(os + (u * C::kRowsPad + row) * kHeadDim + d4);
+        const float4 o = *reinterpret_cast<const float4*>(os + (u * C::kRowsPad + row) * C::kOStride + d4);
         acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
       }
     }
