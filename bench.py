@@ -173,9 +173,15 @@ def max_over_ranks(x: float, world: int) -> float:
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_step_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job rate: the units all ranks processed / the slowest rank's time per step."""
+    return units_per_step_per_rank * world / (ms_max * 1e-3)
 
 
 # --------------------------------------------------------------------------- caches
@@ -790,7 +796,7 @@ def main():
     kern_ms = time_kernel(b, max(3, min(args.steps, 50)))
     e2e_ms, h2d, d2h = time_e2e(b, max(3, min(args.steps, 200)), 3)
     assert kvattn.kvattn_device_error() == 0
-    value = b.bytes_per_step * world / (ms * 1e-3) / 1e9
+    value = job_throughput(b.bytes_per_step, world, ms) / 1e9
     achieved = b.bytes_per_layer / (kern_ms * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
