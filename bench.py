@@ -222,7 +222,40 @@ def event_pair():
 
 
 # --------------------------------------------------------------------------- decode workloads
-class DecodeBench:
+class GraphStep:
+    """One step's launches through the C ABI, optionally captured once as a CUDA graph and
+    replayed: the same kernels on the same buffers, without the host's per-launch cost (a
+    decode step is ~50 launches of ~50 us each)."""
+
+    graph = None
+
+    def launch_step(self):
+        for l in range(self.w.layers):
+            self.layer(l)
+
+    def capture(self):
+        import torch
+
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.launch_step()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.launch_step()
+        torch.cuda.synchronize()
+        self.graph = g
+
+    def step(self):
+        if self.graph is not None:
+            self.graph.replay()
+        else:
+            self.launch_step()
+
+
+class DecodeBench(GraphStep):
     def __init__(self, kv, wname, device, layers=0):
         import dataclasses
 
@@ -259,12 +292,8 @@ class DecodeBench:
         if timed is not None:
             timed[1].record()
 
-    def step(self):
-        for l in range(self.w.layers):
-            self.layer(l)
 
-
-class VerifyBench:
+class VerifyBench(GraphStep):
     """MTP verify at 262,144 context: per layer, select 256 + 128 recent blocks (+ the tail
     page) with the block summaries, append the 4 verify tokens, decode n_q = 4 over the
     selected pages."""
@@ -320,10 +349,6 @@ class VerifyBench:
                          self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
         if timed is not None:
             timed[1].record()
-
-    def step(self):
-        for l in range(self.w.layers):
-            self.layer(l)
 
 
 class PrefillBench:
@@ -642,7 +667,7 @@ def time_e2e(bench, steps, warmup):
         bench.q.copy_(hq, non_blocking=True)
         bench.k_new.copy_(hk, non_blocking=True)
         bench.v_new.copy_(hv, non_blocking=True)
-        bench.step()
+        bench.launch_step()  # the C-ABI calls themselves, no graph
         ho.copy_(bench.out, non_blocking=True)
         hl.copy_(bench.lse, non_blocking=True)
 
@@ -789,6 +814,11 @@ def main():
 
     # ---------------- headline: decode at 131K ----------------
     b = DecodeBench(kvattn, "decode131k", device, layers=args.layers)
+    launch_mode = "one CUDA graph per step (3 launches per layer, programmatic dependent launch)"
+    try:
+        b.capture()
+    except Exception as exc:  # report and time the direct launches instead
+        launch_mode = f"direct launches (graph capture failed: {exc!r})"
     clocks = ClockSampler(local)
     clocks.start()
     ms = time_steps(b, args.steps, args.warmup, world)
@@ -805,7 +835,8 @@ def main():
         "config": {"workload": "decode131k", "layers": b.w.layers, "kv_heads": b.w.kv_heads,
                    "q_heads": b.w.q_heads, "context": b.ctx, "n_q": 1, "k_fmt": "q8_0", "v_fmt": "q4_0",
                    "outliers": "1% of channels x8", "parallelism": f"{world} independent decodes (one per GPU)",
-                   "l2": "inputs larger than L2 (218 MB of KV per layer launch, 3.49 GB per step)"},
+                   "l2": "inputs larger than L2 (218 MB of KV per layer launch, 3.49 GB per step)",
+                   "launch": launch_mode},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": profiled_traffic("decode_kernel_decode131k.md"), "kernel": "decode_kernel<1,false,false>",
                      "peak_kind": f"{peak_kind} copy bandwidth (hbm_gbs)",
@@ -825,6 +856,7 @@ def main():
     if not args.no_extra:
         try:
             b2 = DecodeBench(kvattn, "decode131k_q8q8", device)
+            b2.capture()
             ms2 = time_steps(b2, args.extra_steps, 5, world)
             k2 = time_kernel(b2, 10)
             extra["decode131k_q8q8"] = {"GB/s": b2.bytes_per_step / (ms2 * 1e-3) / 1e9, "ms_per_step": ms2,
@@ -833,6 +865,7 @@ def main():
             del b2
             torch.cuda.empty_cache()
             b3 = VerifyBench(kvattn, device)
+            b3.capture()
             ms3 = time_steps(b3, args.extra_steps, 5, world)
             k3 = time_kernel(b3, 10)
             extra["verify262k"] = {"GB/s": b3.bytes_per_step / (ms3 * 1e-3) / 1e9, "ms_per_step": ms3,

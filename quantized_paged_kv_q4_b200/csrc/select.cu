@@ -93,6 +93,40 @@ constexpr int kSelThreads = 1024;
 constexpr int kMaxCand = 16384;
 constexpr int kMaxTotal = 65536;
 
+// Exclusive prefix sum of one int per thread over the CTA (kSelThreads threads); `warp_tot`
+// is shared scratch of kSelThreads / 32 ints.  Returns this thread's exclusive prefix and
+// writes the CTA total to *total (shared).
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int t = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    warp_tot[lane] = t;  // inclusive over warps
+    if (lane == 31) *total = t;
+  }
+  __syncthreads();
+  const int r = x - v + (warp > 0 ? warp_tot[warp - 1] : 0);
+  __syncthreads();  // warp_tot may be reused by the caller
+  return r;
+}
+
+// Top-`budget` candidates by (score desc, block index asc), plus the recent window and the
+// tail, compacted into ascending logical ids.  The `take`-th largest 64-bit order key is found
+// by an 8-bit radix select (eight histogram passes); candidates above it are taken, and those
+// equal to it are taken in index order until `take` are chosen, which is exactly the first
+// `take` of a sort by (score desc, index asc).
 __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const double* __restrict__ scores, int n_blocks,
                                                                  int n_cand, int n_total, int budget,
                                                                  const int32_t* __restrict__ page_table,
@@ -100,71 +134,96 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const double* 
                                                                  int32_t* __restrict__ sel_phys,
                                                                  int32_t* __restrict__ n_sel, int cap) {
   extern __shared__ __align__(16) uint8_t sm[];
+  __shared__ int hist[256];
+  __shared__ int warp_tot[kSelThreads / 32];
+  __shared__ int s_total, s_digit, s_need;
   const int unit = blockIdx.x;
-  int npad = 1;
-  while (npad < n_cand) npad <<= 1;
-  unsigned long long* key = reinterpret_cast<unsigned long long*>(sm);
-  int* idx = reinterpret_cast<int*>(key + npad);
-  int* counts = idx + npad;                                   // [kSelThreads + 1]
-  uint32_t* bits = reinterpret_cast<uint32_t*>(counts + kSelThreads + 1);  // [n_total / 32]
+  unsigned long long* key = reinterpret_cast<unsigned long long*>(sm);           // [n_cand]
+  uint32_t* bits = reinterpret_cast<uint32_t*>(key + (n_cand > 0 ? n_cand : 1));  // [n_total / 32]
   const double* sc = scores + static_cast<long long>(unit) * n_blocks;
-  for (int i = threadIdx.x; i < npad; i += kSelThreads) {
-    if (i < n_cand) {
-      key[i] = order_key(sc[i]);
-      idx[i] = i;
-    } else {
-      key[i] = 0ull;
-      idx[i] = INT_MAX;
-    }
-  }
+  for (int i = threadIdx.x; i < n_cand; i += kSelThreads) key[i] = order_key(sc[i]);
+  const int take = min(budget, n_cand);
+  unsigned long long prefix = 0ull, mask = 0ull;
+  int need = take;  // how many still to take among keys matching prefix under mask
   __syncthreads();
-  // bitonic sort: descending key, ascending index
-  for (int k = 2; k <= npad; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < npad; i += kSelThreads) {
-        const int l = i ^ j;
-        if (l > i) {
-          const unsigned long long ki = key[i], kl = key[l];
-          const int ii = idx[i], il = idx[l];
-          const bool i_first = ki > kl || (ki == kl && ii < il);  // i precedes l in the target order
-          const bool up = (i & k) == 0;
-          if (up != i_first) {
-            key[i] = kl; key[l] = ki;
-            idx[i] = il; idx[l] = ii;
+  if (take > 0 && take < n_cand) {
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      for (int b = threadIdx.x; b < 256; b += kSelThreads) hist[b] = 0;
+      __syncthreads();
+      for (int i = threadIdx.x; i < n_cand; i += kSelThreads) {
+        const unsigned long long k = key[i];
+        if ((k & mask) == prefix) atomicAdd(&hist[static_cast<int>((k >> shift) & 255ull)], 1);
+      }
+      __syncthreads();
+      if (threadIdx.x < 32) {
+        // lane l owns bins 255 - 8l - e (e = 0..7), highest first; find the digit whose bin
+        // holds the need-th largest remaining key
+        const int lane = threadIdx.x;
+        int c[8], sum = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          c[e] = hist[255 - 8 * lane - e];
+          sum += c[e];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        int before = incl - sum;  // keys in higher bins than this lane's
+        if (before < need && need <= incl) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (before < need && need <= before + c[e]) {
+              s_digit = 255 - 8 * lane - e;
+              s_need = need - before;
+            }
+            before += c[e];
           }
         }
       }
       __syncthreads();
+      prefix |= static_cast<unsigned long long>(s_digit) << shift;
+      mask |= 255ull << shift;
+      need = s_need;
+      __syncthreads();
     }
   }
-  // mark the chosen candidates in a bitmap over [0, n_total)
-  const int take = min(budget, n_cand);
-  const int* chosen = idx;
+  // mark: keys above the threshold, and the first `need` keys equal to it in index order
+  // (contiguous index ranges per thread, ranks of equal keys by a block scan)
   const int words = (n_total + 31) / 32;
   for (int w = threadIdx.x; w < words; w += kSelThreads) bits[w] = 0u;
   __syncthreads();
-  for (int i = threadIdx.x; i < take; i += kSelThreads) atomicOr(&bits[chosen[i] >> 5], 1u << (chosen[i] & 31));
+  {
+    const int per = (n_cand + kSelThreads - 1) / kSelThreads;
+    const int i0 = min(n_cand, threadIdx.x * per), i1 = min(n_cand, i0 + per);
+    int eq = 0;
+    if (take > 0 && take < n_cand)
+      for (int i = i0; i < i1; ++i) eq += key[i] == prefix;
+    int rank = block_exclusive_scan(eq, warp_tot, &s_total);
+    for (int i = i0; i < i1; ++i) {
+      bool sel;
+      if (take >= n_cand) {
+        sel = true;
+      } else if (take <= 0) {
+        sel = false;
+      } else {
+        const unsigned long long k = key[i];
+        sel = k > prefix || (k == prefix && rank++ < need);
+      }
+      if (sel) atomicOr(&bits[i >> 5], 1u << (i & 31));
+    }
+  }
   for (int b = n_cand + threadIdx.x; b < n_total; b += kSelThreads) atomicOr(&bits[b >> 5], 1u << (b & 31));
   __syncthreads();
-  // each thread owns a contiguous range of words; exclusive scan of their popcounts
+  // compaction into ascending ids
   const int per = (words + kSelThreads - 1) / kSelThreads;
-  const int w0 = threadIdx.x * per, w1 = min(words, w0 + per);
+  const int w0 = min(words, threadIdx.x * per), w1 = min(words, w0 + per);
   int cnt = 0;
   for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
-  counts[threadIdx.x] = cnt;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int i = 0; i < kSelThreads; ++i) {
-      const int c = counts[i];
-      counts[i] = run;
-      run += c;
-    }
-    counts[kSelThreads] = run;
-  }
-  __syncthreads();
-  int pos = counts[threadIdx.x];
-  const int total = counts[kSelThreads];
+  int pos = block_exclusive_scan(cnt, warp_tot, &s_total);
+  const int total = s_total;
   int32_t* out_l = sel_logical + static_cast<long long>(unit) * cap;
   int32_t* out_p = sel_phys + static_cast<long long>(unit) * cap;
   const int32_t* pt = page_table + static_cast<long long>(unit) * n_blocks;
@@ -195,9 +254,7 @@ cudaError_t launch_block_summaries(const kvattn_kv_desc& d, const int32_t* page_
 }
 
 size_t select_smem_bytes(int n_cand, int n_total) {
-  int npad = 1;
-  while (npad < n_cand) npad <<= 1;
-  return static_cast<size_t>(npad) * 12 + (kSelThreads + 1) * 4 + static_cast<size_t>((n_total + 31) / 32) * 4;
+  return static_cast<size_t>(n_cand > 0 ? n_cand : 1) * 8 + static_cast<size_t>((n_total + 31) / 32) * 4;
 }
 
 cudaError_t prepare_select_kernels() {
