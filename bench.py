@@ -565,6 +565,87 @@ class StreamBench:
             self._gather(l, cs)
 
 
+class ResidentStreamBench(StreamBench):
+    """The streamed step with resident-page reuse: every (layer, KV head) keeps a pool of 256
+    device slots across steps; per layer, kvattn_resident_update maps the new selection onto
+    the pool and only the misses cross PCIe (layer L+1's on the side stream while layer L
+    decodes).  `queries` per-step retrieval queries are cycled: 1 = the per-turn query KVMem
+    uses (the working set is fixed during a turn), more = a drifting query."""
+
+    def __init__(self, kv, device, queries=1, drift=0.0, layers=0, context=0):
+        import torch
+
+        super().__init__(kv, device, layers=layers, context=context)
+        w, L, H = self.w, self.w.layers, self.w.kv_heads
+        self.units = L * H
+        self.n_res = self.units * self.budget                 # resident pool pages, then the tails
+        P = self.PAGE
+        self.slots = torch.zeros((self.n_res + self.units, P), dtype=torch.uint8, device=device)
+        for l in range(L):
+            for h in range(H):
+                self.slots[self.n_res + l * H + h].copy_(self.host[(l * H + h) * self.nb + self.n_full])
+        self.n_slots = self.slots.shape[0]
+        self.desc = kv.make_desc(H, w.q_heads, self.slots, self.slots.data_ptr() + 34816, self.n_slots,
+                                 k_page_stride=P, v_page_stride=P)
+        self.tail_slot = torch.tensor([[self.n_res + l * H + h for h in range(H)] for l in range(L)],
+                                      dtype=torch.int32, device=device)
+        self.tail_tab = self.tail_slot[:, :, None].expand(L, H, self.nb).contiguous()
+        self.sob = torch.full((self.units, self.nb), -1, dtype=torch.int32, device=device)
+        self.bos = torch.full((self.units, self.budget), -1, dtype=torch.int32, device=device)
+        self.plist_r = torch.zeros((L, H, self.cap), dtype=torch.int32, device=device)
+        self.copy_host = torch.zeros((L, H, self.cap), dtype=torch.int32, device=device)
+        self.copy_dst = torch.full((L, H, self.cap), -1, dtype=torch.int32, device=device)
+        self.n_copies = torch.zeros((L, H), dtype=torch.int32, device=device)
+        # per-step retrieval queries: q_0 = the workload's, q_t = q_{t-1} + drift * N(0, 1)
+        qs = [self.q]
+        for t in range(1, queries):
+            qs.append(qs[-1] + drift * torch_normal(derived_seed(w.seed, 30, t), tuple(self.q.shape), device))
+        self.qs = [q.contiguous() for q in qs]
+        self.qgs = [q[:, 0].reshape(L, H, w.group, 256).contiguous() for q in qs]
+        self.t = 0
+
+    def _select(self, l):
+        w, H = self.w, self.w.kv_heads
+        qg = self.qgs[self.t % len(self.qgs)]
+        self.kv.kvattn_select_blocks(self.summ[l * H:(l + 1) * H], qg[l], H, w.group, self.nb, self.n_full, self.nb,
+                                     self.budget, 0, self.host_table[l], self.sel_l[l], self.sel_p[l], self.n_sel[l],
+                                     self.cap, self.sws[l], self.sws_bytes)
+        self.kv.kvattn_resident_update(self.sel_l[l], self.n_sel[l], self.cap, H, self.nb, self.n_full,
+                                       self.sob[l * H:(l + 1) * H], self.bos[l * H:(l + 1) * H], self.budget,
+                                       self.host_table[l], l * H * self.budget, self.tail_slot[l], self.plist_r[l],
+                                       self.copy_host[l], self.copy_dst[l], self.n_copies[l])
+
+    def _gather(self, l, stream):
+        H = self.w.kv_heads
+        self.kv.kvattn_gather_pages(self.host, self.PAGE, self.host.shape[0], self.slots, self.PAGE, self.n_slots,
+                                    self.PAGE, self.copy_host[l], self.copy_dst[l], H * self.cap, self.gather_ctas,
+                                    stream)
+
+    def _attend(self, l, timed=None):
+        kv, w = self.kv, self.w
+        q = self.qs[self.t % len(self.qs)]
+        kv.kvattn_quantize_append(self.desc, self.k_new[l], self.v_new[l], 1, self.pos, self.tail_tab[l], self.nb)
+        kv.kvattn_decode(self.desc, q[l], 1, self.q_pos, self.plist_r[l], self.sel_l[l], self.n_sel[l], self.cap,
+                         self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
+        kv.kvattn_scatter_pages(self.host, self.PAGE, self.host.shape[0], self.slots, self.PAGE, self.n_slots,
+                                self.PAGE, self.tail_host[l], self.tail_slot[l], w.kv_heads, 4)
+
+    def step(self, stream_pages=True, timed=None):
+        super().step(stream_pages, timed)
+        self.t += 1
+
+    def copies_per_step(self, steps):
+        """Pages copied per step over `steps` steps (read back after each; untimed)."""
+        import torch
+
+        n = []
+        for _ in range(steps):
+            self.step()
+            torch.cuda.synchronize()
+            n.append(int(self.n_copies.sum()))
+        return n
+
+
 def time_stream(b, steps, warmup):
     """T_stream (pipelined), T_resident (no page copies), T_copy (copies alone), decode time."""
     import torch
@@ -898,6 +979,19 @@ def main():
                 "host_pool_GB": b5.host.numel() / 1e9}
             del b5
             torch.cuda.empty_cache()
+            res = {}
+            for name, nq, drift in (("per_turn_query", 1, 0.0), ("drifting_query", 16, 0.05)):
+                b6 = ResidentStreamBench(kvattn, device, queries=nq, drift=drift)
+                first = b6.copies_per_step(1)[0]          # the cold step copies the whole working set
+                warm = b6.copies_per_step(max(2 * nq, 4))
+                full = b6.w.layers * b6.w.kv_heads * b6.budget
+                ms6 = time_steps(b6, max(8, args.extra_steps // 5), 2, world)
+                res[name] = {"ms_per_step": ms6, "pages_copied_first_step": first,
+                             "pages_copied_per_step": statistics.mean(warm), "hit_rate": 1.0 - statistics.mean(warm) / full,
+                             "queries_cycled": nq, "drift": drift}
+                del b6
+                torch.cuda.empty_cache()
+            extra["stream524k"]["resident_reuse"] = res
         except Exception as exc:  # report, do not hide
             extra["error"] = repr(exc)
         assert kvattn.kvattn_device_error() == 0

@@ -275,6 +275,37 @@ KVATTN_API int kvattn_scatter_pages(void* host_pool, int64_t host_stride, int64_
                                     int64_t dev_stride, int64_t n_slots, int64_t page_bytes, const int32_t* host_ids,
                                     const int32_t* dev_slots, int n, int n_ctas, kvattn_stream_t stream);
 
+/* ---- resident-page reuse ([KVMEM] recall section: the GPU working set follows the
+ * retrieval query; a block already on the GPU is not copied again) ---------------------
+ * Per unit (layer, KV head) a pool of n_slots device pages, pool page first_page + unit *
+ * n_slots + s for slot s.  For the selection of each unit (sel_logical, ascending and unique,
+ * as kvattn_select_blocks writes it):
+ *   - a selected block that is resident keeps its slot;
+ *   - free slots are the empty ones and those holding a block that is not selected;
+ *   - misses (selected, not resident), in ascending block order, take the free slots in
+ *     ascending slot order; blocks evicted this way are no longer resident.
+ * Blocks >= n_full (the tail page) are not managed; their page-list entry is
+ * extra_page[unit].
+ *   sel_logical   device int32 [n_units][cap];  n_sel device int32 [n_units]
+ *   slot_of_block device int32 [n_units][n_blocks], -1 = not resident (state; the caller
+ *                 fills it with -1 once and then only passes it back)
+ *   block_of_slot device int32 [n_units][n_slots], -1 = empty (state, likewise)
+ *   host_page_of_block device int32 [n_units][n_blocks]: host page id of each block
+ *   page_list     device int32 [n_units][cap] out: pool page holding each selected block
+ *                 (a kvattn_decode page list, with sel_logical as its page_logical)
+ *   copy_host, copy_dst device int32 [n_units][cap] out: host page and pool page of every
+ *                 miss, copy_dst = -1 past n_copies[unit] (ready for kvattn_gather_pages
+ *                 with n = n_units * cap)
+ *   n_copies      device int32 [n_units] out
+ * n_slots must be >= the number of managed selected blocks; otherwise the unit is left
+ * unchanged, n_copies = 0 and KVATTN_ERR_INVALID_ARG is set in the device error word.
+ * Limits: n_blocks <= 262,144, n_slots <= 16,384.  Asynchronous on `stream`. */
+KVATTN_API int kvattn_resident_update(const int32_t* sel_logical, const int32_t* n_sel, int cap, int n_units,
+                                      int n_blocks, int n_full, int32_t* slot_of_block, int32_t* block_of_slot,
+                                      int n_slots, const int32_t* host_page_of_block, int64_t first_page,
+                                      const int32_t* extra_page, int32_t* page_list, int32_t* copy_host,
+                                      int32_t* copy_dst, int32_t* n_copies, kvattn_stream_t stream);
+
 /* Polls `event` until it completes or timeout_ms elapses (KVATTN_ERR_TIMEOUT). */
 KVATTN_API int kvattn_stream_wait(kvattn_event_t event, int timeout_ms);
 

@@ -11,6 +11,10 @@ namespace kvattn {
 cudaError_t launch_quantize_append(const kvattn_kv_desc&, const float*, const float*, int, int32_t, const int32_t*,
                                    int, cudaStream_t);
 cudaError_t prepare_select_kernels();
+cudaError_t prepare_resident_kernels();
+cudaError_t launch_resident_update(const int32_t*, const int32_t*, int, int, int, int, int32_t*, int32_t*, int,
+                                   const int32_t*, int64_t, const int32_t*, int32_t*, int32_t*, int32_t*, int32_t*,
+                                   cudaStream_t);
 cudaError_t prepare_prefill_kernels();
 struct PrefillParams;
 cudaError_t launch_merge_lse(const float*, const float*, int, int, int, float*, float*, int, cudaStream_t);
@@ -114,6 +118,7 @@ KVATTN_API int kvattn_init(int device) {
   if ((e = prepare_decode_kernels()) != cudaSuccess) return cuda_fail(e);
   if ((e = prepare_select_kernels()) != cudaSuccess) return cuda_fail(e);
   if ((e = prepare_prefill_kernels()) != cudaSuccess) return cuda_fail(e);
+  if ((e = prepare_resident_kernels()) != cudaSuccess) return cuda_fail(e);
   g_sm_count[device] = prop.multiProcessorCount;
   g_inited[device] = true;
   return KVATTN_OK;
@@ -389,6 +394,27 @@ KVATTN_API int kvattn_scatter_pages(void* host_pool, int64_t host_stride, int64_
                                     const int32_t* dev_slots, int n, int n_ctas, kvattn_stream_t stream) {
   return page_copy_common(host_pool, host_stride, n_host_pages, const_cast<void*>(dev_pool), dev_stride, n_slots,
                           page_bytes, host_ids, dev_slots, n, n_ctas, 0, stream);
+}
+
+KVATTN_API int kvattn_resident_update(const int32_t* sel_logical, const int32_t* n_sel, int cap, int n_units,
+                                      int n_blocks, int n_full, int32_t* slot_of_block, int32_t* block_of_slot,
+                                      int n_slots, const int32_t* host_page_of_block, int64_t first_page,
+                                      const int32_t* extra_page, int32_t* page_list, int32_t* copy_host,
+                                      int32_t* copy_dst, int32_t* n_copies, kvattn_stream_t stream) {
+  if (!sel_logical || !n_sel || !slot_of_block || !block_of_slot || !host_page_of_block || !extra_page ||
+      !page_list || !copy_host || !copy_dst || !n_copies)
+    return KVATTN_ERR_INVALID_ARG;
+  if (cap < 1 || n_units < 1 || n_units > 65535 || n_blocks < 1 || n_blocks > 262144 || n_full < 0 ||
+      n_full > n_blocks || n_slots < 1 || n_slots > 16384 || first_page < 0 ||
+      first_page + static_cast<int64_t>(n_units) * n_slots > INT32_MAX)
+    return KVATTN_ERR_INVALID_ARG;
+  int dev;
+  int st = current_device_checked(&dev);
+  if (st) return st;
+  cudaError_t e = launch_resident_update(sel_logical, n_sel, cap, n_units, n_blocks, n_full, slot_of_block,
+                                         block_of_slot, n_slots, host_page_of_block, first_page, extra_page,
+                                         page_list, copy_host, copy_dst, n_copies, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVATTN_OK : cuda_fail(e);
 }
 
 KVATTN_API int kvattn_stream_wait(kvattn_event_t event, int timeout_ms) {

@@ -77,6 +77,9 @@ _SIGS = {
                                      c_void_p, c_int, c_int, c_void_p]),
     "kvattn_stream_plan": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int]),
     "kvattn_stream_wait": (c_int, [c_void_p, c_int]),
+    "kvattn_resident_update": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_int,
+                                       c_void_p, c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_void_p]),
 }
 
 _lib = None
@@ -225,6 +228,18 @@ def kvattn_scatter_pages(host_pool, host_stride, n_host_pages, dev_pool, dev_str
     _check(lib().kvattn_scatter_pages(_p(host_pool), host_stride, n_host_pages, _p(dev_pool), dev_stride, n_slots,
                                       page_bytes, _p(host_ids), _p(dev_slots), n, n_ctas, _s(stream)),
            "kvattn_scatter_pages")
+
+
+def kvattn_resident_update(sel_logical, n_sel, cap, n_units, n_blocks, n_full, slot_of_block, block_of_slot,
+                           n_slots, host_page_of_block, first_page, extra_page, page_list, copy_host, copy_dst,
+                           n_copies, stream=None) -> None:
+    """Resident-page reuse: update each unit's slot pool for its new selection and write the
+    decode page list and the copy list of the misses (all device arrays)."""
+    _check(lib().kvattn_resident_update(_p(sel_logical), _p(n_sel), cap, n_units, n_blocks, n_full,
+                                        _p(slot_of_block), _p(block_of_slot), n_slots, _p(host_page_of_block),
+                                        first_page, _p(extra_page), _p(page_list), _p(copy_host), _p(copy_dst),
+                                        _p(n_copies), _s(stream)),
+           "kvattn_resident_update")
 
 
 def _host_i32(a):

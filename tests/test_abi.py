@@ -116,3 +116,23 @@ def test_stream_plan_coalesces_runs(lib):
     assert kvattn.kvattn_stream_plan(host, dev) == [(0, 3), (3, 2), (5, 2), (7, 1)]
     with pytest.raises(kvattn.KVAttnError):
         kvattn.kvattn_stream_pages(16, 64, 16, 64, 64, [1, -1], [0, 1], copy_stream=0)
+
+
+def test_resident_update_validation(lib):
+    f = kvattn.lib().kvattn_resident_update
+    one = 16  # any non-null address: validation fails before anything is read
+    args = [one, one, 8, 2, 100, 90, one, one, 16, one, 0, one, one, one, one, one, None]
+    bad = [
+        (2, 0),        # cap
+        (3, 0),        # n_units
+        (4, 0),        # n_blocks
+        (5, 101),      # n_full > n_blocks
+        (8, 0),        # n_slots
+        (8, 16385),    # n_slots over the limit
+        (10, -1),      # first_page
+        (0, None),     # null selection
+    ]
+    for i, v in bad:
+        a = list(args)
+        a[i] = v
+        assert f(*a) == kvattn.ERR_INVALID_ARG
