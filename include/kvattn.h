@@ -275,6 +275,17 @@ KVATTN_API int kvattn_scatter_pages(void* host_pool, int64_t host_stride, int64_
                                     int64_t dev_stride, int64_t n_slots, int64_t page_bytes, const int32_t* host_ids,
                                     const int32_t* dev_slots, int n, int n_ctas, kvattn_stream_t stream);
 
+/* ---- attention rotation (Vulkan/ROCm long-context report, section on attention
+ * rotation: the rotation improves the precision of quantized KV) --------------------------
+ * out[r] = in[r] R for `rows` rows of 256 fp32 values, R = H_256 / 16 with H the
+ * Sylvester-Hadamard matrix (H[i][j] = (-1)^popcount(i & j)).  R is symmetric, orthonormal
+ * and its own inverse.  The rotated pipeline: rotate K and V before kvattn_quantize_append,
+ * rotate Q before kvattn_decode / kvattn_prefill_chunk (scores are unchanged in exact
+ * arithmetic), rotate the output back with the same call; outlier channels are spread across
+ * the block before quantization.  in == out is allowed; both 16-byte aligned.  fp32
+ * butterflies: each output is within ~8 ulp-scale roundings of the exact product. */
+KVATTN_API int kvattn_hadamard(const float* in, float* out, int64_t rows, kvattn_stream_t stream);
+
 /* ---- resident-page reuse ([KVMEM] recall section: the GPU working set follows the
  * retrieval query; a block already on the GPU is not copied again) ---------------------
  * Per unit (layer, KV head) a pool of n_slots device pages, pool page first_page + unit *

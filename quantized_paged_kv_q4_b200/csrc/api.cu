@@ -12,6 +12,7 @@ cudaError_t launch_quantize_append(const kvattn_kv_desc&, const float*, const fl
                                    int, cudaStream_t);
 cudaError_t prepare_select_kernels();
 cudaError_t prepare_resident_kernels();
+cudaError_t launch_hadamard(const float*, float*, long long, cudaStream_t);
 cudaError_t launch_resident_update(const int32_t*, const int32_t*, int, int, int, int, int32_t*, int32_t*, int,
                                    const int32_t*, int64_t, const int32_t*, int32_t*, int32_t*, int32_t*, int32_t*,
                                    cudaStream_t);
@@ -394,6 +395,16 @@ KVATTN_API int kvattn_scatter_pages(void* host_pool, int64_t host_stride, int64_
                                     const int32_t* dev_slots, int n, int n_ctas, kvattn_stream_t stream) {
   return page_copy_common(host_pool, host_stride, n_host_pages, const_cast<void*>(dev_pool), dev_stride, n_slots,
                           page_bytes, host_ids, dev_slots, n, n_ctas, 0, stream);
+}
+
+KVATTN_API int kvattn_hadamard(const float* in, float* out, int64_t rows, kvattn_stream_t stream) {
+  if (rows < 0 || (rows > 0 && (!in || !out)) || rows > (1ll << 40)) return KVATTN_ERR_INVALID_ARG;
+  if (rows > 0 && (!aligned16(in) || !aligned16(out))) return KVATTN_ERR_INVALID_ARG;
+  int dev;
+  int st = current_device_checked(&dev);
+  if (st) return st;
+  cudaError_t e = launch_hadamard(in, out, rows, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVATTN_OK : cuda_fail(e);
 }
 
 KVATTN_API int kvattn_resident_update(const int32_t* sel_logical, const int32_t* n_sel, int cap, int n_units,

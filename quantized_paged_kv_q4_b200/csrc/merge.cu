@@ -73,3 +73,50 @@ cudaError_t launch_merge_lse(const float* o_parts, const float* lse_parts, int n
 }
 
 }  // namespace kvattn
+
+namespace kvattn {
+
+// x R for rows of 256 fp32 values, R = H_256 / 16 with H the Sylvester-Hadamard matrix
+// (symmetric, orthonormal, its own inverse): the attention rotation of the Vulkan/ROCm
+// long-context report (section on attention rotation), which spreads outlier channels
+// before quantization.  One warp per row; lane l holds elements 8l .. 8l + 7: the three low
+// index bits are butterflied in registers, the five high ones across lanes by shuffles.
+// `in` may equal `out`.
+__global__ void __launch_bounds__(256) hadamard_kernel(const float* __restrict__ in, float* __restrict__ out,
+                                                       long long rows) {
+  const int lane = threadIdx.x & 31;
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const float4* src = reinterpret_cast<const float4*>(in + row * kHeadDim + lane * 8);
+  const float4 a = src[0], b = src[1];
+  float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int m = 1; m < 8; m <<= 1)
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (!(e & m)) {
+        const float u = x[e], w = x[e | m];
+        x[e] = u + w;
+        x[e | m] = u - w;
+      }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = lane & m;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float y = __shfl_xor_sync(0xffffffffu, x[e], m);
+      x[e] = upper ? y - x[e] : x[e] + y;
+    }
+  }
+  float4* dst = reinterpret_cast<float4*>(out + row * kHeadDim + lane * 8);
+  dst[0] = make_float4(x[0] * 0.0625f, x[1] * 0.0625f, x[2] * 0.0625f, x[3] * 0.0625f);
+  dst[1] = make_float4(x[4] * 0.0625f, x[5] * 0.0625f, x[6] * 0.0625f, x[7] * 0.0625f);
+}
+
+cudaError_t launch_hadamard(const float* in, float* out, long long rows, cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  hadamard_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(in, out, rows);
+  return cudaGetLastError();
+}
+
+}  // namespace kvattn

@@ -77,6 +77,7 @@ _SIGS = {
                                      c_void_p, c_int, c_int, c_void_p]),
     "kvattn_stream_plan": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int]),
     "kvattn_stream_wait": (c_int, [c_void_p, c_int]),
+    "kvattn_hadamard": (c_int, [c_void_p, c_void_p, c_int64, c_void_p]),
     "kvattn_resident_update": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_int,
                                        c_void_p, c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                        c_void_p]),
@@ -228,6 +229,14 @@ def kvattn_scatter_pages(host_pool, host_stride, n_host_pages, dev_pool, dev_str
     _check(lib().kvattn_scatter_pages(_p(host_pool), host_stride, n_host_pages, _p(dev_pool), dev_stride, n_slots,
                                       page_bytes, _p(host_ids), _p(dev_slots), n, n_ctas, _s(stream)),
            "kvattn_scatter_pages")
+
+
+def kvattn_hadamard(x, out=None, rows=None, stream=None):
+    """out = x R over rows of 256 fp32 values (R = H_256 / 16); in place when out is None."""
+    out = x if out is None else out
+    n = rows if rows is not None else x.numel() // 256
+    _check(lib().kvattn_hadamard(_p(x), _p(out), n, _s(stream)), "kvattn_hadamard")
+    return out
 
 
 def kvattn_resident_update(sel_logical, n_sel, cap, n_units, n_blocks, n_full, slot_of_block, block_of_slot,
