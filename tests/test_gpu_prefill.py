@@ -126,3 +126,15 @@ def test_prefill_bad_page_id_is_skipped_and_reported(kv_gpu):
     keys = keys[(keys < 3 * 128) | (keys >= 4 * 128)]
     o_ref, l_ref = OracleCache(k, v, "q4_0").attend(q, q_pos, 0, 6, key_idx=keys)
     compare(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref)
+
+
+def test_prefill_empty_page_list_for_one_head(kv_gpu):
+    """Head 0 lists no page: its rows see no key (o = 0, lse = -inf); head 1 is unaffected."""
+    H, n_prior, n_q = 2, 600, 20
+    rng, k, v, q, cache, T = _case(1600, H, n_prior, n_q, outliers=False)
+    q_pos = np.arange(n_prior, T)
+    nb = cache.n_blocks
+    out, lse = _prefill(kv_gpu, cache, 6 * H, q, q_pos, cache.page_table_np, 256, None, [0, nb], nb)
+    assert np.all(out[:, :6] == 0) and np.all(np.isneginf(lse[:, :6]))
+    o_ref, l_ref = OracleCache(k, v, "q4_0").attend(q, q_pos, 1, 6)
+    compare(out[:, 6:], lse[:, 6:], o_ref, l_ref)
