@@ -1,4 +1,4 @@
-"""CPU oracle for quantized paged-KV attention (Q8_0 keys, Q4_0 or Q8_0 values).
+"""CPU oracle for quantized paged-KV attention (Q8_0 or Q4_0 keys, Q4_0 or Q8_0 values).
 
 TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import anything

@@ -5,7 +5,7 @@ A page holds the K (or V) rows of 128 consecutive tokens of one (layer, KV head)
 pages fix only the bits per element; the arrangement below is this library's own
 storage spec, written so that one 16-byte load per thread feeds tensor-core
 fragments directly.  Bytes per page equal the AoS block sizes the pages print:
-K Q8_0 = 128 x 8 x 34 = 34,816; V Q4_0 = 128 x 8 x 18 = 18,432; V Q8_0 = 34,816.
+K Q8_0 = 128 x 8 x 34 = 34,816; K Q4_0 = V Q4_0 = 128 x 8 x 18 = 18,432; V Q8_0 = 34,816.
 
 Notation: tok in [0,128) is the token slot inside the page, dim in [0,256) the
 channel, b = dim // 32 the block, d[tok][b] the fp16 block scale.  Tokens are
@@ -17,6 +17,13 @@ K page, Q8_0 (34,816 bytes)
   holds the int8 code of token 16G + 8H + R, channel 64P + 32*(j // 8) + 8T + (j % 8).
   scales, bytes [32768, 34816): fp16 at 32768 + 2*((((G*8 + R)*2 + H)*8) + b)
   holds d[16G + 8H + R][b].
+
+K page, Q4_0 (18,432 bytes)
+  nibbles, bytes [0, 16384): the little-endian 32-bit word at byte
+      4 * (((((G*2 + Q)*2 + H)*8 + R)*4 + T)*4 + c)       (Q<2, H<2, R<8, T<4, c<4)
+  belongs to token 16G + 8H + R and block b = 4Q + c; it holds the 4-bit codes of the
+  channels 32b + 8T + i (i < 8), channel i at bit 4*(i // 2) + 16*(i % 2).
+  scales, bytes [16384, 18432): same arrangement as the Q8_0 K scales.
 
 V page, Q4_0 (18,432 bytes)
   nibbles, bytes [0, 16384): byte at
@@ -43,6 +50,7 @@ HEAD_DIM = 256
 N_BLOCKS = HEAD_DIM // 32
 
 K_Q8_BYTES = 34816
+K_Q4_BYTES = 18432
 V_Q4_BYTES = 18432
 V_Q8_BYTES = 34816
 
@@ -50,6 +58,8 @@ V_Q8_BYTES = 34816
 def page_bytes(role: str, fmt: str) -> int:
     if role == "k" and fmt == "q8_0":
         return K_Q8_BYTES
+    if role == "k" and fmt == "q4_0":
+        return K_Q4_BYTES
     if role == "v" and fmt == "q4_0":
         return V_Q4_BYTES
     if role == "v" and fmt == "q8_0":
@@ -89,6 +99,18 @@ def _v4_nibble_map():
     return off.ravel(), tok.ravel(), lo.ravel(), (lo + 8).ravel()
 
 
+def _k4_nibble_map():
+    """(byte offset, shift, token, channel) of every K Q4_0 code."""
+    G, Q, H, R, T, c, i = np.meshgrid(np.arange(8), np.arange(2), np.arange(2), np.arange(8),
+                                      np.arange(4), np.arange(4), np.arange(8), indexing="ij")
+    word = ((((G * 2 + Q) * 2 + H) * 8 + R) * 4 + T) * 4 + c
+    bit = 4 * (i // 2) + 16 * (i % 2)
+    off = 4 * word + bit // 8
+    tok = 16 * G + 8 * H + R
+    dim = 32 * (4 * Q + c) + 8 * T + i
+    return off.ravel(), (bit % 8).ravel(), tok.ravel(), dim.ravel()
+
+
 def _v8_code_map():
     G, b, R, T, w, y = np.meshgrid(np.arange(8), np.arange(8), np.arange(8), np.arange(4),
                                    np.arange(4), np.arange(4), indexing="ij")
@@ -103,6 +125,7 @@ _K_SCALES = _k_scale_map()
 _V_SCALES = _v_scale_map()
 _V4_NIBBLES = _v4_nibble_map()
 _V8_CODES = _v8_code_map()
+_K4_NIBBLES = _k4_nibble_map()
 
 
 def _flat_codes(codes: np.ndarray) -> np.ndarray:
@@ -117,7 +140,15 @@ def encode_page(role: str, fmt: str, codes: np.ndarray, d: np.ndarray) -> np.nda
     out = np.zeros(n, dtype=np.uint8)
     c = _flat_codes(codes)
     d16 = np.asarray(d, dtype=np.float16).view(np.uint16)
-    if role == "k":
+    if role == "k" and fmt == "q4_0":
+        off, sh, tok, dim = _K4_NIBBLES
+        c8 = c.astype(np.uint8)
+        if np.any(c8 > 15):
+            raise ValueError("Q4_0 codes must be in [0, 15]")
+        np.bitwise_or.at(out, off, (c8[tok, dim] << sh).astype(np.uint8))
+        idx, tok, b = _K_SCALES
+        scale_base = 16384
+    elif role == "k":
         off, tok, dim = _K_CODES
         out[off] = c[tok, dim].astype(np.int8).view(np.uint8)
         idx, tok, b = _K_SCALES
@@ -147,7 +178,12 @@ def decode_page(role: str, fmt: str, page: np.ndarray):
     if page.size != page_bytes(role, fmt):
         raise ValueError("wrong page size")
     c = np.zeros((PAGE_TOKENS, HEAD_DIM), dtype=np.int16)
-    if role == "k":
+    if role == "k" and fmt == "q4_0":
+        off, sh, tok, dim = _K4_NIBBLES
+        c[tok, dim] = (page[off] >> sh) & 0xF
+        idx, tok, b = _K_SCALES
+        scale_base = 16384
+    elif role == "k":
         off, tok, dim = _K_CODES
         c[tok, dim] = page[off].view(np.int8)
         idx, tok, b = _K_SCALES

@@ -26,11 +26,12 @@ import math
 import numpy as np
 
 
-def block_summaries(codes: np.ndarray, d: np.ndarray) -> np.ndarray:
-    """Mean dequantised Q8_0 key of each block.
+def block_summaries(codes: np.ndarray, d: np.ndarray, fmt: str = "q8_0") -> np.ndarray:
+    """Mean dequantised key of each block, keys stored as Q8_0 or Q4_0.
 
-    codes: int8 [n_blocks][128][8][32]; d: float16 [n_blocks][128][8].
-    Returns fp32 [n_blocks][256].
+    codes: [n_blocks][128][8][32] (int8 for Q8_0, 0..15 for Q4_0); d: float16
+    [n_blocks][128][8].  Returns fp32 [n_blocks][256].  The key value is q * d for Q8_0
+    and (q - 8) * d for Q4_0.
 
     Each product d * q is exact in float64 (11 + 8 significant bits) and is a
     multiple of the block's smallest scale grid; when the sum of magnitudes stays
@@ -41,7 +42,10 @@ def block_summaries(codes: np.ndarray, d: np.ndarray) -> np.ndarray:
     codes = np.asarray(codes)
     nb = codes.shape[0]
     d64 = np.asarray(d, dtype=np.float16).astype(np.float64)          # [nb][128][8]
-    prod = codes.astype(np.float64) * d64[..., None]                  # [nb][128][8][32]
+    q = codes.astype(np.float64) - (8.0 if fmt == "q4_0" else 0.0)
+    if fmt not in ("q8_0", "q4_0"):
+        raise ValueError(f"unsupported key format {fmt}")
+    prod = q * d64[..., None]                                         # [nb][128][8][32]
     # exactness certificate
     _, e = np.frexp(np.where(d64 == 0, 1.0, d64))
     grid = np.ldexp(1.0, e - 11)

@@ -27,12 +27,12 @@ def lib():
 class GpuCache:
     """Device page pools for one layer (H_kv units) filled through kvattn_quantize_append."""
 
-    def __init__(self, H_kv, H_q, n_blocks, v_fmt="q4_0", n_phys=None, perm=None, device="cuda"):
+    def __init__(self, H_kv, H_q, n_blocks, v_fmt="q4_0", n_phys=None, perm=None, device="cuda", k_fmt="q8_0"):
         torch = torch_mod()
         kv = lib()
-        self.H_kv, self.H_q, self.n_blocks, self.v_fmt = H_kv, H_q, n_blocks, v_fmt
+        self.H_kv, self.H_q, self.n_blocks, self.v_fmt, self.k_fmt = H_kv, H_q, n_blocks, v_fmt, k_fmt
         self.n_phys = n_phys or H_kv * n_blocks
-        kb = olay.page_bytes("k", "q8_0")
+        kb = olay.page_bytes("k", k_fmt)
         vb = olay.page_bytes("v", v_fmt)
         self.k_pool = torch.zeros((self.n_phys, kb), dtype=torch.uint8, device=device)
         self.v_pool = torch.zeros((self.n_phys, vb), dtype=torch.uint8, device=device)
@@ -40,7 +40,7 @@ class GpuCache:
             perm = np.arange(self.n_phys, dtype=np.int32)
         self.page_table_np = np.asarray(perm[: H_kv * n_blocks], dtype=np.int32).reshape(H_kv, n_blocks)
         self.page_table = torch.from_numpy(self.page_table_np.copy()).to(device)
-        self.desc = kv.make_desc(H_kv, H_q, self.k_pool, self.v_pool, self.n_phys, v_fmt=v_fmt)
+        self.desc = kv.make_desc(H_kv, H_q, self.k_pool, self.v_pool, self.n_phys, v_fmt=v_fmt, k_fmt=k_fmt)
 
     def append(self, k, v, pos0):
         """k, v: fp32 arrays [n][H_kv][256] (numpy or torch)."""
@@ -53,15 +53,15 @@ class GpuCache:
 class OracleCache:
     """The oracle's quantised view of one layer: codes and scales per unit and token."""
 
-    def __init__(self, k, v, v_fmt="q4_0"):
+    def __init__(self, k, v, v_fmt="q4_0", k_fmt="q8_0"):
         # k, v: fp32 [T][H_kv][256]
-        self.v_fmt = v_fmt
-        self.kc, self.kd = oq.q8_0_quantize(np.asarray(k, np.float32))          # [T][H][8][32], [T][H][8]
+        self.v_fmt, self.k_fmt = v_fmt, k_fmt
+        self.kc, self.kd = oq.quantize(np.asarray(k, np.float32), k_fmt)        # [T][H][8][32], [T][H][8]
         self.vc, self.vd = oq.quantize(np.asarray(v, np.float32), v_fmt)
         self.T = k.shape[0]
 
     def khat(self, h):
-        return oq.q8_0_dequantize(self.kc[:, h], self.kd[:, h])
+        return oq.dequantize(self.kc[:, h], self.kd[:, h], self.k_fmt)
 
     def vhat(self, h):
         return oq.dequantize(self.vc[:, h], self.vd[:, h], self.v_fmt)
@@ -70,11 +70,11 @@ class OracleCache:
         """Expected bytes of logical block `blk` of unit h (tokens beyond T stay zero codes)."""
         a, b = blk * 128, min((blk + 1) * 128, self.T)
         if role == "k":
-            codes = np.zeros((128, 8, 32), np.int8)
+            codes = np.zeros((128, 8, 32), np.int8 if self.k_fmt == "q8_0" else np.uint8)
             d = np.zeros((128, 8), np.float16)
             codes[: b - a] = self.kc[a:b, h]
             d[: b - a] = self.kd[a:b, h]
-            return olay.encode_page("k", "q8_0", codes, d)
+            return olay.encode_page("k", self.k_fmt, codes, d)
         codes = np.zeros((128, 8, 32), np.int8 if self.v_fmt == "q8_0" else np.uint8)
         d = np.zeros((128, 8), np.float16)
         codes[: b - a] = self.vc[a:b, h]

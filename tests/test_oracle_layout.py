@@ -16,7 +16,7 @@ def _page(fmt, seed):
     return quant.quantize(x, fmt)
 
 
-@pytest.mark.parametrize("role,fmt", [("k", "q8_0"), ("v", "q4_0"), ("v", "q8_0")])
+@pytest.mark.parametrize("role,fmt", [("k", "q8_0"), ("k", "q4_0"), ("v", "q4_0"), ("v", "q8_0")])
 def test_round_trip(role, fmt):
     codes, d = _page(fmt, 11)
     page = layout.encode_page(role, fmt, codes, d)
@@ -41,6 +41,28 @@ def test_k_code_offsets(tok, dim, off):
     codes, d = _one_hot("q8_0", tok, dim, 7)
     page = layout.encode_page("k", "q8_0", codes, d)
     assert np.flatnonzero(page).tolist() == [off]
+
+
+# K Q4_0: word 4*((((G*2+Q)*2+H)*8+R)*4+T)*4+c) for token 16G+8H+R, block 4Q+c; channel
+# 32b+8T+i sits at bit 4*(i//2) + 16*(i%2) of the little-endian word (offsets worked by hand)
+@pytest.mark.parametrize("tok,dim,off,shift", [
+    (0, 0, 0, 0), (0, 1, 2, 0), (0, 2, 0, 4), (0, 3, 2, 4), (0, 4, 1, 0), (0, 5, 3, 0),
+    (0, 6, 1, 4), (0, 7, 3, 4), (0, 8, 16, 0), (0, 32, 4, 0), (0, 128, 1024, 0), (1, 0, 64, 0),
+    (8, 0, 512, 0), (16, 0, 2048, 0), (5, 200, 1368, 0),
+])
+def test_k_q4_nibble_offsets(tok, dim, off, shift):
+    codes = np.zeros((128, 8, 32), np.uint8)
+    codes[tok, dim // 32, dim % 32] = 9
+    page = layout.encode_page("k", "q4_0", codes, np.zeros((128, 8), np.float16))
+    assert np.flatnonzero(page).tolist() == [off]
+    assert page[off] == 9 << shift
+
+
+def test_k_q4_scales_follow_the_q8_k_arrangement():
+    d = np.zeros((128, 8), np.float16)
+    d[9, 3] = 1.0          # same index 27 as the Q8_0 K page, after 16,384 bytes of nibbles
+    page = layout.encode_page("k", "q4_0", np.zeros((128, 8, 32), np.uint8), d)
+    assert np.flatnonzero(page).tolist() == [16384 + 2 * 27 + 1]
 
 
 def test_k_scale_offsets():

@@ -31,6 +31,21 @@ def test_summaries_equal_correctly_rounded_mean():
             assert s[b, c] == ref
 
 
+def test_q4_0_key_summaries_equal_correctly_rounded_mean():
+    x = normal_f32(np_rng(24), (2, 128, 256))
+    x[..., [5, 77]] *= 8
+    qs, d = quant.q4_0_quantize(x)
+    s = select.block_summaries(qs, d, "q4_0")
+    k = quant.q4_0_dequantize(qs, d)
+    for b in range(2):
+        for c in range(0, 256, 5):
+            assert s[b, c] == np.float32(math.fsum(k[b, :, c].tolist()) / 128.0)
+    # code 3 of a Q4_0 block is the value (3 - 8) * d
+    const = select.block_summaries(np.full((1, 128, 8, 32), 3, np.uint8), np.full((1, 128, 8), np.float16(0.5)),
+                                   "q4_0")
+    assert np.all(const == np.float32(-2.5))
+
+
 def test_summary_of_a_constant_block():
     qs = np.full((1, 128, 8, 32), -5, np.int8)
     d = np.full((1, 128, 8), np.float16(0.375))
