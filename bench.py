@@ -31,7 +31,12 @@ if ROOT not in sys.path:
 from synth import WORKLOADS, derived_seed, np_rng, page_permutation, torch_normal, workload_layer_kv  # noqa: E402
 
 METRIC = "quantized paged KV attention: decode HBM GB/s & prefill TFLOP/s vs roofline"
-BYTES_PER_TOKEN_HEAD = {"q4_0": 34816 // 128 + 18432 // 128, "q8_0": 34816 // 128 + 34816 // 128}  # 416 / 544
+PAGE_BYTES = {("k", "q8_0"): 34816, ("k", "q4_0"): 18432, ("v", "q4_0"): 18432, ("v", "q8_0"): 34816}
+
+
+def bytes_per_token_head(k_fmt: str, v_fmt: str) -> int:
+    """K + V bytes of one token of one KV head: 416 (Q8_0/Q4_0), 544 (Q8_0/Q8_0), 288 (Q4_0/Q4_0)."""
+    return (PAGE_BYTES[("k", k_fmt)] + PAGE_BYTES[("v", v_fmt)]) // 128
 
 
 def parse_args():
@@ -195,7 +200,7 @@ class DecodeCache:
         L, H = w.layers, w.kv_heads
         self.L, self.H, self.nb = L, H, n_blocks_per_unit
         n_phys = L * H * n_blocks_per_unit
-        kb = kv.kvattn_page_bytes(kv.ROLE_K, kv.FMT_Q8_0)
+        kb = kv.kvattn_page_bytes(kv.ROLE_K, kv.FMT[w.k_fmt])
         vb = kv.kvattn_page_bytes(kv.ROLE_V, kv.FMT[w.v_fmt])
         self.k_pool = torch.empty((n_phys, kb), dtype=torch.uint8, device=device)
         self.v_pool = torch.empty((n_phys, vb), dtype=torch.uint8, device=device)
@@ -204,7 +209,7 @@ class DecodeCache:
         rng = np_rng(w.seed, 1)
         perm = page_permutation(rng, n_phys).reshape(L, H, n_blocks_per_unit)
         self.page_table = torch.from_numpy(perm).to(device)        # [L][H][nb]
-        self.desc = kv.make_desc(H, w.q_heads, self.k_pool, self.v_pool, n_phys, v_fmt=w.v_fmt)
+        self.desc = kv.make_desc(H, w.q_heads, self.k_pool, self.v_pool, n_phys, v_fmt=w.v_fmt, k_fmt=w.k_fmt)
         self.needles = {}
         for l in range(L):
             k, v, nd = workload_layer_kv(w, l, tokens, device, q_for_needles[l] if with_needles else None)
@@ -278,7 +283,7 @@ class DecodeBench(GraphStep):
         self.lse = torch.empty((L, 1, Hq), device=device)
         self.ws_bytes = kv.kvattn_decode_workspace_size(self.cache.desc, 1, self.nb)
         self.ws = torch.zeros((L, max(self.ws_bytes, 256)), dtype=torch.uint8, device=device)
-        self.bytes_per_layer = self.ctx * H * BYTES_PER_TOKEN_HEAD[w.v_fmt]
+        self.bytes_per_layer = self.ctx * H * bytes_per_token_head(w.k_fmt, w.v_fmt)
         self.bytes_per_step = self.bytes_per_layer * L
         self.launches_per_step = 3 * L  # quantize-append, decode, split merge
 
@@ -332,7 +337,7 @@ class VerifyBench(GraphStep):
         self.ws_bytes = kv.kvattn_decode_workspace_size(c.desc, w.n_q, self.cap)
         self.ws = torch.zeros((L, max(self.ws_bytes, 256)), dtype=torch.uint8, device=device)
         tokens = (w.budget_blocks + w.recent_blocks) * 128 + w.n_q
-        self.bytes_per_layer = tokens * H * BYTES_PER_TOKEN_HEAD[w.v_fmt]
+        self.bytes_per_layer = tokens * H * bytes_per_token_head(w.k_fmt, w.v_fmt)
         self.bytes_per_step = self.bytes_per_layer * L
         self.select_bytes_per_layer = H * (self.n_full - w.recent_blocks) * 256 * 4
         self.launches_per_step = 5 * L  # block scores, top-k, quantize-append, decode, split merge
@@ -501,7 +506,7 @@ class StreamBench:
         self.ev_dec = [torch.cuda.Event() for _ in range(L)]
         self.copy_bytes_per_step = L * H * self.budget * P
         tokens = self.budget * 128 + 1
-        self.attn_bytes_per_step = L * H * tokens * BYTES_PER_TOKEN_HEAD["q4_0"]
+        self.attn_bytes_per_step = L * H * tokens * bytes_per_token_head("q8_0", "q4_0")
         self.launches_per_step = 5 * L
         self.gather_ctas = 16
 
@@ -782,7 +787,7 @@ def _oracle_inputs(wname, n_tokens):
         v = rng.standard_normal((n_tokens, 256), dtype=np.float32)
         q = rng.standard_normal((w.group, 256), dtype=np.float32)
         _ORACLE_INPUTS.clear()
-        _ORACLE_INPUTS[key] = (q, oq.q8_0_quantize(k), oq.quantize(v, w.v_fmt))
+        _ORACLE_INPUTS[key] = (q, oq.quantize(k, w.k_fmt), oq.quantize(v, w.v_fmt))
     return _ORACLE_INPUTS[key]
 
 
@@ -813,13 +818,13 @@ def oracle_decode_sample(wname, n_tokens, reps_min_s=10.0, max_reps=200):
     t_total, reps = 0.0, 0
     while reps < max_reps and (reps == 0 or t_total < reps_min_s):
         t0 = time.perf_counter()
-        kh = oq.q8_0_dequantize(kc, kd)
+        kh = oq.dequantize(kc, kd, w.k_fmt)
         vh = oq.dequantize(vc, vd, w.v_fmt)
         oatt.attend(q, kh, vh, pos, np.full(w.group, w.context - 1), 1.0 / 16)
         t_total += time.perf_counter() - t0
         reps += 1
     secs = t_total / reps
-    gbs = n_tokens * BYTES_PER_TOKEN_HEAD[w.v_fmt] / secs / 1e9
+    gbs = n_tokens * bytes_per_token_head(w.k_fmt, w.v_fmt) / secs / 1e9
     threads = _blas_threads()
     sample = (f"1 of {w.layers * w.kv_heads} (layer, KV head) units, {n_tokens} of {w.context} tokens, "
               f"{w.group} query heads, timed {reps} times ({t_total:.1f} s of CPU work)")
@@ -841,7 +846,7 @@ def reference_arm(args, world, rank):
         if i >= args.warmup:
             times.append(s)
     secs = statistics.mean(times)
-    value = n_tok * BYTES_PER_TOKEN_HEAD[w.v_fmt] / secs / 1e9
+    value = n_tok * bytes_per_token_head(w.k_fmt, w.v_fmt) / secs / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3, "higher_is_better": True,
@@ -944,6 +949,16 @@ def main():
                                         "kernel_GB/s": b2.bytes_per_layer / (k2 * 1e-3) / 1e9,
                                         "kernel_frac_hbm": b2.bytes_per_layer / (k2 * 1e-3) / 1e9 / hbm}
             del b2
+            torch.cuda.empty_cache()
+            b4 = DecodeBench(kvattn, "decode131k_q4q4", device)
+            b4.capture()
+            ms4 = time_steps(b4, args.extra_steps, 5, world)
+            k4 = time_kernel(b4, 10)
+            extra["decode131k_q4q4"] = {"GB/s": b4.bytes_per_step / (ms4 * 1e-3) / 1e9, "ms_per_step": ms4,
+                                        "kernel_GB/s": b4.bytes_per_layer / (k4 * 1e-3) / 1e9,
+                                        "kernel_frac_hbm": b4.bytes_per_layer / (k4 * 1e-3) / 1e9 / hbm,
+                                        "tokens/s": job_throughput(1, world, ms4)}
+            del b4
             torch.cuda.empty_cache()
             b3 = VerifyBench(kvattn, device)
             b3.capture()

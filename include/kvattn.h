@@ -16,21 +16,28 @@
  *           streamed pages merged by online log-sum-exp; layer L+1 transfers overlapped
  *           with layer L compute).
  *  [GUIDE]  Adaptive KV Streaming six-step validation guide (alphalab.site): streaming needs
- *           flash attention with Q8_0 K / Q4_0 V.
+ *           flash attention with Q8_0 K / Q4_0 V; its build step compiles the q4_0-q4_0 and
+ *           q8_0-q4_0 flash-attention KV pairs among others.
  *  [VULKAN] Vulkan speculative-decoding report, 7900 XTX (lcz.me/topic/1398): model structure
  *           (16 layers x 4 KV heads x 256 = 16,384 elements per token), pitfalls (q4_0 =
  *           18 bytes per 32 elements; only legacy block quants are valid KV formats) and
- *           configs (q8_0 = 8.5 bits per element).
+ *           configs (q8_0 = 8.5 bits per element); summary (a q4_0/q4_0 cache holds the most
+ *           tokens).
  *
  * Data formats (fixed by this library; the pages fix only the bits per element):
  *  - head_dim = 256, page = 128 tokens of one (layer, KV head).
  *  - Q8_0: blocks of 32 int8 codes + one fp16 scale d; value = q * d.
  *    Q4_0: blocks of 32 4-bit codes q in [0,15] + fp16 d; value = (q - 8) * d.
- *  - K pages are Q8_0 (34,816 B); V pages are Q4_0 (18,432 B) or Q8_0 (34,816 B).  Inside a
+ *  - Format pairs: Q8_0 K with Q4_0 or Q8_0 V, and Q4_0 K with Q4_0 V.  K pages are Q8_0
+ *    (34,816 B) or Q4_0 (18,432 B); V pages are Q4_0 (18,432 B) or Q8_0 (34,816 B).  Inside a
  *    page, codes come first and fp16 scales after them, both in tensor-core fragment order
  *    (tok = slot in page, c = channel, b = c/32, G = tok/16):
  *      K Q8_0 code  (tok = 16G+8H+R, c = 64P+32(j/8)+8T+j%8) at ((((G*4+P)*2+H)*8+R)*4+T)*16+j
- *      K scale      d[16G+8H+R][b] at 32768 + 2*(((G*8+R)*2+H)*8+b)
+ *      K Q4_0 word  (tok = 16G+8H+R, b = 4Q+c, channels 32b+8T+i, i < 8) is the little-endian
+ *                   uint32 at 4*(((((G*2+Q)*2+H)*8+R)*4+T)*4+c); channel i's 4-bit code sits
+ *                   at bit 4*(i/2) + 16*(i%2)
+ *      K scale      d[16G+8H+R][b] at S + 2*(((G*8+R)*2+H)*8+b), S = 32768 (Q8_0) or 16384
+ *                   (Q4_0)
  *      V Q4_0 byte  ((((G*4+C)*8+R)*4+T)*16 + 4w + y: block b = 2C+w/2, token
  *                   16G+2T+8(w%2)+y/2; low nibble c = 32b+16(y%2)+R, high nibble c+8
  *      V Q8_0 code  (tok = 16G+2T+8(w%2)+y%2, c = 32b+16(w/2)+8(y/2)+R) at
@@ -41,7 +48,7 @@
  *  - Pages live in caller-owned pools: page p's K bytes start at k_pool + p * k_page_stride
  *    and its V bytes at v_pool + p * v_page_stride.  Pool bases and strides are multiples
  *    of 16 bytes.  K and V of one page may be interleaved in one allocation by choosing
- *    v_pool = k_pool + 34816 and equal strides.
+ *    v_pool = k_pool + (K page bytes) and equal strides.
  *  - A page list names, per KV head, the physical pages to attend over and (optionally)
  *    their logical block indices; key positions are logical * 128 + slot.
  *
@@ -91,7 +98,7 @@ typedef struct kvattn_kv_desc {
   int32_t n_q_heads;      /* H_q, a multiple of H_kv; the GQA group is H_q / H_kv       */
   int32_t head_dim;       /* must be 256                                                */
   int32_t page_tokens;    /* must be 128                                                */
-  int32_t k_fmt;          /* KVATTN_FMT_Q8_0                                            */
+  int32_t k_fmt;          /* KVATTN_FMT_Q8_0, or KVATTN_FMT_Q4_0 (then v_fmt must be Q4_0) */
   int32_t v_fmt;          /* KVATTN_FMT_Q4_0 or KVATTN_FMT_Q8_0                         */
   void* k_pool;           /* device memory, 16-byte aligned                              */
   void* v_pool;           /* device memory, 16-byte aligned                              */
@@ -188,7 +195,8 @@ KVATTN_API int kvattn_merge_lse(const float* o_parts, const float* lse_parts, in
 
 /* ---- KVMem block summaries and selection ([KVMEM]) ---------------------------------
  * Summary of a full 128-token block = mean dequantized key per channel, rounded once to
- * fp32 (the per-block sum is exact in fp64 for scales within 2^28 of each other).
+ * fp32 (the per-block sum is exact in fp64 for scales within 2^28 of each other).  Keys may
+ * be Q8_0 or Q4_0.
  *   page_table  device int32 [n_units][n_blocks] (a unit is one (layer, KV head))
  *   summaries   device fp32 [n_units][n_blocks][256]; blocks [block_begin, block_end) of
  *               every unit are written, others untouched. */
@@ -221,7 +229,8 @@ KVATTN_API int kvattn_select_blocks(const float* summaries, const float* q_group
  * tcgen05 tensor cores with fp32 accumulation in tensor memory.  The keys are taken in
  * splits of kv_split_tokens (a multiple of 128, at most 65,536; a CTA may walk several
  * consecutive splits); partial results are merged by log-sum-exp.  A page id outside
- * [0, n_pages) skips its page and records KVATTN_ERR_BAD_PAGE.
+ * [0, n_pages) skips its page and records KVATTN_ERR_BAD_PAGE.  Needs Q8_0 K / Q4_0 V pages
+ * (UNSUPPORTED_FORMAT otherwise).
  *   q      device bf16 bits [n_q][H_q][256];  out device fp32 [n_q][H_q][256];
  *   lse    device fp32 [n_q][H_q];  page arguments as for kvattn_decode.
  *   ws     device workspace of kvattn_prefill_workspace_size() bytes. */

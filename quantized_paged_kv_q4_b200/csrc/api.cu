@@ -63,6 +63,7 @@ int sm_count_for_planning() {
 
 int64_t page_bytes_of(int role, int fmt) {
   if (role == KVATTN_ROLE_K && fmt == KVATTN_FMT_Q8_0) return kKPageBytes;
+  if (role == KVATTN_ROLE_K && fmt == KVATTN_FMT_Q4_0) return kK4PageBytes;
   if (role == KVATTN_ROLE_V && fmt == KVATTN_FMT_Q4_0) return kV4PageBytes;
   if (role == KVATTN_ROLE_V && fmt == KVATTN_FMT_Q8_0) return kV8PageBytes;
   return 0;
@@ -75,6 +76,8 @@ int validate_desc(const kvattn_kv_desc* d) {
   if (d->head_dim != kHeadDim || d->page_tokens != kPageTokens) return KVATTN_ERR_UNSUPPORTED_FORMAT;
   const int64_t kb = page_bytes_of(KVATTN_ROLE_K, d->k_fmt), vb = page_bytes_of(KVATTN_ROLE_V, d->v_fmt);
   if (!kb || !vb) return KVATTN_ERR_UNSUPPORTED_FORMAT;
+  // Q4_0 keys come with Q4_0 values only
+  if (d->k_fmt == KVATTN_FMT_Q4_0 && d->v_fmt != KVATTN_FMT_Q4_0) return KVATTN_ERR_UNSUPPORTED_FORMAT;
   if (!d->k_pool || !d->v_pool || !aligned16(d->k_pool) || !aligned16(d->v_pool)) return KVATTN_ERR_INVALID_ARG;
   if (d->k_page_stride < kb || d->v_page_stride < vb || (d->k_page_stride & 15) || (d->v_page_stride & 15))
     return KVATTN_ERR_INVALID_ARG;
@@ -218,8 +221,8 @@ KVATTN_API int kvattn_decode(const kvattn_kv_desc* desc, const float* q, int n_q
   prm.n_qh = desc->n_q_heads;
   prm.max_pages = max_pages;
   prm.n_splits = plan.n_splits;
-  cudaError_t e = launch_decode(prm, desc->n_kv_heads, desc->v_fmt == KVATTN_FMT_Q8_0,
-                                static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_decode(prm, desc->n_kv_heads, desc->k_fmt == KVATTN_FMT_Q4_0,
+                                desc->v_fmt == KVATTN_FMT_Q8_0, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVATTN_OK : cuda_fail(e);
 }
 
@@ -462,7 +465,7 @@ KVATTN_API int kvattn_prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* 
                                     size_t ws_bytes, kvattn_stream_t stream) {
   int st = validate_desc(desc);
   if (st) return st;
-  if (desc->v_fmt != KVATTN_FMT_Q4_0) return KVATTN_ERR_UNSUPPORTED_FORMAT;
+  if (desc->k_fmt != KVATTN_FMT_Q8_0 || desc->v_fmt != KVATTN_FMT_Q4_0) return KVATTN_ERR_UNSUPPORTED_FORMAT;
   if (n_q < 1 || max_pages < 0 || !q || !q_pos || !out || !lse || (max_pages > 0 && !page_list))
     return KVATTN_ERR_INVALID_ARG;
   if (kv_split_tokens < kPageTokens || kv_split_tokens % kPageTokens || kv_split_tokens > 65536)

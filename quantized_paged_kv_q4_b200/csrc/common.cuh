@@ -17,6 +17,8 @@ constexpr int kHeadDim = 256;
 constexpr int kPageTokens = 128;
 constexpr int kBlocks = kHeadDim / 32;  // quantisation blocks per row
 constexpr int kKPageBytes = 34816;      // Q8_0: 128 x 8 x (32 + 2)
+constexpr int kK4PageBytes = 18432;     // Q4_0 keys: 128 x 8 x (16 + 2)
+constexpr int kK4ScaleOffset = 16384;
 constexpr int kV4PageBytes = 18432;     // Q4_0: 128 x 8 x (16 + 2)
 constexpr int kV8PageBytes = 34816;     // Q8_0 values
 constexpr int kKScaleOffset = 32768;    // K page: codes first, then fp16 scales

@@ -1,4 +1,6 @@
-// Split-KV flash decode over Q8_0 K / Q4_0 (or Q8_0) V pages, for one query token or an
+// Split-KV flash decode over Q8_0 K / Q4_0 (or Q8_0) V pages, or Q4_0 K / Q4_0 V pages (the
+// q4_0/q4_0 cache of the Vulkan report's summary; q4_0-q4_0 is one of the flash-attention KV
+// pairs built in the six-step validation guide's build step), for one query token or an
 // MTP verify batch of up to 4 (Adaptive KV Streaming + RDNA 4 announcement, wqu.guru,
 // method list: "paged decode attention extended to verify batches").
 //
@@ -23,15 +25,19 @@
 namespace kvattn {
 
 
-template <int NT, bool PAIR, bool VQ8>
+template <int NT, bool PAIR, bool VQ8, bool KQ4>
 struct DecodeCfg {
   static constexpr int kConsumerWarps = 8;
   static constexpr int kThreads = kConsumerWarps * 32;  // lane 0 of warp 0 also issues the copies
   static constexpr int kNB = PAIR ? 4 : 8;      // 32-channel blocks per warp
   static constexpr int kTilesPerWarp = PAIR ? 2 : 1;
+  static constexpr int kKBytes = KQ4 ? kK4PageBytes : kKPageBytes;
+  static constexpr int kKScaleOff = KQ4 ? kK4ScaleOffset : kKScaleOffset;
   static constexpr int kVBytes = VQ8 ? kV8PageBytes : kV4PageBytes;
-  static constexpr int kStageBytes = kKPageBytes + kVBytes;
-  static constexpr int kStages = PAIR ? (VQ8 ? 2 : 3) : (VQ8 ? 3 : 4);
+  static constexpr int kStageBytes = kKBytes + kVBytes;
+  // as many page stages as fit beside the pair exchange buffer and the barriers (at most 6)
+  static constexpr int kStagesFit = (PAIR ? 190000 : 214000) / kStageBytes;
+  static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
   static constexpr int kUnits = PAIR ? 4 : 8;   // independent softmax streams per CTA
   static constexpr int kRowsPad = NT * 8;
   static constexpr int kXBytes = PAIR ? 4 * 2 * 2 * NT * 32 * 16 : 0;  // pair S exchange
@@ -53,9 +59,9 @@ constexpr uint32_t kHalf2_1152 = 0x64806480u;  // 1024 + 128
 constexpr uint32_t kHalf2_1_16 = 0x2C002C00u;  // 1/16
 constexpr uint32_t kHalf2_m72 = 0xD480D480u;   // -(64 + 8)
 
-template <int NT, bool PAIR, bool VQ8>
-__global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_kernel(const DecodeParams p) {
-  using C = DecodeCfg<NT, PAIR, VQ8>;
+template <int NT, bool PAIR, bool VQ8, bool KQ4>
+__global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KQ4>::kThreads, 1) decode_kernel(const DecodeParams p) {
+  using C = DecodeCfg<NT, PAIR, VQ8, KQ4>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   uint64_t* xbar = full + C::kStages;   // [4] pair exchange barriers (PAIR only)
@@ -135,8 +141,8 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
       st_valid[s] = 1;
       uint8_t* stage = smem + s * C::kStageBytes;
       mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-      bulk_g2s(stage, p.k_pool + static_cast<int64_t>(page) * p.k_stride, kKPageBytes, &full[s]);
-      bulk_g2s(stage + kKPageBytes, p.v_pool + static_cast<int64_t>(page) * p.v_stride, C::kVBytes, &full[s]);
+      bulk_g2s(stage, p.k_pool + static_cast<int64_t>(page) * p.k_stride, C::kKBytes, &full[s]);
+      bulk_g2s(stage + C::kKBytes, p.v_pool + static_cast<int64_t>(page) * p.v_stride, C::kVBytes, &full[s]);
     }
     *reinterpret_cast<volatile int*>(s_issued) = i + 1;
   };
@@ -230,7 +236,7 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
       }
       if (st_valid[s]) {
         const uint32_t kb = smem_u32(smem + s * C::kStageBytes);
-        const uint32_t vb = kb + kKPageBytes;
+        const uint32_t vb = kb + C::kKBytes;
         const int logical = st_logical[s];
         const bool need_mask = static_cast<long long>(logical) * kPageTokens + (kPageTokens - 1) > qpos_min;
 #pragma unroll
@@ -246,7 +252,7 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
           uint32_t dk2[2][C::kNB];
 #pragma unroll
           for (int H = 0; H < 2; ++H) {
-            const uint32_t a = kb + kKScaleOffset + (((G * 8 + g) * 2 + H) * 8 + blk0) * 2;
+            const uint32_t a = kb + C::kKScaleOff + (((G * 8 + g) * 2 + H) * 8 + blk0) * 2;
             uint32_t w[4];
             if constexpr (C::kNB == 8) {
               const uint4 v = lds128(a);
@@ -261,6 +267,38 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
               dk2[H][2 * e + 1] = prmt(w[e], 0u, 0x3232u);
             }
           }
+          if constexpr (KQ4) {
+            // Q4_0 keys: one 32-bit word per (token, block) and lane holds channels 8t + i,
+            // channel i at bit 4 * (i / 2) + 16 * (i % 2); a shift by 8 * ks and two masks give
+            // the f16 pairs (4ks, 4ks + 1) and (4ks + 2, 4ks + 3) of k-step ks.  The nibble
+            // q becomes q - 8 exactly (1024 + q - 1032, or (1024 + 16q) / 16 - 72), then the
+            // block scale (one f16 rounding).
+#pragma unroll
+            for (int qq = 0; qq < C::kNB / 4; ++qq) {
+              const int Q = blk0 / 4 + qq;
+              const uint4 ka = lds128(kb + (((((G * 2 + Q) * 2 + 0) * 8 + g) * 4 + t) * 16));
+              const uint4 kc = lds128(kb + (((((G * 2 + Q) * 2 + 1) * 8 + g) * 4 + t) * 16));
+              const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
+              const uint32_t wc[4] = {kc.x, kc.y, kc.z, kc.w};
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const int bl = 4 * qq + c;
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                  const uint32_t xa = wa[c] >> (8 * ks), xc = wc[c] >> (8 * ks);
+                  const uint32_t A0 = hmul2(hsub2(and_or(xa, 0x000F000Fu, kHalf2Magic), kHalf2_1032), dk2[0][bl]);
+                  const uint32_t A2 =
+                      hmul2(hfma2(and_or(xa, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kHalf2_m72), dk2[0][bl]);
+                  const uint32_t A1 = hmul2(hsub2(and_or(xc, 0x000F000Fu, kHalf2Magic), kHalf2_1032), dk2[1][bl]);
+                  const uint32_t A3 =
+                      hmul2(hfma2(and_or(xc, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kHalf2_m72), dk2[1][bl]);
+#pragma unroll
+                  for (int nt = 0; nt < NT; ++nt)
+                    mma_f16(sacc[nt], A0, A1, A2, A3, qf[bl][ks][nt][0], qf[bl][ks][nt][1]);
+                }
+              }
+            }
+          } else {
 #pragma unroll
           for (int pp = 0; pp < C::kNB / 2; ++pp) {
             const int P = blk0 / 2 + pp;
@@ -282,6 +320,7 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8>::kThreads, 1) decode_
                 for (int nt = 0; nt < NT; ++nt) mma_f16(sacc[nt], A0, A1, A2, A3, qf[bl][ks][nt][0], qf[bl][ks][nt][1]);
               }
             }
+          }
           }
           if constexpr (PAIR) {
             // exchange partial scores with the partner warp (other channel half)
@@ -609,9 +648,9 @@ __global__ void __launch_bounds__(kMergeThreads, kMinBlocks) decode_merge_kernel
 }
 
 // ---------------------------------------------------------------------------------------
-template <int NT, bool PAIR, bool VQ8>
+template <int NT, bool PAIR, bool VQ8, bool KQ4>
 static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream_t stream) {
-  using C = DecodeCfg<NT, PAIR, VQ8>;
+  using C = DecodeCfg<NT, PAIR, VQ8, KQ4>;
   // programmatic dependent launch: the grid may start while the previous kernel on the
   // stream drains; the kernel waits for it (griddepcontrol.wait) before reading any input
   cudaLaunchConfig_t cfg = {};
@@ -624,7 +663,7 @@ static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<NT, PAIR, VQ8>, prm);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<NT, PAIR, VQ8, KQ4>, prm);
   if (e != cudaSuccess || prm.n_splits == 1) return e;
   cfg.gridDim = dim3(prm.group * prm.n_q, n_kv);
   cfg.blockDim = dim3(kMergeThreads);
@@ -638,21 +677,34 @@ int decode_rows_pad(int rows) { return ((rows + 7) / 8) * 8; }
 
 cudaError_t prepare_decode_kernels() {
   cudaError_t e;
-#define KV_SET(NT, PAIR, VQ8)                                                                   \
-  e = cudaFuncSetAttribute(decode_kernel<NT, PAIR, VQ8>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                           DecodeCfg<NT, PAIR, VQ8>::kSmemBytes);                               \
+#define KV_SET(NT, PAIR, VQ8, KQ4)                                                                   \
+  e = cudaFuncSetAttribute(decode_kernel<NT, PAIR, VQ8, KQ4>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                           DecodeCfg<NT, PAIR, VQ8, KQ4>::kSmemBytes);                               \
   if (e != cudaSuccess) return e;
-  KV_SET(1, false, false) KV_SET(1, false, true) KV_SET(2, true, false) KV_SET(2, true, true)
-  KV_SET(3, true, false) KV_SET(3, true, true)
+  KV_SET(1, false, false, false) KV_SET(1, false, true, false) KV_SET(2, true, false, false)
+  KV_SET(2, true, true, false) KV_SET(3, true, false, false) KV_SET(3, true, true, false)
+  KV_SET(1, false, false, true) KV_SET(2, true, false, true) KV_SET(3, true, false, true)
 #undef KV_SET
   return cudaSuccess;
 }
 
-cudaError_t launch_decode(const DecodeParams& prm, int n_kv, bool vq8, cudaStream_t stream) {
+// Q8_0 keys with Q4_0 or Q8_0 values, and Q4_0 keys with Q4_0 values.
+cudaError_t launch_decode(const DecodeParams& prm, int n_kv, bool kq4, bool vq8, cudaStream_t stream) {
   const int nt = decode_rows_pad(prm.group * prm.n_q) / 8;
-  if (nt == 1) return vq8 ? launch_decode_t<1, false, true>(prm, n_kv, stream) : launch_decode_t<1, false, false>(prm, n_kv, stream);
-  if (nt == 2) return vq8 ? launch_decode_t<2, true, true>(prm, n_kv, stream) : launch_decode_t<2, true, false>(prm, n_kv, stream);
-  return vq8 ? launch_decode_t<3, true, true>(prm, n_kv, stream) : launch_decode_t<3, true, false>(prm, n_kv, stream);
+  if (kq4) {
+    if (vq8) return cudaErrorInvalidValue;
+    if (nt == 1) return launch_decode_t<1, false, false, true>(prm, n_kv, stream);
+    if (nt == 2) return launch_decode_t<2, true, false, true>(prm, n_kv, stream);
+    return launch_decode_t<3, true, false, true>(prm, n_kv, stream);
+  }
+  if (nt == 1)
+    return vq8 ? launch_decode_t<1, false, true, false>(prm, n_kv, stream)
+               : launch_decode_t<1, false, false, false>(prm, n_kv, stream);
+  if (nt == 2)
+    return vq8 ? launch_decode_t<2, true, true, false>(prm, n_kv, stream)
+               : launch_decode_t<2, true, false, false>(prm, n_kv, stream);
+  return vq8 ? launch_decode_t<3, true, true, false>(prm, n_kv, stream)
+             : launch_decode_t<3, true, false, false>(prm, n_kv, stream);
 }
 
 }  // namespace kvattn

@@ -11,7 +11,7 @@
 // (no FMA contraction), so the codes equal those of any correct fp32 implementation.
 //
 // One warp encodes one (token, KV head) row: lane l owns channels [8l, 8l+8), four lanes
-// form one 32-element block.
+// form one 32-element block.  Keys are stored as Q8_0 or Q4_0, values as Q4_0 or Q8_0.
 #include "common.cuh"
 
 namespace kvattn {
@@ -41,13 +41,39 @@ __device__ __forceinline__ float q8_scale(const float (&x)[8], float* inv) {
   return d;
 }
 
+// Q4_0 block scale of this lane's block (channels 8 * lane + e): the signed element of
+// largest magnitude, first index on ties, over the four lanes of the block; returns
+// d = m / -8 (fp32) and writes 1/d to *inv.
+__device__ __forceinline__ float q4_scale(const float (&x)[8], int lane, float* inv) {
+  float best = x[0];
+  int bidx = lane * 8;
+#pragma unroll
+  for (int e = 1; e < 8; ++e)
+    if (fabsf(x[e]) > fabsf(best)) {
+      best = x[e];
+      bidx = lane * 8 + e;
+    }
+#pragma unroll
+  for (int s = 1; s <= 2; s <<= 1) {
+    const float ob = __shfl_xor_sync(0xffffffffu, best, s);
+    const int oi = __shfl_xor_sync(0xffffffffu, bidx, s);
+    if (fabsf(ob) > fabsf(best) || (fabsf(ob) == fabsf(best) && oi < bidx)) {
+      best = ob;
+      bidx = oi;
+    }
+  }
+  const float d = __fdiv_rn(best, -8.f);
+  *inv = d != 0.f ? __frcp_rn(d) : 0.f;
+  return d;
+}
+
 __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __restrict__ k,
                                                               const float* __restrict__ v, int n_tok,
                                                               int n_kv, int32_t pos0,
                                                               const int32_t* __restrict__ page_table,
                                                               int n_blocks, uint8_t* k_pool, int64_t k_stride,
                                                               uint8_t* v_pool, int64_t v_stride, int64_t n_pages,
-                                                              int v_q8) {
+                                                              int k_q4, int v_q8) {
   // a kernel launched behind this one with programmatic dependent launch (decode) may start
   // its setup now; it waits for this grid to complete before reading the pages
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -73,8 +99,26 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
   const int G = tok >> 4, tl = tok & 15, H = tl >> 3, R = tok & 7;
   const int b = lane >> 2;  // this lane's block
 
+  // ---------------- K: Q4_0 ----------------
+  if (k_q4) {
+    const float x[8] = {kx0.x, kx0.y, kx0.z, kx0.w, kx1.x, kx1.y, kx1.z, kx1.w};
+    float inv;
+    const float d = q4_scale(x, lane, &inv);
+    // one 32-bit word per lane: channel 8T + e at bit 4 * (e / 2) + 16 * (e % 2)
+    uint32_t w = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) w |= static_cast<uint32_t>(q4_code(x[e], inv)) << (4 * (e >> 1) + 16 * (e & 1));
+    uint8_t* pg = k_pool + static_cast<int64_t>(page) * k_stride;
+    const int T = lane & 3;
+    const int word = ((((G * 2 + (b >> 2)) * 2 + H) * 8 + R) * 4 + T) * 4 + (b & 3);
+    *reinterpret_cast<uint32_t*>(pg + 4 * word) = w;
+    if ((lane & 3) == 0) {
+      const int so = kK4ScaleOffset + 2 * (((G * 8 + R) * 2 + H) * 8 + b);
+      *reinterpret_cast<__half*>(pg + so) = __float2half_rn(d);
+    }
+  }
   // ---------------- K: Q8_0 ----------------
-  {
+  else {
     const float x[8] = {kx0.x, kx0.y, kx0.z, kx0.w, kx1.x, kx1.y, kx1.z, kx1.w};
     float inv;
     const float d = q8_scale(x, &inv);
@@ -103,26 +147,8 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
     float d;
     int codes[8];
     if (!v_q8) {
-      // signed element of largest magnitude, first index on ties
-      float best = x[0];
-      int bidx = lane * 8;
-#pragma unroll
-      for (int e = 1; e < 8; ++e)
-        if (fabsf(x[e]) > fabsf(best)) {
-          best = x[e];
-          bidx = lane * 8 + e;
-        }
-#pragma unroll
-      for (int s = 1; s <= 2; s <<= 1) {
-        const float ob = __shfl_xor_sync(0xffffffffu, best, s);
-        const int oi = __shfl_xor_sync(0xffffffffu, bidx, s);
-        if (fabsf(ob) > fabsf(best) || (fabsf(ob) == fabsf(best) && oi < bidx)) {
-          best = ob;
-          bidx = oi;
-        }
-      }
-      d = __fdiv_rn(best, -8.f);
-      const float inv = d != 0.f ? __frcp_rn(d) : 0.f;
+      float inv;
+      d = q4_scale(x, lane, &inv);
 #pragma unroll
       for (int e = 0; e < 8; ++e) codes[e] = q4_code(x[e], inv);
       // lanes cl = 0,1 share bytes (lo, hi nibble) with y%2 = 0; lanes 2,3 with y%2 = 1
@@ -179,6 +205,7 @@ cudaError_t launch_quantize_append(const kvattn_kv_desc& desc, const float* k, c
   return cudaLaunchKernelEx(&cfg, quantize_append_kernel, k, v, n_tok, desc.n_kv_heads, pos0, page_table, n_blocks,
                             static_cast<uint8_t*>(desc.k_pool), desc.k_page_stride,
                             static_cast<uint8_t*>(desc.v_pool), desc.v_page_stride, desc.n_pages,
+                            static_cast<int>(desc.k_fmt == KVATTN_FMT_Q4_0),
                             static_cast<int>(desc.v_fmt == KVATTN_FMT_Q8_0));
 }
 

@@ -20,7 +20,7 @@ namespace kvattn {
 __global__ void __launch_bounds__(256) block_summary_kernel(const uint8_t* __restrict__ k_pool, int64_t k_stride,
                                                             int64_t n_pages, const int32_t* __restrict__ page_table,
                                                             int n_blocks, int block_begin, int n_range,
-                                                            float* __restrict__ summaries) {
+                                                            int k_q4, float* __restrict__ summaries) {
   __shared__ __align__(16) uint8_t page[kKPageBytes];
   const int unit = blockIdx.y;
   const int b = block_begin + blockIdx.x;
@@ -31,16 +31,28 @@ __global__ void __launch_bounds__(256) block_summary_kernel(const uint8_t* __res
   }
   const uint4* src = reinterpret_cast<const uint4*>(k_pool + static_cast<int64_t>(pg) * k_stride);
   uint4* dst = reinterpret_cast<uint4*>(page);
-  for (int i = threadIdx.x; i < kKPageBytes / 16; i += blockDim.x) dst[i] = src[i];
+  const int bytes = k_q4 ? kK4PageBytes : kKPageBytes;
+  const int scale_off = k_q4 ? kK4ScaleOffset : kKScaleOffset;
+  for (int i = threadIdx.x; i < bytes / 16; i += blockDim.x) dst[i] = src[i];
   __syncthreads();
   const int c = threadIdx.x;  // channel
   const int blk = c >> 5;
+  // Q8_0 key byte: token-row base + 16 * T + j; Q4_0 key word: base + T * 4 + (blk & 3), then
+  // the nibble of channel i = c & 7 at bit 4 * (i / 2) + 16 * (i % 2)
   const int P = c >> 6, cc = c & 63, T = (cc & 31) >> 3, j = 8 * (cc >> 5) + (cc & 7);
+  const int i8 = c & 7, nib_shift = 4 * (i8 >> 1) + 16 * (i8 & 1);
   long long acc = 0;
   for (int tok = 0; tok < kPageTokens; ++tok) {
     const int G = tok >> 4, H = (tok & 15) >> 3, R = tok & 7;
-    const int q = static_cast<int8_t>(page[((((G * 4 + P) * 2 + H) * 8 + R) * 4 + T) * 16 + j]);
-    const uint16_t hb = *reinterpret_cast<const uint16_t*>(page + kKScaleOffset + 2 * (((G * 8 + R) * 2 + H) * 8 + blk));
+    int q;
+    if (k_q4) {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(
+          page + 4 * (((((G * 2 + (blk >> 2)) * 2 + H) * 8 + R) * 4 + T) * 4 + (blk & 3)));
+      q = static_cast<int>((w >> nib_shift) & 15u) - 8;
+    } else {
+      q = static_cast<int8_t>(page[((((G * 4 + P) * 2 + H) * 8 + R) * 4 + T) * 16 + j]);
+    }
+    const uint16_t hb = *reinterpret_cast<const uint16_t*>(page + scale_off + 2 * (((G * 8 + R) * 2 + H) * 8 + blk));
     const int e = (hb >> 10) & 31;
     const int mant = hb & 1023;
     const int m = e ? (1024 | mant) : mant;
@@ -249,7 +261,8 @@ cudaError_t launch_block_summaries(const kvattn_kv_desc& d, const int32_t* page_
   if (n <= 0 || n_units <= 0) return cudaSuccess;
   dim3 grid(n, n_units);
   block_summary_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(d.k_pool), d.k_page_stride, d.n_pages,
-                                                 page_table, n_blocks, block_begin, n, summaries);
+                                                 page_table, n_blocks, block_begin, n,
+                                                 static_cast<int>(d.k_fmt == KVATTN_FMT_Q4_0), summaries);
   return cudaGetLastError();
 }
 

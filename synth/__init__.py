@@ -157,6 +157,8 @@ WORKLOADS = {
                            outlier_frac=0.01, seed=2002),
     "decode131k_q8q8": Workload("decode131k_q8q8", layers=16, kv_heads=4, q_heads=24, context=131072,
                                 n_q=1, v_fmt="q8_0", outlier_frac=0.01, seed=2003),
+    "decode131k_q4q4": Workload("decode131k_q4q4", layers=16, kv_heads=4, q_heads=24, context=131072,
+                                n_q=1, k_fmt="q4_0", v_fmt="q4_0", outlier_frac=0.01, seed=2004),
     # 262,144 prior tokens, 4 verify tokens, 20 needles, budget 256 + recent 128 blocks.
     "verify262k": Workload("verify262k", layers=16, kv_heads=4, q_heads=24, context=262144, n_q=4,
                            needles=20, budget_blocks=256, recent_blocks=128, seed=3003),

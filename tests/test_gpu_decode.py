@@ -9,7 +9,7 @@ from synth import normal_f32, np_rng, page_permutation
 pytestmark = pytest.mark.gpu
 
 
-def _layer(seed, H, T, v_fmt, n_blocks=None, spare=0, outliers=True):
+def _layer(seed, H, T, v_fmt, n_blocks=None, spare=0, outliers=True, k_fmt="q8_0"):
     rng = np_rng(seed)
     k = normal_f32(rng, (T, H, 256))
     v = normal_f32(rng, (T, H, 256))
@@ -20,7 +20,7 @@ def _layer(seed, H, T, v_fmt, n_blocks=None, spare=0, outliers=True):
             v[:, h, ch] *= 8
     n_blocks = n_blocks or (T + 127) // 128
     n_phys = H * n_blocks + spare
-    cache = GpuCache(H, 6 * H, n_blocks, v_fmt, n_phys=n_phys, perm=page_permutation(rng, n_phys))
+    cache = GpuCache(H, 6 * H, n_blocks, v_fmt, n_phys=n_phys, perm=page_permutation(rng, n_phys), k_fmt=k_fmt)
     return rng, k, v, cache
 
 
@@ -42,16 +42,16 @@ def _run_decode(kv, cache, H_q, q, q_pos, page_list, page_logical=None, n_pages=
     return out.cpu().numpy(), lse.cpu().numpy(), (qd, qp, pl, lg, npg, out, lse, ws, wsb)
 
 
-@pytest.mark.parametrize("v_fmt", ["q4_0", "q8_0"])
+@pytest.mark.parametrize("k_fmt,v_fmt", [("q8_0", "q4_0"), ("q8_0", "q8_0"), ("q4_0", "q4_0")])
 @pytest.mark.parametrize("n_q", [1, 2, 3, 4])
-def test_decode_matches_oracle(kv_gpu, v_fmt, n_q):
+def test_decode_matches_oracle(kv_gpu, k_fmt, v_fmt, n_q):
     H, H_q, T = 4, 24, 37 * 128 + 77          # ragged tail page
-    rng, k, v, cache = _layer(600 + n_q, H, T, v_fmt, spare=5)
+    rng, k, v, cache = _layer(600 + n_q, H, T, v_fmt, spare=5, k_fmt=k_fmt)
     cache.append(k, v, 0)
     q = normal_f32(rng, (n_q, H_q, 256))
     q_pos = [T - n_q + i for i in range(n_q)]
     out, lse, keep = _run_decode(kv_gpu, cache, H_q, q, q_pos, cache.page_table_np)
-    oc = OracleCache(k, v, v_fmt)
+    oc = OracleCache(k, v, v_fmt, k_fmt)
     for h in range(H):
         o_ref, l_ref = oc.attend(q, q_pos, h, 6)
         compare(out[:, 6 * h:6 * h + 6], lse[:, 6 * h:6 * h + 6], o_ref, l_ref)

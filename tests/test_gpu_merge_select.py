@@ -31,7 +31,7 @@ def test_merge_lse(kv_gpu, n_parts, rows, dim):
     assert np.all(out.cpu().numpy()[0] == 0)
 
 
-def _select_case(seed, H, n_full, tail, budget, recent, needles, group=6):
+def _select_case(seed, H, n_full, tail, budget, recent, needles, group=6, k_fmt="q8_0"):
     rng = np_rng(seed)
     T = n_full * 128 + tail
     n_blocks = n_full + (1 if tail else 0)
@@ -47,16 +47,18 @@ def _select_case(seed, H, n_full, tail, budget, recent, needles, group=6):
         plant_needles(kh, nb, q[h].astype(np.float64).sum(0), rng, cosine=0.9)
         k[:, h] = kh
     n_phys = H * n_blocks + 2
-    cache = GpuCache(H, H * group, n_blocks, "q4_0", n_phys=n_phys, perm=page_permutation(rng, n_phys))
+    cache = GpuCache(H, H * group, n_blocks, "q4_0", n_phys=n_phys, perm=page_permutation(rng, n_phys), k_fmt=k_fmt)
     cache.append(k, v, 0)
     return rng, k, v, q, cache, needle_sets, n_blocks, T
 
 
-@pytest.mark.parametrize("seed,n_full,tail,budget,recent", [(900, 300, 37, 64, 32), (901, 2048, 4, 256, 128),
-                                                            (902, 50, 0, 80, 10), (903, 40, 100, 8, 0)])
-def test_summaries_and_selection_bit_exact(kv_gpu, seed, n_full, tail, budget, recent):
+@pytest.mark.parametrize("seed,n_full,tail,budget,recent,k_fmt", [
+    (900, 300, 37, 64, 32, "q8_0"), (901, 2048, 4, 256, 128, "q8_0"), (902, 50, 0, 80, 10, "q8_0"),
+    (903, 40, 100, 8, 0, "q8_0"), (904, 300, 37, 64, 32, "q4_0")])
+def test_summaries_and_selection_bit_exact(kv_gpu, seed, n_full, tail, budget, recent, k_fmt):
     H = 4
-    rng, k, v, q, cache, needle_sets, n_blocks, T = _select_case(seed, H, n_full, tail, budget, recent, 20 if n_full > 100 else 3)
+    rng, k, v, q, cache, needle_sets, n_blocks, T = _select_case(seed, H, n_full, tail, budget, recent,
+                                                                 20 if n_full > 100 else 3, k_fmt=k_fmt)
     summ = torch.zeros((H, n_blocks, 256), device="cuda")
     kv_gpu.kvattn_block_summaries(cache.desc, cache.page_table, H, n_blocks, 0, n_full, summ)
     n_cand = n_full - min(recent, n_full)
@@ -70,12 +72,12 @@ def test_summaries_and_selection_bit_exact(kv_gpu, seed, n_full, tail, budget, r
     kv_gpu.kvattn_select_blocks(summ, qg, H, 6, n_blocks, n_full, n_blocks, budget, recent, cache.page_table,
                                 sel_l, sel_p, n_sel, cap, ws, wsb)
     torch.cuda.synchronize()
-    oc = OracleCache(k, v, "q4_0")
+    oc = OracleCache(k, v, "q4_0", k_fmt)
     s_gpu = summ.cpu().numpy()
     for h in range(H):
         kc = oc.kc[: n_full * 128, h].reshape(n_full, 128, 8, 32)
         kd = oc.kd[: n_full * 128, h].reshape(n_full, 128, 8)
-        s_ref = osel.block_summaries(kc, kd)
+        s_ref = osel.block_summaries(kc, kd, k_fmt)
         assert np.array_equal(s_gpu[h, :n_full].view(np.uint32), s_ref.view(np.uint32))
         scores = osel.block_scores(s_ref[:n_cand], q[h])
         sel, gap = osel.select_blocks(scores, n_full, n_blocks, budget, recent)

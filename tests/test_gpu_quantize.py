@@ -9,8 +9,8 @@ from synth import normal_f32, np_rng, page_permutation
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("v_fmt", ["q4_0", "q8_0"])
-def test_append_bytes_bit_exact(kv_gpu, v_fmt):
+@pytest.mark.parametrize("k_fmt,v_fmt", [("q8_0", "q4_0"), ("q8_0", "q8_0"), ("q4_0", "q4_0")])
+def test_append_bytes_bit_exact(kv_gpu, k_fmt, v_fmt):
     rng = np_rng(501)
     H, T, n_blocks = 4, 3 * 128 + 50, 5
     k = normal_f32(rng, (T, H, 256))
@@ -28,11 +28,11 @@ def test_append_bytes_bit_exact(kv_gpu, v_fmt):
     v[11, 0, :32] = 3.0                      # ties of the largest magnitude: first index wins
     v[11, 0, 4] = -3.0
     n_phys = H * n_blocks + 3
-    cache = GpuCache(H, 24, n_blocks, v_fmt, n_phys=n_phys, perm=page_permutation(rng, n_phys))
+    cache = GpuCache(H, 24, n_blocks, v_fmt, n_phys=n_phys, perm=page_permutation(rng, n_phys), k_fmt=k_fmt)
     for a, b in ((0, 100), (100, 101), (101, 300), (300, T)):
         cache.append(k[a:b], v[a:b], a)
     torch.cuda.synchronize()
-    oc = OracleCache(k, v, v_fmt)
+    oc = OracleCache(k, v, v_fmt, k_fmt)
     kp = cache.k_pool.cpu().numpy()
     vp = cache.v_pool.cpu().numpy()
     used = set()
