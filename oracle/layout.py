@@ -5,7 +5,8 @@ A page holds the K (or V) rows of 128 consecutive tokens of one (layer, KV head)
 pages fix only the bits per element; the arrangement below is this library's own
 storage spec, written so that one 16-byte load per thread feeds tensor-core
 fragments directly.  Bytes per page equal the AoS block sizes the pages print:
-K Q8_0 = 128 x 8 x 34 = 34,816; K Q4_0 = V Q4_0 = 128 x 8 x 18 = 18,432; V Q8_0 = 34,816.
+K Q8_0 = 128 x 8 x 34 = 34,816; K Q4_0 = V Q4_0 = 128 x 8 x 18 = 18,432; K Q5_1 = 128 x 8 x 24
+= 24,576; V Q8_0 = 34,816.
 
 Notation: tok in [0,128) is the token slot inside the page, dim in [0,256) the
 channel, b = dim // 32 the block, d[tok][b] the fp16 block scale.  Tokens are
@@ -24,6 +25,15 @@ K page, Q4_0 (18,432 bytes)
   belongs to token 16G + 8H + R and block b = 4Q + c; it holds the 4-bit codes of the
   channels 32b + 8T + i (i < 8), channel i at bit 4*(i // 2) + 16*(i % 2).
   scales, bytes [16384, 18432): same arrangement as the Q8_0 K scales.
+
+K page, Q5_1 (24,576 bytes)
+  low nibbles, bytes [0, 16384): the low 4 bits of every code, arranged as the K Q4_0 nibbles.
+  fifth bits, bytes [16384, 20480): the little-endian 32-bit word at byte
+      16384 + 4 * ((((G*2 + Q)*2 + H)*8 + R)*4 + T)
+  holds bit 4 of the codes of token 16G + 8H + R, channels 32(4Q + c) + 8T + i (c < 4, i < 8),
+  channel (c, i) at bit 16*(i % 2) + 4c + i // 2.
+  scales d, bytes [20480, 22528), and minima m, bytes [22528, 24576): fp16 at base + 2*idx
+  with idx the K Q8_0 scale index ((G*8 + R)*2 + H)*8 + b.  The value is q * d + m.
 
 V page, Q4_0 (18,432 bytes)
   nibbles, bytes [0, 16384): byte at
@@ -51,6 +61,7 @@ N_BLOCKS = HEAD_DIM // 32
 
 K_Q8_BYTES = 34816
 K_Q4_BYTES = 18432
+K_Q51_BYTES = 24576
 V_Q4_BYTES = 18432
 V_Q8_BYTES = 34816
 
@@ -60,6 +71,8 @@ def page_bytes(role: str, fmt: str) -> int:
         return K_Q8_BYTES
     if role == "k" and fmt == "q4_0":
         return K_Q4_BYTES
+    if role == "k" and fmt == "q5_1":
+        return K_Q51_BYTES
     if role == "v" and fmt == "q4_0":
         return V_Q4_BYTES
     if role == "v" and fmt == "q8_0":
@@ -111,6 +124,18 @@ def _k4_nibble_map():
     return off.ravel(), (bit % 8).ravel(), tok.ravel(), dim.ravel()
 
 
+def _k5_high_bit_map():
+    """(byte offset, bit in byte, token, channel) of bit 4 of every K Q5_1 code."""
+    G, Q, H, R, T, c, i = np.meshgrid(np.arange(8), np.arange(2), np.arange(2), np.arange(8),
+                                      np.arange(4), np.arange(4), np.arange(8), indexing="ij")
+    word = (((G * 2 + Q) * 2 + H) * 8 + R) * 4 + T
+    bit = 16 * (i % 2) + 4 * c + i // 2
+    off = 16384 + 4 * word + bit // 8
+    tok = 16 * G + 8 * H + R
+    dim = 32 * (4 * Q + c) + 8 * T + i
+    return off.ravel(), (bit % 8).ravel(), tok.ravel(), dim.ravel()
+
+
 def _v8_code_map():
     G, b, R, T, w, y = np.meshgrid(np.arange(8), np.arange(8), np.arange(8), np.arange(4),
                                    np.arange(4), np.arange(4), indexing="ij")
@@ -126,6 +151,7 @@ _V_SCALES = _v_scale_map()
 _V4_NIBBLES = _v4_nibble_map()
 _V8_CODES = _v8_code_map()
 _K4_NIBBLES = _k4_nibble_map()
+_K5_HIGH = _k5_high_bit_map()
 
 
 def _flat_codes(codes: np.ndarray) -> np.ndarray:
@@ -134,12 +160,26 @@ def _flat_codes(codes: np.ndarray) -> np.ndarray:
 
 
 def encode_page(role: str, fmt: str, codes: np.ndarray, d: np.ndarray) -> np.ndarray:
-    """Encode one page.  codes: [128][8][32] (int8 for Q8_0, 0..15 for Q4_0);
-    d: [128][8] float16.  Returns uint8[page_bytes]."""
+    """Encode one page.  codes: [128][8][32] (int8 for Q8_0, 0..15 for Q4_0, 0..31 for Q5_1);
+    d: [128][8] float16 ([128][8][2] (d, m) for Q5_1).  Returns uint8[page_bytes]."""
     n = page_bytes(role, fmt)
     out = np.zeros(n, dtype=np.uint8)
     c = _flat_codes(codes)
     d16 = np.asarray(d, dtype=np.float16).view(np.uint16)
+    if role == "k" and fmt == "q5_1":
+        c8 = c.astype(np.uint8)
+        if np.any(c8 > 31):
+            raise ValueError("Q5_1 codes must be in [0, 31]")
+        off, sh, tok, dim = _K4_NIBBLES
+        np.bitwise_or.at(out, off, ((c8[tok, dim] & 15) << sh).astype(np.uint8))
+        off, sh, tok, dim = _K5_HIGH
+        np.bitwise_or.at(out, off, ((c8[tok, dim] >> 4) << sh).astype(np.uint8))
+        idx, tok, b = _K_SCALES
+        for base, part in ((20480, d16[..., 0]), (22528, d16[..., 1])):
+            sv = part[tok, b]
+            out[base + 2 * idx] = (sv & 0xFF).astype(np.uint8)
+            out[base + 2 * idx + 1] = (sv >> 8).astype(np.uint8)
+        return out
     if role == "k" and fmt == "q4_0":
         off, sh, tok, dim = _K4_NIBBLES
         c8 = c.astype(np.uint8)
@@ -178,6 +218,16 @@ def decode_page(role: str, fmt: str, page: np.ndarray):
     if page.size != page_bytes(role, fmt):
         raise ValueError("wrong page size")
     c = np.zeros((PAGE_TOKENS, HEAD_DIM), dtype=np.int16)
+    if role == "k" and fmt == "q5_1":
+        off, sh, tok, dim = _K4_NIBBLES
+        c[tok, dim] = (page[off] >> sh) & 0xF
+        off, sh, tok, dim = _K5_HIGH
+        c[tok, dim] |= ((page[off] >> sh) & 1).astype(np.int16) << 4
+        idx, tok, b = _K_SCALES
+        dm = np.zeros((PAGE_TOKENS, N_BLOCKS, 2), dtype=np.uint16)
+        for j, base in enumerate((20480, 22528)):
+            dm[tok, b, j] = page[base + 2 * idx].astype(np.uint16) | (page[base + 2 * idx + 1].astype(np.uint16) << 8)
+        return c.astype(np.uint8).reshape(PAGE_TOKENS, N_BLOCKS, 32), dm.view(np.float16)
     if role == "k" and fmt == "q4_0":
         off, sh, tok, dim = _K4_NIBBLES
         c[tok, dim] = (page[off] >> sh) & 0xF

@@ -1,4 +1,4 @@
-"""Q8_0 and Q4_0 block quantisation -- CPU oracle (test infrastructure only).
+"""Q8_0, Q4_0 and Q5_1 block quantisation -- CPU oracle (test infrastructure only).
 
 Both formats split a row into blocks of 32 elements and store one fp16 scale
 ``d`` per block (Vulkan speculative-decoding report, lcz.me/topic/1398, section
@@ -16,6 +16,15 @@ The pages do not spell out the encoders.  The readings used here:
   largest magnitude (first one on ties), ``d = m / -8`` in fp32, ``q =
   min(15, floor(x * (1/d) + 8.5))`` with the product and the sum each rounded to
   fp32; the element m maps to q = 0.  ``m == 0`` gives d = 0 and q = 8.
+
+* Q5_1 (section "pitfalls" of the same report: a 5-bit format with a zero point,
+  6 bits per element, i.e. 32 x 5 bits + fp16 scale + fp16 minimum = 24 bytes per
+  block; the report pairs Q5_1 keys with Q4_0 values): value = q * d + m with q in
+  [0, 31].  ``m`` = the block minimum, ``d = (max - min) / 31`` (the difference and the
+  quotient each rounded to fp32), ``q = min(31, floor((x - m) * (1/d) + 0.5))`` with the
+  difference, the product and the sum each rounded to fp32; d and m are stored as fp16.
+  ``max == min`` gives d = 0 and q = 0.  The scale pair is carried as one float16 array
+  [..., n, 2] holding (d, m).
 
 Every rounding that decides an integer code is done in fp32, exactly as an IEEE
 fp32 unit would do it, so a GPU encoder can match the codes bit for bit.
@@ -86,14 +95,35 @@ def q4_0_dequantize(q: np.ndarray, d: np.ndarray) -> np.ndarray:
     return v.reshape(v.shape[:-2] + (-1,))
 
 
+def q5_1_quantize(x: np.ndarray):
+    """x: fp32 [..., 32n] -> (q uint8 in [0,31] [..., n, 32], (d, m) float16 [..., n, 2])."""
+    xb = _blocks(x)
+    mn = np.min(xb, axis=-1)
+    mx = np.max(xb, axis=-1)
+    d32 = ((mx - mn).astype(F32) / F32(31.0)).astype(F32)
+    inv = _recip_f32(d32)
+    y = ((xb - mn[..., None]).astype(F32) * inv[..., None]).astype(F32)
+    z = (y + F32(0.5)).astype(F32)
+    q = np.minimum(31, np.floor(z.astype(np.float64)))
+    dm = np.stack([d32.astype(np.float16), mn.astype(np.float16)], axis=-1)
+    return q.astype(np.uint8), dm
+
+
+def q5_1_dequantize(q: np.ndarray, dm: np.ndarray) -> np.ndarray:
+    """(q [..., n, 32], (d, m) [..., n, 2]) -> float64 [..., 32n], value = q * d + m."""
+    dm = np.asarray(dm, dtype=np.float16).astype(np.float64)
+    v = q.astype(np.float64) * dm[..., 0][..., None] + dm[..., 1][..., None]
+    return v.reshape(v.shape[:-2] + (-1,))
+
+
 def quantize(x: np.ndarray, fmt: str):
-    return {"q8_0": q8_0_quantize, "q4_0": q4_0_quantize}[fmt](x)
+    return {"q8_0": q8_0_quantize, "q4_0": q4_0_quantize, "q5_1": q5_1_quantize}[fmt](x)
 
 
 def dequantize(codes: np.ndarray, d: np.ndarray, fmt: str) -> np.ndarray:
-    return {"q8_0": q8_0_dequantize, "q4_0": q4_0_dequantize}[fmt](codes, d)
+    return {"q8_0": q8_0_dequantize, "q4_0": q4_0_dequantize, "q5_1": q5_1_dequantize}[fmt](codes, d)
 
 
 def block_bytes(fmt: str) -> int:
-    """Bytes of one 32-element block: fp16 scale + codes."""
-    return {"q8_0": 2 + 32, "q4_0": 2 + 16}[fmt]
+    """Bytes of one 32-element block: fp16 scale (and fp16 minimum) + codes."""
+    return {"q8_0": 2 + 32, "q4_0": 2 + 16, "q5_1": 2 + 2 + 20}[fmt]

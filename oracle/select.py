@@ -26,34 +26,46 @@ import math
 import numpy as np
 
 
+def _grid(v: np.ndarray) -> np.ndarray:
+    """Spacing of the float16 grid at |v| (11 significant bits), inf where v == 0; smaller
+    than the true spacing for fp16 subnormals, which only makes the check stricter."""
+    _, e = np.frexp(np.where(v == 0, 1.0, v))
+    return np.where(v == 0, np.inf, np.ldexp(1.0, e - 11))
+
+
 def block_summaries(codes: np.ndarray, d: np.ndarray, fmt: str = "q8_0") -> np.ndarray:
-    """Mean dequantised key of each block, keys stored as Q8_0 or Q4_0.
+    """Mean dequantised key of each block, keys stored as Q8_0, Q4_0 or Q5_1.
 
-    codes: [n_blocks][128][8][32] (int8 for Q8_0, 0..15 for Q4_0); d: float16
-    [n_blocks][128][8].  Returns fp32 [n_blocks][256].  The key value is q * d for Q8_0
-    and (q - 8) * d for Q4_0.
+    codes: [n_blocks][128][8][32] (int8 for Q8_0, 0..15 for Q4_0, 0..31 for Q5_1); d:
+    float16 [n_blocks][128][8] ([n_blocks][128][8][2] = (d, m) for Q5_1).  Returns fp32
+    [n_blocks][256].  The key value is q * d for Q8_0, (q - 8) * d for Q4_0 and q * d + m
+    for Q5_1.
 
-    Each product d * q is exact in float64 (11 + 8 significant bits) and is a
-    multiple of the block's smallest scale grid; when the sum of magnitudes stays
-    below 2**53 grid steps every partial sum is exact, so the float64 sum below is
-    the exact sum (checked, not assumed).  Division by 128 is exact; the one
+    Each product d * q is exact in float64 (11 + 8 significant bits) and, like each
+    minimum m, a multiple of the block's smallest fp16 grid step; when the sum of
+    magnitudes stays below 2**53 grid steps every partial sum is exact, so the float64 sum
+    below is the exact sum (checked, not assumed).  Division by 128 is exact; the one
     rounding is the final conversion to fp32.
     """
+    if fmt not in ("q8_0", "q4_0", "q5_1"):
+        raise ValueError(f"unsupported key format {fmt}")
     codes = np.asarray(codes)
     nb = codes.shape[0]
-    d64 = np.asarray(d, dtype=np.float16).astype(np.float64)          # [nb][128][8]
+    dd = np.asarray(d, dtype=np.float16).astype(np.float64)
+    d64 = dd[..., 0] if fmt == "q5_1" else dd                         # [nb][128][8]
     q = codes.astype(np.float64) - (8.0 if fmt == "q4_0" else 0.0)
-    if fmt not in ("q8_0", "q4_0"):
-        raise ValueError(f"unsupported key format {fmt}")
-    prod = q * d64[..., None]                                         # [nb][128][8][32]
+    terms = [q * d64[..., None]]                                      # [nb][128][8][32]
+    grids = [_grid(d64)]
+    if fmt == "q5_1":
+        m64 = dd[..., 1]
+        terms.append(np.broadcast_to(m64[..., None], q.shape))
+        grids.append(_grid(m64))
     # exactness certificate
-    _, e = np.frexp(np.where(d64 == 0, 1.0, d64))
-    grid = np.ldexp(1.0, e - 11)
-    grid = np.where(d64 == 0, np.inf, grid).reshape(nb, -1).min(axis=1)
-    mag = np.abs(prod).reshape(nb, -1).sum(axis=1)
+    grid = np.minimum.reduce([g.reshape(nb, -1).min(axis=1) for g in grids])
+    mag = sum(np.abs(t).reshape(nb, -1).sum(axis=1) for t in terms)
     if np.any(np.isfinite(grid) & (mag >= np.ldexp(grid, 53))):
         raise ArithmeticError("block sum not exactly representable in float64")
-    s = prod.sum(axis=1)                                              # [nb][8][32] exact
+    s = sum(t.sum(axis=1) for t in terms)                            # [nb][8][32] exact
     return (s / 128.0).reshape(nb, -1).astype(np.float32)
 
 

@@ -71,7 +71,7 @@ class OracleCache:
         a, b = blk * 128, min((blk + 1) * 128, self.T)
         if role == "k":
             codes = np.zeros((128, 8, 32), np.int8 if self.k_fmt == "q8_0" else np.uint8)
-            d = np.zeros((128, 8), np.float16)
+            d = np.zeros((128,) + self.kd.shape[2:], np.float16)  # (d, m) pairs for Q5_1
             codes[: b - a] = self.kc[a:b, h]
             d[: b - a] = self.kd[a:b, h]
             return olay.encode_page("k", self.k_fmt, codes, d)

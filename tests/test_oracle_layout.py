@@ -16,7 +16,7 @@ def _page(fmt, seed):
     return quant.quantize(x, fmt)
 
 
-@pytest.mark.parametrize("role,fmt", [("k", "q8_0"), ("k", "q4_0"), ("v", "q4_0"), ("v", "q8_0")])
+@pytest.mark.parametrize("role,fmt", [("k", "q8_0"), ("k", "q4_0"), ("k", "q5_1"), ("v", "q4_0"), ("v", "q8_0")])
 def test_round_trip(role, fmt):
     codes, d = _page(fmt, 11)
     page = layout.encode_page(role, fmt, codes, d)
@@ -63,6 +63,34 @@ def test_k_q4_scales_follow_the_q8_k_arrangement():
     d[9, 3] = 1.0          # same index 27 as the Q8_0 K page, after 16,384 bytes of nibbles
     page = layout.encode_page("k", "q4_0", np.zeros((128, 8, 32), np.uint8), d)
     assert np.flatnonzero(page).tolist() == [16384 + 2 * 27 + 1]
+
+
+# K Q5_1: bit 4 of the code of token 16G+8H+R, channel 32(4Q+c)+8T+i sits in the word at
+# 16384 + 4*((((G*2+Q)*2+H)*8+R)*4+T), bit 16*(i%2) + 4c + i//2 (worked by hand)
+@pytest.mark.parametrize("tok,dim,off,bit", [
+    (0, 0, 16384, 0), (0, 1, 16386, 0), (0, 2, 16384, 1), (0, 32, 16384, 4), (0, 96, 16385, 4),
+    (0, 103, 16387, 7), (0, 8, 16388, 0), (0, 128, 16640, 0), (1, 0, 16400, 0), (8, 0, 16512, 0),
+    (16, 0, 16896, 0),
+])
+def test_k_q5_1_fifth_bit_offsets(tok, dim, off, bit):
+    codes = np.zeros((128, 8, 32), np.uint8)
+    codes[tok, dim // 32, dim % 32] = 16
+    page = layout.encode_page("k", "q5_1", codes, np.zeros((128, 8, 2), np.float16))
+    assert np.flatnonzero(page).tolist() == [off]
+    assert page[off] == 1 << bit
+    codes[tok, dim // 32, dim % 32] = 17      # the low nibble goes where a Q4_0 key nibble goes
+    page2 = layout.encode_page("k", "q5_1", codes, np.zeros((128, 8, 2), np.float16))
+    nib = layout.encode_page("k", "q4_0", np.where(codes > 0, 1, 0).astype(np.uint8), np.zeros((128, 8), np.float16))
+    assert np.array_equal(page2[:16384], nib[:16384]) and np.array_equal(page2[16384:], page[16384:])
+
+
+def test_k_q5_1_scale_and_minimum_offsets():
+    dm = np.zeros((128, 8, 2), np.float16)
+    dm[9, 3, 0] = 1.0      # index 27 of the K scale arrangement
+    dm[9, 3, 1] = 2.0      # 0x4000
+    page = layout.encode_page("k", "q5_1", np.zeros((128, 8, 32), np.uint8), dm)
+    assert np.flatnonzero(page).tolist() == [20480 + 2 * 27 + 1, 22528 + 2 * 27 + 1]
+    assert page[20480 + 55] == 0x3C and page[22528 + 55] == 0x40
 
 
 def test_k_scale_offsets():

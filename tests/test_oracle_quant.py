@@ -130,3 +130,58 @@ def test_q4_0_zero_block():
 def test_block_bytes_match_bits_per_element():
     assert quant.block_bytes("q8_0") * 8 / 32 == 8.5
     assert quant.block_bytes("q4_0") * 8 / 32 == 4.5
+    assert quant.block_bytes("q5_1") * 8 / 32 == 6.0
+
+
+def test_q5_1_bits_are_a_third_more_than_q4_0():
+    # the Vulkan report's pitfalls section: Q5_1 keys give a third more key precision (bits)
+    # than Q4_0 keys
+    assert Fraction(quant.block_bytes("q5_1"), quant.block_bytes("q4_0")) == Fraction(4, 3)
+
+
+@pytest.mark.parametrize("outliers", [False, True])
+def test_q5_1_error_bound(outliers):
+    x = _x(7, 256, outliers).reshape(-1, 32)
+    q, dm = quant.q5_1_quantize(x)
+    xh = quant.q5_1_dequantize(q, dm).reshape(-1, 32)
+    mn = x.min(axis=1).astype(np.float64)
+    d32 = ((x.max(axis=1) - x.min(axis=1)).astype(np.float32) / np.float32(31)).astype(np.float32).astype(np.float64)
+    d16 = dm[:, 0, 0].astype(np.float64)
+    m16 = dm[:, 0, 1].astype(np.float64)
+    bound = d32 * (0.5 + 1e-5) + 31 * np.abs(d32 - d16) + np.abs(mn - m16)
+    assert np.all(np.abs(x - xh) <= bound[:, None])
+    assert np.all(q <= 31)
+
+
+def test_q5_1_extremes_map_to_codes_0_and_31():
+    x = _x(8, 64).reshape(-1, 32)
+    q, _ = quant.q5_1_quantize(x)
+    q = q.reshape(-1, 32)
+    rows = np.arange(x.shape[0])
+    assert np.all(q[rows, np.argmin(x, axis=1)] == 0)
+    assert np.all(q[rows, np.argmax(x, axis=1)] == 31)
+
+
+def test_q5_1_round_trip_and_halves():
+    rng = np_rng(9)
+    d, m = 0.25, -1.0
+    q = rng.integers(0, 32, size=(8, 32)).astype(np.uint8)
+    q[:, 0], q[:, 1] = 0, 31                   # the block's minimum and maximum
+    x = (q.astype(np.float32) * np.float32(d) + np.float32(m)).astype(np.float32)
+    qq, dm = quant.q5_1_quantize(x)
+    assert np.array_equal(qq.reshape(q.shape), q)
+    assert np.all(dm[..., 0].astype(np.float64) == d) and np.all(dm[..., 1].astype(np.float64) == m)
+    assert np.array_equal(quant.q5_1_dequantize(qq, dm).reshape(q.shape), x.astype(np.float64))
+    # exact halves round up: (x - m) / d = 0.5 -> 1, 30.5 -> 31, 2.25 -> 2
+    x = np.zeros(32, np.float32)
+    x[0], x[1] = m, m + 31 * d
+    x[2:5] = [m + 0.5 * d, m + 30.5 * d, m + 2.25 * d]
+    qq, _ = quant.q5_1_quantize(x)
+    assert list(qq[0, :5]) == [0, 31, 1, 31, 2]
+    assert qq[0, 5] == 4                       # x = 0: (0 - m) / d = 4
+
+
+def test_q5_1_constant_block():
+    q, dm = quant.q5_1_quantize(np.full(32, 1.5, np.float32))
+    assert dm[0, 0] == 0 and dm[0, 1] == np.float16(1.5) and np.all(q == 0)
+    assert np.all(quant.q5_1_dequantize(q, dm) == 1.5)

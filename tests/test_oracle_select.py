@@ -46,6 +46,22 @@ def test_q4_0_key_summaries_equal_correctly_rounded_mean():
     assert np.all(const == np.float32(-2.5))
 
 
+def test_q5_1_key_summaries_equal_correctly_rounded_mean():
+    x = normal_f32(np_rng(25), (2, 128, 256))
+    x[..., [9, 130]] *= 8
+    qs, dm = quant.q5_1_quantize(x)
+    s = select.block_summaries(qs, dm, "q5_1")
+    k = quant.q5_1_dequantize(qs, dm)
+    for b in range(2):
+        for c in range(0, 256, 5):
+            assert s[b, c] == np.float32(math.fsum(k[b, :, c].tolist()) / 128.0)
+    # code 3 with d = 0.5 and m = -4 is the value -2.5
+    dm1 = np.zeros((1, 128, 8, 2), np.float16)
+    dm1[..., 0], dm1[..., 1] = 0.5, -4.0
+    const = select.block_summaries(np.full((1, 128, 8, 32), 3, np.uint8), dm1, "q5_1")
+    assert np.all(const == np.float32(-2.5))
+
+
 def test_summary_of_a_constant_block():
     qs = np.full((1, 128, 8, 32), -5, np.int8)
     d = np.full((1, 128, 8), np.float16(0.375))
