@@ -31,11 +31,13 @@ if ROOT not in sys.path:
 from synth import WORKLOADS, derived_seed, np_rng, page_permutation, torch_normal, workload_layer_kv  # noqa: E402
 
 METRIC = "quantized paged KV attention: decode HBM GB/s & prefill TFLOP/s vs roofline"
-PAGE_BYTES = {("k", "q8_0"): 34816, ("k", "q4_0"): 18432, ("v", "q4_0"): 18432, ("v", "q8_0"): 34816}
+PAGE_BYTES = {("k", "q8_0"): 34816, ("k", "q4_0"): 18432, ("k", "q5_1"): 24576, ("v", "q4_0"): 18432,
+              ("v", "q8_0"): 34816}
 
 
 def bytes_per_token_head(k_fmt: str, v_fmt: str) -> int:
-    """K + V bytes of one token of one KV head: 416 (Q8_0/Q4_0), 544 (Q8_0/Q8_0), 288 (Q4_0/Q4_0)."""
+    """K + V bytes of one token of one KV head: 416 (Q8_0/Q4_0), 544 (Q8_0/Q8_0), 288 (Q4_0/Q4_0),
+    336 (Q5_1/Q4_0)."""
     return (PAGE_BYTES[("k", k_fmt)] + PAGE_BYTES[("v", v_fmt)]) // 128
 
 
@@ -924,7 +926,7 @@ def main():
                    "l2": "inputs larger than L2 (218 MB of KV per layer launch, 3.49 GB per step)",
                    "launch": launch_mode},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": profiled_traffic("decode_kernel_decode131k.md"), "kernel": "decode_kernel<1,false,false>",
+                     "traffic": profiled_traffic("decode_kernel_decode131k.md"), "kernel": "decode_kernel<1,false,false,0>",
                      "peak_kind": f"{peak_kind} copy bandwidth (hbm_gbs)",
                      "algorithmic_bytes_per_launch": b.bytes_per_layer, "avg_launch_ms": kern_ms},
         "e2e": {"value": b.bytes_per_step * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
@@ -941,25 +943,18 @@ def main():
     extra = {}
     if not args.no_extra:
         try:
-            b2 = DecodeBench(kvattn, "decode131k_q8q8", device)
-            b2.capture()
-            ms2 = time_steps(b2, args.extra_steps, 5, world)
-            k2 = time_kernel(b2, 10)
-            extra["decode131k_q8q8"] = {"GB/s": b2.bytes_per_step / (ms2 * 1e-3) / 1e9, "ms_per_step": ms2,
-                                        "kernel_GB/s": b2.bytes_per_layer / (k2 * 1e-3) / 1e9,
-                                        "kernel_frac_hbm": b2.bytes_per_layer / (k2 * 1e-3) / 1e9 / hbm}
-            del b2
-            torch.cuda.empty_cache()
-            b4 = DecodeBench(kvattn, "decode131k_q4q4", device)
-            b4.capture()
-            ms4 = time_steps(b4, args.extra_steps, 5, world)
-            k4 = time_kernel(b4, 10)
-            extra["decode131k_q4q4"] = {"GB/s": b4.bytes_per_step / (ms4 * 1e-3) / 1e9, "ms_per_step": ms4,
-                                        "kernel_GB/s": b4.bytes_per_layer / (k4 * 1e-3) / 1e9,
-                                        "kernel_frac_hbm": b4.bytes_per_layer / (k4 * 1e-3) / 1e9 / hbm,
-                                        "tokens/s": job_throughput(1, world, ms4)}
-            del b4
-            torch.cuda.empty_cache()
+            # the same decode step over the other KV format pairs
+            for wn in ("decode131k_q8q8", "decode131k_q4q4", "decode131k_q51q4"):
+                b2 = DecodeBench(kvattn, wn, device)
+                b2.capture()
+                ms2 = time_steps(b2, args.extra_steps, 5, world)
+                k2 = time_kernel(b2, 10)
+                extra[wn] = {"GB/s": b2.bytes_per_step / (ms2 * 1e-3) / 1e9, "ms_per_step": ms2,
+                             "kernel_GB/s": b2.bytes_per_layer / (k2 * 1e-3) / 1e9,
+                             "kernel_frac_hbm": b2.bytes_per_layer / (k2 * 1e-3) / 1e9 / hbm,
+                             "kernel_ms": k2, "bytes_per_token_head": bytes_per_token_head(b2.w.k_fmt, b2.w.v_fmt)}
+                del b2
+                torch.cuda.empty_cache()
             b3 = VerifyBench(kvattn, device)
             b3.capture()
             ms3 = time_steps(b3, args.extra_steps, 5, world)

@@ -28,16 +28,23 @@
  *  - head_dim = 256, page = 128 tokens of one (layer, KV head).
  *  - Q8_0: blocks of 32 int8 codes + one fp16 scale d; value = q * d.
  *    Q4_0: blocks of 32 4-bit codes q in [0,15] + fp16 d; value = (q - 8) * d.
- *  - Format pairs: Q8_0 K with Q4_0 or Q8_0 V, and Q4_0 K with Q4_0 V.  K pages are Q8_0
- *    (34,816 B) or Q4_0 (18,432 B); V pages are Q4_0 (18,432 B) or Q8_0 (34,816 B).  Inside a
+ *    Q5_1: blocks of 32 5-bit codes q in [0,31] + fp16 d + fp16 minimum m; value = q * d + m
+ *    ([VULKAN] pitfalls: 6 bits per element, a zero point; paired with Q4_0 values).
+ *  - Format pairs: Q8_0 K with Q4_0 or Q8_0 V, and Q4_0 or Q5_1 K with Q4_0 V.  K pages are
+ *    Q8_0 (34,816 B), Q4_0 (18,432 B) or Q5_1 (24,576 B); V pages are Q4_0 (18,432 B) or Q8_0
+ *    (34,816 B).  Inside a
  *    page, codes come first and fp16 scales after them, both in tensor-core fragment order
  *    (tok = slot in page, c = channel, b = c/32, G = tok/16):
  *      K Q8_0 code  (tok = 16G+8H+R, c = 64P+32(j/8)+8T+j%8) at ((((G*4+P)*2+H)*8+R)*4+T)*16+j
  *      K Q4_0 word  (tok = 16G+8H+R, b = 4Q+c, channels 32b+8T+i, i < 8) is the little-endian
  *                   uint32 at 4*(((((G*2+Q)*2+H)*8+R)*4+T)*4+c); channel i's 4-bit code sits
  *                   at bit 4*(i/2) + 16*(i%2)
- *      K scale      d[16G+8H+R][b] at S + 2*(((G*8+R)*2+H)*8+b), S = 32768 (Q8_0) or 16384
- *                   (Q4_0)
+ *      K Q5_1       low 4 bits of each code as the K Q4_0 word; bit 4 of the codes of token
+ *                   16G+8H+R, channels 32(4Q+c)+8T+i in the uint32 at
+ *                   16384 + 4*((((G*2+Q)*2+H)*8+R)*4+T), channel (c, i) at bit 16(i%2)+4c+i/2;
+ *                   minimum m[16G+8H+R][b] at 22528 + 2*(((G*8+R)*2+H)*8+b)
+ *      K scale      d[16G+8H+R][b] at S + 2*(((G*8+R)*2+H)*8+b), S = 32768 (Q8_0), 16384
+ *                   (Q4_0) or 20480 (Q5_1)
  *      V Q4_0 byte  ((((G*4+C)*8+R)*4+T)*16 + 4w + y: block b = 2C+w/2, token
  *                   16G+2T+8(w%2)+y/2; low nibble c = 32b+16(y%2)+R, high nibble c+8
  *      V Q8_0 code  (tok = 16G+2T+8(w%2)+y%2, c = 32b+16(w/2)+8(y/2)+R) at
@@ -90,7 +97,7 @@ enum kvattn_status {
   KVATTN_ERR_NOT_INITIALIZED = -9     /* kvattn_init was not called for the current device  */
 };
 
-enum kvattn_format { KVATTN_FMT_Q4_0 = 4, KVATTN_FMT_Q8_0 = 8 };
+enum kvattn_format { KVATTN_FMT_Q4_0 = 4, KVATTN_FMT_Q8_0 = 8, KVATTN_FMT_Q5_1 = 51 };
 enum kvattn_role { KVATTN_ROLE_K = 0, KVATTN_ROLE_V = 1 };
 
 typedef struct kvattn_kv_desc {
@@ -98,7 +105,7 @@ typedef struct kvattn_kv_desc {
   int32_t n_q_heads;      /* H_q, a multiple of H_kv; the GQA group is H_q / H_kv       */
   int32_t head_dim;       /* must be 256                                                */
   int32_t page_tokens;    /* must be 128                                                */
-  int32_t k_fmt;          /* KVATTN_FMT_Q8_0, or KVATTN_FMT_Q4_0 (then v_fmt must be Q4_0) */
+  int32_t k_fmt;          /* KVATTN_FMT_Q8_0, or Q4_0 / Q5_1 (then v_fmt must be Q4_0)  */
   int32_t v_fmt;          /* KVATTN_FMT_Q4_0 or KVATTN_FMT_Q8_0                         */
   void* k_pool;           /* device memory, 16-byte aligned                              */
   void* v_pool;           /* device memory, 16-byte aligned                              */
@@ -128,10 +135,12 @@ KVATTN_API int kvattn_device_error(kvattn_stream_t stream);
 KVATTN_API int64_t kvattn_page_bytes(int role, int fmt);
 
 /* ---- cache write path ----------------------------------------------------------------
- * Quantizes n_tok new tokens and writes them into their pages (the Q8_0 / Q4_0 encoders of
- * [VULKAN] pitfalls).  Q8_0: d = amax/127, q = round-half-away(x * fp32(1/d)), clamped to
- * +-127.  Q4_0: m = the element of largest magnitude, d = m/-8, q = min(15, floor(x * fp32(1/d)
- * + 8.5)).  Every step that decides a code is rounded to fp32; scales are stored as fp16.
+ * Quantizes n_tok new tokens and writes them into their pages (the Q8_0 / Q4_0 / Q5_1
+ * encoders of [VULKAN] pitfalls).  Q8_0: d = amax/127, q = round-half-away(x * fp32(1/d)),
+ * clamped to +-127.  Q4_0: m = the element of largest magnitude, d = m/-8, q = min(15,
+ * floor(x * fp32(1/d) + 8.5)).  Q5_1: m = the block minimum, d = (max - m)/31, q = min(31,
+ * floor((x - m) * fp32(1/d) + 0.5)).  Every step that decides a code is rounded to fp32;
+ * scales and minima are stored as fp16.
  *   k, v        device fp32 [n_tok][H_kv][256]
  *   pos0        position of the first token; token i goes to logical block (pos0+i)/128,
  *               slot (pos0+i)%128
@@ -196,7 +205,7 @@ KVATTN_API int kvattn_merge_lse(const float* o_parts, const float* lse_parts, in
 /* ---- KVMem block summaries and selection ([KVMEM]) ---------------------------------
  * Summary of a full 128-token block = mean dequantized key per channel, rounded once to
  * fp32 (the per-block sum is exact in fp64 for scales within 2^28 of each other).  Keys may
- * be Q8_0 or Q4_0.
+ * be Q8_0, Q4_0 or Q5_1.
  *   page_table  device int32 [n_units][n_blocks] (a unit is one (layer, KV head))
  *   summaries   device fp32 [n_units][n_blocks][256]; blocks [block_begin, block_end) of
  *               every unit are written, others untouched. */

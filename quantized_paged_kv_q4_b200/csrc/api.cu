@@ -64,6 +64,7 @@ int sm_count_for_planning() {
 int64_t page_bytes_of(int role, int fmt) {
   if (role == KVATTN_ROLE_K && fmt == KVATTN_FMT_Q8_0) return kKPageBytes;
   if (role == KVATTN_ROLE_K && fmt == KVATTN_FMT_Q4_0) return kK4PageBytes;
+  if (role == KVATTN_ROLE_K && fmt == KVATTN_FMT_Q5_1) return kK5PageBytes;
   if (role == KVATTN_ROLE_V && fmt == KVATTN_FMT_Q4_0) return kV4PageBytes;
   if (role == KVATTN_ROLE_V && fmt == KVATTN_FMT_Q8_0) return kV8PageBytes;
   return 0;
@@ -76,8 +77,8 @@ int validate_desc(const kvattn_kv_desc* d) {
   if (d->head_dim != kHeadDim || d->page_tokens != kPageTokens) return KVATTN_ERR_UNSUPPORTED_FORMAT;
   const int64_t kb = page_bytes_of(KVATTN_ROLE_K, d->k_fmt), vb = page_bytes_of(KVATTN_ROLE_V, d->v_fmt);
   if (!kb || !vb) return KVATTN_ERR_UNSUPPORTED_FORMAT;
-  // Q4_0 keys come with Q4_0 values only
-  if (d->k_fmt == KVATTN_FMT_Q4_0 && d->v_fmt != KVATTN_FMT_Q4_0) return KVATTN_ERR_UNSUPPORTED_FORMAT;
+  // Q4_0 and Q5_1 keys come with Q4_0 values only
+  if (d->k_fmt != KVATTN_FMT_Q8_0 && d->v_fmt != KVATTN_FMT_Q4_0) return KVATTN_ERR_UNSUPPORTED_FORMAT;
   if (!d->k_pool || !d->v_pool || !aligned16(d->k_pool) || !aligned16(d->v_pool)) return KVATTN_ERR_INVALID_ARG;
   if (d->k_page_stride < kb || d->v_page_stride < vb || (d->k_page_stride & 15) || (d->v_page_stride & 15))
     return KVATTN_ERR_INVALID_ARG;
@@ -221,8 +222,9 @@ KVATTN_API int kvattn_decode(const kvattn_kv_desc* desc, const float* q, int n_q
   prm.n_qh = desc->n_q_heads;
   prm.max_pages = max_pages;
   prm.n_splits = plan.n_splits;
-  cudaError_t e = launch_decode(prm, desc->n_kv_heads, desc->k_fmt == KVATTN_FMT_Q4_0,
-                                desc->v_fmt == KVATTN_FMT_Q8_0, static_cast<cudaStream_t>(stream));
+  const int kf = desc->k_fmt == KVATTN_FMT_Q4_0 ? kKeyQ4 : desc->k_fmt == KVATTN_FMT_Q5_1 ? kKeyQ51 : kKeyQ8;
+  cudaError_t e = launch_decode(prm, desc->n_kv_heads, kf, desc->v_fmt == KVATTN_FMT_Q8_0,
+                                static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVATTN_OK : cuda_fail(e);
 }
 

@@ -19,6 +19,12 @@ constexpr int kBlocks = kHeadDim / 32;  // quantisation blocks per row
 constexpr int kKPageBytes = 34816;      // Q8_0: 128 x 8 x (32 + 2)
 constexpr int kK4PageBytes = 18432;     // Q4_0 keys: 128 x 8 x (16 + 2)
 constexpr int kK4ScaleOffset = 16384;
+constexpr int kK5PageBytes = 24576;     // Q5_1 keys: 128 x 8 x (20 + 2 + 2)
+constexpr int kK5HighOffset = 16384;    // fifth code bits, after the low nibbles
+constexpr int kK5ScaleOffset = 20480;
+constexpr int kK5MinOffset = 22528;
+// key formats as kernel template / flag values
+constexpr int kKeyQ8 = 0, kKeyQ4 = 1, kKeyQ51 = 2;
 constexpr int kV4PageBytes = 18432;     // Q4_0: 128 x 8 x (16 + 2)
 constexpr int kV8PageBytes = 34816;     // Q8_0 values
 constexpr int kKScaleOffset = 32768;    // K page: codes first, then fp16 scales
@@ -114,6 +120,12 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
@@ -160,6 +172,13 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
 __device__ __forceinline__ uint32_t and_or(uint32_t x, uint32_t mask, uint32_t orv) {
   uint32_t r;
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(x), "r"(mask), "r"(orv));
+  return r;
+}
+
+// x | (y & mask)
+__device__ __forceinline__ uint32_t or_and(uint32_t x, uint32_t y, uint32_t mask) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xF8;" : "=r"(r) : "r"(x), "r"(y), "r"(mask));
   return r;
 }
 

@@ -25,14 +25,14 @@
 namespace kvattn {
 
 
-template <int NT, bool PAIR, bool VQ8, bool KQ4>
+template <int NT, bool PAIR, bool VQ8, int KF>
 struct DecodeCfg {
   static constexpr int kConsumerWarps = 8;
   static constexpr int kThreads = kConsumerWarps * 32;  // lane 0 of warp 0 also issues the copies
   static constexpr int kNB = PAIR ? 4 : 8;      // 32-channel blocks per warp
   static constexpr int kTilesPerWarp = PAIR ? 2 : 1;
-  static constexpr int kKBytes = KQ4 ? kK4PageBytes : kKPageBytes;
-  static constexpr int kKScaleOff = KQ4 ? kK4ScaleOffset : kKScaleOffset;
+  static constexpr int kKBytes = KF == kKeyQ4 ? kK4PageBytes : KF == kKeyQ51 ? kK5PageBytes : kKPageBytes;
+  static constexpr int kKScaleOff = KF == kKeyQ4 ? kK4ScaleOffset : KF == kKeyQ51 ? kK5ScaleOffset : kKScaleOffset;
   static constexpr int kVBytes = VQ8 ? kV8PageBytes : kV4PageBytes;
   static constexpr int kStageBytes = kKBytes + kVBytes;
   // as many page stages as fit beside the pair exchange buffer and the barriers (at most 6)
@@ -58,10 +58,11 @@ constexpr uint32_t kHalf2_1032 = 0x64086408u;  // 1024 + 8
 constexpr uint32_t kHalf2_1152 = 0x64806480u;  // 1024 + 128
 constexpr uint32_t kHalf2_1_16 = 0x2C002C00u;  // 1/16
 constexpr uint32_t kHalf2_m72 = 0xD480D480u;   // -(64 + 8)
+constexpr uint32_t kHalf2_m64 = 0xD400D400u;   // -64
 
-template <int NT, bool PAIR, bool VQ8, bool KQ4>
-__global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KQ4>::kThreads, 1) decode_kernel(const DecodeParams p) {
-  using C = DecodeCfg<NT, PAIR, VQ8, KQ4>;
+template <int NT, bool PAIR, bool VQ8, int KF>
+__global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KF>::kThreads, 1) decode_kernel(const DecodeParams p) {
+  using C = DecodeCfg<NT, PAIR, VQ8, KF>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   uint64_t* xbar = full + C::kStages;   // [4] pair exchange barriers (PAIR only)
@@ -267,7 +268,68 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KQ4>::kThreads, 1) de
               dk2[H][2 * e + 1] = prmt(w[e], 0u, 0x3232u);
             }
           }
-          if constexpr (KQ4) {
+          if constexpr (KF == kKeyQ51) {
+            // Q5_1 keys: the low nibbles as for Q4_0 keys; the fifth bits of the lane's four
+            // blocks of one token in one word, channel (c, i) at bit 16(i%2) + 4c + i/2, shifted
+            // to bit 4 (f16 pair 1024 + q) or bit 8 (pair 1024 + 16q) of each half.  q is exact
+            // in f16; the value q * d + m takes one f16 rounding (fma).
+            uint32_t mk2[2][C::kNB];
+#pragma unroll
+            for (int H = 0; H < 2; ++H) {
+              const uint32_t a = kb + kK5MinOffset + (((G * 8 + g) * 2 + H) * 8 + blk0) * 2;
+              uint32_t w[4];
+              if constexpr (C::kNB == 8) {
+                const uint4 v = lds128(a);
+                w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+              } else {
+                asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(a));
+                w[2] = w[3] = 0u;
+              }
+#pragma unroll
+              for (int e = 0; e < C::kNB / 2; ++e) {
+                mk2[H][2 * e] = prmt(w[e], 0u, 0x1010u);
+                mk2[H][2 * e + 1] = prmt(w[e], 0u, 0x3232u);
+              }
+            }
+#pragma unroll
+            for (int qq = 0; qq < C::kNB / 4; ++qq) {
+              const int Q = blk0 / 4 + qq;
+              const int row0 = (((G * 2 + Q) * 2 + 0) * 8 + g) * 4 + t;
+              const int row1 = (((G * 2 + Q) * 2 + 1) * 8 + g) * 4 + t;
+              const uint4 ka = lds128(kb + row0 * 16);
+              const uint4 kc = lds128(kb + row1 * 16);
+              const uint32_t xa5 = lds32(kb + kK5HighOffset + row0 * 4);
+              const uint32_t xc5 = lds32(kb + kK5HighOffset + row1 * 4);
+              const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
+              const uint32_t wc[4] = {kc.x, kc.y, kc.z, kc.w};
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const int bl = 4 * qq + c;
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                  const uint32_t xa = wa[c] >> (8 * ks), xc = wc[c] >> (8 * ks);
+                  const int slo = 4 - (4 * c + 2 * ks), shi = 7 - (4 * c + 2 * ks);
+                  const uint32_t ha_lo = slo >= 0 ? xa5 << slo : xa5 >> -slo;
+                  const uint32_t ha_hi = shi >= 0 ? xa5 << shi : xa5 >> -shi;
+                  const uint32_t hc_lo = slo >= 0 ? xc5 << slo : xc5 >> -slo;
+                  const uint32_t hc_hi = shi >= 0 ? xc5 << shi : xc5 >> -shi;
+                  const uint32_t qa0 = hsub2(or_and(and_or(xa, 0x000F000Fu, kHalf2Magic), ha_lo, 0x00100010u), kHalf2Magic);
+                  const uint32_t qa2 =
+                      hfma2(or_and(and_or(xa, 0x00F000F0u, kHalf2Magic), ha_hi, 0x01000100u), kHalf2_1_16, kHalf2_m64);
+                  const uint32_t qc1 = hsub2(or_and(and_or(xc, 0x000F000Fu, kHalf2Magic), hc_lo, 0x00100010u), kHalf2Magic);
+                  const uint32_t qc3 =
+                      hfma2(or_and(and_or(xc, 0x00F000F0u, kHalf2Magic), hc_hi, 0x01000100u), kHalf2_1_16, kHalf2_m64);
+                  const uint32_t A0 = hfma2(qa0, dk2[0][bl], mk2[0][bl]);
+                  const uint32_t A2 = hfma2(qa2, dk2[0][bl], mk2[0][bl]);
+                  const uint32_t A1 = hfma2(qc1, dk2[1][bl], mk2[1][bl]);
+                  const uint32_t A3 = hfma2(qc3, dk2[1][bl], mk2[1][bl]);
+#pragma unroll
+                  for (int nt = 0; nt < NT; ++nt)
+                    mma_f16(sacc[nt], A0, A1, A2, A3, qf[bl][ks][nt][0], qf[bl][ks][nt][1]);
+                }
+              }
+            }
+          } else if constexpr (KF == kKeyQ4) {
             // Q4_0 keys: one 32-bit word per (token, block) and lane holds channels 8t + i,
             // channel i at bit 4 * (i / 2) + 16 * (i % 2); a shift by 8 * ks and two masks give
             // the f16 pairs (4ks, 4ks + 1) and (4ks + 2, 4ks + 3) of k-step ks.  The nibble
@@ -648,9 +710,9 @@ __global__ void __launch_bounds__(kMergeThreads, kMinBlocks) decode_merge_kernel
 }
 
 // ---------------------------------------------------------------------------------------
-template <int NT, bool PAIR, bool VQ8, bool KQ4>
+template <int NT, bool PAIR, bool VQ8, int KF>
 static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream_t stream) {
-  using C = DecodeCfg<NT, PAIR, VQ8, KQ4>;
+  using C = DecodeCfg<NT, PAIR, VQ8, KF>;
   // programmatic dependent launch: the grid may start while the previous kernel on the
   // stream drains; the kernel waits for it (griddepcontrol.wait) before reading any input
   cudaLaunchConfig_t cfg = {};
@@ -663,7 +725,7 @@ static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<NT, PAIR, VQ8, KQ4>, prm);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<NT, PAIR, VQ8, KF>, prm);
   if (e != cudaSuccess || prm.n_splits == 1) return e;
   cfg.gridDim = dim3(prm.group * prm.n_q, n_kv);
   cfg.blockDim = dim3(kMergeThreads);
@@ -677,34 +739,35 @@ int decode_rows_pad(int rows) { return ((rows + 7) / 8) * 8; }
 
 cudaError_t prepare_decode_kernels() {
   cudaError_t e;
-#define KV_SET(NT, PAIR, VQ8, KQ4)                                                                   \
-  e = cudaFuncSetAttribute(decode_kernel<NT, PAIR, VQ8, KQ4>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                           DecodeCfg<NT, PAIR, VQ8, KQ4>::kSmemBytes);                               \
+#define KV_SET(NT, PAIR, VQ8, KF)                                                                   \
+  e = cudaFuncSetAttribute(decode_kernel<NT, PAIR, VQ8, KF>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                           DecodeCfg<NT, PAIR, VQ8, KF>::kSmemBytes);                               \
   if (e != cudaSuccess) return e;
-  KV_SET(1, false, false, false) KV_SET(1, false, true, false) KV_SET(2, true, false, false)
-  KV_SET(2, true, true, false) KV_SET(3, true, false, false) KV_SET(3, true, true, false)
-  KV_SET(1, false, false, true) KV_SET(2, true, false, true) KV_SET(3, true, false, true)
+  KV_SET(1, false, false, kKeyQ8) KV_SET(1, false, true, kKeyQ8) KV_SET(2, true, false, kKeyQ8)
+  KV_SET(2, true, true, kKeyQ8) KV_SET(3, true, false, kKeyQ8) KV_SET(3, true, true, kKeyQ8)
+  KV_SET(1, false, false, kKeyQ4) KV_SET(2, true, false, kKeyQ4) KV_SET(3, true, false, kKeyQ4)
+  KV_SET(1, false, false, kKeyQ51) KV_SET(2, true, false, kKeyQ51) KV_SET(3, true, false, kKeyQ51)
 #undef KV_SET
   return cudaSuccess;
 }
 
-// Q8_0 keys with Q4_0 or Q8_0 values, and Q4_0 keys with Q4_0 values.
-cudaError_t launch_decode(const DecodeParams& prm, int n_kv, bool kq4, bool vq8, cudaStream_t stream) {
+// Q8_0 keys with Q4_0 or Q8_0 values; Q4_0 or Q5_1 keys with Q4_0 values.
+template <int KF>
+static cudaError_t launch_decode_v4(const DecodeParams& prm, int n_kv, int nt, cudaStream_t stream) {
+  if (nt == 1) return launch_decode_t<1, false, false, KF>(prm, n_kv, stream);
+  if (nt == 2) return launch_decode_t<2, true, false, KF>(prm, n_kv, stream);
+  return launch_decode_t<3, true, false, KF>(prm, n_kv, stream);
+}
+
+cudaError_t launch_decode(const DecodeParams& prm, int n_kv, int key_fmt, bool vq8, cudaStream_t stream) {
   const int nt = decode_rows_pad(prm.group * prm.n_q) / 8;
-  if (kq4) {
-    if (vq8) return cudaErrorInvalidValue;
-    if (nt == 1) return launch_decode_t<1, false, false, true>(prm, n_kv, stream);
-    if (nt == 2) return launch_decode_t<2, true, false, true>(prm, n_kv, stream);
-    return launch_decode_t<3, true, false, true>(prm, n_kv, stream);
-  }
-  if (nt == 1)
-    return vq8 ? launch_decode_t<1, false, true, false>(prm, n_kv, stream)
-               : launch_decode_t<1, false, false, false>(prm, n_kv, stream);
-  if (nt == 2)
-    return vq8 ? launch_decode_t<2, true, true, false>(prm, n_kv, stream)
-               : launch_decode_t<2, true, false, false>(prm, n_kv, stream);
-  return vq8 ? launch_decode_t<3, true, true, false>(prm, n_kv, stream)
-             : launch_decode_t<3, true, false, false>(prm, n_kv, stream);
+  if (key_fmt != kKeyQ8 && vq8) return cudaErrorInvalidValue;
+  if (key_fmt == kKeyQ4) return launch_decode_v4<kKeyQ4>(prm, n_kv, nt, stream);
+  if (key_fmt == kKeyQ51) return launch_decode_v4<kKeyQ51>(prm, n_kv, nt, stream);
+  if (!vq8) return launch_decode_v4<kKeyQ8>(prm, n_kv, nt, stream);
+  if (nt == 1) return launch_decode_t<1, false, true, kKeyQ8>(prm, n_kv, stream);
+  if (nt == 2) return launch_decode_t<2, true, true, kKeyQ8>(prm, n_kv, stream);
+  return launch_decode_t<3, true, true, kKeyQ8>(prm, n_kv, stream);
 }
 
 }  // namespace kvattn

@@ -21,7 +21,7 @@ struct DecodeParams {
   int n_q, group, n_qh, max_pages, n_splits;
 };
 
-cudaError_t launch_decode(const DecodeParams& prm, int n_kv, bool kq4, bool vq8, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams& prm, int n_kv, int key_fmt, bool vq8, cudaStream_t stream);
 cudaError_t prepare_decode_kernels();
 
 }  // namespace kvattn

@@ -1,4 +1,4 @@
-// Q8_0 / Q4_0 encoders that append new tokens into their KV pages.
+// Q8_0 / Q4_0 / Q5_1 encoders that append new tokens into their KV pages.
 //
 // Formats (Vulkan speculative-decoding report, lcz.me/topic/1398, "pitfalls" and
 // "configs"): 32-element blocks with one fp16 scale; Q8_0 stores int8 codes (8.5 bits per
@@ -7,11 +7,14 @@
 //   Q8_0: d = amax / 127, q = round-half-away(x * fp32(1/d)), |q| <= 127.
 //   Q4_0: m = the signed element of largest magnitude (first on ties), d = m / -8,
 //         q = min(15, floor(fp32(fp32(x * fp32(1/d)) + 8.5))).
+//   Q5_1 (same report, pitfalls: 5-bit codes with a zero point, 6 bits per element):
+//         m = the block minimum, d = fp32(fp32(max - m) / 31),
+//         q = min(31, floor(fp32(fp32(fp32(x - m) * fp32(1/d)) + 0.5))), value q * d + m.
 // Every operation that decides a code is an IEEE fp32 operation with round-to-nearest
 // (no FMA contraction), so the codes equal those of any correct fp32 implementation.
 //
 // One warp encodes one (token, KV head) row: lane l owns channels [8l, 8l+8), four lanes
-// form one 32-element block.  Keys are stored as Q8_0 or Q4_0, values as Q4_0 or Q8_0.
+// form one 32-element block.  Keys are stored as Q8_0, Q4_0 or Q5_1, values as Q4_0 or Q8_0.
 #include "common.cuh"
 
 namespace kvattn {
@@ -67,13 +70,18 @@ __device__ __forceinline__ float q4_scale(const float (&x)[8], int lane, float* 
   return d;
 }
 
+__device__ __forceinline__ int q51_code(float x, float mn, float inv) {
+  const float y = __fmul_rn(__fsub_rn(x, mn), inv);
+  return min(31, __float2int_rz(__fadd_rn(y, 0.5f)));  // y >= 0, so truncation is floor
+}
+
 __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __restrict__ k,
                                                               const float* __restrict__ v, int n_tok,
                                                               int n_kv, int32_t pos0,
                                                               const int32_t* __restrict__ page_table,
                                                               int n_blocks, uint8_t* k_pool, int64_t k_stride,
                                                               uint8_t* v_pool, int64_t v_stride, int64_t n_pages,
-                                                              int k_q4, int v_q8) {
+                                                              int k_fmt, int v_q8) {
   // a kernel launched behind this one with programmatic dependent launch (decode) may start
   // its setup now; it waits for this grid to complete before reading the pages
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -99,8 +107,46 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
   const int G = tok >> 4, tl = tok & 15, H = tl >> 3, R = tok & 7;
   const int b = lane >> 2;  // this lane's block
 
+  // ---------------- K: Q5_1 ----------------
+  if (k_fmt == kKeyQ51) {
+    const float x[8] = {kx0.x, kx0.y, kx0.z, kx0.w, kx1.x, kx1.y, kx1.z, kx1.w};
+    float mn = x[0], mx = x[0];
+#pragma unroll
+    for (int e = 1; e < 8; ++e) {
+      mn = fminf(mn, x[e]);
+      mx = fmaxf(mx, x[e]);
+    }
+#pragma unroll
+    for (int s = 1; s <= 2; s <<= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, s));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
+    }
+    const float d = __fdiv_rn(__fsub_rn(mx, mn), 31.f);
+    const float inv = d != 0.f ? __frcp_rn(d) : 0.f;
+    const int T = lane & 3, c = b & 3, Q = b >> 2;
+    // low nibbles as the Q4_0 key word; fifth bits of the four blocks 4Q..4Q+3 of this T
+    // (lanes T + 4c + 16Q) gathered into one word, channel (c, e) at bit 16(e%2) + 4c + e/2
+    uint32_t w = 0, hb = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t q = static_cast<uint32_t>(q51_code(x[e], mn, inv));
+      w |= (q & 15u) << (4 * (e >> 1) + 16 * (e & 1));
+      hb |= (q >> 4) << (16 * (e & 1) + 4 * c + (e >> 1));
+    }
+    hb |= __shfl_xor_sync(0xffffffffu, hb, 4);
+    hb |= __shfl_xor_sync(0xffffffffu, hb, 8);
+    uint8_t* pg = k_pool + static_cast<int64_t>(page) * k_stride;
+    const int row = (((G * 2 + Q) * 2 + H) * 8 + R) * 4 + T;
+    *reinterpret_cast<uint32_t*>(pg + 4 * (row * 4 + c)) = w;
+    if (c == 0) *reinterpret_cast<uint32_t*>(pg + kK5HighOffset + 4 * row) = hb;
+    if ((lane & 3) == 0) {
+      const int si = 2 * (((G * 8 + R) * 2 + H) * 8 + b);
+      *reinterpret_cast<__half*>(pg + kK5ScaleOffset + si) = __float2half_rn(d);
+      *reinterpret_cast<__half*>(pg + kK5MinOffset + si) = __float2half_rn(mn);
+    }
+  }
   // ---------------- K: Q4_0 ----------------
-  if (k_q4) {
+  else if (k_fmt == kKeyQ4) {
     const float x[8] = {kx0.x, kx0.y, kx0.z, kx0.w, kx1.x, kx1.y, kx1.z, kx1.w};
     float inv;
     const float d = q4_scale(x, lane, &inv);
@@ -205,7 +251,7 @@ cudaError_t launch_quantize_append(const kvattn_kv_desc& desc, const float* k, c
   return cudaLaunchKernelEx(&cfg, quantize_append_kernel, k, v, n_tok, desc.n_kv_heads, pos0, page_table, n_blocks,
                             static_cast<uint8_t*>(desc.k_pool), desc.k_page_stride,
                             static_cast<uint8_t*>(desc.v_pool), desc.v_page_stride, desc.n_pages,
-                            static_cast<int>(desc.k_fmt == KVATTN_FMT_Q4_0),
+                            desc.k_fmt == KVATTN_FMT_Q4_0 ? kKeyQ4 : desc.k_fmt == KVATTN_FMT_Q5_1 ? kKeyQ51 : kKeyQ8,
                             static_cast<int>(desc.v_fmt == KVATTN_FMT_Q8_0));
 }
 

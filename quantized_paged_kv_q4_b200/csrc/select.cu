@@ -3,11 +3,12 @@
 // fill a 32,768-token GPU budget, and a 16,384-token recent reserve is always kept).
 //
 // Readings (the pages do not define the ranking):
-//   summary[b][c] = mean over the block's 128 tokens of the dequantized key, rounded once
-//                   to fp32.  Computed exactly: each fp16 scale is split into an 11-bit
-//                   integer significand and an exponent, every code x significand product is
-//                   shifted onto a common 2^-24 grid and summed in int64 (< 2^54, no
-//                   overflow), then converted to fp32 with one rounding.
+//   summary[b][c] = mean over the block's 128 tokens of the dequantized key (Q8_0, Q4_0 or
+//                   Q5_1), rounded once to fp32.  Computed exactly: each fp16 scale (and
+//                   Q5_1 minimum) is split into an 11-bit integer significand and an
+//                   exponent, every code x significand product is shifted onto a common
+//                   2^-24 grid and summed in int64 (< 2^54, no overflow), then converted to
+//                   fp32 with one rounding.
 //   score[b]      = sum_c (sum_j q[j][c]) * summary[b][c] in fp64.
 //   selection     = the `budget` highest scores among blocks older than the recent window
 //                   (ties: lower block index), plus the recent window and partial tail
@@ -17,10 +18,21 @@
 namespace kvattn {
 
 // ---------------------------------------------------------------- summaries
+// q * h for an fp16 bit pattern h, exactly, in units of 2^-24 (the fp16 subnormal step):
+// h = +-m * 2^(eff - 25) with m the 11-bit significand.  |q| <= 127 keeps it below 2^47.
+__device__ __forceinline__ long long fp16_grid_units(uint16_t h, int q) {
+  const int e = (h >> 10) & 31;
+  const int mant = h & 1023;
+  const int m = e ? (1024 | mant) : mant;
+  const int eff = e ? e : 1;
+  const long long term = static_cast<long long>(q * m) * (1ll << (eff - 1));
+  return (h & 0x8000) ? -term : term;
+}
+
 __global__ void __launch_bounds__(256) block_summary_kernel(const uint8_t* __restrict__ k_pool, int64_t k_stride,
                                                             int64_t n_pages, const int32_t* __restrict__ page_table,
                                                             int n_blocks, int block_begin, int n_range,
-                                                            int k_q4, float* __restrict__ summaries) {
+                                                            int k_fmt, float* __restrict__ summaries) {
   __shared__ __align__(16) uint8_t page[kKPageBytes];
   const int unit = blockIdx.y;
   const int b = block_begin + blockIdx.x;
@@ -31,8 +43,8 @@ __global__ void __launch_bounds__(256) block_summary_kernel(const uint8_t* __res
   }
   const uint4* src = reinterpret_cast<const uint4*>(k_pool + static_cast<int64_t>(pg) * k_stride);
   uint4* dst = reinterpret_cast<uint4*>(page);
-  const int bytes = k_q4 ? kK4PageBytes : kKPageBytes;
-  const int scale_off = k_q4 ? kK4ScaleOffset : kKScaleOffset;
+  const int bytes = k_fmt == kKeyQ4 ? kK4PageBytes : k_fmt == kKeyQ51 ? kK5PageBytes : kKPageBytes;
+  const int scale_off = k_fmt == kKeyQ4 ? kK4ScaleOffset : k_fmt == kKeyQ51 ? kK5ScaleOffset : kKScaleOffset;
   for (int i = threadIdx.x; i < bytes / 16; i += blockDim.x) dst[i] = src[i];
   __syncthreads();
   const int c = threadIdx.x;  // channel
@@ -45,20 +57,22 @@ __global__ void __launch_bounds__(256) block_summary_kernel(const uint8_t* __res
   for (int tok = 0; tok < kPageTokens; ++tok) {
     const int G = tok >> 4, H = (tok & 15) >> 3, R = tok & 7;
     int q;
-    if (k_q4) {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(
-          page + 4 * (((((G * 2 + (blk >> 2)) * 2 + H) * 8 + R) * 4 + T) * 4 + (blk & 3)));
-      q = static_cast<int>((w >> nib_shift) & 15u) - 8;
+    if (k_fmt != kKeyQ8) {
+      const int row = (((G * 2 + (blk >> 2)) * 2 + H) * 8 + R) * 4 + T;
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(page + 4 * (row * 4 + (blk & 3)));
+      q = static_cast<int>((w >> nib_shift) & 15u);
+      if (k_fmt == kKeyQ4) {
+        q -= 8;
+      } else {
+        const uint32_t fifth = *reinterpret_cast<const uint32_t*>(page + kK5HighOffset + 4 * row);
+        q |= static_cast<int>((fifth >> (16 * (i8 & 1) + 4 * (blk & 3) + (i8 >> 1))) & 1u) << 4;
+      }
     } else {
       q = static_cast<int8_t>(page[((((G * 4 + P) * 2 + H) * 8 + R) * 4 + T) * 16 + j]);
     }
-    const uint16_t hb = *reinterpret_cast<const uint16_t*>(page + scale_off + 2 * (((G * 8 + R) * 2 + H) * 8 + blk));
-    const int e = (hb >> 10) & 31;
-    const int mant = hb & 1023;
-    const int m = e ? (1024 | mant) : mant;
-    const int eff = e ? e : 1;
-    const long long term = static_cast<long long>(q * m) * (1ll << (eff - 1));
-    acc += (hb & 0x8000) ? -term : term;
+    const int si = 2 * (((G * 8 + R) * 2 + H) * 8 + blk);
+    acc += fp16_grid_units(*reinterpret_cast<const uint16_t*>(page + scale_off + si), q);
+    if (k_fmt == kKeyQ51) acc += fp16_grid_units(*reinterpret_cast<const uint16_t*>(page + kK5MinOffset + si), 1);
   }
   // value = acc * 2^-24 / 128
   const float r = __ll2float_rn(acc) * 4.656612873077392578125e-10f;  // 2^-31
@@ -262,7 +276,10 @@ cudaError_t launch_block_summaries(const kvattn_kv_desc& d, const int32_t* page_
   dim3 grid(n, n_units);
   block_summary_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(d.k_pool), d.k_page_stride, d.n_pages,
                                                  page_table, n_blocks, block_begin, n,
-                                                 static_cast<int>(d.k_fmt == KVATTN_FMT_Q4_0), summaries);
+                                                 d.k_fmt == KVATTN_FMT_Q4_0   ? kKeyQ4
+                                                 : d.k_fmt == KVATTN_FMT_Q5_1 ? kKeyQ51
+                                                                              : kKeyQ8,
+                                                 summaries);
   return cudaGetLastError();
 }
 

@@ -28,9 +28,10 @@ ERR_NOT_INITIALIZED = -9
 
 FMT_Q4_0 = 4
 FMT_Q8_0 = 8
+FMT_Q5_1 = 51
 ROLE_K = 0
 ROLE_V = 1
-FMT = {"q4_0": FMT_Q4_0, "q8_0": FMT_Q8_0}
+FMT = {"q4_0": FMT_Q4_0, "q8_0": FMT_Q8_0, "q5_1": FMT_Q5_1}
 
 
 class KVAttnError(RuntimeError):

@@ -159,6 +159,8 @@ WORKLOADS = {
                                 n_q=1, v_fmt="q8_0", outlier_frac=0.01, seed=2003),
     "decode131k_q4q4": Workload("decode131k_q4q4", layers=16, kv_heads=4, q_heads=24, context=131072,
                                 n_q=1, k_fmt="q4_0", v_fmt="q4_0", outlier_frac=0.01, seed=2004),
+    "decode131k_q51q4": Workload("decode131k_q51q4", layers=16, kv_heads=4, q_heads=24, context=131072,
+                                 n_q=1, k_fmt="q5_1", v_fmt="q4_0", outlier_frac=0.01, seed=2005),
     # 262,144 prior tokens, 4 verify tokens, 20 needles, budget 256 + recent 128 blocks.
     "verify262k": Workload("verify262k", layers=16, kv_heads=4, q_heads=24, context=262144, n_q=4,
                            needles=20, budget_blocks=256, recent_blocks=128, seed=3003),

@@ -52,6 +52,8 @@ def test_status_strings_and_page_sizes(lib):
     assert kvattn.kvattn_page_bytes(kvattn.ROLE_V, kvattn.FMT_Q4_0) == 18432
     assert kvattn.kvattn_page_bytes(kvattn.ROLE_V, kvattn.FMT_Q8_0) == 34816
     assert kvattn.kvattn_page_bytes(kvattn.ROLE_K, kvattn.FMT_Q4_0) == 18432
+    assert kvattn.kvattn_page_bytes(kvattn.ROLE_K, kvattn.FMT_Q5_1) == 24576
+    assert kvattn.kvattn_page_bytes(kvattn.ROLE_V, kvattn.FMT_Q5_1) == 0
     assert kvattn.kvattn_page_bytes(kvattn.ROLE_K, 5) == 0
 
 
@@ -80,11 +82,14 @@ def test_host_validation_rejects_bad_arguments(lib):
     bad = _desc(v_fmt="q8_0")
     bad.k_fmt = kvattn.FMT_Q4_0
     assert L.kvattn_decode(by(bad), 16, 1, 16, 16, None, None, 1, 16, 16, None, 0, None) == kvattn.ERR_UNSUPPORTED_FORMAT
-    # Q4_0 keys: decode and the summaries take them; chunked prefill refuses them
-    k4 = _desc(k_fmt="q4_0")
-    assert L.kvattn_decode_workspace_size(by(k4), 1, 1024) == L.kvattn_decode_workspace_size(by(d), 1, 1024)
-    assert L.kvattn_prefill_chunk(by(k4), 16, 1, 16, 16, None, None, 1, 4096, 16, 16, 16, 1 << 20, None) == \
-        kvattn.ERR_UNSUPPORTED_FORMAT
+    # Q4_0 / Q5_1 keys: decode and the summaries take them; chunked prefill refuses them
+    for kf in ("q4_0", "q5_1"):
+        kd = _desc(k_fmt=kf)
+        assert L.kvattn_decode_workspace_size(by(kd), 1, 1024) == L.kvattn_decode_workspace_size(by(d), 1, 1024)
+        assert L.kvattn_prefill_chunk(by(kd), 16, 1, 16, 16, None, None, 1, 4096, 16, 16, 16, 1 << 20, None) == \
+            kvattn.ERR_UNSUPPORTED_FORMAT
+    bad = _desc(k_fmt="q5_1", v_fmt="q8_0")
+    assert L.kvattn_decode(by(bad), 16, 1, 16, 16, None, None, 1, 16, 16, None, 0, None) == kvattn.ERR_UNSUPPORTED_FORMAT
     bad = _desc(n_q_heads=25)
     assert L.kvattn_decode(by(bad), 16, 1, 16, 16, None, None, 1, 16, 16, None, 0, None) == kvattn.ERR_INVALID_ARG
     bad = _desc(k_pool=16 * 1000 + 8)

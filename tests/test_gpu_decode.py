@@ -42,7 +42,7 @@ def _run_decode(kv, cache, H_q, q, q_pos, page_list, page_logical=None, n_pages=
     return out.cpu().numpy(), lse.cpu().numpy(), (qd, qp, pl, lg, npg, out, lse, ws, wsb)
 
 
-@pytest.mark.parametrize("k_fmt,v_fmt", [("q8_0", "q4_0"), ("q8_0", "q8_0"), ("q4_0", "q4_0")])
+@pytest.mark.parametrize("k_fmt,v_fmt", [("q8_0", "q4_0"), ("q8_0", "q8_0"), ("q4_0", "q4_0"), ("q5_1", "q4_0")])
 @pytest.mark.parametrize("n_q", [1, 2, 3, 4])
 def test_decode_matches_oracle(kv_gpu, k_fmt, v_fmt, n_q):
     H, H_q, T = 4, 24, 37 * 128 + 77          # ragged tail page

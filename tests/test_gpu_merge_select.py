@@ -54,7 +54,7 @@ def _select_case(seed, H, n_full, tail, budget, recent, needles, group=6, k_fmt=
 
 @pytest.mark.parametrize("seed,n_full,tail,budget,recent,k_fmt", [
     (900, 300, 37, 64, 32, "q8_0"), (901, 2048, 4, 256, 128, "q8_0"), (902, 50, 0, 80, 10, "q8_0"),
-    (903, 40, 100, 8, 0, "q8_0"), (904, 300, 37, 64, 32, "q4_0")])
+    (903, 40, 100, 8, 0, "q8_0"), (904, 300, 37, 64, 32, "q4_0"), (905, 300, 37, 64, 32, "q5_1")])
 def test_summaries_and_selection_bit_exact(kv_gpu, seed, n_full, tail, budget, recent, k_fmt):
     H = 4
     rng, k, v, q, cache, needle_sets, n_blocks, T = _select_case(seed, H, n_full, tail, budget, recent,

@@ -9,7 +9,7 @@ from synth import normal_f32, np_rng, page_permutation
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("k_fmt,v_fmt", [("q8_0", "q4_0"), ("q8_0", "q8_0"), ("q4_0", "q4_0")])
+@pytest.mark.parametrize("k_fmt,v_fmt", [("q8_0", "q4_0"), ("q8_0", "q8_0"), ("q4_0", "q4_0"), ("q5_1", "q4_0")])
 def test_append_bytes_bit_exact(kv_gpu, k_fmt, v_fmt):
     rng = np_rng(501)
     H, T, n_blocks = 4, 3 * 128 + 50, 5
@@ -27,6 +27,8 @@ def test_append_bytes_bit_exact(kv_gpu, k_fmt, v_fmt):
     v[9, 3, 1:4] = [-0.125, 0.125, 1.875]
     v[11, 0, :32] = 3.0                      # ties of the largest magnitude: first index wins
     v[11, 0, 4] = -3.0
+    k[13, 1, 32:64] = 0.0                    # Q5_1 halves: m = -1, d = 0.25, (x - m) / d = k + 0.5
+    k[13, 1, 32:37] = [-1.0, 6.75, -0.875, 6.625, -0.4375]
     n_phys = H * n_blocks + 3
     cache = GpuCache(H, 24, n_blocks, v_fmt, n_phys=n_phys, perm=page_permutation(rng, n_phys), k_fmt=k_fmt)
     for a, b in ((0, 100), (100, 101), (101, 300), (300, T)):
