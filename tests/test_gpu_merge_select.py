@@ -76,7 +76,7 @@ def test_summaries_and_selection_bit_exact(kv_gpu, seed, n_full, tail, budget, r
     s_gpu = summ.cpu().numpy()
     for h in range(H):
         kc = oc.kc[: n_full * 128, h].reshape(n_full, 128, 8, 32)
-        kd = oc.kd[: n_full * 128, h].reshape(n_full, 128, 8)
+        kd = oc.kd[: n_full * 128, h].reshape((n_full, 128) + oc.kd.shape[2:])  # (d, m) pairs for Q5_1
         s_ref = osel.block_summaries(kc, kd, k_fmt)
         assert np.array_equal(s_gpu[h, :n_full].view(np.uint32), s_ref.view(np.uint32))
         scores = osel.block_scores(s_ref[:n_cand], q[h])
