@@ -4,8 +4,8 @@ Each test builds one layer of a benchmark workload through the benchmark's own c
 context length, head counts, page table, split plan and launch sequence as every timed
 layer), runs that layer once, and checks outputs against the oracle:
 
-* decode, 131,072 tokens (Q8_0 K with Q4_0 or Q8_0 V): every output row of the layer, plus
-  page bytes of sampled blocks bit-exact;
+* decode, 131,072 tokens (Q8_0 K with Q4_0 or Q8_0 V, Q4_0 or Q5_1 K with Q4_0 V): every
+  output row of the layer, plus page bytes of sampled blocks bit-exact;
 * MTP verify, 262,144 tokens + 4: the selection bit-exact (needles included) and the 4 x 24
   rows over the selected blocks, for two sampled KV heads;
 * chunked prefill, 524,288 prior tokens + the 2,048-token chunk: 64 seeded (token, query head)
@@ -34,16 +34,16 @@ def _head(x, h):
     return x[:, h].contiguous().cpu().numpy()
 
 
-def _oracle_unit(k, v, h, v_fmt, k_tail=None, v_tail=None):
+def _oracle_unit(k, v, h, v_fmt, k_tail=None, v_tail=None, k_fmt="q8_0"):
     """OracleCache of KV head h: the workload's draws, then the appended tokens."""
     kh, vh = _head(k, h), _head(v, h)
     if k_tail is not None:
         kh = np.concatenate([kh, k_tail[:, h].cpu().numpy()], 0)
         vh = np.concatenate([vh, v_tail[:, h].cpu().numpy()], 0)
-    return OracleCache(kh[:, None], vh[:, None], v_fmt)
+    return OracleCache(kh[:, None], vh[:, None], v_fmt, k_fmt)
 
 
-@pytest.mark.parametrize("wname", ["decode131k", "decode131k_q8q8"])
+@pytest.mark.parametrize("wname", ["decode131k", "decode131k_q8q8", "decode131k_q4q4", "decode131k_q51q4"])
 def test_decode_full_context(kv_gpu, wname):
     b = bench.DecodeBench(kv_gpu, wname, torch.device(DEV), layers=1)
     b.layer(0)
@@ -59,7 +59,7 @@ def test_decode_full_context(kv_gpu, wname):
     pt = b.cache.page_table[0].cpu().numpy()
     rng = np_rng(7100)
     for h in range(w.kv_heads):
-        oc = _oracle_unit(k, v, h, w.v_fmt)
+        oc = _oracle_unit(k, v, h, w.v_fmt, k_fmt=w.k_fmt)
         for blk in [0, b.nb - 1] + rng.choice(b.nb, 4, replace=False).tolist():
             phys = int(pt[h, blk])
             assert np.array_equal(b.cache.k_pool[phys].cpu().numpy(), oc.page_bytes(0, blk, "k"))
