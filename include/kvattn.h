@@ -88,7 +88,7 @@ enum kvattn_status {
   KVATTN_OK = 0,
   KVATTN_ERR_INVALID_ARG = -1,        /* null pointer, bad size or alignment, bad range     */
   KVATTN_ERR_UNSUPPORTED_ARCH = -2,   /* device is not compute capability 10.0 (sm_100)     */
-  KVATTN_ERR_UNSUPPORTED_FORMAT = -3, /* format / head_dim / page size this build lacks     */
+  KVATTN_ERR_UNSUPPORTED_FORMAT = -3, /* format / head_dim / page size not supported        */
   KVATTN_ERR_BAD_PAGE = -4,           /* a page id outside [0, n_pages) (device-side check) */
   KVATTN_ERR_WORKSPACE_TOO_SMALL = -5,
   KVATTN_ERR_CUDA = -6,               /* a CUDA runtime call failed; see kvattn_last_cuda_error */
