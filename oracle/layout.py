@@ -6,7 +6,7 @@ pages fix only the bits per element; the arrangement below is this library's own
 storage spec, written so that one 16-byte load per thread feeds tensor-core
 fragments directly.  Bytes per page equal the AoS block sizes the pages print:
 K Q8_0 = 128 x 8 x 34 = 34,816; K Q4_0 = V Q4_0 = 128 x 8 x 18 = 18,432; K Q5_1 = 128 x 8 x 24
-= 24,576; V Q8_0 = 34,816.
+= 24,576; K Q5_0 = 128 x 8 x 22 = 22,528; V Q4_1 = 128 x 8 x 20 = 20,480; V Q8_0 = 34,816.
 
 Notation: tok in [0,128) is the token slot inside the page, dim in [0,256) the
 channel, b = dim // 32 the block, d[tok][b] the fp16 block scale.  Tokens are
@@ -35,6 +35,10 @@ K page, Q5_1 (24,576 bytes)
   scales d, bytes [20480, 22528), and minima m, bytes [22528, 24576): fp16 at base + 2*idx
   with idx the K Q8_0 scale index ((G*8 + R)*2 + H)*8 + b.  The value is q * d + m.
 
+K page, Q5_0 (22,528 bytes)
+  low nibbles and fifth bits as the K Q5_1 page, bytes [0, 20480); scales d, bytes
+  [20480, 22528), as the K Q5_1 scales.  The value is (q - 16) * d.
+
 V page, Q4_0 (18,432 bytes)
   nibbles, bytes [0, 16384): byte at
       ((((G*4 + C)*8 + R)*4 + T)*16 + 4*w + y            (C<4, R<8, T<4, w<4, y<4)
@@ -43,6 +47,10 @@ V page, Q4_0 (18,432 bytes)
   A nibble stores q in [0, 15]; the value is (q - 8) * d.
   scales, bytes [16384, 18432): fp16 at 16384 + 2*((((G*4 + T)*8 + b)*4) + k)
   holds d[16G + 2T + (k % 2) + 8*(k // 2)][b]                (k < 4).
+
+V page, Q4_1 (20,480 bytes)
+  nibbles, bytes [0, 16384), and scales d, bytes [16384, 18432), as the V Q4_0 page; minima m,
+  bytes [18432, 20480), in the arrangement of the scales.  The value is q * d + m.
 
 V page, Q8_0 (34,816 bytes)
   codes, bytes [0, 32768): byte at
@@ -62,6 +70,8 @@ N_BLOCKS = HEAD_DIM // 32
 K_Q8_BYTES = 34816
 K_Q4_BYTES = 18432
 K_Q51_BYTES = 24576
+K_Q50_BYTES = 22528
+V_Q41_BYTES = 20480
 V_Q4_BYTES = 18432
 V_Q8_BYTES = 34816
 
@@ -73,6 +83,10 @@ def page_bytes(role: str, fmt: str) -> int:
         return K_Q4_BYTES
     if role == "k" and fmt == "q5_1":
         return K_Q51_BYTES
+    if role == "k" and fmt == "q5_0":
+        return K_Q50_BYTES
+    if role == "v" and fmt == "q4_1":
+        return V_Q41_BYTES
     if role == "v" and fmt == "q4_0":
         return V_Q4_BYTES
     if role == "v" and fmt == "q8_0":
@@ -160,22 +174,36 @@ def _flat_codes(codes: np.ndarray) -> np.ndarray:
 
 
 def encode_page(role: str, fmt: str, codes: np.ndarray, d: np.ndarray) -> np.ndarray:
-    """Encode one page.  codes: [128][8][32] (int8 for Q8_0, 0..15 for Q4_0, 0..31 for Q5_1);
-    d: [128][8] float16 ([128][8][2] (d, m) for Q5_1).  Returns uint8[page_bytes]."""
+    """Encode one page.  codes: [128][8][32] (int8 for Q8_0, 0..15 for Q4_0 / Q4_1, 0..31 for
+    Q5_0 / Q5_1); d: [128][8] float16 ([128][8][2] (d, m) for Q4_1 and Q5_1).  Returns
+    uint8[page_bytes]."""
     n = page_bytes(role, fmt)
     out = np.zeros(n, dtype=np.uint8)
     c = _flat_codes(codes)
     d16 = np.asarray(d, dtype=np.float16).view(np.uint16)
-    if role == "k" and fmt == "q5_1":
+    if role == "k" and fmt in ("q5_1", "q5_0"):
         c8 = c.astype(np.uint8)
         if np.any(c8 > 31):
-            raise ValueError("Q5_1 codes must be in [0, 31]")
+            raise ValueError("5-bit codes must be in [0, 31]")
         off, sh, tok, dim = _K4_NIBBLES
         np.bitwise_or.at(out, off, ((c8[tok, dim] & 15) << sh).astype(np.uint8))
         off, sh, tok, dim = _K5_HIGH
         np.bitwise_or.at(out, off, ((c8[tok, dim] >> 4) << sh).astype(np.uint8))
         idx, tok, b = _K_SCALES
-        for base, part in ((20480, d16[..., 0]), (22528, d16[..., 1])):
+        parts = ((20480, d16[..., 0]), (22528, d16[..., 1])) if fmt == "q5_1" else ((20480, d16),)
+        for base, part in parts:
+            sv = part[tok, b]
+            out[base + 2 * idx] = (sv & 0xFF).astype(np.uint8)
+            out[base + 2 * idx + 1] = (sv >> 8).astype(np.uint8)
+        return out
+    if role == "v" and fmt == "q4_1":
+        off, tok, lo, hi = _V4_NIBBLES
+        c8 = c.astype(np.uint8)
+        if np.any(c8 > 15):
+            raise ValueError("Q4_1 codes must be in [0, 15]")
+        out[off] = c8[tok, lo] | (c8[tok, hi] << 4)
+        idx, tok, b = _V_SCALES
+        for base, part in ((16384, d16[..., 0]), (18432, d16[..., 1])):
             sv = part[tok, b]
             out[base + 2 * idx] = (sv & 0xFF).astype(np.uint8)
             out[base + 2 * idx + 1] = (sv >> 8).astype(np.uint8)
@@ -218,14 +246,25 @@ def decode_page(role: str, fmt: str, page: np.ndarray):
     if page.size != page_bytes(role, fmt):
         raise ValueError("wrong page size")
     c = np.zeros((PAGE_TOKENS, HEAD_DIM), dtype=np.int16)
-    if role == "k" and fmt == "q5_1":
+    if role == "k" and fmt in ("q5_1", "q5_0"):
         off, sh, tok, dim = _K4_NIBBLES
         c[tok, dim] = (page[off] >> sh) & 0xF
         off, sh, tok, dim = _K5_HIGH
         c[tok, dim] |= ((page[off] >> sh) & 1).astype(np.int16) << 4
         idx, tok, b = _K_SCALES
+        bases = (20480, 22528) if fmt == "q5_1" else (20480,)
+        dm = np.zeros((PAGE_TOKENS, N_BLOCKS, len(bases)), dtype=np.uint16)
+        for j, base in enumerate(bases):
+            dm[tok, b, j] = page[base + 2 * idx].astype(np.uint16) | (page[base + 2 * idx + 1].astype(np.uint16) << 8)
+        dm = dm.view(np.float16)
+        return c.astype(np.uint8).reshape(PAGE_TOKENS, N_BLOCKS, 32), (dm if fmt == "q5_1" else dm[..., 0])
+    if role == "v" and fmt == "q4_1":
+        off, tok, lo, hi = _V4_NIBBLES
+        c[tok, lo] = page[off] & 0xF
+        c[tok, hi] = page[off] >> 4
+        idx, tok, b = _V_SCALES
         dm = np.zeros((PAGE_TOKENS, N_BLOCKS, 2), dtype=np.uint16)
-        for j, base in enumerate((20480, 22528)):
+        for j, base in enumerate((16384, 18432)):
             dm[tok, b, j] = page[base + 2 * idx].astype(np.uint16) | (page[base + 2 * idx + 1].astype(np.uint16) << 8)
         return c.astype(np.uint8).reshape(PAGE_TOKENS, N_BLOCKS, 32), dm.view(np.float16)
     if role == "k" and fmt == "q4_0":

@@ -1,4 +1,4 @@
-"""Q8_0, Q4_0 and Q5_1 block quantisation -- CPU oracle (test infrastructure only).
+"""Q8_0, Q4_0, Q5_0, Q4_1 and Q5_1 block quantisation -- CPU oracle (test infrastructure only).
 
 Both formats split a row into blocks of 32 elements and store one fp16 scale
 ``d`` per block (Vulkan speculative-decoding report, lcz.me/topic/1398, section
@@ -25,6 +25,13 @@ The pages do not spell out the encoders.  The readings used here:
   difference, the product and the sum each rounded to fp32; d and m are stored as fp16.
   ``max == min`` gives d = 0 and q = 0.  The scale pair is carried as one float16 array
   [..., n, 2] holding (d, m).
+
+* Q5_0 and Q4_1 (named with Q5_1 in the same section's list of KV formats; the MTP tuning
+  notes on one 7900 XTX, lcz.me/topic/593, run a Q5_0 K / Q4_1 V cache at 128K): Q5_0 is
+  Q4_0 with 5-bit codes, value = (q - 16) * d, ``d = m / -16``, ``q = min(31, floor(x *
+  (1/d) + 16.5))`` (22 bytes per block); Q4_1 is Q5_1 with 4-bit codes, value = q * d + m,
+  ``d = (max - min) / 15``, ``q = min(15, floor((x - m) * (1/d) + 0.5))`` (20 bytes per
+  block).  Same rounding rules as Q4_0 and Q5_1.
 
 Every rounding that decides an integer code is done in fp32, exactly as an IEEE
 fp32 unit would do it, so a GPU encoder can match the codes bit for bit.
@@ -76,17 +83,38 @@ def q8_0_dequantize(qs: np.ndarray, d: np.ndarray) -> np.ndarray:
     return v.reshape(v.shape[:-2] + (-1,))
 
 
-def q4_0_quantize(x: np.ndarray):
-    """x: fp32 [..., 32n] -> (q uint8 in [0,15] [..., n, 32], d float16 [..., n])."""
+def _offset_quantize(x: np.ndarray, half: int):
+    """Symmetric codes with offset `half` (8 for Q4_0, 16 for Q5_0): m = the signed element of
+    largest magnitude (first on ties), d = m / -half, q = min(2 half - 1, floor(x/d + half + .5))."""
     xb = _blocks(x)
     idx = np.argmax(np.abs(xb), axis=-1)
     m = np.take_along_axis(xb, idx[..., None], axis=-1)[..., 0]
-    d32 = (m / F32(-8.0)).astype(F32)
+    d32 = (m / F32(-half)).astype(F32)
     inv = _recip_f32(d32)
     y = (xb * inv[..., None]).astype(F32)
-    z = (y + F32(8.5)).astype(F32)
-    q = np.minimum(15, np.floor(z.astype(np.float64)))
+    z = (y + F32(half + 0.5)).astype(F32)
+    q = np.minimum(2 * half - 1, np.floor(z.astype(np.float64)))
     return q.astype(np.uint8), d32.astype(np.float16)
+
+
+def _min_quantize(x: np.ndarray, top: int):
+    """Codes with a zero point (top = 15 for Q4_1, 31 for Q5_1): m = the block minimum,
+    d = (max - m) / top, q = min(top, floor((x - m)/d + 0.5)); returns (q, (d, m))."""
+    xb = _blocks(x)
+    mn = np.min(xb, axis=-1)
+    mx = np.max(xb, axis=-1)
+    d32 = ((mx - mn).astype(F32) / F32(top)).astype(F32)
+    inv = _recip_f32(d32)
+    y = ((xb - mn[..., None]).astype(F32) * inv[..., None]).astype(F32)
+    z = (y + F32(0.5)).astype(F32)
+    q = np.minimum(top, np.floor(z.astype(np.float64)))
+    dm = np.stack([d32.astype(np.float16), mn.astype(np.float16)], axis=-1)
+    return q.astype(np.uint8), dm
+
+
+def q4_0_quantize(x: np.ndarray):
+    """x: fp32 [..., 32n] -> (q uint8 in [0,15] [..., n, 32], d float16 [..., n])."""
+    return _offset_quantize(x, 8)
 
 
 def q4_0_dequantize(q: np.ndarray, d: np.ndarray) -> np.ndarray:
@@ -95,35 +123,51 @@ def q4_0_dequantize(q: np.ndarray, d: np.ndarray) -> np.ndarray:
     return v.reshape(v.shape[:-2] + (-1,))
 
 
+def q5_0_quantize(x: np.ndarray):
+    """x: fp32 [..., 32n] -> (q uint8 in [0,31] [..., n, 32], d float16 [..., n])."""
+    return _offset_quantize(x, 16)
+
+
+def q5_0_dequantize(q: np.ndarray, d: np.ndarray) -> np.ndarray:
+    """(q [..., n, 32], d [..., n]) -> float64 [..., 32n], value = (q - 16) * d."""
+    v = (q.astype(np.float64) - 16.0) * d.astype(np.float64)[..., None]
+    return v.reshape(v.shape[:-2] + (-1,))
+
+
 def q5_1_quantize(x: np.ndarray):
     """x: fp32 [..., 32n] -> (q uint8 in [0,31] [..., n, 32], (d, m) float16 [..., n, 2])."""
-    xb = _blocks(x)
-    mn = np.min(xb, axis=-1)
-    mx = np.max(xb, axis=-1)
-    d32 = ((mx - mn).astype(F32) / F32(31.0)).astype(F32)
-    inv = _recip_f32(d32)
-    y = ((xb - mn[..., None]).astype(F32) * inv[..., None]).astype(F32)
-    z = (y + F32(0.5)).astype(F32)
-    q = np.minimum(31, np.floor(z.astype(np.float64)))
-    dm = np.stack([d32.astype(np.float16), mn.astype(np.float16)], axis=-1)
-    return q.astype(np.uint8), dm
+    return _min_quantize(x, 31)
 
 
-def q5_1_dequantize(q: np.ndarray, dm: np.ndarray) -> np.ndarray:
-    """(q [..., n, 32], (d, m) [..., n, 2]) -> float64 [..., 32n], value = q * d + m."""
+def q4_1_quantize(x: np.ndarray):
+    """x: fp32 [..., 32n] -> (q uint8 in [0,15] [..., n, 32], (d, m) float16 [..., n, 2])."""
+    return _min_quantize(x, 15)
+
+
+def min_dequantize(q: np.ndarray, dm: np.ndarray) -> np.ndarray:
+    """Q4_1 / Q5_1: (q [..., n, 32], (d, m) [..., n, 2]) -> float64 [..., 32n], value = q * d + m."""
     dm = np.asarray(dm, dtype=np.float16).astype(np.float64)
     v = q.astype(np.float64) * dm[..., 0][..., None] + dm[..., 1][..., None]
     return v.reshape(v.shape[:-2] + (-1,))
 
 
+q5_1_dequantize = min_dequantize
+q4_1_dequantize = min_dequantize
+
+_QUANT = {"q8_0": q8_0_quantize, "q4_0": q4_0_quantize, "q5_0": q5_0_quantize, "q4_1": q4_1_quantize,
+          "q5_1": q5_1_quantize}
+_DEQUANT = {"q8_0": q8_0_dequantize, "q4_0": q4_0_dequantize, "q5_0": q5_0_dequantize,
+            "q4_1": min_dequantize, "q5_1": min_dequantize}
+
+
 def quantize(x: np.ndarray, fmt: str):
-    return {"q8_0": q8_0_quantize, "q4_0": q4_0_quantize, "q5_1": q5_1_quantize}[fmt](x)
+    return _QUANT[fmt](x)
 
 
 def dequantize(codes: np.ndarray, d: np.ndarray, fmt: str) -> np.ndarray:
-    return {"q8_0": q8_0_dequantize, "q4_0": q4_0_dequantize, "q5_1": q5_1_dequantize}[fmt](codes, d)
+    return _DEQUANT[fmt](codes, d)
 
 
 def block_bytes(fmt: str) -> int:
     """Bytes of one 32-element block: fp16 scale (and fp16 minimum) + codes."""
-    return {"q8_0": 2 + 32, "q4_0": 2 + 16, "q5_1": 2 + 2 + 20}[fmt]
+    return {"q8_0": 2 + 32, "q4_0": 2 + 16, "q5_0": 2 + 20, "q4_1": 2 + 2 + 16, "q5_1": 2 + 2 + 20}[fmt]

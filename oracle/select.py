@@ -34,12 +34,12 @@ def _grid(v: np.ndarray) -> np.ndarray:
 
 
 def block_summaries(codes: np.ndarray, d: np.ndarray, fmt: str = "q8_0") -> np.ndarray:
-    """Mean dequantised key of each block, keys stored as Q8_0, Q4_0 or Q5_1.
+    """Mean dequantised key of each block, keys stored as Q8_0, Q4_0, Q5_0 or Q5_1.
 
-    codes: [n_blocks][128][8][32] (int8 for Q8_0, 0..15 for Q4_0, 0..31 for Q5_1); d:
-    float16 [n_blocks][128][8] ([n_blocks][128][8][2] = (d, m) for Q5_1).  Returns fp32
-    [n_blocks][256].  The key value is q * d for Q8_0, (q - 8) * d for Q4_0 and q * d + m
-    for Q5_1.
+    codes: [n_blocks][128][8][32] (int8 for Q8_0, 0..15 for Q4_0, 0..31 for Q5_0 / Q5_1);
+    d: float16 [n_blocks][128][8] ([n_blocks][128][8][2] = (d, m) for Q5_1).  Returns fp32
+    [n_blocks][256].  The key value is q * d for Q8_0, (q - 8) * d for Q4_0, (q - 16) * d
+    for Q5_0 and q * d + m for Q5_1.
 
     Each product d * q is exact in float64 (11 + 8 significant bits) and, like each
     minimum m, a multiple of the block's smallest fp16 grid step; when the sum of
@@ -47,13 +47,13 @@ def block_summaries(codes: np.ndarray, d: np.ndarray, fmt: str = "q8_0") -> np.n
     below is the exact sum (checked, not assumed).  Division by 128 is exact; the one
     rounding is the final conversion to fp32.
     """
-    if fmt not in ("q8_0", "q4_0", "q5_1"):
+    if fmt not in ("q8_0", "q4_0", "q5_0", "q5_1"):
         raise ValueError(f"unsupported key format {fmt}")
     codes = np.asarray(codes)
     nb = codes.shape[0]
     dd = np.asarray(d, dtype=np.float16).astype(np.float64)
     d64 = dd[..., 0] if fmt == "q5_1" else dd                         # [nb][128][8]
-    q = codes.astype(np.float64) - (8.0 if fmt == "q4_0" else 0.0)
+    q = codes.astype(np.float64) - {"q4_0": 8.0, "q5_0": 16.0}.get(fmt, 0.0)
     terms = [q * d64[..., None]]                                      # [nb][128][8][32]
     grids = [_grid(d64)]
     if fmt == "q5_1":

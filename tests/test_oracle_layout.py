@@ -16,7 +16,8 @@ def _page(fmt, seed):
     return quant.quantize(x, fmt)
 
 
-@pytest.mark.parametrize("role,fmt", [("k", "q8_0"), ("k", "q4_0"), ("k", "q5_1"), ("v", "q4_0"), ("v", "q8_0")])
+@pytest.mark.parametrize("role,fmt", [("k", "q8_0"), ("k", "q4_0"), ("k", "q5_1"), ("k", "q5_0"), ("v", "q4_0"),
+                                      ("v", "q8_0"), ("v", "q4_1")])
 def test_round_trip(role, fmt):
     codes, d = _page(fmt, 11)
     page = layout.encode_page(role, fmt, codes, d)
@@ -91,6 +92,29 @@ def test_k_q5_1_scale_and_minimum_offsets():
     page = layout.encode_page("k", "q5_1", np.zeros((128, 8, 32), np.uint8), dm)
     assert np.flatnonzero(page).tolist() == [20480 + 2 * 27 + 1, 22528 + 2 * 27 + 1]
     assert page[20480 + 55] == 0x3C and page[22528 + 55] == 0x40
+
+
+def test_k_q5_0_matches_q5_1_codes_and_scales_without_minima():
+    codes = np.zeros((128, 8, 32), np.uint8)
+    codes[5, 6, 8], codes[9, 3, 31] = 16, 27
+    d = np.zeros((128, 8), np.float16)
+    d[9, 3] = 1.0
+    dm = np.zeros((128, 8, 2), np.float16)
+    dm[..., 0] = d
+    p50 = layout.encode_page("k", "q5_0", codes, d)
+    p51 = layout.encode_page("k", "q5_1", codes, dm)
+    assert p50.size == 22528 and np.array_equal(p50, p51[:22528]) and not p51[22528:].any()
+
+
+def test_v_q4_1_matches_q4_0_nibbles_and_scales_plus_minima():
+    codes = np.zeros((128, 8, 32), np.uint8)
+    codes[10, 2, 17] = 6
+    dm = np.zeros((128, 8, 2), np.float16)
+    dm[10, 2, 0], dm[10, 2, 1] = 1.0, 2.0     # token 10 of block 2 -> scale index 42
+    p41 = layout.encode_page("v", "q4_1", codes, dm)
+    p40 = layout.encode_page("v", "q4_0", codes, dm[..., 0])
+    assert p41.size == 20480 and np.array_equal(p41[:18432], p40)
+    assert np.flatnonzero(p41[18432:]).tolist() == [2 * 42 + 1] and p41[18432 + 85] == 0x40
 
 
 def test_k_scale_offsets():

@@ -185,3 +185,81 @@ def test_q5_1_constant_block():
     q, dm = quant.q5_1_quantize(np.full(32, 1.5, np.float32))
     assert dm[0, 0] == 0 and dm[0, 1] == np.float16(1.5) and np.all(q == 0)
     assert np.all(quant.q5_1_dequantize(q, dm) == 1.5)
+
+
+def test_q5_0_and_q4_1_bits_per_element():
+    assert quant.block_bytes("q5_0") * 8 / 32 == 5.5
+    assert quant.block_bytes("q4_1") * 8 / 32 == 5.0
+
+
+@pytest.mark.parametrize("outliers", [False, True])
+def test_q5_0_error_bound(outliers):
+    x = _x(10, 256, outliers).reshape(-1, 32)
+    q, d = quant.q5_0_quantize(x)
+    xh = quant.q5_0_dequantize(q, d).reshape(-1, 32)
+    idx = np.argmax(np.abs(x), axis=1)
+    m = x[np.arange(x.shape[0]), idx]
+    d32 = (m / np.float32(-16)).astype(np.float32).astype(np.float64)
+    d16 = d.astype(np.float64).reshape(-1)
+    # |x - (q - 16) d32| <= |d32| / 2 (1 at the clamp q = 31) plus rounding slack, then the
+    # fp16 scale moves each value by at most 16 |d32 - d16|
+    err = np.abs(x - xh)
+    bound = np.abs(d32) * (1.0 + 1e-5) + 16 * np.abs(d32 - d16)
+    assert np.all(err <= bound[:, None])
+    assert np.all(q <= 31)
+    # the largest-magnitude element maps to code 0, and m = -16 d up to the fp16 rounding
+    assert np.all(q.reshape(-1, 32)[np.arange(x.shape[0]), idx] == 0)
+    assert np.allclose(-16.0 * d16, m, rtol=2.0 ** -11)
+
+
+def test_q5_0_round_trip_halves_and_zero_block():
+    rng = np_rng(11)
+    d = 0.125
+    q = rng.integers(0, 32, size=(8, 32)).astype(np.uint8)
+    q[:, 5] = 0                               # value -16 d: the largest magnitude
+    x = ((q.astype(np.float32) - 16) * np.float32(d))
+    qq, dd = quant.q5_0_quantize(x)
+    assert np.array_equal(qq.reshape(q.shape), q) and np.all(dd.astype(np.float64) == d)
+    # exact halves: y = -0.5 -> 16, +0.5 -> 17, 15.5 -> clamp 31
+    x = np.zeros(32, np.float32)
+    x[0] = -16 * d
+    x[1:4] = [-0.5 * d, 0.5 * d, 15.5 * d]
+    qq, _ = quant.q5_0_quantize(x)
+    assert list(qq[0, :4]) == [0, 16, 17, 31]
+    q0, d0 = quant.q5_0_quantize(np.zeros(32, np.float32))
+    assert d0[0] == 0 and np.all(q0 == 16) and np.all(quant.q5_0_dequantize(q0, d0) == 0)
+
+
+@pytest.mark.parametrize("outliers", [False, True])
+def test_q4_1_error_bound_and_extremes(outliers):
+    x = _x(12, 256, outliers).reshape(-1, 32)
+    q, dm = quant.q4_1_quantize(x)
+    xh = quant.q4_1_dequantize(q, dm).reshape(-1, 32)
+    mn = x.min(axis=1).astype(np.float64)
+    d32 = ((x.max(axis=1) - x.min(axis=1)).astype(np.float32) / np.float32(15)).astype(np.float32).astype(np.float64)
+    d16 = dm[:, 0, 0].astype(np.float64)
+    m16 = dm[:, 0, 1].astype(np.float64)
+    bound = d32 * (0.5 + 1e-5) + 15 * np.abs(d32 - d16) + np.abs(mn - m16)
+    assert np.all(np.abs(x - xh) <= bound[:, None])
+    q = q.reshape(-1, 32)
+    rows = np.arange(x.shape[0])
+    assert np.all(q[rows, np.argmin(x, axis=1)] == 0) and np.all(q[rows, np.argmax(x, axis=1)] == 15)
+
+
+def test_q4_1_round_trip_halves_and_constant_block():
+    rng = np_rng(13)
+    d, m = 0.5, -3.0
+    q = rng.integers(0, 16, size=(8, 32)).astype(np.uint8)
+    q[:, 0], q[:, 1] = 0, 15
+    x = (q.astype(np.float32) * np.float32(d) + np.float32(m)).astype(np.float32)
+    qq, dm = quant.q4_1_quantize(x)
+    assert np.array_equal(qq.reshape(q.shape), q)
+    assert np.array_equal(quant.q4_1_dequantize(qq, dm).reshape(q.shape), x.astype(np.float64))
+    # exact halves round up: (x - m) / d = 0.5 -> 1, 14.5 -> 15, 6.25 -> 6
+    x = np.zeros(32, np.float32)
+    x[0], x[1] = m, m + 15 * d
+    x[2:5] = [m + 0.5 * d, m + 14.5 * d, m + 6.25 * d]
+    qq, _ = quant.q4_1_quantize(x)
+    assert list(qq[0, :5]) == [0, 15, 1, 15, 6]
+    q0, dm0 = quant.q4_1_quantize(np.full(32, -0.75, np.float32))
+    assert dm0[0, 0] == 0 and dm0[0, 1] == np.float16(-0.75) and np.all(q0 == 0)

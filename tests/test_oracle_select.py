@@ -62,6 +62,20 @@ def test_q5_1_key_summaries_equal_correctly_rounded_mean():
     assert np.all(const == np.float32(-2.5))
 
 
+def test_q5_0_key_summaries_equal_correctly_rounded_mean():
+    x = normal_f32(np_rng(26), (2, 128, 256))
+    qs, d = quant.q5_0_quantize(x)
+    s = select.block_summaries(qs, d, "q5_0")
+    k = quant.q5_0_dequantize(qs, d)
+    for b in range(2):
+        for c in range(0, 256, 7):
+            assert s[b, c] == np.float32(math.fsum(k[b, :, c].tolist()) / 128.0)
+    # code 11 of a Q5_0 block is the value (11 - 16) * d
+    const = select.block_summaries(np.full((1, 128, 8, 32), 11, np.uint8), np.full((1, 128, 8), np.float16(0.25)),
+                                   "q5_0")
+    assert np.all(const == np.float32(-1.25))
+
+
 def test_summary_of_a_constant_block():
     qs = np.full((1, 128, 8, 32), -5, np.int8)
     d = np.full((1, 128, 8), np.float16(0.375))
