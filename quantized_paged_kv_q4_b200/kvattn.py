@@ -1,7 +1,9 @@
 """Thin ctypes binding of libkvattn (include/kvattn.h).
 
 Argument marshalling only: every computation runs in the CUDA library.  Pointer arguments
-accept torch tensors (their data_ptr), plain integers (raw addresses) or None; stream
+accept torch tensors (their data_ptr), plain integers (raw addresses) or None; a tensor must
+be contiguous, on the GPU for device-memory arguments and on the host for the pinned host
+pools (anything else raises ValueError before the library is called); stream
 arguments accept torch.cuda.Stream objects, raw handles or None (the current torch
 stream).  A nonzero status raises KVAttnError.  If libkvattn.so is missing the import of
 any entry point fails loudly: there is no fallback implementation.
@@ -102,11 +104,26 @@ def lib():
     return _lib
 
 
-def _p(x):
-    if x is None:
-        return None
-    if isinstance(x, int):
+def _d(x):
+    """A device-memory argument: a contiguous CUDA tensor, a raw address (int) or None.  A CPU
+    tensor is refused here: its address would reach a kernel as device memory."""
+    if x is None or isinstance(x, int):
         return x
+    if not x.is_cuda:
+        raise ValueError(f"expected a CUDA tensor for a device-memory argument, got one on {x.device}")
+    if not x.is_contiguous():
+        raise ValueError("expected a contiguous tensor (the library reads dense row-major arrays)")
+    return x.data_ptr()
+
+
+def _h(x):
+    """A host-memory argument (pinned pools): a contiguous CPU tensor, a raw address or None."""
+    if x is None or isinstance(x, int):
+        return x
+    if x.is_cuda:
+        raise ValueError("expected a host (pinned CPU) tensor for a host-memory argument")
+    if not x.is_contiguous():
+        raise ValueError("expected a contiguous tensor (the library reads dense row-major arrays)")
     return x.data_ptr()
 
 
@@ -133,7 +150,7 @@ def status_string(status: int) -> str:
 def make_desc(n_kv_heads, n_q_heads, k_pool, v_pool, n_pages, v_fmt="q4_0", k_page_stride=None,
               v_page_stride=None, head_dim=256, page_tokens=128, k_fmt="q8_0") -> kvattn_kv_desc:
     kf, vf = FMT[k_fmt] if isinstance(k_fmt, str) else k_fmt, FMT[v_fmt] if isinstance(v_fmt, str) else v_fmt
-    return kvattn_kv_desc(n_kv_heads, n_q_heads, head_dim, page_tokens, kf, vf, _p(k_pool), _p(v_pool),
+    return kvattn_kv_desc(n_kv_heads, n_q_heads, head_dim, page_tokens, kf, vf, _d(k_pool), _d(v_pool),
                           k_page_stride or kvattn_page_bytes(ROLE_K, kf), v_page_stride or kvattn_page_bytes(ROLE_V, vf),
                           n_pages)
 
@@ -160,7 +177,7 @@ def kvattn_page_bytes(role: int, fmt: int) -> int:
 
 
 def kvattn_quantize_append(desc, k, v, n_tok, pos0, page_table, n_blocks, stream=None) -> None:
-    _check(lib().kvattn_quantize_append(ctypes.byref(desc), _p(k), _p(v), n_tok, pos0, _p(page_table), n_blocks,
+    _check(lib().kvattn_quantize_append(ctypes.byref(desc), _d(k), _d(v), n_tok, pos0, _d(page_table), n_blocks,
                                         _s(stream)), "kvattn_quantize_append")
 
 
@@ -170,28 +187,28 @@ def kvattn_decode_workspace_size(desc, n_q, max_pages) -> int:
 
 def kvattn_decode(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pages, out, lse, ws, ws_bytes,
                   stream=None) -> None:
-    _check(lib().kvattn_decode(ctypes.byref(desc), _p(q), n_q, _p(q_pos), _p(page_list), _p(page_logical),
-                               _p(n_pages), max_pages, _p(out), _p(lse), _p(ws), ws_bytes, _s(stream)),
+    _check(lib().kvattn_decode(ctypes.byref(desc), _d(q), n_q, _d(q_pos), _d(page_list), _d(page_logical),
+                               _d(n_pages), max_pages, _d(out), _d(lse), _d(ws), ws_bytes, _s(stream)),
            "kvattn_decode")
 
 
 def kvattn_decode_noalloc(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pages, out, lse,
                           stream=None) -> None:
     """kvattn_decode without a caller workspace (scratch in a fixed device array of the library)."""
-    _check(lib().kvattn_decode_noalloc(ctypes.byref(desc), _p(q), n_q, _p(q_pos), _p(page_list), _p(page_logical),
-                                       _p(n_pages), max_pages, _p(out), _p(lse), _s(stream)),
+    _check(lib().kvattn_decode_noalloc(ctypes.byref(desc), _d(q), n_q, _d(q_pos), _d(page_list), _d(page_logical),
+                                       _d(n_pages), max_pages, _d(out), _d(lse), _s(stream)),
            "kvattn_decode_noalloc")
 
 
 def kvattn_merge_lse(o_parts, lse_parts, n_parts, rows, dim, out, lse, stream=None) -> None:
-    _check(lib().kvattn_merge_lse(_p(o_parts), _p(lse_parts), n_parts, rows, dim, _p(out), _p(lse), _s(stream)),
+    _check(lib().kvattn_merge_lse(_d(o_parts), _d(lse_parts), n_parts, rows, dim, _d(out), _d(lse), _s(stream)),
            "kvattn_merge_lse")
 
 
 def kvattn_block_summaries(desc, page_table, n_units, n_blocks, block_begin, block_end, summaries,
                            stream=None) -> None:
-    _check(lib().kvattn_block_summaries(ctypes.byref(desc), _p(page_table), n_units, n_blocks, block_begin,
-                                        block_end, _p(summaries), _s(stream)), "kvattn_block_summaries")
+    _check(lib().kvattn_block_summaries(ctypes.byref(desc), _d(page_table), n_units, n_blocks, block_begin,
+                                        block_end, _d(summaries), _s(stream)), "kvattn_block_summaries")
 
 
 def kvattn_select_workspace_size(n_units, n_blocks) -> int:
@@ -200,8 +217,8 @@ def kvattn_select_workspace_size(n_units, n_blocks) -> int:
 
 def kvattn_select_blocks(summaries, q_group, n_units, group, n_blocks, n_full, n_total, budget, recent, page_table,
                          sel_logical, sel_phys, n_sel, cap, ws, ws_bytes, stream=None) -> None:
-    _check(lib().kvattn_select_blocks(_p(summaries), _p(q_group), n_units, group, n_blocks, n_full, n_total, budget,
-                                      recent, _p(page_table), _p(sel_logical), _p(sel_phys), _p(n_sel), cap, _p(ws),
+    _check(lib().kvattn_select_blocks(_d(summaries), _d(q_group), n_units, group, n_blocks, n_full, n_total, budget,
+                                      recent, _d(page_table), _d(sel_logical), _d(sel_phys), _d(n_sel), cap, _d(ws),
                                       ws_bytes, _s(stream)), "kvattn_select_blocks")
 
 
@@ -211,24 +228,24 @@ def kvattn_prefill_workspace_size(desc, n_q, max_pages, kv_split_tokens) -> int:
 
 def kvattn_prefill_chunk(desc, q_bf16, n_q, q_pos, page_list, page_logical, n_pages, max_pages, kv_split_tokens, out,
                          lse, ws, ws_bytes, stream=None) -> None:
-    _check(lib().kvattn_prefill_chunk(ctypes.byref(desc), _p(q_bf16), n_q, _p(q_pos), _p(page_list),
-                                      _p(page_logical), _p(n_pages), max_pages, kv_split_tokens, _p(out), _p(lse),
-                                      _p(ws), ws_bytes, _s(stream)), "kvattn_prefill_chunk")
+    _check(lib().kvattn_prefill_chunk(ctypes.byref(desc), _d(q_bf16), n_q, _d(q_pos), _d(page_list),
+                                      _d(page_logical), _d(n_pages), max_pages, kv_split_tokens, _d(out), _d(lse),
+                                      _d(ws), ws_bytes, _s(stream)), "kvattn_prefill_chunk")
 
 
 def kvattn_gather_pages(host_pool, host_stride, n_host_pages, dev_pool, dev_stride, n_slots, page_bytes, host_ids,
                         dev_slots, n, n_ctas=0, stream=None) -> None:
     """Host (pinned, mapped) -> device page copy driven by device-side page lists."""
-    _check(lib().kvattn_gather_pages(_p(host_pool), host_stride, n_host_pages, _p(dev_pool), dev_stride, n_slots,
-                                     page_bytes, _p(host_ids), _p(dev_slots), n, n_ctas, _s(stream)),
+    _check(lib().kvattn_gather_pages(_h(host_pool), host_stride, n_host_pages, _d(dev_pool), dev_stride, n_slots,
+                                     page_bytes, _d(host_ids), _d(dev_slots), n, n_ctas, _s(stream)),
            "kvattn_gather_pages")
 
 
 def kvattn_scatter_pages(host_pool, host_stride, n_host_pages, dev_pool, dev_stride, n_slots, page_bytes, host_ids,
                          dev_slots, n, n_ctas=0, stream=None) -> None:
     """Device -> host (pinned, mapped) page copy driven by device-side page lists."""
-    _check(lib().kvattn_scatter_pages(_p(host_pool), host_stride, n_host_pages, _p(dev_pool), dev_stride, n_slots,
-                                      page_bytes, _p(host_ids), _p(dev_slots), n, n_ctas, _s(stream)),
+    _check(lib().kvattn_scatter_pages(_h(host_pool), host_stride, n_host_pages, _d(dev_pool), dev_stride, n_slots,
+                                      page_bytes, _d(host_ids), _d(dev_slots), n, n_ctas, _s(stream)),
            "kvattn_scatter_pages")
 
 
@@ -236,7 +253,7 @@ def kvattn_hadamard(x, out=None, rows=None, stream=None):
     """out = x R over rows of 256 fp32 values (R = H_256 / 16); in place when out is None."""
     out = x if out is None else out
     n = rows if rows is not None else x.numel() // 256
-    _check(lib().kvattn_hadamard(_p(x), _p(out), n, _s(stream)), "kvattn_hadamard")
+    _check(lib().kvattn_hadamard(_d(x), _d(out), n, _s(stream)), "kvattn_hadamard")
     return out
 
 
@@ -245,10 +262,10 @@ def kvattn_resident_update(sel_logical, n_sel, cap, n_units, n_blocks, n_full, s
                            n_copies, stream=None) -> None:
     """Resident-page reuse: update each unit's slot pool for its new selection and write the
     decode page list and the copy list of the misses (all device arrays)."""
-    _check(lib().kvattn_resident_update(_p(sel_logical), _p(n_sel), cap, n_units, n_blocks, n_full,
-                                        _p(slot_of_block), _p(block_of_slot), n_slots, _p(host_page_of_block),
-                                        first_page, _p(extra_page), _p(page_list), _p(copy_host), _p(copy_dst),
-                                        _p(n_copies), _s(stream)),
+    _check(lib().kvattn_resident_update(_d(sel_logical), _d(n_sel), cap, n_units, n_blocks, n_full,
+                                        _d(slot_of_block), _d(block_of_slot), n_slots, _d(host_page_of_block),
+                                        first_page, _d(extra_page), _d(page_list), _d(copy_host), _d(copy_dst),
+                                        _d(n_copies), _s(stream)),
            "kvattn_resident_update")
 
 
@@ -293,7 +310,7 @@ def kvattn_stream_pages(host_pool, host_stride, dev_pool, dev_stride, page_bytes
     d, dp = _host_i32(dev_slots)
     n_copies = c_int(0)
     ev = None if done is None else _event_handle(done, copy_stream)
-    _check(lib().kvattn_stream_pages(_p(host_pool), host_stride, _p(dev_pool), dev_stride, page_bytes, hp, dp,
+    _check(lib().kvattn_stream_pages(_h(host_pool), host_stride, _d(dev_pool), dev_stride, page_bytes, hp, dp,
                                      int(h.size), _s(copy_stream), ev, ctypes.byref(n_copies)),
            "kvattn_stream_pages")
     return n_copies.value

@@ -147,3 +147,21 @@ def test_resident_update_validation(lib):
         a = list(args)
         a[i] = v
         assert f(*a) == kvattn.ERR_INVALID_ARG
+
+
+def test_binding_refuses_host_tensors_for_device_arguments(lib):
+    import torch
+
+    d = _desc()
+    q_cpu = torch.zeros((1, 24, 256))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        kvattn.kvattn_decode(d, q_cpu, 1, 16, 16, None, None, 1, 16, 16, None, 0, stream=0)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        kvattn.kvattn_hadamard(torch.zeros((2, 256)), stream=0)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        kvattn.make_desc(1, 6, torch.zeros(64, dtype=torch.uint8), 16, 1)
+    # a host pool must be a host tensor
+    with pytest.raises(ValueError, match="host"):
+        kvattn._h(type("FakeCuda", (), {"is_cuda": True})())
+    with pytest.raises(ValueError, match="contiguous"):
+        kvattn._h(torch.zeros((4, 4)).t())
