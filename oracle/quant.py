@@ -53,10 +53,18 @@ def _blocks(x: np.ndarray) -> np.ndarray:
 
 
 def _recip_f32(d: np.ndarray) -> np.ndarray:
-    """1/d rounded to fp32, and 0 where d == 0."""
+    """1/d rounded to fp32, and 0 where d == 0.
+
+    A nonzero fp32 scale whose reciprocal overflows (|d| below about 2.9e-39: a block whose
+    elements, or whose spread for the zero-point formats, are all below about 1e-36) has no
+    defined codes under these readings; such blocks are outside the supported input range and
+    are refused."""
     out = np.zeros_like(d, dtype=F32)
     nz = d != 0
-    out[nz] = F32(1.0) / d[nz]
+    with np.errstate(over="ignore"):
+        out[nz] = F32(1.0) / d[nz]
+    if not np.all(np.isfinite(out)):
+        raise ValueError("block scale so small that 1/d overflows fp32: outside the supported input range")
     return out
 
 
