@@ -140,7 +140,9 @@ KVATTN_API int64_t kvattn_page_bytes(int role, int fmt);
  * clamped to +-127.  Q4_0: m = the element of largest magnitude, d = m/-8, q = min(15,
  * floor(x * fp32(1/d) + 8.5)).  Q5_1: m = the block minimum, d = (max - m)/31, q = min(31,
  * floor((x - m) * fp32(1/d) + 0.5)).  Every step that decides a code is rounded to fp32;
- * scales and minima are stored as fp16.
+ * scales and minima are stored as fp16.  A block whose fp32 scale is nonzero but has no
+ * finite fp32 reciprocal (all elements, or for Q5_1 the spread, below about 1e-36) is outside
+ * the supported range: its codes are unspecified and it decodes to 0.
  *   k, v        device fp32 [n_tok][H_kv][256]
  *   pos0        position of the first token; token i goes to logical block (pos0+i)/128,
  *               slot (pos0+i)%128
