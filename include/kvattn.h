@@ -295,8 +295,8 @@ KVATTN_API int kvattn_scatter_pages(void* host_pool, int64_t host_stride, int64_
                                     int64_t dev_stride, int64_t n_slots, int64_t page_bytes, const int32_t* host_ids,
                                     const int32_t* dev_slots, int n, int n_ctas, kvattn_stream_t stream);
 
-/* ---- attention rotation (Vulkan/ROCm long-context report, section on attention
- * rotation: the rotation improves the precision of quantized KV) --------------------------
+/* ---- attention rotation ([VULKAN] pitfalls, the attention-rotation item: the rotation
+ * improves the precision of quantized KV) ------------------------------------------------
  * out[r] = in[r] R for `rows` rows of 256 fp32 values, R = H_256 / 16 with H the
  * Sylvester-Hadamard matrix (H[i][j] = (-1)^popcount(i & j)).  R is symmetric, orthonormal
  * and its own inverse.  The rotated pipeline: rotate K and V before kvattn_quantize_append,

@@ -2,9 +2,9 @@
 
 Test infrastructure only.
 
-The Vulkan/ROCm long-context report (lcz.me/topic/1398, section on attention rotation) runs
-q8_0 / q5_1 / q4_0 KV caches with the attention rotation on and notes that the rotation
-improves the precision of the quantized KV.  The page does not write the transform out; the
+The Vulkan speculative-decoding report, 7900 XTX (lcz.me/topic/1398), in its pitfalls
+section (the item on attention rotation), runs q8_0 / q5_1 / q4_0 KV caches with the
+attention rotation on and notes that the rotation improves the precision of the quantized KV.  The page does not write the transform out; the
 reading used here (the plainest one, and the one that keeps attention unchanged in exact
 arithmetic):
 

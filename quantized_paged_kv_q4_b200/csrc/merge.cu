@@ -77,8 +77,8 @@ cudaError_t launch_merge_lse(const float* o_parts, const float* lse_parts, int n
 namespace kvattn {
 
 // x R for rows of 256 fp32 values, R = H_256 / 16 with H the Sylvester-Hadamard matrix
-// (symmetric, orthonormal, its own inverse): the attention rotation of the Vulkan/ROCm
-// long-context report (section on attention rotation), which spreads outlier channels
+// (symmetric, orthonormal, its own inverse): the attention rotation of the Vulkan
+// speculative-decoding report (pitfalls section, attention-rotation item), which spreads outlier channels
 // before quantization.  One warp per row; lane l holds elements 8l .. 8l + 7: the three low
 // index bits are butterflied in registers, the five high ones across lanes by shuffles.
 // `in` may equal `out`.
