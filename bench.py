@@ -4,10 +4,11 @@
 Headline (one JSON line on rank 0): decode at 131,072 context -- 16 layers x 4 KV heads x
 head_dim 256, 24 query heads, 1 query token, Q8_0 K / Q4_0 V pages in a seeded shuffled page
 table.  One step = for every layer: quantize-append the new token's K/V, then split-KV decode
-(with the fused LSE merge).  value = algorithmic KV bytes read per step (416 B per token, KV
-head and layer) / device time per step, in GB/s.  The other workloads (Q8_0/Q8_0 decode,
-MTP verify at 262K with block selection, ...) are measured in the same run and reported under
-"extra".
+(with its split-merge grid).  value = algorithmic KV bytes read per step (416 B per token, KV
+head and layer) / device time per step, in GB/s.  The other workloads (the Q8_0/Q8_0,
+Q4_0/Q4_0 and Q5_1/Q4_0 decodes, MTP verify at 262K with block selection, chunked prefill at
+524K, host-streamed decode with and without resident-page reuse) are measured in the same run
+and reported under "extra".
 
 --impl reference times the CPU oracle (float64 NumPy) on the host cores on the same workload
 and metric, each step a bounded sample of it.
