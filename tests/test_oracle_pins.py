@@ -29,6 +29,8 @@ def test_sizes_printed_on_the_pages():
     bpe_q4 = quant.block_bytes("q4_0") / 32
     assert per_token * 2 * bpe_q4 == g["q4_0_kv_bytes_per_token"]
     assert quant.block_bytes("q8_0") * 8 * 2 // 32 == g["q8_0_bits_per_element_x2"]
+    assert quant.block_bytes("q5_1") * 8 / 32 == g["q5_1_bits_per_element"]
+    assert round(100 * (quant.block_bytes("q5_1") / quant.block_bytes("q4_0") - 1)) == g["q5_1_over_q4_0_key_bits_pct"]
     bt = g["block_tokens"]
     assert 62080 // bt == g["blocks_in_62080_tokens"] and 62080 % bt == 0
     assert 32768 // bt == g["blocks_in_budget_32768"]
@@ -42,6 +44,10 @@ def test_page_sizes_follow_block_sizes():
     assert layout.page_bytes("k", "q8_0") == 128 * 8 * quant.block_bytes("q8_0") == 34816
     assert layout.page_bytes("v", "q4_0") == 128 * 8 * quant.block_bytes("q4_0") == 18432
     assert layout.page_bytes("v", "q8_0") == 34816
+    assert layout.page_bytes("k", "q4_0") == 18432
+    assert layout.page_bytes("k", "q5_1") == 128 * 8 * quant.block_bytes("q5_1") == 24576
+    assert layout.page_bytes("k", "q5_0") == 128 * 8 * quant.block_bytes("q5_0") == 22528
+    assert layout.page_bytes("v", "q4_1") == 128 * 8 * quant.block_bytes("q4_1") == 20480
 
 
 def test_decode_bytes_per_step():
