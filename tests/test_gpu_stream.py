@@ -137,3 +137,16 @@ def test_streamed_working_set_decode(kv_gpu):
         keys = keys[keys < T]
         o_ref, l_ref = oc.attend(q, [T - 1], h, g, key_idx=keys)
         compare(out[:, g * h:g * h + g].cpu().numpy(), lse[:, g * h:g * h + g].cpu().numpy(), o_ref, l_ref)
+
+
+def test_stream_wait_times_out_then_completes(kv_gpu):
+    """An event behind a bounded busy kernel (at least 0.75 s) has not fired after 20 ms:
+    the wait returns TIMEOUT and the context stays usable; a longer wait then succeeds."""
+    s = torch.cuda.Stream()
+    ev = torch.cuda.Event()
+    with torch.cuda.stream(s):
+        torch.cuda._sleep(int(1.5e9))          # clock cycles; ends by itself
+        ev.record(s)
+    assert kv_gpu.kvattn_stream_wait(ev, 20) == kv_gpu.ERR_TIMEOUT
+    assert kv_gpu.kvattn_stream_wait(ev, 10000) == kv_gpu.OK
+    assert kv_gpu.kvattn_device_error() == 0
