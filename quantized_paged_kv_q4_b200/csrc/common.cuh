@@ -23,9 +23,13 @@ constexpr int kK5PageBytes = 24576;     // Q5_1 keys: 128 x 8 x (20 + 2 + 2)
 constexpr int kK5HighOffset = 16384;    // fifth code bits, after the low nibbles
 constexpr int kK5ScaleOffset = 20480;
 constexpr int kK5MinOffset = 22528;
-// key formats as kernel template / flag values
-constexpr int kKeyQ8 = 0, kKeyQ4 = 1, kKeyQ51 = 2;
+constexpr int kK50PageBytes = 22528;    // Q5_0 keys: 128 x 8 x (20 + 2); nibbles and fifth bits as Q5_1
+// key and value formats as kernel template / flag values
+constexpr int kKeyQ8 = 0, kKeyQ4 = 1, kKeyQ51 = 2, kKeyQ50 = 3;
+constexpr int kValQ4 = 0, kValQ8 = 1, kValQ41 = 2;
 constexpr int kV4PageBytes = 18432;     // Q4_0: 128 x 8 x (16 + 2)
+constexpr int kV41PageBytes = 20480;    // Q4_1 values: 128 x 8 x (16 + 2 + 2)
+constexpr int kV41MinOffset = 18432;    // Q4_1 minima, after the scales
 constexpr int kV8PageBytes = 34816;     // Q8_0 values
 constexpr int kKScaleOffset = 32768;    // K page: codes first, then fp16 scales
 constexpr int kV4ScaleOffset = 16384;
@@ -143,13 +147,13 @@ __device__ __forceinline__ float4 lds128f(uint32_t addr) {
   return v;
 }
 
-// D = A(16x32 s8, row) * B(32x8 s8, col) + C, int32 accumulate (exact).
-__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                       uint32_t b0, uint32_t b1, const int (&c)[4]) {
-  asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%10,%11,%12,%13};"
-      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c[0]), "r"(c[1]), "r"(c[2]), "r"(c[3]));
+// D = A(16x16 f16, row) * B(16x8 f16, col), fp32 accumulate, starting from zero.
+__device__ __forceinline__ void mma_f16_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
 }
 
 // D += A(16x16 f16, row) * B(16x8 f16, col), fp32 accumulate.

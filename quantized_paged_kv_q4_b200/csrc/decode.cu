@@ -1,42 +1,57 @@
-// Split-KV flash decode over Q8_0 K / Q4_0 (or Q8_0) V pages, or Q4_0 K / Q4_0 V pages (the
-// q4_0/q4_0 cache of the Vulkan report's summary; q4_0-q4_0 is one of the flash-attention KV
-// pairs built in the six-step validation guide's build step), for one query token or an
-// MTP verify batch of up to 4 (Adaptive KV Streaming + RDNA 4 announcement, wqu.guru,
-// method list: "paged decode attention extended to verify batches").
+// Split-KV flash decode over block-quantized KV pages, for one query token or an MTP verify
+// batch of up to 4 (Adaptive KV Streaming + RDNA 4 announcement, wqu.guru, method list:
+// "paged decode attention extended to verify batches").  Key formats Q8_0, Q4_0, Q5_1 and
+// Q5_0, value formats Q4_0, Q8_0 and Q4_1 (Vulkan speculative-decoding report, lcz.me/topic/
+// 1398, "pitfalls": the legacy block quants valid as KV types; the q4_0/q4_0 and K q5_1 /
+// V q4_0 caches; MTP tuning notes on one 7900 XTX, lcz.me/topic/593: a q5_0 / q4_1 cache).
 //
-// Grid: (split, KV head).  One CTA per SM: warp 8 streams whole pages into a shared-memory
-// ring with bulk async copies (TMA engine, one 34,816 B K copy and one V copy per page);
+// Grid: (split, KV head).  One CTA per SM: lanes of warp 0 stream whole pages into a
+// shared-memory ring with bulk async copies (TMA engine, one K copy and one V copy per page);
 // warps 0-7 consume them.  All query rows of the KV head's group (group x n_q <= 24) are
 // packed into the N dimension of legacy tensor-core MMAs so every KV byte is read once per
-// group:
-//   QK^T: f16 MMA (m16n8k16), A = Q8_0 key codes dequantized in registers (int8 -> f16 by
-//         byte permutes, exact; times the fp16 block scale, one f16 rounding), 16 tokens on
-//         M; B = the query row divided by its largest magnitude, in f16.
-//   PV:   f16 MMA (m16n8k16), A = V^T decoded in registers from nibbles (value q - 8, exact
-//         in f16), B = P^T (probabilities, transposed in registers with movmatrix) times the
-//         V block scale.
+// group.  The arithmetic keeps the dequantized operands exact:
+//   QK^T: f16 MMA (m16n8k16), A = the key codes decoded in registers (integers, exact in
+//         f16), 16 tokens on M; B = the query row divided by its largest magnitude, as an f16
+//         high part and an f16 low part (the rounded remainder: about 22 significant bits
+//         together).  Each 32-channel block is accumulated on its own and multiplied by the
+//         block's fp16 scale in fp32 (plus minimum x query block sum for zero-point keys).
+//   PV:   f16 MMA (m16n8k16), A = V^T codes decoded in registers (exact), B = P^T (fp32
+//         probabilities split into f16 high and low parts, transposed in registers with
+//         movmatrix) times the per-token V block scale, again as an exact-product high part
+//         and a low part.  Zero-point values add sum_t p_t m_t per block through an all-ones
+//         A operand.
 // The online softmax keeps a per-row running maximum and rescales the accumulators only
 // when the maximum grows by more than 2^8 (p stays <= 256, safe in f16); the exact
-// cross-lane maximum is only computed when a warp vote says some score crossed that bound.  Warps merge their
-// partial states in shared memory; CTAs write (o, lse) partials that a small follow-up grid
-// (programmatic dependent launch) merges by log-sum-exp, the arithmetic of kvattn_merge_lse.
+// cross-lane maximum is only computed when a warp vote says some score crossed that bound.
+// Warps merge their partial states in shared memory; CTAs write (o, lse) partials that a
+// small follow-up grid (programmatic dependent launch) merges by log-sum-exp, the arithmetic
+// of kvattn_merge_lse.
 #include "decode.cuh"
 
 namespace kvattn {
 
 
-template <int NT, bool PAIR, bool VQ8, int KF>
+template <int KF, int VF, int NT, bool PAIR>
 struct DecodeCfg {
   static constexpr int kConsumerWarps = 8;
   static constexpr int kThreads = kConsumerWarps * 32;  // lane 0 of warp 0 also issues the copies
   static constexpr int kNB = PAIR ? 4 : 8;      // 32-channel blocks per warp
   static constexpr int kTilesPerWarp = PAIR ? 2 : 1;
-  static constexpr int kKBytes = KF == kKeyQ4 ? kK4PageBytes : KF == kKeyQ51 ? kK5PageBytes : kKPageBytes;
-  static constexpr int kKScaleOff = KF == kKeyQ4 ? kK4ScaleOffset : KF == kKeyQ51 ? kK5ScaleOffset : kKScaleOffset;
-  static constexpr int kVBytes = VQ8 ? kV8PageBytes : kV4PageBytes;
+  static constexpr bool kK5 = KF == kKeyQ51 || KF == kKeyQ50;  // 5-bit key codes
+  static constexpr bool kKMin = KF == kKeyQ51;                 // keys with a zero point
+  static constexpr bool kVMin = VF == kValQ41;                 // values with a zero point
+  static constexpr int kKBytes =
+      KF == kKeyQ4 ? kK4PageBytes : KF == kKeyQ51 ? kK5PageBytes : KF == kKeyQ50 ? kK50PageBytes : kKPageBytes;
+  static constexpr int kKScaleOff = KF == kKeyQ4 ? kK4ScaleOffset : kK5 ? kK5ScaleOffset : kKScaleOffset;
+  static constexpr int kVBytes = VF == kValQ8 ? kV8PageBytes : VF == kValQ41 ? kV41PageBytes : kV4PageBytes;
+  static constexpr int kVScaleOff = VF == kValQ8 ? kV8ScaleOffset : kV4ScaleOffset;
   static constexpr int kStageBytes = kKBytes + kVBytes;
+  // the paired shapes (16 and 24 query rows) keep the query B fragments in shared memory:
+  // [half][block][k-step][n-tile][lane][hi0, hi1, lo0, lo1]
+  static constexpr bool kQSmem = PAIR;
+  static constexpr int kQBytes = kQSmem ? 2 * 4 * 2 * NT * 32 * 16 : 0;
   // as many page stages as fit beside the pair exchange buffer and the barriers (at most 6)
-  static constexpr int kStagesFit = (PAIR ? 190000 : 214000) / kStageBytes;
+  static constexpr int kStagesFit = ((PAIR ? 190000 : 214000) - kQBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
   static constexpr int kUnits = PAIR ? 4 : 8;   // independent softmax streams per CTA
   static constexpr int kRowsPad = NT * 8;
@@ -47,7 +62,8 @@ struct DecodeCfg {
   static constexpr int kOStride = kHeadDim + 4;
   static constexpr int kMergeBytes = kUnits * kRowsPad * (kOStride + 2) * 4;
   static_assert(kMergeBytes <= kRingBytes, "merge buffer must fit in the ring");
-  static constexpr int kBarOffset = kRingBytes + kXBytes;
+  static constexpr int kQOffset = kRingBytes + kXBytes;
+  static constexpr int kBarOffset = kQOffset + kQBytes;
   static constexpr int kSmemBytes = kBarOffset + 256;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -55,14 +71,33 @@ struct DecodeCfg {
 constexpr uint32_t kHalf2Magic = 0x64006400u;  // f16 1024.0 in both halves
 constexpr uint32_t kByte64x4 = 0x64646464u;    // high byte of f16 1024.0, for byte permutes
 constexpr uint32_t kHalf2_1032 = 0x64086408u;  // 1024 + 8
+constexpr uint32_t kHalf2_1040 = 0x64106410u;  // 1024 + 16
 constexpr uint32_t kHalf2_1152 = 0x64806480u;  // 1024 + 128
 constexpr uint32_t kHalf2_1_16 = 0x2C002C00u;  // 1/16
 constexpr uint32_t kHalf2_m72 = 0xD480D480u;   // -(64 + 8)
 constexpr uint32_t kHalf2_m64 = 0xD400D400u;   // -64
+constexpr uint32_t kHalf2_m80 = 0xD500D500u;   // -(64 + 16)
+constexpr uint32_t kHalf2_One = 0x3C003C00u;   // 1.0
+constexpr uint32_t kHalf2_Sign = 0x80008000u;
 
-template <int NT, bool PAIR, bool VQ8, int KF>
-__global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KF>::kThreads, 1) decode_kernel(const DecodeParams p) {
-  using C = DecodeCfg<NT, PAIR, VQ8, KF>;
+// B operand (probabilities times a per-token fp16 factor f) as an unevaluated f16 sum hi + lo:
+// hi = f16(ph * f); ph * f - hi is exact in f16 (an 11 x 11-bit product rounded to 11 bits
+// leaves at most 11 bits), and lo adds pl * f with one rounding.  hi + lo equals (ph + pl) * f
+// to about 2^-22 relative.
+__device__ __forceinline__ void split_scaled(uint32_t ph, uint32_t pl, uint32_t f, uint32_t& hi, uint32_t& lo) {
+  hi = hmul2(ph, f);
+  lo = hfma2(pl, f, hfma2(ph, f, hi ^ kHalf2_Sign));
+}
+
+// fp32 pair -> f16 hi part (round to nearest) and f16 lo part (the rounded remainder).
+__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  hi = pack_half2(x0, x1);
+  lo = pack_half2(x0 - half_lo(hi), x1 - half_hi(hi));
+}
+
+template <int KF, int VF, int NT, bool PAIR>
+__global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) decode_kernel(const DecodeParams p) {
+  using C = DecodeCfg<KF, VF, NT, PAIR>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   uint64_t* xbar = full + C::kStages;   // [4] pair exchange barriers (PAIR only)
@@ -106,6 +141,9 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KF>::kThreads, 1) dec
   // per-warp softmax state (consumers)
   float m_run[NT][2], l_run[NT][2];
   float oacc[2 * C::kNB][NT][4];
+  // values with a zero point: sum over tokens of p * m per (block, query row), kept apart
+  // from oacc (every dimension of a block gets the same term) and added at the end
+  float macc[C::kVMin ? C::kNB : 1][NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -119,11 +157,17 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KF>::kThreads, 1) dec
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) oacc[i][nt][e] = 0.f;
+#pragma unroll
+  for (int i = 0; i < (C::kVMin ? C::kNB : 1); ++i)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) macc[i][nt][e] = 0.f;
 
   const int half = PAIR ? (warp & 1) : 0;
   const int blk0 = PAIR ? 4 * half : 0;
 
-  // Page copies: the first kStages pages are issued up front by lane 0 of warp 0; after
+  // Page copies: the first kStages pages are issued up front by lanes of warp 0; after
   // that, the warp that is the last of the eight to finish with a stage refills it at
   // once with the page kStages further on, so kStages - 1 pages stay in flight while one
   // is being consumed.  Pages are issued in increasing order.
@@ -157,11 +201,16 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KF>::kThreads, 1) dec
   {
     // ------------------------------------------------------------------ consumers
     // query rows of this KV head: r = qi * group + j  ->  q[qi][h * group + j][:]
-    // B fragments: the query row divided by its largest magnitude, in f16, per block, k-step
-    // and n-tile (two regs each); crow[nt][c] = amax / 16 * log2(e) turns a dot product with
-    // the normalised row into a base-2 softmax score.
-    uint32_t qf[C::kNB][2][NT][2];
+    // B fragments: the query row divided by its largest magnitude, split into an f16 high
+    // part and an f16 low part (the rounded remainder), per block, k-step and n-tile (two
+    // regs each); crow[nt][c] = amax / 16 * log2(e) turns a dot product with the normalised
+    // row into a base-2 softmax score.
+    uint32_t qh[C::kQSmem ? 1 : C::kNB][2][NT][2];
+    uint32_t ql[C::kQSmem ? 1 : C::kNB][2][NT][2];
     float crow[NT][2];
+    // zero-point keys: per block, the sum of the normalised query row's channels (for the
+    // query rows 2t, 2t + 1 of each n-tile)
+    float qsum[C::kKMin ? C::kNB : 1][NT][2];
     // query positions of this thread's accumulator rows, loaded first: every global read of
     // the setup is issued before any of them is used
     int qpos_row[NT][2];
@@ -172,6 +221,7 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KF>::kThreads, 1) dec
         const int rr = nt * 8 + 2 * t + c;
         qpos_row[nt][c] = rr < n_rows ? p.q_pos[rr / p.group] : INT_MAX;
       }
+    const uint32_t q_s = smem_u32(smem + C::kQOffset);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int r = nt * 8 + g;
@@ -206,15 +256,46 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KF>::kThreads, 1) dec
 #pragma unroll
         for (int e = 0; e < 8; ++e) xv[e] = ((PAIR && half) ? x[(4 + bl) % kBlocks][e] : x[bl][e]) * inv;
         // k-step 0 of the block: channels 8t+0..3, k-step 1: 8t+4..7 (k = 2t, 2t+1 | 2t+8, 2t+9)
-        qf[bl][0][nt][0] = pack_half2(xv[0], xv[1]);
-        qf[bl][0][nt][1] = pack_half2(xv[2], xv[3]);
-        qf[bl][1][nt][0] = pack_half2(xv[4], xv[5]);
-        qf[bl][1][nt][1] = pack_half2(xv[6], xv[7]);
+        uint32_t hi[2][2], lo[2][2];
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          split_pair(xv[4 * ks], xv[4 * ks + 1], hi[ks][0], lo[ks][0]);
+          split_pair(xv[4 * ks + 2], xv[4 * ks + 3], hi[ks][1], lo[ks][1]);
+        }
+        if constexpr (C::kQSmem) {
+          // warps of the same half hold the same values; warps 0 and 1 write them
+          if (warp < 2) {
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks)
+              asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                               q_s + (((((half * 4 + bl) * 2 + ks) * NT + nt) * 32 + lane) * 16)),
+                           "r"(hi[ks][0]), "r"(hi[ks][1]), "r"(lo[ks][0]), "r"(lo[ks][1])
+                           : "memory");
+          }
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+            qh[bl][ks][nt][0] = hi[ks][0];
+            qh[bl][ks][nt][1] = hi[ks][1];
+            ql[bl][ks][nt][0] = lo[ks][0];
+            ql[bl][ks][nt][1] = lo[ks][1];
+          }
+        }
+        if constexpr (C::kKMin) {
+          float sm = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) sm += xv[e];
+          sm += __shfl_xor_sync(0xffffffffu, sm, 1);
+          sm += __shfl_xor_sync(0xffffffffu, sm, 2);
+          qsum[bl][nt][0] = __shfl_sync(0xffffffffu, sm, (2 * t) * 4);
+          qsum[bl][nt][1] = __shfl_sync(0xffffffffu, sm, (2 * t + 1) * 4);
+        }
       }
       const float cr = amax * (1.0f / 16.0f) * 1.4426950408889634f;
       crow[nt][0] = __shfl_sync(0xffffffffu, cr, (2 * t) * 4);
       crow[nt][1] = __shfl_sync(0xffffffffu, cr, (2 * t + 1) * 4);
     }
+    if constexpr (C::kQSmem) __syncthreads();
     // the smallest query position over all rows (the four t-lanes of a quad hold all rows)
     int qpos_min = INT_MAX;
 #pragma unroll
@@ -227,6 +308,15 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KF>::kThreads, 1) dec
     int xpar = 0;
     uint32_t xphase = 0;
     bool aborted = false;
+
+    // the B fragments (hi0, hi1, lo0, lo1) of block bl, k-step ks, n-tile nt
+    auto qfrag = [&](int bl, int ks, int nt) -> uint4 {
+      if constexpr (C::kQSmem) {
+        return lds128(q_s + (((((half * 4 + bl) * 2 + ks) * NT + nt) * 32 + lane) * 16));
+      } else {
+        return make_uint4(qh[bl][ks][nt][0], qh[bl][ks][nt][1], ql[bl][ks][nt][0], ql[bl][ks][nt][1]);
+      }
+    };
 
     for (int i = 0; i < count; ++i) {
       const int s = i % C::kStages;
@@ -244,53 +334,99 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KF>::kThreads, 1) dec
         for (int tt = 0; tt < C::kTilesPerWarp; ++tt) {
           const int G = PAIR ? (2 * pair + tt) : warp;
           // ---------------- S = K Q^T over this warp's channel blocks ----------------
+          // Key codes enter the MMA exactly (integers in f16).  Each 32-channel block is
+          // accumulated on its own (four MMAs: two k-steps, query high and low parts) and then
+          // scaled by the block's fp32 scale (and, with a zero point, plus the block minimum
+          // times the query block sum) into S.
           float sacc[NT][4];
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-          // key scales of rows g (H=0) and g+8 (H=1) for this warp's blocks, as f16 pairs
-          uint32_t dk2[2][C::kNB];
+          // key scales (and minima) of rows g (H=0) and g+8 (H=1) for this warp's blocks, fp32
+          float dkf[2][C::kNB];
+          float mkf[2][C::kKMin ? C::kNB : 1];
 #pragma unroll
           for (int H = 0; H < 2; ++H) {
             const uint32_t a = kb + C::kKScaleOff + (((G * 8 + g) * 2 + H) * 8 + blk0) * 2;
-            uint32_t w[4];
+            uint32_t w[4], wm[4];
             if constexpr (C::kNB == 8) {
               const uint4 v = lds128(a);
               w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+              if constexpr (C::kKMin) {
+                const uint4 vm = lds128(a + (kK5MinOffset - kK5ScaleOffset));
+                wm[0] = vm.x; wm[1] = vm.y; wm[2] = vm.z; wm[3] = vm.w;
+              }
             } else {
               asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(a));
               w[2] = w[3] = 0u;
+              if constexpr (C::kKMin) {
+                asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
+                             : "=r"(wm[0]), "=r"(wm[1])
+                             : "r"(a + (kK5MinOffset - kK5ScaleOffset)));
+                wm[2] = wm[3] = 0u;
+              }
             }
 #pragma unroll
             for (int e = 0; e < C::kNB / 2; ++e) {
-              dk2[H][2 * e] = prmt(w[e], 0u, 0x1010u);
-              dk2[H][2 * e + 1] = prmt(w[e], 0u, 0x3232u);
+              dkf[H][2 * e] = half_lo(w[e]);
+              dkf[H][2 * e + 1] = half_hi(w[e]);
+              if constexpr (C::kKMin) {
+                mkf[H][2 * e] = half_lo(wm[e]);
+                mkf[H][2 * e + 1] = half_hi(wm[e]);
+              }
             }
           }
-          if constexpr (KF == kKeyQ51) {
-            // Q5_1 keys: the low nibbles as for Q4_0 keys; the fifth bits of the lane's four
-            // blocks of one token in one word, channel (c, i) at bit 16(i%2) + 4c + i/2, shifted
-            // to bit 4 (f16 pair 1024 + q) or bit 8 (pair 1024 + 16q) of each half.  q is exact
-            // in f16; the value q * d + m takes one f16 rounding (fma).
-            uint32_t mk2[2][C::kNB];
+          // one block: four MMAs into xb, then S += d * xb (+ m * qsum)
+          auto block_qk = [&](int bl, const uint32_t (&A)[2][4]) {
+            float xb[NT][4];
 #pragma unroll
-            for (int H = 0; H < 2; ++H) {
-              const uint32_t a = kb + kK5MinOffset + (((G * 8 + g) * 2 + H) * 8 + blk0) * 2;
-              uint32_t w[4];
-              if constexpr (C::kNB == 8) {
-                const uint4 v = lds128(a);
-                w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-              } else {
-                asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(a));
-                w[2] = w[3] = 0u;
+            for (int nt = 0; nt < NT; ++nt) {
+              const uint4 f0 = qfrag(bl, 0, nt), f1 = qfrag(bl, 1, nt);
+              mma_f16_z(xb[nt], A[0][0], A[0][1], A[0][2], A[0][3], f0.x, f0.y);
+              mma_f16(xb[nt], A[0][0], A[0][1], A[0][2], A[0][3], f0.z, f0.w);
+              mma_f16(xb[nt], A[1][0], A[1][1], A[1][2], A[1][3], f1.x, f1.y);
+              mma_f16(xb[nt], A[1][0], A[1][1], A[1][2], A[1][3], f1.z, f1.w);
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                sacc[nt][e] = fmaf(dkf[e >> 1][bl], xb[nt][e], sacc[nt][e]);
+                if constexpr (C::kKMin) sacc[nt][e] = fmaf(mkf[e >> 1][bl], qsum[bl][nt][e & 1], sacc[nt][e]);
               }
+          };
+          if constexpr (KF == kKeyQ8) {
 #pragma unroll
-              for (int e = 0; e < C::kNB / 2; ++e) {
-                mk2[H][2 * e] = prmt(w[e], 0u, 0x1010u);
-                mk2[H][2 * e + 1] = prmt(w[e], 0u, 0x3232u);
+            for (int pp = 0; pp < C::kNB / 2; ++pp) {
+              const int P = blk0 / 2 + pp;
+              const uint4 ka = lds128(kb + ((((G * 4 + P) * 2 + 0) * 8 + g) * 4 + t) * 16);
+              const uint4 kc = lds128(kb + ((((G * 4 + P) * 2 + 1) * 8 + g) * 4 + t) * 16);
+              const uint32_t wg[4] = {ka.x ^ 0x80808080u, ka.y ^ 0x80808080u, ka.z ^ 0x80808080u,
+                                      ka.w ^ 0x80808080u};
+              const uint32_t w8[4] = {kc.x ^ 0x80808080u, kc.y ^ 0x80808080u, kc.z ^ 0x80808080u,
+                                      kc.w ^ 0x80808080u};
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                uint32_t A[2][4];
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                  // exact int8 -> f16: 1024 + (q + 128) - 1152
+                  A[ks][0] = hsub2(prmt(wg[2 * e + ks], kByte64x4, 0x4140u), kHalf2_1152);
+                  A[ks][2] = hsub2(prmt(wg[2 * e + ks], kByte64x4, 0x4342u), kHalf2_1152);
+                  A[ks][1] = hsub2(prmt(w8[2 * e + ks], kByte64x4, 0x4140u), kHalf2_1152);
+                  A[ks][3] = hsub2(prmt(w8[2 * e + ks], kByte64x4, 0x4342u), kHalf2_1152);
+                }
+                block_qk(2 * pp + e, A);
               }
             }
+          } else {
+            // 4- and 5-bit keys: one 32-bit word per (token, block) and lane holds channels 8t + i,
+            // channel i at bit 4 * (i / 2) + 16 * (i % 2); a shift by 8 * ks and two masks give
+            // the f16 pairs (4ks, 4ks + 1) and (4ks + 2, 4ks + 3) of k-step ks (1024 + q and
+            // 1024 + 16q).  5-bit keys: the fifth bits of the lane's four blocks of one token
+            // sit in one word, channel (c, i) at bit 16(i%2) + 4c + i/2, and are shifted to bit 4
+            // or bit 8 of each half.  The code (minus 8 for Q4_0, 16 for Q5_0) is exact in f16.
 #pragma unroll
             for (int qq = 0; qq < C::kNB / 4; ++qq) {
               const int Q = blk0 / 4 + qq;
@@ -298,91 +434,43 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KF>::kThreads, 1) dec
               const int row1 = (((G * 2 + Q) * 2 + 1) * 8 + g) * 4 + t;
               const uint4 ka = lds128(kb + row0 * 16);
               const uint4 kc = lds128(kb + row1 * 16);
-              const uint32_t xa5 = lds32(kb + kK5HighOffset + row0 * 4);
-              const uint32_t xc5 = lds32(kb + kK5HighOffset + row1 * 4);
+              uint32_t xa5 = 0, xc5 = 0;
+              if constexpr (C::kK5) {
+                xa5 = lds32(kb + kK5HighOffset + row0 * 4);
+                xc5 = lds32(kb + kK5HighOffset + row1 * 4);
+              }
               const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
               const uint32_t wc[4] = {kc.x, kc.y, kc.z, kc.w};
 #pragma unroll
               for (int c = 0; c < 4; ++c) {
-                const int bl = 4 * qq + c;
+                uint32_t A[2][4];
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks) {
                   const uint32_t xa = wa[c] >> (8 * ks), xc = wc[c] >> (8 * ks);
-                  const int slo = 4 - (4 * c + 2 * ks), shi = 7 - (4 * c + 2 * ks);
-                  const uint32_t ha_lo = slo >= 0 ? xa5 << slo : xa5 >> -slo;
-                  const uint32_t ha_hi = shi >= 0 ? xa5 << shi : xa5 >> -shi;
-                  const uint32_t hc_lo = slo >= 0 ? xc5 << slo : xc5 >> -slo;
-                  const uint32_t hc_hi = shi >= 0 ? xc5 << shi : xc5 >> -shi;
-                  const uint32_t qa0 = hsub2(or_and(and_or(xa, 0x000F000Fu, kHalf2Magic), ha_lo, 0x00100010u), kHalf2Magic);
-                  const uint32_t qa2 =
-                      hfma2(or_and(and_or(xa, 0x00F000F0u, kHalf2Magic), ha_hi, 0x01000100u), kHalf2_1_16, kHalf2_m64);
-                  const uint32_t qc1 = hsub2(or_and(and_or(xc, 0x000F000Fu, kHalf2Magic), hc_lo, 0x00100010u), kHalf2Magic);
-                  const uint32_t qc3 =
-                      hfma2(or_and(and_or(xc, 0x00F000F0u, kHalf2Magic), hc_hi, 0x01000100u), kHalf2_1_16, kHalf2_m64);
-                  const uint32_t A0 = hfma2(qa0, dk2[0][bl], mk2[0][bl]);
-                  const uint32_t A2 = hfma2(qa2, dk2[0][bl], mk2[0][bl]);
-                  const uint32_t A1 = hfma2(qc1, dk2[1][bl], mk2[1][bl]);
-                  const uint32_t A3 = hfma2(qc3, dk2[1][bl], mk2[1][bl]);
-#pragma unroll
-                  for (int nt = 0; nt < NT; ++nt)
-                    mma_f16(sacc[nt], A0, A1, A2, A3, qf[bl][ks][nt][0], qf[bl][ks][nt][1]);
+                  if constexpr (KF == kKeyQ4) {
+                    A[ks][0] = hsub2(and_or(xa, 0x000F000Fu, kHalf2Magic), kHalf2_1032);
+                    A[ks][2] = hfma2(and_or(xa, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kHalf2_m72);
+                    A[ks][1] = hsub2(and_or(xc, 0x000F000Fu, kHalf2Magic), kHalf2_1032);
+                    A[ks][3] = hfma2(and_or(xc, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kHalf2_m72);
+                  } else {
+                    const int slo = 4 - (4 * c + 2 * ks), shi = 7 - (4 * c + 2 * ks);
+                    const uint32_t ha_lo = slo >= 0 ? xa5 << slo : xa5 >> -slo;
+                    const uint32_t ha_hi = shi >= 0 ? xa5 << shi : xa5 >> -shi;
+                    const uint32_t hc_lo = slo >= 0 ? xc5 << slo : xc5 >> -slo;
+                    const uint32_t hc_hi = shi >= 0 ? xc5 << shi : xc5 >> -shi;
+                    constexpr uint32_t kSubLo = KF == kKeyQ50 ? kHalf2_1040 : kHalf2Magic;
+                    constexpr uint32_t kAddHi = KF == kKeyQ50 ? kHalf2_m80 : kHalf2_m64;
+                    A[ks][0] = hsub2(or_and(and_or(xa, 0x000F000Fu, kHalf2Magic), ha_lo, 0x00100010u), kSubLo);
+                    A[ks][2] = hfma2(or_and(and_or(xa, 0x00F000F0u, kHalf2Magic), ha_hi, 0x01000100u), kHalf2_1_16,
+                                     kAddHi);
+                    A[ks][1] = hsub2(or_and(and_or(xc, 0x000F000Fu, kHalf2Magic), hc_lo, 0x00100010u), kSubLo);
+                    A[ks][3] = hfma2(or_and(and_or(xc, 0x00F000F0u, kHalf2Magic), hc_hi, 0x01000100u), kHalf2_1_16,
+                                     kAddHi);
+                  }
                 }
+                block_qk(4 * qq + c, A);
               }
             }
-          } else if constexpr (KF == kKeyQ4) {
-            // Q4_0 keys: one 32-bit word per (token, block) and lane holds channels 8t + i,
-            // channel i at bit 4 * (i / 2) + 16 * (i % 2); a shift by 8 * ks and two masks give
-            // the f16 pairs (4ks, 4ks + 1) and (4ks + 2, 4ks + 3) of k-step ks.  The nibble
-            // q becomes q - 8 exactly (1024 + q - 1032, or (1024 + 16q) / 16 - 72), then the
-            // block scale (one f16 rounding).
-#pragma unroll
-            for (int qq = 0; qq < C::kNB / 4; ++qq) {
-              const int Q = blk0 / 4 + qq;
-              const uint4 ka = lds128(kb + (((((G * 2 + Q) * 2 + 0) * 8 + g) * 4 + t) * 16));
-              const uint4 kc = lds128(kb + (((((G * 2 + Q) * 2 + 1) * 8 + g) * 4 + t) * 16));
-              const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
-              const uint32_t wc[4] = {kc.x, kc.y, kc.z, kc.w};
-#pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                const int bl = 4 * qq + c;
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks) {
-                  const uint32_t xa = wa[c] >> (8 * ks), xc = wc[c] >> (8 * ks);
-                  const uint32_t A0 = hmul2(hsub2(and_or(xa, 0x000F000Fu, kHalf2Magic), kHalf2_1032), dk2[0][bl]);
-                  const uint32_t A2 =
-                      hmul2(hfma2(and_or(xa, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kHalf2_m72), dk2[0][bl]);
-                  const uint32_t A1 = hmul2(hsub2(and_or(xc, 0x000F000Fu, kHalf2Magic), kHalf2_1032), dk2[1][bl]);
-                  const uint32_t A3 =
-                      hmul2(hfma2(and_or(xc, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kHalf2_m72), dk2[1][bl]);
-#pragma unroll
-                  for (int nt = 0; nt < NT; ++nt)
-                    mma_f16(sacc[nt], A0, A1, A2, A3, qf[bl][ks][nt][0], qf[bl][ks][nt][1]);
-                }
-              }
-            }
-          } else {
-#pragma unroll
-          for (int pp = 0; pp < C::kNB / 2; ++pp) {
-            const int P = blk0 / 2 + pp;
-            const uint4 ka = lds128(kb + ((((G * 4 + P) * 2 + 0) * 8 + g) * 4 + t) * 16);
-            const uint4 kc = lds128(kb + ((((G * 4 + P) * 2 + 1) * 8 + g) * 4 + t) * 16);
-            const uint32_t wg[4] = {ka.x ^ 0x80808080u, ka.y ^ 0x80808080u, ka.z ^ 0x80808080u, ka.w ^ 0x80808080u};
-            const uint32_t w8[4] = {kc.x ^ 0x80808080u, kc.y ^ 0x80808080u, kc.z ^ 0x80808080u, kc.w ^ 0x80808080u};
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int bl = 2 * pp + e;
-#pragma unroll
-              for (int ks = 0; ks < 2; ++ks) {
-                // exact int8 -> f16 (1024 + u - 1152), then the block scale (one f16 rounding)
-                const uint32_t A0 = hmul2(hsub2(prmt(wg[2 * e + ks], kByte64x4, 0x4140u), kHalf2_1152), dk2[0][bl]);
-                const uint32_t A2 = hmul2(hsub2(prmt(wg[2 * e + ks], kByte64x4, 0x4342u), kHalf2_1152), dk2[0][bl]);
-                const uint32_t A1 = hmul2(hsub2(prmt(w8[2 * e + ks], kByte64x4, 0x4140u), kHalf2_1152), dk2[1][bl]);
-                const uint32_t A3 = hmul2(hsub2(prmt(w8[2 * e + ks], kByte64x4, 0x4342u), kHalf2_1152), dk2[1][bl]);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) mma_f16(sacc[nt], A0, A1, A2, A3, qf[bl][ks][nt][0], qf[bl][ks][nt][1]);
-              }
-            }
-          }
           }
           if constexpr (PAIR) {
             // exchange partial scores with the partner warp (other channel half)
@@ -451,11 +539,19 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KF>::kThreads, 1) dec
                     oacc[mt][nt][c] *= alpha;
                     oacc[mt][nt][c + 2] *= alpha;
                   }
+                  if constexpr (C::kVMin) {
+#pragma unroll
+                    for (int bl = 0; bl < C::kNB; ++bl) {
+                      macc[bl][nt][c] *= alpha;
+                      macc[bl][nt][c + 2] *= alpha;
+                    }
+                  }
                   m_run[nt][c] = mx;
                 }
               }
           }
-          uint32_t pb[NT][2];
+          // P as f16 high and low parts, transposed in registers into B fragments
+          uint32_t pbh[NT][2], pbl[NT][2];
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             float pr[4];
@@ -466,35 +562,62 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KF>::kThreads, 1) dec
               pr[c + 2] = fast_exp2(sv[nt][c + 2] - mu);
               l_run[nt][c] += pr[c] + pr[c + 2];
             }
-            pb[nt][0] = movmatrix_t(pack_half2(pr[0], pr[1]));
-            pb[nt][1] = movmatrix_t(pack_half2(pr[2], pr[3]));
+            uint32_t h01, l01, h23, l23;
+            split_pair(pr[0], pr[1], h01, l01);
+            split_pair(pr[2], pr[3], h23, l23);
+            pbh[nt][0] = movmatrix_t(h01);
+            pbh[nt][1] = movmatrix_t(h23);
+            pbl[nt][0] = movmatrix_t(l01);
+            pbl[nt][1] = movmatrix_t(l23);
           }
           // ---------------- O^T += V^T P^T ----------------
-          if constexpr (!VQ8) {
+          // V codes enter the MMA exactly; the per-token block scale multiplies P (as a high
+          // and a low f16 part), two MMAs per 16-dimension half.
+          if constexpr (VF != kValQ8) {
 #pragma unroll
             for (int cc = 0; cc < C::kNB / 2; ++cc) {
               const int Cc = blk0 / 2 + cc;
               const uint4 vw = lds128(vb + ((((G * 4 + Cc) * 8 + g) * 4 + t) * 16));
-              const uint4 dv = lds128(vb + kV4ScaleOffset + (((G * 4 + t) * 8 + 2 * Cc) * 4) * 2);
+              const uint32_t sidx = vb + C::kVScaleOff + (((G * 4 + t) * 8 + 2 * Cc) * 4) * 2;
+              const uint4 dv = lds128(sidx);
+              uint4 mv = make_uint4(0u, 0u, 0u, 0u);
+              if constexpr (C::kVMin) mv = lds128(sidx + (kV41MinOffset - kV4ScaleOffset));
 #pragma unroll
               for (int e = 0; e < 2; ++e) {
                 const int bl = 2 * cc + e;
                 const uint32_t W0 = e ? vw.z : vw.x, W1 = e ? vw.w : vw.y;
                 const uint32_t d0 = e ? dv.z : dv.x, d1 = e ? dv.w : dv.y;
                 const uint32_t W0s = W0 >> 8, W1s = W1 >> 8;
-                const uint32_t a00 = hsub2(and_or(W0, 0x000F000Fu, kHalf2Magic), kHalf2_1032);
-                const uint32_t a01 = hfma2(and_or(W0, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kHalf2_m72);
-                const uint32_t a02 = hsub2(and_or(W1, 0x000F000Fu, kHalf2Magic), kHalf2_1032);
-                const uint32_t a03 = hfma2(and_or(W1, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kHalf2_m72);
-                const uint32_t a10 = hsub2(and_or(W0s, 0x000F000Fu, kHalf2Magic), kHalf2_1032);
-                const uint32_t a11 = hfma2(and_or(W0s, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kHalf2_m72);
-                const uint32_t a12 = hsub2(and_or(W1s, 0x000F000Fu, kHalf2Magic), kHalf2_1032);
-                const uint32_t a13 = hfma2(and_or(W1s, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kHalf2_m72);
+                // Q4_0: q - 8 (1024 + q - 1032, or (1024 + 16q) / 16 - 72); Q4_1: q
+                constexpr uint32_t kSubLo = C::kVMin ? kHalf2Magic : kHalf2_1032;
+                constexpr uint32_t kAddHi = C::kVMin ? kHalf2_m64 : kHalf2_m72;
+                const uint32_t a00 = hsub2(and_or(W0, 0x000F000Fu, kHalf2Magic), kSubLo);
+                const uint32_t a01 = hfma2(and_or(W0, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kAddHi);
+                const uint32_t a02 = hsub2(and_or(W1, 0x000F000Fu, kHalf2Magic), kSubLo);
+                const uint32_t a03 = hfma2(and_or(W1, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kAddHi);
+                const uint32_t a10 = hsub2(and_or(W0s, 0x000F000Fu, kHalf2Magic), kSubLo);
+                const uint32_t a11 = hfma2(and_or(W0s, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kAddHi);
+                const uint32_t a12 = hsub2(and_or(W1s, 0x000F000Fu, kHalf2Magic), kSubLo);
+                const uint32_t a13 = hfma2(and_or(W1s, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kAddHi);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                  const uint32_t b0 = hmul2(pb[nt][0], d0), b1 = hmul2(pb[nt][1], d1);
-                  mma_f16(oacc[2 * bl][nt], a00, a01, a02, a03, b0, b1);
-                  mma_f16(oacc[2 * bl + 1][nt], a10, a11, a12, a13, b0, b1);
+                  uint32_t bh0, bl0, bh1, bl1;
+                  split_scaled(pbh[nt][0], pbl[nt][0], d0, bh0, bl0);
+                  split_scaled(pbh[nt][1], pbl[nt][1], d1, bh1, bl1);
+                  mma_f16(oacc[2 * bl][nt], a00, a01, a02, a03, bh0, bh1);
+                  mma_f16(oacc[2 * bl][nt], a00, a01, a02, a03, bl0, bl1);
+                  mma_f16(oacc[2 * bl + 1][nt], a10, a11, a12, a13, bh0, bh1);
+                  mma_f16(oacc[2 * bl + 1][nt], a10, a11, a12, a13, bl0, bl1);
+                  if constexpr (C::kVMin) {
+                    // sum over the tile's tokens of p * m, the same for every dimension of the
+                    // block: an all-ones A operand
+                    const uint32_t m0 = e ? mv.z : mv.x, m1 = e ? mv.w : mv.y;
+                    uint32_t mh0, ml0, mh1, ml1;
+                    split_scaled(pbh[nt][0], pbl[nt][0], m0, mh0, ml0);
+                    split_scaled(pbh[nt][1], pbl[nt][1], m1, mh1, ml1);
+                    mma_f16(macc[bl][nt], kHalf2_One, kHalf2_One, kHalf2_One, kHalf2_One, mh0, mh1);
+                    mma_f16(macc[bl][nt], kHalf2_One, kHalf2_One, kHalf2_One, kHalf2_One, ml0, ml1);
+                  }
                 }
               }
             }
@@ -517,9 +640,13 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KF>::kThreads, 1) dec
               }
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt) {
-                const uint32_t b0 = hmul2(pb[nt][0], d0), b1 = hmul2(pb[nt][1], d1);
-                mma_f16(oacc[2 * bl][nt], a[0][0], a[0][1], a[1][0], a[1][1], b0, b1);
-                mma_f16(oacc[2 * bl + 1][nt], a[2][0], a[2][1], a[3][0], a[3][1], b0, b1);
+                uint32_t bh0, bl0, bh1, bl1;
+                split_scaled(pbh[nt][0], pbl[nt][0], d0, bh0, bl0);
+                split_scaled(pbh[nt][1], pbl[nt][1], d1, bh1, bl1);
+                mma_f16(oacc[2 * bl][nt], a[0][0], a[0][1], a[1][0], a[1][1], bh0, bh1);
+                mma_f16(oacc[2 * bl][nt], a[0][0], a[0][1], a[1][0], a[1][1], bl0, bl1);
+                mma_f16(oacc[2 * bl + 1][nt], a[2][0], a[2][1], a[3][0], a[3][1], bh0, bh1);
+                mma_f16(oacc[2 * bl + 1][nt], a[2][0], a[2][1], a[3][0], a[3][1], bl0, bl1);
               }
             }
           }
@@ -587,7 +714,9 @@ __global__ void __launch_bounds__(DecodeCfg<NT, PAIR, VQ8, KF>::kThreads, 1) dec
         for (int e = 0; e < 4; ++e) {
           const int row = nt * 8 + 2 * t + (e & 1);
           const int dim = 32 * b + 16 * hb + g + 8 * (e >> 1);
-          os[(unit * C::kRowsPad + row) * C::kOStride + dim] = oacc[mt][nt][e];
+          float v = oacc[mt][nt][e];
+          if constexpr (C::kVMin) v += macc[mt >> 1][nt][e];
+          os[(unit * C::kRowsPad + row) * C::kOStride + dim] = v;
         }
     }
   }
@@ -710,9 +839,29 @@ __global__ void __launch_bounds__(kMergeThreads, kMinBlocks) decode_merge_kernel
 }
 
 // ---------------------------------------------------------------------------------------
-template <int NT, bool PAIR, bool VQ8, int KF>
+int decode_rows_pad(int rows) { return ((rows + 7) / 8) * 8; }
+
+// The merge grid of a decode plan with more than one split (a no-op for one split, where the
+// split grid wrote out and lse itself).
+cudaError_t launch_decode_merge(const DecodeParams& prm, int n_kv, cudaStream_t stream) {
+  if (prm.n_splits == 1) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(prm.group * prm.n_q, n_kv);
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_merge_kernel<16, 1>, static_cast<const float*>(prm.part_o),
+                            static_cast<const float*>(prm.part_lse), prm.n_splits,
+                            decode_rows_pad(prm.group * prm.n_q), prm.group, prm.n_qh, prm.out, prm.lse);
+}
+
+template <int KF, int VF, int NT, bool PAIR>
 static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream_t stream) {
-  using C = DecodeCfg<NT, PAIR, VQ8, KF>;
+  using C = DecodeCfg<KF, VF, NT, PAIR>;
   // programmatic dependent launch: the grid may start while the previous kernel on the
   // stream drains; the kernel waits for it (griddepcontrol.wait) before reading any input
   cudaLaunchConfig_t cfg = {};
@@ -725,49 +874,49 @@ static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<NT, PAIR, VQ8, KF>, prm);
-  if (e != cudaSuccess || prm.n_splits == 1) return e;
-  cfg.gridDim = dim3(prm.group * prm.n_q, n_kv);
-  cfg.blockDim = dim3(kMergeThreads);
-  cfg.dynamicSmemBytes = 0;
-  return cudaLaunchKernelEx(&cfg, decode_merge_kernel<16, 1>, static_cast<const float*>(prm.part_o),
-                            static_cast<const float*>(prm.part_lse), prm.n_splits, C::kRowsPad, prm.group, prm.n_qh,
-                            prm.out, prm.lse);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<KF, VF, NT, PAIR>, prm);
 }
 
-int decode_rows_pad(int rows) { return ((rows + 7) / 8) * 8; }
+// The supported (key, value) format pairs: Q8_0 keys with Q4_0 or Q8_0 values, Q4_0 and Q5_1
+// keys with Q4_0 or Q8_0 values, Q5_0 keys with Q4_1 values.
+#define KVATTN_DECODE_PAIRS(X) \
+  X(kKeyQ8, kValQ4) X(kKeyQ8, kValQ8) X(kKeyQ4, kValQ4) X(kKeyQ4, kValQ8) X(kKeyQ51, kValQ4) \
+  X(kKeyQ51, kValQ8) X(kKeyQ50, kValQ41)
+
+bool decode_pair_supported(int key_fmt, int val_fmt) {
+#define KV_PAIR_OK(KF, VF) if (key_fmt == KF && val_fmt == VF) return true;
+  KVATTN_DECODE_PAIRS(KV_PAIR_OK)
+#undef KV_PAIR_OK
+  return false;
+}
 
 cudaError_t prepare_decode_kernels() {
   cudaError_t e;
-#define KV_SET(NT, PAIR, VQ8, KF)                                                                   \
-  e = cudaFuncSetAttribute(decode_kernel<NT, PAIR, VQ8, KF>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                           DecodeCfg<NT, PAIR, VQ8, KF>::kSmemBytes);                               \
+#define KV_SET1(KF, VF, NT, PAIR)                                                                   \
+  e = cudaFuncSetAttribute(decode_kernel<KF, VF, NT, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                           DecodeCfg<KF, VF, NT, PAIR>::kSmemBytes);                               \
   if (e != cudaSuccess) return e;
-  KV_SET(1, false, false, kKeyQ8) KV_SET(1, false, true, kKeyQ8) KV_SET(2, true, false, kKeyQ8)
-  KV_SET(2, true, true, kKeyQ8) KV_SET(3, true, false, kKeyQ8) KV_SET(3, true, true, kKeyQ8)
-  KV_SET(1, false, false, kKeyQ4) KV_SET(2, true, false, kKeyQ4) KV_SET(3, true, false, kKeyQ4)
-  KV_SET(1, false, false, kKeyQ51) KV_SET(2, true, false, kKeyQ51) KV_SET(3, true, false, kKeyQ51)
+#define KV_SET(KF, VF) KV_SET1(KF, VF, 1, false) KV_SET1(KF, VF, 2, true) KV_SET1(KF, VF, 3, true)
+  KVATTN_DECODE_PAIRS(KV_SET)
 #undef KV_SET
+#undef KV_SET1
   return cudaSuccess;
 }
 
-// Q8_0 keys with Q4_0 or Q8_0 values; Q4_0 or Q5_1 keys with Q4_0 values.
-template <int KF>
-static cudaError_t launch_decode_v4(const DecodeParams& prm, int n_kv, int nt, cudaStream_t stream) {
-  if (nt == 1) return launch_decode_t<1, false, false, KF>(prm, n_kv, stream);
-  if (nt == 2) return launch_decode_t<2, true, false, KF>(prm, n_kv, stream);
-  return launch_decode_t<3, true, false, KF>(prm, n_kv, stream);
+template <int KF, int VF>
+static cudaError_t launch_decode_fmt(const DecodeParams& prm, int n_kv, int nt, cudaStream_t stream) {
+  if (nt == 1) return launch_decode_t<KF, VF, 1, false>(prm, n_kv, stream);
+  if (nt == 2) return launch_decode_t<KF, VF, 2, true>(prm, n_kv, stream);
+  return launch_decode_t<KF, VF, 3, true>(prm, n_kv, stream);
 }
 
-cudaError_t launch_decode(const DecodeParams& prm, int n_kv, int key_fmt, bool vq8, cudaStream_t stream) {
+cudaError_t launch_decode(const DecodeParams& prm, int n_kv, int key_fmt, int val_fmt, cudaStream_t stream) {
   const int nt = decode_rows_pad(prm.group * prm.n_q) / 8;
-  if (key_fmt != kKeyQ8 && vq8) return cudaErrorInvalidValue;
-  if (key_fmt == kKeyQ4) return launch_decode_v4<kKeyQ4>(prm, n_kv, nt, stream);
-  if (key_fmt == kKeyQ51) return launch_decode_v4<kKeyQ51>(prm, n_kv, nt, stream);
-  if (!vq8) return launch_decode_v4<kKeyQ8>(prm, n_kv, nt, stream);
-  if (nt == 1) return launch_decode_t<1, false, true, kKeyQ8>(prm, n_kv, stream);
-  if (nt == 2) return launch_decode_t<2, true, true, kKeyQ8>(prm, n_kv, stream);
-  return launch_decode_t<3, true, true, kKeyQ8>(prm, n_kv, stream);
+#define KV_LAUNCH(KF, VF) \
+  if (key_fmt == KF && val_fmt == VF) return launch_decode_fmt<KF, VF>(prm, n_kv, nt, stream);
+  KVATTN_DECODE_PAIRS(KV_LAUNCH)
+#undef KV_LAUNCH
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace kvattn

@@ -21,7 +21,15 @@ struct DecodeParams {
   int n_q, group, n_qh, max_pages, n_splits;
 };
 
-cudaError_t launch_decode(const DecodeParams& prm, int n_kv, int key_fmt, bool vq8, cudaStream_t stream);
+// The split grid of a decode (partials into the workspace, or out / lse for one split) ...
+cudaError_t launch_decode(const DecodeParams& prm, int n_kv, int key_fmt, int val_fmt, cudaStream_t stream);
+// ... and the grid that merges the partials (nothing for one split).
+cudaError_t launch_decode_merge(const DecodeParams& prm, int n_kv, cudaStream_t stream);
+int decode_rows_pad(int rows);
+bool decode_pair_supported(int key_fmt, int val_fmt);
+// kvattn_kv_desc format codes -> kernel format ids (-1 if not a key / value format)
+int key_format_id(int k_fmt);
+int value_format_id(int v_fmt);
 cudaError_t prepare_decode_kernels();
 
 }  // namespace kvattn

@@ -1,21 +1,26 @@
-// Q8_0 / Q4_0 / Q5_1 encoders that append new tokens into their KV pages.
+// Q8_0 / Q4_0 / Q5_1 / Q5_0 / Q4_1 encoders that append new tokens into their KV pages.
 //
 // Formats (Vulkan speculative-decoding report, lcz.me/topic/1398, "pitfalls" and
 // "configs"): 32-element blocks with one fp16 scale; Q8_0 stores int8 codes (8.5 bits per
-// element), Q4_0 stores 4-bit codes q with value (q - 8) * d (18 bytes per block).
+// element), Q4_0 stores 4-bit codes q with value (q - 8) * d (18 bytes per block); the same
+// list names q4_1, q5_0 and q5_1 as KV types.
 // Encoder readings (the pages do not spell them out):
 //   Q8_0: d = amax / 127, q = round-half-away(x * fp32(1/d)), |q| <= 127.
 //   Q4_0: m = the signed element of largest magnitude (first on ties), d = m / -8,
 //         q = min(15, floor(fp32(fp32(x * fp32(1/d)) + 8.5))).
+//   Q5_0: as Q4_0 with 5-bit codes: d = m / -16, q = min(31, floor(x * fp32(1/d) + 16.5)),
+//         value (q - 16) * d.
 //   Q5_1 (same report, pitfalls: 5-bit codes with a zero point, 6 bits per element):
 //         m = the block minimum, d = fp32(fp32(max - m) / 31),
 //         q = min(31, floor(fp32(fp32(fp32(x - m) * fp32(1/d)) + 0.5))), value q * d + m.
+//   Q4_1: as Q5_1 with 4-bit codes: d = (max - m) / 15, q = min(15, ...).
 // Every operation that decides a code is an IEEE fp32 operation with round-to-nearest
 // (no FMA contraction), so the codes equal those of any correct fp32 implementation.
 //
 // One warp encodes one (token, KV head) row: lane l owns channels [8l, 8l+8), four lanes
-// form one 32-element block.  Keys are stored as Q8_0, Q4_0 or Q5_1, values as Q4_0 or Q8_0.
-#include "common.cuh"
+// form one 32-element block.  Keys are stored as Q8_0, Q4_0, Q5_1 or Q5_0, values as Q4_0,
+// Q8_0 or Q4_1.
+#include "decode.cuh"
 
 namespace kvattn {
 
@@ -26,11 +31,14 @@ __device__ __forceinline__ int q8_code(float x, float inv) {
   return static_cast<int>(r);
 }
 
-__device__ __forceinline__ int q4_code(float x, float inv) {
+// Offset codes: min(2 half - 1, floor(fp32(fp32(x * inv) + half + 0.5))) (half = 8: Q4_0, 16: Q5_0).
+template <int HALF>
+__device__ __forceinline__ int offset_code(float x, float inv) {
   const float y = __fmul_rn(x, inv);
-  const float z = __fadd_rn(y, 8.5f);
-  return min(15, __float2int_rz(z));  // z > 0, so truncation is floor
+  const float z = __fadd_rn(y, HALF + 0.5f);
+  return min(2 * HALF - 1, __float2int_rz(z));  // z > 0, so truncation is floor
 }
+__device__ __forceinline__ int q4_code(float x, float inv) { return offset_code<8>(x, inv); }
 
 // Q8_0 block scale of this lane's block: returns d (fp32) and writes 1/d to *inv.
 __device__ __forceinline__ float q8_scale(const float (&x)[8], float* inv) {
@@ -44,10 +52,11 @@ __device__ __forceinline__ float q8_scale(const float (&x)[8], float* inv) {
   return d;
 }
 
-// Q4_0 block scale of this lane's block (channels 8 * lane + e): the signed element of
-// largest magnitude, first index on ties, over the four lanes of the block; returns
-// d = m / -8 (fp32) and writes 1/d to *inv.
-__device__ __forceinline__ float q4_scale(const float (&x)[8], int lane, float* inv) {
+// Offset-format block scale of this lane's block: the signed element of largest magnitude,
+// first index on ties, over the four lanes of the block; returns d = m / -half (fp32) and
+// writes 1/d to *inv (half = 8: Q4_0, 16: Q5_0).
+template <int HALF>
+__device__ __forceinline__ float offset_scale(const float (&x)[8], int lane, float* inv) {
   float best = x[0];
   int bidx = lane * 8;
 #pragma unroll
@@ -65,15 +74,41 @@ __device__ __forceinline__ float q4_scale(const float (&x)[8], int lane, float* 
       bidx = oi;
     }
   }
-  const float d = __fdiv_rn(best, -8.f);
+  const float d = __fdiv_rn(best, -static_cast<float>(HALF));
   *inv = d != 0.f ? __frcp_rn(d) : 0.f;
   return d;
 }
-
-__device__ __forceinline__ int q51_code(float x, float mn, float inv) {
-  const float y = __fmul_rn(__fsub_rn(x, mn), inv);
-  return min(31, __float2int_rz(__fadd_rn(y, 0.5f)));  // y >= 0, so truncation is floor
+__device__ __forceinline__ float q4_scale(const float (&x)[8], int lane, float* inv) {
+  return offset_scale<8>(x, lane, inv);
 }
+
+// Zero-point block scale of this lane's block (TOP = 31: Q5_1, 15: Q4_1): writes the block
+// minimum to *mn and 1/d to *inv, returns d = fp32(fp32(max - min) / TOP).
+template <int TOP>
+__device__ __forceinline__ float min_scale(const float (&x)[8], float* mn_out, float* inv) {
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int e = 1; e < 8; ++e) {
+    mn = fminf(mn, x[e]);
+    mx = fmaxf(mx, x[e]);
+  }
+#pragma unroll
+  for (int s = 1; s <= 2; s <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, s));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
+  }
+  const float d = __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(TOP));
+  *inv = d != 0.f ? __frcp_rn(d) : 0.f;
+  *mn_out = mn;
+  return d;
+}
+
+template <int TOP>
+__device__ __forceinline__ int min_code(float x, float mn, float inv) {
+  const float y = __fmul_rn(__fsub_rn(x, mn), inv);
+  return min(TOP, __float2int_rz(__fadd_rn(y, 0.5f)));  // y >= 0, so truncation is floor
+}
+
 
 __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __restrict__ k,
                                                               const float* __restrict__ v, int n_tok,
@@ -81,7 +116,7 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
                                                               const int32_t* __restrict__ page_table,
                                                               int n_blocks, uint8_t* k_pool, int64_t k_stride,
                                                               uint8_t* v_pool, int64_t v_stride, int64_t n_pages,
-                                                              int k_fmt, int v_q8) {
+                                                              int k_fmt, int v_fmt) {
   // a kernel launched behind this one with programmatic dependent launch (decode) may start
   // its setup now; it waits for this grid to complete before reading the pages
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -107,29 +142,23 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
   const int G = tok >> 4, tl = tok & 15, H = tl >> 3, R = tok & 7;
   const int b = lane >> 2;  // this lane's block
 
-  // ---------------- K: Q5_1 ----------------
-  if (k_fmt == kKeyQ51) {
+  // ---------------- K: Q5_1 / Q5_0 ----------------
+  if (k_fmt == kKeyQ51 || k_fmt == kKeyQ50) {
     const float x[8] = {kx0.x, kx0.y, kx0.z, kx0.w, kx1.x, kx1.y, kx1.z, kx1.w};
-    float mn = x[0], mx = x[0];
-#pragma unroll
-    for (int e = 1; e < 8; ++e) {
-      mn = fminf(mn, x[e]);
-      mx = fmaxf(mx, x[e]);
+    float mn = 0.f, inv, d;
+    if (k_fmt == kKeyQ51) {
+      d = min_scale<31>(x, &mn, &inv);
+    } else {
+      d = offset_scale<16>(x, lane, &inv);
     }
-#pragma unroll
-    for (int s = 1; s <= 2; s <<= 1) {
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, s));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
-    }
-    const float d = __fdiv_rn(__fsub_rn(mx, mn), 31.f);
-    const float inv = d != 0.f ? __frcp_rn(d) : 0.f;
     const int T = lane & 3, c = b & 3, Q = b >> 2;
     // low nibbles as the Q4_0 key word; fifth bits of the four blocks 4Q..4Q+3 of this T
     // (lanes T + 4c + 16Q) gathered into one word, channel (c, e) at bit 16(e%2) + 4c + e/2
     uint32_t w = 0, hb = 0;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const uint32_t q = static_cast<uint32_t>(q51_code(x[e], mn, inv));
+      const uint32_t q = static_cast<uint32_t>(k_fmt == kKeyQ51 ? min_code<31>(x[e], mn, inv)
+                                                                : offset_code<16>(x[e], inv));
       w |= (q & 15u) << (4 * (e >> 1) + 16 * (e & 1));
       hb |= (q >> 4) << (16 * (e & 1) + 4 * c + (e >> 1));
     }
@@ -142,7 +171,7 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
     if ((lane & 3) == 0) {
       const int si = 2 * (((G * 8 + R) * 2 + H) * 8 + b);
       *reinterpret_cast<__half*>(pg + kK5ScaleOffset + si) = __float2half_rn(d);
-      *reinterpret_cast<__half*>(pg + kK5MinOffset + si) = __float2half_rn(mn);
+      if (k_fmt == kKeyQ51) *reinterpret_cast<__half*>(pg + kK5MinOffset + si) = __float2half_rn(mn);
     }
   }
   // ---------------- K: Q4_0 ----------------
@@ -183,7 +212,7 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
     }
   }
 
-  // ---------------- V: Q4_0 or Q8_0 ----------------
+  // ---------------- V: Q4_0, Q4_1 or Q8_0 ----------------
   {
     const float x[8] = {vx0.x, vx0.y, vx0.z, vx0.w, vx1.x, vx1.y, vx1.z, vx1.w};
     uint8_t* pg = v_pool + static_cast<int64_t>(page) * v_stride;
@@ -192,11 +221,17 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
     const int cl = lane & 3;  // which 8-channel group of the block
     float d;
     int codes[8];
-    if (!v_q8) {
-      float inv;
-      d = q4_scale(x, lane, &inv);
+    if (v_fmt != kValQ8) {
+      float inv, mn = 0.f;
+      if (v_fmt == kValQ41) {
+        d = min_scale<15>(x, &mn, &inv);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) codes[e] = q4_code(x[e], inv);
+        for (int e = 0; e < 8; ++e) codes[e] = min_code<15>(x[e], mn, inv);
+      } else {
+        d = q4_scale(x, lane, &inv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) codes[e] = q4_code(x[e], inv);
+      }
       // lanes cl = 0,1 share bytes (lo, hi nibble) with y%2 = 0; lanes 2,3 with y%2 = 1
       int other[8];
 #pragma unroll
@@ -212,6 +247,8 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
       if (cl == 0) {
         const int so = kV4ScaleOffset + 2 * (((G * 4 + T) * 8 + b) * 4 + k_slot);
         *reinterpret_cast<__half*>(pg + so) = __float2half_rn(d);
+        if (v_fmt == kValQ41)
+          *reinterpret_cast<__half*>(pg + so + (kV41MinOffset - kV4ScaleOffset)) = __float2half_rn(mn);
       }
     } else {
       float inv;
@@ -251,8 +288,7 @@ cudaError_t launch_quantize_append(const kvattn_kv_desc& desc, const float* k, c
   return cudaLaunchKernelEx(&cfg, quantize_append_kernel, k, v, n_tok, desc.n_kv_heads, pos0, page_table, n_blocks,
                             static_cast<uint8_t*>(desc.k_pool), desc.k_page_stride,
                             static_cast<uint8_t*>(desc.v_pool), desc.v_page_stride, desc.n_pages,
-                            desc.k_fmt == KVATTN_FMT_Q4_0 ? kKeyQ4 : desc.k_fmt == KVATTN_FMT_Q5_1 ? kKeyQ51 : kKeyQ8,
-                            static_cast<int>(desc.v_fmt == KVATTN_FMT_Q8_0));
+                            key_format_id(desc.k_fmt), value_format_id(desc.v_fmt));
 }
 
 }  // namespace kvattn

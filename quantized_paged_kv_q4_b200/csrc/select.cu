@@ -3,7 +3,7 @@
 // fill a 32,768-token GPU budget, and a 16,384-token recent reserve is always kept).
 //
 // Readings (the pages do not define the ranking):
-//   summary[b][c] = mean over the block's 128 tokens of the dequantized key (Q8_0, Q4_0 or
+//   summary[b][c] = mean over the block's 128 tokens of the dequantized key (Q8_0, Q4_0, Q5_0 or
 //                   Q5_1), rounded once to fp32.  Computed exactly: each fp16 scale (and
 //                   Q5_1 minimum) is split into an 11-bit integer significand and an
 //                   exponent, every code x significand product is shifted onto a common
@@ -13,7 +13,7 @@
 //   selection     = the `budget` highest scores among blocks older than the recent window
 //                   (ties: lower block index), plus the recent window and partial tail
 //                   blocks, written in ascending order.
-#include "common.cuh"
+#include "decode.cuh"
 
 namespace kvattn {
 
@@ -43,8 +43,11 @@ __global__ void __launch_bounds__(256) block_summary_kernel(const uint8_t* __res
   }
   const uint4* src = reinterpret_cast<const uint4*>(k_pool + static_cast<int64_t>(pg) * k_stride);
   uint4* dst = reinterpret_cast<uint4*>(page);
-  const int bytes = k_fmt == kKeyQ4 ? kK4PageBytes : k_fmt == kKeyQ51 ? kK5PageBytes : kKPageBytes;
-  const int scale_off = k_fmt == kKeyQ4 ? kK4ScaleOffset : k_fmt == kKeyQ51 ? kK5ScaleOffset : kKScaleOffset;
+  const int bytes = k_fmt == kKeyQ4    ? kK4PageBytes
+                    : k_fmt == kKeyQ51 ? kK5PageBytes
+                    : k_fmt == kKeyQ50 ? kK50PageBytes
+                                       : kKPageBytes;
+  const int scale_off = k_fmt == kKeyQ4 ? kK4ScaleOffset : k_fmt == kKeyQ8 ? kKScaleOffset : kK5ScaleOffset;
   for (int i = threadIdx.x; i < bytes / 16; i += blockDim.x) dst[i] = src[i];
   __syncthreads();
   const int c = threadIdx.x;  // channel
@@ -66,6 +69,7 @@ __global__ void __launch_bounds__(256) block_summary_kernel(const uint8_t* __res
       } else {
         const uint32_t fifth = *reinterpret_cast<const uint32_t*>(page + kK5HighOffset + 4 * row);
         q |= static_cast<int>((fifth >> (16 * (i8 & 1) + 4 * (blk & 3) + (i8 >> 1))) & 1u) << 4;
+        if (k_fmt == kKeyQ50) q -= 16;
       }
     } else {
       q = static_cast<int8_t>(page[((((G * 4 + P) * 2 + H) * 8 + R) * 4 + T) * 16 + j]);
@@ -276,9 +280,7 @@ cudaError_t launch_block_summaries(const kvattn_kv_desc& d, const int32_t* page_
   dim3 grid(n, n_units);
   block_summary_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(d.k_pool), d.k_page_stride, d.n_pages,
                                                  page_table, n_blocks, block_begin, n,
-                                                 d.k_fmt == KVATTN_FMT_Q4_0   ? kKeyQ4
-                                                 : d.k_fmt == KVATTN_FMT_Q5_1 ? kKeyQ51
-                                                                              : kKeyQ8,
+                                                 key_format_id(d.k_fmt),
                                                  summaries);
   return cudaGetLastError();
 }

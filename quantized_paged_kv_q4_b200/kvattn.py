@@ -31,9 +31,11 @@ ERR_NOT_INITIALIZED = -9
 FMT_Q4_0 = 4
 FMT_Q8_0 = 8
 FMT_Q5_1 = 51
+FMT_Q5_0 = 50
+FMT_Q4_1 = 41
 ROLE_K = 0
 ROLE_V = 1
-FMT = {"q4_0": FMT_Q4_0, "q8_0": FMT_Q8_0, "q5_1": FMT_Q5_1}
+FMT = {"q4_0": FMT_Q4_0, "q8_0": FMT_Q8_0, "q5_1": FMT_Q5_1, "q5_0": FMT_Q5_0, "q4_1": FMT_Q4_1}
 
 
 class KVAttnError(RuntimeError):
@@ -61,6 +63,10 @@ _SIGS = {
     "kvattn_decode_workspace_size": (c_size_t, [POINTER(kvattn_kv_desc), c_int, c_int]),
     "kvattn_decode": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                               c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "kvattn_decode_splits": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_int, c_void_p, c_void_p, c_void_p,
+                                     c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "kvattn_decode_merge_splits": (c_int, [POINTER(kvattn_kv_desc), c_int, c_int, c_void_p, c_void_p, c_void_p,
+                                           c_size_t, c_void_p]),
     "kvattn_decode_noalloc": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_int, c_void_p, c_void_p, c_void_p,
                                       c_void_p, c_int, c_void_p, c_void_p, c_void_p]),
     "kvattn_merge_lse": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
@@ -190,6 +196,20 @@ def kvattn_decode(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pag
     _check(lib().kvattn_decode(ctypes.byref(desc), _d(q), n_q, _d(q_pos), _d(page_list), _d(page_logical),
                                _d(n_pages), max_pages, _d(out), _d(lse), _d(ws), ws_bytes, _s(stream)),
            "kvattn_decode")
+
+
+def kvattn_decode_splits(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pages, out, lse, ws, ws_bytes,
+                         stream=None) -> None:
+    """The split grid of kvattn_decode alone (partials into the workspace)."""
+    _check(lib().kvattn_decode_splits(ctypes.byref(desc), _d(q), n_q, _d(q_pos), _d(page_list), _d(page_logical),
+                                      _d(n_pages), max_pages, _d(out), _d(lse), _d(ws), ws_bytes, _s(stream)),
+           "kvattn_decode_splits")
+
+
+def kvattn_decode_merge_splits(desc, n_q, max_pages, out, lse, ws, ws_bytes, stream=None) -> None:
+    """The merge grid of kvattn_decode alone (partials in the workspace -> out, lse)."""
+    _check(lib().kvattn_decode_merge_splits(ctypes.byref(desc), n_q, max_pages, _d(out), _d(lse), _d(ws), ws_bytes,
+                                            _s(stream)), "kvattn_decode_merge_splits")
 
 
 def kvattn_decode_noalloc(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pages, out, lse,

@@ -161,6 +161,13 @@ WORKLOADS = {
                                 n_q=1, k_fmt="q4_0", v_fmt="q4_0", outlier_frac=0.01, seed=2004),
     "decode131k_q51q4": Workload("decode131k_q51q4", layers=16, kv_heads=4, q_heads=24, context=131072,
                                  n_q=1, k_fmt="q5_1", v_fmt="q4_0", outlier_frac=0.01, seed=2005),
+    # Q8_0 values under 4- and 5-bit keys, and the Q5_0 K / Q4_1 V cache of the MTP tuning notes.
+    "decode131k_q4q8": Workload("decode131k_q4q8", layers=16, kv_heads=4, q_heads=24, context=131072,
+                                n_q=1, k_fmt="q4_0", v_fmt="q8_0", outlier_frac=0.01, seed=2006),
+    "decode131k_q51q8": Workload("decode131k_q51q8", layers=16, kv_heads=4, q_heads=24, context=131072,
+                                 n_q=1, k_fmt="q5_1", v_fmt="q8_0", outlier_frac=0.01, seed=2007),
+    "decode131k_q50q41": Workload("decode131k_q50q41", layers=16, kv_heads=4, q_heads=24, context=131072,
+                                  n_q=1, k_fmt="q5_0", v_fmt="q4_1", outlier_frac=0.01, seed=2008),
     # 262,144 prior tokens, 4 verify tokens, 20 needles, budget 256 + recent 128 blocks.
     "verify262k": Workload("verify262k", layers=16, kv_heads=4, q_heads=24, context=262144, n_q=4,
                            needles=20, budget_blocks=256, recent_blocks=128, seed=3003),

@@ -54,6 +54,10 @@ def test_status_strings_and_page_sizes(lib):
     assert kvattn.kvattn_page_bytes(kvattn.ROLE_K, kvattn.FMT_Q4_0) == 18432
     assert kvattn.kvattn_page_bytes(kvattn.ROLE_K, kvattn.FMT_Q5_1) == 24576
     assert kvattn.kvattn_page_bytes(kvattn.ROLE_V, kvattn.FMT_Q5_1) == 0
+    assert kvattn.kvattn_page_bytes(kvattn.ROLE_K, kvattn.FMT_Q5_0) == 22528
+    assert kvattn.kvattn_page_bytes(kvattn.ROLE_V, kvattn.FMT_Q4_1) == 20480
+    assert kvattn.kvattn_page_bytes(kvattn.ROLE_V, kvattn.FMT_Q5_0) == 0
+    assert kvattn.kvattn_page_bytes(kvattn.ROLE_K, kvattn.FMT_Q4_1) == 0
     assert kvattn.kvattn_page_bytes(kvattn.ROLE_K, 5) == 0
 
 
@@ -79,17 +83,23 @@ def test_host_validation_rejects_bad_arguments(lib):
     bad = _desc()
     bad.head_dim = 128
     assert L.kvattn_decode(by(bad), 16, 1, 16, 16, None, None, 1, 16, 16, None, 0, None) == kvattn.ERR_UNSUPPORTED_FORMAT
-    bad = _desc(v_fmt="q8_0")
-    bad.k_fmt = kvattn.FMT_Q4_0
+    # format pairs outside the supported set
+    for kf, vf in (("q5_0", "q4_0"), ("q8_0", "q4_1"), ("q4_0", "q4_1"), ("q5_0", "q8_0")):
+        bad = _desc(k_fmt=kf, v_fmt=vf)
+        assert L.kvattn_decode(by(bad), 16, 1, 16, 16, None, None, 1, 16, 16, None, 0, None) == \
+            kvattn.ERR_UNSUPPORTED_FORMAT, (kf, vf)
+    bad = _desc(v_fmt="q5_1")
     assert L.kvattn_decode(by(bad), 16, 1, 16, 16, None, None, 1, 16, 16, None, 0, None) == kvattn.ERR_UNSUPPORTED_FORMAT
-    # Q4_0 / Q5_1 keys: decode and the summaries take them; chunked prefill refuses them
+    # Q4_0 / Q5_1 keys: decode and the summaries take them; chunked prefill takes Q8_0 or Q4_0
+    # keys with Q4_0 values and refuses the rest
     for kf in ("q4_0", "q5_1"):
         kd = _desc(k_fmt=kf)
         assert L.kvattn_decode_workspace_size(by(kd), 1, 1024) == L.kvattn_decode_workspace_size(by(d), 1, 1024)
-        assert L.kvattn_prefill_chunk(by(kd), 16, 1, 16, 16, None, None, 1, 4096, 16, 16, 16, 1 << 20, None) == \
-            kvattn.ERR_UNSUPPORTED_FORMAT
-    bad = _desc(k_fmt="q5_1", v_fmt="q8_0")
-    assert L.kvattn_decode(by(bad), 16, 1, 16, 16, None, None, 1, 16, 16, None, 0, None) == kvattn.ERR_UNSUPPORTED_FORMAT
+    for kf, vf, ok in (("q8_0", "q4_0", True), ("q4_0", "q4_0", True), ("q5_1", "q4_0", False),
+                       ("q8_0", "q8_0", False), ("q5_0", "q4_1", False)):
+        kd = _desc(k_fmt=kf, v_fmt=vf)
+        st = L.kvattn_prefill_chunk(by(kd), 16, 1, 16, 16, None, None, 1, 4096, 16, 16, 16, 1 << 20, None)
+        assert (st != kvattn.ERR_UNSUPPORTED_FORMAT) if ok else (st == kvattn.ERR_UNSUPPORTED_FORMAT), (kf, vf, st)
     bad = _desc(n_q_heads=25)
     assert L.kvattn_decode(by(bad), 16, 1, 16, 16, None, None, 1, 16, 16, None, 0, None) == kvattn.ERR_INVALID_ARG
     bad = _desc(k_pool=16 * 1000 + 8)

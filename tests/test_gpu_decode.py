@@ -42,7 +42,11 @@ def _run_decode(kv, cache, H_q, q, q_pos, page_list, page_logical=None, n_pages=
     return out.cpu().numpy(), lse.cpu().numpy(), (qd, qp, pl, lg, npg, out, lse, ws, wsb)
 
 
-@pytest.mark.parametrize("k_fmt,v_fmt", [("q8_0", "q4_0"), ("q8_0", "q8_0"), ("q4_0", "q4_0"), ("q5_1", "q4_0")])
+FORMAT_PAIRS = [("q8_0", "q4_0"), ("q8_0", "q8_0"), ("q4_0", "q4_0"), ("q4_0", "q8_0"), ("q5_1", "q4_0"),
+                ("q5_1", "q8_0"), ("q5_0", "q4_1")]
+
+
+@pytest.mark.parametrize("k_fmt,v_fmt", FORMAT_PAIRS)
 @pytest.mark.parametrize("n_q", [1, 2, 3, 4])
 def test_decode_matches_oracle(kv_gpu, k_fmt, v_fmt, n_q):
     H, H_q, T = 4, 24, 37 * 128 + 77          # ragged tail page
@@ -58,6 +62,24 @@ def test_decode_matches_oracle(kv_gpu, k_fmt, v_fmt, n_q):
     # a second launch reuses the workspace (split counters are left at zero) bit-identically
     qd, qp, pl, lg, npg, o2, l2, ws, wsb = keep
     kv_gpu.kvattn_decode(cache.desc, qd, n_q, qp, pl, lg, npg, pl.shape[1], o2, l2, ws, wsb)
+    torch.cuda.synchronize()
+    assert np.array_equal(o2.cpu().numpy(), out) and np.array_equal(l2.cpu().numpy(), lse)
+
+
+@pytest.mark.parametrize("n_q", [1, 4])
+def test_split_and_merge_calls_equal_decode(kv_gpu, n_q):
+    """kvattn_decode_splits then kvattn_decode_merge_splits: bit-identical to kvattn_decode."""
+    H, H_q, T = 4, 24, 20 * 128 + 9
+    rng, k, v, cache = _layer(650 + n_q, H, T, "q4_0")
+    cache.append(k, v, 0)
+    q = normal_f32(rng, (n_q, H_q, 256))
+    q_pos = [T - n_q + i for i in range(n_q)]
+    out, lse, keep = _run_decode(kv_gpu, cache, H_q, q, q_pos, cache.page_table_np)
+    qd, qp, pl, lg, npg, o2, l2, ws, wsb = keep
+    o2.fill_(float("nan"))
+    l2.fill_(float("nan"))
+    kv_gpu.kvattn_decode_splits(cache.desc, qd, n_q, qp, pl, lg, npg, pl.shape[1], o2, l2, ws, wsb)
+    kv_gpu.kvattn_decode_merge_splits(cache.desc, n_q, pl.shape[1], o2, l2, ws, wsb)
     torch.cuda.synchronize()
     assert np.array_equal(o2.cpu().numpy(), out) and np.array_equal(l2.cpu().numpy(), lse)
 
@@ -111,14 +133,19 @@ def test_causal_and_fully_masked_rows(kv_gpu):
     assert np.all(out[2] == 0) and np.all(np.isneginf(lse[2]))
 
 
-def test_single_short_page_and_empty_list(kv_gpu):
-    rng, k, v, cache = _layer(720, 1, 5, "q4_0", n_blocks=1)
+@pytest.mark.parametrize("k_fmt,v_fmt", FORMAT_PAIRS)
+@pytest.mark.parametrize("n_q", [1, 4])
+def test_single_short_page_and_empty_list(kv_gpu, k_fmt, v_fmt, n_q):
+    """Five keys with x8 outlier channels: outputs of magnitude up to ~25 that average few
+    values, the case where f16 rounding of any operand would show."""
+    rng, k, v, cache = _layer(720, 1, 5, v_fmt, n_blocks=1, k_fmt=k_fmt)
     cache.append(k, v, 0)
-    q = normal_f32(rng, (1, 6, 256))
-    out, lse, _ = _run_decode(kv_gpu, cache, 6, q, [4], cache.page_table_np)
-    o_ref, l_ref = OracleCache(k, v, "q4_0").attend(q, [4], 0, 6)
-    compare(out, lse, o_ref, l_ref, magnitude_scaled=True)   # 5 keys: outputs of size ~1-10
-    out, lse, _ = _run_decode(kv_gpu, cache, 6, q, [4], np.zeros((1, 1), np.int32), n_pages=[0], max_pages=1)
+    q = normal_f32(rng, (n_q, 6, 256))
+    q_pos = [5 - n_q + i for i in range(n_q)]
+    out, lse, _ = _run_decode(kv_gpu, cache, 6, q, q_pos, cache.page_table_np)
+    o_ref, l_ref = OracleCache(k, v, v_fmt, k_fmt).attend(q, q_pos, 0, 6)
+    compare(out, lse, o_ref, l_ref)
+    out, lse, _ = _run_decode(kv_gpu, cache, 6, q, q_pos, np.zeros((1, 1), np.int32), n_pages=[0], max_pages=1)
     assert np.all(out == 0) and np.all(np.isneginf(lse))
 
 

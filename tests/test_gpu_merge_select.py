@@ -47,14 +47,16 @@ def _select_case(seed, H, n_full, tail, budget, recent, needles, group=6, k_fmt=
         plant_needles(kh, nb, q[h].astype(np.float64).sum(0), rng, cosine=0.9)
         k[:, h] = kh
     n_phys = H * n_blocks + 2
-    cache = GpuCache(H, H * group, n_blocks, "q4_0", n_phys=n_phys, perm=page_permutation(rng, n_phys), k_fmt=k_fmt)
+    v_fmt = "q4_1" if k_fmt == "q5_0" else "q4_0"
+    cache = GpuCache(H, H * group, n_blocks, v_fmt, n_phys=n_phys, perm=page_permutation(rng, n_phys), k_fmt=k_fmt)
     cache.append(k, v, 0)
     return rng, k, v, q, cache, needle_sets, n_blocks, T
 
 
 @pytest.mark.parametrize("seed,n_full,tail,budget,recent,k_fmt", [
     (900, 300, 37, 64, 32, "q8_0"), (901, 2048, 4, 256, 128, "q8_0"), (902, 50, 0, 80, 10, "q8_0"),
-    (903, 40, 100, 8, 0, "q8_0"), (904, 300, 37, 64, 32, "q4_0"), (905, 300, 37, 64, 32, "q5_1")])
+    (903, 40, 100, 8, 0, "q8_0"), (904, 300, 37, 64, 32, "q4_0"), (905, 300, 37, 64, 32, "q5_1"),
+    (906, 300, 37, 64, 32, "q5_0")])
 def test_summaries_and_selection_bit_exact(kv_gpu, seed, n_full, tail, budget, recent, k_fmt):
     H = 4
     rng, k, v, q, cache, needle_sets, n_blocks, T = _select_case(seed, H, n_full, tail, budget, recent,
@@ -72,7 +74,7 @@ def test_summaries_and_selection_bit_exact(kv_gpu, seed, n_full, tail, budget, r
     kv_gpu.kvattn_select_blocks(summ, qg, H, 6, n_blocks, n_full, n_blocks, budget, recent, cache.page_table,
                                 sel_l, sel_p, n_sel, cap, ws, wsb)
     torch.cuda.synchronize()
-    oc = OracleCache(k, v, "q4_0", k_fmt)
+    oc = OracleCache(k, v, "q4_1" if k_fmt == "q5_0" else "q4_0", k_fmt)
     s_gpu = summ.cpu().numpy()
     for h in range(H):
         kc = oc.kc[: n_full * 128, h].reshape(n_full, 128, 8, 32)

@@ -9,7 +9,8 @@ from synth import normal_f32, np_rng, page_permutation
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("k_fmt,v_fmt", [("q8_0", "q4_0"), ("q8_0", "q8_0"), ("q4_0", "q4_0"), ("q5_1", "q4_0")])
+@pytest.mark.parametrize("k_fmt,v_fmt", [("q8_0", "q4_0"), ("q8_0", "q8_0"), ("q4_0", "q4_0"), ("q4_0", "q8_0"),
+                                         ("q5_1", "q4_0"), ("q5_1", "q8_0"), ("q5_0", "q4_1")])
 def test_append_bytes_bit_exact(kv_gpu, k_fmt, v_fmt):
     rng = np_rng(501)
     H, T, n_blocks = 4, 3 * 128 + 50, 5
@@ -29,6 +30,11 @@ def test_append_bytes_bit_exact(kv_gpu, k_fmt, v_fmt):
     v[11, 0, 4] = -3.0
     k[13, 1, 32:64] = 0.0                    # Q5_1 halves: m = -1, d = 0.25, (x - m) / d = k + 0.5
     k[13, 1, 32:37] = [-1.0, 6.75, -0.875, 6.625, -0.4375]
+    k[15, 3, 64:96] = 0.0                    # Q5_0 halves: m = -4, d = 0.25, x / d + 16.5 = q + 1
+    k[15, 3, 64:68] = [-4.0, 0.125, -0.375, 3.625]
+    v[15, 2, 96:128] = 0.5                   # Q4_1: a constant block gives d = 0, q = 0, m = 0.5
+    v[17, 2, 0:32] = 0.0                     # Q4_1 halves: m = -1, d = 0.25, (x - m) / d + 0.5 = k + 1
+    v[17, 2, 0:6] = [-1.0, 2.75, -0.875, -0.125, 0.875, 2.625]
     n_phys = H * n_blocks + 3
     cache = GpuCache(H, 24, n_blocks, v_fmt, n_phys=n_phys, perm=page_permutation(rng, n_phys), k_fmt=k_fmt)
     for a, b in ((0, 100), (100, 101), (101, 300), (300, T)):
