@@ -1,27 +1,34 @@
-// Chunked prefill over Q8_0 K / Q4_0 V pages on tcgen05 tensor cores (Adaptive KV
-// Streaming + RDNA 4 announcement, wqu.guru, method list: "online log-sum-exp prefill":
-// the prefill of a chunk is computed across streamed KV pages and the partial results are
-// accumulated by online log-sum-exp).
+// Chunked prefill over block-quantized KV pages (Q8_0 or Q4_0 keys, Q4_0 values) on
+// tcgen05 tensor cores (Adaptive KV Streaming + RDNA 4 announcement, wqu.guru, method list:
+// "online log-sum-exp prefill": the prefill of a chunk is computed across streamed KV pages
+// and the partial results are accumulated by online log-sum-exp; the six-step validation
+// guide, alphalab.site, build step: the q8_0-q4_0 and q4_0-q4_0 flash-attention KV pairs).
 //
-// Work unit (one CTA): a KV head h, an M-tile of 128 query rows of that head's group
-// (row r = token t * group + j: all query heads of a group share the K/V tiles, so each
-// dequantized tile serves 128 rows), and one KV split of kv_split_tokens keys, walked in
-// 64-key tiles (half pages).  Roles:
+// Work unit: a cluster of two CTAs = a KV head, two M-tiles of 128 query rows of that head's
+// group (row r = token t * group + j: all query heads of a group share the K/V tiles), and
+// one run of KV splits, walked in 64-key tiles (half pages).  The pair issues CTA-pair MMAs
+// (cta_group::2, M = 256): each CTA holds the accumulators and A operands of its own 128 rows
+// in its tensor memory, and half of every B operand in its shared memory, so each CTA
+// dequantizes half of every tile (K^ of 32 keys, V^T of 128 dimensions) and nothing is
+// copied between the CTAs.  Roles per CTA:
 //
-//   producer (1 thread)   bulk async copies (TMA engine) of a tile's raw Q8_0 K / Q4_0 V
-//                         bytes (26 KB) into a two-stage shared-memory ring
-//   dequant warps (8)     raw -> f16 with the block scales folded in (one f16 rounding):
-//                         K^ [64 keys][256] and V^T [256 dims][64 keys], K-major, 128-byte
-//                         swizzle, double-buffered
-//   MMA issuer (1 thread) S = Q K^T  (M = 128 rows, N = 64 keys, K = 256; Q from tensor memory)
-//                         O += P V   (M = 128 rows, N = 256 dims, K = 64 keys; P from tensor
-//                         memory), both accumulated in tensor memory
+//   producer (1 thread)   bulk async copies (TMA engine) of its raw K / V bytes of a tile
+//                         into a two-stage shared-memory ring
+//   dequant warps (8)     raw -> K^ and V^T, each as an f16 high part (code x scale rounded
+//                         once) and an f16 low part (the remainder, exact): together the
+//                         dequantized values exactly; K-major, 128-byte swizzle, three deep
+//   MMA issuer (1 warp,   S = Q K^T (N = 64 keys, K = 256) as Q K^_hi^T + Q K^_lo^T, and
+//     even CTA only)      O += P V (N = 256 dims, K = 64 keys) as P_hi V^_hi + P_lo V^_hi +
+//                         P_hi V^_lo; Q and P from tensor memory
 //   softmax warps (4)     thread = query row = TMEM lane: S -> causal mask -> running max
 //                         (the row of O is rescaled only when its max grows by more than
-//                         2^8) -> P = exp2(S - m) as f16 into tensor memory, over S
+//                         2^8) -> P = exp2(S log2(e) - m) split into f16 high and low parts
+//                         written over S
 //
-// Q (bf16) is converted to f16 and pre-scaled by log2(e)/16, so S is a base-2 score.  The
-// CTA writes a normalised partial (o, lse) per row; a second grid merges the splits.
+// Q (bf16) is stored as Q/16 in f16, which is exact; log2(e) is applied in fp32 to S.  Every
+// operand therefore carries the dequantized values to about 22 significant bits and the
+// products accumulate in fp32.  The CTA writes a normalised partial (o, lse) per row; a
+// second grid merges the splits.
 #include "decode.cuh"
 #include "tcgen05.cuh"
 
@@ -46,7 +53,7 @@ struct PrefillParams {
 namespace pf {
 constexpr int kRows = 128;
 constexpr int kKeys = 64;
-constexpr int kPairKeys = kKeys / 2;  // keys of a tile each CTA of a pair dequantizes
+constexpr int kHalfKeys = kKeys / 2;  // keys of a tile whose K^ this CTA holds
 constexpr int kSoftmaxWarps = 4;      // warps 0-3: TMEM lane quarters 0-3
 constexpr int kMmaWarp = 4;
 constexpr int kLoadWarp = 5;
@@ -56,32 +63,39 @@ constexpr int kDq0 = (kSoftmaxWarps + 2) * 32;  // first dequant thread
 // raw bytes a CTA copies per 64-key tile: K codes and scales of its 32 keys (contiguous in
 // the page), V codes of its 128 head dimensions for all 64 keys (four 1 KB pieces, one per
 // 16-key group), and all V scales of the tile
-constexpr int kRawKc = 8192, kRawKs = 512, kRawVc = 4096, kRawVs = 1024;
-constexpr int kRawBytes = kRawKc + kRawKs + kRawVc + kRawVs;  // 13,824
-constexpr uint32_t kHalfBytes = 16384;  // K^ or V^T bytes a CTA receives from its peer per tile
+template <int KF>
+struct Raw {
+  static constexpr int kKc = KF == kKeyQ4 ? 2048 : 8192;
+  static constexpr int kKs = 512, kVc = 4096, kVs = 1024;
+  static constexpr int kBytes = kKc + kKs + kVc + kVs;
+};
+constexpr int kRawStageBytes = Raw<kKeyQ8>::kBytes;  // 13,824 (the larger layout)
 constexpr int kRawStages = 2;
-constexpr int kBufs = 3;  // K^ and V^T buffers: dequant runs up to two tiles ahead of the MMAs
+constexpr int kBufs = 3;          // K^ / V^T buffer sets: dequant runs up to two tiles ahead of the MMAs
+constexpr int kPart = 16384;      // one of K^_hi, K^_lo (4 atoms x [32 keys][128 B]), V^T_hi, V^T_lo ([128][128 B])
+constexpr int kSet = 2 * kPart;   // hi + lo
 // a CTA walks at most this many 64-key tiles (the host plan keeps pages per CTA <= 256)
 constexpr int kMaxTiles = 512;
 // shared memory map (bytes)
-constexpr int kKOff = 0;                                  // kBufs buffers x 4 atoms x [64 keys][128 B]
-constexpr int kVOff = kKOff + kBufs * 32768;              // kBufs buffers x [256 dims][128 B]
-constexpr int kRawOff = kVOff + kBufs * 32768;            // kRawStages stages of raw tile bytes
-constexpr int kTileOff = kRawOff + kRawStages * kRawBytes;  // int2 [kMaxTiles]: page, 2*logical+half
+constexpr int kKOff = 0;                                  // kBufs x (K^_hi, K^_lo)
+constexpr int kVOff = kKOff + kBufs * kSet;               // kBufs x (V^T_hi, V^T_lo)
+constexpr int kRawOff = kVOff + kBufs * kSet;             // kRawStages stages of raw tile bytes
+constexpr int kTileOff = kRawOff + kRawStages * kRawStageBytes;  // int2 [kMaxTiles]: page, 2*logical+half
 constexpr int kMiscOff = kTileOff + 8 * kMaxTiles;
 constexpr int kSmemBytes = kMiscOff + 512;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSCol0 = 0;    // S buffers [0,64), [64,128); P (f16 pairs) over their first 32
+constexpr uint32_t kSCol0 = 0;    // S buffers [0,64), [64,128); P_hi over the first 32, P_lo over the next 32
 constexpr uint32_t kOCol0 = 128;  // O [row][256 dims]: [128, 384)
-constexpr uint32_t kQCol0 = 384;  // Q [row][256 dims] as f16 pairs: [384, 512)
-constexpr uint32_t kIdescQK = tc::idesc_f16(128, kKeys, 0, 0);
-constexpr uint32_t kIdescPV = tc::idesc_f16(128, 256, 0, 0);
+constexpr uint32_t kQCol0 = 384;  // Q / 16 [row][256 dims] as f16 pairs: [384, 512)
+constexpr uint32_t kIdescQK = tc::idesc_f16(2 * kRows, kKeys, 0, 0);
+constexpr uint32_t kIdescPV = tc::idesc_f16(2 * kRows, 256, 0, 0);
+constexpr float kLog2e = 1.4426950408889634f;
 }  // namespace pf
 
-// ---- the CTA pair (a cluster of two): shared-memory addresses in the peer, remote stores
-// and barrier arrivals, cluster-scope waits ----
+// ---- the CTA pair (a cluster of two): shared-memory addresses in the peer, barrier
+// arrivals, cluster-scope waits ----
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -93,15 +107,6 @@ __device__ __forceinline__ uint32_t map_shared(uint32_t a, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
   return r;
 }
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
-}
-// Orders this thread's shared-memory writes (its own CTA's and the peer's) before later
-// tensor-core reads of them.
-__device__ __forceinline__ void fence_proxy_async_cluster() {
-  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
-}
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
@@ -109,19 +114,6 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
 }
 __device__ __forceinline__ void sts128u(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-// Copy engine: `bytes` of this CTA's shared memory at `src` to the peer's shared memory at
-// shared::cluster address `dst`, completing the peer's barrier at `bar` by byte count.
-// Addresses and size are multiples of 16.
-__device__ __forceinline__ void bulk_s2peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-      "r"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-// Waits until every bulk copy this thread issued has completed.
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
 }
 // Named barrier over `n` threads that also ANDs a flag over them.
 __device__ __forceinline__ bool bar_and(int id, int n, bool v) {
@@ -166,8 +158,8 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
 }
 
 // The CTA's i-th candidate tile (2 per listed page): 1 if it holds a key that some row of
-// the M-tile may see (*page, *lh = 2 * logical block + half), 0 if not, -1 if its page id is
-// out of range.
+// the M-tile pair may see (*page, *lh = 2 * logical block + half), 0 if not, -1 if its page
+// id is out of range.
 __device__ __forceinline__ int pf_candidate(const PrefillParams& p, int h, int ks, int i, int np, int max_qpos,
                                             int* page_out, int* lh_out) {
   const int idx = ks * p.pages_per_split + (i >> 1);
@@ -192,10 +184,9 @@ __device__ __forceinline__ uint32_t tmem_lane(uint32_t tmem, int warp) {
   return tmem + ((static_cast<uint32_t>(warp & 3) * 32) << 16);
 }
 
-
 // Softmax pieces for one 64-key tile of S: this thread's row, loaded from tensor memory as
 // two 32-column halves.  Independent partial maxima and sums keep dependency chains short;
-// packed f32x2 arithmetic halves the subtractions and additions.
+// packed f32x2 arithmetic halves the instruction count.
 __device__ __forceinline__ void pf_mask32(uint32_t (&v)[32], int lim, int c0) {
 #pragma unroll
   for (int c = 0; c < 32; ++c)
@@ -215,20 +206,23 @@ __device__ __forceinline__ uint64_t f32x2_pack(uint32_t lo, uint32_t hi) {
   return r;
 }
 
-// P = exp2(S - mu) for 32 columns as 16 f16 pairs; returns the sum of the 32 values of P.
-__device__ __forceinline__ float pf_p32(const uint32_t (&v)[32], uint32_t mu_bits, uint32_t (&w)[16]) {
-  const uint64_t mm = f32x2_pack(mu_bits, mu_bits);
+// P = exp2(S log2(e) - mu) for 32 columns, as 16 f16 pairs of high parts (wh) and 16 of low
+// parts (wl: the rounded remainder); returns the sum of the 32 fp32 values of P.
+__device__ __forceinline__ float pf_p32(const uint32_t (&v)[32], float mu, uint32_t (&wh)[16], uint32_t (&wl)[16]) {
+  const uint64_t l2 = f32x2_pack(__float_as_uint(pf::kLog2e), __float_as_uint(pf::kLog2e));
+  const uint64_t nm = f32x2_pack(__float_as_uint(-mu), __float_as_uint(-mu));
   uint64_t acc[2] = {0ull, 0ull};  // two f32x2 partial sums (0.0f bit patterns)
 #pragma unroll
   for (int c = 0; c < 16; ++c) {
     uint64_t x = f32x2_pack(v[2 * c], v[2 * c + 1]);
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(x) : "l"(x), "l"(mm));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(x) : "l"(x), "l"(l2), "l"(nm));
     uint32_t d0, d1;
     asm("mov.b64 {%0, %1}, %2;" : "=r"(d0), "=r"(d1) : "l"(x));
     const float p0 = fast_exp2(__uint_as_float(d0)), p1 = fast_exp2(__uint_as_float(d1));
     const uint64_t pp = f32x2_pack(__float_as_uint(p0), __float_as_uint(p1));
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(acc[c & 1]) : "l"(acc[c & 1]), "l"(pp));
-    w[c] = pack_half2(p0, p1);
+    wh[c] = pack_half2(p0, p1);
+    wl[c] = pack_half2(p0 - half_lo(wh[c]), p1 - half_hi(wh[c]));
   }
   uint64_t t;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(acc[0]), "l"(acc[1]));
@@ -237,20 +231,29 @@ __device__ __forceinline__ float pf_p32(const uint32_t (&v)[32], uint32_t mu_bit
   return __uint_as_float(a) + __uint_as_float(b);
 }
 
+// f16 pair of a dequantized value as an exact high + low split: hi = f16(c * d) and
+// lo = c * d - hi (exact in f16: c has at most 8 significant bits, d 11).
+__device__ __forceinline__ void split_product(uint32_t code, uint32_t d, uint32_t& hi, uint32_t& lo) {
+  hi = hmul2(code, d);
+  lo = hfma2(code, d, hi ^ 0x80008000u);
+}
+
+template <int KF>
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillParams p) {
+  using RawF = pf::Raw<KF>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pf::kMiscOff);
   uint64_t* rawfull = bars + 0;    // [2] producer (tx bytes) -> dequant
   uint64_t* rawempty = bars + 2;   // [2] dequant -> producer
-  uint64_t* kready = bars + 4;     // [3] both halves of K^ in place (local + peer copy) -> MMA
-  uint64_t* vready = bars + 7;     // [3]
-  uint64_t* kfree = bars + 10;     // [3] QK done in both CTAs -> dequant
-  uint64_t* vfreep = bars + 13;    // [3] PV done in both CTAs -> dequant
-  uint64_t* vfree = bars + 16;     // one phase per PV of this CTA -> softmax (rescale of O)
-  uint64_t* sready = bars + 17;    // [2] MMA -> softmax
-  uint64_t* pready = bars + 19;    // [2] softmax -> MMA
-  uint64_t* ofinal = bars + 21;    // MMA -> softmax (epilogue)
-  uint64_t* qready = bars + 22;    // softmax (Q in TMEM) -> MMA
+  uint64_t* kready = bars + 4;     // [3] even CTA: K^ halves of both CTAs in place -> MMA
+  uint64_t* vready = bars + 7;     // [3] even CTA: V^T halves in place -> MMA
+  uint64_t* kfree = bars + 10;     // [3] QK done (pair commit) -> dequant
+  uint64_t* vfree = bars + 13;     // [3] PV done (pair commit) -> dequant
+  uint64_t* vdone = bars + 16;     // one phase per PV (pair commit) -> softmax (rescale of O)
+  uint64_t* sready = bars + 17;    // [2] QK done (pair commit) -> softmax
+  uint64_t* pready = bars + 19;    // [2] even CTA: P of both CTAs written -> MMA
+  uint64_t* ofinal = bars + 21;    // every MMA done (pair commit) -> epilogue, tensor-memory release
+  uint64_t* qready = bars + 22;    // even CTA: Q of both CTAs in tensor memory -> MMA
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bars + 23);
   int* s_abort = reinterpret_cast<int*>(tmem_base_s + 1);
   int* s_ntiles = s_abort + 1;
@@ -262,15 +265,16 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
   const int row0 = mt * pf::kRows;
   int np = p.max_pages;
   if (p.n_pages_arr) np = min(max(p.n_pages_arr[h], 0), p.max_pages);
-  // largest query position among this M-tile's rows: keys beyond it are never visible
-  // (over both M-tiles of the pair: the two CTAs walk the same tiles)
+  // largest query position among the rows of the M-tile pair: keys beyond it are never
+  // visible (the two CTAs walk the same tiles)
   int max_qpos = INT_MIN;
   {
     const int pair_row0 = (mt & ~1) * pf::kRows;
     const int t0 = pair_row0 / p.group, t1 = min(n_rows - 1, pair_row0 + 2 * pf::kRows - 1) / p.group;
     for (int t = t0; t <= t1; ++t) max_qpos = max(max_qpos, p.q_pos[t]);
   }
-  const uint32_t crank = cluster_rank(), peer = crank ^ 1u;
+  const uint32_t crank = cluster_rank();
+  const bool leader = crank == 0;
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < pf::kRawStages; ++b) {
@@ -278,18 +282,18 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       mbar_init(&rawempty[b], pf::kDequantWarps);
     }
     for (int b = 0; b < pf::kBufs; ++b) {
-      mbar_init(&kready[b], 1);  // + the peer's half as transaction bytes
-      mbar_init(&vready[b], 1);
-      mbar_init(&kfree[b], 2);
-      mbar_init(&vfreep[b], 2);
+      mbar_init(&kready[b], 2);  // one arrival from the dequant warps of each CTA
+      mbar_init(&vready[b], 2);
+      mbar_init(&kfree[b], 1);
+      mbar_init(&vfree[b], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sready[b], 1);
-      mbar_init(&pready[b], pf::kSoftmaxWarps);
+      mbar_init(&pready[b], 2 * pf::kSoftmaxWarps);
     }
-    mbar_init(vfree, 1);
+    mbar_init(vdone, 1);
     mbar_init(ofinal, 1);
-    mbar_init(qready, pf::kSoftmaxWarps);
+    mbar_init(qready, 2 * pf::kSoftmaxWarps);
     *s_abort = 0;
     if (smem_u32(smem) & 1023) record_error(KVATTN_ERR_INVALID_ARG);
     fence_barrier_init();
@@ -314,12 +318,12 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     if (lane == 0) *s_ntiles = cnt;
   }
   if (warp == pf::kMmaWarp) {
-    tc::tmem_alloc(tmem_base_s, pf::kTmemCols);
-    tc::tmem_relinquish();
+    tc::tmem_alloc_pair(tmem_base_s, pf::kTmemCols);
+    tc::tmem_relinquish_pair();
   }
   tc::fence_before_sync();
   __syncthreads();
-  cluster_sync();  // both CTAs' barriers are initialised before any remote arrival or store
+  cluster_sync();  // both CTAs' barriers are initialised before any remote arrival
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_base_s;
   const int n_tiles = *s_ntiles;
@@ -337,16 +341,17 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         }
         // K: this CTA's 32 keys of the tile (quarter q of the page); V: its 128 dimensions
         const int half = tl.y & 1, q = 2 * half + static_cast<int>(crank);
-        uint8_t* st = smem + pf::kRawOff + r * pf::kRawBytes;
+        uint8_t* st = smem + pf::kRawOff + r * pf::kRawStageBytes;
         const uint8_t* kp = p.k_pool + static_cast<int64_t>(tl.x) * p.k_stride;
         const uint8_t* vp = p.v_pool + static_cast<int64_t>(tl.x) * p.v_stride;
-        mbar_arrive_expect_tx(&rawfull[r], pf::kRawBytes);
-        bulk_g2s(st, kp + q * pf::kRawKc, pf::kRawKc, &rawfull[r]);
-        bulk_g2s(st + pf::kRawKc, kp + kKScaleOffset + q * pf::kRawKs, pf::kRawKs, &rawfull[r]);
+        constexpr int kScaleOff = KF == kKeyQ4 ? kK4ScaleOffset : kKScaleOffset;
+        mbar_arrive_expect_tx(&rawfull[r], RawF::kBytes);
+        bulk_g2s(st, kp + q * RawF::kKc, RawF::kKc, &rawfull[r]);
+        bulk_g2s(st + RawF::kKc, kp + kScaleOff + q * RawF::kKs, RawF::kKs, &rawfull[r]);
         for (int g = 0; g < 4; ++g)
-          bulk_g2s(st + pf::kRawKc + pf::kRawKs + g * 1024, vp + half * 8192 + g * 2048 + crank * 1024, 1024,
+          bulk_g2s(st + RawF::kKc + RawF::kKs + g * 1024, vp + half * 8192 + g * 2048 + crank * 1024, 1024,
                    &rawfull[r]);
-        bulk_g2s(st + pf::kRawKc + pf::kRawKs + pf::kRawVc, vp + kV4ScaleOffset + half * pf::kRawVs, pf::kRawVs,
+        bulk_g2s(st + RawF::kKc + RawF::kKs + RawF::kVc, vp + kV4ScaleOffset + half * RawF::kVs, RawF::kVs,
                  &rawfull[r]);
       }
       // every copy issued must land before the CTA may exit
@@ -354,19 +359,19 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         mbar_wait(&rawfull[jj % pf::kRawStages], (jj / pf::kRawStages) & 1);
     }
   } else if (warp == pf::kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ MMA issuer (even CTA)
     // The whole warp runs this loop (one elected lane issues each instruction); barrier
     // checks are made warp-uniform so the lanes never diverge around elect.sync.  Each pass
-    // issues whichever is ready of QK of the next tile (once its K^ is in place and the S
-    // buffer it overwrites was consumed by PV two tiles back) and PV of the oldest tile whose
-    // P is written, so a late K^ does not hold back a ready PV.
-    {
+    // issues whichever is ready of QK of the next tile (once both CTAs' K^ halves are in
+    // place and the S buffer it overwrites was consumed by PV two tiles back) and PV of the
+    // oldest tile whose P is written in both CTAs.
+    if (leader) {
       const uint32_t k_base = smem_u32(smem + pf::kKOff);
       const uint32_t v_base = smem_u32(smem + pf::kVOff);
       auto ready_all = [&](uint64_t* bar, uint32_t par) -> bool {
         return __all_sync(0xffffffffu, mbar_try_wait_cluster(bar, par, 0u));
       };
-      bool ok = __all_sync(0xffffffffu, mbar_wait(qready, 0));
+      bool ok = __all_sync(0xffffffffu, mbar_wait_cluster(qready, 0));
       int jq = 0, jp = 0;  // next QK, next PV
       unsigned long long t_idle = 0;
       while (ok && jp < n_tiles) {
@@ -376,12 +381,13 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
           tc::fence_after_sync();
 #pragma unroll
           for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-            const uint64_t bd = tc::sw128_desc(k_base + b * 32768 + (kk >> 2) * 8192 + (kk & 3) * 32, 1024, 16);
-            tc::mma_f16_ts_warp(tmem + pf::kSCol0 + s2 * pf::kKeys, tmem + pf::kQCol0 + kk * 8, bd, pf::kIdescQK,
-                                kk > 0 ? 1u : 0u);
+            const uint32_t ka = k_base + b * pf::kSet + (kk >> 2) * 4096 + (kk & 3) * 32;
+            const uint32_t dcol = tmem + pf::kSCol0 + s2 * pf::kKeys, qcol = tmem + pf::kQCol0 + kk * 8;
+            tc::mma_f16_ts_pair_warp(dcol, qcol, tc::sw128_desc(ka, 1024, 16), pf::kIdescQK, kk > 0 ? 1u : 0u);
+            tc::mma_f16_ts_pair_warp(dcol, qcol, tc::sw128_desc(ka + pf::kPart, 1024, 16), pf::kIdescQK, 1u);
           }
-          tc::commit_warp(&sready[s2]);
-          tc::commit_pair_warp(&kfree[b]);
+          tc::commit_pair2_warp(&sready[s2]);
+          tc::commit_pair2_warp(&kfree[b]);
           ++jq;
           did = true;
         } else if (jp < jq && ready_all(&pready[jp & 1], (jp >> 1) & 1) &&
@@ -390,12 +396,15 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
           tc::fence_after_sync();
 #pragma unroll
           for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
-            const uint64_t bd = tc::sw128_desc(v_base + b * 32768 + kk * 32, 1024, 16);
-            tc::mma_f16_ts_warp(tmem + pf::kOCol0, tmem + pf::kSCol0 + s2 * pf::kKeys + kk * 8, bd, pf::kIdescPV,
-                                (jp > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t va = v_base + b * pf::kSet + kk * 32;
+            const uint32_t ph = tmem + pf::kSCol0 + s2 * pf::kKeys + kk * 8, pl = ph + pf::kKeys / 2;
+            const uint64_t vh = tc::sw128_desc(va, 1024, 16), vl = tc::sw128_desc(va + pf::kPart, 1024, 16);
+            tc::mma_f16_ts_pair_warp(tmem + pf::kOCol0, ph, vh, pf::kIdescPV, (jp > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_f16_ts_pair_warp(tmem + pf::kOCol0, pl, vh, pf::kIdescPV, 1u);
+            tc::mma_f16_ts_pair_warp(tmem + pf::kOCol0, ph, vl, pf::kIdescPV, 1u);
           }
-          tc::commit_warp(vfree);
-          tc::commit_pair_warp(&vfreep[b]);
+          tc::commit_pair2_warp(vdone);
+          tc::commit_pair2_warp(&vfree[b]);
           ++jp;
           did = true;
         }
@@ -414,23 +423,25 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         ok = __all_sync(0xffffffffu, ok);
       }
       if (!ok && lane == 0) *s_abort = 1;
-      tc::commit_warp(ofinal);  // arrives when every MMA above has completed
-      __all_sync(0xffffffffu, mbar_wait(ofinal, 0));  // no MMA may still run when TMEM is freed
+      tc::commit_pair2_warp(ofinal);  // arrives in both CTAs when every MMA above has completed
     }
+    // no MMA may still write this CTA's tensor memory when it is freed
+    __all_sync(0xffffffffu, mbar_wait_cluster(ofinal, 0));
   } else if (warp < pf::kSoftmaxWarps) {
     // ------------------------------------------------------------ softmax (thread = row)
     const int r = threadIdx.x;  // 0..127 == TMEM lane
     const int R = row0 + r;
     const int qpos = R < n_rows ? p.q_pos[R / p.group] : INT_MAX;
     const uint32_t lane_base = tmem_lane(tmem, warp);
-    // ---- Q row: bf16 -> f16 * log2(e)/16 into tensor memory (A operand of S = Q K^T) ----
+    const uint32_t qready_lead = map_shared(smem_u32(qready), 0);
+    const uint32_t pready_lead = map_shared(smem_u32(&pready[0]), 0);
+    // ---- Q row: bf16 -> f16 of q / 16 (exact) into tensor memory (A operand of S = Q K^T) ----
     {
       const uint16_t* src = nullptr;
       if (R < n_rows) {
         const int t = R / p.group, jq = R % p.group;
         src = p.q + (static_cast<long long>(t) * p.n_qh + h * p.group + jq) * kHeadDim;
       }
-      const float sc = 1.4426950408889634f / 16.0f;
       for (int c0 = 0; c0 < 4; ++c0) {  // 64 channels = 32 columns at a time
         uint32_t w[32];
 #pragma unroll
@@ -440,27 +451,28 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
           const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            w[c * 4 + e] = pack_half2(__uint_as_float(in[e] << 16) * sc, __uint_as_float(in[e] & 0xFFFF0000u) * sc);
+            w[c * 4 + e] =
+                pack_half2(__uint_as_float(in[e] << 16) * 0.0625f, __uint_as_float(in[e] & 0xFFFF0000u) * 0.0625f);
         }
         tc::st32(lane_base + pf::kQCol0 + c0 * 32, w);
       }
       tc::wait_st();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(qready);
+      if (lane == 0) mbar_arrive_cluster(qready_lead);
     }
-    float m_ref = -INFINITY, l_sum = 0.f;
+    float m_ref = -INFINITY, l_sum = 0.f;  // base-2 units
     int j = 0;
     bool ok = true;
     for (; j < n_tiles && ok; ++j) {
       const int2 tl = tiles[j];
       const int b = j & 1;
-      if (!mbar_wait(&sready[b], (j >> 1) & 1)) {
+      if (!mbar_wait_cluster(&sready[b], (j >> 1) & 1)) {
         ok = false;
         break;
       }
       tc::fence_after_sync();
-      // the 64 scores in one tensor-memory round trip; P overwrites their first 32 columns
+      // the 64 scores in one tensor-memory round trip; P overwrites them
       const int lim = qpos - tl.y * pf::kKeys;  // columns beyond lim are in this row's future
       const uint32_t scol = lane_base + pf::kSCol0 + b * pf::kKeys;
       uint32_t v0[32], v1[32];
@@ -471,7 +483,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         pf_mask32(v0, lim, 0);
         pf_mask32(v1, lim, 32);
       }
-      const float mx = fmaxf(pf_max32(v0), pf_max32(v1));
+      const float mx = fmaxf(pf_max32(v0), pf_max32(v1)) * pf::kLog2e;
       float alpha = 1.f;
       bool resc = false;
       if (mx > m_ref + 8.f) {
@@ -482,16 +494,18 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       }
       const float mu = m_ref == -INFINITY ? 0.f : m_ref;
       {
-        uint32_t w[16];
-        l_sum += pf_p32(v0, __float_as_uint(mu), w);
-        tc::st16(scol, w);
-        l_sum += pf_p32(v1, __float_as_uint(mu), w);
-        tc::st16(scol + 16, w);
+        uint32_t wh[16], wl[16];
+        l_sum += pf_p32(v0, mu, wh, wl);
+        tc::st16(scol, wh);
+        tc::st16(scol + 32, wl);
+        l_sum += pf_p32(v1, mu, wh, wl);
+        tc::st16(scol + 16, wh);
+        tc::st16(scol + 48, wl);
       }
       if (__any_sync(0xffffffffu, resc)) {
         // O is rescaled to the new maximum before PV of this tile accumulates into it; this
         // warp's rows of O hold the previous tile's PV only once that completed
-        if (!mbar_wait(vfree, (j - 1) & 1)) {
+        if (!mbar_wait_cluster(vdone, (j - 1) & 1)) {
           ok = false;
           break;
         }
@@ -509,12 +523,12 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       tc::wait_st();
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&pready[b]);
+      if (lane == 0) mbar_arrive_cluster(pready_lead + 8 * b);
     }
     // ---- epilogue: normalised partial (o, lse) of this row ----
     bool have = false;
     if (ok && j > 0) {
-      have = mbar_wait(ofinal, 0);
+      have = mbar_wait_cluster(ofinal, 0);
       ok = have;
     }
     if (!ok) *s_abort = 1;
@@ -560,16 +574,14 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     }
   } else if (warp >= pf::kDq0 / 32) {
     // ------------------------------------------------------------ dequant (256 threads)
-    // This CTA dequantizes half of every tile (K^: its 32 keys; V^T: its 128 dimensions) into
-    // its own buffers; one thread then copies that half into the peer's buffers with the
-    // copy engine, which completes the peer's barrier by byte count.
+    // This CTA dequantizes its half of every tile (K^: its 32 keys; V^T: its 128 dimensions)
+    // into its own buffers, as exact high + low f16 parts, then one thread tells the even CTA.
     const int d = threadIdx.x - pf::kDq0;
     // K task: key kl of this CTA's 32, channel quarter kP (blocks 2kP, 2kP+1), raw chunks
     // 2cp and 2cp+1 of the four; 8 consecutive threads take 8 consecutive keys, so their
     // swizzled 16-byte stores hit 8 different bank groups.
     const int kl = d & 31, kP = (d >> 5) & 3, cp = d >> 7;
     const int kGl = kl >> 4, kH = (kl >> 3) & 1, kR = kl & 7;
-    const int kn = pf::kPairKeys * static_cast<int>(crank) + kl;  // row of K^ (key within the tile)
     // V task: channel row vR (channels vR + 8k of block 2vC + ve, vC = 2 * rank + vCl), key
     // half vh of token group vG (16 keys)
     const int vR = d & 7, vh = (d >> 3) & 1, vCl = (d >> 4) & 1, vG = (d >> 5) & 3, ve = d >> 7;
@@ -577,9 +589,9 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     // 16-byte chunks are read in an order rotated by (row / 2): 8 threads at a 64-byte
     // stride then touch 8 different bank groups
     const int rotK = kR >> 1, rotV = vR >> 1;
-    const uint32_t own = smem_u32(smem), other = map_shared(own, peer);
-    const uint32_t kready_peer = map_shared(smem_u32(&kready[0]), peer);
-    const uint32_t vready_peer = map_shared(smem_u32(&vready[0]), peer);
+    const uint32_t own = smem_u32(smem);
+    const uint32_t kready_lead = map_shared(smem_u32(&kready[0]), 0);
+    const uint32_t vready_lead = map_shared(smem_u32(&vready[0]), 0);
     int j = 0;
     bool ok = true;
     for (; j < n_tiles && ok; ++j) {
@@ -587,49 +599,79 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       // every wait result is combined over the 256 dequant threads at the named barriers, so
       // all of them stop at the same tile when one gives up
       bool wok = mbar_wait(&rawfull[r], (j / pf::kRawStages) & 1);
-      const uint32_t stu = own + pf::kRawOff + r * pf::kRawBytes;
+      const uint32_t stu = own + pf::kRawOff + r * pf::kRawStageBytes;
       // ---------------- raw K, V -> registers; the stage is then released ----------------
-      uint4 kraw[2] = {};
+      uint32_t kw[2][4] = {};  // per chunk i: the 4 words (8 codes of block 2kP, 8 of 2kP + 1)
       uint32_t dkw = 0;
       uint2 vraw[4] = {}, dvr[4] = {};
       if (wok) {
-        const uint32_t kbase = stu + ((((kGl * 4 + kP) * 2 + kH) * 8 + kR) * 4) * 16;
+        if constexpr (KF == kKeyQ4) {
+          // Q4_0 key words of token kl, blocks 2kP, 2kP + 1 (c = 2kP % 4, 2kP % 4 + 1) of block
+          // quad Q = kP / 2, lane column T: one 8-byte load per chunk
 #pragma unroll
-        for (int i = 0; i < 2; ++i) kraw[i] = lds128(kbase + (((2 * cp + i + rotK) & 3) << 4));
+          for (int i = 0; i < 2; ++i) {
+            const int T = (2 * cp + i + rotK) & 3;
+            const uint2 w2 =
+                lds64(stu + 4 * (((((kGl * 2 + (kP >> 1)) * 2 + kH) * 8 + kR) * 4 + T) * 4 + ((2 * kP) & 3)));
+            kw[i][0] = w2.x;
+            kw[i][1] = w2.y;
+          }
+        } else {
+          const uint32_t kbase = stu + ((((kGl * 4 + kP) * 2 + kH) * 8 + kR) * 4) * 16;
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const uint4 c = lds128(kbase + (((2 * cp + i + rotK) & 3) << 4));
+            kw[i][0] = c.x; kw[i][1] = c.y; kw[i][2] = c.z; kw[i][3] = c.w;
+          }
+        }
         asm volatile("ld.shared.u32 %0, [%1];"
                      : "=r"(dkw)
-                     : "r"(stu + pf::kRawKc + ((kGl * 8 + kR) * 2 + kH) * 16 + 4 * kP));
+                     : "r"(stu + RawF::kKc + ((kGl * 8 + kR) * 2 + kH) * 16 + 4 * kP));
         // this thread's two words (block 2vC + ve, both key halves) of each raw chunk and of
         // the scales of each token pair
-        const uint32_t vbase = stu + pf::kRawKc + pf::kRawKs + vG * 1024 + ((vCl * 8 + vR) * 4) * 16 + 8 * ve;
+        const uint32_t vbase = stu + RawF::kKc + RawF::kKs + vG * 1024 + ((vCl * 8 + vR) * 4) * 16 + 8 * ve;
 #pragma unroll
         for (int ii = 0; ii < 4; ++ii) vraw[ii] = lds64(vbase + (((ii + rotV) & 3) << 4));
 #pragma unroll
         for (int T = 0; T < 4; ++T)
-          dvr[T] = lds64(stu + pf::kRawKc + pf::kRawKs + pf::kRawVc + ((vG * 4 + T) * 8 + 2 * vC) * 8 + 8 * ve);
+          dvr[T] = lds64(stu + RawF::kKc + RawF::kKs + RawF::kVc + ((vG * 4 + T) * 8 + 2 * vC) * 8 + 8 * ve);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&rawempty[r]);
-      // ---------------- K^ (both CTAs' buffers are free once both QK(j - 3) completed) ----
+      // ---------------- K^ (this CTA's buffer is free once QK(j - 3) completed) ----
       if (wok && j >= pf::kBufs) wok = mbar_wait_cluster(&kfree[b], ((j / pf::kBufs) - 1) & 1);
-      const uint32_t katom0 = pf::kKOff + b * 32768;
+      const uint32_t katom = own + pf::kKOff + b * pf::kSet + kP * 4096;
       if (wok) {
         const uint32_t dlo = prmt(dkw, 0u, 0x1010u), dhi = prmt(dkw, 0u, 0x3232u);
-        const uint32_t katom = katom0 + kP * 8192;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           const int T = (2 * cp + i + rotK) & 3;
-          const uint32_t w[4] = {kraw[i].x ^ 0x80808080u, kraw[i].y ^ 0x80808080u, kraw[i].z ^ 0x80808080u,
-                                 kraw[i].w ^ 0x80808080u};
-          uint32_t o[8];
+          uint32_t c[8];  // exact codes as f16 pairs: c[0..3] block 2kP, c[4..7] block 2kP + 1
+          if constexpr (KF == kKeyQ4) {
+            // channel i' of a word at bit 4(i'/2) + 16(i'%2): pairs (0,1), (2,3), (4,5), (6,7)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t sc = e < 2 ? dlo : dhi;
-            o[2 * e] = hmul2(hsub2(prmt(w[e], 0x64646464u, 0x4140u), 0x64806480u), sc);
-            o[2 * e + 1] = hmul2(hsub2(prmt(w[e], 0x64646464u, 0x4342u), 0x64806480u), sc);
+            for (int e = 0; e < 2; ++e) {
+              const uint32_t w = kw[i][e], ws = w >> 8;
+              c[4 * e + 0] = hsub2(and_or(w, 0x000F000Fu, 0x64006400u), 0x64086408u);
+              c[4 * e + 1] = hfma2(and_or(w, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
+              c[4 * e + 2] = hsub2(and_or(ws, 0x000F000Fu, 0x64006400u), 0x64086408u);
+              c[4 * e + 3] = hfma2(and_or(ws, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t w = kw[i][e] ^ 0x80808080u;
+              c[2 * e] = hsub2(prmt(w, 0x64646464u, 0x4140u), 0x64806480u);
+              c[2 * e + 1] = hsub2(prmt(w, 0x64646464u, 0x4342u), 0x64806480u);
+            }
           }
-          sts128u(own + katom + swz(kn, T), o[0], o[1], o[2], o[3]);
-          sts128u(own + katom + swz(kn, 4 + T), o[4], o[5], o[6], o[7]);
+          uint32_t oh[8], ol[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) split_product(c[e], e < 4 ? dlo : dhi, oh[e], ol[e]);
+          sts128u(katom + swz(kl, T), oh[0], oh[1], oh[2], oh[3]);
+          sts128u(katom + swz(kl, 4 + T), oh[4], oh[5], oh[6], oh[7]);
+          sts128u(katom + pf::kPart + swz(kl, T), ol[0], ol[1], ol[2], ol[3]);
+          sts128u(katom + pf::kPart + swz(kl, 4 + T), ol[4], ol[5], ol[6], ol[7]);
         }
         tc::fence_proxy_async_smem();
       }
@@ -637,19 +679,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         ok = false;
         break;
       }
-      if (d == 0) {
-        // this CTA's 32 rows of each of the four K^ atoms -> the peer; the peer's half comes
-        // the other way as transaction bytes on kready
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          const uint32_t off = katom0 + a * 8192 + crank * 4096;
-          bulk_s2peer(other + off, own + off, 4096, kready_peer + 8 * b);
-        }
-        mbar_arrive_expect_tx(&kready[b], pf::kHalfBytes);
-      }
-      // ---------------- V^T: rows 128 * rank .. of the buffer ----------------
-      if (j >= pf::kBufs) wok = mbar_wait_cluster(&vfreep[b], ((j / pf::kBufs) - 1) & 1);
-      const uint32_t vt = pf::kVOff + b * 32768;
+      if (d == 0) mbar_arrive_cluster(kready_lead + 8 * b);
+      // ---------------- V^T: this CTA's 128 dimensions ----------------
+      if (j >= pf::kBufs) wok = mbar_wait_cluster(&vfree[b], ((j / pf::kBufs) - 1) & 1);
+      const uint32_t vt = own + pf::kVOff + b * pf::kSet;
       if (wok) {
         // chunk ii holds token pair (ii + rotV) & 3: two select stages undo the rotation so
         // that wv[T] is token pair T (an array indexed by the runtime rotation would be
@@ -661,7 +694,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         for (int x = 0; x < 4; ++x) t[x] = (rotV & 1) ? wv[(x + 3) & 3] : wv[x];
 #pragma unroll
         for (int x = 0; x < 4; ++x) wv[x] = (rotV & 2) ? t[(x + 2) & 3] : t[x];
-        uint32_t o[4][4];  // [k][T]
+        uint32_t oh[4][4], ol[4][4];  // [k][T]
 #pragma unroll
         for (int T = 0; T < 4; ++T) {
           const uint32_t W = wv[T];
@@ -671,15 +704,16 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
           const uint32_t v1 = hfma2(and_or(W, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
           const uint32_t v2 = hsub2(and_or(Ws, 0x000F000Fu, 0x64006400u), 0x64086408u);
           const uint32_t v3 = hfma2(and_or(Ws, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
-          o[0][T] = hmul2(v0, dv);
-          o[1][T] = hmul2(v1, dv);
-          o[2][T] = hmul2(v2, dv);
-          o[3][T] = hmul2(v3, dv);
+          split_product(v0, dv, oh[0][T], ol[0][T]);
+          split_product(v1, dv, oh[1][T], ol[1][T]);
+          split_product(v2, dv, oh[2][T], ol[2][T]);
+          split_product(v3, dv, oh[3][T], ol[3][T]);
         }
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int dim = 32 * (2 * vC + ve) + 8 * k + vR;
-          sts128u(own + vt + swz(dim, 2 * vG + vh), o[k][0], o[k][1], o[k][2], o[k][3]);
+          const int row = 32 * (2 * vCl + ve) + 8 * k + vR;  // dimension - 128 * rank
+          sts128u(vt + swz(row, 2 * vG + vh), oh[k][0], oh[k][1], oh[k][2], oh[k][3]);
+          sts128u(vt + pf::kPart + swz(row, 2 * vG + vh), ol[k][0], ol[k][1], ol[k][2], ol[k][3]);
         }
         tc::fence_proxy_async_smem();
       }
@@ -687,30 +721,27 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         ok = false;
         break;
       }
-      if (d == 0) {
-        const uint32_t off = vt + crank * pf::kHalfBytes;
-        bulk_s2peer(other + off, own + off, pf::kHalfBytes, vready_peer + 8 * b);
-        mbar_arrive_expect_tx(&vready[b], pf::kHalfBytes);
-      }
+      if (d == 0) mbar_arrive_cluster(vready_lead + 8 * b);
     }
     if (!ok) *s_abort = 1;
-    // the copies this CTA sent must have landed before either CTA may leave
-    if (d == 0) bulk_wait_all();
   }
 
   tc::fence_before_sync();
   __syncthreads();
-  // the peer stores into and arrives on this CTA's shared memory until it gets here
+  // the peer arrives on this CTA's barriers until it gets here
   cluster_sync();
   if (*s_abort && threadIdx.x == 0) record_error(KVATTN_ERR_TIMEOUT);
   if (warp == pf::kMmaWarp) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, pf::kTmemCols);
+    tc::tmem_dealloc_pair(tmem, pf::kTmemCols);
   }
 }
 
 cudaError_t prepare_prefill_kernels() {
-  return cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<kKeyQ8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       pf::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(prefill_kernel<kKeyQ4>, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::kSmemBytes);
 }
 
 struct PrefillPlan {
@@ -741,7 +772,7 @@ PrefillPlan plan_prefill(int n_kv, int group, int n_q, int max_pages, int kv_spl
   return pl;
 }
 
-cudaError_t launch_prefill(const PrefillParams& prm0, int n_kv, cudaStream_t stream) {
+cudaError_t launch_prefill(const PrefillParams& prm0, int n_kv, int key_fmt, cudaStream_t stream) {
   PrefillParams prm = prm0;
   const int rows = prm.n_q * prm.group;
   {
@@ -757,7 +788,8 @@ cudaError_t launch_prefill(const PrefillParams& prm0, int n_kv, cudaStream_t str
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_kernel, prm);
+    cudaError_t e = key_fmt == kKeyQ4 ? cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ4>, prm)
+                                      : cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ8>, prm);
     if (e != cudaSuccess || prm.n_ks == 1) return e;
   }
   cudaLaunchConfig_t cfg = {};

@@ -1,6 +1,6 @@
 // Thin inline-PTX wrappers for the sm_100a tensor-core path: tensor-memory allocation,
-// tcgen05.mma (kind::f16, single CTA), commits to mbarriers, tensor-memory loads/stores,
-// shared-memory matrix descriptors and instruction descriptors.
+// tcgen05.mma (kind::f16, one CTA or a CTA pair), commits to mbarriers, tensor-memory
+// loads/stores, shared-memory matrix descriptors and instruction descriptors.
 #pragma once
 
 #include "common.cuh"
@@ -20,6 +20,20 @@ __device__ __forceinline__ void tmem_relinquish() {
 }
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// The same for a CTA pair (cta_group::2): one warp with the same warp index in each of the two
+// CTAs of the cluster calls it; both get the same columns of their own tensor memory.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
 __device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -53,6 +67,34 @@ __device__ __forceinline__ void mma_f16_ts_warp(uint32_t d_tmem, uint32_t a_tmem
       "setp.ne.b32 p, %4, 0;\n\t"
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// CTA-pair MMA (cta_group::2, issued by the even CTA of the cluster for both): D rows
+// [0, M/2) in the even CTA's tensor memory and [M/2, M) in the odd CTA's, A likewise from
+// each CTA's own tensor memory at the same address; B's N columns split in halves, the first
+// in the even CTA's shared memory and the second in the odd CTA's, both at the address of
+// b_desc.  Executed by a whole converged warp; one elected lane issues.
+__device__ __forceinline__ void mma_f16_ts_pair_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                     uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrives on the barrier at the same shared-memory offset in both CTAs of the pair once all
+// CTA-pair MMAs issued so far by this thread complete (from a converged warp, one lane).
+__device__ __forceinline__ void commit_pair2_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t.reg .b16 m;\n\t"
+      "mov.b16 m, 3;\n\t"
+      "elect.sync r|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
+          smem_u32(bar))
       : "memory");
 }
 
