@@ -23,6 +23,8 @@
  *           18 bytes per 32 elements; only legacy block quants are valid KV formats) and
  *           configs (q8_0 = 8.5 bits per element); summary (a q4_0/q4_0 cache holds the most
  *           tokens).
+ *  [MTP]    7900 XTX llama.cpp MTP tuning notes (lcz.me/topic/593): a server command with a
+ *           q5_0 K / q4_1 V cache at 131,072 context.
  *
  * Data formats (fixed by this library; the pages fix only the bits per element):
  *  - head_dim = 256, page = 128 tokens of one (layer, KV head).
@@ -30,27 +32,31 @@
  *    Q4_0: blocks of 32 4-bit codes q in [0,15] + fp16 d; value = (q - 8) * d.
  *    Q5_1: blocks of 32 5-bit codes q in [0,31] + fp16 d + fp16 minimum m; value = q * d + m
  *    ([VULKAN] pitfalls: 6 bits per element, a zero point; paired with Q4_0 values).
- *  - Format pairs: Q8_0 K with Q4_0 or Q8_0 V, and Q4_0 or Q5_1 K with Q4_0 V.  K pages are
- *    Q8_0 (34,816 B), Q4_0 (18,432 B) or Q5_1 (24,576 B); V pages are Q4_0 (18,432 B) or Q8_0
- *    (34,816 B).  Inside a
+ *    Q5_0: 5-bit codes q in [0,31] + fp16 d; value = (q - 16) * d.  Q4_1: 4-bit codes q in
+ *    [0,15] + fp16 d + fp16 minimum m; value = q * d + m ([VULKAN] pitfalls lists both among
+ *    the KV types; [MTP] runs a Q5_0 K / Q4_1 V cache).
+ *  - Format pairs: Q8_0, Q4_0 or Q5_1 K with Q4_0 or Q8_0 V, and Q5_0 K with Q4_1 V.  K pages
+ *    are Q8_0 (34,816 B), Q4_0 (18,432 B), Q5_1 (24,576 B) or Q5_0 (22,528 B); V pages are Q4_0
+ *    (18,432 B), Q8_0 (34,816 B) or Q4_1 (20,480 B).  Inside a
  *    page, codes come first and fp16 scales after them, both in tensor-core fragment order
  *    (tok = slot in page, c = channel, b = c/32, G = tok/16):
  *      K Q8_0 code  (tok = 16G+8H+R, c = 64P+32(j/8)+8T+j%8) at ((((G*4+P)*2+H)*8+R)*4+T)*16+j
  *      K Q4_0 word  (tok = 16G+8H+R, b = 4Q+c, channels 32b+8T+i, i < 8) is the little-endian
  *                   uint32 at 4*(((((G*2+Q)*2+H)*8+R)*4+T)*4+c); channel i's 4-bit code sits
  *                   at bit 4*(i/2) + 16*(i%2)
- *      K Q5_1       low 4 bits of each code as the K Q4_0 word; bit 4 of the codes of token
+ *      K Q5_1/Q5_0  low 4 bits of each code as the K Q4_0 word; bit 4 of the codes of token
  *                   16G+8H+R, channels 32(4Q+c)+8T+i in the uint32 at
  *                   16384 + 4*((((G*2+Q)*2+H)*8+R)*4+T), channel (c, i) at bit 16(i%2)+4c+i/2;
- *                   minimum m[16G+8H+R][b] at 22528 + 2*(((G*8+R)*2+H)*8+b)
+ *                   Q5_1 minimum m[16G+8H+R][b] at 22528 + 2*(((G*8+R)*2+H)*8+b)
  *      K scale      d[16G+8H+R][b] at S + 2*(((G*8+R)*2+H)*8+b), S = 32768 (Q8_0), 16384
- *                   (Q4_0) or 20480 (Q5_1)
+ *                   (Q4_0) or 20480 (Q5_1, Q5_0)
  *      V Q4_0 byte  ((((G*4+C)*8+R)*4+T)*16 + 4w + y: block b = 2C+w/2, token
  *                   16G+2T+8(w%2)+y/2; low nibble c = 32b+16(y%2)+R, high nibble c+8
  *      V Q8_0 code  (tok = 16G+2T+8(w%2)+y%2, c = 32b+16(w/2)+8(y/2)+R) at
  *                   ((((G*8+b)*8+R)*4+T)*16 + 4w + y
- *      V scale      d[16G+2T+k%2+8(k/2)][b] at S + 2*(((G*4+T)*8+b)*4+k), S = 16384 (Q4_0)
- *                   or 32768 (Q8_0)
+ *      V Q4_1 byte  as the V Q4_0 byte (the code is q, not q - 8)
+ *      V scale      d[16G+2T+k%2+8(k/2)][b] at S + 2*(((G*4+T)*8+b)*4+k), S = 16384 (Q4_0,
+ *                   Q4_1) or 32768 (Q8_0); Q4_1 minima in the same arrangement at 18432
  *    kvattn_quantize_append is the supported writer.
  *  - Pages live in caller-owned pools: page p's K bytes start at k_pool + p * k_page_stride
  *    and its V bytes at v_pool + p * v_page_stride.  Pool bases and strides are multiples
@@ -97,7 +103,13 @@ enum kvattn_status {
   KVATTN_ERR_NOT_INITIALIZED = -9     /* kvattn_init was not called for the current device  */
 };
 
-enum kvattn_format { KVATTN_FMT_Q4_0 = 4, KVATTN_FMT_Q8_0 = 8, KVATTN_FMT_Q5_1 = 51 };
+enum kvattn_format {
+  KVATTN_FMT_Q4_0 = 4,
+  KVATTN_FMT_Q8_0 = 8,
+  KVATTN_FMT_Q5_1 = 51,
+  KVATTN_FMT_Q5_0 = 50, /* keys only  */
+  KVATTN_FMT_Q4_1 = 41  /* values only */
+};
 enum kvattn_role { KVATTN_ROLE_K = 0, KVATTN_ROLE_V = 1 };
 
 typedef struct kvattn_kv_desc {
@@ -105,8 +117,8 @@ typedef struct kvattn_kv_desc {
   int32_t n_q_heads;      /* H_q, a multiple of H_kv; the GQA group is H_q / H_kv       */
   int32_t head_dim;       /* must be 256                                                */
   int32_t page_tokens;    /* must be 128                                                */
-  int32_t k_fmt;          /* KVATTN_FMT_Q8_0, or Q4_0 / Q5_1 (then v_fmt must be Q4_0)  */
-  int32_t v_fmt;          /* KVATTN_FMT_Q4_0 or KVATTN_FMT_Q8_0                         */
+  int32_t k_fmt;          /* KVATTN_FMT_Q8_0, Q4_0, Q5_1 (values Q4_0 or Q8_0) or Q5_0  */
+  int32_t v_fmt;          /* KVATTN_FMT_Q4_0 or Q8_0, or Q4_1 (with Q5_0 keys only)     */
   void* k_pool;           /* device memory, 16-byte aligned                              */
   void* v_pool;           /* device memory, 16-byte aligned                              */
   int64_t k_page_stride;  /* bytes between consecutive K pages (>= K page bytes, %16==0) */
@@ -166,6 +178,10 @@ KVATTN_API int kvattn_quantize_append(const kvattn_kv_desc* desc, const float* k
  *   out          device fp32 [n_q][H_q][256]: softmax(q.k/16) v
  *   lse          device fp32 [n_q][H_q]: natural-log log-sum-exp of the scaled scores
  *                (-inf and out = 0 for a row that sees no key)
+ * Key and value codes enter the tensor-core MMAs exactly; block scales are applied in fp32
+ * (keys) or folded into P as an exact f16 product plus a remainder (values), and the query
+ * and P are split into f16 high and low parts, so the result matches exact attention over
+ * the dequantized cache to about 2^-20 relative.
  *   ws, ws_bytes device workspace of at least kvattn_decode_workspace_size() bytes (256-byte
  *                aligned; may be NULL when that size is 0).  The keys of each KV head are
  *                split across CTAs; per-split (o, lse) partials go to the workspace and a
@@ -181,6 +197,19 @@ KVATTN_API int kvattn_decode(const kvattn_kv_desc* desc, const float* q, int n_q
                              const int32_t* n_pages, int max_pages, float* out, float* lse,
                              void* ws, size_t ws_bytes, kvattn_stream_t stream);
 
+/* The two grids of kvattn_decode, as separate calls (same arguments; kvattn_decode is
+ * kvattn_decode_splits followed by kvattn_decode_merge_splits on the same stream and
+ * workspace).  kvattn_decode_splits runs the split grid: per-split (o, lse) partials into ws,
+ * or out / lse directly when the plan has one split.  kvattn_decode_merge_splits merges them
+ * into out / lse (nothing to do for one split); it reads only the workspace, so other work may
+ * run on the stream in between, as long as the workspace is not reused. */
+KVATTN_API int kvattn_decode_splits(const kvattn_kv_desc* desc, const float* q, int n_q, const int32_t* q_pos,
+                                    const int32_t* page_list, const int32_t* page_logical,
+                                    const int32_t* n_pages, int max_pages, float* out, float* lse,
+                                    void* ws, size_t ws_bytes, kvattn_stream_t stream);
+KVATTN_API int kvattn_decode_merge_splits(const kvattn_kv_desc* desc, int n_q, int max_pages, float* out,
+                                          float* lse, void* ws, size_t ws_bytes, kvattn_stream_t stream);
+
 /* Same computation and arguments as kvattn_decode, for callers that cannot allocate device
  * memory (for example code hosted by a framework whose memory pool owns the device memory
  * and forbids cudaMalloc, or loops that must never enter the allocator).  It has no
@@ -190,7 +219,10 @@ KVATTN_API int kvattn_decode(const kvattn_kv_desc* desc, const float* q, int n_q
  * address (with that device current) and should come before any stream capture.  All calls
  * on a device share that device's array, which keeps the last call's contents: calls on one
  * device whose GPU work overlaps (for example on two streams) race, so order them on one
- * stream.  Calls no allocating routine. */
+ * stream.  Calls no allocating routine.  Shapes kvattn_decode refuses return the same status
+ * here (UNSUPPORTED_SHAPE for group * n_q > 24).  The looked-up address does not survive a
+ * device reset (cudaDeviceReset): the library is then unusable on that device in this
+ * process, as for every other entry point. */
 KVATTN_API int kvattn_decode_noalloc(const kvattn_kv_desc* desc, const float* q, int n_q, const int32_t* q_pos,
                                      const int32_t* page_list, const int32_t* page_logical,
                                      const int32_t* n_pages, int max_pages, float* out, float* lse,
@@ -235,13 +267,16 @@ KVATTN_API int kvattn_select_blocks(const float* summaries, const float* q_group
 
 /* ---- chunked prefill on tcgen05 ([STREAM] method list) -----------------------------
  * Attention of n_q bf16 query tokens (positions q_pos[i], device int32 [n_q]) over the
- * listed pages, causal.  K/V tiles are dequantized to f16 (block scales folded in) in
- * shared memory and Q is rounded to f16 after scaling by log2(e)/16; QK^T and PV run on
- * tcgen05 tensor cores with fp32 accumulation in tensor memory.  The keys are taken in
- * splits of kv_split_tokens (a multiple of 128, at most 65,536; a CTA may walk several
- * consecutive splits); partial results are merged by log-sum-exp.  A page id outside
- * [0, n_pages) skips its page and records KVATTN_ERR_BAD_PAGE.  Needs Q8_0 K / Q4_0 V pages
- * (UNSUPPORTED_FORMAT otherwise).
+ * listed pages, causal.  K/V tiles are dequantized in shared memory into an f16 high part
+ * (code x scale rounded once) and an f16 low part (the exact remainder); Q enters as Q/16 in
+ * f16 (exact) and P as an f16 high part plus the rounded remainder.  QK^T (two MMAs per
+ * k-step) and PV (three) run on tcgen05 tensor cores as CTA-pair MMAs with fp32
+ * accumulation in tensor memory, so every operand carries about 22 significant bits.  The
+ * keys are taken in splits of kv_split_tokens (a multiple of 128, at most 65,536; a CTA may
+ * walk several consecutive splits); partial results are merged by log-sum-exp.  A page id
+ * outside [0, n_pages) skips its page and records KVATTN_ERR_BAD_PAGE.  Needs Q8_0 or Q4_0
+ * K with Q4_0 V pages (UNSUPPORTED_FORMAT otherwise; [GUIDE] build step: the q8_0-q4_0 and
+ * q4_0-q4_0 pairs).
  *   q      device bf16 bits [n_q][H_q][256];  out device fp32 [n_q][H_q][256];
  *   lse    device fp32 [n_q][H_q];  page arguments as for kvattn_decode.
  *   ws     device workspace of kvattn_prefill_workspace_size() bytes. */

@@ -1,6 +1,8 @@
 // C ABI of libkvattn: argument validation, split planning and kernel launches.
 // No entry point allocates memory; every GPU action is stream-ordered on the caller's stream
 // except kvattn_init and kvattn_device_error, which synchronise.
+#include <nvtx3/nvToolsExt.h>
+
 #include <chrono>
 #include <thread>
 
@@ -24,6 +26,39 @@ cudaError_t launch_select(const float*, const float*, int, int, int, int, int, i
                           int32_t*, int32_t*, int, double*, cudaStream_t);
 cudaError_t launch_page_copy(const void*, int64_t, int64_t, void*, int64_t, int64_t, int64_t, const int32_t*,
                              const int32_t*, int, int, int, cudaStream_t);
+
+}  // namespace kvattn
+
+namespace kvattn {
+
+// An NVTX range named after the entry point around each call that launches GPU work, so a
+// profiler timeline shows which library call every kernel belongs to (header-only NVTX 3: the
+// push / pop cost a pointer check when no tool is attached).
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
+
+int key_format_id(int k_fmt) {
+  switch (k_fmt) {
+    case KVATTN_FMT_Q8_0: return kKeyQ8;
+    case KVATTN_FMT_Q4_0: return kKeyQ4;
+    case KVATTN_FMT_Q5_1: return kKeyQ51;
+    case KVATTN_FMT_Q5_0: return kKeyQ50;
+    default: return -1;
+  }
+}
+
+int value_format_id(int v_fmt) {
+  switch (v_fmt) {
+    case KVATTN_FMT_Q4_0: return kValQ4;
+    case KVATTN_FMT_Q8_0: return kValQ8;
+    case KVATTN_FMT_Q4_1: return kValQ41;
+    default: return -1;
+  }
+}
 
 }  // namespace kvattn
 
@@ -65,8 +100,10 @@ int64_t page_bytes_of(int role, int fmt) {
   if (role == KVATTN_ROLE_K && fmt == KVATTN_FMT_Q8_0) return kKPageBytes;
   if (role == KVATTN_ROLE_K && fmt == KVATTN_FMT_Q4_0) return kK4PageBytes;
   if (role == KVATTN_ROLE_K && fmt == KVATTN_FMT_Q5_1) return kK5PageBytes;
+  if (role == KVATTN_ROLE_K && fmt == KVATTN_FMT_Q5_0) return kK50PageBytes;
   if (role == KVATTN_ROLE_V && fmt == KVATTN_FMT_Q4_0) return kV4PageBytes;
   if (role == KVATTN_ROLE_V && fmt == KVATTN_FMT_Q8_0) return kV8PageBytes;
+  if (role == KVATTN_ROLE_V && fmt == KVATTN_FMT_Q4_1) return kV41PageBytes;
   return 0;
 }
 
@@ -77,8 +114,7 @@ int validate_desc(const kvattn_kv_desc* d) {
   if (d->head_dim != kHeadDim || d->page_tokens != kPageTokens) return KVATTN_ERR_UNSUPPORTED_FORMAT;
   const int64_t kb = page_bytes_of(KVATTN_ROLE_K, d->k_fmt), vb = page_bytes_of(KVATTN_ROLE_V, d->v_fmt);
   if (!kb || !vb) return KVATTN_ERR_UNSUPPORTED_FORMAT;
-  // Q4_0 and Q5_1 keys come with Q4_0 values only
-  if (d->k_fmt != KVATTN_FMT_Q8_0 && d->v_fmt != KVATTN_FMT_Q4_0) return KVATTN_ERR_UNSUPPORTED_FORMAT;
+  if (!decode_pair_supported(key_format_id(d->k_fmt), value_format_id(d->v_fmt))) return KVATTN_ERR_UNSUPPORTED_FORMAT;
   if (!d->k_pool || !d->v_pool || !aligned16(d->k_pool) || !aligned16(d->v_pool)) return KVATTN_ERR_INVALID_ARG;
   if (d->k_page_stride < kb || d->v_page_stride < vb || (d->k_page_stride & 15) || (d->v_page_stride & 15))
     return KVATTN_ERR_INVALID_ARG;
@@ -165,6 +201,7 @@ KVATTN_API int kvattn_device_error(kvattn_stream_t stream) {
 KVATTN_API int kvattn_quantize_append(const kvattn_kv_desc* desc, const float* k, const float* v, int n_tok,
                                       int32_t pos0, const int32_t* page_table, int n_blocks,
                                       kvattn_stream_t stream) {
+  const CallRange range_("kvattn_quantize_append");
   int st = validate_desc(desc);
   if (st) return st;
   if (n_tok < 0 || pos0 < 0 || n_blocks < 0) return KVATTN_ERR_INVALID_ARG;
@@ -183,10 +220,14 @@ KVATTN_API size_t kvattn_decode_workspace_size(const kvattn_kv_desc* desc, int n
   return plan_decode(desc, n_q, max_pages).bytes;
 }
 
-KVATTN_API int kvattn_decode(const kvattn_kv_desc* desc, const float* q, int n_q, const int32_t* q_pos,
-                             const int32_t* page_list, const int32_t* page_logical, const int32_t* n_pages,
-                             int max_pages, float* out, float* lse, void* ws, size_t ws_bytes,
-                             kvattn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Validates the arguments of a decode and fills its parameters (the split plan included).
+int decode_setup(const kvattn_kv_desc* desc, const float* q, int n_q, const int32_t* q_pos, const int32_t* page_list,
+                 const int32_t* page_logical, const int32_t* n_pages, int max_pages, float* out, float* lse, void* ws,
+                 size_t ws_bytes, DecodeParams* prm) {
   int st = validate_desc(desc);
   if (st) return st;
   if (n_q < 1 || max_pages < 0 || !q || !q_pos || !out || !lse || (max_pages > 0 && !page_list))
@@ -201,35 +242,80 @@ KVATTN_API int kvattn_decode(const kvattn_kv_desc* desc, const float* q, int n_q
   }
   int dev;
   if ((st = current_device_checked(&dev))) return st;
-  DecodeParams prm{};
-  prm.k_pool = static_cast<const uint8_t*>(desc->k_pool);
-  prm.v_pool = static_cast<const uint8_t*>(desc->v_pool);
-  prm.k_stride = desc->k_page_stride;
-  prm.v_stride = desc->v_page_stride;
-  prm.n_pages = desc->n_pages;
-  prm.q = q;
-  prm.q_pos = q_pos;
-  prm.page_list = page_list;
-  prm.page_logical = page_logical;
-  prm.n_pages_arr = n_pages;
-  prm.out = out;
-  prm.lse = lse;
+  *prm = DecodeParams{};
+  prm->k_pool = static_cast<const uint8_t*>(desc->k_pool);
+  prm->v_pool = static_cast<const uint8_t*>(desc->v_pool);
+  prm->k_stride = desc->k_page_stride;
+  prm->v_stride = desc->v_page_stride;
+  prm->n_pages = desc->n_pages;
+  prm->q = q;
+  prm->q_pos = q_pos;
+  prm->page_list = page_list;
+  prm->page_logical = page_logical;
+  prm->n_pages_arr = n_pages;
+  prm->out = out;
+  prm->lse = lse;
   uint8_t* w = static_cast<uint8_t*>(ws);
-  prm.part_lse = plan.bytes ? reinterpret_cast<float*>(w + plan.lse_off) : nullptr;
-  prm.part_o = plan.bytes ? reinterpret_cast<float*>(w + plan.o_off) : nullptr;
-  prm.n_q = n_q;
-  prm.group = group;
-  prm.n_qh = desc->n_q_heads;
-  prm.max_pages = max_pages;
-  prm.n_splits = plan.n_splits;
-  const int kf = desc->k_fmt == KVATTN_FMT_Q4_0 ? kKeyQ4 : desc->k_fmt == KVATTN_FMT_Q5_1 ? kKeyQ51 : kKeyQ8;
-  cudaError_t e = launch_decode(prm, desc->n_kv_heads, kf, desc->v_fmt == KVATTN_FMT_Q8_0,
+  prm->part_lse = plan.bytes ? reinterpret_cast<float*>(w + plan.lse_off) : nullptr;
+  prm->part_o = plan.bytes ? reinterpret_cast<float*>(w + plan.o_off) : nullptr;
+  prm->n_q = n_q;
+  prm->group = group;
+  prm->n_qh = desc->n_q_heads;
+  prm->max_pages = max_pages;
+  prm->n_splits = plan.n_splits;
+  return KVATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+KVATTN_API int kvattn_decode(const kvattn_kv_desc* desc, const float* q, int n_q, const int32_t* q_pos,
+                             const int32_t* page_list, const int32_t* page_logical, const int32_t* n_pages,
+                             int max_pages, float* out, float* lse, void* ws, size_t ws_bytes,
+                             kvattn_stream_t stream) {
+  const CallRange range_("kvattn_decode");
+  DecodeParams prm;
+  const int st =
+      decode_setup(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pages, out, lse, ws, ws_bytes, &prm);
+  if (st) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_decode(prm, desc->n_kv_heads, key_format_id(desc->k_fmt), value_format_id(desc->v_fmt), s);
+  if (e == cudaSuccess) e = launch_decode_merge(prm, desc->n_kv_heads, s);
+  return e == cudaSuccess ? KVATTN_OK : cuda_fail(e);
+}
+
+KVATTN_API int kvattn_decode_splits(const kvattn_kv_desc* desc, const float* q, int n_q, const int32_t* q_pos,
+                                    const int32_t* page_list, const int32_t* page_logical, const int32_t* n_pages,
+                                    int max_pages, float* out, float* lse, void* ws, size_t ws_bytes,
+                                    kvattn_stream_t stream) {
+  const CallRange range_("kvattn_decode_splits");
+  DecodeParams prm;
+  const int st =
+      decode_setup(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pages, out, lse, ws, ws_bytes, &prm);
+  if (st) return st;
+  cudaError_t e = launch_decode(prm, desc->n_kv_heads, key_format_id(desc->k_fmt), value_format_id(desc->v_fmt),
                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVATTN_OK : cuda_fail(e);
+}
+
+KVATTN_API int kvattn_decode_merge_splits(const kvattn_kv_desc* desc, int n_q, int max_pages, float* out, float* lse,
+                                          void* ws, size_t ws_bytes, kvattn_stream_t stream) {
+  const CallRange range_("kvattn_decode_merge_splits");
+  // the same validation as the split grid's call; q, q_pos and the page list are not read
+  static const float kDummy[4] __attribute__((aligned(16))) = {0.f, 0.f, 0.f, 0.f};
+  static const int32_t kDummyI[1] = {0};
+  DecodeParams prm;
+  const int st = decode_setup(desc, kDummy, n_q, kDummyI, kDummyI, nullptr, nullptr, max_pages, out, lse, ws,
+                              ws_bytes, &prm);
+  if (st) return st;
+  cudaError_t e = launch_decode_merge(prm, desc->n_kv_heads, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVATTN_OK : cuda_fail(e);
 }
 
 KVATTN_API int kvattn_merge_lse(const float* o_parts, const float* lse_parts, int n_parts, int rows, int dim,
                                 float* out, float* lse, kvattn_stream_t stream) {
+  const CallRange range_("kvattn_merge_lse");
   if (n_parts < 0 || rows < 0 || dim < 4 || (dim & 3)) return KVATTN_ERR_INVALID_ARG;
   if (rows == 0) return KVATTN_OK;
   if (!out || !lse || (n_parts > 0 && (!o_parts || !lse_parts))) return KVATTN_ERR_INVALID_ARG;
@@ -244,6 +330,7 @@ KVATTN_API int kvattn_merge_lse(const float* o_parts, const float* lse_parts, in
 KVATTN_API int kvattn_block_summaries(const kvattn_kv_desc* desc, const int32_t* page_table, int n_units,
                                       int n_blocks, int block_begin, int block_end, float* summaries,
                                       kvattn_stream_t stream) {
+  const CallRange range_("kvattn_block_summaries");
   int st = validate_desc(desc);
   if (st) return st;
   if (n_units < 0 || n_blocks < 0 || block_begin < 0 || block_end < block_begin || block_end > n_blocks)
@@ -266,6 +353,7 @@ KVATTN_API int kvattn_select_blocks(const float* summaries, const float* q_group
                                     int n_blocks, int n_full, int n_total, int budget, int recent,
                                     const int32_t* page_table, int32_t* sel_logical, int32_t* sel_phys,
                                     int32_t* n_sel, int cap, void* ws, size_t ws_bytes, kvattn_stream_t stream) {
+  const CallRange range_("kvattn_select_blocks");
   if (n_units < 0 || group < 1 || n_blocks < 0 || n_full < 0 || n_total < n_full || n_total > n_blocks ||
       budget < 0 || recent < 0 || cap < 0)
     return KVATTN_ERR_INVALID_ARG;
@@ -309,6 +397,7 @@ KVATTN_API int kvattn_stream_plan(const int32_t* host_ids, const int32_t* dev_sl
 KVATTN_API int kvattn_stream_pages(const void* host_pool, int64_t host_stride, void* dev_pool, int64_t dev_stride,
                                    int64_t page_bytes, const int32_t* host_ids, const int32_t* dev_slots, int n,
                                    kvattn_stream_t copy_stream, kvattn_event_t done, int* n_copies) {
+  const CallRange range_("kvattn_stream_pages");
   if (n < 0 || page_bytes <= 0 || host_stride < page_bytes || dev_stride < page_bytes) return KVATTN_ERR_INVALID_ARG;
   if (n > 0 && (!host_pool || !dev_pool || !host_ids || !dev_slots)) return KVATTN_ERR_INVALID_ARG;
   for (int i = 0; i < n; ++i)
@@ -391,6 +480,7 @@ extern "C" {
 KVATTN_API int kvattn_gather_pages(const void* host_pool, int64_t host_stride, int64_t n_host_pages, void* dev_pool,
                                    int64_t dev_stride, int64_t n_slots, int64_t page_bytes, const int32_t* host_ids,
                                    const int32_t* dev_slots, int n, int n_ctas, kvattn_stream_t stream) {
+  const CallRange range_("kvattn_gather_pages");
   return page_copy_common(host_pool, host_stride, n_host_pages, dev_pool, dev_stride, n_slots, page_bytes, host_ids,
                           dev_slots, n, n_ctas, 1, stream);
 }
@@ -398,11 +488,13 @@ KVATTN_API int kvattn_gather_pages(const void* host_pool, int64_t host_stride, i
 KVATTN_API int kvattn_scatter_pages(void* host_pool, int64_t host_stride, int64_t n_host_pages, const void* dev_pool,
                                     int64_t dev_stride, int64_t n_slots, int64_t page_bytes, const int32_t* host_ids,
                                     const int32_t* dev_slots, int n, int n_ctas, kvattn_stream_t stream) {
+  const CallRange range_("kvattn_scatter_pages");
   return page_copy_common(host_pool, host_stride, n_host_pages, const_cast<void*>(dev_pool), dev_stride, n_slots,
                           page_bytes, host_ids, dev_slots, n, n_ctas, 0, stream);
 }
 
 KVATTN_API int kvattn_hadamard(const float* in, float* out, int64_t rows, kvattn_stream_t stream) {
+  const CallRange range_("kvattn_hadamard");
   if (rows < 0 || (rows > 0 && (!in || !out)) || rows > (1ll << 40)) return KVATTN_ERR_INVALID_ARG;
   if (rows > 0 && (!aligned16(in) || !aligned16(out))) return KVATTN_ERR_INVALID_ARG;
   int dev;
@@ -417,6 +509,7 @@ KVATTN_API int kvattn_resident_update(const int32_t* sel_logical, const int32_t*
                                       int n_slots, const int32_t* host_page_of_block, int64_t first_page,
                                       const int32_t* extra_page, int32_t* page_list, int32_t* copy_host,
                                       int32_t* copy_dst, int32_t* n_copies, kvattn_stream_t stream) {
+  const CallRange range_("kvattn_resident_update");
   if (!sel_logical || !n_sel || !slot_of_block || !block_of_slot || !host_page_of_block || !extra_page ||
       !page_list || !copy_host || !copy_dst || !n_copies)
     return KVATTN_ERR_INVALID_ARG;
@@ -465,9 +558,11 @@ KVATTN_API int kvattn_prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* 
                                     const int32_t* page_list, const int32_t* page_logical, const int32_t* n_pages,
                                     int max_pages, int kv_split_tokens, float* out, float* lse, void* ws,
                                     size_t ws_bytes, kvattn_stream_t stream) {
+  const CallRange range_("kvattn_prefill_chunk");
   int st = validate_desc(desc);
   if (st) return st;
-  if (desc->k_fmt != KVATTN_FMT_Q8_0 || desc->v_fmt != KVATTN_FMT_Q4_0) return KVATTN_ERR_UNSUPPORTED_FORMAT;
+  if ((desc->k_fmt != KVATTN_FMT_Q8_0 && desc->k_fmt != KVATTN_FMT_Q4_0) || desc->v_fmt != KVATTN_FMT_Q4_0)
+    return KVATTN_ERR_UNSUPPORTED_FORMAT;
   if (n_q < 1 || max_pages < 0 || !q || !q_pos || !out || !lse || (max_pages > 0 && !page_list))
     return KVATTN_ERR_INVALID_ARG;
   if (kv_split_tokens < kPageTokens || kv_split_tokens % kPageTokens || kv_split_tokens > 65536)
@@ -508,7 +603,7 @@ KVATTN_API int kvattn_prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* 
   prm.pages_per_split = plan.pps;
   prm.n_ks = plan.n_ks;
   prm.rows_pad = plan.rows_pad;
-  cudaError_t e = launch_prefill(prm, desc->n_kv_heads, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_prefill(prm, desc->n_kv_heads, key_format_id(desc->k_fmt), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVATTN_OK : cuda_fail(e);
 }
 

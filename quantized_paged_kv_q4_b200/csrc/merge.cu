@@ -81,9 +81,9 @@ namespace kvattn {
 // speculative-decoding report (pitfalls section, attention-rotation item), which spreads outlier channels
 // before quantization.  One warp per row; lane l holds elements 8l .. 8l + 7: the three low
 // index bits are butterflied in registers, the five high ones across lanes by shuffles.
-// `in` may equal `out`.
-__global__ void __launch_bounds__(256) hadamard_kernel(const float* __restrict__ in, float* __restrict__ out,
-                                                       long long rows) {
+// `in` may equal `out` (each warp reads its whole row before writing it), so neither pointer
+// is declared restrict.
+__global__ void __launch_bounds__(256) hadamard_kernel(const float* in, float* out, long long rows) {
   const int lane = threadIdx.x & 31;
   const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;

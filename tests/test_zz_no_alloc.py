@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers_kv import ATOL, GpuCache
+from helpers_kv import GpuCache
 from synth import normal_f32, np_rng, page_permutation
 
 pytestmark = pytest.mark.gpu
@@ -37,5 +37,22 @@ def test_noalloc_decode_matches_decode(kv_gpu, n_q):
         lse = torch.full((n_q, 6 * H), float("nan"), device="cuda")
         kv_gpu.kvattn_decode_noalloc(cache.desc, q, n_q, q_pos, cache.page_table, None, None, nb, out, lse)
         torch.cuda.synchronize()
-        assert np.abs(out.cpu().numpy() - ref_o.cpu().numpy()).max() <= ATOL, call
-        assert np.abs(lse.cpu().numpy() - ref_l.cpu().numpy()).max() <= ATOL, call
+        # the same kernels with the same split plan: bit-identical results
+        assert np.array_equal(out.cpu().numpy(), ref_o.cpu().numpy()), call
+        assert np.array_equal(lse.cpu().numpy(), ref_l.cpu().numpy()), call
+
+
+def test_noalloc_refuses_unsupported_shape_untouched(kv_gpu):
+    """GQA 6 with 5 query tokens (30 rows per KV head) is refused as an unsupported shape, as
+    kvattn_decode refuses it, and the outputs are left untouched."""
+    H, T, n_q = 1, 300, 5
+    rng, cache, nb = _cache(9200, H, T)
+    q = torch.from_numpy(normal_f32(rng, (n_q, 6 * H, 256))).cuda()
+    q_pos = torch.arange(T - n_q, T, dtype=torch.int32, device="cuda")
+    out = torch.full((n_q, 6 * H, 256), 7.0, device="cuda")
+    lse = torch.full((n_q, 6 * H), 7.0, device="cuda")
+    with pytest.raises(kv_gpu.KVAttnError) as e:
+        kv_gpu.kvattn_decode_noalloc(cache.desc, q, n_q, q_pos, cache.page_table, None, None, nb, out, lse)
+    assert e.value.status == kv_gpu.ERR_UNSUPPORTED_SHAPE
+    torch.cuda.synchronize()
+    assert bool((out == 7.0).all()) and bool((lse == 7.0).all())
