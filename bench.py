@@ -33,13 +33,13 @@ if ROOT not in sys.path:
 from synth import WORKLOADS, derived_seed, np_rng, page_permutation, torch_normal, workload_layer_kv  # noqa: E402
 
 METRIC = "quantized paged KV attention: decode HBM GB/s & prefill TFLOP/s vs roofline"
-PAGE_BYTES = {("k", "q8_0"): 34816, ("k", "q4_0"): 18432, ("k", "q5_1"): 24576, ("v", "q4_0"): 18432,
-              ("v", "q8_0"): 34816}
+PAGE_BYTES = {("k", "q8_0"): 34816, ("k", "q4_0"): 18432, ("k", "q5_1"): 24576, ("k", "q5_0"): 22528,
+              ("v", "q4_0"): 18432, ("v", "q8_0"): 34816, ("v", "q4_1"): 20480}
 
 
 def bytes_per_token_head(k_fmt: str, v_fmt: str) -> int:
     """K + V bytes of one token of one KV head: 416 (Q8_0/Q4_0), 544 (Q8_0/Q8_0), 288 (Q4_0/Q4_0),
-    336 (Q5_1/Q4_0)."""
+    416 (Q4_0/Q8_0), 336 (Q5_1/Q4_0), 464 (Q5_1/Q8_0), 336 (Q5_0/Q4_1)."""
     return (PAGE_BYTES[("k", k_fmt)] + PAGE_BYTES[("v", v_fmt)]) // 128
 
 
@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="only the headline workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extra-steps", type=int, default=100)
+    ap.add_argument("--stream-steps", type=int, default=0,
+                    help="decode steps of the host-streamed generation to time (0 = the workload's 512)")
     ap.add_argument("--prefill-layers", type=int, default=0, help="layers of the prefill workload (0 = 16)")
     ap.add_argument("--profile", choices=["none", "decode", "prefill", "verify", "stream"], default="none",
                     help="profiling only: run just this workload's steps (no JSON bench line)")
@@ -124,7 +126,7 @@ class ClockSampler:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                          "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
                                          stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -295,14 +297,20 @@ class DecodeBench(GraphStep):
         self.launches_per_step = 3 * L  # quantize-append, decode, split merge
 
     def layer(self, l, timed=None):
+        """One layer: quantize-append the new token, then kvattn_decode.  With `timed` (three
+        events) the decode runs as its two grids with an event before, between and after them."""
         kv, c = self.kv, self.cache
         kv.kvattn_quantize_append(c.desc, self.k_new[l], self.v_new[l], 1, self.pos, c.page_table[l], self.nb)
-        if timed is not None:
-            timed[0].record()
-        kv.kvattn_decode(c.desc, self.q[l], 1, self.q_pos, c.page_table[l], None, None, self.nb, self.out[l],
-                         self.lse[l], self.ws[l], self.ws_bytes)
-        if timed is not None:
-            timed[1].record()
+        if timed is None:
+            kv.kvattn_decode(c.desc, self.q[l], 1, self.q_pos, c.page_table[l], None, None, self.nb, self.out[l],
+                             self.lse[l], self.ws[l], self.ws_bytes)
+            return
+        timed[0].record()
+        kv.kvattn_decode_splits(c.desc, self.q[l], 1, self.q_pos, c.page_table[l], None, None, self.nb, self.out[l],
+                                self.lse[l], self.ws[l], self.ws_bytes)
+        timed[1].record()
+        kv.kvattn_decode_merge_splits(c.desc, 1, self.nb, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
+        timed[2].record()
 
 
 class VerifyBench(GraphStep):
@@ -355,12 +363,16 @@ class VerifyBench(GraphStep):
                                 self.nb, self.n_full, self.nb, w.budget_blocks, w.recent_blocks, c.page_table[l],
                                 self.sel_l[l], self.sel_p[l], self.n_sel[l], self.cap, self.sws, self.sws_bytes)
         kv.kvattn_quantize_append(c.desc, self.k_new[l], self.v_new[l], w.n_q, self.pos0, c.page_table[l], self.nb)
-        if timed is not None:
-            timed[0].record()
-        kv.kvattn_decode(c.desc, self.q[l], w.n_q, self.q_pos, self.sel_p[l], self.sel_l[l], self.n_sel[l], self.cap,
-                         self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
-        if timed is not None:
-            timed[1].record()
+        if timed is None:
+            kv.kvattn_decode(c.desc, self.q[l], w.n_q, self.q_pos, self.sel_p[l], self.sel_l[l], self.n_sel[l],
+                             self.cap, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
+            return
+        timed[0].record()
+        kv.kvattn_decode_splits(c.desc, self.q[l], w.n_q, self.q_pos, self.sel_p[l], self.sel_l[l], self.n_sel[l],
+                                self.cap, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
+        timed[1].record()
+        kv.kvattn_decode_merge_splits(c.desc, w.n_q, self.cap, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
+        timed[2].record()
 
 
 class PrefillBench:
@@ -394,6 +406,9 @@ class PrefillBench:
         self.ws = torch.zeros(max(self.ws_bytes, 256), dtype=torch.uint8, device=device)
         g = w.group
         self.flops_per_layer = 4.0 * Hq * 256 * (w.n_q * w.context + w.n_q * (w.n_q + 1) / 2)
+        # tensor-core work per algorithmic flop: QK^T as two MMAs (K^ high and low parts) and PV
+        # as three (P_hi V^_hi, P_lo V^_hi, P_hi V^_lo)
+        self.mma_work_factor = (2 + 3) / 2
         self.flops_per_step = self.flops_per_layer * L
         self.launches_per_step = L * (1 + 2 * (w.n_q // w.ubatch))
 
@@ -417,15 +432,17 @@ class PrefillBench:
 
 class StreamBench:
     """Host-streamed decode: the full 524,288-token cache of 16 layers x 4 KV heads sits in
-    pinned host RAM (K|V interleaved per page); per layer the retrieval query selects 256
-    blocks per KV head, a copy kernel brings those pages into device slots on a side stream
-    (layer L+1 while layer L decodes; the tail page stays resident), the new token is
-    quantize-appended into the tail page and written back to host RAM, and decode attends over
-    the 256 + 1 pages."""
+    pinned host RAM (K|V interleaved per page).  A generation is `steps` decode steps (512)
+    whose position advances by one each step.  Per step and layer the step's retrieval query
+    selects 256 blocks per KV head among the prompt's full blocks, a copy kernel brings those
+    pages into device slots on a side stream (layer L+1 while layer L decodes), the step's new
+    token is quantize-appended into the generated-token pages (resident on the device: the
+    generation reserve) and that page is written back to host RAM, and decode attends over the
+    256 selected pages plus the generated-token pages so far."""
 
     PAGE = 34816 + 18432
 
-    def __init__(self, kv, device, layers=0, context=0):
+    def __init__(self, kv, device, layers=0, context=0, steps=0):
         import dataclasses
 
         import torch
@@ -435,12 +452,15 @@ class StreamBench:
             w = dataclasses.replace(w, layers=layers)
         if context:
             w = dataclasses.replace(w, context=context)
+        if steps:
+            w = dataclasses.replace(w, steps=steps)
         self.kv, self.w, self.device = kv, w, device
         L, H, Hq, g = w.layers, w.kv_heads, w.q_heads, w.group
         self.n_full = w.context // 128
-        self.nb = self.n_full + 1
+        self.n_tail = (w.context % 128 + w.steps + 127) // 128     # pages the generated tokens fill
+        self.nb = self.n_full + self.n_tail
         self.budget = w.budget_blocks
-        self.cap = self.budget + 1
+        self.cap = self.budget + self.n_tail
         P = self.PAGE
         # ---- build: per layer on the device, then into pinned host RAM ----
         self.host = torch.empty((L * H * self.nb, P), dtype=torch.uint8).pin_memory()
@@ -459,16 +479,18 @@ class StreamBench:
         torch.cuda.synchronize()
         # host page ids per (layer, head, block)
         self.host_table = torch.arange(L * H * self.nb, dtype=torch.int32, device=device).view(L, H, self.nb)
-        # ---- device slots: 2 buffers x H x budget streamed pages + L x H resident tail pages ----
+        # ---- device slots: 2 buffers x H x budget streamed pages + L x H x n_tail resident pages
+        # of the generated tokens ----
         self.n_stream_slots = 2 * H * self.budget
-        self.n_slots = self.n_stream_slots + L * H
+        self.n_slots = self.n_stream_slots + L * H * self.n_tail
         self.slots = torch.zeros((self.n_slots, P), dtype=torch.uint8, device=device)
-        for l in range(L):
-            for h in range(H):
-                self.slots[self.n_stream_slots + l * H + h].copy_(self.host[(l * H + h) * self.nb + self.n_full])
+        self.tail_slots = torch.tensor([[[self.n_stream_slots + (l * H + h) * self.n_tail + k for k in range(self.n_tail)]
+                                         for h in range(H)] for l in range(L)], dtype=torch.int32, device=device)
+        self.tail_hosts = self.host_table[:, :, self.n_full:].contiguous()
+        self.reset()
         self.desc = kv.make_desc(H, Hq, self.slots, self.slots.data_ptr() + 34816, self.n_slots, k_page_stride=P,
                                  v_page_stride=P)
-        # per buffer: gather destinations (-1 for the tail entry) and the decode page lists
+        # per buffer: gather destinations (-1 for the generated-token entries) and the decode page lists
         self.dst = []
         self.plist = []
         for b in range(2):
@@ -479,17 +501,11 @@ class StreamBench:
             b = l % 2
             base = b * H * self.budget
             self.plist.append(torch.tensor([[base + h * self.budget + i if i < self.budget
-                                             else self.n_stream_slots + l * H + h for i in range(self.cap)]
+                                             else int(self.tail_slots[l, h, i - self.budget]) for i in range(self.cap)]
                                             for h in range(H)], dtype=torch.int32, device=device))
-        # tail page table for the append: logical block n_full -> the layer's tail slot
-        self.tail_tab = torch.full((L, H, self.nb), 0, dtype=torch.int32, device=device)
-        for l in range(L):
-            for h in range(H):
-                self.tail_tab[l, h, :] = self.n_stream_slots + l * H + h
-        self.tail_host = torch.tensor([[(l * H + h) * self.nb + self.n_full for h in range(H)] for l in range(L)],
-                                      dtype=torch.int32, device=device)
-        self.tail_slot = torch.tensor([[self.n_stream_slots + l * H + h for h in range(H)] for l in range(L)],
-                                      dtype=torch.int32, device=device)
+        # append page table: logical block n_full + k -> generated-token slot k of the unit
+        self.tail_tab = torch.zeros((L, H, self.nb), dtype=torch.int32, device=device)
+        self.tail_tab[:, :, self.n_full:] = self.tail_slots
         # selection outputs and workspaces
         self.sel_l = torch.zeros((L, H, self.cap), dtype=torch.int32, device=device)
         self.sel_p = torch.zeros((L, H, self.cap), dtype=torch.int32, device=device)
@@ -498,13 +514,17 @@ class StreamBench:
         self.sws = torch.zeros((L, self.sws_bytes), dtype=torch.uint8, device=device)
         self.ws_bytes = kv.kvattn_decode_workspace_size(self.desc, 1, self.cap)
         self.ws = torch.zeros((L, max(self.ws_bytes, 256)), dtype=torch.uint8, device=device)
-        # per-step inputs
-        self.q = torch_normal(derived_seed(w.seed, 20), (L, 1, Hq, 256), device)
-        self.q_group = self.q[:, 0].reshape(L, H, g, 256).contiguous()
-        self.k_new = torch_normal(derived_seed(w.seed, 21), (L, 1, H, 256), device)
-        self.v_new = torch_normal(derived_seed(w.seed, 22), (L, 1, H, 256), device)
+        # per-step inputs of the whole generation: query, new K and V of every step and layer
+        S = w.steps
+        self.q_all = torch_normal(derived_seed(w.seed, 20), (S, L, 1, Hq, 256), device)
+        self.qg_all = self.q_all[:, :, 0].reshape(S, L, H, g, 256).contiguous()
+        self.k_all = torch_normal(derived_seed(w.seed, 21), (S, L, 1, H, 256), device)
+        self.v_all = torch_normal(derived_seed(w.seed, 22), (S, L, 1, H, 256), device)
+        self.pos_all = torch.arange(w.context, w.context + S, dtype=torch.int32, device=device)
+        # step 0's views, kept for the fixed-position subclass
+        self.q, self.q_group, self.k_new, self.v_new = self.q_all[0], self.qg_all[0], self.k_all[0], self.v_all[0]
         self.pos = w.context
-        self.q_pos = torch.tensor([self.pos], dtype=torch.int32, device=device)
+        self.q_pos = self.pos_all[:1]
         self.out = torch.empty((L, 1, Hq, 256), device=device)
         self.lse = torch.empty((L, 1, Hq), device=device)
         self.copy_stream = torch.cuda.Stream(device=device)
@@ -512,17 +532,36 @@ class StreamBench:
         self.ev_copy = [torch.cuda.Event() for _ in range(L)]
         self.ev_dec = [torch.cuda.Event() for _ in range(L)]
         self.copy_bytes_per_step = L * H * self.budget * P
-        tokens = self.budget * 128 + 1
-        self.attn_bytes_per_step = L * H * tokens * bytes_per_token_head("q8_0", "q4_0")
-        self.launches_per_step = 5 * L
+        self.launches_per_step = 6 * L  # scores, top-k, copy, append, decode (+ merge), write-back
         self.gather_ctas = 16
 
-    def _select(self, l):
+    def reset(self):
+        """Back to the first step of the generation: the generated-token pages hold the prompt's
+        partial tail (if any), as in host RAM before the generation."""
+        L, H = self.w.layers, self.w.kv_heads
+        self.gen_t = 0
+        self.slots[self.n_stream_slots:].zero_()
+        if self.w.context % 128:
+            for l in range(L):
+                for h in range(H):
+                    self.slots[int(self.tail_slots[l, h, 0])].copy_(self.host[(l * H + h) * self.nb + self.n_full])
+
+    def attn_bytes(self, t):
+        """Quantized KV bytes the decode launches of step t read (all layers)."""
         w = self.w
-        self.kv.kvattn_select_blocks(self.summ[l * w.kv_heads:(l + 1) * w.kv_heads], self.q_group[l], w.kv_heads,
-                                     w.group, self.nb, self.n_full, self.nb, self.budget, 0, self.host_table[l],
-                                     self.sel_l[l], self.sel_p[l], self.n_sel[l], self.cap, self.sws[l],
-                                     self.sws_bytes)
+        tokens = self.budget * 128 + w.context % 128 + t + 1
+        return w.layers * w.kv_heads * tokens * bytes_per_token_head(w.k_fmt, w.v_fmt)
+
+    def _n_total(self):
+        """Blocks of the unit so far: the prompt's full blocks and the generated-token pages."""
+        return self.n_full + (self.w.context % 128 + self.gen_t) // 128 + 1
+
+    def _select(self, l):
+        w, t = self.w, self.gen_t
+        self.kv.kvattn_select_blocks(self.summ[l * w.kv_heads:(l + 1) * w.kv_heads], self.qg_all[t, l], w.kv_heads,
+                                     w.group, self.nb, self.n_full, self._n_total(), self.budget, 0,
+                                     self.host_table[l], self.sel_l[l], self.sel_p[l], self.n_sel[l], self.cap,
+                                     self.sws[l], self.sws_bytes)
 
     def _gather(self, l, stream):
         H = self.w.kv_heads
@@ -531,18 +570,22 @@ class StreamBench:
                                     stream)
 
     def _attend(self, l, timed=None):
-        kv, w = self.kv, self.w
-        kv.kvattn_quantize_append(self.desc, self.k_new[l], self.v_new[l], 1, self.pos, self.tail_tab[l], self.nb)
+        kv, w, t = self.kv, self.w, self.gen_t
+        pos = w.context + t
+        kv.kvattn_quantize_append(self.desc, self.k_all[t, l], self.v_all[t, l], 1, pos, self.tail_tab[l], self.nb)
         if timed is not None:
             timed[0].record()
-        kv.kvattn_decode(self.desc, self.q[l], 1, self.q_pos, self.plist[l], self.sel_l[l], self.n_sel[l], self.cap,
-                         self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
+        kv.kvattn_decode(self.desc, self.q_all[t, l], 1, self.pos_all[t:t + 1], self.plist[l], self.sel_l[l],
+                         self.n_sel[l], self.cap, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
         if timed is not None:
             timed[1].record()
+        k = (w.context % 128 + t) // 128     # the generated-token page the token went to
         kv.kvattn_scatter_pages(self.host, self.PAGE, self.host.shape[0], self.slots, self.PAGE, self.n_slots,
-                                self.PAGE, self.tail_host[l], self.tail_slot[l], w.kv_heads, 4)
+                                self.PAGE, self.tail_hosts[l, :, k], self.tail_slots[l, :, k], w.kv_heads, 4)
 
     def step(self, stream_pages=True, timed=None):
+        """One decode step of all layers at the current position; the position then advances
+        (after the last step of the generation it stays there)."""
         import torch
 
         L = self.w.layers
@@ -568,6 +611,7 @@ class StreamBench:
                 main.wait_event(self.ev_copy[l])
             self._attend(l, timed[l] if timed is not None else None)
             self.ev_dec[l].record(main)
+        self.gen_t = min(self.gen_t + 1, self.w.steps - 1)
 
     def copies_only(self):
         import torch
@@ -587,7 +631,7 @@ class ResidentStreamBench(StreamBench):
     def __init__(self, kv, device, queries=1, drift=0.0, layers=0, context=0):
         import torch
 
-        super().__init__(kv, device, layers=layers, context=context)
+        super().__init__(kv, device, layers=layers, context=context, steps=1)
         w, L, H = self.w, self.w.layers, self.w.kv_heads
         self.units = L * H
         self.n_res = self.units * self.budget                 # resident pool pages, then the tails
@@ -602,6 +646,7 @@ class ResidentStreamBench(StreamBench):
         self.tail_slot = torch.tensor([[self.n_res + l * H + h for h in range(H)] for l in range(L)],
                                       dtype=torch.int32, device=device)
         self.tail_tab = self.tail_slot[:, :, None].expand(L, H, self.nb).contiguous()
+        self.tail_host = self.tail_hosts[:, :, 0].contiguous()
         self.sob = torch.full((self.units, self.nb), -1, dtype=torch.int32, device=device)
         self.bos = torch.full((self.units, self.budget), -1, dtype=torch.int32, device=device)
         self.plist_r = torch.zeros((L, H, self.cap), dtype=torch.int32, device=device)
@@ -659,12 +704,12 @@ class ResidentStreamBench(StreamBench):
 
 
 def time_stream(b, steps, warmup):
-    """T_stream (pipelined), T_resident (no page copies), T_copy (copies alone), decode time."""
+    """A generation of `steps` advancing decode steps, pipelined (T_stream per step); the same
+    steps without page copies (T_resident), the copies alone (T_copy), and the decode launches
+    of one step.  Warm-up steps run first and the generation then restarts at its first step."""
     import torch
 
-    def timed(fn, n, w_):
-        for _ in range(w_):
-            fn()
+    def timed(fn, n):
         torch.cuda.synchronize()
         e0, e1 = event_pair()
         e0.record()
@@ -674,13 +719,21 @@ def time_stream(b, steps, warmup):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / n
 
-    t_stream = timed(lambda: b.step(True), steps, warmup)
-    t_res = timed(lambda: b.step(False), steps, warmup)
-    t_copy = timed(b.copies_only, steps, warmup)
+    b.reset()
+    for _ in range(warmup):
+        b.step(True)
+    b.reset()
+    t_stream = timed(lambda: b.step(True), steps)
+    short = min(steps, 32)
+    b.reset()
+    t_res = timed(lambda: b.step(False), short)
+    t_copy = timed(b.copies_only, short)
+    b.reset()
     pairs = [event_pair() for _ in range(b.w.layers)]
     b.step(True, timed=pairs)
     torch.cuda.synchronize()
     t_dec = sum(a.elapsed_time(c) for a, c in pairs)
+    b.reset()
     return t_stream, t_res, t_copy, t_dec
 
 
@@ -732,7 +785,24 @@ def time_steps(bench, steps, warmup, world):
 
 
 def time_kernel(bench, steps):
-    """Average device duration of the decode launches (events on the launching stream)."""
+    """Average device duration of the decode split grid and of its merge grid, per layer launch
+    (events on the launching stream before, between and after the two grids)."""
+    import torch
+
+    trip = []
+    for _ in range(steps):
+        for l in range(bench.w.layers):
+            p = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                 torch.cuda.Event(enable_timing=True))
+            bench.layer(l, timed=p)
+            trip.append(p)
+    torch.cuda.synchronize()
+    return (statistics.mean(a.elapsed_time(b) for a, b, _ in trip),
+            statistics.mean(b.elapsed_time(c) for _, b, c in trip))
+
+
+def time_layers(bench, steps):
+    """Average device duration of one layer's prefill calls (events before and after them)."""
     import torch
 
     pairs = []
@@ -860,7 +930,8 @@ def reference_arm(args, world, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": "decode131k", "layers": w.layers, "kv_heads": w.kv_heads, "q_heads": w.q_heads,
                    "context": w.context, "n_q": 1, "k_fmt": w.k_fmt, "v_fmt": w.v_fmt},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": len(os.sched_getaffinity(0)), "blas_threads": threads,
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -912,28 +983,33 @@ def main():
         b.capture()
     except Exception as exc:  # report and time the direct launches instead
         launch_mode = f"direct launches (graph capture failed: {exc!r})"
+    # clocks are sampled over the whole headline section: warm-up, timed steps, the per-grid
+    # timing and the end-to-end steps
     clocks = ClockSampler(local)
     clocks.start()
     ms = time_steps(b, args.steps, args.warmup, world)
-    clk = clocks.stop()
-    kern_ms = time_kernel(b, max(3, min(args.steps, 50)))
+    kern_ms, merge_ms = time_kernel(b, max(3, min(args.steps, 50)))
     e2e_ms, h2d, d2h = time_e2e(b, max(3, min(args.steps, 200)), 3)
+    clk = clocks.stop()
     assert kvattn.kvattn_device_error() == 0
     value = job_throughput(b.bytes_per_step, world, ms) / 1e9
     achieved = b.bytes_per_layer / (kern_ms * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "s8/f16 MMA, f32 accumulate", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f16 MMA (exact hi+lo f16 operands), f32 accumulate", "data": "synthetic",
         "config": {"workload": "decode131k", "layers": b.w.layers, "kv_heads": b.w.kv_heads,
                    "q_heads": b.w.q_heads, "context": b.ctx, "n_q": 1, "k_fmt": "q8_0", "v_fmt": "q4_0",
                    "outliers": "1% of channels x8", "parallelism": f"{world} independent decodes (one per GPU)",
                    "l2": "inputs larger than L2 (218 MB of KV per layer launch, 3.49 GB per step)",
                    "launch": launch_mode},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": profiled_traffic("decode_kernel_decode131k.md"), "kernel": "decode_kernel<1,false,false,0>",
+                     "traffic": profiled_traffic("decode_kernel_decode131k.md"),
+                     "kernel": "decode_kernel<Q8_0 K, Q4_0 V, 8 rows> (the split grid alone)",
                      "peak_kind": f"{peak_kind} copy bandwidth (hbm_gbs)",
-                     "algorithmic_bytes_per_launch": b.bytes_per_layer, "avg_launch_ms": kern_ms},
+                     "algorithmic_bytes_per_launch": b.bytes_per_layer, "avg_launch_ms": kern_ms,
+                     "merge_grid_ms": merge_ms, "step_ms_per_layer": ms / b.w.layers,
+                     "step_frac": value / world / hbm},
         "e2e": {"value": b.bytes_per_step * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": b.launches_per_step * args.steps,
@@ -949,44 +1025,52 @@ def main():
     if not args.no_extra:
         try:
             # the same decode step over the other KV format pairs
-            for wn in ("decode131k_q8q8", "decode131k_q4q4", "decode131k_q51q4"):
+            for wn in ("decode131k_q8q8", "decode131k_q4q4", "decode131k_q4q8", "decode131k_q51q4",
+                       "decode131k_q51q8", "decode131k_q50q41"):
                 b2 = DecodeBench(kvattn, wn, device)
                 b2.capture()
                 ms2 = time_steps(b2, args.extra_steps, 5, world)
-                k2 = time_kernel(b2, 10)
+                k2, m2 = time_kernel(b2, 10)
                 extra[wn] = {"GB/s": b2.bytes_per_step / (ms2 * 1e-3) / 1e9, "ms_per_step": ms2,
                              "kernel_GB/s": b2.bytes_per_layer / (k2 * 1e-3) / 1e9,
                              "kernel_frac_hbm": b2.bytes_per_layer / (k2 * 1e-3) / 1e9 / hbm,
-                             "kernel_ms": k2, "bytes_per_token_head": bytes_per_token_head(b2.w.k_fmt, b2.w.v_fmt)}
+                             "kernel_ms": k2, "merge_ms": m2, "k_fmt": b2.w.k_fmt, "v_fmt": b2.w.v_fmt,
+                             "bytes_per_token_head": bytes_per_token_head(b2.w.k_fmt, b2.w.v_fmt)}
                 del b2
                 torch.cuda.empty_cache()
             b3 = VerifyBench(kvattn, device)
             b3.capture()
             ms3 = time_steps(b3, args.extra_steps, 5, world)
-            k3 = time_kernel(b3, 10)
+            k3, m3 = time_kernel(b3, 10)
             extra["verify262k"] = {"GB/s": b3.bytes_per_step / (ms3 * 1e-3) / 1e9, "ms_per_step": ms3,
                                    "decode_kernel_GB/s": b3.bytes_per_layer / (k3 * 1e-3) / 1e9,
                                    "decode_kernel_frac_hbm": b3.bytes_per_layer / (k3 * 1e-3) / 1e9 / hbm,
+                                   "decode_kernel_ms": k3, "merge_ms": m3,
                                    "selected_tokens_per_unit": (b3.w.budget_blocks + b3.w.recent_blocks) * 128 + 4}
             del b3
             torch.cuda.empty_cache()
             b4 = PrefillBench(kvattn, device, layers=args.prefill_layers)
             ms4 = time_steps(b4, max(1, args.extra_steps // 50), 1, world)
-            k4 = time_kernel(b4, 1)
+            k4 = time_layers(b4, 1)
             tf = b4.flops_per_layer / (k4 * 1e-3) / 1e12
             extra["prefill524k"] = {"TFLOP/s": b4.flops_per_step / (ms4 * 1e-3) / 1e12, "ms_per_step": ms4,
                                     "layers": b4.w.layers, "kernel_TFLOP/s": tf, "kernel_frac_bf16": tf / bf16,
-                                    "flop_per_layer": b4.flops_per_layer,
+                                    "layer_ms": k4, "flop_per_layer": b4.flops_per_layer,
+                                    "executed_TFLOP/s": tf * b4.mma_work_factor,
+                                    "executed_frac_bf16": tf * b4.mma_work_factor / bf16,
+                                    "mma_work_factor": b4.mma_work_factor,
                                     "peak": f"{peak_kind} dense bf16 (f16 operands run at the same rate)"}
             del b4
             torch.cuda.empty_cache()
             b5 = StreamBench(kvattn, device)
-            ts, tr, tcp, td = time_stream(b5, max(3, args.extra_steps // 5), 2)
+            n_gen = args.stream_steps or b5.w.steps
+            ts, tr, tcp, td = time_stream(b5, n_gen, 2)
             tm, tenq, ncp = time_memcpy_route(b5)
             extra["stream524k"] = {
                 "ms_per_step": ts, "ms_per_step_resident": tr, "ms_copies_only": tcp, "ms_decode": td,
                 "pcie_GB/s": b5.copy_bytes_per_step / (tcp * 1e-3) / 1e9,
-                "hbm_GB/s_decode": b5.attn_bytes_per_step / (td * 1e-3) / 1e9,
+                "hbm_GB/s_decode": b5.attn_bytes(0) / (td * 1e-3) / 1e9,
+                "generation_steps_timed": n_gen, "positions": [b5.w.context, b5.w.context + n_gen - 1],
                 "hidden_copy_fraction": max(0.0, 1.0 - (ts - tr) / tcp) if tcp > 0 else None,
                 "copy_bytes_per_step": b5.copy_bytes_per_step,
                 "memcpy_route": {"ms_device": tm, "ms_host_enqueue": tenq, "copies": ncp,
@@ -1014,7 +1098,8 @@ def main():
 
     if rank == 0 and not args.no_cpu_baseline:
         gbs, secs, threads, sample = oracle_decode_sample("decode131k", 131072)
-        line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample,
+        line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": len(os.sched_getaffinity(0)),
+                                "blas_threads": threads, "kind": "oracle", "sample": sample,
                                 "seconds_per_sample": secs}
     if rank == 0:
         print(json.dumps(line), flush=True)

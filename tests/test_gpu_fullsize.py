@@ -4,13 +4,15 @@ Each test builds one layer of a benchmark workload through the benchmark's own c
 context length, head counts, page table, split plan and launch sequence as every timed
 layer), runs that layer once, and checks outputs against the oracle:
 
-* decode, 131,072 tokens (Q8_0 K with Q4_0 or Q8_0 V, Q4_0 or Q5_1 K with Q4_0 V): every
+* decode, 131,072 tokens (every supported K / V format pair): every
   output row of the layer, plus page bytes of sampled blocks bit-exact;
 * MTP verify, 262,144 tokens + 4: the selection bit-exact (needles included) and the 4 x 24
   rows over the selected blocks, for two sampled KV heads;
 * chunked prefill, 524,288 prior tokens + the 2,048-token chunk: 64 seeded (token, query head)
   rows over the full context;
-* the streamed 524,288-token working set: selection and decode rows of two KV heads.
+* the host-streamed generation over 524,288 prompt tokens: 512 advancing steps, selection and
+  decode rows of two KV heads at steps 0, 255 and 511, and the host bytes of every generated
+  token's pages.
 
 The oracle's inputs are the same seeded draws (made on the device by torch's generator and
 copied to the host) with the oracle's own quantisation; nothing the CUDA library computes
@@ -43,7 +45,8 @@ def _oracle_unit(k, v, h, v_fmt, k_tail=None, v_tail=None, k_fmt="q8_0"):
     return OracleCache(kh[:, None], vh[:, None], v_fmt, k_fmt)
 
 
-@pytest.mark.parametrize("wname", ["decode131k", "decode131k_q8q8", "decode131k_q4q4", "decode131k_q51q4"])
+@pytest.mark.parametrize("wname", ["decode131k", "decode131k_q8q8", "decode131k_q4q4", "decode131k_q4q8",
+                                   "decode131k_q51q4", "decode131k_q51q8", "decode131k_q50q41"])
 def test_decode_full_context(kv_gpu, wname):
     b = bench.DecodeBench(kv_gpu, wname, torch.device(DEV), layers=1)
     b.layer(0)
@@ -121,24 +124,44 @@ def test_prefill_full_context_sampled_rows(kv_gpu):
 
 
 def test_stream_full_context(kv_gpu):
+    """The host-streamed generation at full size (one layer): 512 decode steps whose position
+    advances from 524,288; steps 0, 255 and 511 are checked against the oracle (selection
+    bit-exact, decode rows within the tolerance) and, after the generation, the host bytes of
+    every appended token's pages bit-exact."""
     b = bench.StreamBench(kv_gpu, torch.device(DEV), layers=1)
-    b.step(True)
+    w, g = b.w, b.w.group
+    ctx, S = w.context, w.steps
+    checks = {0: None, 255: None, 511: None}
+    for t in range(S):
+        b.step(True)
+        if t in checks:
+            torch.cuda.synchronize()
+            checks[t] = (b.out[0].cpu().numpy(), b.lse[0].cpu().numpy(), b.sel_l[0].cpu().numpy(),
+                         b.n_sel[0].cpu().numpy())
     torch.cuda.synchronize()
     assert kv_gpu.kvattn_device_error() == 0
-    w, g = b.w, b.w.group
-    ctx = w.context
-    T = ctx + 1
     k, v, _ = workload_layer_kv(w, 0, ctx, DEV)
-    q = b.q[0].cpu().numpy()
-    out, lse = b.out[0].cpu().numpy(), b.lse[0].cpu().numpy()
-    sel_l, n_sel = b.sel_l[0].cpu().numpy(), b.n_sel[0].cpu().numpy()
+    k_gen, v_gen = b.k_all[:, 0, 0], b.v_all[:, 0, 0]            # [S][H][256]
+    q_all = b.q_all[:, 0, 0].cpu().numpy()                        # [S][Hq][256]
+    host = b.host.numpy()
     for h in (1, 2):
-        oc = _oracle_unit(k, v, h, w.v_fmt, b.k_new[0], b.v_new[0])
+        oc = _oracle_unit(k, v, h, w.v_fmt, k_gen, v_gen)
         kc = oc.kc[: b.n_full * 128, 0].reshape(b.n_full, 128, 8, 32)
         kd = oc.kd[: b.n_full * 128, 0].reshape(b.n_full, 128, 8)
-        sc = osel.block_scores(osel.block_summaries(kc, kd), q[0, h * g:(h + 1) * g])
-        ref_sel, gap = osel.select_blocks(sc, b.n_full, b.nb, w.budget_blocks, 0)
-        assert gap > 1e-9 * np.abs(sc).max()
-        assert sel_l[h, : n_sel[h]].tolist() == ref_sel.tolist()
-        o_ref, l_ref = oc.attend(q[:, h * g:(h + 1) * g], [ctx], 0, g, key_idx=_selected_keys(ref_sel, T))
-        compare(out[:, h * g:(h + 1) * g], lse[:, h * g:(h + 1) * g], o_ref, l_ref)
+        summ = osel.block_summaries(kc, kd)
+        for t, (out, lse, sel_l, n_sel) in checks.items():
+            T = ctx + t + 1
+            n_total = b.n_full + t // 128 + 1
+            sc = osel.block_scores(summ, q_all[t, h * g:(h + 1) * g])
+            ref_sel, gap = osel.select_blocks(sc, b.n_full, n_total, w.budget_blocks, 0)
+            assert gap > 1e-9 * np.abs(sc).max()
+            assert sel_l[h, : n_sel[h]].tolist() == ref_sel.tolist(), t
+            o_ref, l_ref = oc.attend(q_all[t:t + 1, h * g:(h + 1) * g], [ctx + t], 0, g,
+                                     key_idx=_selected_keys(ref_sel, T))
+            compare(out[:, h * g:(h + 1) * g], lse[:, h * g:(h + 1) * g], o_ref, l_ref)
+        # every generated token's page in host RAM, bit-exact (the pages the generation filled)
+        for kk in range(b.n_tail):
+            blk = b.n_full + kk
+            page = host[int(b.tail_hosts[0, h, kk])]
+            assert np.array_equal(page[:34816], oc.page_bytes(0, blk, "k")), (h, kk, "k")
+            assert np.array_equal(page[34816:], oc.page_bytes(0, blk, "v")), (h, kk, "v")
