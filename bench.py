@@ -487,6 +487,9 @@ class StreamBench:
         self.tail_slots = torch.tensor([[[self.n_stream_slots + (l * H + h) * self.n_tail + k for k in range(self.n_tail)]
                                          for h in range(H)] for l in range(L)], dtype=torch.int32, device=device)
         self.tail_hosts = self.host_table[:, :, self.n_full:].contiguous()
+        # per (layer, generated-token page): the H host pages and device slots, contiguous
+        self.tail_hosts_k = self.tail_hosts.permute(0, 2, 1).contiguous()
+        self.tail_slots_k = self.tail_slots.permute(0, 2, 1).contiguous()
         self.reset()
         self.desc = kv.make_desc(H, Hq, self.slots, self.slots.data_ptr() + 34816, self.n_slots, k_page_stride=P,
                                  v_page_stride=P)
@@ -581,7 +584,7 @@ class StreamBench:
             timed[1].record()
         k = (w.context % 128 + t) // 128     # the generated-token page the token went to
         kv.kvattn_scatter_pages(self.host, self.PAGE, self.host.shape[0], self.slots, self.PAGE, self.n_slots,
-                                self.PAGE, self.tail_hosts[l, :, k], self.tail_slots[l, :, k], w.kv_heads, 4)
+                                self.PAGE, self.tail_hosts_k[l, k], self.tail_slots_k[l, k], w.kv_heads, 4)
 
     def step(self, stream_pages=True, timed=None):
         """One decode step of all layers at the current position; the position then advances

@@ -65,7 +65,7 @@ constexpr int kDq0 = (kSoftmaxWarps + 2) * 32;  // first dequant thread
 // 16-key group), and all V scales of the tile
 template <int KF>
 struct Raw {
-  static constexpr int kKc = KF == kKeyQ4 ? 2048 : 8192;
+  static constexpr int kKc = KF == kKeyQ4 ? 4096 : 8192;  // 32 keys x 128 or 256 bytes
   static constexpr int kKs = 512, kVc = 4096, kVs = 1024;
   static constexpr int kBytes = kKc + kKs + kVc + kVs;
 };

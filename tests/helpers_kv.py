@@ -76,7 +76,7 @@ class OracleCache:
             d[: b - a] = self.kd[a:b, h]
             return olay.encode_page("k", self.k_fmt, codes, d)
         codes = np.zeros((128, 8, 32), np.int8 if self.v_fmt == "q8_0" else np.uint8)
-        d = np.zeros((128, 8), np.float16)
+        d = np.zeros((128,) + self.vd.shape[2:], np.float16)  # (d, m) pairs for Q4_1
         codes[: b - a] = self.vc[a:b, h]
         d[: b - a] = self.vd[a:b, h]
         return olay.encode_page("v", self.v_fmt, codes, d)
