@@ -31,12 +31,17 @@
 namespace kvattn {
 
 
-template <int KF, int VF, int NT, bool PAIR>
+template <int KF, int VF, int NT, int SPLIT>
 struct DecodeCfg {
-  static constexpr int kConsumerWarps = 8;
-  static constexpr int kThreads = kConsumerWarps * 32;  // lane 0 of warp 0 also issues the copies
-  static constexpr int kNB = PAIR ? 4 : 8;      // 32-channel blocks per warp
-  static constexpr int kTilesPerWarp = PAIR ? 2 : 1;
+  // SPLIT warps share each 16-token tile, each taking 8 / SPLIT of the 32-channel blocks, and
+  // add their partial scores through shared memory.  Split tiles run 16 warps (at most 128
+  // registers each): four warps per scheduler hide the latency of the dequantize -> MMA
+  // chains.  Unsplit tiles run 8 warps.
+  static constexpr int kConsumerWarps = SPLIT == 1 ? 8 : 16;
+  static constexpr int kThreads = kConsumerWarps * 32;  // lanes of warp 0 also issue the copies
+  static constexpr int kNB = 8 / SPLIT;                 // 32-channel blocks per warp
+  static constexpr int kGroups = kConsumerWarps / SPLIT;  // warps groups, one softmax stream each
+  static constexpr int kTilesPerWarp = 8 / kGroups;
   static constexpr bool kK5 = KF == kKeyQ51 || KF == kKeyQ50;  // 5-bit key codes
   static constexpr bool kKMin = KF == kKeyQ51;                 // keys with a zero point
   static constexpr bool kVMin = VF == kValQ41;                 // values with a zero point
@@ -46,16 +51,18 @@ struct DecodeCfg {
   static constexpr int kVBytes = VF == kValQ8 ? kV8PageBytes : VF == kValQ41 ? kV41PageBytes : kV4PageBytes;
   static constexpr int kVScaleOff = VF == kValQ8 ? kV8ScaleOffset : kV4ScaleOffset;
   static constexpr int kStageBytes = kKBytes + kVBytes;
-  // the paired shapes (16 and 24 query rows) keep the query B fragments in shared memory:
-  // [half][block][k-step][n-tile][lane][hi0, hi1, lo0, lo1]
-  static constexpr bool kQSmem = PAIR;
-  static constexpr int kQBytes = kQSmem ? 2 * 4 * 2 * NT * 32 * 16 : 0;
-  // as many page stages as fit beside the pair exchange buffer and the barriers (at most 6)
-  static constexpr int kStagesFit = ((PAIR ? 190000 : 214000) - kQBytes) / kStageBytes;
-  static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
-  static constexpr int kUnits = PAIR ? 4 : 8;   // independent softmax streams per CTA
+  // split tiles keep the query B fragments in shared memory:
+  // [block][k-step][n-tile][lane][hi0, hi1, lo0, lo1]
+  static constexpr bool kQSmem = SPLIT > 1;
+  static constexpr int kQBytes = kQSmem ? 8 * 2 * NT * 32 * 16 : 0;
+  static constexpr int kUnits = kGroups;   // independent softmax streams per CTA
   static constexpr int kRowsPad = NT * 8;
-  static constexpr int kXBytes = PAIR ? 4 * 2 * 2 * NT * 32 * 16 : 0;  // pair S exchange
+  // partial-score exchange: [group][part][parity][n-tile][lane][4 floats]
+  static constexpr int kXBytes = SPLIT > 1 ? kGroups * SPLIT * 2 * NT * 32 * 16 : 0;
+  // as many page stages as fit beside the pair exchange buffer, the query fragments and the
+  // barriers (at most 6)
+  static constexpr int kStagesFit = (227 * 1024 - 256 - kXBytes - kQBytes) / kStageBytes;
+  static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
   static constexpr int kRingBytes = kStages * kStageBytes;
   // rows of the output merge buffer are padded by 4 floats: the four lanes of an MMA quad
   // store rows 2t, 2t+1 of the same dims and then fall into different banks
@@ -95,13 +102,13 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uin
   lo = pack_half2(x0 - half_lo(hi), x1 - half_hi(hi));
 }
 
-template <int KF, int VF, int NT, bool PAIR>
-__global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) decode_kernel(const DecodeParams p) {
-  using C = DecodeCfg<KF, VF, NT, PAIR>;
+template <int KF, int VF, int NT, int SPLIT>
+__global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) decode_kernel(const DecodeParams p) {
+  using C = DecodeCfg<KF, VF, NT, SPLIT>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
-  uint64_t* xbar = full + C::kStages;   // [4] pair exchange barriers (PAIR only)
-  int* rel_cnt = reinterpret_cast<int*>(xbar + 4);  // [kStages] warps done with the stage
+  uint64_t* xbar = full + C::kStages;   // [kGroups] score-exchange barriers (split tiles only)
+  int* rel_cnt = reinterpret_cast<int*>(xbar + C::kGroups);  // [kStages] warps done with the stage
   int* s_issued = rel_cnt + C::kStages;              // pages issued so far
   int* st_logical = s_issued + 1;
   int* st_valid = st_logical + C::kStages;
@@ -122,7 +129,7 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) deco
       rel_cnt[s] = 0;
     }
     *s_issued = 0;
-    for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 2);
+    for (int i = 0; i < C::kGroups; ++i) mbar_init(&xbar[i], SPLIT);
     s_flags[0] = 0;
     fence_barrier_init();
   }
@@ -164,8 +171,9 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) deco
 #pragma unroll
       for (int e = 0; e < 4; ++e) macc[i][nt][e] = 0.f;
 
-  const int half = PAIR ? (warp & 1) : 0;
-  const int blk0 = PAIR ? 4 * half : 0;
+  const int part = warp & (SPLIT - 1);  // this warp's share of the channel blocks
+  const int grp = warp / SPLIT;          // the warps that share a tile
+  const int blk0 = C::kNB * part;
 
   // Page copies: the first kStages pages are issued up front by lanes of warp 0; after
   // that, the warp that is the last of the eight to finish with a stage refills it at
@@ -254,7 +262,15 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) deco
       for (int bl = 0; bl < C::kNB; ++bl) {
         float xv[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) xv[e] = ((PAIR && half) ? x[(4 + bl) % kBlocks][e] : x[bl][e]) * inv;
+        for (int e = 0; e < 8; ++e) {
+          // block blk0 + bl, selected with constant indices (a runtime index would put x in
+          // local memory)
+          float xe = x[bl][e];
+#pragma unroll
+          for (int pp = 1; pp < SPLIT; ++pp)
+            if (part == pp) xe = x[pp * C::kNB + bl][e];
+          xv[e] = xe * inv;
+        }
         // k-step 0 of the block: channels 8t+0..3, k-step 1: 8t+4..7 (k = 2t, 2t+1 | 2t+8, 2t+9)
         uint32_t hi[2][2], lo[2][2];
 #pragma unroll
@@ -263,12 +279,12 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) deco
           split_pair(xv[4 * ks + 2], xv[4 * ks + 3], hi[ks][1], lo[ks][1]);
         }
         if constexpr (C::kQSmem) {
-          // warps of the same half hold the same values; warps 0 and 1 write them
-          if (warp < 2) {
+          // the warps of every group hold the same values; those of group 0 write them
+          if (warp < SPLIT) {
 #pragma unroll
             for (int ks = 0; ks < 2; ++ks)
               asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
-                               q_s + (((((half * 4 + bl) * 2 + ks) * NT + nt) * 32 + lane) * 16)),
+                               q_s + (((((blk0 + bl) * 2 + ks) * NT + nt) * 32 + lane) * 16)),
                            "r"(hi[ks][0]), "r"(hi[ks][1]), "r"(lo[ks][0]), "r"(lo[ks][1])
                            : "memory");
           }
@@ -303,7 +319,6 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) deco
     qpos_min = min(qpos_min, __shfl_xor_sync(0xffffffffu, qpos_min, 1));
     qpos_min = min(qpos_min, __shfl_xor_sync(0xffffffffu, qpos_min, 2));
 
-    const int pair = PAIR ? (warp >> 1) : 0;
     float* xbuf = reinterpret_cast<float*>(smem + C::kRingBytes);
     int xpar = 0;
     uint32_t xphase = 0;
@@ -312,7 +327,7 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) deco
     // the B fragments (hi0, hi1, lo0, lo1) of block bl, k-step ks, n-tile nt
     auto qfrag = [&](int bl, int ks, int nt) -> uint4 {
       if constexpr (C::kQSmem) {
-        return lds128(q_s + (((((half * 4 + bl) * 2 + ks) * NT + nt) * 32 + lane) * 16));
+        return lds128(q_s + (((((blk0 + bl) * 2 + ks) * NT + nt) * 32 + lane) * 16));
       } else {
         return make_uint4(qh[bl][ks][nt][0], qh[bl][ks][nt][1], ql[bl][ks][nt][0], ql[bl][ks][nt][1]);
       }
@@ -332,7 +347,7 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) deco
         const bool need_mask = static_cast<long long>(logical) * kPageTokens + (kPageTokens - 1) > qpos_min;
 #pragma unroll
         for (int tt = 0; tt < C::kTilesPerWarp; ++tt) {
-          const int G = PAIR ? (2 * pair + tt) : warp;
+          const int G = SPLIT > 1 ? (C::kTilesPerWarp * grp + tt) : warp;
           // ---------------- S = K Q^T over this warp's channel blocks ----------------
           // Key codes enter the MMA exactly (integers in f16).  Each 32-channel block is
           // accumulated on its own (four MMAs: two k-steps, query high and low parts) and then
@@ -357,7 +372,7 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) deco
                 const uint4 vm = lds128(a + (kK5MinOffset - kK5ScaleOffset));
                 wm[0] = vm.x; wm[1] = vm.y; wm[2] = vm.z; wm[3] = vm.w;
               }
-            } else {
+            } else if constexpr (C::kNB == 4) {
               asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(a));
               w[2] = w[3] = 0u;
               if constexpr (C::kKMin) {
@@ -365,6 +380,13 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) deco
                              : "=r"(wm[0]), "=r"(wm[1])
                              : "r"(a + (kK5MinOffset - kK5ScaleOffset)));
                 wm[2] = wm[3] = 0u;
+              }
+            } else {
+              w[0] = lds32(a);
+              w[1] = w[2] = w[3] = 0u;
+              if constexpr (C::kKMin) {
+                wm[0] = lds32(a + (kK5MinOffset - kK5ScaleOffset));
+                wm[1] = wm[2] = wm[3] = 0u;
               }
             }
 #pragma unroll
@@ -427,22 +449,37 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) deco
             // 1024 + 16q).  5-bit keys: the fifth bits of the lane's four blocks of one token
             // sit in one word, channel (c, i) at bit 16(i%2) + 4c + i/2, and are shifted to bit 4
             // or bit 8 of each half.  The code (minus 8 for Q4_0, 16 for Q5_0) is exact in f16.
+            // A warp with two blocks of a block quad reads their two words, at word c0 = blk0 % 4,
+            // and shifts the fifth-bit word right by 4 c0 so that its blocks sit at c = 0, 1.
+            constexpr int kWords = C::kNB < 4 ? C::kNB : 4;
+            const int c0 = blk0 & 3;
 #pragma unroll
-            for (int qq = 0; qq < C::kNB / 4; ++qq) {
+            for (int qq = 0; qq < (C::kNB + 3) / 4; ++qq) {
               const int Q = blk0 / 4 + qq;
               const int row0 = (((G * 2 + Q) * 2 + 0) * 8 + g) * 4 + t;
               const int row1 = (((G * 2 + Q) * 2 + 1) * 8 + g) * 4 + t;
-              const uint4 ka = lds128(kb + row0 * 16);
-              const uint4 kc = lds128(kb + row1 * 16);
+              uint32_t wa[4], wc[4];
+              if constexpr (kWords == 4) {
+                const uint4 ka = lds128(kb + row0 * 16);
+                const uint4 kc = lds128(kb + row1 * 16);
+                wa[0] = ka.x; wa[1] = ka.y; wa[2] = ka.z; wa[3] = ka.w;
+                wc[0] = kc.x; wc[1] = kc.y; wc[2] = kc.z; wc[3] = kc.w;
+              } else {
+                asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(wa[0]), "=r"(wa[1]) : "r"(kb + row0 * 16 + 4 * c0));
+                asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(wc[0]), "=r"(wc[1]) : "r"(kb + row1 * 16 + 4 * c0));
+                wa[2] = wa[3] = wc[2] = wc[3] = 0u;
+              }
               uint32_t xa5 = 0, xc5 = 0;
               if constexpr (C::kK5) {
                 xa5 = lds32(kb + kK5HighOffset + row0 * 4);
                 xc5 = lds32(kb + kK5HighOffset + row1 * 4);
+                if constexpr (kWords < 4) {
+                  xa5 >>= 4 * c0;
+                  xc5 >>= 4 * c0;
+                }
               }
-              const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
-              const uint32_t wc[4] = {kc.x, kc.y, kc.z, kc.w};
 #pragma unroll
-              for (int c = 0; c < 4; ++c) {
+              for (int c = 0; c < kWords; ++c) {
                 uint32_t A[2][4];
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks) {
@@ -472,17 +509,19 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) deco
               }
             }
           }
-          if constexpr (PAIR) {
-            // exchange partial scores with the partner warp (other channel half)
-            float* mine = xbuf + ((((pair * 2 + half) * 2 + xpar) * NT) * 32) * 4;
-            float* theirs = xbuf + ((((pair * 2 + (half ^ 1)) * 2 + xpar) * NT) * 32) * 4;
+          if constexpr (SPLIT > 1) {
+            // exchange partial scores with the other warps of the group (the other channel
+            // blocks); every warp adds the SPLIT parts in the same order (its own part from its
+            // registers), so all of them hold bit-identical sums
+            auto slot = [&](int q) { return xbuf + ((((grp * SPLIT + q) * 2 + xpar) * NT) * 32) * 4; };
+            float* mine = slot(part);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
               *reinterpret_cast<float4*>(mine + (nt * 32 + lane) * 4) =
                   make_float4(sacc[nt][0], sacc[nt][1], sacc[nt][2], sacc[nt][3]);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&xbar[pair]);
-            if (!mbar_wait(&xbar[pair], xphase)) {
+            if (lane == 0) mbar_arrive(&xbar[grp]);
+            if (!mbar_wait(&xbar[grp], xphase)) {
               s_flags[0] = 1;
               aborted = true;
               break;
@@ -490,14 +529,22 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) deco
             xphase ^= 1;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              const float4 o = *reinterpret_cast<const float4*>(theirs + (nt * 32 + lane) * 4);
-              // same operands in both warps, so both get bit-identical sums
-              if (half == 0) {
-                sacc[nt][0] += o.x; sacc[nt][1] += o.y; sacc[nt][2] += o.z; sacc[nt][3] += o.w;
-              } else {
-                sacc[nt][0] = o.x + sacc[nt][0]; sacc[nt][1] = o.y + sacc[nt][1];
-                sacc[nt][2] = o.z + sacc[nt][2]; sacc[nt][3] = o.w + sacc[nt][3];
+              float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+              for (int q = 0; q < SPLIT; ++q) {
+                float4 o;
+                if (q == part) {
+                  o = make_float4(sacc[nt][0], sacc[nt][1], sacc[nt][2], sacc[nt][3]);
+                } else {
+                  o = *reinterpret_cast<const float4*>(slot(q) + (nt * 32 + lane) * 4);
+                }
+                if (q == 0) {
+                  acc = o;
+                } else {
+                  acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+                }
               }
+              sacc[nt][0] = acc.x; sacc[nt][1] = acc.y; sacc[nt][2] = acc.z; sacc[nt][3] = acc.w;
             }
             xpar ^= 1;
           }
@@ -695,8 +742,8 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, PAIR>::kThreads, 1) deco
   float* ls = ms + C::kUnits * C::kRowsPad;
   float* os = ls + C::kUnits * C::kRowsPad;
   {
-    const int unit = PAIR ? (warp >> 1) : warp;
-    if (g == 0 && half == 0) {
+    const int unit = SPLIT > 1 ? grp : warp;
+    if (g == 0 && part == 0) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -859,9 +906,9 @@ cudaError_t launch_decode_merge(const DecodeParams& prm, int n_kv, cudaStream_t 
                             decode_rows_pad(prm.group * prm.n_q), prm.group, prm.n_qh, prm.out, prm.lse);
 }
 
-template <int KF, int VF, int NT, bool PAIR>
+template <int KF, int VF, int NT, int SPLIT>
 static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream_t stream) {
-  using C = DecodeCfg<KF, VF, NT, PAIR>;
+  using C = DecodeCfg<KF, VF, NT, SPLIT>;
   // programmatic dependent launch: the grid may start while the previous kernel on the
   // stream drains; the kernel waits for it (griddepcontrol.wait) before reading any input
   cudaLaunchConfig_t cfg = {};
@@ -874,7 +921,7 @@ static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<KF, VF, NT, PAIR>, prm);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<KF, VF, NT, SPLIT>, prm);
 }
 
 // The supported (key, value) format pairs: Q8_0 keys with Q4_0 or Q8_0 values, Q4_0 and Q5_1
@@ -892,11 +939,11 @@ bool decode_pair_supported(int key_fmt, int val_fmt) {
 
 cudaError_t prepare_decode_kernels() {
   cudaError_t e;
-#define KV_SET1(KF, VF, NT, PAIR)                                                                   \
-  e = cudaFuncSetAttribute(decode_kernel<KF, VF, NT, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                           DecodeCfg<KF, VF, NT, PAIR>::kSmemBytes);                               \
+#define KV_SET1(KF, VF, NT, SPLIT)                                                                   \
+  e = cudaFuncSetAttribute(decode_kernel<KF, VF, NT, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                           DecodeCfg<KF, VF, NT, SPLIT>::kSmemBytes);                               \
   if (e != cudaSuccess) return e;
-#define KV_SET(KF, VF) KV_SET1(KF, VF, 1, false) KV_SET1(KF, VF, 2, true) KV_SET1(KF, VF, 3, true)
+#define KV_SET(KF, VF) KV_SET1(KF, VF, 1, 2) KV_SET1(KF, VF, 2, 4) KV_SET1(KF, VF, 3, 4)
   KVATTN_DECODE_PAIRS(KV_SET)
 #undef KV_SET
 #undef KV_SET1
@@ -905,9 +952,9 @@ cudaError_t prepare_decode_kernels() {
 
 template <int KF, int VF>
 static cudaError_t launch_decode_fmt(const DecodeParams& prm, int n_kv, int nt, cudaStream_t stream) {
-  if (nt == 1) return launch_decode_t<KF, VF, 1, false>(prm, n_kv, stream);
-  if (nt == 2) return launch_decode_t<KF, VF, 2, true>(prm, n_kv, stream);
-  return launch_decode_t<KF, VF, 3, true>(prm, n_kv, stream);
+  if (nt == 1) return launch_decode_t<KF, VF, 1, 2>(prm, n_kv, stream);
+  if (nt == 2) return launch_decode_t<KF, VF, 2, 4>(prm, n_kv, stream);
+  return launch_decode_t<KF, VF, 3, 4>(prm, n_kv, stream);
 }
 
 cudaError_t launch_decode(const DecodeParams& prm, int n_kv, int key_fmt, int val_fmt, cudaStream_t stream) {
