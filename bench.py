@@ -294,17 +294,19 @@ class DecodeBench(GraphStep):
         self.ws = torch.zeros((L, max(self.ws_bytes, 256)), dtype=torch.uint8, device=device)
         self.bytes_per_layer = self.ctx * H * bytes_per_token_head(w.k_fmt, w.v_fmt)
         self.bytes_per_step = self.bytes_per_layer * L
-        self.launches_per_step = 3 * L  # quantize-append, decode, split merge
+        self.launches_per_step = 2 * L  # decode with the append fused in, split merge
 
     def layer(self, l, timed=None):
-        """One layer: quantize-append the new token, then kvattn_decode.  With `timed` (three
-        events) the decode runs as its two grids with an event before, between and after them."""
+        """One layer: append the new token and attend, as one kvattn_append_decode (its split
+        grid, then the merge grid).  With `timed` (three events) the append is its own kernel
+        and the decode runs as its two grids with an event before, between and after them."""
         kv, c = self.kv, self.cache
-        kv.kvattn_quantize_append(c.desc, self.k_new[l], self.v_new[l], 1, self.pos, c.page_table[l], self.nb)
         if timed is None:
-            kv.kvattn_decode(c.desc, self.q[l], 1, self.q_pos, c.page_table[l], None, None, self.nb, self.out[l],
-                             self.lse[l], self.ws[l], self.ws_bytes)
+            kv.kvattn_append_decode(c.desc, self.k_new[l], self.v_new[l], 1, self.pos, c.page_table[l], self.nb,
+                                    self.q[l], 1, self.q_pos, c.page_table[l], None, None, self.nb, self.out[l],
+                                    self.lse[l], self.ws[l], self.ws_bytes)
             return
+        kv.kvattn_quantize_append(c.desc, self.k_new[l], self.v_new[l], 1, self.pos, c.page_table[l], self.nb)
         timed[0].record()
         kv.kvattn_decode_splits(c.desc, self.q[l], 1, self.q_pos, c.page_table[l], None, None, self.nb, self.out[l],
                                 self.lse[l], self.ws[l], self.ws_bytes)
@@ -355,18 +357,19 @@ class VerifyBench(GraphStep):
         self.bytes_per_layer = tokens * H * bytes_per_token_head(w.k_fmt, w.v_fmt)
         self.bytes_per_step = self.bytes_per_layer * L
         self.select_bytes_per_layer = H * (self.n_full - w.recent_blocks) * 256 * 4
-        self.launches_per_step = 5 * L  # block scores, top-k, quantize-append, decode, split merge
+        self.launches_per_step = 4 * L  # block scores, top-k, decode with the append fused in, split merge
 
     def layer(self, l, timed=None):
         kv, c, w = self.kv, self.cache, self.w
         kv.kvattn_select_blocks(self.summ[l * w.kv_heads:(l + 1) * w.kv_heads], self.q_group[l], w.kv_heads, w.group,
                                 self.nb, self.n_full, self.nb, w.budget_blocks, w.recent_blocks, c.page_table[l],
                                 self.sel_l[l], self.sel_p[l], self.n_sel[l], self.cap, self.sws, self.sws_bytes)
-        kv.kvattn_quantize_append(c.desc, self.k_new[l], self.v_new[l], w.n_q, self.pos0, c.page_table[l], self.nb)
         if timed is None:
-            kv.kvattn_decode(c.desc, self.q[l], w.n_q, self.q_pos, self.sel_p[l], self.sel_l[l], self.n_sel[l],
-                             self.cap, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
+            kv.kvattn_append_decode(c.desc, self.k_new[l], self.v_new[l], w.n_q, self.pos0, c.page_table[l], self.nb,
+                                    self.q[l], w.n_q, self.q_pos, self.sel_p[l], self.sel_l[l], self.n_sel[l],
+                                    self.cap, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
             return
+        kv.kvattn_quantize_append(c.desc, self.k_new[l], self.v_new[l], w.n_q, self.pos0, c.page_table[l], self.nb)
         timed[0].record()
         kv.kvattn_decode_splits(c.desc, self.q[l], w.n_q, self.q_pos, self.sel_p[l], self.sel_l[l], self.n_sel[l],
                                 self.cap, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
@@ -535,7 +538,7 @@ class StreamBench:
         self.ev_copy = [torch.cuda.Event() for _ in range(L)]
         self.ev_dec = [torch.cuda.Event() for _ in range(L)]
         self.copy_bytes_per_step = L * H * self.budget * P
-        self.launches_per_step = 6 * L  # scores, top-k, copy, append, decode (+ merge), write-back
+        self.launches_per_step = 6 * L  # scores, top-k, copy, decode with the append (+ merge), write-back
         self.gather_ctas = 16
 
     def reset(self):
@@ -575,12 +578,16 @@ class StreamBench:
     def _attend(self, l, timed=None):
         kv, w, t = self.kv, self.w, self.gen_t
         pos = w.context + t
-        kv.kvattn_quantize_append(self.desc, self.k_all[t, l], self.v_all[t, l], 1, pos, self.tail_tab[l], self.nb)
-        if timed is not None:
+        if timed is None:
+            kv.kvattn_append_decode(self.desc, self.k_all[t, l], self.v_all[t, l], 1, pos, self.tail_tab[l], self.nb,
+                                    self.q_all[t, l], 1, self.pos_all[t:t + 1], self.plist[l], self.sel_l[l],
+                                    self.n_sel[l], self.cap, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
+        else:
+            kv.kvattn_quantize_append(self.desc, self.k_all[t, l], self.v_all[t, l], 1, pos, self.tail_tab[l],
+                                      self.nb)
             timed[0].record()
-        kv.kvattn_decode(self.desc, self.q_all[t, l], 1, self.pos_all[t:t + 1], self.plist[l], self.sel_l[l],
-                         self.n_sel[l], self.cap, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
-        if timed is not None:
+            kv.kvattn_decode(self.desc, self.q_all[t, l], 1, self.pos_all[t:t + 1], self.plist[l], self.sel_l[l],
+                             self.n_sel[l], self.cap, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
             timed[1].record()
         k = (w.context % 128 + t) // 128     # the generated-token page the token went to
         kv.kvattn_scatter_pages(self.host, self.PAGE, self.host.shape[0], self.slots, self.PAGE, self.n_slots,
@@ -981,7 +988,7 @@ def main():
 
     # ---------------- headline: decode at 131K ----------------
     b = DecodeBench(kvattn, "decode131k", device, layers=args.layers)
-    launch_mode = "one CUDA graph per step (3 launches per layer, programmatic dependent launch)"
+    launch_mode = "one CUDA graph per step (2 launches per layer: kvattn_append_decode's two grids, programmatic dependent launch)"
     try:
         b.capture()
     except Exception as exc:  # report and time the direct launches instead

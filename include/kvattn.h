@@ -197,6 +197,20 @@ KVATTN_API int kvattn_decode(const kvattn_kv_desc* desc, const float* q, int n_q
                              const int32_t* n_pages, int max_pages, float* out, float* lse,
                              void* ws, size_t ws_bytes, kvattn_stream_t stream);
 
+/* kvattn_quantize_append of n_new tokens followed by kvattn_decode, in one grid: the same
+ * bytes land in the pages and the same outputs result, without the append kernel and its
+ * dependency on the stream.  The first CTA of every KV head encodes the new tokens into their
+ * pages in global memory; a CTA that streams such a page encodes the token again into its
+ * shared-memory copy before reading it, so no CTA waits for another.  Arguments are those of
+ * the two calls (k_new, v_new device fp32 [n_new][H_kv][256] at positions pos0 .. pos0 +
+ * n_new - 1, pages from page_table [H_kv][n_blocks]), with 1 <= n_new <= 8.  Errors as for
+ * both calls. */
+KVATTN_API int kvattn_append_decode(const kvattn_kv_desc* desc, const float* k_new, const float* v_new, int n_new,
+                                    int32_t pos0, const int32_t* page_table, int n_blocks, const float* q,
+                                    int n_q, const int32_t* q_pos, const int32_t* page_list,
+                                    const int32_t* page_logical, const int32_t* n_pages, int max_pages,
+                                    float* out, float* lse, void* ws, size_t ws_bytes, kvattn_stream_t stream);
+
 /* The two grids of kvattn_decode, as separate calls (same arguments; kvattn_decode is
  * kvattn_decode_splits followed by kvattn_decode_merge_splits on the same stream and
  * workspace).  kvattn_decode_splits runs the split grid: per-split (o, lse) partials into ws,

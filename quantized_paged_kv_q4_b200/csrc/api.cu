@@ -285,6 +285,31 @@ KVATTN_API int kvattn_decode(const kvattn_kv_desc* desc, const float* q, int n_q
   return e == cudaSuccess ? KVATTN_OK : cuda_fail(e);
 }
 
+KVATTN_API int kvattn_append_decode(const kvattn_kv_desc* desc, const float* k_new, const float* v_new, int n_new,
+                                    int32_t pos0, const int32_t* page_table, int n_blocks, const float* q, int n_q,
+                                    const int32_t* q_pos, const int32_t* page_list, const int32_t* page_logical,
+                                    const int32_t* n_pages, int max_pages, float* out, float* lse, void* ws,
+                                    size_t ws_bytes, kvattn_stream_t stream) {
+  const CallRange range_("kvattn_append_decode");
+  if (n_new < 1 || n_new > kMaxAppend || pos0 < 0 || n_blocks < 0) return KVATTN_ERR_INVALID_ARG;
+  if (!k_new || !v_new || !page_table || !aligned16(k_new) || !aligned16(v_new)) return KVATTN_ERR_INVALID_ARG;
+  if ((static_cast<int64_t>(pos0) + n_new - 1) / kPageTokens >= n_blocks) return KVATTN_ERR_INVALID_ARG;
+  DecodeParams prm;
+  const int st =
+      decode_setup(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pages, out, lse, ws, ws_bytes, &prm);
+  if (st) return st;
+  prm.k_new = k_new;
+  prm.v_new = v_new;
+  prm.n_new = n_new;
+  prm.new_pos0 = pos0;
+  prm.new_table = page_table;
+  prm.new_blocks = n_blocks;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_decode(prm, desc->n_kv_heads, key_format_id(desc->k_fmt), value_format_id(desc->v_fmt), s);
+  if (e == cudaSuccess) e = launch_decode_merge(prm, desc->n_kv_heads, s);
+  return e == cudaSuccess ? KVATTN_OK : cuda_fail(e);
+}
+
 KVATTN_API int kvattn_decode_splits(const kvattn_kv_desc* desc, const float* q, int n_q, const int32_t* q_pos,
                                     const int32_t* page_list, const int32_t* page_logical, const int32_t* n_pages,
                                     int max_pages, float* out, float* lse, void* ws, size_t ws_bytes,

@@ -34,13 +34,15 @@ namespace kvattn {
 template <int KF, int VF, int NT, int SPLIT>
 struct DecodeCfg {
   // SPLIT warps share each 16-token tile, each taking 8 / SPLIT of the 32-channel blocks, and
-  // add their partial scores through shared memory.  Split tiles run 16 warps (at most 128
-  // registers each): four warps per scheduler hide the latency of the dequantize -> MMA
-  // chains.  Unsplit tiles run 8 warps.
-  static constexpr int kConsumerWarps = SPLIT == 1 ? 8 : 16;
+  // add their partial scores through shared memory; a group of SPLIT warps walks SPLIT tiles
+  // of every page.  The 8-row shape runs unsplit tiles (SPLIT = 1); the 16- and 24-row shapes
+  // split them in two, which halves the accumulators per warp.  (Sixteen warps in the split
+  // arrangement measured slower for 8 rows: the duplicated softmax and the exchange cost more
+  // instructions than the extra warps hid.)
+  static constexpr int kConsumerWarps = 8;
   static constexpr int kThreads = kConsumerWarps * 32;  // lanes of warp 0 also issue the copies
   static constexpr int kNB = 8 / SPLIT;                 // 32-channel blocks per warp
-  static constexpr int kGroups = kConsumerWarps / SPLIT;  // warps groups, one softmax stream each
+  static constexpr int kGroups = kConsumerWarps / SPLIT;  // warp groups, one softmax stream each
   static constexpr int kTilesPerWarp = 8 / kGroups;
   static constexpr bool kK5 = KF == kKeyQ51 || KF == kKeyQ50;  // 5-bit key codes
   static constexpr bool kKMin = KF == kKeyQ51;                 // keys with a zero point
@@ -205,6 +207,27 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
     __syncwarp();
     if (lane == 0) *reinterpret_cast<volatile int*>(s_issued) = count < C::kStages ? count : C::kStages;
   }
+  // Appended tokens: split 0 of every head encodes them into their pages in global memory, one
+  // warp per token (warps 1 ..).  A CTA that streams such a page encodes the token again into
+  // its shared-memory copy before using it (below), so no CTA waits for another.
+  if (p.n_new > 0 && split == 0 && warp >= 1 && warp <= p.n_new) {
+    const int i = warp - 1;
+    const int pos = p.new_pos0 + i;
+    const long long row = (static_cast<long long>(i) * gridDim.y + h) * kHeadDim;
+    const float4* ks = reinterpret_cast<const float4*>(p.k_new + row + lane * 8);
+    const float4* vs = reinterpret_cast<const float4*>(p.v_new + row + lane * 8);
+    const float4 k0 = ks[0], k1 = ks[1], v0 = vs[0], v1 = vs[1];
+    const int page = p.new_table[static_cast<long long>(h) * p.new_blocks + pos / kPageTokens];
+    if (page < 0 || page >= p.n_pages) {
+      if (lane == 0) record_error(KVATTN_ERR_BAD_PAGE);
+    } else {
+      const float kx[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+      const float vx[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      encode_token(kx, vx, lane, const_cast<uint8_t*>(p.k_pool) + static_cast<int64_t>(page) * p.k_stride,
+                   const_cast<uint8_t*>(p.v_pool) + static_cast<int64_t>(page) * p.v_stride, pos % kPageTokens, KF,
+                   VF, 0xffffffffu);
+    }
+  }
 
   {
     // ------------------------------------------------------------------ consumers
@@ -348,6 +371,29 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
 #pragma unroll
         for (int tt = 0; tt < C::kTilesPerWarp; ++tt) {
           const int G = SPLIT > 1 ? (C::kTilesPerWarp * grp + tt) : warp;
+          if (p.n_new > 0) {
+            // an appended token in this tile: encode it into the stage (this warp's channel
+            // blocks), as split 0 encodes it into the page in global memory
+            const int pos_lo = logical * kPageTokens + 16 * G;
+#pragma unroll 1
+            for (int i = 0; i < p.n_new; ++i) {
+              const int pos = p.new_pos0 + i;
+              if (pos < pos_lo || pos >= pos_lo + 16) continue;
+              const long long row = (static_cast<long long>(i) * gridDim.y + h) * kHeadDim;
+              const float4* ks = reinterpret_cast<const float4*>(p.k_new + row + lane * 8);
+              const float4* vs = reinterpret_cast<const float4*>(p.v_new + row + lane * 8);
+              const float4 k0 = ks[0], k1 = ks[1], v0 = vs[0], v1 = vs[1];
+              const float kx[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+              const float vx[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+              constexpr int kLanes = 32 / SPLIT;  // lanes 4b .. 4b + 3 hold block b
+              const uint32_t mask = SPLIT == 1 ? 0xffffffffu : (((1u << kLanes) - 1u) << (kLanes * part));
+              uint8_t* stage = smem + s * C::kStageBytes;
+              encode_token(kx, vx, lane, stage, stage + C::kKBytes, pos - logical * kPageTokens, KF, VF, mask);
+              // the stage is later refilled by the copy engine (async proxy)
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+              __syncwarp();
+            }
+          }
           // ---------------- S = K Q^T over this warp's channel blocks ----------------
           // Key codes enter the MMA exactly (integers in f16).  Each 32-channel block is
           // accumulated on its own (four MMAs: two k-steps, query high and low parts) and then
@@ -943,7 +989,7 @@ cudaError_t prepare_decode_kernels() {
   e = cudaFuncSetAttribute(decode_kernel<KF, VF, NT, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                            DecodeCfg<KF, VF, NT, SPLIT>::kSmemBytes);                               \
   if (e != cudaSuccess) return e;
-#define KV_SET(KF, VF) KV_SET1(KF, VF, 1, 2) KV_SET1(KF, VF, 2, 4) KV_SET1(KF, VF, 3, 4)
+#define KV_SET(KF, VF) KV_SET1(KF, VF, 1, 1) KV_SET1(KF, VF, 2, 2) KV_SET1(KF, VF, 3, 2)
   KVATTN_DECODE_PAIRS(KV_SET)
 #undef KV_SET
 #undef KV_SET1
@@ -952,9 +998,9 @@ cudaError_t prepare_decode_kernels() {
 
 template <int KF, int VF>
 static cudaError_t launch_decode_fmt(const DecodeParams& prm, int n_kv, int nt, cudaStream_t stream) {
-  if (nt == 1) return launch_decode_t<KF, VF, 1, 2>(prm, n_kv, stream);
-  if (nt == 2) return launch_decode_t<KF, VF, 2, 4>(prm, n_kv, stream);
-  return launch_decode_t<KF, VF, 3, 4>(prm, n_kv, stream);
+  if (nt == 1) return launch_decode_t<KF, VF, 1, 1>(prm, n_kv, stream);
+  if (nt == 2) return launch_decode_t<KF, VF, 2, 2>(prm, n_kv, stream);
+  return launch_decode_t<KF, VF, 3, 2>(prm, n_kv, stream);
 }
 
 cudaError_t launch_decode(const DecodeParams& prm, int n_kv, int key_fmt, int val_fmt, cudaStream_t stream) {

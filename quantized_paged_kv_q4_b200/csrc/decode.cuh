@@ -19,7 +19,16 @@ struct DecodeParams {
   float* part_o;    // [H_kv][n_splits][rows_pad][256]
   float* part_lse;  // [H_kv][n_splits][rows_pad]   (log2 units)
   int n_q, group, n_qh, max_pages, n_splits;
+  // tokens to append before attending (0 for a plain decode): fp32 [n_new][H_kv][256] K and V
+  // at positions new_pos0 + i, pages from new_table [H_kv][new_blocks]
+  const float* k_new;
+  const float* v_new;
+  const int32_t* new_table;
+  int n_new, new_pos0, new_blocks;
 };
+
+// Most tokens kvattn_append_decode appends in one call.
+constexpr int kMaxAppend = 8;
 
 // The split grid of a decode (partials into the workspace, or out / lse for one split) ...
 cudaError_t launch_decode(const DecodeParams& prm, int n_kv, int key_fmt, int val_fmt, cudaStream_t stream);

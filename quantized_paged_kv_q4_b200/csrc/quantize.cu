@@ -110,6 +110,146 @@ __device__ __forceinline__ int min_code(float x, float mn, float inv) {
 }
 
 
+// Encodes one token of one KV head into slot `tok` of its K page (kpg) and V page (vpg), in
+// any memory space (global pages, or a page's copy in shared memory).  The 32 lanes of the
+// calling warp each hold 8 channels: kx / vx are channels 8 lane .. 8 lane + 7 of K and V.
+// Every lane takes part in the shuffles; only lanes whose bit is set in store_mask write, so
+// a warp may write just its own 32-channel blocks (lanes 4b .. 4b + 3 hold block b).
+__device__ __forceinline__ void encode_token(const float (&kx)[8], const float (&vx)[8], int lane, uint8_t* kpg,
+                                             uint8_t* vpg, int tok, int k_fmt, int v_fmt, uint32_t store_mask) {
+  const bool st = (store_mask >> lane) & 1u;
+  const int G = tok >> 4, tl = tok & 15, H = tl >> 3, R = tok & 7;
+  const int b = lane >> 2;  // this lane's block
+
+  // ---------------- K: Q5_1 / Q5_0 ----------------
+  if (k_fmt == kKeyQ51 || k_fmt == kKeyQ50) {
+    const float (&x)[8] = kx;
+    float mn = 0.f, inv, d;
+    if (k_fmt == kKeyQ51) {
+      d = min_scale<31>(x, &mn, &inv);
+    } else {
+      d = offset_scale<16>(x, lane, &inv);
+    }
+    const int T = lane & 3, c = b & 3, Q = b >> 2;
+    // low nibbles as the Q4_0 key word; fifth bits of the four blocks 4Q..4Q+3 of this T
+    // (lanes T + 4c + 16Q) gathered into one word, channel (c, e) at bit 16(e%2) + 4c + e/2
+    uint32_t w = 0, hb = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t q = static_cast<uint32_t>(k_fmt == kKeyQ51 ? min_code<31>(x[e], mn, inv)
+                                                                : offset_code<16>(x[e], inv));
+      w |= (q & 15u) << (4 * (e >> 1) + 16 * (e & 1));
+      hb |= (q >> 4) << (16 * (e & 1) + 4 * c + (e >> 1));
+    }
+    hb |= __shfl_xor_sync(0xffffffffu, hb, 4);
+    hb |= __shfl_xor_sync(0xffffffffu, hb, 8);
+    uint8_t* pg = kpg;
+    const int row = (((G * 2 + Q) * 2 + H) * 8 + R) * 4 + T;
+    if (st) *reinterpret_cast<uint32_t*>(pg + 4 * (row * 4 + c)) = w;
+    if (st && c == 0) *reinterpret_cast<uint32_t*>(pg + kK5HighOffset + 4 * row) = hb;
+    if (st && (lane & 3) == 0) {
+      const int si = 2 * (((G * 8 + R) * 2 + H) * 8 + b);
+      *reinterpret_cast<__half*>(pg + kK5ScaleOffset + si) = __float2half_rn(d);
+      if (k_fmt == kKeyQ51) *reinterpret_cast<__half*>(pg + kK5MinOffset + si) = __float2half_rn(mn);
+    }
+  }
+  // ---------------- K: Q4_0 ----------------
+  else if (k_fmt == kKeyQ4) {
+    const float (&x)[8] = kx;
+    float inv;
+    const float d = q4_scale(x, lane, &inv);
+    // one 32-bit word per lane: channel 8T + e at bit 4 * (e / 2) + 16 * (e % 2)
+    uint32_t w = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) w |= static_cast<uint32_t>(q4_code(x[e], inv)) << (4 * (e >> 1) + 16 * (e & 1));
+    uint8_t* pg = kpg;
+    const int T = lane & 3;
+    const int word = ((((G * 2 + (b >> 2)) * 2 + H) * 8 + R) * 4 + T) * 4 + (b & 3);
+    if (st) *reinterpret_cast<uint32_t*>(pg + 4 * word) = w;
+    if (st && (lane & 3) == 0) {
+      const int so = kK4ScaleOffset + 2 * (((G * 8 + R) * 2 + H) * 8 + b);
+      *reinterpret_cast<__half*>(pg + so) = __float2half_rn(d);
+    }
+  }
+  // ---------------- K: Q8_0 ----------------
+  else {
+    const float (&x)[8] = kx;
+    float inv;
+    const float d = q8_scale(x, &inv);
+    uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w0 |= (static_cast<uint32_t>(q8_code(x[e], inv)) & 0xFFu) << (8 * e);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w1 |= (static_cast<uint32_t>(q8_code(x[4 + e], inv)) & 0xFFu) << (8 * e);
+    uint8_t* pg = kpg;
+    const int P = lane >> 3, T = lane & 3, jhi = (lane & 7) >> 2;
+    const int off = ((((G * 4 + P) * 2 + H) * 8 + R) * 4 + T) * 16 + 8 * jhi;
+    if (st) *reinterpret_cast<uint2*>(pg + off) = make_uint2(w0, w1);
+    if (st && (lane & 3) == 0) {
+      const int so = kKScaleOffset + 2 * (((G * 8 + R) * 2 + H) * 8 + b);
+      *reinterpret_cast<__half*>(pg + so) = __float2half_rn(d);
+    }
+  }
+
+  // ---------------- V: Q4_0, Q4_1 or Q8_0 ----------------
+  {
+    const float (&x)[8] = vx;
+    uint8_t* pg = vpg;
+    const int T = (tl & 7) >> 1, wlo = tl >> 3, ylo = tl & 1;
+    const int k_slot = ylo + 2 * wlo;
+    const int cl = lane & 3;  // which 8-channel group of the block
+    float d;
+    int codes[8];
+    if (v_fmt != kValQ8) {
+      float inv, mn = 0.f;
+      if (v_fmt == kValQ41) {
+        d = min_scale<15>(x, &mn, &inv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) codes[e] = min_code<15>(x[e], mn, inv);
+      } else {
+        d = q4_scale(x, lane, &inv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) codes[e] = q4_code(x[e], inv);
+      }
+      // lanes cl = 0,1 share bytes (lo, hi nibble) with y%2 = 0; lanes 2,3 with y%2 = 1
+      int other[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) other[e] = __shfl_xor_sync(0xffffffffu, codes[e], 1);
+      if (st && (cl & 1) == 0) {
+        const int C = b >> 1, w = 2 * (b & 1) + wlo, y = 2 * ylo + (cl >> 1);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int off = ((((G * 4 + C) * 8 + e) * 4 + T) * 16) + 4 * w + y;
+          pg[off] = static_cast<uint8_t>(codes[e] | (other[e] << 4));
+        }
+      }
+      if (st && cl == 0) {
+        const int so = kV4ScaleOffset + 2 * (((G * 4 + T) * 8 + b) * 4 + k_slot);
+        *reinterpret_cast<__half*>(pg + so) = __float2half_rn(d);
+        if (v_fmt == kValQ41)
+          *reinterpret_cast<__half*>(pg + so + (kV41MinOffset - kV4ScaleOffset)) = __float2half_rn(mn);
+      }
+    } else {
+      float inv;
+      d = q8_scale(x, &inv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) codes[e] = q8_code(x[e], inv);
+      const int w = 2 * (cl >> 1) + wlo, y = 2 * (cl & 1) + ylo;
+      if (st) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int off = ((((G * 8 + b) * 8 + e) * 4 + T) * 16) + 4 * w + y;
+          pg[off] = static_cast<uint8_t>(codes[e] & 0xFF);
+        }
+      }
+      if (st && cl == 0) {
+        const int so = kV8ScaleOffset + 2 * (((G * 4 + T) * 8 + b) * 4 + k_slot);
+        *reinterpret_cast<__half*>(pg + so) = __float2half_rn(d);
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __restrict__ k,
                                                               const float* __restrict__ v, int n_tok,
                                                               int n_kv, int32_t pos0,
@@ -139,134 +279,10 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const float* __res
     if (lane == 0) record_error(KVATTN_ERR_BAD_PAGE);
     return;
   }
-  const int G = tok >> 4, tl = tok & 15, H = tl >> 3, R = tok & 7;
-  const int b = lane >> 2;  // this lane's block
-
-  // ---------------- K: Q5_1 / Q5_0 ----------------
-  if (k_fmt == kKeyQ51 || k_fmt == kKeyQ50) {
-    const float x[8] = {kx0.x, kx0.y, kx0.z, kx0.w, kx1.x, kx1.y, kx1.z, kx1.w};
-    float mn = 0.f, inv, d;
-    if (k_fmt == kKeyQ51) {
-      d = min_scale<31>(x, &mn, &inv);
-    } else {
-      d = offset_scale<16>(x, lane, &inv);
-    }
-    const int T = lane & 3, c = b & 3, Q = b >> 2;
-    // low nibbles as the Q4_0 key word; fifth bits of the four blocks 4Q..4Q+3 of this T
-    // (lanes T + 4c + 16Q) gathered into one word, channel (c, e) at bit 16(e%2) + 4c + e/2
-    uint32_t w = 0, hb = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const uint32_t q = static_cast<uint32_t>(k_fmt == kKeyQ51 ? min_code<31>(x[e], mn, inv)
-                                                                : offset_code<16>(x[e], inv));
-      w |= (q & 15u) << (4 * (e >> 1) + 16 * (e & 1));
-      hb |= (q >> 4) << (16 * (e & 1) + 4 * c + (e >> 1));
-    }
-    hb |= __shfl_xor_sync(0xffffffffu, hb, 4);
-    hb |= __shfl_xor_sync(0xffffffffu, hb, 8);
-    uint8_t* pg = k_pool + static_cast<int64_t>(page) * k_stride;
-    const int row = (((G * 2 + Q) * 2 + H) * 8 + R) * 4 + T;
-    *reinterpret_cast<uint32_t*>(pg + 4 * (row * 4 + c)) = w;
-    if (c == 0) *reinterpret_cast<uint32_t*>(pg + kK5HighOffset + 4 * row) = hb;
-    if ((lane & 3) == 0) {
-      const int si = 2 * (((G * 8 + R) * 2 + H) * 8 + b);
-      *reinterpret_cast<__half*>(pg + kK5ScaleOffset + si) = __float2half_rn(d);
-      if (k_fmt == kKeyQ51) *reinterpret_cast<__half*>(pg + kK5MinOffset + si) = __float2half_rn(mn);
-    }
-  }
-  // ---------------- K: Q4_0 ----------------
-  else if (k_fmt == kKeyQ4) {
-    const float x[8] = {kx0.x, kx0.y, kx0.z, kx0.w, kx1.x, kx1.y, kx1.z, kx1.w};
-    float inv;
-    const float d = q4_scale(x, lane, &inv);
-    // one 32-bit word per lane: channel 8T + e at bit 4 * (e / 2) + 16 * (e % 2)
-    uint32_t w = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) w |= static_cast<uint32_t>(q4_code(x[e], inv)) << (4 * (e >> 1) + 16 * (e & 1));
-    uint8_t* pg = k_pool + static_cast<int64_t>(page) * k_stride;
-    const int T = lane & 3;
-    const int word = ((((G * 2 + (b >> 2)) * 2 + H) * 8 + R) * 4 + T) * 4 + (b & 3);
-    *reinterpret_cast<uint32_t*>(pg + 4 * word) = w;
-    if ((lane & 3) == 0) {
-      const int so = kK4ScaleOffset + 2 * (((G * 8 + R) * 2 + H) * 8 + b);
-      *reinterpret_cast<__half*>(pg + so) = __float2half_rn(d);
-    }
-  }
-  // ---------------- K: Q8_0 ----------------
-  else {
-    const float x[8] = {kx0.x, kx0.y, kx0.z, kx0.w, kx1.x, kx1.y, kx1.z, kx1.w};
-    float inv;
-    const float d = q8_scale(x, &inv);
-    uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) w0 |= (static_cast<uint32_t>(q8_code(x[e], inv)) & 0xFFu) << (8 * e);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) w1 |= (static_cast<uint32_t>(q8_code(x[4 + e], inv)) & 0xFFu) << (8 * e);
-    uint8_t* pg = k_pool + static_cast<int64_t>(page) * k_stride;
-    const int P = lane >> 3, T = lane & 3, jhi = (lane & 7) >> 2;
-    const int off = ((((G * 4 + P) * 2 + H) * 8 + R) * 4 + T) * 16 + 8 * jhi;
-    *reinterpret_cast<uint2*>(pg + off) = make_uint2(w0, w1);
-    if ((lane & 3) == 0) {
-      const int so = kKScaleOffset + 2 * (((G * 8 + R) * 2 + H) * 8 + b);
-      *reinterpret_cast<__half*>(pg + so) = __float2half_rn(d);
-    }
-  }
-
-  // ---------------- V: Q4_0, Q4_1 or Q8_0 ----------------
-  {
-    const float x[8] = {vx0.x, vx0.y, vx0.z, vx0.w, vx1.x, vx1.y, vx1.z, vx1.w};
-    uint8_t* pg = v_pool + static_cast<int64_t>(page) * v_stride;
-    const int T = (tl & 7) >> 1, wlo = tl >> 3, ylo = tl & 1;
-    const int k_slot = ylo + 2 * wlo;
-    const int cl = lane & 3;  // which 8-channel group of the block
-    float d;
-    int codes[8];
-    if (v_fmt != kValQ8) {
-      float inv, mn = 0.f;
-      if (v_fmt == kValQ41) {
-        d = min_scale<15>(x, &mn, &inv);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) codes[e] = min_code<15>(x[e], mn, inv);
-      } else {
-        d = q4_scale(x, lane, &inv);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) codes[e] = q4_code(x[e], inv);
-      }
-      // lanes cl = 0,1 share bytes (lo, hi nibble) with y%2 = 0; lanes 2,3 with y%2 = 1
-      int other[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) other[e] = __shfl_xor_sync(0xffffffffu, codes[e], 1);
-      if ((cl & 1) == 0) {
-        const int C = b >> 1, w = 2 * (b & 1) + wlo, y = 2 * ylo + (cl >> 1);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int off = ((((G * 4 + C) * 8 + e) * 4 + T) * 16) + 4 * w + y;
-          pg[off] = static_cast<uint8_t>(codes[e] | (other[e] << 4));
-        }
-      }
-      if (cl == 0) {
-        const int so = kV4ScaleOffset + 2 * (((G * 4 + T) * 8 + b) * 4 + k_slot);
-        *reinterpret_cast<__half*>(pg + so) = __float2half_rn(d);
-        if (v_fmt == kValQ41)
-          *reinterpret_cast<__half*>(pg + so + (kV41MinOffset - kV4ScaleOffset)) = __float2half_rn(mn);
-      }
-    } else {
-      float inv;
-      d = q8_scale(x, &inv);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) codes[e] = q8_code(x[e], inv);
-      const int w = 2 * (cl >> 1) + wlo, y = 2 * (cl & 1) + ylo;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int off = ((((G * 8 + b) * 8 + e) * 4 + T) * 16) + 4 * w + y;
-        pg[off] = static_cast<uint8_t>(codes[e] & 0xFF);
-      }
-      if (cl == 0) {
-        const int so = kV8ScaleOffset + 2 * (((G * 4 + T) * 8 + b) * 4 + k_slot);
-        *reinterpret_cast<__half*>(pg + so) = __float2half_rn(d);
-      }
-    }
-  }
+  const float kx[8] = {kx0.x, kx0.y, kx0.z, kx0.w, kx1.x, kx1.y, kx1.z, kx1.w};
+  const float vx[8] = {vx0.x, vx0.y, vx0.z, vx0.w, vx1.x, vx1.y, vx1.z, vx1.w};
+  encode_token(kx, vx, lane, k_pool + static_cast<int64_t>(page) * k_stride, v_pool + static_cast<int64_t>(page) * v_stride,
+               tok, k_fmt, v_fmt, 0xffffffffu);
 }
 
 cudaError_t launch_quantize_append(const kvattn_kv_desc& desc, const float* k, const float* v, int n_tok,

@@ -63,6 +63,9 @@ _SIGS = {
     "kvattn_decode_workspace_size": (c_size_t, [POINTER(kvattn_kv_desc), c_int, c_int]),
     "kvattn_decode": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                               c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "kvattn_append_decode": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_void_p, c_int, c_int32, c_void_p, c_int,
+                                     c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_void_p,
+                                     c_void_p, c_void_p, c_size_t, c_void_p]),
     "kvattn_decode_splits": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_int, c_void_p, c_void_p, c_void_p,
                                      c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "kvattn_decode_merge_splits": (c_int, [POINTER(kvattn_kv_desc), c_int, c_int, c_void_p, c_void_p, c_void_p,
@@ -196,6 +199,14 @@ def kvattn_decode(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pag
     _check(lib().kvattn_decode(ctypes.byref(desc), _d(q), n_q, _d(q_pos), _d(page_list), _d(page_logical),
                                _d(n_pages), max_pages, _d(out), _d(lse), _d(ws), ws_bytes, _s(stream)),
            "kvattn_decode")
+
+
+def kvattn_append_decode(desc, k_new, v_new, n_new, pos0, page_table, n_blocks, q, n_q, q_pos, page_list,
+                         page_logical, n_pages, max_pages, out, lse, ws, ws_bytes, stream=None) -> None:
+    """kvattn_quantize_append of n_new tokens and kvattn_decode in one grid."""
+    _check(lib().kvattn_append_decode(ctypes.byref(desc), _d(k_new), _d(v_new), n_new, pos0, _d(page_table), n_blocks,
+                                      _d(q), n_q, _d(q_pos), _d(page_list), _d(page_logical), _d(n_pages), max_pages,
+                                      _d(out), _d(lse), _d(ws), ws_bytes, _s(stream)), "kvattn_append_decode")
 
 
 def kvattn_decode_splits(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pages, out, lse, ws, ws_bytes,

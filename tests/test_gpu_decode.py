@@ -84,6 +84,71 @@ def test_split_and_merge_calls_equal_decode(kv_gpu, n_q):
     assert np.array_equal(o2.cpu().numpy(), out) and np.array_equal(l2.cpu().numpy(), lse)
 
 
+@pytest.mark.parametrize("k_fmt,v_fmt", FORMAT_PAIRS)
+@pytest.mark.parametrize("n_new,subset", [(1, False), (4, False), (4, True)])
+def test_append_decode_equals_append_then_decode(kv_gpu, k_fmt, v_fmt, n_new, subset):
+    """kvattn_append_decode against kvattn_quantize_append + kvattn_decode on a copy of the same
+    cache: bit-identical outputs and pages.  Four new tokens straddle a page boundary; with
+    `subset` the decode lists only some of the older pages, so the new tokens' pages are written
+    but not attended."""
+    H, H_q, T0 = 4, 24, 20 * 128 + 126
+    rng, k, v, cache = _layer(660 + n_new, H, T0 + n_new, v_fmt, spare=3, k_fmt=k_fmt)
+    cache.append(k[:T0], v[:T0], 0)
+    kp2, vp2 = cache.k_pool.clone(), cache.v_pool.clone()
+    desc2 = kv_gpu.make_desc(H, H_q, kp2, vp2, cache.n_phys, v_fmt=v_fmt, k_fmt=k_fmt)
+    nb = cache.n_blocks
+    k_new = torch.from_numpy(np.ascontiguousarray(k[T0:])).cuda()
+    v_new = torch.from_numpy(np.ascontiguousarray(v[T0:])).cuda()
+    q = torch.from_numpy(normal_f32(rng, (n_new, H_q, 256))).cuda()
+    qp = torch.arange(T0, T0 + n_new, dtype=torch.int32, device="cuda")
+    if subset:
+        blocks = np.sort(rng.choice(nb - 2, 9, replace=False))
+        pl = torch.from_numpy(np.ascontiguousarray(cache.page_table_np[:, blocks])).cuda()
+        lg = torch.from_numpy(np.tile(blocks.astype(np.int32), (H, 1))).cuda()
+    else:
+        pl, lg = cache.page_table, None
+    mp = pl.shape[1]
+    wsb = kv_gpu.kvattn_decode_workspace_size(cache.desc, n_new, mp)
+    outs = []
+    for fused, desc in ((False, cache.desc), (True, desc2)):
+        ws = torch.zeros(max(wsb, 256), dtype=torch.uint8, device="cuda")
+        out = torch.full((n_new, H_q, 256), float("nan"), device="cuda")
+        lse = torch.full((n_new, H_q), float("nan"), device="cuda")
+        if fused:
+            kv_gpu.kvattn_append_decode(desc, k_new, v_new, n_new, T0, cache.page_table, nb, q, n_new, qp, pl, lg,
+                                        None, mp, out, lse, ws, wsb)
+        else:
+            kv_gpu.kvattn_quantize_append(desc, k_new, v_new, n_new, T0, cache.page_table, nb)
+            kv_gpu.kvattn_decode(desc, q, n_new, qp, pl, lg, None, mp, out, lse, ws, wsb)
+        torch.cuda.synchronize()
+        outs.append((out.cpu().numpy(), lse.cpu().numpy()))
+    assert kv_gpu.kvattn_device_error() == 0
+    assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+    assert torch.equal(cache.k_pool, kp2) and torch.equal(cache.v_pool, vp2)
+    if not subset:
+        oc = OracleCache(k, v, v_fmt, k_fmt)
+        qn = q.cpu().numpy()
+        for h in range(H):
+            o_ref, l_ref = oc.attend(qn, list(range(T0, T0 + n_new)), h, 6)
+            compare(outs[1][0][:, 6 * h:6 * h + 6], outs[1][1][:, 6 * h:6 * h + 6], o_ref, l_ref)
+
+
+def test_append_decode_rejects_bad_arguments(kv_gpu):
+    rng, k, v, cache = _layer(670, 1, 300, "q4_0", n_blocks=3)
+    x = torch.zeros((1, 1, 256), device="cuda")
+    q = torch.zeros((1, 6, 256), device="cuda")
+    qp = torch.tensor([300], dtype=torch.int32, device="cuda")
+    out = torch.empty((1, 6, 256), device="cuda")
+    lse = torch.empty((1, 6), device="cuda")
+    wsb = kv_gpu.kvattn_decode_workspace_size(cache.desc, 1, 3)
+    ws = torch.zeros(max(wsb, 256), dtype=torch.uint8, device="cuda")
+    for n_new, pos0 in ((0, 300), (9, 300), (1, 3 * 128)):   # none, too many, past the table
+        with pytest.raises(kv_gpu.KVAttnError) as e:
+            kv_gpu.kvattn_append_decode(cache.desc, x, x, n_new, pos0, cache.page_table, 3, q, 1, qp,
+                                        cache.page_table, None, None, 3, out, lse, ws, wsb)
+        assert e.value.status == kv_gpu.ERR_INVALID_ARG
+
+
 def test_tiny_workload(kv_gpu):
     # 1 layer, 1 KV head, 6 query heads, 4,096 tokens in 32 shuffled pages, 1 query token
     rng, k, v, cache = _layer(1001, 1, 4096, "q4_0", outliers=False)
