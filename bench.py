@@ -494,8 +494,11 @@ class StreamBench:
         self.tail_hosts_k = self.tail_hosts.permute(0, 2, 1).contiguous()
         self.tail_slots_k = self.tail_slots.permute(0, 2, 1).contiguous()
         self.reset()
+        # the page copy runs on gather_ctas SMs beside the decode: the decode grid leaves them free
+        self.gather_ctas = 16
+        sms = torch.cuda.get_device_properties(device).multi_processor_count
         self.desc = kv.make_desc(H, Hq, self.slots, self.slots.data_ptr() + 34816, self.n_slots, k_page_stride=P,
-                                 v_page_stride=P)
+                                 v_page_stride=P, sm_budget=sms - self.gather_ctas)
         # per buffer: gather destinations (-1 for the generated-token entries) and the decode page lists
         self.dst = []
         self.plist = []
@@ -539,7 +542,6 @@ class StreamBench:
         self.ev_dec = [torch.cuda.Event() for _ in range(L)]
         self.copy_bytes_per_step = L * H * self.budget * P
         self.launches_per_step = 6 * L  # scores, top-k, copy, decode with the append (+ merge), write-back
-        self.gather_ctas = 16
 
     def reset(self):
         """Back to the first step of the generation: the generated-token pages hold the prompt's
@@ -651,8 +653,9 @@ class ResidentStreamBench(StreamBench):
             for h in range(H):
                 self.slots[self.n_res + l * H + h].copy_(self.host[(l * H + h) * self.nb + self.n_full])
         self.n_slots = self.slots.shape[0]
+        sms = torch.cuda.get_device_properties(device).multi_processor_count
         self.desc = kv.make_desc(H, w.q_heads, self.slots, self.slots.data_ptr() + 34816, self.n_slots,
-                                 k_page_stride=P, v_page_stride=P)
+                                 k_page_stride=P, v_page_stride=P, sm_budget=sms - self.gather_ctas)
         self.tail_slot = torch.tensor([[self.n_res + l * H + h for h in range(H)] for l in range(L)],
                                       dtype=torch.int32, device=device)
         self.tail_tab = self.tail_slot[:, :, None].expand(L, H, self.nb).contiguous()

@@ -124,6 +124,12 @@ typedef struct kvattn_kv_desc {
   int64_t k_page_stride;  /* bytes between consecutive K pages (>= K page bytes, %16==0) */
   int64_t v_page_stride;  /* bytes between consecutive V pages (>= V page bytes, %16==0) */
   int64_t n_pages;        /* physical pages addressable in both pools                   */
+  int32_t sm_budget;      /* 0: decode and prefill grids are sized to every SM; n > 0:   */
+                          /* at most n SMs' worth of CTAs (fewer KV splits), leaving the */
+                          /* other SMs to kernels that run at the same time on another   */
+                          /* stream, e.g. the page copy of the streamed working set.     */
+                          /* Workspace sizes follow the same plan.  Must be >= 0.        */
+  int32_t reserved;       /* must be 0                                                  */
 } kvattn_kv_desc;
 
 /* ---- setup and status ------------------------------------------------------------- */
@@ -253,7 +259,7 @@ KVATTN_API int kvattn_merge_lse(const float* o_parts, const float* lse_parts, in
 /* ---- KVMem block summaries and selection ([KVMEM]) ---------------------------------
  * Summary of a full 128-token block = mean dequantized key per channel, rounded once to
  * fp32 (the per-block sum is exact in fp64 for scales within 2^28 of each other).  Keys may
- * be Q8_0, Q4_0 or Q5_1.
+ * be Q8_0, Q4_0, Q5_1 or Q5_0.
  *   page_table  device int32 [n_units][n_blocks] (a unit is one (layer, KV head))
  *   summaries   device fp32 [n_units][n_blocks][256]; blocks [block_begin, block_end) of
  *               every unit are written, others untouched. */
@@ -271,7 +277,13 @@ KVATTN_API int kvattn_block_summaries(const kvattn_kv_desc* desc, const int32_t*
  *   sel_logical device int32 [n_units][cap], sel_phys device int32 [n_units][cap],
  *   n_sel       device int32 [n_units]; cap >= min(budget, candidates) + recent + tail.
  *   ws          device workspace of kvattn_select_workspace_size(n_units, n_blocks) bytes.
- * Candidates per unit <= 16384. */
+ * Candidates per unit <= 16384.
+ * Scores are fp64 sums of the 256 x group products, accumulated by fused multiply-adds in a
+ * fixed order; a correctly rounded sum can differ from them by at most about
+ * 256 x group x 2^-53 x sum|products|.  The ids therefore equal those of an exact ranking
+ * wherever the gap between the budget-th and the next candidate's score is larger than that
+ * (the tests take 1e-9 of the largest score as the margin and check it per seed); blocks
+ * closer than that may be ordered either way. */
 KVATTN_API size_t kvattn_select_workspace_size(int n_units, int n_blocks);
 KVATTN_API int kvattn_select_blocks(const float* summaries, const float* q_group, int n_units,
                                     int group, int n_blocks, int n_full, int n_total, int budget,

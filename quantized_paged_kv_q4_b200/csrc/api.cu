@@ -96,6 +96,12 @@ int sm_count_for_planning() {
   return 148;
 }
 
+// The SMs a grid planned for this cache may take: every SM, or the descriptor's budget.
+int sm_budget_of(const kvattn_kv_desc* d) {
+  const int sms = sm_count_for_planning();
+  return d->sm_budget > 0 && d->sm_budget < sms ? d->sm_budget : sms;
+}
+
 int64_t page_bytes_of(int role, int fmt) {
   if (role == KVATTN_ROLE_K && fmt == KVATTN_FMT_Q8_0) return kKPageBytes;
   if (role == KVATTN_ROLE_K && fmt == KVATTN_FMT_Q4_0) return kK4PageBytes;
@@ -119,6 +125,7 @@ int validate_desc(const kvattn_kv_desc* d) {
   if (d->k_page_stride < kb || d->v_page_stride < vb || (d->k_page_stride & 15) || (d->v_page_stride & 15))
     return KVATTN_ERR_INVALID_ARG;
   if (d->n_pages < 1 || d->n_pages > (int64_t{1} << 31) - 1) return KVATTN_ERR_INVALID_ARG;
+  if (d->sm_budget < 0 || d->reserved != 0) return KVATTN_ERR_INVALID_ARG;
   return KVATTN_OK;
 }
 
@@ -133,7 +140,7 @@ DecodePlan plan_decode(const kvattn_kv_desc* d, int n_q, int max_pages) {
   DecodePlan p{};
   const int group = d->n_q_heads / d->n_kv_heads;
   p.rows_pad = ((group * n_q + 7) / 8) * 8;
-  const int sms = sm_count_for_planning();
+  const int sms = sm_budget_of(d);
   int s = sms / d->n_kv_heads;
   if (s < 1) s = 1;
   if (s > max_pages) s = max_pages < 1 ? 1 : max_pages;
@@ -575,7 +582,7 @@ KVATTN_API size_t kvattn_prefill_workspace_size(const kvattn_kv_desc* desc, int 
       kv_split_tokens % kPageTokens || kv_split_tokens > 65536)
     return 0;
   return plan_prefill(desc->n_kv_heads, desc->n_q_heads / desc->n_kv_heads, n_q, max_pages, kv_split_tokens,
-                      sm_count_for_planning())
+                      sm_budget_of(desc))
       .bytes;
 }
 
@@ -597,7 +604,7 @@ KVATTN_API int kvattn_prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* 
   const long long rows = static_cast<long long>(n_q) * group;
   if (rows > (1ll << 24)) return KVATTN_ERR_UNSUPPORTED_SHAPE;
   const PrefillPlan plan =
-      plan_prefill(desc->n_kv_heads, group, n_q, max_pages, kv_split_tokens, sm_count_for_planning());
+      plan_prefill(desc->n_kv_heads, group, n_q, max_pages, kv_split_tokens, sm_budget_of(desc));
   if (plan.n_ks > 65535 || plan.n_mt > (1 << 30)) return KVATTN_ERR_UNSUPPORTED_SHAPE;
   if (plan.bytes) {
     if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return KVATTN_ERR_INVALID_ARG;

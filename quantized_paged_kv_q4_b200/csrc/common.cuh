@@ -110,6 +110,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// Waits until a shared-memory word written by another warp equals `want`; gives up after
+// kWaitTimeoutNs, records KVATTN_ERR_TIMEOUT and returns false.
+__device__ __forceinline__ bool wait_tag(const int* tag, int want) {
+  const volatile int* v = tag;
+  if (*v == want) return true;
+  const unsigned long long t0 = global_timer_ns();
+  while (*v != want) {
+    if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      record_error(KVATTN_ERR_TIMEOUT);
+      return false;
+    }
+    __nanosleep(64);
+  }
+  return true;
+}
+
 // One contiguous global -> shared bulk copy (TMA engine), completion counted on `bar`.
 // dst, src and bytes must be multiples of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

@@ -28,22 +28,29 @@
 // of kvattn_merge_lse.
 #include "decode.cuh"
 
+#ifndef KVATTN_DECODE_WARPS1
+#define KVATTN_DECODE_WARPS1 12  // consumer warps of the unsplit (8-row) shape
+#endif
+
 namespace kvattn {
 
 
 template <int KF, int VF, int NT, int SPLIT>
 struct DecodeCfg {
   // SPLIT warps share each 16-token tile, each taking 8 / SPLIT of the 32-channel blocks, and
-  // add their partial scores through shared memory; a group of SPLIT warps walks SPLIT tiles
-  // of every page.  The 8-row shape runs unsplit tiles (SPLIT = 1); the 16- and 24-row shapes
-  // split them in two, which halves the accumulators per warp.  (Sixteen warps in the split
-  // arrangement measured slower for 8 rows: the duplicated softmax and the exchange cost more
-  // instructions than the extra warps hid.)
-  static constexpr int kConsumerWarps = 8;
+  // add their partial scores through shared memory.  The groups of SPLIT warps take the
+  // 16-token tiles of the CTA's pages round robin (tile j = 8 x page + tile in page goes to
+  // group j mod kGroups).  The 8-row shape runs unsplit tiles (SPLIT = 1) on twelve warps,
+  // three per scheduler, with the query fragments in shared memory so that a thread needs
+  // at most 168 registers; the 16- and 24-row shapes split the tiles in two, which halves the
+  // accumulators per warp.  (Sixteen warps in the split arrangement measured slower for 8
+  // rows: the duplicated softmax and the exchange cost more instructions than the extra
+  // warps hid.)
+  static constexpr int kConsumerWarps = SPLIT == 1 ? KVATTN_DECODE_WARPS1 : 8;
   static constexpr int kThreads = kConsumerWarps * 32;  // lanes of warp 0 also issue the copies
   static constexpr int kNB = 8 / SPLIT;                 // 32-channel blocks per warp
   static constexpr int kGroups = kConsumerWarps / SPLIT;  // warp groups, one softmax stream each
-  static constexpr int kTilesPerWarp = 8 / kGroups;
+  static constexpr int kReleases = 8 * SPLIT;             // (warp, tile) pairs per page
   static constexpr bool kK5 = KF == kKeyQ51 || KF == kKeyQ50;  // 5-bit key codes
   static constexpr bool kKMin = KF == kKeyQ51;                 // keys with a zero point
   static constexpr bool kVMin = VF == kValQ41;                 // values with a zero point
@@ -55,7 +62,7 @@ struct DecodeCfg {
   static constexpr int kStageBytes = kKBytes + kVBytes;
   // split tiles keep the query B fragments in shared memory:
   // [block][k-step][n-tile][lane][hi0, hi1, lo0, lo1]
-  static constexpr bool kQSmem = SPLIT > 1;
+  static constexpr bool kQSmem = SPLIT > 1 || kConsumerWarps > 8;
   static constexpr int kQBytes = kQSmem ? 8 * 2 * NT * 32 * 16 : 0;
   static constexpr int kUnits = kGroups;   // independent softmax streams per CTA
   static constexpr int kRowsPad = NT * 8;
@@ -74,6 +81,7 @@ struct DecodeCfg {
   static constexpr int kQOffset = kRingBytes + kXBytes;
   static constexpr int kBarOffset = kQOffset + kQBytes;
   static constexpr int kSmemBytes = kBarOffset + 256;
+  static_assert(8 * (kStages + kGroups) + 4 * (4 * kStages + 1) <= 256, "stage bookkeeping");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -104,16 +112,61 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uin
   lo = pack_half2(x0 - half_lo(hi), x1 - half_hi(hi));
 }
 
+// Encodes the appended tokens that fall in tokens [pos_lo, pos_lo + 16) of a page held in a
+// shared-memory stage (K bytes at `stage`, V bytes k_bytes further on) into that copy, for the
+// lanes of store_mask.  Kept out of line: it runs for one tile in thousands, and inlined it
+// would take registers from the tile loop.
+// Arguments are scalars: a reference to the kernel's parameter block would make every thread
+// copy that block to its stack.
+__device__ __noinline__ void patch_stage(const float* k_new, const float* v_new, int n_new, int new_pos0, int h,
+                                         int n_kv, int lane, uint8_t* stage, int k_bytes, int logical, int pos_lo,
+                                         int k_fmt, int v_fmt, uint32_t mask) {
+  for (int n = 0; n < n_new; ++n) {
+    const int pos = new_pos0 + n;
+    if (pos < pos_lo || pos >= pos_lo + 16) continue;
+    const long long row = (static_cast<long long>(n) * n_kv + h) * kHeadDim;
+    const float4* ks = reinterpret_cast<const float4*>(k_new + row + lane * 8);
+    const float4* vs = reinterpret_cast<const float4*>(v_new + row + lane * 8);
+    const float4 k0 = ks[0], k1 = ks[1], v0 = vs[0], v1 = vs[1];
+    const float kx[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+    const float vx[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    encode_token(kx, vx, lane, stage, stage + k_bytes, pos - logical * kPageTokens, k_fmt, v_fmt, mask);
+    // the stage is later refilled by the copy engine (async proxy)
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+  }
+}
+
+// Encodes appended token n of KV head h into its page in global memory (one warp).
+__device__ __noinline__ void append_global(const float* k_new, const float* v_new, const int32_t* table,
+                                           int table_blocks, uint8_t* k_pool, uint8_t* v_pool, int64_t k_stride,
+                                           int64_t v_stride, int64_t n_pages, int pos, int h, int n_kv, int lane,
+                                           int n, int k_fmt, int v_fmt) {
+  const long long row = (static_cast<long long>(n) * n_kv + h) * kHeadDim;
+  const float4* ks = reinterpret_cast<const float4*>(k_new + row + lane * 8);
+  const float4* vs = reinterpret_cast<const float4*>(v_new + row + lane * 8);
+  const float4 k0 = ks[0], k1 = ks[1], v0 = vs[0], v1 = vs[1];
+  const int page = table[static_cast<long long>(h) * table_blocks + pos / kPageTokens];
+  if (page < 0 || page >= n_pages) {
+    if (lane == 0) record_error(KVATTN_ERR_BAD_PAGE);
+    return;
+  }
+  const float kx[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+  const float vx[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  encode_token(kx, vx, lane, k_pool + static_cast<int64_t>(page) * k_stride, v_pool + static_cast<int64_t>(page) * v_stride,
+               pos % kPageTokens, k_fmt, v_fmt, 0xffffffffu);
+}
+
 template <int KF, int VF, int NT, int SPLIT>
 __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) decode_kernel(const DecodeParams p) {
   using C = DecodeCfg<KF, VF, NT, SPLIT>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   uint64_t* xbar = full + C::kStages;   // [kGroups] score-exchange barriers (split tiles only)
-  int* rel_cnt = reinterpret_cast<int*>(xbar + C::kGroups);  // [kStages] warps done with the stage
-  int* s_issued = rel_cnt + C::kStages;              // pages issued so far
-  int* st_logical = s_issued + 1;
-  int* st_valid = st_logical + C::kStages;
+  int* rel_cnt = reinterpret_cast<int*>(xbar + C::kGroups);  // [kStages] (warp, tile) pairs done
+  int* st_page = rel_cnt + C::kStages;     // [kStages] the page last issued into the stage, -1: none
+  int* st_logical = st_page + C::kStages;  // [kStages]
+  int* st_valid = st_logical + C::kStages;  // [kStages]
   int* s_flags = st_valid + C::kStages;  // [0] abort
 
   // the LSE-merge grid that follows may start launching now; it waits for this grid's data
@@ -129,8 +182,8 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       rel_cnt[s] = 0;
+      st_page[s] = -1;
     }
-    *s_issued = 0;
     for (int i = 0; i < C::kGroups; ++i) mbar_init(&xbar[i], SPLIT);
     s_flags[0] = 0;
     fence_barrier_init();
@@ -178,16 +231,15 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
   const int blk0 = C::kNB * part;
 
   // Page copies: the first kStages pages are issued up front by lanes of warp 0; after
-  // that, the warp that is the last of the eight to finish with a stage refills it at
-  // once with the page kStages further on, so kStages - 1 pages stay in flight while one
-  // is being consumed.  Pages are issued in increasing order.
+  // that, the warp that finishes the last of a page's tiles refills its stage at once with
+  // the page kStages further on, so kStages - 1 pages stay in flight while one is being
+  // consumed.  Each stage carries the number of the page last issued into it.
   const int32_t* plist = p.page_list + static_cast<long long>(h) * p.max_pages;
   const int32_t* plog = p.page_logical ? p.page_logical + static_cast<long long>(h) * p.max_pages : nullptr;
-  auto issue = [&](int i) {
+  auto issue_page = [&](int i, int page, int logical) {
     const int s = i % C::kStages;
-    const int idx = first + i;
-    const int page = plist[idx];
-    st_logical[s] = plog ? plog[idx] : idx;
+    *reinterpret_cast<volatile int*>(&st_page[s]) = i;
+    st_logical[s] = logical;
     if (page < 0 || page >= p.n_pages) {
       record_error(KVATTN_ERR_BAD_PAGE);
       st_valid[s] = 0;
@@ -199,35 +251,29 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
       bulk_g2s(stage, p.k_pool + static_cast<int64_t>(page) * p.k_stride, C::kKBytes, &full[s]);
       bulk_g2s(stage + C::kKBytes, p.v_pool + static_cast<int64_t>(page) * p.v_stride, C::kVBytes, &full[s]);
     }
-    *reinterpret_cast<volatile int*>(s_issued) = i + 1;
   };
-  // the first stages are issued by parallel lanes: their page-table reads overlap
-  if (warp == 0) {
-    if (lane < C::kStages && lane < count) issue(lane);
-    __syncwarp();
-    if (lane == 0) *reinterpret_cast<volatile int*>(s_issued) = count < C::kStages ? count : C::kStages;
+  auto issue = [&](int i) {
+    const int idx = first + i;
+    issue_page(i, plist[idx], plog ? plog[idx] : idx);
+  };
+  // The first stages: lanes of warp 0 read their page ids in parallel; lane 0 issues the first
+  // page before the others issue theirs, so that of all the CTAs' first requests, which reach
+  // the memory system together, each CTA's first page comes first and its warps can start.
+  if (warp == 0 && lane < C::kStages && lane < count) {
+    const int idx = first + lane;
+    const int page = plist[idx];
+    const int logical = plog ? plog[idx] : idx;
+    if (lane == 0) issue_page(0, page, logical);
+    __syncwarp((1u << (count < C::kStages ? count : C::kStages)) - 1u);
+    if (lane > 0) issue_page(lane, page, logical);
   }
   // Appended tokens: split 0 of every head encodes them into their pages in global memory, one
   // warp per token (warps 1 ..).  A CTA that streams such a page encodes the token again into
   // its shared-memory copy before using it (below), so no CTA waits for another.
-  if (p.n_new > 0 && split == 0 && warp >= 1 && warp <= p.n_new) {
-    const int i = warp - 1;
-    const int pos = p.new_pos0 + i;
-    const long long row = (static_cast<long long>(i) * gridDim.y + h) * kHeadDim;
-    const float4* ks = reinterpret_cast<const float4*>(p.k_new + row + lane * 8);
-    const float4* vs = reinterpret_cast<const float4*>(p.v_new + row + lane * 8);
-    const float4 k0 = ks[0], k1 = ks[1], v0 = vs[0], v1 = vs[1];
-    const int page = p.new_table[static_cast<long long>(h) * p.new_blocks + pos / kPageTokens];
-    if (page < 0 || page >= p.n_pages) {
-      if (lane == 0) record_error(KVATTN_ERR_BAD_PAGE);
-    } else {
-      const float kx[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-      const float vx[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      encode_token(kx, vx, lane, const_cast<uint8_t*>(p.k_pool) + static_cast<int64_t>(page) * p.k_stride,
-                   const_cast<uint8_t*>(p.v_pool) + static_cast<int64_t>(page) * p.v_stride, pos % kPageTokens, KF,
-                   VF, 0xffffffffu);
-    }
-  }
+  if (p.n_new > 0 && split == 0 && warp >= 1 && warp <= p.n_new)
+    append_global(p.k_new, p.v_new, p.new_table, p.new_blocks, const_cast<uint8_t*>(p.k_pool),
+                  const_cast<uint8_t*>(p.v_pool), p.k_stride, p.v_stride, p.n_pages, p.new_pos0 + warp - 1, h,
+                  gridDim.y, lane, warp - 1, KF, VF);
 
   {
     // ------------------------------------------------------------------ consumers
@@ -356,10 +402,20 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
       }
     };
 
-    for (int i = 0; i < count; ++i) {
+    // Tiles in increasing order, group grp taking j = grp, grp + kGroups, ...: page i = j / 8,
+    // tile G = j % 8.  With more groups than tiles per page a group skips pages, so the parity
+    // of a stage's barrier alone cannot tell page i from page i - kStages.  A group therefore
+    // first waits until the stage's tag names page i (issued only after every tile of page
+    // i - kStages is done, so that page's phase has completed), then for the barrier phase of
+    // page i (which cannot move on before this group's tile of page i is done).
+    const int new_lo = p.new_pos0, new_hi = p.new_pos0 + p.n_new;  // appended positions
+    const int n_tiles = 8 * count;
+    for (int j = grp; j < n_tiles; j += C::kGroups) {
+      const int i = j >> 3;
+      const int G = j & 7;
       const int s = i % C::kStages;
       const uint32_t par = (i / C::kStages) & 1;
-      if (!mbar_wait(&full[s], par)) {
+      if (!wait_tag(&st_page[s], i) || !mbar_wait(&full[s], par)) {
         s_flags[0] = 1;
         break;
       }
@@ -368,31 +424,16 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
         const uint32_t vb = kb + C::kKBytes;
         const int logical = st_logical[s];
         const bool need_mask = static_cast<long long>(logical) * kPageTokens + (kPageTokens - 1) > qpos_min;
-#pragma unroll
-        for (int tt = 0; tt < C::kTilesPerWarp; ++tt) {
-          const int G = SPLIT > 1 ? (C::kTilesPerWarp * grp + tt) : warp;
-          if (p.n_new > 0) {
+        {
+          const int pos_lo = logical * kPageTokens + 16 * G;
+          if (pos_lo < new_hi && pos_lo + 16 > new_lo) {
             // an appended token in this tile: encode it into the stage (this warp's channel
-            // blocks), as split 0 encodes it into the page in global memory
-            const int pos_lo = logical * kPageTokens + 16 * G;
-#pragma unroll 1
-            for (int i = 0; i < p.n_new; ++i) {
-              const int pos = p.new_pos0 + i;
-              if (pos < pos_lo || pos >= pos_lo + 16) continue;
-              const long long row = (static_cast<long long>(i) * gridDim.y + h) * kHeadDim;
-              const float4* ks = reinterpret_cast<const float4*>(p.k_new + row + lane * 8);
-              const float4* vs = reinterpret_cast<const float4*>(p.v_new + row + lane * 8);
-              const float4 k0 = ks[0], k1 = ks[1], v0 = vs[0], v1 = vs[1];
-              const float kx[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-              const float vx[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-              constexpr int kLanes = 32 / SPLIT;  // lanes 4b .. 4b + 3 hold block b
-              const uint32_t mask = SPLIT == 1 ? 0xffffffffu : (((1u << kLanes) - 1u) << (kLanes * part));
-              uint8_t* stage = smem + s * C::kStageBytes;
-              encode_token(kx, vx, lane, stage, stage + C::kKBytes, pos - logical * kPageTokens, KF, VF, mask);
-              // the stage is later refilled by the copy engine (async proxy)
-              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-              __syncwarp();
-            }
+            // blocks; lanes 4b .. 4b + 3 hold block b), as split 0 encodes it into the page in
+            // global memory
+            constexpr int kLanes = 32 / SPLIT;
+            const uint32_t mask = SPLIT == 1 ? 0xffffffffu : (((1u << kLanes) - 1u) << (kLanes * part));
+            patch_stage(p.k_new, p.v_new, p.n_new, p.new_pos0, h, gridDim.y, lane, smem + s * C::kStageBytes,
+                        C::kKBytes, logical, pos_lo, KF, VF, mask);
           }
           // ---------------- S = K Q^T over this warp's channel blocks ----------------
           // Key codes enter the MMA exactly (integers in f16).  Each 32-channel block is
@@ -748,7 +789,7 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
       if (aborted) break;
       __syncwarp();
       if (lane == 0) {
-        if (atomicAdd(&rel_cnt[s], 1) == C::kConsumerWarps - 1) {
+        if (atomicAdd(&rel_cnt[s], 1) == C::kReleases - 1) {
           rel_cnt[s] = 0;
           if (i + C::kStages < count) issue(i + C::kStages);
         }
@@ -771,10 +812,11 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
   if (s_flags[0]) {
     // A bounded wait expired: wait (bounded) for the copies still in flight, then leave.
     if (threadIdx.x == 0) {
-      const int next = *reinterpret_cast<volatile int*>(s_issued);
-      for (int pg = next - C::kStages < 0 ? 0 : next - C::kStages; pg < next; ++pg) {
+      for (int s = 0; s < C::kStages; ++s) {
+        const int pg = *reinterpret_cast<volatile int*>(&st_page[s]);
+        if (pg < 0) continue;
         const unsigned long long t0 = global_timer_ns();
-        while (!mbar_try_wait(&full[pg % C::kStages], (pg / C::kStages) & 1)) {
+        while (!mbar_try_wait(&full[s], (pg / C::kStages) & 1)) {
           if (global_timer_ns() - t0 > kWaitTimeoutNs) break;
         }
       }

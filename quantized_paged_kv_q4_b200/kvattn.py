@@ -49,6 +49,7 @@ class kvattn_kv_desc(ctypes.Structure):
         ("n_kv_heads", c_int32), ("n_q_heads", c_int32), ("head_dim", c_int32), ("page_tokens", c_int32),
         ("k_fmt", c_int32), ("v_fmt", c_int32), ("k_pool", c_void_p), ("v_pool", c_void_p),
         ("k_page_stride", c_int64), ("v_page_stride", c_int64), ("n_pages", c_int64),
+        ("sm_budget", c_int32), ("reserved", c_int32),
     ]
 
 
@@ -157,11 +158,11 @@ def status_string(status: int) -> str:
 
 
 def make_desc(n_kv_heads, n_q_heads, k_pool, v_pool, n_pages, v_fmt="q4_0", k_page_stride=None,
-              v_page_stride=None, head_dim=256, page_tokens=128, k_fmt="q8_0") -> kvattn_kv_desc:
+              v_page_stride=None, head_dim=256, page_tokens=128, k_fmt="q8_0", sm_budget=0) -> kvattn_kv_desc:
     kf, vf = FMT[k_fmt] if isinstance(k_fmt, str) else k_fmt, FMT[v_fmt] if isinstance(v_fmt, str) else v_fmt
     return kvattn_kv_desc(n_kv_heads, n_q_heads, head_dim, page_tokens, kf, vf, _d(k_pool), _d(v_pool),
                           k_page_stride or kvattn_page_bytes(ROLE_K, kf), v_page_stride or kvattn_page_bytes(ROLE_V, vf),
-                          n_pages)
+                          n_pages, sm_budget, 0)
 
 
 # ---------------------------------------------------------------- entry points

@@ -127,6 +127,22 @@ def test_decode_workspace_plan(lib):
         pytest.skip("workspace planned for a different SM count on this machine")
     assert kvattn.kvattn_decode_workspace_size(d, 1, 1) == 0       # one page: no split, no workspace
     assert kvattn.kvattn_decode_workspace_size(d, 4, 1024) > got
+    # an SM budget of 132 leaves 16 SMs free: 33 splits per KV head; a budget above the SM
+    # count plans for every SM
+    d.sm_budget = 132
+    want_b = ((4 * 33 * rows * 4 + 255) // 256) * 256 + 4 * 33 * rows * 256 * 4
+    assert kvattn.kvattn_decode_workspace_size(d, 1, 1024) == want_b
+    d.sm_budget = 1000
+    assert kvattn.kvattn_decode_workspace_size(d, 1, 1024) == got
+
+
+def test_descriptor_budget_fields_checked(lib):
+    L = lib
+    by = ctypes.byref
+    for field, value in (("sm_budget", -1), ("reserved", 1)):
+        d = _desc()
+        setattr(d, field, value)
+        assert L.kvattn_decode(by(d), 16, 1, 16, 16, None, None, 1, 16, 16, None, 0, None) == kvattn.ERR_INVALID_ARG
 
 
 def test_stream_plan_coalesces_runs(lib):
