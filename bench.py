@@ -65,7 +65,7 @@ def parse_args():
 
 # --------------------------------------------------------------------------- plumbing
 KERNEL_SOURCES = {
-    "decode_kernel_decode131k.md": ["common.cuh", "decode.cuh", "decode.cu"],
+    "decode_kernel_decode131k.md": ["common.cuh", "decode.cuh", "quantize.cu", "decode.cu"],
     "prefill_kernel_prefill65k.md": ["common.cuh", "tcgen05.cuh", "decode.cuh", "prefill.cu"],
 }
 
