@@ -28,7 +28,9 @@
  *
  * Data formats (fixed by this library; the pages fix only the bits per element):
  *  - head_dim = 256, page = 128 tokens of one (layer, KV head).
- *  - Q8_0: blocks of 32 int8 codes + one fp16 scale d; value = q * d.
+ *  - Q8_0: blocks of 32 codes q in [-127,127] + one fp16 scale d; value = q * d.  A code is
+ *    stored offset-binary, as the byte q + 128 (a zero byte, in a slot never written, is the
+ *    code -128 with the scale 0).
  *    Q4_0: blocks of 32 4-bit codes q in [0,15] + fp16 d; value = (q - 8) * d.
  *    Q5_1: blocks of 32 5-bit codes q in [0,31] + fp16 d + fp16 minimum m; value = q * d + m
  *    ([VULKAN] pitfalls: 6 bits per element, a zero point; paired with Q4_0 values).
@@ -40,7 +42,8 @@
  *    (18,432 B), Q8_0 (34,816 B) or Q4_1 (20,480 B).  Inside a
  *    page, codes come first and fp16 scales after them, both in tensor-core fragment order
  *    (tok = slot in page, c = channel, b = c/32, G = tok/16):
- *      K Q8_0 code  (tok = 16G+8H+R, c = 64P+32(j/8)+8T+j%8) at ((((G*4+P)*2+H)*8+R)*4+T)*16+j
+ *      K Q8_0 byte  q + 128 (tok = 16G+8H+R, c = 64P+32(j/8)+8T+j%8) at
+ *                   ((((G*4+P)*2+H)*8+R)*4+T)*16+j
  *      K Q4_0 word  (tok = 16G+8H+R, b = 4Q+c, channels 32b+8T+i, i < 8) is the little-endian
  *                   uint32 at 4*(((((G*2+Q)*2+H)*8+R)*4+T)*4+c); channel i's 4-bit code sits
  *                   at bit 4*(i/2) + 16*(i%2)
@@ -52,7 +55,7 @@
  *                   (Q4_0) or 20480 (Q5_1, Q5_0)
  *      V Q4_0 byte  ((((G*4+C)*8+R)*4+T)*16 + 4w + y: block b = 2C+w/2, token
  *                   16G+2T+8(w%2)+y/2; low nibble c = 32b+16(y%2)+R, high nibble c+8
- *      V Q8_0 code  (tok = 16G+2T+8(w%2)+y%2, c = 32b+16(w/2)+8(y/2)+R) at
+ *      V Q8_0 byte  q + 128 (tok = 16G+2T+8(w%2)+y%2, c = 32b+16(w/2)+8(y/2)+R) at
  *                   ((((G*8+b)*8+R)*4+T)*16 + 4w + y
  *      V Q4_1 byte  as the V Q4_0 byte (the code is q, not q - 8)
  *      V scale      d[16G+2T+k%2+8(k/2)][b] at S + 2*(((G*4+T)*8+b)*4+k), S = 16384 (Q4_0,

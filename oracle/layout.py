@@ -15,7 +15,10 @@ grouped in sixteens: G = tok // 16.
 K page, Q8_0 (34,816 bytes)
   codes, bytes [0, 32768): byte at
       ((((G*4 + P)*2 + H)*8 + R)*4 + T)*16 + j          (P<4, H<2, R<8, T<4, j<16)
-  holds the int8 code of token 16G + 8H + R, channel 64P + 32*(j // 8) + 8T + (j % 8).
+  holds the code q (in [-127, 127]) of token 16G + 8H + R, channel
+  64P + 32*(j // 8) + 8T + (j % 8), stored offset-binary as the byte q + 128 (the value of the
+  byte XOR 0x80 read as int8; a zero byte is the code -128, so an unwritten slot, whose
+  scale is zero too, holds the value 0).
   scales, bytes [32768, 34816): fp16 at 32768 + 2*((((G*8 + R)*2 + H)*8) + b)
   holds d[16G + 8H + R][b].
 
@@ -55,8 +58,8 @@ V page, Q4_1 (20,480 bytes)
 V page, Q8_0 (34,816 bytes)
   codes, bytes [0, 32768): byte at
       ((((G*8 + b)*8 + R)*4 + T)*16 + 4*w + y            (b<8, R<8, T<4, w<4, y<4)
-  holds the int8 code of token 16G + 2T + 8*(w % 2) + y % 2, channel
-  32b + 16*(w // 2) + 8*(y // 2) + R.
+  holds the code of token 16G + 2T + 8*(w % 2) + y % 2, channel
+  32b + 16*(w // 2) + 8*(y // 2) + R, offset-binary as for the K Q8_0 codes.
   scales, bytes [32768, 34816): same arrangement as the Q4_0 V scales.
 """
 from __future__ import annotations
@@ -173,6 +176,14 @@ def _flat_codes(codes: np.ndarray) -> np.ndarray:
     return np.asarray(codes).reshape(PAGE_TOKENS, HEAD_DIM)
 
 
+def _offset_binary(q: np.ndarray) -> np.ndarray:
+    """Q8_0 codes in [-128, 127] -> their stored bytes q + 128."""
+    q = np.asarray(q).astype(np.int16)
+    if np.any(q < -128) or np.any(q > 127):
+        raise ValueError("Q8_0 codes must be in [-128, 127]")
+    return (q + 128).astype(np.uint8)
+
+
 def encode_page(role: str, fmt: str, codes: np.ndarray, d: np.ndarray) -> np.ndarray:
     """Encode one page.  codes: [128][8][32] (int8 for Q8_0, 0..15 for Q4_0 / Q4_1, 0..31 for
     Q5_0 / Q5_1); d: [128][8] float16 ([128][8][2] (d, m) for Q4_1 and Q5_1).  Returns
@@ -218,7 +229,7 @@ def encode_page(role: str, fmt: str, codes: np.ndarray, d: np.ndarray) -> np.nda
         scale_base = 16384
     elif role == "k":
         off, tok, dim = _K_CODES
-        out[off] = c[tok, dim].astype(np.int8).view(np.uint8)
+        out[off] = _offset_binary(c[tok, dim])
         idx, tok, b = _K_SCALES
         scale_base = 32768
     elif fmt == "q4_0":
@@ -231,7 +242,7 @@ def encode_page(role: str, fmt: str, codes: np.ndarray, d: np.ndarray) -> np.nda
         scale_base = 16384
     else:
         off, tok, dim = _V8_CODES
-        out[off] = c[tok, dim].astype(np.int8).view(np.uint8)
+        out[off] = _offset_binary(c[tok, dim])
         idx, tok, b = _V_SCALES
         scale_base = 32768
     sv = d16[tok, b]
@@ -274,7 +285,7 @@ def decode_page(role: str, fmt: str, page: np.ndarray):
         scale_base = 16384
     elif role == "k":
         off, tok, dim = _K_CODES
-        c[tok, dim] = page[off].view(np.int8)
+        c[tok, dim] = page[off].astype(np.int16) - 128
         idx, tok, b = _K_SCALES
         scale_base = 32768
     elif fmt == "q4_0":
@@ -285,7 +296,7 @@ def decode_page(role: str, fmt: str, page: np.ndarray):
         scale_base = 16384
     else:
         off, tok, dim = _V8_CODES
-        c[tok, dim] = page[off].view(np.int8)
+        c[tok, dim] = page[off].astype(np.int16) - 128
         idx, tok, b = _V_SCALES
         scale_base = 32768
     d16 = np.zeros((PAGE_TOKENS, N_BLOCKS), dtype=np.uint16)

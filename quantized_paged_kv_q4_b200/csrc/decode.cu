@@ -50,7 +50,6 @@ struct DecodeCfg {
   static constexpr int kThreads = kConsumerWarps * 32;  // lanes of warp 0 also issue the copies
   static constexpr int kNB = 8 / SPLIT;                 // 32-channel blocks per warp
   static constexpr int kGroups = kConsumerWarps / SPLIT;  // warp groups, one softmax stream each
-  static constexpr int kReleases = 8 * SPLIT;             // (warp, tile) pairs per page
   static constexpr bool kK5 = KF == kKeyQ51 || KF == kKeyQ50;  // 5-bit key codes
   static constexpr bool kKMin = KF == kKeyQ51;                 // keys with a zero point
   static constexpr bool kVMin = VF == kValQ41;                 // values with a zero point
@@ -60,6 +59,26 @@ struct DecodeCfg {
   static constexpr int kVBytes = VF == kValQ8 ? kV8PageBytes : VF == kValQ41 ? kV41PageBytes : kV4PageBytes;
   static constexpr int kVScaleOff = VF == kValQ8 ? kV8ScaleOffset : kV4ScaleOffset;
   static constexpr int kStageBytes = kKBytes + kVBytes;
+  // Every region of a page (codes, fifth bits, scales, minima) is ordered by 16-token tile
+  // first, so tiles [g0, g1) of a page are one contiguous range of each region: (offset of
+  // the region, bytes per tile).  A stage holds K regions at 0 and V regions at kKBytes.
+  static constexpr int kKRegions = KF == kKeyQ51 ? 4 : KF == kKeyQ50 ? 3 : 2;
+  static constexpr int kVRegions = VF == kValQ41 ? 3 : 2;
+  __host__ __device__ static constexpr int k_reg_off(int r) {
+    return r == 0 ? 0 : r == 1 ? (kK5 ? kK5HighOffset : kKScaleOff) : r == 2 ? kK5ScaleOffset : kK5MinOffset;
+  }
+  __host__ __device__ static constexpr int k_reg_tile(int r) {
+    return r == 0 ? (KF == kKeyQ8 ? 4096 : 2048) : r == 1 && kK5 ? 512 : 256;
+  }
+  __host__ __device__ static constexpr int v_reg_off(int r) { return r == 0 ? 0 : r == 1 ? kVScaleOff : kV41MinOffset; }
+  __host__ __device__ static constexpr int v_reg_tile(int r) { return r == 0 ? (VF == kValQ8 ? 4096 : 2048) : 256; }
+  static_assert(8 * (k_reg_tile(0) + k_reg_tile(1) + (kKRegions > 2 ? k_reg_tile(2) : 0) +
+                     (kKRegions > 3 ? k_reg_tile(3) : 0)) == kKBytes, "K regions");
+  static_assert(8 * (v_reg_tile(0) + v_reg_tile(1) + (kVRegions > 2 ? v_reg_tile(2) : 0)) == kVBytes, "V regions");
+  static_assert(k_reg_off(1) == 8 * k_reg_tile(0) && (kKRegions < 3 || k_reg_off(2) == k_reg_off(1) + 8 * k_reg_tile(1)) &&
+                (kKRegions < 4 || k_reg_off(3) == k_reg_off(2) + 8 * k_reg_tile(2)), "K region offsets");
+  static_assert(v_reg_off(1) == 8 * v_reg_tile(0) && (kVRegions < 3 || v_reg_off(2) == v_reg_off(1) + 8 * v_reg_tile(1)),
+                "V region offsets");
   // split tiles keep the query B fragments in shared memory:
   // [block][k-step][n-tile][lane][hi0, hi1, lo0, lo1]
   static constexpr bool kQSmem = SPLIT > 1 || kConsumerWarps > 8;
@@ -196,9 +215,16 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
 
   int np = p.max_pages;
   if (p.n_pages_arr) np = min(max(p.n_pages_arr[h], 0), p.max_pages);
-  const int first = static_cast<int>(static_cast<long long>(split) * np / p.n_splits);
-  const int last = static_cast<int>(static_cast<long long>(split + 1) * np / p.n_splits);
-  const int count = last - first;
+  // This split's 16-token tiles [t_first, t_last) of the head's 8 np tiles, and the pages they
+  // touch, [first, first + count): the CTAs' shares differ by at most one tile.  The first and
+  // the last page may be shared with the neighbouring splits; each copies only its own tiles.
+  const int t_first = static_cast<int>(static_cast<long long>(split) * 8 * np / p.n_splits);
+  const int t_last = static_cast<int>(static_cast<long long>(split + 1) * 8 * np / p.n_splits);
+  const int first = t_first >> 3;
+  const int count = t_last > t_first ? ((t_last + 7) >> 3) - first : 0;
+  // tiles [tile_lo(i), tile_hi(i)) of the CTA's page i are in its range
+  auto tile_lo = [&](int i) { return i == 0 ? (t_first & 7) : 0; };
+  auto tile_hi = [&](int i) { return i == count - 1 && (t_last & 7) ? (t_last & 7) : 8; };
 
   // per-warp softmax state (consumers)
   float m_run[NT][2], l_run[NT][2];
@@ -244,12 +270,30 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
       record_error(KVATTN_ERR_BAD_PAGE);
       st_valid[s] = 0;
       mbar_arrive(&full[s]);
-    } else {
-      st_valid[s] = 1;
-      uint8_t* stage = smem + s * C::kStageBytes;
+      return;
+    }
+    st_valid[s] = 1;
+    uint8_t* stage = smem + s * C::kStageBytes;
+    const uint8_t* ksrc = p.k_pool + static_cast<int64_t>(page) * p.k_stride;
+    const uint8_t* vsrc = p.v_pool + static_cast<int64_t>(page) * p.v_stride;
+    const int g0 = tile_lo(i), g1 = tile_hi(i);
+    if (g0 == 0 && g1 == 8) {
       mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-      bulk_g2s(stage, p.k_pool + static_cast<int64_t>(page) * p.k_stride, C::kKBytes, &full[s]);
-      bulk_g2s(stage + C::kKBytes, p.v_pool + static_cast<int64_t>(page) * p.v_stride, C::kVBytes, &full[s]);
+      bulk_g2s(stage, ksrc, C::kKBytes, &full[s]);
+      bulk_g2s(stage + C::kKBytes, vsrc, C::kVBytes, &full[s]);
+    } else {
+      // a page shared with a neighbouring split: only tiles [g0, g1) of every region
+      mbar_arrive_expect_tx(&full[s], (g1 - g0) * (C::kStageBytes / 8));
+#pragma unroll
+      for (int r = 0; r < C::kKRegions; ++r) {
+        const int o = C::k_reg_off(r) + g0 * C::k_reg_tile(r);
+        bulk_g2s(stage + o, ksrc + o, (g1 - g0) * C::k_reg_tile(r), &full[s]);
+      }
+#pragma unroll
+      for (int r = 0; r < C::kVRegions; ++r) {
+        const int o = C::v_reg_off(r) + g0 * C::v_reg_tile(r);
+        bulk_g2s(stage + C::kKBytes + o, vsrc + o, (g1 - g0) * C::v_reg_tile(r), &full[s]);
+      }
     }
   };
   auto issue = [&](int i) {
@@ -402,16 +446,19 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
       }
     };
 
-    // Tiles in increasing order, group grp taking j = grp, grp + kGroups, ...: page i = j / 8,
-    // tile G = j % 8.  With more groups than tiles per page a group skips pages, so the parity
+    // The CTA's tiles in increasing order, group grp taking k = grp, grp + kGroups, ... (the
+    // head's tile j = t_first + k: the CTA's page i = j / 8 - first, tile G = j % 8).  A stage
+    // is refilled once every in-range tile of its page is done.  With more groups than tiles
+    // per page a group skips pages, so the parity
     // of a stage's barrier alone cannot tell page i from page i - kStages.  A group therefore
     // first waits until the stage's tag names page i (issued only after every tile of page
     // i - kStages is done, so that page's phase has completed), then for the barrier phase of
     // page i (which cannot move on before this group's tile of page i is done).
     const int new_lo = p.new_pos0, new_hi = p.new_pos0 + p.n_new;  // appended positions
-    const int n_tiles = 8 * count;
-    for (int j = grp; j < n_tiles; j += C::kGroups) {
-      const int i = j >> 3;
+    const int n_tiles = t_last - t_first;
+    for (int k = grp; k < n_tiles; k += C::kGroups) {
+      const int j = t_first + k;  // the head's tile
+      const int i = (j >> 3) - first;
       const int G = j & 7;
       const int s = i % C::kStages;
       const uint32_t par = (i / C::kStages) & 1;
@@ -511,16 +558,15 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
               const int P = blk0 / 2 + pp;
               const uint4 ka = lds128(kb + ((((G * 4 + P) * 2 + 0) * 8 + g) * 4 + t) * 16);
               const uint4 kc = lds128(kb + ((((G * 4 + P) * 2 + 1) * 8 + g) * 4 + t) * 16);
-              const uint32_t wg[4] = {ka.x ^ 0x80808080u, ka.y ^ 0x80808080u, ka.z ^ 0x80808080u,
-                                      ka.w ^ 0x80808080u};
-              const uint32_t w8[4] = {kc.x ^ 0x80808080u, kc.y ^ 0x80808080u, kc.z ^ 0x80808080u,
-                                      kc.w ^ 0x80808080u};
+              // code bytes are offset-binary (q + 128)
+              const uint32_t wg[4] = {ka.x, ka.y, ka.z, ka.w};
+              const uint32_t w8[4] = {kc.x, kc.y, kc.z, kc.w};
 #pragma unroll
               for (int e = 0; e < 2; ++e) {
                 uint32_t A[2][4];
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks) {
-                  // exact int8 -> f16: 1024 + (q + 128) - 1152
+                  // exact code -> f16: 1024 + (q + 128) - 1152
                   A[ks][0] = hsub2(prmt(wg[2 * e + ks], kByte64x4, 0x4140u), kHalf2_1152);
                   A[ks][2] = hsub2(prmt(wg[2 * e + ks], kByte64x4, 0x4342u), kHalf2_1152);
                   A[ks][1] = hsub2(prmt(w8[2 * e + ks], kByte64x4, 0x4140u), kHalf2_1152);
@@ -764,8 +810,7 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
               asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
                            : "=r"(d0), "=r"(d1)
                            : "r"(vb + kV8ScaleOffset + (((G * 4 + t) * 8 + b) * 4) * 2));
-              const uint32_t w[4] = {vw.x ^ 0x80808080u, vw.y ^ 0x80808080u, vw.z ^ 0x80808080u,
-                                     vw.w ^ 0x80808080u};
+              const uint32_t w[4] = {vw.x, vw.y, vw.z, vw.w};  // offset-binary code bytes (q + 128)
               uint32_t a[4][2];
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
@@ -789,7 +834,7 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
       if (aborted) break;
       __syncwarp();
       if (lane == 0) {
-        if (atomicAdd(&rel_cnt[s], 1) == C::kReleases - 1) {
+        if (atomicAdd(&rel_cnt[s], 1) == (tile_hi(i) - tile_lo(i)) * SPLIT - 1) {
           rel_cnt[s] = 0;
           if (i + C::kStages < count) issue(i + C::kStages);
         }

@@ -660,7 +660,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
           } else {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const uint32_t w = kw[i][e] ^ 0x80808080u;
+              const uint32_t w = kw[i][e];  // offset-binary code bytes: 1024 + (q + 128) - 1152 = q
               c[2 * e] = hsub2(prmt(w, 0x64646464u, 0x4140u), 0x64806480u);
               c[2 * e + 1] = hsub2(prmt(w, 0x64646464u, 0x4342u), 0x64806480u);
             }

@@ -176,11 +176,12 @@ __device__ __forceinline__ void encode_token(const float (&kx)[8], const float (
     const float (&x)[8] = kx;
     float inv;
     const float d = q8_scale(x, &inv);
+    // codes are stored offset-binary: the byte q + 128
     uint32_t w0 = 0, w1 = 0;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) w0 |= (static_cast<uint32_t>(q8_code(x[e], inv)) & 0xFFu) << (8 * e);
+    for (int e = 0; e < 4; ++e) w0 |= static_cast<uint32_t>(q8_code(x[e], inv) + 128) << (8 * e);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) w1 |= (static_cast<uint32_t>(q8_code(x[4 + e], inv)) & 0xFFu) << (8 * e);
+    for (int e = 0; e < 4; ++e) w1 |= static_cast<uint32_t>(q8_code(x[4 + e], inv) + 128) << (8 * e);
     uint8_t* pg = kpg;
     const int P = lane >> 3, T = lane & 3, jhi = (lane & 7) >> 2;
     const int off = ((((G * 4 + P) * 2 + H) * 8 + R) * 4 + T) * 16 + 8 * jhi;
@@ -239,7 +240,7 @@ __device__ __forceinline__ void encode_token(const float (&kx)[8], const float (
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int off = ((((G * 8 + b) * 8 + e) * 4 + T) * 16) + 4 * w + y;
-          pg[off] = static_cast<uint8_t>(codes[e] & 0xFF);
+          pg[off] = static_cast<uint8_t>(codes[e] + 128);  // offset-binary, as the K codes
         }
       }
       if (st && cl == 0) {

@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(256) block_summary_kernel(const uint8_t* __res
         if (k_fmt == kKeyQ50) q -= 16;
       }
     } else {
-      q = static_cast<int8_t>(page[((((G * 4 + P) * 2 + H) * 8 + R) * 4 + T) * 16 + j]);
+      q = static_cast<int>(page[((((G * 4 + P) * 2 + H) * 8 + R) * 4 + T) * 16 + j]) - 128;  // offset-binary
     }
     const int si = 2 * (((G * 8 + R) * 2 + H) * 8 + blk);
     acc += fp16_grid_units(*reinterpret_cast<const uint16_t*>(page + scale_off + si), q);

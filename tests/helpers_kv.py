@@ -66,16 +66,23 @@ class OracleCache:
     def vhat(self, h):
         return oq.dequantize(self.vc[:, h], self.vd[:, h], self.v_fmt)
 
+    @staticmethod
+    def _unwritten(fmt):
+        """Codes of slots never written (zero bytes in a zero-filled pool: Q8_0 stores q + 128)."""
+        if fmt == "q8_0":
+            return np.full((128, 8, 32), -128, np.int8)
+        return np.zeros((128, 8, 32), np.uint8)
+
     def page_bytes(self, h, blk, role):
-        """Expected bytes of logical block `blk` of unit h (tokens beyond T stay zero codes)."""
+        """Expected bytes of logical block `blk` of unit h (slots beyond T stay zero bytes)."""
         a, b = blk * 128, min((blk + 1) * 128, self.T)
         if role == "k":
-            codes = np.zeros((128, 8, 32), np.int8 if self.k_fmt == "q8_0" else np.uint8)
+            codes = self._unwritten(self.k_fmt)
             d = np.zeros((128,) + self.kd.shape[2:], np.float16)  # (d, m) pairs for Q5_1
             codes[: b - a] = self.kc[a:b, h]
             d[: b - a] = self.kd[a:b, h]
             return olay.encode_page("k", self.k_fmt, codes, d)
-        codes = np.zeros((128, 8, 32), np.int8 if self.v_fmt == "q8_0" else np.uint8)
+        codes = self._unwritten(self.v_fmt)
         d = np.zeros((128,) + self.vd.shape[2:], np.float16)  # (d, m) pairs for Q4_1
         codes[: b - a] = self.vc[a:b, h]
         d[: b - a] = self.vd[a:b, h]

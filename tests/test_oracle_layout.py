@@ -27,9 +27,10 @@ def test_round_trip(role, fmt):
 
 
 def _one_hot(fmt, tok, dim, code):
+    """A page of zero bytes but for one code (Q8_0: the code -128 is the zero byte)."""
     codes = np.zeros((128, 8, 32), dtype=np.int8 if fmt == "q8_0" else np.uint8)
-    if fmt == "q4_0":
-        codes[:] = 0
+    if fmt == "q8_0":
+        codes[:] = -128
     codes[tok, dim // 32, dim % 32] = code
     return codes, np.zeros((128, 8), np.float16)
 
@@ -42,6 +43,17 @@ def test_k_code_offsets(tok, dim, off):
     codes, d = _one_hot("q8_0", tok, dim, 7)
     page = layout.encode_page("k", "q8_0", codes, d)
     assert np.flatnonzero(page).tolist() == [off]
+    assert page[off] == 7 + 128
+
+
+@pytest.mark.parametrize("code,byte", [(-128, 0x00), (-127, 0x01), (-1, 0x7F), (0, 0x80), (1, 0x81), (127, 0xFF)])
+def test_q8_codes_are_stored_offset_binary(code, byte):
+    for role in ("k", "v"):
+        codes, d = _one_hot("q8_0", 3, 77, code)
+        page = layout.encode_page(role, "q8_0", codes, d)
+        assert page[:32768].tolist().count(byte) == (32768 if code == -128 else 1)
+        c2, _ = layout.decode_page(role, "q8_0", page)
+        assert c2[3, 2, 13] == code and c2.dtype == np.int8
 
 
 # K Q4_0: word 4*((((G*2+Q)*2+H)*8+R)*4+T)*4+c) for token 16G+8H+R, block 4Q+c; channel
@@ -118,7 +130,7 @@ def test_v_q4_1_matches_q4_0_nibbles_and_scales_plus_minima():
 
 
 def test_k_scale_offsets():
-    codes = np.zeros((128, 8, 32), np.int8)
+    codes = np.full((128, 8, 32), -128, np.int8)      # code bytes all zero
     d = np.zeros((128, 8), np.float16)
     d[9, 3] = 1.0          # G=0, R=1, H=1, b=3 -> index ((0*8+1)*2+1)*8+3 = 27
     page = layout.encode_page("k", "q8_0", codes, d)
@@ -146,6 +158,7 @@ def test_v_q8_code_offsets(tok, dim, off):
     codes, d = _one_hot("q8_0", tok, dim, 9)
     page = layout.encode_page("v", "q8_0", codes, d)
     assert np.flatnonzero(page).tolist() == [off]
+    assert page[off] == 9 + 128
 
 
 def test_v_scale_offsets():
@@ -153,7 +166,7 @@ def test_v_scale_offsets():
     d[10, 2] = 1.0        # tok 10 = 2T + k%2 + 8*(k//2) with T=1, k=2 -> index ((0*4+1)*8+2)*4+2 = 42
     for fmt, base in (("q4_0", 16384), ("q8_0", 32768)):
         codes = np.zeros((128, 8, 32), np.int8 if fmt == "q8_0" else np.uint8)
-        if fmt == "q4_0":
-            codes[:] = 0
+        if fmt == "q8_0":
+            codes[:] = -128                            # code bytes all zero
         page = layout.encode_page("v", fmt, codes, d)
         assert np.flatnonzero(page).tolist() == [base + 2 * 42 + 1]
