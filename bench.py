@@ -296,23 +296,23 @@ class DecodeBench(GraphStep):
         self.bytes_per_step = self.bytes_per_layer * L
         self.launches_per_step = 2 * L  # decode with the append fused in, split merge
 
-    def layer(self, l, timed=None):
+    def layer(self, l):
         """One layer: append the new token and attend, as one kvattn_append_decode (its split
-        grid, then the merge grid).  With `timed` (three events) the append is its own kernel
-        and the decode runs as its two grids with an event before, between and after them."""
+        grid, then the merge grid)."""
         kv, c = self.kv, self.cache
-        if timed is None:
-            kv.kvattn_append_decode(c.desc, self.k_new[l], self.v_new[l], 1, self.pos, c.page_table[l], self.nb,
-                                    self.q[l], 1, self.q_pos, c.page_table[l], None, None, self.nb, self.out[l],
-                                    self.lse[l], self.ws[l], self.ws_bytes)
-            return
-        kv.kvattn_quantize_append(c.desc, self.k_new[l], self.v_new[l], 1, self.pos, c.page_table[l], self.nb)
-        timed[0].record()
-        kv.kvattn_decode_splits(c.desc, self.q[l], 1, self.q_pos, c.page_table[l], None, None, self.nb, self.out[l],
+        kv.kvattn_append_decode(c.desc, self.k_new[l], self.v_new[l], 1, self.pos, c.page_table[l], self.nb,
+                                self.q[l], 1, self.q_pos, c.page_table[l], None, None, self.nb, self.out[l],
                                 self.lse[l], self.ws[l], self.ws_bytes)
-        timed[1].record()
-        kv.kvattn_decode_merge_splits(c.desc, 1, self.nb, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
-        timed[2].record()
+
+    def split_grid(self, l):
+        """The layer's decode split grid alone (the token already appended)."""
+        c = self.cache
+        self.kv.kvattn_decode_splits(c.desc, self.q[l], 1, self.q_pos, c.page_table[l], None, None, self.nb,
+                                     self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
+
+    def merge_grid(self, l):
+        self.kv.kvattn_decode_merge_splits(self.cache.desc, 1, self.nb, self.out[l], self.lse[l], self.ws[l],
+                                           self.ws_bytes)
 
 
 class VerifyBench(GraphStep):
@@ -359,23 +359,24 @@ class VerifyBench(GraphStep):
         self.select_bytes_per_layer = H * (self.n_full - w.recent_blocks) * 256 * 4
         self.launches_per_step = 4 * L  # block scores, top-k, decode with the append fused in, split merge
 
-    def layer(self, l, timed=None):
+    def layer(self, l):
         kv, c, w = self.kv, self.cache, self.w
         kv.kvattn_select_blocks(self.summ[l * w.kv_heads:(l + 1) * w.kv_heads], self.q_group[l], w.kv_heads, w.group,
                                 self.nb, self.n_full, self.nb, w.budget_blocks, w.recent_blocks, c.page_table[l],
                                 self.sel_l[l], self.sel_p[l], self.n_sel[l], self.cap, self.sws, self.sws_bytes)
-        if timed is None:
-            kv.kvattn_append_decode(c.desc, self.k_new[l], self.v_new[l], w.n_q, self.pos0, c.page_table[l], self.nb,
-                                    self.q[l], w.n_q, self.q_pos, self.sel_p[l], self.sel_l[l], self.n_sel[l],
-                                    self.cap, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
-            return
-        kv.kvattn_quantize_append(c.desc, self.k_new[l], self.v_new[l], w.n_q, self.pos0, c.page_table[l], self.nb)
-        timed[0].record()
-        kv.kvattn_decode_splits(c.desc, self.q[l], w.n_q, self.q_pos, self.sel_p[l], self.sel_l[l], self.n_sel[l],
+        kv.kvattn_append_decode(c.desc, self.k_new[l], self.v_new[l], w.n_q, self.pos0, c.page_table[l], self.nb,
+                                self.q[l], w.n_q, self.q_pos, self.sel_p[l], self.sel_l[l], self.n_sel[l],
                                 self.cap, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
-        timed[1].record()
-        kv.kvattn_decode_merge_splits(c.desc, w.n_q, self.cap, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
-        timed[2].record()
+
+    def split_grid(self, l):
+        """The layer's decode split grid alone, over the selection of the last step."""
+        c, w = self.cache, self.w
+        self.kv.kvattn_decode_splits(c.desc, self.q[l], w.n_q, self.q_pos, self.sel_p[l], self.sel_l[l],
+                                     self.n_sel[l], self.cap, self.out[l], self.lse[l], self.ws[l], self.ws_bytes)
+
+    def merge_grid(self, l):
+        self.kv.kvattn_decode_merge_splits(self.cache.desc, self.w.n_q, self.cap, self.out[l], self.lse[l],
+                                           self.ws[l], self.ws_bytes)
 
 
 class PrefillBench:
@@ -798,20 +799,37 @@ def time_steps(bench, steps, warmup, world):
 
 
 def time_kernel(bench, steps):
-    """Average device duration of the decode split grid and of its merge grid, per layer launch
-    (events on the launching stream before, between and after the two grids)."""
+    """Average device duration of one launch of the decode split grid and of its merge grid.
+    Each kind is captured as a CUDA graph of its launches for every layer, back to back on one
+    stream (programmatic dependent launch, as in the step), and replayed `steps` times between
+    two events on that stream; the duration is the elapsed time / launches.  The grids run on
+    the state the preceding full steps left (pages with the token appended, selections)."""
     import torch
 
-    trip = []
-    for _ in range(steps):
-        for l in range(bench.w.layers):
-            p = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-                 torch.cuda.Event(enable_timing=True))
-            bench.layer(l, timed=p)
-            trip.append(p)
-    torch.cuda.synchronize()
-    return (statistics.mean(a.elapsed_time(b) for a, b, _ in trip),
-            statistics.mean(b.elapsed_time(c) for _, b, c in trip))
+    out = []
+    for grid in (bench.split_grid, bench.merge_grid):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for l in range(bench.w.layers):
+                grid(l)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for l in range(bench.w.layers):
+                grid(l)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = event_pair()
+        e0.record()
+        for _ in range(steps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        out.append(e0.elapsed_time(e1) / (steps * bench.w.layers))
+        del g
+    return out[0], out[1]
 
 
 def time_layers(bench, steps):
@@ -1018,7 +1036,8 @@ def main():
                    "launch": launch_mode},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": profiled_traffic("decode_kernel_decode131k.md"),
-                     "kernel": "decode_kernel<Q8_0 K, Q4_0 V, 8 rows> (the split grid alone)",
+                     "kernel": ("decode_kernel<Q8_0 K, Q4_0 V, 8 rows>: the split grid alone, one launch per "
+                                "layer back to back in a CUDA graph"),
                      "peak_kind": f"{peak_kind} copy bandwidth (hbm_gbs)",
                      "algorithmic_bytes_per_launch": b.bytes_per_layer, "avg_launch_ms": kern_ms,
                      "merge_grid_ms": merge_ms, "step_ms_per_layer": ms / b.w.layers,
