@@ -28,10 +28,6 @@
 // of kvattn_merge_lse.
 #include "decode.cuh"
 
-#ifndef KVATTN_DECODE_WARPS1
-#define KVATTN_DECODE_WARPS1 12  // consumer warps of the unsplit (8-row) shape
-#endif
-
 namespace kvattn {
 
 
@@ -46,7 +42,7 @@ struct DecodeCfg {
   // accumulators per warp.  (Sixteen warps in the split arrangement measured slower for 8
   // rows: the duplicated softmax and the exchange cost more instructions than the extra
   // warps hid.)
-  static constexpr int kConsumerWarps = SPLIT == 1 ? KVATTN_DECODE_WARPS1 : 8;
+  static constexpr int kConsumerWarps = SPLIT == 1 ? 12 : 8;
   static constexpr int kThreads = kConsumerWarps * 32;  // lanes of warp 0 also issue the copies
   static constexpr int kNB = 8 / SPLIT;                 // 32-channel blocks per warp
   static constexpr int kGroups = kConsumerWarps / SPLIT;  // warp groups, one softmax stream each

@@ -59,11 +59,32 @@ def test_decode_matches_oracle(kv_gpu, k_fmt, v_fmt, n_q):
     for h in range(H):
         o_ref, l_ref = oc.attend(q, q_pos, h, 6)
         compare(out[:, 6 * h:6 * h + 6], lse[:, 6 * h:6 * h + 6], o_ref, l_ref)
-    # a second launch reuses the workspace (split counters are left at zero) bit-identically
+    # a second launch reusing the workspace gives the same bits
     qd, qp, pl, lg, npg, o2, l2, ws, wsb = keep
     kv_gpu.kvattn_decode(cache.desc, qd, n_q, qp, pl, lg, npg, pl.shape[1], o2, l2, ws, wsb)
     torch.cuda.synchronize()
     assert np.array_equal(o2.cpu().numpy(), out) and np.array_equal(l2.cpu().numpy(), lse)
+
+
+@pytest.mark.parametrize("k_fmt,v_fmt", [("q8_0", "q4_0"), ("q5_1", "q8_0"), ("q5_0", "q4_1")])
+@pytest.mark.parametrize("n_q,T,budget", [(1, 3 * 128 + 40, 148), (1, 37 * 128 + 77, 24), (1, 37 * 128 + 77, 9),
+                                          (4, 5 * 128 + 3, 148), (4, 37 * 128 + 77, 20)])
+def test_decode_tile_splits_and_sm_budget(kv_gpu, k_fmt, v_fmt, n_q, T, budget):
+    """Splits are ranges of 16-token tiles: with few pages over many splits most CTAs take part
+    of a page (copied region by region) or nothing at all; a descriptor's SM budget gives fewer
+    splits.  Every partition must agree with the oracle."""
+    H, H_q = 4, 24
+    rng, k, v, cache = _layer(680 + T % 97 + budget, H, T, v_fmt, spare=3, k_fmt=k_fmt)
+    cache.append(k, v, 0)
+    cache.desc.sm_budget = budget
+    q = normal_f32(rng, (n_q, H_q, 256))
+    q_pos = [T - n_q + i for i in range(n_q)]
+    out, lse, _ = _run_decode(kv_gpu, cache, H_q, q, q_pos, cache.page_table_np)
+    assert kv_gpu.kvattn_device_error() == 0
+    oc = OracleCache(k, v, v_fmt, k_fmt)
+    for h in range(H):
+        o_ref, l_ref = oc.attend(q, q_pos, h, 6)
+        compare(out[:, 6 * h:6 * h + 6], lse[:, 6 * h:6 * h + 6], o_ref, l_ref)
 
 
 @pytest.mark.parametrize("n_q", [1, 4])
