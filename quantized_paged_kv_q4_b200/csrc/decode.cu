@@ -5,11 +5,13 @@
 // 1398, "pitfalls": the legacy block quants valid as KV types; the q4_0/q4_0 and K q5_1 /
 // V q4_0 caches; MTP tuning notes on one 7900 XTX, lcz.me/topic/593: a q5_0 / q4_1 cache).
 //
-// Grid: (split, KV head).  One CTA per SM: lanes of warp 0 stream whole pages into a
-// shared-memory ring with bulk async copies (TMA engine, one K copy and one V copy per page);
-// warps 0-7 consume them.  All query rows of the KV head's group (group x n_q <= 24) are
-// packed into the N dimension of legacy tensor-core MMAs so every KV byte is read once per
-// group.  The arithmetic keeps the dequantized operands exact:
+// Grid: (split, KV head), each split a range of 16-token tiles.  One CTA per SM: lanes of warp
+// 0 stream the pages into a shared-memory ring with bulk async copies (TMA engine, one K copy
+// and one V copy per page, or one per region for a page shared with the next split); all warps
+// consume them (twelve for 8 query rows, eight in pairs for 16 and 24).  All query rows of
+// the KV head's group (group x n_q <= 24) are packed into the N dimension of legacy
+// tensor-core MMAs so every KV byte is read once per group.  The arithmetic keeps the
+// dequantized operands exact:
 //   QK^T: f16 MMA (m16n8k16), A = the key codes decoded in registers (integers, exact in
 //         f16), 16 tokens on M; B = the query row divided by its largest magnitude, as an f16
 //         high part and an f16 low part (the rounded remainder: about 22 significant bits
@@ -29,7 +31,6 @@
 #include "decode.cuh"
 
 namespace kvattn {
-
 
 template <int KF, int VF, int NT, int SPLIT>
 struct DecodeCfg {
