@@ -8,9 +8,10 @@
 // Grid: (split, KV head), each split a range of 16-token tiles.  One CTA per SM: lanes of warp
 // 0 stream the pages into a shared-memory ring with bulk async copies (TMA engine, one K copy
 // and one V copy per page, or one per region for a page shared with the next split); all warps
-// consume them (twelve for 8 query rows, eight in pairs for 16 and 24).  All query rows of
-// the KV head's group (group x n_q <= 24) are packed into the N dimension of legacy
-// tensor-core MMAs so every KV byte is read once per group.  The arithmetic keeps the
+// consume them: twelve warps, each holding one 8-row n-tile of the head's query rows, the
+// warps of a group (one per n-tile) sharing each 16-token tile.  All query rows of the KV
+// head's group (group x n_q <= 24) are packed into the N dimension of legacy tensor-core MMAs
+// so every KV byte is read from HBM once per group.  The arithmetic keeps the
 // dequantized operands exact:
 //   QK^T: f16 MMA (m16n8k16), A = the key codes decoded in registers (integers, exact in
 //         f16), 16 tokens on M; B = the query row divided by its largest magnitude, as an f16
@@ -32,21 +33,20 @@
 
 namespace kvattn {
 
-template <int KF, int VF, int NT, int SPLIT>
+template <int KF, int VF, int NT>
 struct DecodeCfg {
-  // SPLIT warps share each 16-token tile, each taking 8 / SPLIT of the 32-channel blocks, and
-  // add their partial scores through shared memory.  The groups of SPLIT warps take the
-  // 16-token tiles of the CTA's pages round robin (tile j = 8 x page + tile in page goes to
-  // group j mod kGroups).  The 8-row shape runs unsplit tiles (SPLIT = 1) on twelve warps,
-  // three per scheduler, with the query fragments in shared memory so that a thread needs
-  // at most 168 registers; the 16- and 24-row shapes split the tiles in two, which halves the
-  // accumulators per warp.  (Sixteen warps in the split arrangement measured slower for 8
-  // rows: the duplicated softmax and the exchange cost more instructions than the extra
-  // warps hid.)
-  static constexpr int kConsumerWarps = SPLIT == 1 ? 12 : 8;
+  // Twelve consumer warps, three per scheduler, so that a thread has at most 168 registers.
+  // Each warp owns one n-tile (8 query rows) of a 16-token tile and all 256 channels; the NT
+  // warps of a group share each tile (one per n-tile), and the groups take the CTA's tiles
+  // round robin (tile k of the CTA goes to group k mod kGroups).  The query fragments sit in
+  // shared memory.  (Sharing a tile between warps by channel halves or quarters, with partial
+  // scores exchanged through shared memory, and sixteen warps at 128 registers, measured
+  // slower.)
+  static constexpr int kConsumerWarps = 12;
   static constexpr int kThreads = kConsumerWarps * 32;  // lanes of warp 0 also issue the copies
-  static constexpr int kNB = 8 / SPLIT;                 // 32-channel blocks per warp
-  static constexpr int kGroups = kConsumerWarps / SPLIT;  // warp groups, one softmax stream each
+  static_assert(kConsumerWarps % NT == 0, "n-tiles per group");
+  static constexpr int kGroups = kConsumerWarps / NT;   // warp groups taking tiles
+  static constexpr int kNB = 8;                          // 32-channel blocks (all, per warp)
   static constexpr bool kK5 = KF == kKeyQ51 || KF == kKeyQ50;  // 5-bit key codes
   static constexpr bool kKMin = KF == kKeyQ51;                 // keys with a zero point
   static constexpr bool kVMin = VF == kValQ41;                 // values with a zero point
@@ -76,28 +76,22 @@ struct DecodeCfg {
                 (kKRegions < 4 || k_reg_off(3) == k_reg_off(2) + 8 * k_reg_tile(2)), "K region offsets");
   static_assert(v_reg_off(1) == 8 * v_reg_tile(0) && (kVRegions < 3 || v_reg_off(2) == v_reg_off(1) + 8 * v_reg_tile(1)),
                 "V region offsets");
-  // split tiles keep the query B fragments in shared memory:
-  // [block][k-step][n-tile][lane][hi0, hi1, lo0, lo1]
-  static constexpr bool kQSmem = SPLIT > 1 || kConsumerWarps > 8;
-  static constexpr int kQBytes = kQSmem ? 8 * 2 * NT * 32 * 16 : 0;
-  static constexpr int kUnits = kGroups;   // independent softmax streams per CTA
+  // the query B fragments: [block][k-step][n-tile][lane][hi0, hi1, lo0, lo1]
+  static constexpr int kQBytes = 8 * 2 * NT * 32 * 16;
   static constexpr int kRowsPad = NT * 8;
-  // partial-score exchange: [group][part][parity][n-tile][lane][4 floats]
-  static constexpr int kXBytes = SPLIT > 1 ? kGroups * SPLIT * 2 * NT * 32 * 16 : 0;
-  // as many page stages as fit beside the pair exchange buffer, the query fragments and the
-  // barriers (at most 6)
-  static constexpr int kStagesFit = (227 * 1024 - 256 - kXBytes - kQBytes) / kStageBytes;
+  // as many page stages as fit beside the query fragments and the barriers (at most 6)
+  static constexpr int kStagesFit = (227 * 1024 - 256 - kQBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
   static constexpr int kRingBytes = kStages * kStageBytes;
   // rows of the output merge buffer are padded by 4 floats: the four lanes of an MMA quad
   // store rows 2t, 2t+1 of the same dims and then fall into different banks
   static constexpr int kOStride = kHeadDim + 4;
-  static constexpr int kMergeBytes = kUnits * kRowsPad * (kOStride + 2) * 4;
+  static constexpr int kMergeBytes = kConsumerWarps * 8 * (kOStride + 2) * 4;  // 8 rows per warp
   static_assert(kMergeBytes <= kRingBytes, "merge buffer must fit in the ring");
-  static constexpr int kQOffset = kRingBytes + kXBytes;
+  static constexpr int kQOffset = kRingBytes;
   static constexpr int kBarOffset = kQOffset + kQBytes;
   static constexpr int kSmemBytes = kBarOffset + 256;
-  static_assert(8 * (kStages + kGroups) + 4 * (4 * kStages + 1) <= 256, "stage bookkeeping");
+  static_assert(8 * kStages + 4 * (4 * kStages + 1) <= 256, "stage bookkeeping");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -173,13 +167,12 @@ __device__ __noinline__ void append_global(const float* k_new, const float* v_ne
                pos % kPageTokens, k_fmt, v_fmt, 0xffffffffu);
 }
 
-template <int KF, int VF, int NT, int SPLIT>
-__global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) decode_kernel(const DecodeParams p) {
-  using C = DecodeCfg<KF, VF, NT, SPLIT>;
+template <int KF, int VF, int NT>
+__global__ void __launch_bounds__(DecodeCfg<KF, VF, NT>::kThreads, 1) decode_kernel(const DecodeParams p) {
+  using C = DecodeCfg<KF, VF, NT>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
-  uint64_t* xbar = full + C::kStages;   // [kGroups] score-exchange barriers (split tiles only)
-  int* rel_cnt = reinterpret_cast<int*>(xbar + C::kGroups);  // [kStages] (warp, tile) pairs done
+  int* rel_cnt = reinterpret_cast<int*>(full + C::kStages);  // [kStages] (warp, tile) pairs done
   int* st_page = rel_cnt + C::kStages;     // [kStages] the page last issued into the stage, -1: none
   int* st_logical = st_page + C::kStages;  // [kStages]
   int* st_valid = st_logical + C::kStages;  // [kStages]
@@ -200,7 +193,6 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
       rel_cnt[s] = 0;
       st_page[s] = -1;
     }
-    for (int i = 0; i < C::kGroups; ++i) mbar_init(&xbar[i], SPLIT);
     s_flags[0] = 0;
     fence_barrier_init();
   }
@@ -223,35 +215,28 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
   auto tile_lo = [&](int i) { return i == 0 ? (t_first & 7) : 0; };
   auto tile_hi = [&](int i) { return i == count - 1 && (t_last & 7) ? (t_last & 7) : 8; };
 
-  // per-warp softmax state (consumers)
-  float m_run[NT][2], l_run[NT][2];
-  float oacc[2 * C::kNB][NT][4];
+  // per-warp softmax state (consumers): rows 2t, 2t + 1 of the warp's n-tile (index c)
+  float m_run[2], l_run[2];
+  float oacc[2 * C::kNB][4];
   // values with a zero point: sum over tokens of p * m per (block, query row), kept apart
   // from oacc (every dimension of a block gets the same term) and added at the end
-  float macc[C::kVMin ? C::kNB : 1][NT][4];
+  float macc[C::kVMin ? C::kNB : 1][4];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      m_run[nt][c] = -INFINITY;
-      l_run[nt][c] = 0.f;
-    }
+  for (int c = 0; c < 2; ++c) {
+    m_run[c] = -INFINITY;
+    l_run[c] = 0.f;
+  }
 #pragma unroll
   for (int i = 0; i < 2 * C::kNB; ++i)
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) oacc[i][nt][e] = 0.f;
+    for (int e = 0; e < 4; ++e) oacc[i][e] = 0.f;
 #pragma unroll
   for (int i = 0; i < (C::kVMin ? C::kNB : 1); ++i)
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) macc[i][nt][e] = 0.f;
+    for (int e = 0; e < 4; ++e) macc[i][e] = 0.f;
 
-  const int part = warp & (SPLIT - 1);  // this warp's share of the channel blocks
-  const int grp = warp / SPLIT;          // the warps that share a tile
-  const int blk0 = C::kNB * part;
+  const int grp = warp / NT;  // the warps that share a tile, one per n-tile
+  const int nt0 = warp % NT;  // this warp's n-tile: query rows 8 nt0 .. 8 nt0 + 7
 
   // Page copies: the first kStages pages are issued up front by lanes of warp 0; after
   // that, the warp that finishes the last of a page's tiles refills its stage at once with
@@ -320,29 +305,24 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
     // ------------------------------------------------------------------ consumers
     // query rows of this KV head: r = qi * group + j  ->  q[qi][h * group + j][:]
     // B fragments: the query row divided by its largest magnitude, split into an f16 high
-    // part and an f16 low part (the rounded remainder), per block, k-step and n-tile (two
-    // regs each); crow[nt][c] = amax / 16 * log2(e) turns a dot product with the normalised
-    // row into a base-2 softmax score.
-    uint32_t qh[C::kQSmem ? 1 : C::kNB][2][NT][2];
-    uint32_t ql[C::kQSmem ? 1 : C::kNB][2][NT][2];
-    float crow[NT][2];
+    // part and an f16 low part (the rounded remainder), per block and k-step (two regs each),
+    // in shared memory for the n-tile's warps; crow[c] = amax / 16 * log2(e) turns a dot
+    // product with the normalised row into a base-2 softmax score.
+    float crow[2];
     // zero-point keys: per block, the sum of the normalised query row's channels (for the
-    // query rows 2t, 2t + 1 of each n-tile)
-    float qsum[C::kKMin ? C::kNB : 1][NT][2];
+    // query rows 2t, 2t + 1 of the n-tile)
+    float qsum[C::kKMin ? C::kNB : 1][2];
     // query positions of this thread's accumulator rows, loaded first: every global read of
     // the setup is issued before any of them is used
-    int qpos_row[NT][2];
+    int qpos_row[2];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int rr = nt * 8 + 2 * t + c;
-        qpos_row[nt][c] = rr < n_rows ? p.q_pos[rr / p.group] : INT_MAX;
-      }
+    for (int c = 0; c < 2; ++c) {
+      const int rr = nt0 * 8 + 2 * t + c;
+      qpos_row[c] = rr < n_rows ? p.q_pos[rr / p.group] : INT_MAX;
+    }
     const uint32_t q_s = smem_u32(smem + C::kQOffset);
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int r = nt * 8 + g;
+    {
+      const int r = nt0 * 8 + g;
       float x[kBlocks][8];
       if (r < n_rows) {
         const int qi = r / p.group, j = r % p.group;
@@ -372,15 +352,7 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
       for (int bl = 0; bl < C::kNB; ++bl) {
         float xv[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          // block blk0 + bl, selected with constant indices (a runtime index would put x in
-          // local memory)
-          float xe = x[bl][e];
-#pragma unroll
-          for (int pp = 1; pp < SPLIT; ++pp)
-            if (part == pp) xe = x[pp * C::kNB + bl][e];
-          xv[e] = xe * inv;
-        }
+        for (int e = 0; e < 8; ++e) xv[e] = x[bl][e] * inv;
         // k-step 0 of the block: channels 8t+0..3, k-step 1: 8t+4..7 (k = 2t, 2t+1 | 2t+8, 2t+9)
         uint32_t hi[2][2], lo[2][2];
 #pragma unroll
@@ -388,24 +360,14 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
           split_pair(xv[4 * ks], xv[4 * ks + 1], hi[ks][0], lo[ks][0]);
           split_pair(xv[4 * ks + 2], xv[4 * ks + 3], hi[ks][1], lo[ks][1]);
         }
-        if constexpr (C::kQSmem) {
-          // the warps of every group hold the same values; those of group 0 write them
-          if (warp < SPLIT) {
+        // every group holds the same values; the warps of group 0 (one per n-tile) write them
+        if (warp < NT) {
 #pragma unroll
-            for (int ks = 0; ks < 2; ++ks)
-              asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
-                               q_s + (((((blk0 + bl) * 2 + ks) * NT + nt) * 32 + lane) * 16)),
-                           "r"(hi[ks][0]), "r"(hi[ks][1]), "r"(lo[ks][0]), "r"(lo[ks][1])
-                           : "memory");
-          }
-        } else {
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            qh[bl][ks][nt][0] = hi[ks][0];
-            qh[bl][ks][nt][1] = hi[ks][1];
-            ql[bl][ks][nt][0] = lo[ks][0];
-            ql[bl][ks][nt][1] = lo[ks][1];
-          }
+          for (int ks = 0; ks < 2; ++ks)
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             q_s + ((((bl * 2 + ks) * NT + nt0) * 32 + lane) * 16)),
+                         "r"(hi[ks][0]), "r"(hi[ks][1]), "r"(lo[ks][0]), "r"(lo[ks][1])
+                         : "memory");
         }
         if constexpr (C::kKMin) {
           float sm = 0.f;
@@ -413,34 +375,23 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
           for (int e = 0; e < 8; ++e) sm += xv[e];
           sm += __shfl_xor_sync(0xffffffffu, sm, 1);
           sm += __shfl_xor_sync(0xffffffffu, sm, 2);
-          qsum[bl][nt][0] = __shfl_sync(0xffffffffu, sm, (2 * t) * 4);
-          qsum[bl][nt][1] = __shfl_sync(0xffffffffu, sm, (2 * t + 1) * 4);
+          qsum[bl][0] = __shfl_sync(0xffffffffu, sm, (2 * t) * 4);
+          qsum[bl][1] = __shfl_sync(0xffffffffu, sm, (2 * t + 1) * 4);
         }
       }
       const float cr = amax * (1.0f / 16.0f) * 1.4426950408889634f;
-      crow[nt][0] = __shfl_sync(0xffffffffu, cr, (2 * t) * 4);
-      crow[nt][1] = __shfl_sync(0xffffffffu, cr, (2 * t + 1) * 4);
+      crow[0] = __shfl_sync(0xffffffffu, cr, (2 * t) * 4);
+      crow[1] = __shfl_sync(0xffffffffu, cr, (2 * t + 1) * 4);
     }
-    if constexpr (C::kQSmem) __syncthreads();
-    // the smallest query position over all rows (the four t-lanes of a quad hold all rows)
-    int qpos_min = INT_MAX;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) qpos_min = min(qpos_min, min(qpos_row[nt][0], qpos_row[nt][1]));
+    __syncthreads();
+    // the smallest query position over the warp's rows (the four t-lanes of a quad hold them)
+    int qpos_min = min(qpos_row[0], qpos_row[1]);
     qpos_min = min(qpos_min, __shfl_xor_sync(0xffffffffu, qpos_min, 1));
     qpos_min = min(qpos_min, __shfl_xor_sync(0xffffffffu, qpos_min, 2));
 
-    float* xbuf = reinterpret_cast<float*>(smem + C::kRingBytes);
-    int xpar = 0;
-    uint32_t xphase = 0;
-    bool aborted = false;
-
-    // the B fragments (hi0, hi1, lo0, lo1) of block bl, k-step ks, n-tile nt
-    auto qfrag = [&](int bl, int ks, int nt) -> uint4 {
-      if constexpr (C::kQSmem) {
-        return lds128(q_s + (((((blk0 + bl) * 2 + ks) * NT + nt) * 32 + lane) * 16));
-      } else {
-        return make_uint4(qh[bl][ks][nt][0], qh[bl][ks][nt][1], ql[bl][ks][nt][0], ql[bl][ks][nt][1]);
-      }
+    // the B fragments (hi0, hi1, lo0, lo1) of block bl, k-step ks
+    auto qfrag = [&](int bl, int ks) -> uint4 {
+      return lds128(q_s + ((((bl * 2 + ks) * NT + nt0) * 32 + lane) * 16));
     };
 
     // The CTA's tiles in increasing order, group grp taking k = grp, grp + kGroups, ... (the
@@ -471,54 +422,30 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
         {
           const int pos_lo = logical * kPageTokens + 16 * G;
           if (pos_lo < new_hi && pos_lo + 16 > new_lo) {
-            // an appended token in this tile: encode it into the stage (this warp's channel
-            // blocks; lanes 4b .. 4b + 3 hold block b), as split 0 encodes it into the page in
-            // global memory
-            constexpr int kLanes = 32 / SPLIT;
-            const uint32_t mask = SPLIT == 1 ? 0xffffffffu : (((1u << kLanes) - 1u) << (kLanes * part));
+            // an appended token in this tile: encode it into the stage, as split 0 encodes it
+            // into the page in global memory.  Each of the tile's warps writes the whole token
+            // (the same bytes) before it reads the tile, so none reads a partial patch.
             patch_stage(p.k_new, p.v_new, p.n_new, p.new_pos0, h, gridDim.y, lane, smem + s * C::kStageBytes,
-                        C::kKBytes, logical, pos_lo, KF, VF, mask);
+                        C::kKBytes, logical, pos_lo, KF, VF, 0xffffffffu);
           }
-          // ---------------- S = K Q^T over this warp's channel blocks ----------------
+          // ---------------- S = K Q^T over the 256 channels ----------------
           // Key codes enter the MMA exactly (integers in f16).  Each 32-channel block is
           // accumulated on its own (four MMAs: two k-steps, query high and low parts) and then
           // scaled by the block's fp32 scale (and, with a zero point, plus the block minimum
           // times the query block sum) into S.
-          float sacc[NT][4];
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-          // key scales (and minima) of rows g (H=0) and g+8 (H=1) for this warp's blocks, fp32
+          float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+          // key scales (and minima) of rows g (H=0) and g+8 (H=1) for the 8 blocks, fp32
           float dkf[2][C::kNB];
           float mkf[2][C::kKMin ? C::kNB : 1];
 #pragma unroll
           for (int H = 0; H < 2; ++H) {
-            const uint32_t a = kb + C::kKScaleOff + (((G * 8 + g) * 2 + H) * 8 + blk0) * 2;
+            const uint32_t a = kb + C::kKScaleOff + (((G * 8 + g) * 2 + H) * 8) * 2;
             uint32_t w[4], wm[4];
-            if constexpr (C::kNB == 8) {
-              const uint4 v = lds128(a);
-              w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-              if constexpr (C::kKMin) {
-                const uint4 vm = lds128(a + (kK5MinOffset - kK5ScaleOffset));
-                wm[0] = vm.x; wm[1] = vm.y; wm[2] = vm.z; wm[3] = vm.w;
-              }
-            } else if constexpr (C::kNB == 4) {
-              asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(a));
-              w[2] = w[3] = 0u;
-              if constexpr (C::kKMin) {
-                asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
-                             : "=r"(wm[0]), "=r"(wm[1])
-                             : "r"(a + (kK5MinOffset - kK5ScaleOffset)));
-                wm[2] = wm[3] = 0u;
-              }
-            } else {
-              w[0] = lds32(a);
-              w[1] = w[2] = w[3] = 0u;
-              if constexpr (C::kKMin) {
-                wm[0] = lds32(a + (kK5MinOffset - kK5ScaleOffset));
-                wm[1] = wm[2] = wm[3] = 0u;
-              }
+            const uint4 v = lds128(a);
+            w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+            if constexpr (C::kKMin) {
+              const uint4 vm = lds128(a + (kK5MinOffset - kK5ScaleOffset));
+              wm[0] = vm.x; wm[1] = vm.y; wm[2] = vm.z; wm[3] = vm.w;
             }
 #pragma unroll
             for (int e = 0; e < C::kNB / 2; ++e) {
@@ -532,27 +459,21 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
           }
           // one block: four MMAs into xb, then S += d * xb (+ m * qsum)
           auto block_qk = [&](int bl, const uint32_t (&A)[2][4]) {
-            float xb[NT][4];
+            float xb[4];
+            const uint4 f0 = qfrag(bl, 0), f1 = qfrag(bl, 1);
+            mma_f16_z(xb, A[0][0], A[0][1], A[0][2], A[0][3], f0.x, f0.y);
+            mma_f16(xb, A[0][0], A[0][1], A[0][2], A[0][3], f0.z, f0.w);
+            mma_f16(xb, A[1][0], A[1][1], A[1][2], A[1][3], f1.x, f1.y);
+            mma_f16(xb, A[1][0], A[1][1], A[1][2], A[1][3], f1.z, f1.w);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              const uint4 f0 = qfrag(bl, 0, nt), f1 = qfrag(bl, 1, nt);
-              mma_f16_z(xb[nt], A[0][0], A[0][1], A[0][2], A[0][3], f0.x, f0.y);
-              mma_f16(xb[nt], A[0][0], A[0][1], A[0][2], A[0][3], f0.z, f0.w);
-              mma_f16(xb[nt], A[1][0], A[1][1], A[1][2], A[1][3], f1.x, f1.y);
-              mma_f16(xb[nt], A[1][0], A[1][1], A[1][2], A[1][3], f1.z, f1.w);
+            for (int e = 0; e < 4; ++e) {
+              sacc[e] = fmaf(dkf[e >> 1][bl], xb[e], sacc[e]);
+              if constexpr (C::kKMin) sacc[e] = fmaf(mkf[e >> 1][bl], qsum[bl][e & 1], sacc[e]);
             }
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                sacc[nt][e] = fmaf(dkf[e >> 1][bl], xb[nt][e], sacc[nt][e]);
-                if constexpr (C::kKMin) sacc[nt][e] = fmaf(mkf[e >> 1][bl], qsum[bl][nt][e & 1], sacc[nt][e]);
-              }
           };
           if constexpr (KF == kKeyQ8) {
 #pragma unroll
-            for (int pp = 0; pp < C::kNB / 2; ++pp) {
-              const int P = blk0 / 2 + pp;
+            for (int P = 0; P < C::kNB / 2; ++P) {
               const uint4 ka = lds128(kb + ((((G * 4 + P) * 2 + 0) * 8 + g) * 4 + t) * 16);
               const uint4 kc = lds128(kb + ((((G * 4 + P) * 2 + 1) * 8 + g) * 4 + t) * 16);
               // code bytes are offset-binary (q + 128)
@@ -569,7 +490,7 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
                   A[ks][1] = hsub2(prmt(w8[2 * e + ks], kByte64x4, 0x4140u), kHalf2_1152);
                   A[ks][3] = hsub2(prmt(w8[2 * e + ks], kByte64x4, 0x4342u), kHalf2_1152);
                 }
-                block_qk(2 * pp + e, A);
+                block_qk(2 * P + e, A);
               }
             }
           } else {
@@ -579,37 +500,21 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
             // 1024 + 16q).  5-bit keys: the fifth bits of the lane's four blocks of one token
             // sit in one word, channel (c, i) at bit 16(i%2) + 4c + i/2, and are shifted to bit 4
             // or bit 8 of each half.  The code (minus 8 for Q4_0, 16 for Q5_0) is exact in f16.
-            // A warp with two blocks of a block quad reads their two words, at word c0 = blk0 % 4,
-            // and shifts the fifth-bit word right by 4 c0 so that its blocks sit at c = 0, 1.
-            constexpr int kWords = C::kNB < 4 ? C::kNB : 4;
-            const int c0 = blk0 & 3;
 #pragma unroll
-            for (int qq = 0; qq < (C::kNB + 3) / 4; ++qq) {
-              const int Q = blk0 / 4 + qq;
+            for (int Q = 0; Q < 2; ++Q) {
               const int row0 = (((G * 2 + Q) * 2 + 0) * 8 + g) * 4 + t;
               const int row1 = (((G * 2 + Q) * 2 + 1) * 8 + g) * 4 + t;
-              uint32_t wa[4], wc[4];
-              if constexpr (kWords == 4) {
-                const uint4 ka = lds128(kb + row0 * 16);
-                const uint4 kc = lds128(kb + row1 * 16);
-                wa[0] = ka.x; wa[1] = ka.y; wa[2] = ka.z; wa[3] = ka.w;
-                wc[0] = kc.x; wc[1] = kc.y; wc[2] = kc.z; wc[3] = kc.w;
-              } else {
-                asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(wa[0]), "=r"(wa[1]) : "r"(kb + row0 * 16 + 4 * c0));
-                asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(wc[0]), "=r"(wc[1]) : "r"(kb + row1 * 16 + 4 * c0));
-                wa[2] = wa[3] = wc[2] = wc[3] = 0u;
-              }
+              const uint4 ka = lds128(kb + row0 * 16);
+              const uint4 kc = lds128(kb + row1 * 16);
+              const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
+              const uint32_t wc[4] = {kc.x, kc.y, kc.z, kc.w};
               uint32_t xa5 = 0, xc5 = 0;
               if constexpr (C::kK5) {
                 xa5 = lds32(kb + kK5HighOffset + row0 * 4);
                 xc5 = lds32(kb + kK5HighOffset + row1 * 4);
-                if constexpr (kWords < 4) {
-                  xa5 >>= 4 * c0;
-                  xc5 >>= 4 * c0;
-                }
               }
 #pragma unroll
-              for (int c = 0; c < kWords; ++c) {
+              for (int c = 0; c < 4; ++c) {
                 uint32_t A[2][4];
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks) {
@@ -635,48 +540,9 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
                                      kAddHi);
                   }
                 }
-                block_qk(4 * qq + c, A);
+                block_qk(4 * Q + c, A);
               }
             }
-          }
-          if constexpr (SPLIT > 1) {
-            // exchange partial scores with the other warps of the group (the other channel
-            // blocks); every warp adds the SPLIT parts in the same order (its own part from its
-            // registers), so all of them hold bit-identical sums
-            auto slot = [&](int q) { return xbuf + ((((grp * SPLIT + q) * 2 + xpar) * NT) * 32) * 4; };
-            float* mine = slot(part);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-              *reinterpret_cast<float4*>(mine + (nt * 32 + lane) * 4) =
-                  make_float4(sacc[nt][0], sacc[nt][1], sacc[nt][2], sacc[nt][3]);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&xbar[grp]);
-            if (!mbar_wait(&xbar[grp], xphase)) {
-              s_flags[0] = 1;
-              aborted = true;
-              break;
-            }
-            xphase ^= 1;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-              for (int q = 0; q < SPLIT; ++q) {
-                float4 o;
-                if (q == part) {
-                  o = make_float4(sacc[nt][0], sacc[nt][1], sacc[nt][2], sacc[nt][3]);
-                } else {
-                  o = *reinterpret_cast<const float4*>(slot(q) + (nt * 32 + lane) * 4);
-                }
-                if (q == 0) {
-                  acc = o;
-                } else {
-                  acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
-                }
-              }
-              sacc[nt][0] = acc.x; sacc[nt][1] = acc.y; sacc[nt][2] = acc.z; sacc[nt][3] = acc.w;
-            }
-            xpar ^= 1;
           }
           // ---------------- online softmax (base 2) ----------------
           // The running maximum m_run of a row is shared by the 8 lanes that hold the row.
@@ -684,76 +550,69 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
           // cross-lane maximum is computed only when some lane sees a score above
           // m_run + 8: one warp vote per tile instead of three shuffles per row.
           const int key0 = logical * kPageTokens + 16 * G + g;  // rows e<2: token g, e>=2: g+8
-          float sv[NT][4], lm[NT][2];
+          float sv[4], lm[2];
           bool need = false;
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
+          for (int e = 0; e < 4; ++e) {
+            sv[e] = sacc[e] * crow[e & 1];
+            if (need_mask && key0 + 8 * (e >> 1) > qpos_row[e & 1]) sv[e] = -INFINITY;
+          }
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              sv[nt][e] = sacc[nt][e] * crow[nt][e & 1];
-              if (need_mask && key0 + 8 * (e >> 1) > qpos_row[nt][e & 1]) sv[nt][e] = -INFINITY;
-            }
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              lm[nt][c] = fmaxf(sv[nt][c], sv[nt][c + 2]);
-              need |= lm[nt][c] > m_run[nt][c] + 8.f;
-            }
+          for (int c = 0; c < 2; ++c) {
+            lm[c] = fmaxf(sv[c], sv[c + 2]);
+            need |= lm[c] > m_run[c] + 8.f;
           }
           if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+            for (int c = 0; c < 2; ++c) {
+              float mx = lm[c];
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+              if (mx > m_run[c] + 8.f) {
+                const float alpha = fast_exp2(m_run[c] - mx);  // 0 when m_run = -inf
+                l_run[c] *= alpha;
 #pragma unroll
-              for (int c = 0; c < 2; ++c) {
-                float mx = lm[nt][c];
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                if (mx > m_run[nt][c] + 8.f) {
-                  const float alpha = fast_exp2(m_run[nt][c] - mx);  // 0 when m_run = -inf
-                  l_run[nt][c] *= alpha;
-#pragma unroll
-                  for (int mt = 0; mt < 2 * C::kNB; ++mt) {
-                    oacc[mt][nt][c] *= alpha;
-                    oacc[mt][nt][c + 2] *= alpha;
-                  }
-                  if constexpr (C::kVMin) {
-#pragma unroll
-                    for (int bl = 0; bl < C::kNB; ++bl) {
-                      macc[bl][nt][c] *= alpha;
-                      macc[bl][nt][c + 2] *= alpha;
-                    }
-                  }
-                  m_run[nt][c] = mx;
+                for (int mt = 0; mt < 2 * C::kNB; ++mt) {
+                  oacc[mt][c] *= alpha;
+                  oacc[mt][c + 2] *= alpha;
                 }
+                if constexpr (C::kVMin) {
+#pragma unroll
+                  for (int bl = 0; bl < C::kNB; ++bl) {
+                    macc[bl][c] *= alpha;
+                    macc[bl][c + 2] *= alpha;
+                  }
+                }
+                m_run[c] = mx;
               }
+            }
           }
           // P as f16 high and low parts, transposed in registers into B fragments
-          uint32_t pbh[NT][2], pbl[NT][2];
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
+          uint32_t pbh[2], pbl[2];
+          {
             float pr[4];
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-              const float mu = m_run[nt][c] == -INFINITY ? 0.f : m_run[nt][c];
-              pr[c] = fast_exp2(sv[nt][c] - mu);
-              pr[c + 2] = fast_exp2(sv[nt][c + 2] - mu);
-              l_run[nt][c] += pr[c] + pr[c + 2];
+              const float mu = m_run[c] == -INFINITY ? 0.f : m_run[c];
+              pr[c] = fast_exp2(sv[c] - mu);
+              pr[c + 2] = fast_exp2(sv[c + 2] - mu);
+              l_run[c] += pr[c] + pr[c + 2];
             }
             uint32_t h01, l01, h23, l23;
             split_pair(pr[0], pr[1], h01, l01);
             split_pair(pr[2], pr[3], h23, l23);
-            pbh[nt][0] = movmatrix_t(h01);
-            pbh[nt][1] = movmatrix_t(h23);
-            pbl[nt][0] = movmatrix_t(l01);
-            pbl[nt][1] = movmatrix_t(l23);
+            pbh[0] = movmatrix_t(h01);
+            pbh[1] = movmatrix_t(h23);
+            pbl[0] = movmatrix_t(l01);
+            pbl[1] = movmatrix_t(l23);
           }
           // ---------------- O^T += V^T P^T ----------------
           // V codes enter the MMA exactly; the per-token block scale multiplies P (as a high
           // and a low f16 part), two MMAs per 16-dimension half.
           if constexpr (VF != kValQ8) {
 #pragma unroll
-            for (int cc = 0; cc < C::kNB / 2; ++cc) {
-              const int Cc = blk0 / 2 + cc;
+            for (int Cc = 0; Cc < C::kNB / 2; ++Cc) {
               const uint4 vw = lds128(vb + ((((G * 4 + Cc) * 8 + g) * 4 + t) * 16));
               const uint32_t sidx = vb + C::kVScaleOff + (((G * 4 + t) * 8 + 2 * Cc) * 4) * 2;
               const uint4 dv = lds128(sidx);
@@ -761,7 +620,7 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
               if constexpr (C::kVMin) mv = lds128(sidx + (kV41MinOffset - kV4ScaleOffset));
 #pragma unroll
               for (int e = 0; e < 2; ++e) {
-                const int bl = 2 * cc + e;
+                const int bl = 2 * Cc + e;
                 const uint32_t W0 = e ? vw.z : vw.x, W1 = e ? vw.w : vw.y;
                 const uint32_t d0 = e ? dv.z : dv.x, d1 = e ? dv.w : dv.y;
                 const uint32_t W0s = W0 >> 8, W1s = W1 >> 8;
@@ -776,32 +635,28 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
                 const uint32_t a11 = hfma2(and_or(W0s, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kAddHi);
                 const uint32_t a12 = hsub2(and_or(W1s, 0x000F000Fu, kHalf2Magic), kSubLo);
                 const uint32_t a13 = hfma2(and_or(W1s, 0x00F000F0u, kHalf2Magic), kHalf2_1_16, kAddHi);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                  uint32_t bh0, bl0, bh1, bl1;
-                  split_scaled(pbh[nt][0], pbl[nt][0], d0, bh0, bl0);
-                  split_scaled(pbh[nt][1], pbl[nt][1], d1, bh1, bl1);
-                  mma_f16(oacc[2 * bl][nt], a00, a01, a02, a03, bh0, bh1);
-                  mma_f16(oacc[2 * bl][nt], a00, a01, a02, a03, bl0, bl1);
-                  mma_f16(oacc[2 * bl + 1][nt], a10, a11, a12, a13, bh0, bh1);
-                  mma_f16(oacc[2 * bl + 1][nt], a10, a11, a12, a13, bl0, bl1);
-                  if constexpr (C::kVMin) {
-                    // sum over the tile's tokens of p * m, the same for every dimension of the
-                    // block: an all-ones A operand
-                    const uint32_t m0 = e ? mv.z : mv.x, m1 = e ? mv.w : mv.y;
-                    uint32_t mh0, ml0, mh1, ml1;
-                    split_scaled(pbh[nt][0], pbl[nt][0], m0, mh0, ml0);
-                    split_scaled(pbh[nt][1], pbl[nt][1], m1, mh1, ml1);
-                    mma_f16(macc[bl][nt], kHalf2_One, kHalf2_One, kHalf2_One, kHalf2_One, mh0, mh1);
-                    mma_f16(macc[bl][nt], kHalf2_One, kHalf2_One, kHalf2_One, kHalf2_One, ml0, ml1);
-                  }
+                uint32_t bh0, bl0, bh1, bl1;
+                split_scaled(pbh[0], pbl[0], d0, bh0, bl0);
+                split_scaled(pbh[1], pbl[1], d1, bh1, bl1);
+                mma_f16(oacc[2 * bl], a00, a01, a02, a03, bh0, bh1);
+                mma_f16(oacc[2 * bl], a00, a01, a02, a03, bl0, bl1);
+                mma_f16(oacc[2 * bl + 1], a10, a11, a12, a13, bh0, bh1);
+                mma_f16(oacc[2 * bl + 1], a10, a11, a12, a13, bl0, bl1);
+                if constexpr (C::kVMin) {
+                  // sum over the tile's tokens of p * m, the same for every dimension of the
+                  // block: an all-ones A operand
+                  const uint32_t m0 = e ? mv.z : mv.x, m1 = e ? mv.w : mv.y;
+                  uint32_t mh0, ml0, mh1, ml1;
+                  split_scaled(pbh[0], pbl[0], m0, mh0, ml0);
+                  split_scaled(pbh[1], pbl[1], m1, mh1, ml1);
+                  mma_f16(macc[bl], kHalf2_One, kHalf2_One, kHalf2_One, kHalf2_One, mh0, mh1);
+                  mma_f16(macc[bl], kHalf2_One, kHalf2_One, kHalf2_One, kHalf2_One, ml0, ml1);
                 }
               }
             }
           } else {
 #pragma unroll
-            for (int bl = 0; bl < C::kNB; ++bl) {
-              const int b = blk0 + bl;
+            for (int b = 0; b < C::kNB; ++b) {
               const uint4 vw = lds128(vb + ((((G * 8 + b) * 8 + g) * 4 + t) * 16));
               uint32_t d0, d1;
               asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
@@ -814,24 +669,20 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
                 a[q][0] = hsub2(prmt(w[q], kByte64x4, 0x4140u), kHalf2_1152);
                 a[q][1] = hsub2(prmt(w[q], kByte64x4, 0x4342u), kHalf2_1152);
               }
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) {
-                uint32_t bh0, bl0, bh1, bl1;
-                split_scaled(pbh[nt][0], pbl[nt][0], d0, bh0, bl0);
-                split_scaled(pbh[nt][1], pbl[nt][1], d1, bh1, bl1);
-                mma_f16(oacc[2 * bl][nt], a[0][0], a[0][1], a[1][0], a[1][1], bh0, bh1);
-                mma_f16(oacc[2 * bl][nt], a[0][0], a[0][1], a[1][0], a[1][1], bl0, bl1);
-                mma_f16(oacc[2 * bl + 1][nt], a[2][0], a[2][1], a[3][0], a[3][1], bh0, bh1);
-                mma_f16(oacc[2 * bl + 1][nt], a[2][0], a[2][1], a[3][0], a[3][1], bl0, bl1);
-              }
+              uint32_t bh0, bl0, bh1, bl1;
+              split_scaled(pbh[0], pbl[0], d0, bh0, bl0);
+              split_scaled(pbh[1], pbl[1], d1, bh1, bl1);
+              mma_f16(oacc[2 * b], a[0][0], a[0][1], a[1][0], a[1][1], bh0, bh1);
+              mma_f16(oacc[2 * b], a[0][0], a[0][1], a[1][0], a[1][1], bl0, bl1);
+              mma_f16(oacc[2 * b + 1], a[2][0], a[2][1], a[3][0], a[3][1], bh0, bh1);
+              mma_f16(oacc[2 * b + 1], a[2][0], a[2][1], a[3][0], a[3][1], bl0, bl1);
             }
           }
         }
       }
-      if (aborted) break;
       __syncwarp();
       if (lane == 0) {
-        if (atomicAdd(&rel_cnt[s], 1) == (tile_hi(i) - tile_lo(i)) * SPLIT - 1) {
+        if (atomicAdd(&rel_cnt[s], 1) == (tile_hi(i) - tile_lo(i)) * NT - 1) {
           rel_cnt[s] = 0;
           if (i + C::kStages < count) issue(i + C::kStages);
         }
@@ -839,15 +690,13 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
     }
     // reduce the per-thread partial sums over the 8 token lanes
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float l = l_run[nt][c];
-        l += __shfl_xor_sync(0xffffffffu, l, 4);
-        l += __shfl_xor_sync(0xffffffffu, l, 8);
-        l += __shfl_xor_sync(0xffffffffu, l, 16);
-        l_run[nt][c] = l;
-      }
+    for (int c = 0; c < 2; ++c) {
+      float l = l_run[c];
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      l_run[c] = l;
+    }
   }
 
   __syncthreads();
@@ -867,34 +716,30 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
   }
 
   // ---------------- merge the CTA's softmax streams in shared memory ----------------
-  // layout: ms[unit][row], ls[unit][row], os[unit][row][kOStride]  (all fp32)
+  // one stream per warp, over the 8 rows of its n-tile (local row lr = row % 8):
+  // ms[warp][lr], ls[warp][lr], os[warp][lr][kOStride]  (all fp32)
   float* ms = reinterpret_cast<float*>(smem);
-  float* ls = ms + C::kUnits * C::kRowsPad;
-  float* os = ls + C::kUnits * C::kRowsPad;
+  float* ls = ms + C::kConsumerWarps * 8;
+  float* os = ls + C::kConsumerWarps * 8;
   {
-    const int unit = SPLIT > 1 ? grp : warp;
-    if (g == 0 && part == 0) {
+    if (g == 0) {
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          ms[unit * C::kRowsPad + nt * 8 + 2 * t + c] = m_run[nt][c];
-          ls[unit * C::kRowsPad + nt * 8 + 2 * t + c] = l_run[nt][c];
-        }
+      for (int c = 0; c < 2; ++c) {
+        ms[warp * 8 + 2 * t + c] = m_run[c];
+        ls[warp * 8 + 2 * t + c] = l_run[c];
+      }
     }
 #pragma unroll
     for (int mt = 0; mt < 2 * C::kNB; ++mt) {
-      const int b = blk0 + (mt >> 1), hb = mt & 1;
+      const int b = mt >> 1, hb = mt & 1;
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int row = nt * 8 + 2 * t + (e & 1);
-          const int dim = 32 * b + 16 * hb + g + 8 * (e >> 1);
-          float v = oacc[mt][nt][e];
-          if constexpr (C::kVMin) v += macc[mt >> 1][nt][e];
-          os[(unit * C::kRowsPad + row) * C::kOStride + dim] = v;
-        }
+      for (int e = 0; e < 4; ++e) {
+        const int lr = 2 * t + (e & 1);
+        const int dim = 32 * b + 16 * hb + g + 8 * (e >> 1);
+        float v = oacc[mt][e];
+        if constexpr (C::kVMin) v += macc[mt >> 1][e];
+        os[(warp * 8 + lr) * C::kOStride + dim] = v;
+      }
     }
   }
   __syncthreads();
@@ -905,17 +750,19 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT, SPLIT>::kThreads, 1) dec
   for (int idx = threadIdx.x; idx < n_rows * (kHeadDim / 4); idx += C::kThreads) {
     const int row = idx / (kHeadDim / 4);
     const int d4 = (idx % (kHeadDim / 4)) * 4;
+    // the streams that hold this row: the warps of its n-tile (warp = n-tile + NT x group)
+    const int lr = row % 8;
     float M = -INFINITY;
 #pragma unroll
-    for (int u = 0; u < C::kUnits; ++u) M = fmaxf(M, ms[u * C::kRowsPad + row]);
+    for (int u = row / 8; u < C::kConsumerWarps; u += NT) M = fmaxf(M, ms[u * 8 + lr]);
     float L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (M != -INFINITY) {
 #pragma unroll
-      for (int u = 0; u < C::kUnits; ++u) {
-        const float w = fast_exp2(ms[u * C::kRowsPad + row] - M);
-        L += w * ls[u * C::kRowsPad + row];
-        const float4 o = *reinterpret_cast<const float4*>(os + (u * C::kRowsPad + row) * C::kOStride + d4);
+      for (int u = row / 8; u < C::kConsumerWarps; u += NT) {
+        const float w = fast_exp2(ms[u * 8 + lr] - M);
+        L += w * ls[u * 8 + lr];
+        const float4 o = *reinterpret_cast<const float4*>(os + (u * 8 + lr) * C::kOStride + d4);
         acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
       }
     }
@@ -1036,9 +883,9 @@ cudaError_t launch_decode_merge(const DecodeParams& prm, int n_kv, cudaStream_t 
                             decode_rows_pad(prm.group * prm.n_q), prm.group, prm.n_qh, prm.out, prm.lse);
 }
 
-template <int KF, int VF, int NT, int SPLIT>
+template <int KF, int VF, int NT>
 static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream_t stream) {
-  using C = DecodeCfg<KF, VF, NT, SPLIT>;
+  using C = DecodeCfg<KF, VF, NT>;
   // programmatic dependent launch: the grid may start while the previous kernel on the
   // stream drains; the kernel waits for it (griddepcontrol.wait) before reading any input
   cudaLaunchConfig_t cfg = {};
@@ -1051,7 +898,7 @@ static cudaError_t launch_decode_t(const DecodeParams& prm, int n_kv, cudaStream
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<KF, VF, NT, SPLIT>, prm);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<KF, VF, NT>, prm);
 }
 
 // The supported (key, value) format pairs: Q8_0 keys with Q4_0 or Q8_0 values, Q4_0 and Q5_1
@@ -1069,11 +916,11 @@ bool decode_pair_supported(int key_fmt, int val_fmt) {
 
 cudaError_t prepare_decode_kernels() {
   cudaError_t e;
-#define KV_SET1(KF, VF, NT, SPLIT)                                                                   \
-  e = cudaFuncSetAttribute(decode_kernel<KF, VF, NT, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                           DecodeCfg<KF, VF, NT, SPLIT>::kSmemBytes);                               \
+#define KV_SET1(KF, VF, NT)                                                                   \
+  e = cudaFuncSetAttribute(decode_kernel<KF, VF, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                           DecodeCfg<KF, VF, NT>::kSmemBytes);                               \
   if (e != cudaSuccess) return e;
-#define KV_SET(KF, VF) KV_SET1(KF, VF, 1, 1) KV_SET1(KF, VF, 2, 2) KV_SET1(KF, VF, 3, 2)
+#define KV_SET(KF, VF) KV_SET1(KF, VF, 1) KV_SET1(KF, VF, 2) KV_SET1(KF, VF, 3)
   KVATTN_DECODE_PAIRS(KV_SET)
 #undef KV_SET
 #undef KV_SET1
@@ -1082,9 +929,9 @@ cudaError_t prepare_decode_kernels() {
 
 template <int KF, int VF>
 static cudaError_t launch_decode_fmt(const DecodeParams& prm, int n_kv, int nt, cudaStream_t stream) {
-  if (nt == 1) return launch_decode_t<KF, VF, 1, 1>(prm, n_kv, stream);
-  if (nt == 2) return launch_decode_t<KF, VF, 2, 2>(prm, n_kv, stream);
-  return launch_decode_t<KF, VF, 3, 2>(prm, n_kv, stream);
+  if (nt == 1) return launch_decode_t<KF, VF, 1>(prm, n_kv, stream);
+  if (nt == 2) return launch_decode_t<KF, VF, 2>(prm, n_kv, stream);
+  return launch_decode_t<KF, VF, 3>(prm, n_kv, stream);
 }
 
 cudaError_t launch_decode(const DecodeParams& prm, int n_kv, int key_fmt, int val_fmt, cudaStream_t stream) {
