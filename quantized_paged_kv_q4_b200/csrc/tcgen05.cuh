@@ -8,22 +8,9 @@
 namespace kvattn {
 namespace tc {
 
-// Allocates `ncols` tensor-memory columns (power of two >= 32); the whole warp must call it.
-// The base address is written to *dst_smem.
-__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
-               "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-// The same for a CTA pair (cta_group::2): one warp with the same warp index in each of the two
-// CTAs of the cluster calls it; both get the same columns of their own tensor memory.
+// Allocates `ncols` tensor-memory columns (power of two >= 32) for a CTA pair (cta_group::2):
+// one warp with the same warp index in each of the two CTAs of the cluster calls it; both get
+// the same columns of their own tensor memory, and the base address is written to *dst_smem.
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
                "r"(ncols)
@@ -42,32 +29,6 @@ __device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence
 // Makes this thread's generic-proxy shared-memory writes visible to the tensor core.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// D[tmem] (+)= A[smem desc] * B[smem desc]; issued by one thread.
-__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                           uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem desc], executed by a whole converged warp: one lane, picked
-// by elect.sync, issues the instruction.  Issuing from a converged warp keeps the operands
-// warp-uniform; a loop run by a single lane issues several times slower when other warps
-// share its scheduler.
-__device__ __forceinline__ void mma_f16_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                                uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred e, p;\n\t.reg .b32 r;\n\t"
-      "elect.sync r|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
 }
 
 // CTA-pair MMA (cta_group::2, issued by the even CTA of the cluster for both): D rows
@@ -96,33 +57,6 @@ __device__ __forceinline__ void commit_pair2_warp(uint64_t* bar) {
       "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
           smem_u32(bar))
       : "memory");
-}
-
-// tcgen05.commit (below) from a converged warp, issued by one elected lane.
-__device__ __forceinline__ void commit_warp(uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
-      "elect.sync r|e, 0xffffffff;\n\t"
-      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
-      : "memory");
-}
-
-// commit_warp to the barrier at the same shared-memory offset in both CTAs of a cluster of
-// two (the signal reaches this CTA and its peer).
-__device__ __forceinline__ void commit_pair_warp(uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t.reg .b16 m;\n\t"
-      "mov.b16 m, 3;\n\t"
-      "elect.sync r|e, 0xffffffff;\n\t"
-      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
-          smem_u32(bar))
-      : "memory");
-}
-
-// Arrives once on `bar` when all previously issued tcgen05.mma of this thread complete.
-__device__ __forceinline__ void commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
 }
 
 // 32 lanes x 32 bit, 32 consecutive columns starting at taddr (warp-collective).
