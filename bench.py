@@ -384,12 +384,12 @@ class PrefillBench:
     16 layers x 4 KV heads, 4,096-token KV splits.  One step = for every layer: append the
     chunk's K/V, then the four ubatch prefill calls."""
 
-    def __init__(self, kv, device, layers=0, context=0):
+    def __init__(self, kv, device, layers=0, context=0, wname="prefill524k"):
         import dataclasses
 
         import torch
 
-        w = WORKLOADS["prefill524k"]
+        w = WORKLOADS[wname]
         if layers:
             w = dataclasses.replace(w, layers=layers)
         if context:
@@ -1094,6 +1094,17 @@ def main():
                                     "peak": f"{peak_kind} dense bf16 (f16 operands run at the same rate)"}
             del b4
             torch.cuda.empty_cache()
+            # the same prefill layer over Q4_0 and Q5_1 keys (one layer: kernel rate only)
+            for wn in ("prefill524k_q4q4", "prefill524k_q51q4"):
+                b6 = PrefillBench(kvattn, device, layers=1, wname=wn)
+                b6.layer(0)
+                k6 = time_layers(b6, 2)
+                tf6 = b6.flops_per_layer / (k6 * 1e-3) / 1e12
+                extra[wn] = {"kernel_TFLOP/s": tf6, "kernel_frac_bf16": tf6 / bf16, "layer_ms": k6,
+                             "executed_frac_bf16": tf6 * b6.mma_work_factor / bf16,
+                             "k_fmt": b6.w.k_fmt, "v_fmt": b6.w.v_fmt}
+                del b6
+                torch.cuda.empty_cache()
             b5 = StreamBench(kvattn, device)
             n_gen = args.stream_steps or b5.w.steps
             ts, tr, tcp, td = time_stream(b5, n_gen, 2)

@@ -1,8 +1,9 @@
-// Chunked prefill over block-quantized KV pages (Q8_0 or Q4_0 keys, Q4_0 values) on
+// Chunked prefill over block-quantized KV pages (Q8_0, Q4_0 or Q5_1 keys, Q4_0 values) on
 // tcgen05 tensor cores (Adaptive KV Streaming + RDNA 4 announcement, wqu.guru, method list:
 // "online log-sum-exp prefill": the prefill of a chunk is computed across streamed KV pages
 // and the partial results are accumulated by online log-sum-exp; the six-step validation
-// guide, alphalab.site, build step: the q8_0-q4_0 and q4_0-q4_0 flash-attention KV pairs).
+// guide, alphalab.site, build step: the q8_0-q4_0 and q4_0-q4_0 flash-attention KV pairs;
+// Vulkan speculative-decoding report, lcz.me/topic/1398, pitfalls: the K q5_1 / V q4_0 cache).
 //
 // Work unit: a cluster of two CTAs = a KV head, two M-tiles of 128 query rows of that head's
 // group (row r = token t * group + j: all query heads of a group share the K/V tiles), and
@@ -16,7 +17,9 @@
 //                         into a two-stage shared-memory ring
 //   dequant warps (8)     raw -> K^ and V^T, each as an f16 high part (code x scale rounded
 //                         once) and an f16 low part (the remainder, exact): together the
-//                         dequantized values exactly; K-major, 128-byte swizzle, three deep
+//                         dequantized values exactly (Q5_1 keys, code x scale + minimum:
+//                         to the one fp32 rounding of the sum); K-major, 128-byte swizzle,
+//                         three deep
 //   MMA issuer (1 warp,   S = Q K^T (N = 64 keys, K = 256) as Q K^_hi^T + Q K^_lo^T, and
 //     even CTA only)      O += P V (N = 256 dims, K = 64 keys) as P_hi V^_hi + P_lo V^_hi +
 //                         P_hi V^_lo; Q and P from tensor memory
@@ -60,16 +63,24 @@ constexpr int kLoadWarp = 5;
 constexpr int kDequantWarps = 8;  // warps 6-13
 constexpr int kThreads = (kSoftmaxWarps + 2 + kDequantWarps) * 32;
 constexpr int kDq0 = (kSoftmaxWarps + 2) * 32;  // first dequant thread
-// raw bytes a CTA copies per 64-key tile: K codes and scales of its 32 keys (contiguous in
-// the page), V codes of its 128 head dimensions for all 64 keys (four 1 KB pieces, one per
-// 16-key group), and all V scales of the tile
+// raw bytes a CTA copies per 64-key tile: K codes (Q5_1: low nibbles, then fifth bits),
+// scales (Q5_1: then minima) of its 32 keys (each region contiguous in the page), V codes of
+// its 128 head dimensions for all 64 keys (four 1 KB pieces, one per 16-key group), and all
+// V scales of the tile; the stage holds them in that order
 template <int KF>
 struct Raw {
-  static constexpr int kKc = KF == kKeyQ4 ? 4096 : 8192;  // 32 keys x 128 or 256 bytes
+  static constexpr int kKc = KF == kKeyQ8 ? 8192 : 4096;  // 32 keys x 256 or 128 bytes
+  static constexpr int kKh = KF == kKeyQ51 ? 1024 : 0;    // fifth bits: 32 keys x 32 bytes
   static constexpr int kKs = 512, kVc = 4096, kVs = 1024;
-  static constexpr int kBytes = kKc + kKs + kVc + kVs;
+  static constexpr int kKm = KF == kKeyQ51 ? 512 : 0;     // minima
+  static constexpr int kKhOff = kKc, kKsOff = kKhOff + kKh, kKmOff = kKsOff + kKs;
+  static constexpr int kVcOff = kKmOff + kKm, kVsOff = kVcOff + kVc;
+  static constexpr int kBytes = kVsOff + kVs;
+  // the regions' offsets in a K page
+  static constexpr int kPageScaleOff = KF == kKeyQ8 ? kKScaleOffset : KF == kKeyQ4 ? kK4ScaleOffset : kK5ScaleOffset;
 };
-constexpr int kRawStageBytes = Raw<kKeyQ8>::kBytes;  // 13,824 (the larger layout)
+constexpr int kRawStageBytes = Raw<kKeyQ8>::kBytes;  // 13,824 (the largest layout)
+static_assert(Raw<kKeyQ51>::kBytes <= kRawStageBytes && Raw<kKeyQ4>::kBytes <= kRawStageBytes, "raw stage");
 constexpr int kRawStages = 2;
 constexpr int kBufs = 3;          // K^ / V^T buffer sets: dequant runs up to two tiles ahead of the MMAs
 constexpr int kPart = 16384;      // one of K^_hi, K^_lo (4 atoms x [32 keys][128 B]), V^T_hi, V^T_lo ([128][128 B])
@@ -238,6 +249,18 @@ __device__ __forceinline__ void split_product(uint32_t code, uint32_t d, uint32_
   lo = hfma2(code, d, hi ^ 0x80008000u);
 }
 
+// The same split of an affine dequantization q * d + m (Q5_1 keys): q * d is exact in fp32
+// (q has at most 5 significant bits, d 11) and the sum is rounded once to fp32; hi = f16 of
+// it and lo = f16 of the exact fp32 remainder carry it to about 22 significant bits.
+__device__ __forceinline__ void split_affine(uint32_t code, float d, float m, uint32_t& hi, uint32_t& lo) {
+  const float v0 = fmaf(half_lo(code), d, m), v1 = fmaf(half_hi(code), d, m);
+  hi = pack_half2(v0, v1);
+  lo = pack_half2(v0 - half_lo(hi), v1 - half_hi(hi));
+}
+
+// x shifted left by s bits (right by -s when s < 0); s is a compile-time constant after unrolling.
+__device__ __forceinline__ uint32_t shl(uint32_t x, int s) { return s >= 0 ? x << s : x >> -s; }
+
 template <int KF>
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillParams p) {
   using RawF = pf::Raw<KF>;
@@ -344,15 +367,16 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         uint8_t* st = smem + pf::kRawOff + r * pf::kRawStageBytes;
         const uint8_t* kp = p.k_pool + static_cast<int64_t>(tl.x) * p.k_stride;
         const uint8_t* vp = p.v_pool + static_cast<int64_t>(tl.x) * p.v_stride;
-        constexpr int kScaleOff = KF == kKeyQ4 ? kK4ScaleOffset : kKScaleOffset;
         mbar_arrive_expect_tx(&rawfull[r], RawF::kBytes);
         bulk_g2s(st, kp + q * RawF::kKc, RawF::kKc, &rawfull[r]);
-        bulk_g2s(st + RawF::kKc, kp + kScaleOff + q * RawF::kKs, RawF::kKs, &rawfull[r]);
+        if constexpr (RawF::kKh > 0)
+          bulk_g2s(st + RawF::kKhOff, kp + kK5HighOffset + q * RawF::kKh, RawF::kKh, &rawfull[r]);
+        bulk_g2s(st + RawF::kKsOff, kp + RawF::kPageScaleOff + q * RawF::kKs, RawF::kKs, &rawfull[r]);
+        if constexpr (RawF::kKm > 0)
+          bulk_g2s(st + RawF::kKmOff, kp + kK5MinOffset + q * RawF::kKm, RawF::kKm, &rawfull[r]);
         for (int g = 0; g < 4; ++g)
-          bulk_g2s(st + RawF::kKc + RawF::kKs + g * 1024, vp + half * 8192 + g * 2048 + crank * 1024, 1024,
-                   &rawfull[r]);
-        bulk_g2s(st + RawF::kKc + RawF::kKs + RawF::kVc, vp + kV4ScaleOffset + half * RawF::kVs, RawF::kVs,
-                 &rawfull[r]);
+          bulk_g2s(st + RawF::kVcOff + g * 1024, vp + half * 8192 + g * 2048 + crank * 1024, 1024, &rawfull[r]);
+        bulk_g2s(st + RawF::kVsOff, vp + kV4ScaleOffset + half * RawF::kVs, RawF::kVs, &rawfull[r]);
       }
       // every copy issued must land before the CTA may exit
       for (int jj = j - pf::kRawStages < 0 ? 0 : j - pf::kRawStages; jj < j; ++jj)
@@ -602,19 +626,23 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       const uint32_t stu = own + pf::kRawOff + r * pf::kRawStageBytes;
       // ---------------- raw K, V -> registers; the stage is then released ----------------
       uint32_t kw[2][4] = {};  // per chunk i: the 4 words (8 codes of block 2kP, 8 of 2kP + 1)
-      uint32_t dkw = 0;
+      uint32_t kh[2] = {};     // Q5_1: per chunk i, the fifth bits of blocks 2kP, 2kP + 1 at bits 0-7, 16-23
+      uint32_t dkw = 0, mkw = 0;
       uint2 vraw[4] = {}, dvr[4] = {};
       if (wok) {
-        if constexpr (KF == kKeyQ4) {
-          // Q4_0 key words of token kl, blocks 2kP, 2kP + 1 (c = 2kP % 4, 2kP % 4 + 1) of block
-          // quad Q = kP / 2, lane column T: one 8-byte load per chunk
+        if constexpr (KF != kKeyQ8) {
+          // 4-bit key words (Q5_1: the low nibbles) of token kl, blocks 2kP, 2kP + 1 (c = 2kP % 4,
+          // 2kP % 4 + 1) of block quad Q = kP / 2, lane column T: one 8-byte load per chunk.
+          // Q5_1: the word of fifth bits of (token, Q, T) holds block c at bits 4c + (0..3) of
+          // each half; shifting it right by 4 * (2kP % 4) brings blocks 2kP, 2kP + 1 to bits 0-7.
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             const int T = (2 * cp + i + rotK) & 3;
-            const uint2 w2 =
-                lds64(stu + 4 * (((((kGl * 2 + (kP >> 1)) * 2 + kH) * 8 + kR) * 4 + T) * 4 + ((2 * kP) & 3)));
+            const int row = (((kGl * 2 + (kP >> 1)) * 2 + kH) * 8 + kR) * 4 + T;
+            const uint2 w2 = lds64(stu + 4 * (row * 4 + ((2 * kP) & 3)));
             kw[i][0] = w2.x;
             kw[i][1] = w2.y;
+            if constexpr (KF == kKeyQ51) kh[i] = lds32(stu + RawF::kKhOff + 4 * row) >> (4 * ((2 * kP) & 3));
           }
         } else {
           const uint32_t kbase = stu + ((((kGl * 4 + kP) * 2 + kH) * 8 + kR) * 4) * 16;
@@ -624,17 +652,17 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
             kw[i][0] = c.x; kw[i][1] = c.y; kw[i][2] = c.z; kw[i][3] = c.w;
           }
         }
-        asm volatile("ld.shared.u32 %0, [%1];"
-                     : "=r"(dkw)
-                     : "r"(stu + RawF::kKc + ((kGl * 8 + kR) * 2 + kH) * 16 + 4 * kP));
+        // scales (Q5_1: and minima) of blocks 2kP, 2kP + 1 of token kl
+        const int sidx = ((kGl * 8 + kR) * 2 + kH) * 16 + 4 * kP;
+        dkw = lds32(stu + RawF::kKsOff + sidx);
+        if constexpr (KF == kKeyQ51) mkw = lds32(stu + RawF::kKmOff + sidx);
         // this thread's two words (block 2vC + ve, both key halves) of each raw chunk and of
         // the scales of each token pair
-        const uint32_t vbase = stu + RawF::kKc + RawF::kKs + vG * 1024 + ((vCl * 8 + vR) * 4) * 16 + 8 * ve;
+        const uint32_t vbase = stu + RawF::kVcOff + vG * 1024 + ((vCl * 8 + vR) * 4) * 16 + 8 * ve;
 #pragma unroll
         for (int ii = 0; ii < 4; ++ii) vraw[ii] = lds64(vbase + (((ii + rotV) & 3) << 4));
 #pragma unroll
-        for (int T = 0; T < 4; ++T)
-          dvr[T] = lds64(stu + RawF::kKc + RawF::kKs + RawF::kVc + ((vG * 4 + T) * 8 + 2 * vC) * 8 + 8 * ve);
+        for (int T = 0; T < 4; ++T) dvr[T] = lds64(stu + RawF::kVsOff + ((vG * 4 + T) * 8 + 2 * vC) * 8 + 8 * ve);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&rawempty[r]);
@@ -657,6 +685,22 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
               c[4 * e + 2] = hsub2(and_or(ws, 0x000F000Fu, 0x64006400u), 0x64086408u);
               c[4 * e + 3] = hfma2(and_or(ws, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
             }
+          } else if constexpr (KF == kKeyQ51) {
+            // as Q4_0, with the fifth bit (channel (e, i) at bit 4e + i / 2 + 16 (i % 2) of kh)
+            // moved to the 16s place of the code: bit 4 of the halves 1024 + q, bit 8 of the
+            // halves 1024 + 16q; the codes q in [0, 31] are exact in f16
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const uint32_t w = kw[i][e], ws = w >> 8, x = kh[i];
+              c[4 * e + 0] = hsub2(or_and(and_or(w, 0x000F000Fu, 0x64006400u), shl(x, 4 - 4 * e), 0x00100010u),
+                                   0x64006400u);
+              c[4 * e + 1] = hfma2(or_and(and_or(w, 0x00F000F0u, 0x64006400u), shl(x, 7 - 4 * e), 0x01000100u),
+                                   0x2C002C00u, 0xD400D400u);
+              c[4 * e + 2] = hsub2(or_and(and_or(ws, 0x000F000Fu, 0x64006400u), shl(x, 2 - 4 * e), 0x00100010u),
+                                   0x64006400u);
+              c[4 * e + 3] = hfma2(or_and(and_or(ws, 0x00F000F0u, 0x64006400u), shl(x, 5 - 4 * e), 0x01000100u),
+                                   0x2C002C00u, 0xD400D400u);
+            }
           } else {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -666,8 +710,15 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
             }
           }
           uint32_t oh[8], ol[8];
+          if constexpr (KF == kKeyQ51) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) split_product(c[e], e < 4 ? dlo : dhi, oh[e], ol[e]);
+            for (int e = 0; e < 8; ++e)
+              split_affine(c[e], e < 4 ? half_lo(dkw) : half_hi(dkw), e < 4 ? half_lo(mkw) : half_hi(mkw), oh[e],
+                           ol[e]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) split_product(c[e], e < 4 ? dlo : dhi, oh[e], ol[e]);
+          }
           sts128u(katom + swz(kl, T), oh[0], oh[1], oh[2], oh[3]);
           sts128u(katom + swz(kl, 4 + T), oh[4], oh[5], oh[6], oh[7]);
           sts128u(katom + pf::kPart + swz(kl, T), ol[0], ol[1], ol[2], ol[3]);
@@ -740,8 +791,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
 cudaError_t prepare_prefill_kernels() {
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel<kKeyQ8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        pf::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_kernel<kKeyQ4>, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::kSmemBytes);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(prefill_kernel<kKeyQ4>, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::kSmemBytes);
+  return cudaFuncSetAttribute(prefill_kernel<kKeyQ51>, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::kSmemBytes);
 }
 
 struct PrefillPlan {
@@ -788,8 +841,9 @@ cudaError_t launch_prefill(const PrefillParams& prm0, int n_kv, int key_fmt, cud
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = key_fmt == kKeyQ4 ? cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ4>, prm)
-                                      : cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ8>, prm);
+    cudaError_t e = key_fmt == kKeyQ4    ? cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ4>, prm)
+                    : key_fmt == kKeyQ51 ? cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ51>, prm)
+                                         : cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ8>, prm);
     if (e != cudaSuccess || prm.n_ks == 1) return e;
   }
   cudaLaunchConfig_t cfg = {};

@@ -46,7 +46,7 @@ def _case(seed, H, n_prior, n_q, outliers=True, k_fmt="q8_0"):
     return rng, k, v, q, cache, T
 
 
-@pytest.mark.parametrize("k_fmt", ["q8_0", "q4_0"])
+@pytest.mark.parametrize("k_fmt", ["q8_0", "q4_0", "q5_1"])
 @pytest.mark.parametrize("n_prior,n_q,split", [(700, 40, 256), (1024, 64, 128), (300, 22, 512), (5000, 130, 1024),
                                                (0, 30, 128), (127, 1, 256)])
 def test_prefill_matches_oracle(kv_gpu, n_prior, n_q, split, k_fmt):
