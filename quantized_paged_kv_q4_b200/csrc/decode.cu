@@ -104,7 +104,6 @@ constexpr uint32_t kHalf2_1_16 = 0x2C002C00u;  // 1/16
 constexpr uint32_t kHalf2_m72 = 0xD480D480u;   // -(64 + 8)
 constexpr uint32_t kHalf2_m64 = 0xD400D400u;   // -64
 constexpr uint32_t kHalf2_m80 = 0xD500D500u;   // -(64 + 16)
-constexpr uint32_t kHalf2_One = 0x3C003C00u;   // 1.0
 constexpr uint32_t kHalf2_Sign = 0x80008000u;
 
 // B operand (probabilities times a per-token fp16 factor f) as an unevaluated f16 sum hi + lo:
@@ -219,8 +218,9 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT>::kThreads, 1) decode_ker
   float m_run[2], l_run[2];
   float oacc[2 * C::kNB][4];
   // values with a zero point: sum over tokens of p * m per (block, query row), kept apart
-  // from oacc (every dimension of a block gets the same term) and added at the end
-  float macc[C::kVMin ? C::kNB : 1][4];
+  // from oacc (every dimension of a block gets the same term) and added at the end; an MMA
+  // accumulator with the 8 blocks as M (rows g: block g, rows g + 8 unused)
+  float racc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
     m_run[c] = -INFINITY;
@@ -230,10 +230,6 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT>::kThreads, 1) decode_ker
   for (int i = 0; i < 2 * C::kNB; ++i)
 #pragma unroll
     for (int e = 0; e < 4; ++e) oacc[i][e] = 0.f;
-#pragma unroll
-  for (int i = 0; i < (C::kVMin ? C::kNB : 1); ++i)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) macc[i][e] = 0.f;
 
   const int grp = warp / NT;  // the warps that share a tile, one per n-tile
   const int nt0 = warp % NT;  // this warp's n-tile: query rows 8 nt0 .. 8 nt0 + 7
@@ -309,9 +305,11 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT>::kThreads, 1) decode_ker
     // in shared memory for the n-tile's warps; crow[c] = amax / 16 * log2(e) turns a dot
     // product with the normalised row into a base-2 softmax score.
     float crow[2];
-    // zero-point keys: per block, the sum of the normalised query row's channels (for the
-    // query rows 2t, 2t + 1 of the n-tile)
-    float qsum[C::kKMin ? C::kNB : 1][2];
+    // zero-point keys: the sums over each block's channels of the normalised query row g of
+    // the n-tile, as the B fragment (k = block 2t, 2t + 1) of an MMA that adds
+    // sum_b m[token][b] qsum[b][row] to S, split into f16 high and low parts
+    uint32_t qsb_hi = 0u, qsb_lo = 0u;
+    float qs0 = 0.f, qs1 = 0.f;
     // query positions of this thread's accumulator rows, loaded first: every global read of
     // the setup is issued before any of them is used
     int qpos_row[2];
@@ -375,10 +373,11 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT>::kThreads, 1) decode_ker
           for (int e = 0; e < 8; ++e) sm += xv[e];
           sm += __shfl_xor_sync(0xffffffffu, sm, 1);
           sm += __shfl_xor_sync(0xffffffffu, sm, 2);
-          qsum[bl][0] = __shfl_sync(0xffffffffu, sm, (2 * t) * 4);
-          qsum[bl][1] = __shfl_sync(0xffffffffu, sm, (2 * t + 1) * 4);
+          if (bl == 2 * t) qs0 = sm;
+          if (bl == 2 * t + 1) qs1 = sm;
         }
       }
+      if constexpr (C::kKMin) split_pair(qs0, qs1, qsb_hi, qsb_lo);
       const float cr = amax * (1.0f / 16.0f) * 1.4426950408889634f;
       crow[0] = __shfl_sync(0xffffffffu, cr, (2 * t) * 4);
       crow[1] = __shfl_sync(0xffffffffu, cr, (2 * t + 1) * 4);
@@ -431,33 +430,28 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT>::kThreads, 1) decode_ker
           // ---------------- S = K Q^T over the 256 channels ----------------
           // Key codes enter the MMA exactly (integers in f16).  Each 32-channel block is
           // accumulated on its own (four MMAs: two k-steps, query high and low parts) and then
-          // scaled by the block's fp32 scale (and, with a zero point, plus the block minimum
-          // times the query block sum) into S.
+          // scaled by the block's fp32 scale into S; with a zero point, two more MMAs add the
+          // block minima times the query block sums.
           float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-          // key scales (and minima) of rows g (H=0) and g+8 (H=1) for the 8 blocks, fp32
+          // key scales of rows g (H=0) and g+8 (H=1) for the 8 blocks, fp32; zero-point keys:
+          // the minima of blocks 2t, 2t + 1 of the same rows (the A fragment of the MMA that
+          // adds the minimum terms)
           float dkf[2][C::kNB];
-          float mkf[2][C::kKMin ? C::kNB : 1];
+          uint32_t mka[2] = {0u, 0u};
 #pragma unroll
           for (int H = 0; H < 2; ++H) {
             const uint32_t a = kb + C::kKScaleOff + (((G * 8 + g) * 2 + H) * 8) * 2;
-            uint32_t w[4], wm[4];
+            uint32_t w[4];
             const uint4 v = lds128(a);
             w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-            if constexpr (C::kKMin) {
-              const uint4 vm = lds128(a + (kK5MinOffset - kK5ScaleOffset));
-              wm[0] = vm.x; wm[1] = vm.y; wm[2] = vm.z; wm[3] = vm.w;
-            }
+            if constexpr (C::kKMin) mka[H] = lds32(a + (kK5MinOffset - kK5ScaleOffset) + 4 * t);
 #pragma unroll
             for (int e = 0; e < C::kNB / 2; ++e) {
               dkf[H][2 * e] = half_lo(w[e]);
               dkf[H][2 * e + 1] = half_hi(w[e]);
-              if constexpr (C::kKMin) {
-                mkf[H][2 * e] = half_lo(wm[e]);
-                mkf[H][2 * e + 1] = half_hi(wm[e]);
-              }
             }
           }
-          // one block: four MMAs into xb, then S += d * xb (+ m * qsum)
+          // one block: four MMAs into xb, then S += d * xb
           auto block_qk = [&](int bl, const uint32_t (&A)[2][4]) {
             float xb[4];
             const uint4 f0 = qfrag(bl, 0), f1 = qfrag(bl, 1);
@@ -466,10 +460,7 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT>::kThreads, 1) decode_ker
             mma_f16(xb, A[1][0], A[1][1], A[1][2], A[1][3], f1.x, f1.y);
             mma_f16(xb, A[1][0], A[1][1], A[1][2], A[1][3], f1.z, f1.w);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              sacc[e] = fmaf(dkf[e >> 1][bl], xb[e], sacc[e]);
-              if constexpr (C::kKMin) sacc[e] = fmaf(mkf[e >> 1][bl], qsum[bl][e & 1], sacc[e]);
-            }
+            for (int e = 0; e < 4; ++e) sacc[e] = fmaf(dkf[e >> 1][bl], xb[e], sacc[e]);
           };
           if constexpr (KF == kKeyQ8) {
 #pragma unroll
@@ -544,6 +535,13 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT>::kThreads, 1) decode_ker
               }
             }
           }
+          if constexpr (C::kKMin) {
+            // S += sum_b m[token][b] qsum[b][row] as one MMA per part of the block sums: A =
+            // the minima (tokens g, g + 8 x blocks 2t, 2t + 1; k = 8..15 is zero, exact in f16),
+            // B = the block sums of the query rows; the products accumulate in fp32
+            mma_f16(sacc, mka[0], mka[1], 0u, 0u, qsb_hi, 0u);
+            mma_f16(sacc, mka[0], mka[1], 0u, 0u, qsb_lo, 0u);
+          }
           // ---------------- online softmax (base 2) ----------------
           // The running maximum m_run of a row is shared by the 8 lanes that hold the row.
           // It only has to bound the scores to within 2^8 (p <= 256 in f16), so the exact
@@ -577,13 +575,7 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT>::kThreads, 1) decode_ker
                   oacc[mt][c] *= alpha;
                   oacc[mt][c + 2] *= alpha;
                 }
-                if constexpr (C::kVMin) {
-#pragma unroll
-                  for (int bl = 0; bl < C::kNB; ++bl) {
-                    macc[bl][c] *= alpha;
-                    macc[bl][c + 2] *= alpha;
-                  }
-                }
+                if constexpr (C::kVMin) racc[c] *= alpha;
                 m_run[c] = mx;
               }
             }
@@ -616,8 +608,6 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT>::kThreads, 1) decode_ker
               const uint4 vw = lds128(vb + ((((G * 4 + Cc) * 8 + g) * 4 + t) * 16));
               const uint32_t sidx = vb + C::kVScaleOff + (((G * 4 + t) * 8 + 2 * Cc) * 4) * 2;
               const uint4 dv = lds128(sidx);
-              uint4 mv = make_uint4(0u, 0u, 0u, 0u);
-              if constexpr (C::kVMin) mv = lds128(sidx + (kV41MinOffset - kV4ScaleOffset));
 #pragma unroll
               for (int e = 0; e < 2; ++e) {
                 const int bl = 2 * Cc + e;
@@ -642,17 +632,18 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT>::kThreads, 1) decode_ker
                 mma_f16(oacc[2 * bl], a00, a01, a02, a03, bl0, bl1);
                 mma_f16(oacc[2 * bl + 1], a10, a11, a12, a13, bh0, bh1);
                 mma_f16(oacc[2 * bl + 1], a10, a11, a12, a13, bl0, bl1);
-                if constexpr (C::kVMin) {
-                  // sum over the tile's tokens of p * m, the same for every dimension of the
-                  // block: an all-ones A operand
-                  const uint32_t m0 = e ? mv.z : mv.x, m1 = e ? mv.w : mv.y;
-                  uint32_t mh0, ml0, mh1, ml1;
-                  split_scaled(pbh[0], pbl[0], m0, mh0, ml0);
-                  split_scaled(pbh[1], pbl[1], m1, mh1, ml1);
-                  mma_f16(macc[bl], kHalf2_One, kHalf2_One, kHalf2_One, kHalf2_One, mh0, mh1);
-                  mma_f16(macc[bl], kHalf2_One, kHalf2_One, kHalf2_One, kHalf2_One, ml0, ml1);
-                }
               }
+            }
+            if constexpr (C::kVMin) {
+              // sum over the tile's tokens of p * m for all 8 blocks at once: A = the minima
+              // (block g x tokens 2t, 2t + 1 | 2t + 8, 2t + 9, exact in f16; blocks 8..15 zero),
+              // B = P^T as its high and low parts
+              uint32_t m01, m89;
+              asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];"
+                           : "=r"(m01), "=r"(m89)
+                           : "r"(vb + kV41MinOffset + (((G * 4 + t) * 8 + g) * 4) * 2));
+              mma_f16(racc, m01, 0u, m89, 0u, pbh[0], pbh[1]);
+              mma_f16(racc, m01, 0u, m89, 0u, pbl[0], pbl[1]);
             }
           } else {
 #pragma unroll
@@ -722,6 +713,14 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT>::kThreads, 1) decode_ker
   float* ls = ms + C::kConsumerWarps * 8;
   float* os = ls + C::kConsumerWarps * 8;
   {
+    // zero-point values: the minimum terms of block b for rows 2t, 2t + 1 sit in lane 4b + t
+    float rv[C::kVMin ? C::kNB : 1][2];
+    if constexpr (C::kVMin) {
+#pragma unroll
+      for (int b = 0; b < C::kNB; ++b)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) rv[b][c] = __shfl_sync(0xffffffffu, racc[c], 4 * b + t);
+    }
     if (g == 0) {
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -737,7 +736,7 @@ __global__ void __launch_bounds__(DecodeCfg<KF, VF, NT>::kThreads, 1) decode_ker
         const int lr = 2 * t + (e & 1);
         const int dim = 32 * b + 16 * hb + g + 8 * (e >> 1);
         float v = oacc[mt][e];
-        if constexpr (C::kVMin) v += macc[mt >> 1][e];
+        if constexpr (C::kVMin) v += rv[mt >> 1][e & 1];
         os[(warp * 8 + lr) * C::kOStride + dim] = v;
       }
     }

@@ -117,8 +117,9 @@ def test_verify_full_context(kv_gpu):
         compare(out[:, h * g:(h + 1) * g], lse[:, h * g:(h + 1) * g], o_ref, l_ref)
 
 
-def test_prefill_full_context_sampled_rows(kv_gpu):
-    b = bench.PrefillBench(kv_gpu, torch.device(DEV), layers=1)
+@pytest.mark.parametrize("wname", ["prefill524k", "prefill524k_q4q4", "prefill524k_q51q4"])
+def test_prefill_full_context_sampled_rows(kv_gpu, wname):
+    b = bench.PrefillBench(kv_gpu, torch.device(DEV), layers=1, wname=wname)
     b.layer(0)
     torch.cuda.synchronize()
     assert kv_gpu.kvattn_device_error() == 0
@@ -130,7 +131,7 @@ def test_prefill_full_context_sampled_rows(kv_gpu):
     q = b.q[0].float().cpu().numpy()                   # bf16 values, exact in fp32
     out, lse = b.out[0].cpu().numpy(), b.lse[0].cpu().numpy()
     for h in heads:
-        oc = _oracle_unit(k, v, int(h), w.v_fmt, b.k_new[0], b.v_new[0])
+        oc = _oracle_unit(k, v, int(h), w.v_fmt, b.k_new[0], b.v_new[0], k_fmt=w.k_fmt)
         t = np.sort(rng.choice(w.n_q, 32, replace=False))
         j = h * g + rng.integers(0, g, 32)
         rows = q[t, j]
