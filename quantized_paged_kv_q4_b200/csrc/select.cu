@@ -87,6 +87,10 @@ __global__ void __launch_bounds__(256) block_summary_kernel(const uint8_t* __res
 __global__ void __launch_bounds__(256) block_score_kernel(const float* __restrict__ summaries,
                                                           const float* __restrict__ q_group, int group, int n_blocks,
                                                           int n_cand, double* __restrict__ scores) {
+  // launched with programmatic dependent launch: the top-k grid behind this one may start
+  // now, and this grid reads the retrieval queries only once the kernel before it completed
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int unit = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x * (blockDim.x >> 5) + warp;
@@ -154,9 +158,11 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* t
 
 // Top-`budget` candidates by (score desc, block index asc), plus the recent window and the
 // tail, compacted into ascending logical ids.  The `take`-th largest 64-bit order key is found
-// by an 8-bit radix select (eight histogram passes); candidates above it are taken, and those
-// equal to it are taken in index order until `take` are chosen, which is exactly the first
-// `take` of a sort by (score desc, index asc).
+// by an 8-bit radix select, most significant digit first; candidates above it are taken, and
+// those equal to it are taken in index order until `take` are chosen, which is exactly the
+// first `take` of a sort by (score desc, index asc).  The select stops after the first pass
+// whose threshold bin holds exactly as many keys as are still to be taken: every key of that
+// bin is then taken, so the remaining digits cannot change the selection.
 __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const double* __restrict__ scores, int n_blocks,
                                                                  int n_cand, int n_total, int budget,
                                                                  const int32_t* __restrict__ page_table,
@@ -166,7 +172,9 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const double* 
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ int hist[256];
   __shared__ int warp_tot[kSelThreads / 32];
-  __shared__ int s_total, s_digit, s_need;
+  __shared__ int s_total, s_digit, s_need, s_bin;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the decode may set up
+  asm volatile("griddepcontrol.wait;" ::: "memory");               // the scores are complete
   const int unit = blockIdx.x;
   unsigned long long* key = reinterpret_cast<unsigned long long*>(sm);           // [n_cand]
   uint32_t* bits = reinterpret_cast<uint32_t*>(key + (n_cand > 0 ? n_cand : 1));  // [n_total / 32]
@@ -208,6 +216,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const double* 
             if (before < need && need <= before + c[e]) {
               s_digit = 255 - 8 * lane - e;
               s_need = need - before;
+              s_bin = c[e];
             }
             before += c[e];
           }
@@ -217,7 +226,9 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const double* 
       prefix |= static_cast<unsigned long long>(s_digit) << shift;
       mask |= 255ull << shift;
       need = s_need;
+      const bool whole_bin = s_bin == s_need;
       __syncthreads();
+      if (whole_bin) break;
     }
   }
   // mark: keys above the threshold, and the first `need` keys equal to it in index order
@@ -230,7 +241,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const double* 
     const int i0 = min(n_cand, threadIdx.x * per), i1 = min(n_cand, i0 + per);
     int eq = 0;
     if (take > 0 && take < n_cand)
-      for (int i = i0; i < i1; ++i) eq += key[i] == prefix;
+      for (int i = i0; i < i1; ++i) eq += (key[i] & mask) == prefix;
     int rank = block_exclusive_scan(eq, warp_tot, &s_total);
     for (int i = i0; i < i1; ++i) {
       bool sel;
@@ -239,7 +250,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const double* 
       } else if (take <= 0) {
         sel = false;
       } else {
-        const unsigned long long k = key[i];
+        const unsigned long long k = key[i] & mask;
         sel = k > prefix || (k == prefix && rank++ < need);
       }
       if (sel) atomicOr(&bits[i >> 5], 1u << (i & 31));
@@ -297,15 +308,30 @@ cudaError_t prepare_select_kernels() {
 cudaError_t launch_select(const float* summaries, const float* q_group, int n_units, int group, int n_blocks,
                           int n_cand, int n_total, int budget, const int32_t* page_table, int32_t* sel_logical,
                           int32_t* sel_phys, int32_t* n_sel, int cap, double* scores, cudaStream_t stream) {
+  // both grids use programmatic dependent launch: each may start while the kernel before it
+  // on the stream drains, and waits for it (griddepcontrol.wait) before reading its inputs
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   if (n_cand > 0) {
-    dim3 grid((n_cand + 7) / 8, n_units);
-    block_score_kernel<<<grid, 256, 0, stream>>>(summaries, q_group, group, n_blocks, n_cand, scores);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((n_cand + 7) / 8, n_units);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, block_score_kernel, summaries, q_group, group, n_blocks, n_cand, scores);
     if (e != cudaSuccess) return e;
   }
-  select_topk_kernel<<<n_units, kSelThreads, select_smem_bytes(max(n_cand, 1), n_total), stream>>>(
-      scores, n_blocks, n_cand, n_total, budget, page_table, sel_logical, sel_phys, n_sel, cap);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_units);
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = select_smem_bytes(max(n_cand, 1), n_total);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, select_topk_kernel, static_cast<const double*>(scores), n_blocks, n_cand, n_total,
+                            budget, page_table, sel_logical, sel_phys, n_sel, cap);
 }
 
 }  // namespace kvattn
