@@ -258,30 +258,40 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const double* 
   }
   for (int b = n_cand + threadIdx.x; b < n_total; b += kSelThreads) atomicOr(&bits[b >> 5], 1u << (b & 31));
   __syncthreads();
-  // compaction into ascending ids
-  const int per = (words + kSelThreads - 1) / kSelThreads;
-  const int w0 = min(words, threadIdx.x * per), w1 = min(words, w0 + per);
-  int cnt = 0;
-  for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
-  int pos = block_exclusive_scan(cnt, warp_tot, &s_total);
-  const int total = s_total;
+  // compaction into ascending ids: each thread takes a contiguous range of at most kCompact
+  // block indices (their page ids are loaded up front, all independent), counts its selected
+  // ones, and writes them at the position an exclusive scan of the counts gives
+  constexpr int kCompact = 4;
+  const int32_t* pt = page_table + static_cast<long long>(unit) * n_blocks;
   int32_t* out_l = sel_logical + static_cast<long long>(unit) * cap;
   int32_t* out_p = sel_phys + static_cast<long long>(unit) * cap;
-  const int32_t* pt = page_table + static_cast<long long>(unit) * n_blocks;
-  for (int w = w0; w < w1; ++w) {
-    uint32_t m = bits[w];
-    while (m) {
-      const int bit = __ffs(m) - 1;
-      m &= m - 1;
-      const int b = w * 32 + bit;
-      if (pos < cap) {
-        out_l[pos] = b;
-        out_p[pos] = pt[b];
+  int run = 0;  // selected blocks in the ranges before this pass
+  for (int base = 0; base < n_total; base += kSelThreads * kCompact) {
+    const int i0 = base + threadIdx.x * kCompact;
+    int32_t pg[kCompact];
+    bool on[kCompact];
+    int cnt = 0;
+#pragma unroll
+    for (int e = 0; e < kCompact; ++e) {
+      const int b = i0 + e;
+      on[e] = b < n_total && ((bits[b >> 5] >> (b & 31)) & 1u);
+      pg[e] = on[e] ? pt[b] : 0;
+      cnt += on[e];
+    }
+    int pos = run + block_exclusive_scan(cnt, warp_tot, &s_total);
+    run += s_total;
+#pragma unroll
+    for (int e = 0; e < kCompact; ++e) {
+      if (on[e]) {
+        if (pos < cap) {
+          out_l[pos] = i0 + e;
+          out_p[pos] = pg[e];
+        }
+        ++pos;
       }
-      ++pos;
     }
   }
-  if (threadIdx.x == 0) n_sel[unit] = min(total, cap);
+  if (threadIdx.x == 0) n_sel[unit] = min(run, cap);
 }
 
 cudaError_t launch_block_summaries(const kvattn_kv_desc& d, const int32_t* page_table, int n_units, int n_blocks,
