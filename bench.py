@@ -55,7 +55,7 @@ def parse_args():
     ap.add_argument("--stream-steps", type=int, default=0,
                     help="decode steps of the host-streamed generation to time (0 = the workload's 512)")
     ap.add_argument("--prefill-layers", type=int, default=0, help="layers of the prefill workload (0 = 16)")
-    ap.add_argument("--profile", choices=["none", "decode", "prefill", "verify", "stream"], default="none",
+    ap.add_argument("--profile", choices=["none", "decode", "prefill", "prefill_f16", "verify", "stream"], default="none",
                     help="profiling only: run just this workload's steps (no JSON bench line)")
     ap.add_argument("--context", type=int, default=0, help="profiling only: prior-context override")
     ap.add_argument("--layers", type=int, default=0,
@@ -384,7 +384,7 @@ class PrefillBench:
     16 layers x 4 KV heads, 4,096-token KV splits.  One step = for every layer: append the
     chunk's K/V, then the four ubatch prefill calls."""
 
-    def __init__(self, kv, device, layers=0, context=0, wname="prefill524k"):
+    def __init__(self, kv, device, layers=0, context=0, wname="prefill524k", f16=False):
         import dataclasses
 
         import torch
@@ -411,8 +411,10 @@ class PrefillBench:
         g = w.group
         self.flops_per_layer = 4.0 * Hq * 256 * (w.n_q * w.context + w.n_q * (w.n_q + 1) / 2)
         # tensor-core work per algorithmic flop: QK^T as two MMAs (K^ high and low parts) and PV
-        # as three (P_hi V^_hi, P_lo V^_hi, P_hi V^_lo)
-        self.mma_work_factor = (2 + 3) / 2
+        # as three (P_hi V^_hi, P_lo V^_hi, P_hi V^_lo); one each with operands rounded once
+        self.f16 = f16
+        self.call = kv.kvattn_prefill_chunk_f16 if f16 else kv.kvattn_prefill_chunk
+        self.mma_work_factor = 1.0 if f16 else (2 + 3) / 2
         self.flops_per_step = self.flops_per_layer * L
         self.launches_per_step = L * (1 + 2 * (w.n_q // w.ubatch))
 
@@ -423,9 +425,8 @@ class PrefillBench:
             timed[0].record()
         for u in range(w.n_q // w.ubatch):
             a, b = u * w.ubatch, (u + 1) * w.ubatch
-            kv.kvattn_prefill_chunk(c.desc, self.q_bits[l, a:b], w.ubatch, self.q_pos[a:b], c.page_table[l], None,
-                                    None, self.nb, w.kv_split_tokens, self.out[l, a:b], self.lse[l, a:b], self.ws,
-                                    self.ws_bytes)
+            self.call(c.desc, self.q_bits[l, a:b], w.ubatch, self.q_pos[a:b], c.page_table[l], None, None, self.nb,
+                      w.kv_split_tokens, self.out[l, a:b], self.lse[l, a:b], self.ws, self.ws_bytes)
         if timed is not None:
             timed[1].record()
 
@@ -999,7 +1000,8 @@ def main():
         elif args.profile == "stream":
             b = StreamBench(kvattn, device, layers=args.layers or 2, context=args.context)
         else:
-            b = PrefillBench(kvattn, device, layers=args.layers or 1, context=args.context)
+            b = PrefillBench(kvattn, device, layers=args.layers or 1, context=args.context,
+                             f16=args.profile == "prefill_f16")
         for _ in range(args.warmup + args.steps):
             b.step()
         torch.cuda.synchronize()
@@ -1087,22 +1089,27 @@ def main():
             tf = b4.flops_per_layer / (k4 * 1e-3) / 1e12
             extra["prefill524k"] = {"TFLOP/s": b4.flops_per_step / (ms4 * 1e-3) / 1e12, "ms_per_step": ms4,
                                     "layers": b4.w.layers, "kernel_TFLOP/s": tf, "kernel_frac_bf16": tf / bf16,
+                                    "kernel_frac_bf16_sustained": tf / bf16_sus,
                                     "layer_ms": k4, "flop_per_layer": b4.flops_per_layer,
                                     "executed_TFLOP/s": tf * b4.mma_work_factor,
                                     "executed_frac_bf16": tf * b4.mma_work_factor / bf16,
                                     "mma_work_factor": b4.mma_work_factor,
-                                    "peak": f"{peak_kind} dense bf16 (f16 operands run at the same rate)"}
+                                    "peak": f"{peak_kind} dense bf16, burst and sustained (f16 operands run at "
+                                            "the same rate; the 16-layer step keeps the GPU at its power cap)"}
             del b4
             torch.cuda.empty_cache()
-            # the same prefill layer over Q4_0 and Q5_1 keys (one layer: kernel rate only)
-            for wn in ("prefill524k_q4q4", "prefill524k_q51q4"):
-                b6 = PrefillBench(kvattn, device, layers=1, wname=wn)
+            # the same prefill layer over Q4_0 and Q5_1 keys, and with operands rounded once to f16
+            # (kvattn_prefill_chunk_f16); one layer each: kernel rate only
+            for wn, f16 in (("prefill524k_q4q4", False), ("prefill524k_q51q4", False), ("prefill524k", True)):
+                b6 = PrefillBench(kvattn, device, layers=1, wname=wn, f16=f16)
                 b6.layer(0)
                 k6 = time_layers(b6, 2)
                 tf6 = b6.flops_per_layer / (k6 * 1e-3) / 1e12
-                extra[wn] = {"kernel_TFLOP/s": tf6, "kernel_frac_bf16": tf6 / bf16, "layer_ms": k6,
-                             "executed_frac_bf16": tf6 * b6.mma_work_factor / bf16,
-                             "k_fmt": b6.w.k_fmt, "v_fmt": b6.w.v_fmt}
+                extra[wn + ("_f16" if f16 else "")] = {
+                    "kernel_TFLOP/s": tf6, "kernel_frac_bf16": tf6 / bf16, "kernel_frac_bf16_sustained": tf6 / bf16_sus,
+                    "layer_ms": k6,
+                    "executed_frac_bf16": tf6 * b6.mma_work_factor / bf16, "k_fmt": b6.w.k_fmt, "v_fmt": b6.w.v_fmt,
+                    "operands": "f16, rounded once" if f16 else "f16 high + low parts (about 22 bits)"}
                 del b6
                 torch.cuda.empty_cache()
             b5 = StreamBench(kvattn, device)

@@ -318,6 +318,20 @@ KVATTN_API int kvattn_prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* 
                                     int max_pages, int kv_split_tokens, float* out, float* lse,
                                     void* ws, size_t ws_bytes, kvattn_stream_t stream);
 
+/* The same chunked prefill (arguments, formats, workspace and errors as kvattn_prefill_chunk)
+ * with each dequantized K/V value and each P rounded once to f16 ([STREAM] method list; the
+ * tiles are dequantized to 16-bit operands in shared memory): QK^T and PV take one MMA pass
+ * each instead of two and three.  Every operand then carries 11 significant bits, so an
+ * output row errs by up to about 2^-11 of the largest |value| it averages when few keys
+ * dominate, and far less when many keys share the weight; kvattn_prefill_chunk keeps about 22
+ * bits. */
+KVATTN_API int kvattn_prefill_chunk_f16(const kvattn_kv_desc* desc, const uint16_t* q, int n_q,
+                                        const int32_t* q_pos, const int32_t* page_list,
+                                        const int32_t* page_logical, const int32_t* n_pages,
+                                        int max_pages, int kv_split_tokens, float* out,
+                                        float* lse, void* ws, size_t ws_bytes,
+                                        kvattn_stream_t stream);
+
 /* ---- host page streaming ([STREAM]: full history in pinned host RAM, working set over
  * PCIe; layer L+1 prefetched while layer L computes) ----------------------------------
  * Copies n pages from a pinned host pool to device slots with cudaMemcpyAsync on

@@ -586,11 +586,16 @@ KVATTN_API size_t kvattn_prefill_workspace_size(const kvattn_kv_desc* desc, int 
       .bytes;
 }
 
-KVATTN_API int kvattn_prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* q, int n_q, const int32_t* q_pos,
-                                    const int32_t* page_list, const int32_t* page_logical, const int32_t* n_pages,
-                                    int max_pages, int kv_split_tokens, float* out, float* lse, void* ws,
-                                    size_t ws_bytes, kvattn_stream_t stream) {
-  const CallRange range_("kvattn_prefill_chunk");
+}  // extern "C"
+
+namespace {
+
+// Validates a prefill call and launches it (exact: the ~22-bit operand splits; else one f16
+// rounding per operand).
+int prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* q, int n_q, const int32_t* q_pos,
+                  const int32_t* page_list, const int32_t* page_logical, const int32_t* n_pages, int max_pages,
+                  int kv_split_tokens, float* out, float* lse, void* ws, size_t ws_bytes, kvattn_stream_t stream,
+                  bool exact) {
   int st = validate_desc(desc);
   if (st) return st;
   if ((desc->k_fmt != KVATTN_FMT_Q8_0 && desc->k_fmt != KVATTN_FMT_Q4_0 && desc->k_fmt != KVATTN_FMT_Q5_1) ||
@@ -636,8 +641,31 @@ KVATTN_API int kvattn_prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* 
   prm.pages_per_split = plan.pps;
   prm.n_ks = plan.n_ks;
   prm.rows_pad = plan.rows_pad;
-  cudaError_t e = launch_prefill(prm, desc->n_kv_heads, key_format_id(desc->k_fmt), static_cast<cudaStream_t>(stream));
+  cudaError_t e =
+      launch_prefill(prm, desc->n_kv_heads, key_format_id(desc->k_fmt), exact, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVATTN_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+KVATTN_API int kvattn_prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* q, int n_q, const int32_t* q_pos,
+                                    const int32_t* page_list, const int32_t* page_logical, const int32_t* n_pages,
+                                    int max_pages, int kv_split_tokens, float* out, float* lse, void* ws,
+                                    size_t ws_bytes, kvattn_stream_t stream) {
+  const CallRange range_("kvattn_prefill_chunk");
+  return prefill_chunk(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pages, kv_split_tokens, out, lse,
+                       ws, ws_bytes, stream, true);
+}
+
+KVATTN_API int kvattn_prefill_chunk_f16(const kvattn_kv_desc* desc, const uint16_t* q, int n_q, const int32_t* q_pos,
+                                        const int32_t* page_list, const int32_t* page_logical, const int32_t* n_pages,
+                                        int max_pages, int kv_split_tokens, float* out, float* lse, void* ws,
+                                        size_t ws_bytes, kvattn_stream_t stream) {
+  const CallRange range_("kvattn_prefill_chunk_f16");
+  return prefill_chunk(desc, q, n_q, q_pos, page_list, page_logical, n_pages, max_pages, kv_split_tokens, out, lse,
+                       ws, ws_bytes, stream, false);
 }
 
 }  // extern "C"

@@ -217,8 +217,9 @@ __device__ __forceinline__ uint64_t f32x2_pack(uint32_t lo, uint32_t hi) {
   return r;
 }
 
-// P = exp2(S log2(e) - mu) for 32 columns, as 16 f16 pairs of high parts (wh) and 16 of low
-// parts (wl: the rounded remainder); returns the sum of the 32 fp32 values of P.
+// P = exp2(S log2(e) - mu) for 32 columns, as 16 f16 pairs of high parts (wh) and, with LO, 16
+// of low parts (wl: the rounded remainder); returns the sum of the 32 fp32 values of P.
+template <bool LO>
 __device__ __forceinline__ float pf_p32(const uint32_t (&v)[32], float mu, uint32_t (&wh)[16], uint32_t (&wl)[16]) {
   const uint64_t l2 = f32x2_pack(__float_as_uint(pf::kLog2e), __float_as_uint(pf::kLog2e));
   const uint64_t nm = f32x2_pack(__float_as_uint(-mu), __float_as_uint(-mu));
@@ -233,7 +234,7 @@ __device__ __forceinline__ float pf_p32(const uint32_t (&v)[32], float mu, uint3
     const uint64_t pp = f32x2_pack(__float_as_uint(p0), __float_as_uint(p1));
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(acc[c & 1]) : "l"(acc[c & 1]), "l"(pp));
     wh[c] = pack_half2(p0, p1);
-    wl[c] = pack_half2(p0 - half_lo(wh[c]), p1 - half_hi(wh[c]));
+    if constexpr (LO) wl[c] = pack_half2(p0 - half_lo(wh[c]), p1 - half_hi(wh[c]));
   }
   uint64_t t;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(acc[0]), "l"(acc[1]));
@@ -261,7 +262,10 @@ __device__ __forceinline__ void split_affine(uint32_t code, float d, float m, ui
 // x shifted left by s bits (right by -s when s < 0); s is a compile-time constant after unrolling.
 __device__ __forceinline__ uint32_t shl(uint32_t x, int s) { return s >= 0 ? x << s : x >> -s; }
 
-template <int KF>
+// EXACT: every operand as an f16 high part plus a low part (about 22 significant bits, QK as
+// two MMA passes, PV as three); otherwise each dequantized value and each P rounded once to
+// f16 (one pass each; the dequant writes, and the MMAs read, the high parts only).
+template <int KF, bool EXACT>
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillParams p) {
   using RawF = pf::Raw<KF>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -408,7 +412,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
             const uint32_t ka = k_base + b * pf::kSet + (kk >> 2) * 4096 + (kk & 3) * 32;
             const uint32_t dcol = tmem + pf::kSCol0 + s2 * pf::kKeys, qcol = tmem + pf::kQCol0 + kk * 8;
             tc::mma_f16_ts_pair_warp(dcol, qcol, tc::sw128_desc(ka, 1024, 16), pf::kIdescQK, kk > 0 ? 1u : 0u);
-            tc::mma_f16_ts_pair_warp(dcol, qcol, tc::sw128_desc(ka + pf::kPart, 1024, 16), pf::kIdescQK, 1u);
+            if constexpr (EXACT)
+              tc::mma_f16_ts_pair_warp(dcol, qcol, tc::sw128_desc(ka + pf::kPart, 1024, 16), pf::kIdescQK, 1u);
           }
           tc::commit_pair2_warp(&sready[s2]);
           tc::commit_pair2_warp(&kfree[b]);
@@ -424,8 +429,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
             const uint32_t ph = tmem + pf::kSCol0 + s2 * pf::kKeys + kk * 8, pl = ph + pf::kKeys / 2;
             const uint64_t vh = tc::sw128_desc(va, 1024, 16), vl = tc::sw128_desc(va + pf::kPart, 1024, 16);
             tc::mma_f16_ts_pair_warp(tmem + pf::kOCol0, ph, vh, pf::kIdescPV, (jp > 0 || kk > 0) ? 1u : 0u);
-            tc::mma_f16_ts_pair_warp(tmem + pf::kOCol0, pl, vh, pf::kIdescPV, 1u);
-            tc::mma_f16_ts_pair_warp(tmem + pf::kOCol0, ph, vl, pf::kIdescPV, 1u);
+            if constexpr (EXACT) {
+              tc::mma_f16_ts_pair_warp(tmem + pf::kOCol0, pl, vh, pf::kIdescPV, 1u);
+              tc::mma_f16_ts_pair_warp(tmem + pf::kOCol0, ph, vl, pf::kIdescPV, 1u);
+            }
           }
           tc::commit_pair2_warp(vdone);
           tc::commit_pair2_warp(&vfree[b]);
@@ -519,12 +526,12 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       const float mu = m_ref == -INFINITY ? 0.f : m_ref;
       {
         uint32_t wh[16], wl[16];
-        l_sum += pf_p32(v0, mu, wh, wl);
+        l_sum += pf_p32<EXACT>(v0, mu, wh, wl);
         tc::st16(scol, wh);
-        tc::st16(scol + 32, wl);
-        l_sum += pf_p32(v1, mu, wh, wl);
+        if constexpr (EXACT) tc::st16(scol + 32, wl);
+        l_sum += pf_p32<EXACT>(v1, mu, wh, wl);
         tc::st16(scol + 16, wh);
-        tc::st16(scol + 48, wl);
+        if constexpr (EXACT) tc::st16(scol + 48, wl);
       }
       if (__any_sync(0xffffffffu, resc)) {
         // O is rescaled to the new maximum before PV of this tile accumulates into it; this
@@ -710,19 +717,29 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
             }
           }
           uint32_t oh[8], ol[8];
-          if constexpr (KF == kKeyQ51) {
+          if constexpr (KF == kKeyQ51 && EXACT) {
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               split_affine(c[e], e < 4 ? half_lo(dkw) : half_hi(dkw), e < 4 ? half_lo(mkw) : half_hi(mkw), oh[e],
                            ol[e]);
-          } else {
+          } else if constexpr (KF == kKeyQ51) {
+            // q * d + m rounded once to f16 (one fused multiply-add)
+            const uint32_t mlo = prmt(mkw, 0u, 0x1010u), mhi = prmt(mkw, 0u, 0x3232u);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) oh[e] = hfma2(c[e], e < 4 ? dlo : dhi, e < 4 ? mlo : mhi);
+          } else if constexpr (EXACT) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) split_product(c[e], e < 4 ? dlo : dhi, oh[e], ol[e]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) oh[e] = hmul2(c[e], e < 4 ? dlo : dhi);
           }
           sts128u(katom + swz(kl, T), oh[0], oh[1], oh[2], oh[3]);
           sts128u(katom + swz(kl, 4 + T), oh[4], oh[5], oh[6], oh[7]);
-          sts128u(katom + pf::kPart + swz(kl, T), ol[0], ol[1], ol[2], ol[3]);
-          sts128u(katom + pf::kPart + swz(kl, 4 + T), ol[4], ol[5], ol[6], ol[7]);
+          if constexpr (EXACT) {
+            sts128u(katom + pf::kPart + swz(kl, T), ol[0], ol[1], ol[2], ol[3]);
+            sts128u(katom + pf::kPart + swz(kl, 4 + T), ol[4], ol[5], ol[6], ol[7]);
+          }
         }
         tc::fence_proxy_async_smem();
       }
@@ -755,16 +772,23 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
           const uint32_t v1 = hfma2(and_or(W, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
           const uint32_t v2 = hsub2(and_or(Ws, 0x000F000Fu, 0x64006400u), 0x64086408u);
           const uint32_t v3 = hfma2(and_or(Ws, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
-          split_product(v0, dv, oh[0][T], ol[0][T]);
-          split_product(v1, dv, oh[1][T], ol[1][T]);
-          split_product(v2, dv, oh[2][T], ol[2][T]);
-          split_product(v3, dv, oh[3][T], ol[3][T]);
+          if constexpr (EXACT) {
+            split_product(v0, dv, oh[0][T], ol[0][T]);
+            split_product(v1, dv, oh[1][T], ol[1][T]);
+            split_product(v2, dv, oh[2][T], ol[2][T]);
+            split_product(v3, dv, oh[3][T], ol[3][T]);
+          } else {
+            oh[0][T] = hmul2(v0, dv);
+            oh[1][T] = hmul2(v1, dv);
+            oh[2][T] = hmul2(v2, dv);
+            oh[3][T] = hmul2(v3, dv);
+          }
         }
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int row = 32 * (2 * vCl + ve) + 8 * k + vR;  // dimension - 128 * rank
           sts128u(vt + swz(row, 2 * vG + vh), oh[k][0], oh[k][1], oh[k][2], oh[k][3]);
-          sts128u(vt + pf::kPart + swz(row, 2 * vG + vh), ol[k][0], ol[k][1], ol[k][2], ol[k][3]);
+          if constexpr (EXACT) sts128u(vt + pf::kPart + swz(row, 2 * vG + vh), ol[k][0], ol[k][1], ol[k][2], ol[k][3]);
         }
         tc::fence_proxy_async_smem();
       }
@@ -788,13 +812,28 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
   }
 }
 
-cudaError_t prepare_prefill_kernels() {
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<kKeyQ8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <bool EXACT>
+static cudaError_t prepare_prefill_t() {
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<kKeyQ8, EXACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        pf::kSmemBytes);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(prefill_kernel<kKeyQ4>, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::kSmemBytes);
+    e = cudaFuncSetAttribute(prefill_kernel<kKeyQ4, EXACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pf::kSmemBytes);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(prefill_kernel<kKeyQ51>, cudaFuncAttributeMaxDynamicSharedMemorySize, pf::kSmemBytes);
+  return cudaFuncSetAttribute(prefill_kernel<kKeyQ51, EXACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              pf::kSmemBytes);
+}
+
+cudaError_t prepare_prefill_kernels() {
+  const cudaError_t e = prepare_prefill_t<true>();
+  return e != cudaSuccess ? e : prepare_prefill_t<false>();
+}
+
+template <bool EXACT>
+static cudaError_t launch_prefill_grid(const cudaLaunchConfig_t& cfg, const PrefillParams& prm, int key_fmt) {
+  return key_fmt == kKeyQ4    ? cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ4, EXACT>, prm)
+         : key_fmt == kKeyQ51 ? cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ51, EXACT>, prm)
+                              : cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ8, EXACT>, prm);
 }
 
 struct PrefillPlan {
@@ -825,7 +864,7 @@ PrefillPlan plan_prefill(int n_kv, int group, int n_q, int max_pages, int kv_spl
   return pl;
 }
 
-cudaError_t launch_prefill(const PrefillParams& prm0, int n_kv, int key_fmt, cudaStream_t stream) {
+cudaError_t launch_prefill(const PrefillParams& prm0, int n_kv, int key_fmt, bool exact, cudaStream_t stream) {
   PrefillParams prm = prm0;
   const int rows = prm.n_q * prm.group;
   {
@@ -841,9 +880,7 @@ cudaError_t launch_prefill(const PrefillParams& prm0, int n_kv, int key_fmt, cud
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = key_fmt == kKeyQ4    ? cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ4>, prm)
-                    : key_fmt == kKeyQ51 ? cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ51>, prm)
-                                         : cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ8>, prm);
+    cudaError_t e = exact ? launch_prefill_grid<true>(cfg, prm, key_fmt) : launch_prefill_grid<false>(cfg, prm, key_fmt);
     if (e != cudaSuccess || prm.n_ks == 1) return e;
   }
   cudaLaunchConfig_t cfg = {};

@@ -82,6 +82,8 @@ _SIGS = {
     "kvattn_prefill_workspace_size": (c_size_t, [POINTER(kvattn_kv_desc), c_int, c_int, c_int]),
     "kvattn_prefill_chunk": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                      c_int, c_int, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "kvattn_prefill_chunk_f16": (c_int, [POINTER(kvattn_kv_desc), c_void_p, c_int, c_void_p, c_void_p, c_void_p,
+                                         c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "kvattn_stream_pages": (c_int, [c_void_p, c_int64, c_void_p, c_int64, c_int64, c_void_p, c_void_p, c_int,
                                     c_void_p, c_void_p, POINTER(c_int)]),
     "kvattn_gather_pages": (c_int, [c_void_p, c_int64, c_int64, c_void_p, c_int64, c_int64, c_int64, c_void_p,
@@ -263,6 +265,13 @@ def kvattn_prefill_chunk(desc, q_bf16, n_q, q_pos, page_list, page_logical, n_pa
     _check(lib().kvattn_prefill_chunk(ctypes.byref(desc), _d(q_bf16), n_q, _d(q_pos), _d(page_list),
                                       _d(page_logical), _d(n_pages), max_pages, kv_split_tokens, _d(out), _d(lse),
                                       _d(ws), ws_bytes, _s(stream)), "kvattn_prefill_chunk")
+
+
+def kvattn_prefill_chunk_f16(desc, q_bf16, n_q, q_pos, page_list, page_logical, n_pages, max_pages, kv_split_tokens,
+                             out, lse, ws, ws_bytes, stream=None) -> None:
+    _check(lib().kvattn_prefill_chunk_f16(ctypes.byref(desc), _d(q_bf16), n_q, _d(q_pos), _d(page_list),
+                                          _d(page_logical), _d(n_pages), max_pages, kv_split_tokens, _d(out), _d(lse),
+                                          _d(ws), ws_bytes, _s(stream)), "kvattn_prefill_chunk_f16")
 
 
 def kvattn_gather_pages(host_pool, host_stride, n_host_pages, dev_pool, dev_stride, n_slots, page_bytes, host_ids,

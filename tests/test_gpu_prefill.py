@@ -9,7 +9,8 @@ from synth import bf16_bits, bf16_round, normal_f32, np_rng, page_permutation
 pytestmark = pytest.mark.gpu
 
 
-def _prefill(kv, cache, H_q, q, q_pos, page_list, split, page_logical=None, n_pages=None, max_pages=None):
+def _prefill(kv, cache, H_q, q, q_pos, page_list, split, page_logical=None, n_pages=None, max_pages=None,
+             f16=False):
     cache.desc.n_q_heads = H_q
     n_q = q.shape[0]
     max_pages = page_list.shape[1] if max_pages is None else max_pages
@@ -22,7 +23,8 @@ def _prefill(kv, cache, H_q, q, q_pos, page_list, split, page_logical=None, n_pa
     pl = torch.as_tensor(page_list, dtype=torch.int32).cuda()
     lg = torch.as_tensor(page_logical, dtype=torch.int32).cuda() if page_logical is not None else None
     npg = torch.as_tensor(n_pages, dtype=torch.int32).cuda() if n_pages is not None else None
-    kv.kvattn_prefill_chunk(cache.desc, qb, n_q, qp, pl, lg, npg, max_pages, split, out, lse, ws, wsb)
+    call = kv.kvattn_prefill_chunk_f16 if f16 else kv.kvattn_prefill_chunk
+    call(cache.desc, qb, n_q, qp, pl, lg, npg, max_pages, split, out, lse, ws, wsb)
     torch.cuda.synchronize()
     assert kv.kvattn_device_error() == 0
     return out.cpu().numpy(), lse.cpu().numpy()
@@ -56,6 +58,21 @@ def test_prefill_matches_oracle(kv_gpu, n_prior, n_q, split, k_fmt):
     rng, k, v, q, cache, T = _case(1200 + n_prior + n_q, H, n_prior, n_q, k_fmt=k_fmt)
     q_pos = np.arange(n_prior, T)
     out, lse = _prefill(kv_gpu, cache, 6 * H, q, q_pos, cache.page_table_np, split)
+    oc = OracleCache(k, v, "q4_0", k_fmt)
+    for h in range(H):
+        o_ref, l_ref = oc.attend(q, q_pos, h, 6)
+        compare(out[:, 6 * h:6 * h + 6], lse[:, 6 * h:6 * h + 6], o_ref, l_ref)
+
+
+@pytest.mark.parametrize("k_fmt", ["q8_0", "q4_0", "q5_1"])
+@pytest.mark.parametrize("n_prior,n_q,split", [(700, 40, 256), (5000, 130, 1024), (0, 30, 128), (4096, 512, 4096)])
+def test_prefill_f16_matches_oracle(kv_gpu, n_prior, n_q, split, k_fmt):
+    """The one-rounding operand mode on the prefill workload's distribution (K, V and Q drawn
+    N(0, 1), no outlier channels): within the same absolute bound as the exact mode."""
+    H = 2
+    rng, k, v, q, cache, T = _case(1700 + n_prior + n_q, H, n_prior, n_q, outliers=False, k_fmt=k_fmt)
+    q_pos = np.arange(n_prior, T)
+    out, lse = _prefill(kv_gpu, cache, 6 * H, q, q_pos, cache.page_table_np, split, f16=True)
     oc = OracleCache(k, v, "q4_0", k_fmt)
     for h in range(H):
         o_ref, l_ref = oc.attend(q, q_pos, h, 6)
