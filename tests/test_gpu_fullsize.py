@@ -117,9 +117,12 @@ def test_verify_full_context(kv_gpu):
         compare(out[:, h * g:(h + 1) * g], lse[:, h * g:(h + 1) * g], o_ref, l_ref)
 
 
-@pytest.mark.parametrize("wname", ["prefill524k", "prefill524k_q4q4", "prefill524k_q51q4"])
-def test_prefill_full_context_sampled_rows(kv_gpu, wname):
-    b = bench.PrefillBench(kv_gpu, torch.device(DEV), layers=1, wname=wname)
+@pytest.mark.parametrize("wname,f16", [("prefill524k", False), ("prefill524k_q4q4", False),
+                                       ("prefill524k_q51q4", False), ("prefill524k", True)])
+def test_prefill_full_context_sampled_rows(kv_gpu, wname, f16):
+    """One layer of the 524,288-key prefill as the bench runs it (the f16 case through
+    kvattn_prefill_chunk_f16): 64 sampled rows of two KV heads against the oracle."""
+    b = bench.PrefillBench(kv_gpu, torch.device(DEV), layers=1, wname=wname, f16=f16)
     b.layer(0)
     torch.cuda.synchronize()
     assert kv_gpu.kvattn_device_error() == 0
