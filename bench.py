@@ -1098,9 +1098,10 @@ def main():
                                             "the same rate; the 16-layer step keeps the GPU at its power cap)"}
             del b4
             torch.cuda.empty_cache()
-            # the same prefill layer over Q4_0 and Q5_1 keys, and with operands rounded once to f16
+            # the same prefill layer over the other format pairs, and with operands rounded once to f16
             # (kvattn_prefill_chunk_f16); one layer each: kernel rate only
-            for wn, f16 in (("prefill524k_q4q4", False), ("prefill524k_q51q4", False), ("prefill524k", True)):
+            for wn, f16 in (("prefill524k_q4q4", False), ("prefill524k_q51q4", False), ("prefill524k_q50q41", False),
+                            ("prefill524k", True)):
                 b6 = PrefillBench(kvattn, device, layers=1, wname=wn, f16=f16)
                 b6.layer(0)
                 k6 = time_layers(b6, 2)

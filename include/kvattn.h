@@ -297,16 +297,17 @@ KVATTN_API int kvattn_select_blocks(const float* summaries, const float* q_group
 /* ---- chunked prefill on tcgen05 ([STREAM] method list) -----------------------------
  * Attention of n_q bf16 query tokens (positions q_pos[i], device int32 [n_q]) over the
  * listed pages, causal.  K/V tiles are dequantized in shared memory into an f16 high part
- * (code x scale rounded once; Q5_1 keys: code x scale + minimum, summed once in fp32) and an
- * f16 low part (the remainder, exact but for Q5_1 keys' fp32 sum); Q enters as Q/16 in
+ * (code x scale rounded once; Q5_1 keys and Q4_1 values: code x scale + minimum, summed once
+ * in fp32) and an f16 low part (the remainder, exact but for that fp32 sum); Q enters as Q/16 in
  * f16 (exact) and P as an f16 high part plus the rounded remainder.  QK^T (two MMAs per
  * k-step) and PV (three) run on tcgen05 tensor cores as CTA-pair MMAs with fp32
  * accumulation in tensor memory, so every operand carries about 22 significant bits.  The
  * keys are taken in splits of kv_split_tokens (a multiple of 128, at most 65,536; a CTA may
  * walk several consecutive splits); partial results are merged by log-sum-exp.  A page id
  * outside [0, n_pages) skips its page and records KVATTN_ERR_BAD_PAGE.  Needs Q8_0, Q4_0 or
- * Q5_1 K with Q4_0 V pages (UNSUPPORTED_FORMAT otherwise; [GUIDE] build step: the q8_0-q4_0
- * and q4_0-q4_0 pairs; [VULKAN] pitfalls: Q5_1 K with Q4_0 V).
+ * Q5_1 K with Q4_0 V pages, or Q5_0 K with Q4_1 V pages (UNSUPPORTED_FORMAT otherwise;
+ * [GUIDE] build step: the q8_0-q4_0 and q4_0-q4_0 pairs; [VULKAN] pitfalls: Q5_1 K with Q4_0
+ * V; [MTP]: the Q5_0 K / Q4_1 V cache).
  *   q      device bf16 bits [n_q][H_q][256];  out device fp32 [n_q][H_q][256];
  *   lse    device fp32 [n_q][H_q];  page arguments as for kvattn_decode.
  *   ws     device workspace of kvattn_prefill_workspace_size() bytes. */

@@ -598,8 +598,10 @@ int prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* q, int n_q, const 
                   bool exact) {
   int st = validate_desc(desc);
   if (st) return st;
-  if ((desc->k_fmt != KVATTN_FMT_Q8_0 && desc->k_fmt != KVATTN_FMT_Q4_0 && desc->k_fmt != KVATTN_FMT_Q5_1) ||
-      desc->v_fmt != KVATTN_FMT_Q4_0)
+  const bool v40_pair = (desc->k_fmt == KVATTN_FMT_Q8_0 || desc->k_fmt == KVATTN_FMT_Q4_0 ||
+                         desc->k_fmt == KVATTN_FMT_Q5_1) &&
+                        desc->v_fmt == KVATTN_FMT_Q4_0;
+  if (!v40_pair && !(desc->k_fmt == KVATTN_FMT_Q5_0 && desc->v_fmt == KVATTN_FMT_Q4_1))
     return KVATTN_ERR_UNSUPPORTED_FORMAT;
   if (n_q < 1 || max_pages < 0 || !q || !q_pos || !out || !lse || (max_pages > 0 && !page_list))
     return KVATTN_ERR_INVALID_ARG;

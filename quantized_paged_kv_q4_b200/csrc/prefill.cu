@@ -1,9 +1,11 @@
-// Chunked prefill over block-quantized KV pages (Q8_0, Q4_0 or Q5_1 keys, Q4_0 values) on
+// Chunked prefill over block-quantized KV pages (Q8_0, Q4_0 or Q5_1 keys with Q4_0 values, Q5_0
+// keys with Q4_1 values) on
 // tcgen05 tensor cores (Adaptive KV Streaming + RDNA 4 announcement, wqu.guru, method list:
 // "online log-sum-exp prefill": the prefill of a chunk is computed across streamed KV pages
 // and the partial results are accumulated by online log-sum-exp; the six-step validation
 // guide, alphalab.site, build step: the q8_0-q4_0 and q4_0-q4_0 flash-attention KV pairs;
-// Vulkan speculative-decoding report, lcz.me/topic/1398, pitfalls: the K q5_1 / V q4_0 cache).
+// Vulkan speculative-decoding report, lcz.me/topic/1398, pitfalls: the K q5_1 / V q4_0 cache;
+// 7900 XTX MTP tuning notes, lcz.me/topic/593: a q5_0 / q4_1 cache).
 //
 // Work unit: a cluster of two CTAs = a KV head, two M-tiles of 128 query rows of that head's
 // group (row r = token t * group + j: all query heads of a group share the K/V tiles), and
@@ -67,20 +69,27 @@ constexpr int kDq0 = (kSoftmaxWarps + 2) * 32;  // first dequant thread
 // scales (Q5_1: then minima) of its 32 keys (each region contiguous in the page), V codes of
 // its 128 head dimensions for all 64 keys (four 1 KB pieces, one per 16-key group), and all
 // V scales of the tile; the stage holds them in that order
+// The value format is fixed by the key format: Q4_0 values under Q8_0, Q4_0 and Q5_1 keys,
+// Q4_1 values under Q5_0 keys (the format pairs chunked prefill takes).
+__host__ __device__ constexpr bool value_q41(int KF) { return KF == kKeyQ50; }
 template <int KF>
 struct Raw {
+  static constexpr bool kK5 = KF == kKeyQ51 || KF == kKeyQ50;
   static constexpr int kKc = KF == kKeyQ8 ? 8192 : 4096;  // 32 keys x 256 or 128 bytes
-  static constexpr int kKh = KF == kKeyQ51 ? 1024 : 0;    // fifth bits: 32 keys x 32 bytes
+  static constexpr int kKh = kK5 ? 1024 : 0;              // fifth bits: 32 keys x 32 bytes
   static constexpr int kKs = 512, kVc = 4096, kVs = 1024;
-  static constexpr int kKm = KF == kKeyQ51 ? 512 : 0;     // minima
+  static constexpr int kKm = KF == kKeyQ51 ? 512 : 0;     // key minima
+  static constexpr int kVm = value_q41(KF) ? 1024 : 0;    // value minima (Q4_1), as the scales
   static constexpr int kKhOff = kKc, kKsOff = kKhOff + kKh, kKmOff = kKsOff + kKs;
-  static constexpr int kVcOff = kKmOff + kKm, kVsOff = kVcOff + kVc;
-  static constexpr int kBytes = kVsOff + kVs;
+  static constexpr int kVcOff = kKmOff + kKm, kVsOff = kVcOff + kVc, kVmOff = kVsOff + kVs;
+  static constexpr int kBytes = kVmOff + kVm;
   // the regions' offsets in a K page
   static constexpr int kPageScaleOff = KF == kKeyQ8 ? kKScaleOffset : KF == kKeyQ4 ? kK4ScaleOffset : kK5ScaleOffset;
 };
 constexpr int kRawStageBytes = Raw<kKeyQ8>::kBytes;  // 13,824 (the largest layout)
-static_assert(Raw<kKeyQ51>::kBytes <= kRawStageBytes && Raw<kKeyQ4>::kBytes <= kRawStageBytes, "raw stage");
+static_assert(Raw<kKeyQ51>::kBytes <= kRawStageBytes && Raw<kKeyQ4>::kBytes <= kRawStageBytes &&
+                  Raw<kKeyQ50>::kBytes <= kRawStageBytes,
+              "raw stage");
 constexpr int kRawStages = 2;
 constexpr int kBufs = 3;          // K^ / V^T buffer sets: dequant runs up to two tiles ahead of the MMAs
 constexpr int kPart = 16384;      // one of K^_hi, K^_lo (4 atoms x [32 keys][128 B]), V^T_hi, V^T_lo ([128][128 B])
@@ -259,6 +268,14 @@ __device__ __forceinline__ void split_affine(uint32_t code, float d, float m, ui
   lo = pack_half2(v0 - half_lo(hi), v1 - half_hi(hi));
 }
 
+// split_affine for a pair of values with a scale and a minimum each (Q4_1 values: the two halves
+// belong to two tokens): hi = f16(q * d + m), lo = f16 of the exact fp32 remainder.
+__device__ __forceinline__ void split_affine2(uint32_t code, uint32_t d, uint32_t m, uint32_t& hi, uint32_t& lo) {
+  const float v0 = fmaf(half_lo(code), half_lo(d), half_lo(m)), v1 = fmaf(half_hi(code), half_hi(d), half_hi(m));
+  hi = pack_half2(v0, v1);
+  lo = pack_half2(v0 - half_lo(hi), v1 - half_hi(hi));
+}
+
 // x shifted left by s bits (right by -s when s < 0); s is a compile-time constant after unrolling.
 __device__ __forceinline__ uint32_t shl(uint32_t x, int s) { return s >= 0 ? x << s : x >> -s; }
 
@@ -268,6 +285,7 @@ __device__ __forceinline__ uint32_t shl(uint32_t x, int s) { return s >= 0 ? x <
 template <int KF, bool EXACT>
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillParams p) {
   using RawF = pf::Raw<KF>;
+  constexpr bool kV41 = pf::value_q41(KF);
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pf::kMiscOff);
   uint64_t* rawfull = bars + 0;    // [2] producer (tx bytes) -> dequant
@@ -381,6 +399,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         for (int g = 0; g < 4; ++g)
           bulk_g2s(st + RawF::kVcOff + g * 1024, vp + half * 8192 + g * 2048 + crank * 1024, 1024, &rawfull[r]);
         bulk_g2s(st + RawF::kVsOff, vp + kV4ScaleOffset + half * RawF::kVs, RawF::kVs, &rawfull[r]);
+        if constexpr (RawF::kVm > 0)
+          bulk_g2s(st + RawF::kVmOff, vp + kV41MinOffset + half * RawF::kVm, RawF::kVm, &rawfull[r]);
       }
       // every copy issued must land before the CTA may exit
       for (int jj = j - pf::kRawStages < 0 ? 0 : j - pf::kRawStages; jj < j; ++jj)
@@ -635,7 +655,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       uint32_t kw[2][4] = {};  // per chunk i: the 4 words (8 codes of block 2kP, 8 of 2kP + 1)
       uint32_t kh[2] = {};     // Q5_1: per chunk i, the fifth bits of blocks 2kP, 2kP + 1 at bits 0-7, 16-23
       uint32_t dkw = 0, mkw = 0;
-      uint2 vraw[4] = {}, dvr[4] = {};
+      uint2 vraw[4] = {}, dvr[4] = {}, mvr[4] = {};
       if (wok) {
         if constexpr (KF != kKeyQ8) {
           // 4-bit key words (Q5_1: the low nibbles) of token kl, blocks 2kP, 2kP + 1 (c = 2kP % 4,
@@ -649,7 +669,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
             const uint2 w2 = lds64(stu + 4 * (row * 4 + ((2 * kP) & 3)));
             kw[i][0] = w2.x;
             kw[i][1] = w2.y;
-            if constexpr (KF == kKeyQ51) kh[i] = lds32(stu + RawF::kKhOff + 4 * row) >> (4 * ((2 * kP) & 3));
+            if constexpr (RawF::kK5) kh[i] = lds32(stu + RawF::kKhOff + 4 * row) >> (4 * ((2 * kP) & 3));
           }
         } else {
           const uint32_t kbase = stu + ((((kGl * 4 + kP) * 2 + kH) * 8 + kR) * 4) * 16;
@@ -670,6 +690,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         for (int ii = 0; ii < 4; ++ii) vraw[ii] = lds64(vbase + (((ii + rotV) & 3) << 4));
 #pragma unroll
         for (int T = 0; T < 4; ++T) dvr[T] = lds64(stu + RawF::kVsOff + ((vG * 4 + T) * 8 + 2 * vC) * 8 + 8 * ve);
+        if constexpr (RawF::kVm > 0) {
+#pragma unroll
+          for (int T = 0; T < 4; ++T) mvr[T] = lds64(stu + RawF::kVmOff + ((vG * 4 + T) * 8 + 2 * vC) * 8 + 8 * ve);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&rawempty[r]);
@@ -692,21 +716,23 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
               c[4 * e + 2] = hsub2(and_or(ws, 0x000F000Fu, 0x64006400u), 0x64086408u);
               c[4 * e + 3] = hfma2(and_or(ws, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
             }
-          } else if constexpr (KF == kKeyQ51) {
+          } else if constexpr (RawF::kK5) {
             // as Q4_0, with the fifth bit (channel (e, i) at bit 4e + i / 2 + 16 (i % 2) of kh)
             // moved to the 16s place of the code: bit 4 of the halves 1024 + q, bit 8 of the
-            // halves 1024 + 16q; the codes q in [0, 31] are exact in f16
+            // halves 1024 + 16q; the codes q in [0, 31] (Q5_1) or q - 16 (Q5_0) are exact in f16
+            constexpr uint32_t kSubLo = KF == kKeyQ50 ? 0x64106410u : 0x64006400u;  // 1024 (+ 16)
+            constexpr uint32_t kAddHi = KF == kKeyQ50 ? 0xD500D500u : 0xD400D400u;  // -64 (- 16)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const uint32_t w = kw[i][e], ws = w >> 8, x = kh[i];
               c[4 * e + 0] = hsub2(or_and(and_or(w, 0x000F000Fu, 0x64006400u), shl(x, 4 - 4 * e), 0x00100010u),
-                                   0x64006400u);
+                                   kSubLo);
               c[4 * e + 1] = hfma2(or_and(and_or(w, 0x00F000F0u, 0x64006400u), shl(x, 7 - 4 * e), 0x01000100u),
-                                   0x2C002C00u, 0xD400D400u);
+                                   0x2C002C00u, kAddHi);
               c[4 * e + 2] = hsub2(or_and(and_or(ws, 0x000F000Fu, 0x64006400u), shl(x, 2 - 4 * e), 0x00100010u),
-                                   0x64006400u);
+                                   kSubLo);
               c[4 * e + 3] = hfma2(or_and(and_or(ws, 0x00F000F0u, 0x64006400u), shl(x, 5 - 4 * e), 0x01000100u),
-                                   0x2C002C00u, 0xD400D400u);
+                                   0x2C002C00u, kAddHi);
             }
           } else {
 #pragma unroll
@@ -768,11 +794,27 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
           const uint32_t W = wv[T];
           const uint32_t Ws = W >> 8;
           const uint32_t dv = vh ? dvr[T].y : dvr[T].x;
-          const uint32_t v0 = hsub2(and_or(W, 0x000F000Fu, 0x64006400u), 0x64086408u);
-          const uint32_t v1 = hfma2(and_or(W, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
-          const uint32_t v2 = hsub2(and_or(Ws, 0x000F000Fu, 0x64006400u), 0x64086408u);
-          const uint32_t v3 = hfma2(and_or(Ws, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
-          if constexpr (EXACT) {
+          // Q4_0: q - 8 (1024 + q - 1032, or (1024 + 16q) / 16 - 72); Q4_1: q
+          constexpr uint32_t kVSubLo = kV41 ? 0x64006400u : 0x64086408u;
+          constexpr uint32_t kVAddHi = kV41 ? 0xD400D400u : 0xD480D480u;
+          const uint32_t v0 = hsub2(and_or(W, 0x000F000Fu, 0x64006400u), kVSubLo);
+          const uint32_t v1 = hfma2(and_or(W, 0x00F000F0u, 0x64006400u), 0x2C002C00u, kVAddHi);
+          const uint32_t v2 = hsub2(and_or(Ws, 0x000F000Fu, 0x64006400u), kVSubLo);
+          const uint32_t v3 = hfma2(and_or(Ws, 0x00F000F0u, 0x64006400u), 0x2C002C00u, kVAddHi);
+          if constexpr (kV41 && EXACT) {
+            // q * d + m per token (each half of the pair has its own scale and minimum)
+            const uint32_t mv = vh ? mvr[T].y : mvr[T].x;
+            split_affine2(v0, dv, mv, oh[0][T], ol[0][T]);
+            split_affine2(v1, dv, mv, oh[1][T], ol[1][T]);
+            split_affine2(v2, dv, mv, oh[2][T], ol[2][T]);
+            split_affine2(v3, dv, mv, oh[3][T], ol[3][T]);
+          } else if constexpr (kV41) {
+            const uint32_t mv = vh ? mvr[T].y : mvr[T].x;
+            oh[0][T] = hfma2(v0, dv, mv);
+            oh[1][T] = hfma2(v1, dv, mv);
+            oh[2][T] = hfma2(v2, dv, mv);
+            oh[3][T] = hfma2(v3, dv, mv);
+          } else if constexpr (EXACT) {
             split_product(v0, dv, oh[0][T], ol[0][T]);
             split_product(v1, dv, oh[1][T], ol[1][T]);
             split_product(v2, dv, oh[2][T], ol[2][T]);
@@ -819,8 +861,11 @@ static cudaError_t prepare_prefill_t() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(prefill_kernel<kKeyQ4, EXACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              pf::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_kernel<kKeyQ51, EXACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pf::kSmemBytes);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(prefill_kernel<kKeyQ51, EXACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(prefill_kernel<kKeyQ50, EXACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               pf::kSmemBytes);
 }
 
@@ -833,6 +878,7 @@ template <bool EXACT>
 static cudaError_t launch_prefill_grid(const cudaLaunchConfig_t& cfg, const PrefillParams& prm, int key_fmt) {
   return key_fmt == kKeyQ4    ? cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ4, EXACT>, prm)
          : key_fmt == kKeyQ51 ? cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ51, EXACT>, prm)
+         : key_fmt == kKeyQ50 ? cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ50, EXACT>, prm)
                               : cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ8, EXACT>, prm);
 }
 

@@ -174,11 +174,14 @@ WORKLOADS = {
     # 2,048-token bf16 chunk (4 ubatches of 512) over 524,288 prior tokens, 4,096-token KV splits.
     "prefill524k": Workload("prefill524k", layers=16, kv_heads=4, q_heads=24, context=524288, n_q=2048,
                             ubatch=512, kv_split_tokens=4096, seed=4004),
-    # the same prefill over the other key formats that chunked prefill takes (Q4_0 values)
+    # the same prefill over the other format pairs that chunked prefill takes
     "prefill524k_q4q4": Workload("prefill524k_q4q4", layers=16, kv_heads=4, q_heads=24, context=524288,
                                  n_q=2048, k_fmt="q4_0", ubatch=512, kv_split_tokens=4096, seed=4005),
     "prefill524k_q51q4": Workload("prefill524k_q51q4", layers=16, kv_heads=4, q_heads=24, context=524288,
                                   n_q=2048, k_fmt="q5_1", ubatch=512, kv_split_tokens=4096, seed=4006),
+    "prefill524k_q50q41": Workload("prefill524k_q50q41", layers=16, kv_heads=4, q_heads=24, context=524288,
+                                   n_q=2048, k_fmt="q5_0", v_fmt="q4_1", ubatch=512, kv_split_tokens=4096,
+                                   seed=4007),
     # 524,288 tokens in pinned host RAM, 256-block working set per (layer, head), 512 steps.
     "stream524k": Workload("stream524k", layers=16, kv_heads=4, q_heads=24, context=524288, n_q=1,
                            budget_blocks=256, recent_blocks=0, steps=512, seed=5005),

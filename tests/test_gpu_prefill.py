@@ -30,7 +30,7 @@ def _prefill(kv, cache, H_q, q, q_pos, page_list, split, page_logical=None, n_pa
     return out.cpu().numpy(), lse.cpu().numpy()
 
 
-def _case(seed, H, n_prior, n_q, outliers=True, k_fmt="q8_0"):
+def _case(seed, H, n_prior, n_q, outliers=True, k_fmt="q8_0", v_fmt="q4_0"):
     rng = np_rng(seed)
     T = n_prior + n_q
     k = normal_f32(rng, (T, H, 256))
@@ -42,38 +42,41 @@ def _case(seed, H, n_prior, n_q, outliers=True, k_fmt="q8_0"):
             v[:, h, ch] *= 8
     n_blocks = (T + 127) // 128
     n_phys = H * n_blocks + 3
-    cache = GpuCache(H, 6 * H, n_blocks, "q4_0", n_phys=n_phys, perm=page_permutation(rng, n_phys), k_fmt=k_fmt)
+    cache = GpuCache(H, 6 * H, n_blocks, v_fmt, n_phys=n_phys, perm=page_permutation(rng, n_phys), k_fmt=k_fmt)
     cache.append(k, v, 0)
     q = bf16_round(normal_f32(rng, (n_q, 6 * H, 256)))
     return rng, k, v, q, cache, T
 
 
-@pytest.mark.parametrize("k_fmt", ["q8_0", "q4_0", "q5_1"])
+PAIRS = [("q8_0", "q4_0"), ("q4_0", "q4_0"), ("q5_1", "q4_0"), ("q5_0", "q4_1")]
+
+
+@pytest.mark.parametrize("k_fmt,v_fmt", PAIRS)
 @pytest.mark.parametrize("n_prior,n_q,split", [(700, 40, 256), (1024, 64, 128), (300, 22, 512), (5000, 130, 1024),
                                                (0, 30, 128), (127, 1, 256)])
-def test_prefill_matches_oracle(kv_gpu, n_prior, n_q, split, k_fmt):
+def test_prefill_matches_oracle(kv_gpu, n_prior, n_q, split, k_fmt, v_fmt):
     """x8 outlier channels and short contexts: outputs of magnitude up to ~25 that average few
     values, where the rounding of any f16 operand would show."""
     H = 2
-    rng, k, v, q, cache, T = _case(1200 + n_prior + n_q, H, n_prior, n_q, k_fmt=k_fmt)
+    rng, k, v, q, cache, T = _case(1200 + n_prior + n_q, H, n_prior, n_q, k_fmt=k_fmt, v_fmt=v_fmt)
     q_pos = np.arange(n_prior, T)
     out, lse = _prefill(kv_gpu, cache, 6 * H, q, q_pos, cache.page_table_np, split)
-    oc = OracleCache(k, v, "q4_0", k_fmt)
+    oc = OracleCache(k, v, v_fmt, k_fmt)
     for h in range(H):
         o_ref, l_ref = oc.attend(q, q_pos, h, 6)
         compare(out[:, 6 * h:6 * h + 6], lse[:, 6 * h:6 * h + 6], o_ref, l_ref)
 
 
-@pytest.mark.parametrize("k_fmt", ["q8_0", "q4_0", "q5_1"])
+@pytest.mark.parametrize("k_fmt,v_fmt", PAIRS)
 @pytest.mark.parametrize("n_prior,n_q,split", [(700, 40, 256), (5000, 130, 1024), (0, 30, 128), (4096, 512, 4096)])
-def test_prefill_f16_matches_oracle(kv_gpu, n_prior, n_q, split, k_fmt):
+def test_prefill_f16_matches_oracle(kv_gpu, n_prior, n_q, split, k_fmt, v_fmt):
     """The one-rounding operand mode on the prefill workload's distribution (K, V and Q drawn
     N(0, 1), no outlier channels): within the same absolute bound as the exact mode."""
     H = 2
-    rng, k, v, q, cache, T = _case(1700 + n_prior + n_q, H, n_prior, n_q, outliers=False, k_fmt=k_fmt)
+    rng, k, v, q, cache, T = _case(1700 + n_prior + n_q, H, n_prior, n_q, outliers=False, k_fmt=k_fmt, v_fmt=v_fmt)
     q_pos = np.arange(n_prior, T)
     out, lse = _prefill(kv_gpu, cache, 6 * H, q, q_pos, cache.page_table_np, split, f16=True)
-    oc = OracleCache(k, v, "q4_0", k_fmt)
+    oc = OracleCache(k, v, v_fmt, k_fmt)
     for h in range(H):
         o_ref, l_ref = oc.attend(q, q_pos, h, 6)
         compare(out[:, 6 * h:6 * h + 6], lse[:, 6 * h:6 * h + 6], o_ref, l_ref)
