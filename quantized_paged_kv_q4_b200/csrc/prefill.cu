@@ -1,6 +1,6 @@
 // Chunked prefill over block-quantized KV pages (Q8_0, Q4_0 or Q5_1 keys with Q4_0 values, Q5_0
-// keys with Q4_1 values) on
-// tcgen05 tensor cores (Adaptive KV Streaming + RDNA 4 announcement, wqu.guru, method list:
+// keys with Q4_1 values) on tcgen05 tensor cores (Adaptive KV Streaming + RDNA 4 announcement,
+// wqu.guru, method list:
 // "online log-sum-exp prefill": the prefill of a chunk is computed across streamed KV pages
 // and the partial results are accumulated by online log-sum-exp; the six-step validation
 // guide, alphalab.site, build step: the q8_0-q4_0 and q4_0-q4_0 flash-attention KV pairs;
