@@ -1101,7 +1101,7 @@ def main():
             # the same prefill layer over the other format pairs, and with operands rounded once to f16
             # (kvattn_prefill_chunk_f16); one layer each: kernel rate only
             for wn, f16 in (("prefill524k_q4q4", False), ("prefill524k_q51q4", False), ("prefill524k_q50q41", False),
-                            ("prefill524k", True)):
+                            ("prefill524k_q8q8", False), ("prefill524k", True)):
                 b6 = PrefillBench(kvattn, device, layers=1, wname=wn, f16=f16)
                 b6.layer(0)
                 k6 = time_layers(b6, 2)

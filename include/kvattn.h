@@ -304,9 +304,9 @@ KVATTN_API int kvattn_select_blocks(const float* summaries, const float* q_group
  * accumulation in tensor memory, so every operand carries about 22 significant bits.  The
  * keys are taken in splits of kv_split_tokens (a multiple of 128, at most 65,536; a CTA may
  * walk several consecutive splits); partial results are merged by log-sum-exp.  A page id
- * outside [0, n_pages) skips its page and records KVATTN_ERR_BAD_PAGE.  Needs Q8_0, Q4_0 or
- * Q5_1 K with Q4_0 V pages, or Q5_0 K with Q4_1 V pages (UNSUPPORTED_FORMAT otherwise;
- * [GUIDE] build step: the q8_0-q4_0 and q4_0-q4_0 pairs; [VULKAN] pitfalls: Q5_1 K with Q4_0
+ * outside [0, n_pages) skips its page and records KVATTN_ERR_BAD_PAGE.  Takes every format
+ * pair of the descriptor: Q8_0, Q4_0 or Q5_1 K with Q4_0 or Q8_0 V, and Q5_0 K with Q4_1 V
+ * ([GUIDE] build step: the q8_0-q4_0 and q4_0-q4_0 pairs; [VULKAN] pitfalls: Q5_1 K with Q4_0
  * V; [MTP]: the Q5_0 K / Q4_1 V cache).
  *   q      device bf16 bits [n_q][H_q][256];  out device fp32 [n_q][H_q][256];
  *   lse    device fp32 [n_q][H_q];  page arguments as for kvattn_decode.

@@ -598,10 +598,7 @@ int prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* q, int n_q, const 
                   bool exact) {
   int st = validate_desc(desc);
   if (st) return st;
-  const bool v40_pair = (desc->k_fmt == KVATTN_FMT_Q8_0 || desc->k_fmt == KVATTN_FMT_Q4_0 ||
-                         desc->k_fmt == KVATTN_FMT_Q5_1) &&
-                        desc->v_fmt == KVATTN_FMT_Q4_0;
-  if (!v40_pair && !(desc->k_fmt == KVATTN_FMT_Q5_0 && desc->v_fmt == KVATTN_FMT_Q4_1))
+  if (!prefill_pair_supported(key_format_id(desc->k_fmt), value_format_id(desc->v_fmt)))
     return KVATTN_ERR_UNSUPPORTED_FORMAT;
   if (n_q < 1 || max_pages < 0 || !q || !q_pos || !out || !lse || (max_pages > 0 && !page_list))
     return KVATTN_ERR_INVALID_ARG;
@@ -644,7 +641,8 @@ int prefill_chunk(const kvattn_kv_desc* desc, const uint16_t* q, int n_q, const 
   prm.n_ks = plan.n_ks;
   prm.rows_pad = plan.rows_pad;
   cudaError_t e =
-      launch_prefill(prm, desc->n_kv_heads, key_format_id(desc->k_fmt), exact, static_cast<cudaStream_t>(stream));
+      launch_prefill(prm, desc->n_kv_heads, key_format_id(desc->k_fmt), value_format_id(desc->v_fmt), exact,
+                     static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVATTN_OK : cuda_fail(e);
 }
 

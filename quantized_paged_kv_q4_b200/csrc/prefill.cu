@@ -69,41 +69,42 @@ constexpr int kDq0 = (kSoftmaxWarps + 2) * 32;  // first dequant thread
 // scales (Q5_1: then minima) of its 32 keys (each region contiguous in the page), V codes of
 // its 128 head dimensions for all 64 keys (four 1 KB pieces, one per 16-key group), and all
 // V scales of the tile; the stage holds them in that order
-// The value format is fixed by the key format: Q4_0 values under Q8_0, Q4_0 and Q5_1 keys,
-// Q4_1 values under Q5_0 keys (the format pairs chunked prefill takes).
-__host__ __device__ constexpr bool value_q41(int KF) { return KF == kKeyQ50; }
-template <int KF>
+template <int KF, int VF>
 struct Raw {
   static constexpr bool kK5 = KF == kKeyQ51 || KF == kKeyQ50;
   static constexpr int kKc = KF == kKeyQ8 ? 8192 : 4096;  // 32 keys x 256 or 128 bytes
   static constexpr int kKh = kK5 ? 1024 : 0;              // fifth bits: 32 keys x 32 bytes
-  static constexpr int kKs = 512, kVc = 4096, kVs = 1024;
+  static constexpr int kKs = 512, kVs = 1024;
   static constexpr int kKm = KF == kKeyQ51 ? 512 : 0;     // key minima
-  static constexpr int kVm = value_q41(KF) ? 1024 : 0;    // value minima (Q4_1), as the scales
+  static constexpr int kVc = VF == kValQ8 ? 8192 : 4096;  // 128 dimensions x 64 keys, 8 or 4 bits
+  static constexpr int kVm = VF == kValQ41 ? 1024 : 0;    // value minima (Q4_1), as the scales
   static constexpr int kKhOff = kKc, kKsOff = kKhOff + kKh, kKmOff = kKsOff + kKs;
   static constexpr int kVcOff = kKmOff + kKm, kVsOff = kVcOff + kVc, kVmOff = kVsOff + kVs;
   static constexpr int kBytes = kVmOff + kVm;
-  // the regions' offsets in a K page
+  // the regions' offsets in a page
   static constexpr int kPageScaleOff = KF == kKeyQ8 ? kKScaleOffset : KF == kKeyQ4 ? kK4ScaleOffset : kK5ScaleOffset;
+  static constexpr int kPageVScaleOff = VF == kValQ8 ? kV8ScaleOffset : kV4ScaleOffset;
 };
-constexpr int kRawStageBytes = Raw<kKeyQ8>::kBytes;  // 13,824 (the largest layout)
-static_assert(Raw<kKeyQ51>::kBytes <= kRawStageBytes && Raw<kKeyQ4>::kBytes <= kRawStageBytes &&
-                  Raw<kKeyQ50>::kBytes <= kRawStageBytes,
-              "raw stage");
 constexpr int kRawStages = 2;
-constexpr int kBufs = 3;          // K^ / V^T buffer sets: dequant runs up to two tiles ahead of the MMAs
 constexpr int kPart = 16384;      // one of K^_hi, K^_lo (4 atoms x [32 keys][128 B]), V^T_hi, V^T_lo ([128][128 B])
 constexpr int kSet = 2 * kPart;   // hi + lo
 // a CTA walks at most this many 64-key tiles (the host plan keeps pages per CTA <= 256)
 constexpr int kMaxTiles = 512;
-// shared memory map (bytes)
-constexpr int kKOff = 0;                                  // kBufs x (K^_hi, K^_lo)
-constexpr int kVOff = kKOff + kBufs * kSet;               // kBufs x (V^T_hi, V^T_lo)
-constexpr int kRawOff = kVOff + kBufs * kSet;             // kRawStages stages of raw tile bytes
-constexpr int kTileOff = kRawOff + kRawStages * kRawStageBytes;  // int2 [kMaxTiles]: page, 2*logical+half
-constexpr int kMiscOff = kTileOff + 8 * kMaxTiles;
-constexpr int kSmemBytes = kMiscOff + 512;
-static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+// Shared memory map (bytes) of a format pair.  Three K^ / V^T buffer sets let the dequant run
+// up to two tiles ahead of the MMAs; Q8_0 values double the raw bytes of a tile, and two sets
+// then fit.
+template <int KF, int VF>
+struct Layout {
+  static constexpr int kBufs = VF == kValQ8 ? 2 : 3;
+  static constexpr int kRawStageBytes = Raw<KF, VF>::kBytes;
+  static constexpr int kKOff = 0;                                  // kBufs x (K^_hi, K^_lo)
+  static constexpr int kVOff = kKOff + kBufs * kSet;               // kBufs x (V^T_hi, V^T_lo)
+  static constexpr int kRawOff = kVOff + kBufs * kSet;             // kRawStages stages of raw tile bytes
+  static constexpr int kTileOff = kRawOff + kRawStages * kRawStageBytes;  // int2 [kMaxTiles]: page, 2*logical+half
+  static constexpr int kMiscOff = kTileOff + 8 * kMaxTiles;
+  static constexpr int kSmemBytes = kMiscOff + 512;
+  static_assert(kRawStageBytes % 16 == 0 && kSmemBytes <= 227 * 1024, "shared memory");
+};
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol0 = 0;    // S buffers [0,64), [64,128); P_hi over the first 32, P_lo over the next 32
@@ -282,12 +283,13 @@ __device__ __forceinline__ uint32_t shl(uint32_t x, int s) { return s >= 0 ? x <
 // EXACT: every operand as an f16 high part plus a low part (about 22 significant bits, QK as
 // two MMA passes, PV as three); otherwise each dequantized value and each P rounded once to
 // f16 (one pass each; the dequant writes, and the MMAs read, the high parts only).
-template <int KF, bool EXACT>
+template <int KF, int VF, bool EXACT>
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillParams p) {
-  using RawF = pf::Raw<KF>;
-  constexpr bool kV41 = pf::value_q41(KF);
+  using RawF = pf::Raw<KF, VF>;
+  using L = pf::Layout<KF, VF>;
+  constexpr bool kV41 = VF == kValQ41, kV8 = VF == kValQ8;
   extern __shared__ __align__(1024) uint8_t smem[];
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + pf::kMiscOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kMiscOff);
   uint64_t* rawfull = bars + 0;    // [2] producer (tx bytes) -> dequant
   uint64_t* rawempty = bars + 2;   // [2] dequant -> producer
   uint64_t* kready = bars + 4;     // [3] even CTA: K^ halves of both CTAs in place -> MMA
@@ -302,7 +304,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(bars + 23);
   int* s_abort = reinterpret_cast<int*>(tmem_base_s + 1);
   int* s_ntiles = s_abort + 1;
-  const int2* tiles = reinterpret_cast<const int2*>(smem + pf::kTileOff);
+  const int2* tiles = reinterpret_cast<const int2*>(smem + L::kTileOff);
 
   const int mt = blockIdx.x, ks = blockIdx.y, h = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -326,7 +328,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       mbar_init(&rawfull[b], 1);
       mbar_init(&rawempty[b], pf::kDequantWarps);
     }
-    for (int b = 0; b < pf::kBufs; ++b) {
+    for (int b = 0; b < L::kBufs; ++b) {
       mbar_init(&kready[b], 2);  // one arrival from the dequant warps of each CTA
       mbar_init(&vready[b], 2);
       mbar_init(&kfree[b], 1);
@@ -345,7 +347,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
   }
   if (warp == 0) {
     // the CTA's tiles in key order, compacted once: (page, 2 * logical block + half)
-    int2* list = reinterpret_cast<int2*>(smem + pf::kTileOff);
+    int2* list = reinterpret_cast<int2*>(smem + L::kTileOff);
     int n_cand = 2 * p.pages_per_split;
     if (n_cand > pf::kMaxTiles) {
       if (lane == 0) record_error(KVATTN_ERR_INVALID_ARG);
@@ -386,7 +388,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         }
         // K: this CTA's 32 keys of the tile (quarter q of the page); V: its 128 dimensions
         const int half = tl.y & 1, q = 2 * half + static_cast<int>(crank);
-        uint8_t* st = smem + pf::kRawOff + r * pf::kRawStageBytes;
+        uint8_t* st = smem + L::kRawOff + r * L::kRawStageBytes;
         const uint8_t* kp = p.k_pool + static_cast<int64_t>(tl.x) * p.k_stride;
         const uint8_t* vp = p.v_pool + static_cast<int64_t>(tl.x) * p.v_stride;
         mbar_arrive_expect_tx(&rawfull[r], RawF::kBytes);
@@ -396,9 +398,13 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         bulk_g2s(st + RawF::kKsOff, kp + RawF::kPageScaleOff + q * RawF::kKs, RawF::kKs, &rawfull[r]);
         if constexpr (RawF::kKm > 0)
           bulk_g2s(st + RawF::kKmOff, kp + kK5MinOffset + q * RawF::kKm, RawF::kKm, &rawfull[r]);
+        // V codes: per 16-key group g of the tile half, this CTA's half of the group's bytes (the
+        // 1 KB of its two block pairs in Q4 pages, the 2 KB of its four blocks in Q8_0 pages)
+        constexpr int kVPiece = RawF::kVc / 4, kVGroup = 2 * kVPiece;
         for (int g = 0; g < 4; ++g)
-          bulk_g2s(st + RawF::kVcOff + g * 1024, vp + half * 8192 + g * 2048 + crank * 1024, 1024, &rawfull[r]);
-        bulk_g2s(st + RawF::kVsOff, vp + kV4ScaleOffset + half * RawF::kVs, RawF::kVs, &rawfull[r]);
+          bulk_g2s(st + RawF::kVcOff + g * kVPiece, vp + (4 * half + g) * kVGroup + crank * kVPiece, kVPiece,
+                   &rawfull[r]);
+        bulk_g2s(st + RawF::kVsOff, vp + RawF::kPageVScaleOff + half * RawF::kVs, RawF::kVs, &rawfull[r]);
         if constexpr (RawF::kVm > 0)
           bulk_g2s(st + RawF::kVmOff, vp + kV41MinOffset + half * RawF::kVm, RawF::kVm, &rawfull[r]);
       }
@@ -414,8 +420,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     // place and the S buffer it overwrites was consumed by PV two tiles back) and PV of the
     // oldest tile whose P is written in both CTAs.
     if (leader) {
-      const uint32_t k_base = smem_u32(smem + pf::kKOff);
-      const uint32_t v_base = smem_u32(smem + pf::kVOff);
+      const uint32_t k_base = smem_u32(smem + L::kKOff);
+      const uint32_t v_base = smem_u32(smem + L::kVOff);
       auto ready_all = [&](uint64_t* bar, uint32_t par) -> bool {
         return __all_sync(0xffffffffu, mbar_try_wait_cluster(bar, par, 0u));
       };
@@ -424,8 +430,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       unsigned long long t_idle = 0;
       while (ok && jp < n_tiles) {
         bool did = false;
-        if (jq < n_tiles && jq <= jp + 1 && ready_all(&kready[jq % pf::kBufs], (jq / pf::kBufs) & 1)) {
-          const int b = jq % pf::kBufs, s2 = jq & 1;
+        if (jq < n_tiles && jq <= jp + 1 && ready_all(&kready[jq % L::kBufs], (jq / L::kBufs) & 1)) {
+          const int b = jq % L::kBufs, s2 = jq & 1;
           tc::fence_after_sync();
 #pragma unroll
           for (int kk = 0; kk < kHeadDim / 16; ++kk) {
@@ -440,8 +446,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
           ++jq;
           did = true;
         } else if (jp < jq && ready_all(&pready[jp & 1], (jp >> 1) & 1) &&
-                   ready_all(&vready[jp % pf::kBufs], (jp / pf::kBufs) & 1)) {
-          const int b = jp % pf::kBufs, s2 = jp & 1;
+                   ready_all(&vready[jp % L::kBufs], (jp / L::kBufs) & 1)) {
+          const int b = jp % L::kBufs, s2 = jp & 1;
           tc::fence_after_sync();
 #pragma unroll
           for (int kk = 0; kk < pf::kKeys / 16; ++kk) {
@@ -637,6 +643,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     // half vh of token group vG (16 keys)
     const int vR = d & 7, vh = (d >> 3) & 1, vCl = (d >> 4) & 1, vG = (d >> 5) & 3, ve = d >> 7;
     const int vC = 2 * static_cast<int>(crank) + vCl;
+    // Q8_0 V task: channel row vR8 (channels vR8 + 8k of this CTA's block vb8), key half vh8 of
+    // token group vG8: the byte pairs of tokens 2T, 2T + 1 (T = 0..3) sit in words vh8 and
+    // vh8 + 2 of raw chunk T of (vG8, vb8, vR8)
+    const int vR8 = d & 7, vh8 = (d >> 3) & 1, vb8 = (d >> 4) & 3, vG8 = (d >> 6) & 3;
     // 16-byte chunks are read in an order rotated by (row / 2): 8 threads at a 64-byte
     // stride then touch 8 different bank groups
     const int rotK = kR >> 1, rotV = vR >> 1;
@@ -646,16 +656,17 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
     int j = 0;
     bool ok = true;
     for (; j < n_tiles && ok; ++j) {
-      const int b = j % pf::kBufs, r = j % pf::kRawStages;
+      const int b = j % L::kBufs, r = j % pf::kRawStages;
       // every wait result is combined over the 256 dequant threads at the named barriers, so
       // all of them stop at the same tile when one gives up
       bool wok = mbar_wait(&rawfull[r], (j / pf::kRawStages) & 1);
-      const uint32_t stu = own + pf::kRawOff + r * pf::kRawStageBytes;
+      const uint32_t stu = own + L::kRawOff + r * L::kRawStageBytes;
       // ---------------- raw K, V -> registers; the stage is then released ----------------
       uint32_t kw[2][4] = {};  // per chunk i: the 4 words (8 codes of block 2kP, 8 of 2kP + 1)
       uint32_t kh[2] = {};     // Q5_1: per chunk i, the fifth bits of blocks 2kP, 2kP + 1 at bits 0-7, 16-23
       uint32_t dkw = 0, mkw = 0;
       uint2 vraw[4] = {}, dvr[4] = {}, mvr[4] = {};
+      uint32_t v8w[4][2] = {}, d8[4] = {};  // Q8_0 values: per token pair T, words vh8, vh8 + 2; scales
       if (wok) {
         if constexpr (KF != kKeyQ8) {
           // 4-bit key words (Q5_1: the low nibbles) of token kl, blocks 2kP, 2kP + 1 (c = 2kP % 4,
@@ -685,21 +696,32 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
         if constexpr (KF == kKeyQ51) mkw = lds32(stu + RawF::kKmOff + sidx);
         // this thread's two words (block 2vC + ve, both key halves) of each raw chunk and of
         // the scales of each token pair
-        const uint32_t vbase = stu + RawF::kVcOff + vG * 1024 + ((vCl * 8 + vR) * 4) * 16 + 8 * ve;
+        if constexpr (kV8) {
+          const uint32_t v8base = stu + RawF::kVcOff + vG8 * 2048 + ((vb8 * 8 + vR8) * 4) * 16;
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) vraw[ii] = lds64(vbase + (((ii + rotV) & 3) << 4));
+          for (int T = 0; T < 4; ++T) {
+            v8w[T][0] = lds32(v8base + T * 16 + 4 * vh8);
+            v8w[T][1] = lds32(v8base + T * 16 + 4 * (vh8 + 2));
+            d8[T] = lds32(stu + RawF::kVsOff + ((vG8 * 4 + T) * 8 + 4 * static_cast<int>(crank) + vb8) * 8 + 4 * vh8);
+          }
+        } else {
+          const uint32_t vbase = stu + RawF::kVcOff + vG * 1024 + ((vCl * 8 + vR) * 4) * 16 + 8 * ve;
 #pragma unroll
-        for (int T = 0; T < 4; ++T) dvr[T] = lds64(stu + RawF::kVsOff + ((vG * 4 + T) * 8 + 2 * vC) * 8 + 8 * ve);
-        if constexpr (RawF::kVm > 0) {
+          for (int ii = 0; ii < 4; ++ii) vraw[ii] = lds64(vbase + (((ii + rotV) & 3) << 4));
 #pragma unroll
-          for (int T = 0; T < 4; ++T) mvr[T] = lds64(stu + RawF::kVmOff + ((vG * 4 + T) * 8 + 2 * vC) * 8 + 8 * ve);
+          for (int T = 0; T < 4; ++T) dvr[T] = lds64(stu + RawF::kVsOff + ((vG * 4 + T) * 8 + 2 * vC) * 8 + 8 * ve);
+          if constexpr (RawF::kVm > 0) {
+#pragma unroll
+            for (int T = 0; T < 4; ++T)
+              mvr[T] = lds64(stu + RawF::kVmOff + ((vG * 4 + T) * 8 + 2 * vC) * 8 + 8 * ve);
+          }
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&rawempty[r]);
       // ---------------- K^ (this CTA's buffer is free once QK(j - 3) completed) ----
-      if (wok && j >= pf::kBufs) wok = mbar_wait_cluster(&kfree[b], ((j / pf::kBufs) - 1) & 1);
-      const uint32_t katom = own + pf::kKOff + b * pf::kSet + kP * 4096;
+      if (wok && j >= L::kBufs) wok = mbar_wait_cluster(&kfree[b], ((j / L::kBufs) - 1) & 1);
+      const uint32_t katom = own + L::kKOff + b * pf::kSet + kP * 4096;
       if (wok) {
         const uint32_t dlo = prmt(dkw, 0u, 0x1010u), dhi = prmt(dkw, 0u, 0x3232u);
 #pragma unroll
@@ -775,62 +797,89 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
       }
       if (d == 0) mbar_arrive_cluster(kready_lead + 8 * b);
       // ---------------- V^T: this CTA's 128 dimensions ----------------
-      if (j >= pf::kBufs) wok = mbar_wait_cluster(&vfree[b], ((j / pf::kBufs) - 1) & 1);
-      const uint32_t vt = own + pf::kVOff + b * pf::kSet;
+      if (j >= L::kBufs) wok = mbar_wait_cluster(&vfree[b], ((j / L::kBufs) - 1) & 1);
+      const uint32_t vt = own + L::kVOff + b * pf::kSet;
       if (wok) {
-        // chunk ii holds token pair (ii + rotV) & 3: two select stages undo the rotation so
-        // that wv[T] is token pair T (an array indexed by the runtime rotation would be
-        // placed in local memory)
-        uint32_t wv[4], t[4];
+        if constexpr (kV8) {
+          // Q8_0 values: offset-binary code bytes 2(k % 2), 2(k % 2) + 1 of word k / 2 are channel
+          // vR8 + 8k of tokens 2T, 2T + 1 (1024 + (q + 128) - 1152 = q, exact in f16)
+          uint32_t oh[4][4], ol[4][4];  // [k][T]
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) wv[ii] = vh ? vraw[ii].y : vraw[ii].x;
+          for (int T = 0; T < 4; ++T) {
 #pragma unroll
-        for (int x = 0; x < 4; ++x) t[x] = (rotV & 1) ? wv[(x + 3) & 3] : wv[x];
-#pragma unroll
-        for (int x = 0; x < 4; ++x) wv[x] = (rotV & 2) ? t[(x + 2) & 3] : t[x];
-        uint32_t oh[4][4], ol[4][4];  // [k][T]
-#pragma unroll
-        for (int T = 0; T < 4; ++T) {
-          const uint32_t W = wv[T];
-          const uint32_t Ws = W >> 8;
-          const uint32_t dv = vh ? dvr[T].y : dvr[T].x;
-          // Q4_0: q - 8 (1024 + q - 1032, or (1024 + 16q) / 16 - 72); Q4_1: q
-          constexpr uint32_t kVSubLo = kV41 ? 0x64006400u : 0x64086408u;
-          constexpr uint32_t kVAddHi = kV41 ? 0xD400D400u : 0xD480D480u;
-          const uint32_t v0 = hsub2(and_or(W, 0x000F000Fu, 0x64006400u), kVSubLo);
-          const uint32_t v1 = hfma2(and_or(W, 0x00F000F0u, 0x64006400u), 0x2C002C00u, kVAddHi);
-          const uint32_t v2 = hsub2(and_or(Ws, 0x000F000Fu, 0x64006400u), kVSubLo);
-          const uint32_t v3 = hfma2(and_or(Ws, 0x00F000F0u, 0x64006400u), 0x2C002C00u, kVAddHi);
-          if constexpr (kV41 && EXACT) {
-            // q * d + m per token (each half of the pair has its own scale and minimum)
-            const uint32_t mv = vh ? mvr[T].y : mvr[T].x;
-            split_affine2(v0, dv, mv, oh[0][T], ol[0][T]);
-            split_affine2(v1, dv, mv, oh[1][T], ol[1][T]);
-            split_affine2(v2, dv, mv, oh[2][T], ol[2][T]);
-            split_affine2(v3, dv, mv, oh[3][T], ol[3][T]);
-          } else if constexpr (kV41) {
-            const uint32_t mv = vh ? mvr[T].y : mvr[T].x;
-            oh[0][T] = hfma2(v0, dv, mv);
-            oh[1][T] = hfma2(v1, dv, mv);
-            oh[2][T] = hfma2(v2, dv, mv);
-            oh[3][T] = hfma2(v3, dv, mv);
-          } else if constexpr (EXACT) {
-            split_product(v0, dv, oh[0][T], ol[0][T]);
-            split_product(v1, dv, oh[1][T], ol[1][T]);
-            split_product(v2, dv, oh[2][T], ol[2][T]);
-            split_product(v3, dv, oh[3][T], ol[3][T]);
-          } else {
-            oh[0][T] = hmul2(v0, dv);
-            oh[1][T] = hmul2(v1, dv);
-            oh[2][T] = hmul2(v2, dv);
-            oh[3][T] = hmul2(v3, dv);
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t code =
+                  hsub2(prmt(v8w[T][k >> 1], 0x64646464u, (k & 1) ? 0x4342u : 0x4140u), 0x64806480u);
+              if constexpr (EXACT) {
+                split_product(code, d8[T], oh[k][T], ol[k][T]);
+              } else {
+                oh[k][T] = hmul2(code, d8[T]);
+              }
+            }
           }
-        }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int row = 32 * (2 * vCl + ve) + 8 * k + vR;  // dimension - 128 * rank
-          sts128u(vt + swz(row, 2 * vG + vh), oh[k][0], oh[k][1], oh[k][2], oh[k][3]);
-          if constexpr (EXACT) sts128u(vt + pf::kPart + swz(row, 2 * vG + vh), ol[k][0], ol[k][1], ol[k][2], ol[k][3]);
+          for (int k = 0; k < 4; ++k) {
+            const int row = 32 * vb8 + 8 * k + vR8;  // dimension - 128 * rank
+            sts128u(vt + swz(row, 2 * vG8 + vh8), oh[k][0], oh[k][1], oh[k][2], oh[k][3]);
+            if constexpr (EXACT)
+              sts128u(vt + pf::kPart + swz(row, 2 * vG8 + vh8), ol[k][0], ol[k][1], ol[k][2], ol[k][3]);
+          }
+        } else {
+          // chunk ii holds token pair (ii + rotV) & 3: two select stages undo the rotation so
+          // that wv[T] is token pair T (an array indexed by the runtime rotation would be
+          // placed in local memory)
+          uint32_t wv[4], t[4];
+#pragma unroll
+          for (int ii = 0; ii < 4; ++ii) wv[ii] = vh ? vraw[ii].y : vraw[ii].x;
+#pragma unroll
+          for (int x = 0; x < 4; ++x) t[x] = (rotV & 1) ? wv[(x + 3) & 3] : wv[x];
+#pragma unroll
+          for (int x = 0; x < 4; ++x) wv[x] = (rotV & 2) ? t[(x + 2) & 3] : t[x];
+          uint32_t oh[4][4], ol[4][4];  // [k][T]
+#pragma unroll
+          for (int T = 0; T < 4; ++T) {
+            const uint32_t W = wv[T];
+            const uint32_t Ws = W >> 8;
+            const uint32_t dv = vh ? dvr[T].y : dvr[T].x;
+            // Q4_0: q - 8 (1024 + q - 1032, or (1024 + 16q) / 16 - 72); Q4_1: q
+            constexpr uint32_t kVSubLo = kV41 ? 0x64006400u : 0x64086408u;
+            constexpr uint32_t kVAddHi = kV41 ? 0xD400D400u : 0xD480D480u;
+            const uint32_t v0 = hsub2(and_or(W, 0x000F000Fu, 0x64006400u), kVSubLo);
+            const uint32_t v1 = hfma2(and_or(W, 0x00F000F0u, 0x64006400u), 0x2C002C00u, kVAddHi);
+            const uint32_t v2 = hsub2(and_or(Ws, 0x000F000Fu, 0x64006400u), kVSubLo);
+            const uint32_t v3 = hfma2(and_or(Ws, 0x00F000F0u, 0x64006400u), 0x2C002C00u, kVAddHi);
+            if constexpr (kV41 && EXACT) {
+              // q * d + m per token (each half of the pair has its own scale and minimum)
+              const uint32_t mv = vh ? mvr[T].y : mvr[T].x;
+              split_affine2(v0, dv, mv, oh[0][T], ol[0][T]);
+              split_affine2(v1, dv, mv, oh[1][T], ol[1][T]);
+              split_affine2(v2, dv, mv, oh[2][T], ol[2][T]);
+              split_affine2(v3, dv, mv, oh[3][T], ol[3][T]);
+            } else if constexpr (kV41) {
+              const uint32_t mv = vh ? mvr[T].y : mvr[T].x;
+              oh[0][T] = hfma2(v0, dv, mv);
+              oh[1][T] = hfma2(v1, dv, mv);
+              oh[2][T] = hfma2(v2, dv, mv);
+              oh[3][T] = hfma2(v3, dv, mv);
+            } else if constexpr (EXACT) {
+              split_product(v0, dv, oh[0][T], ol[0][T]);
+              split_product(v1, dv, oh[1][T], ol[1][T]);
+              split_product(v2, dv, oh[2][T], ol[2][T]);
+              split_product(v3, dv, oh[3][T], ol[3][T]);
+            } else {
+              oh[0][T] = hmul2(v0, dv);
+              oh[1][T] = hmul2(v1, dv);
+              oh[2][T] = hmul2(v2, dv);
+              oh[3][T] = hmul2(v3, dv);
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int row = 32 * (2 * vCl + ve) + 8 * k + vR;  // dimension - 128 * rank
+            sts128u(vt + swz(row, 2 * vG + vh), oh[k][0], oh[k][1], oh[k][2], oh[k][3]);
+            if constexpr (EXACT)
+              sts128u(vt + pf::kPart + swz(row, 2 * vG + vh), ol[k][0], ol[k][1], ol[k][2], ol[k][3]);
+          }
         }
         tc::fence_proxy_async_smem();
       }
@@ -854,32 +903,37 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_kernel(const PrefillP
   }
 }
 
-template <bool EXACT>
-static cudaError_t prepare_prefill_t() {
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<kKeyQ8, EXACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       pf::kSmemBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(prefill_kernel<kKeyQ4, EXACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             pf::kSmemBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(prefill_kernel<kKeyQ51, EXACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             pf::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(prefill_kernel<kKeyQ50, EXACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              pf::kSmemBytes);
+// The format pairs chunked prefill takes: Q8_0, Q4_0 and Q5_1 keys with Q4_0 or Q8_0 values,
+// Q5_0 keys with Q4_1 values.
+#define KVATTN_PREFILL_PAIRS(X)                                                                      \
+  X(kKeyQ8, kValQ4) X(kKeyQ4, kValQ4) X(kKeyQ51, kValQ4) X(kKeyQ50, kValQ41) X(kKeyQ8, kValQ8) \
+  X(kKeyQ4, kValQ8) X(kKeyQ51, kValQ8)
+
+bool prefill_pair_supported(int key_fmt, int val_fmt) {
+#define PF_PAIR_OK(KF, VF) if (key_fmt == KF && val_fmt == VF) return true;
+  KVATTN_PREFILL_PAIRS(PF_PAIR_OK)
+#undef PF_PAIR_OK
+  return false;
 }
 
 cudaError_t prepare_prefill_kernels() {
-  const cudaError_t e = prepare_prefill_t<true>();
-  return e != cudaSuccess ? e : prepare_prefill_t<false>();
+  cudaError_t e = cudaSuccess;
+#define PF_SET1(KF, VF, EX)                                                                          \
+  if (e == cudaSuccess)                                                                              \
+    e = cudaFuncSetAttribute(prefill_kernel<KF, VF, EX>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             pf::Layout<KF, VF>::kSmemBytes);
+#define PF_SET(KF, VF) PF_SET1(KF, VF, true) PF_SET1(KF, VF, false)
+  KVATTN_PREFILL_PAIRS(PF_SET)
+#undef PF_SET
+#undef PF_SET1
+  return e;
 }
 
-template <bool EXACT>
-static cudaError_t launch_prefill_grid(const cudaLaunchConfig_t& cfg, const PrefillParams& prm, int key_fmt) {
-  return key_fmt == kKeyQ4    ? cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ4, EXACT>, prm)
-         : key_fmt == kKeyQ51 ? cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ51, EXACT>, prm)
-         : key_fmt == kKeyQ50 ? cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ50, EXACT>, prm)
-                              : cudaLaunchKernelEx(&cfg, prefill_kernel<kKeyQ8, EXACT>, prm);
+template <int KF, int VF>
+static cudaError_t launch_prefill_grid(cudaLaunchConfig_t cfg, const PrefillParams& prm, bool exact) {
+  cfg.dynamicSmemBytes = pf::Layout<KF, VF>::kSmemBytes;
+  return exact ? cudaLaunchKernelEx(&cfg, prefill_kernel<KF, VF, true>, prm)
+               : cudaLaunchKernelEx(&cfg, prefill_kernel<KF, VF, false>, prm);
 }
 
 struct PrefillPlan {
@@ -910,14 +964,14 @@ PrefillPlan plan_prefill(int n_kv, int group, int n_q, int max_pages, int kv_spl
   return pl;
 }
 
-cudaError_t launch_prefill(const PrefillParams& prm0, int n_kv, int key_fmt, bool exact, cudaStream_t stream) {
+cudaError_t launch_prefill(const PrefillParams& prm0, int n_kv, int key_fmt, int val_fmt, bool exact,
+                           cudaStream_t stream) {
   PrefillParams prm = prm0;
   const int rows = prm.n_q * prm.group;
   {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(prm.rows_pad / pf::kRows, prm.n_ks, n_kv);
     cfg.blockDim = dim3(pf::kThreads);
-    cfg.dynamicSmemBytes = pf::kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -926,7 +980,11 @@ cudaError_t launch_prefill(const PrefillParams& prm0, int n_kv, int key_fmt, boo
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = exact ? launch_prefill_grid<true>(cfg, prm, key_fmt) : launch_prefill_grid<false>(cfg, prm, key_fmt);
+    cudaError_t e = cudaErrorInvalidValue;
+#define PF_LAUNCH(KF, VF) \
+  if (key_fmt == KF && val_fmt == VF) e = launch_prefill_grid<KF, VF>(cfg, prm, exact);
+    KVATTN_PREFILL_PAIRS(PF_LAUNCH)
+#undef PF_LAUNCH
     if (e != cudaSuccess || prm.n_ks == 1) return e;
   }
   cudaLaunchConfig_t cfg = {};

@@ -182,6 +182,8 @@ WORKLOADS = {
     "prefill524k_q50q41": Workload("prefill524k_q50q41", layers=16, kv_heads=4, q_heads=24, context=524288,
                                    n_q=2048, k_fmt="q5_0", v_fmt="q4_1", ubatch=512, kv_split_tokens=4096,
                                    seed=4007),
+    "prefill524k_q8q8": Workload("prefill524k_q8q8", layers=16, kv_heads=4, q_heads=24, context=524288,
+                                 n_q=2048, v_fmt="q8_0", ubatch=512, kv_split_tokens=4096, seed=4008),
     # 524,288 tokens in pinned host RAM, 256-block working set per (layer, head), 512 steps.
     "stream524k": Workload("stream524k", layers=16, kv_heads=4, q_heads=24, context=524288, n_q=1,
                            budget_blocks=256, recent_blocks=0, steps=512, seed=5005),

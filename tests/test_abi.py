@@ -90,14 +90,14 @@ def test_host_validation_rejects_bad_arguments(lib):
             kvattn.ERR_UNSUPPORTED_FORMAT, (kf, vf)
     bad = _desc(v_fmt="q5_1")
     assert L.kvattn_decode(by(bad), 16, 1, 16, 16, None, None, 1, 16, 16, None, 0, None) == kvattn.ERR_UNSUPPORTED_FORMAT
-    # Q4_0 / Q5_1 keys: decode and the summaries take them; chunked prefill takes Q8_0, Q4_0 or
-    # Q5_1 keys with Q4_0 values, and Q5_0 keys with Q4_1 values, and refuses the rest
+    # Q4_0 / Q5_1 keys: decode and the summaries take them; chunked prefill takes every format
+    # pair the descriptor accepts and refuses the rest
     for kf in ("q4_0", "q5_1"):
         kd = _desc(k_fmt=kf)
         assert L.kvattn_decode_workspace_size(by(kd), 1, 1024) == L.kvattn_decode_workspace_size(by(d), 1, 1024)
     for kf, vf, ok in (("q8_0", "q4_0", True), ("q4_0", "q4_0", True), ("q5_1", "q4_0", True),
-                       ("q5_0", "q4_1", True), ("q8_0", "q8_0", False), ("q5_1", "q8_0", False),
-                       ("q4_0", "q8_0", False)):
+                       ("q5_0", "q4_1", True), ("q8_0", "q8_0", True), ("q5_1", "q8_0", True),
+                       ("q4_0", "q8_0", True), ("q5_0", "q4_0", False), ("q8_0", "q4_1", False)):
         kd = _desc(k_fmt=kf, v_fmt=vf)
         st = L.kvattn_prefill_chunk(by(kd), 16, 1, 16, 16, None, None, 1, 4096, 16, 16, 16, 1 << 20, None)
         assert (st != kvattn.ERR_UNSUPPORTED_FORMAT) if ok else (st == kvattn.ERR_UNSUPPORTED_FORMAT), (kf, vf, st)

@@ -119,7 +119,7 @@ def test_verify_full_context(kv_gpu):
 
 @pytest.mark.parametrize("wname,f16", [("prefill524k", False), ("prefill524k_q4q4", False),
                                        ("prefill524k_q51q4", False), ("prefill524k_q50q41", False),
-                                       ("prefill524k", True)])
+                                       ("prefill524k_q8q8", False), ("prefill524k", True)])
 def test_prefill_full_context_sampled_rows(kv_gpu, wname, f16):
     """One layer of the 524,288-key prefill as the bench runs it (the f16 case through
     kvattn_prefill_chunk_f16): 64 sampled rows of two KV heads against the oracle."""

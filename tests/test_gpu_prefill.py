@@ -48,7 +48,8 @@ def _case(seed, H, n_prior, n_q, outliers=True, k_fmt="q8_0", v_fmt="q4_0"):
     return rng, k, v, q, cache, T
 
 
-PAIRS = [("q8_0", "q4_0"), ("q4_0", "q4_0"), ("q5_1", "q4_0"), ("q5_0", "q4_1")]
+PAIRS = [("q8_0", "q4_0"), ("q4_0", "q4_0"), ("q5_1", "q4_0"), ("q5_0", "q4_1"), ("q8_0", "q8_0"), ("q4_0", "q8_0"),
+         ("q5_1", "q8_0")]
 
 
 @pytest.mark.parametrize("k_fmt,v_fmt", PAIRS)
