@@ -1,9 +1,9 @@
-// Chunked prefill over block-quantized KV pages (Q8_0, Q4_0 or Q5_1 keys with Q4_0 values, Q5_0
-// keys with Q4_1 values) on tcgen05 tensor cores (Adaptive KV Streaming + RDNA 4 announcement,
-// wqu.guru, method list:
-// "online log-sum-exp prefill": the prefill of a chunk is computed across streamed KV pages
-// and the partial results are accumulated by online log-sum-exp; the six-step validation
-// guide, alphalab.site, build step: the q8_0-q4_0 and q4_0-q4_0 flash-attention KV pairs;
+// Chunked prefill over block-quantized KV pages (Q8_0, Q4_0 or Q5_1 keys with Q4_0 or Q8_0
+// values, Q5_0 keys with Q4_1 values) on tcgen05 tensor cores (Adaptive KV Streaming + RDNA 4
+// announcement, wqu.guru, method list: "online log-sum-exp prefill": the prefill of a chunk is
+// computed across streamed KV pages and the partial results are accumulated by online
+// log-sum-exp; the six-step validation guide, alphalab.site, build step: the q8_0-q4_0 and
+// q4_0-q4_0 flash-attention KV pairs;
 // Vulkan speculative-decoding report, lcz.me/topic/1398, pitfalls: the K q5_1 / V q4_0 cache;
 // 7900 XTX MTP tuning notes, lcz.me/topic/593: a q5_0 / q4_1 cache).
 //
@@ -19,9 +19,10 @@
 //                         into a two-stage shared-memory ring
 //   dequant warps (8)     raw -> K^ and V^T, each as an f16 high part (code x scale rounded
 //                         once) and an f16 low part (the remainder, exact): together the
-//                         dequantized values exactly (Q5_1 keys, code x scale + minimum:
-//                         to the one fp32 rounding of the sum); K-major, 128-byte swizzle,
-//                         three deep
+//                         dequantized values exactly (Q5_1 keys and Q4_1 values, code x
+//                         scale + minimum: to the one fp32 rounding of the sum); K-major,
+//                         128-byte swizzle,
+//                         three deep (two with Q8_0 values)
 //   MMA issuer (1 warp,   S = Q K^T (N = 64 keys, K = 256) as Q K^_hi^T + Q K^_lo^T, and
 //     even CTA only)      O += P V (N = 256 dims, K = 64 keys) as P_hi V^_hi + P_lo V^_hi +
 //                         P_hi V^_lo; Q and P from tensor memory
@@ -33,7 +34,8 @@
 // Q (bf16) is stored as Q/16 in f16, which is exact; log2(e) is applied in fp32 to S.  Every
 // operand therefore carries the dequantized values to about 22 significant bits and the
 // products accumulate in fp32.  The CTA writes a normalised partial (o, lse) per row; a
-// second grid merges the splits.
+// second grid merges the splits.  With EXACT false (kvattn_prefill_chunk_f16) every operand is
+// rounded once to f16 instead, and QK and PV take one MMA pass each.
 #include "decode.cuh"
 #include "tcgen05.cuh"
 
