@@ -84,6 +84,8 @@ __global__ void __launch_bounds__(256) block_summary_kernel(const uint8_t* __res
 }
 
 // ---------------------------------------------------------------- scores
+// One warp per block.  The CTA first sums the group's query rows per channel (fp64, over the
+// rows in order) into shared memory; lane l then takes channels 4l..4l+3 and 128 + 4l..4l+3.
 __global__ void __launch_bounds__(256) block_score_kernel(const float* __restrict__ summaries,
                                                           const float* __restrict__ q_group, int group, int n_blocks,
                                                           int n_cand, double* __restrict__ scores) {
@@ -91,26 +93,29 @@ __global__ void __launch_bounds__(256) block_score_kernel(const float* __restric
   // now, and this grid reads the retrieval queries only once the kernel before it completed
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ double u_s[kHeadDim];
   const int unit = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* qg = q_group + static_cast<long long>(unit) * group * kHeadDim;
+  {
+    const int c = threadIdx.x;  // blockDim.x == kHeadDim
+    double u = 0.0;
+    for (int j = 0; j < group; ++j) u += qg[j * kHeadDim + c];
+    u_s[c] = u;
+  }
+  __syncthreads();
   const int b = blockIdx.x * (blockDim.x >> 5) + warp;
   if (b >= n_cand) return;
-  const float* qg = q_group + static_cast<long long>(unit) * group * kHeadDim;
   const float* sm = summaries + (static_cast<long long>(unit) * n_blocks + b) * kHeadDim;
   double acc = 0.0;
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const int c0 = lane * 4 + 128 * k;
     const float4 sv = *reinterpret_cast<const float4*>(sm + c0);
-    double u[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int j = 0; j < group; ++j) {
-      const float4 qv = *reinterpret_cast<const float4*>(qg + j * kHeadDim + c0);
-      u[0] += qv.x; u[1] += qv.y; u[2] += qv.z; u[3] += qv.w;
-    }
-    acc = fma(u[0], static_cast<double>(sv.x), acc);
-    acc = fma(u[1], static_cast<double>(sv.y), acc);
-    acc = fma(u[2], static_cast<double>(sv.z), acc);
-    acc = fma(u[3], static_cast<double>(sv.w), acc);
+    acc = fma(u_s[c0], static_cast<double>(sv.x), acc);
+    acc = fma(u_s[c0 + 1], static_cast<double>(sv.y), acc);
+    acc = fma(u_s[c0 + 2], static_cast<double>(sv.z), acc);
+    acc = fma(u_s[c0 + 3], static_cast<double>(sv.w), acc);
   }
 #pragma unroll
   for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
