@@ -19,6 +19,7 @@ cudaError_t launch_resident_update(const int32_t*, const int32_t*, int, int, int
                                    const int32_t*, int64_t, const int32_t*, int32_t*, int32_t*, int32_t*, int32_t*,
                                    cudaStream_t);
 cudaError_t prepare_prefill_kernels();
+bool prefill_pair_supported(int key_fmt, int val_fmt);
 struct PrefillParams;
 cudaError_t launch_merge_lse(const float*, const float*, int, int, int, float*, float*, int, cudaStream_t);
 cudaError_t launch_block_summaries(const kvattn_kv_desc&, const int32_t*, int, int, int, int, float*, cudaStream_t);
