@@ -79,14 +79,19 @@ struct DecodeCfg {
   // the query B fragments: [block][k-step][n-tile][lane][hi0, hi1, lo0, lo1]
   static constexpr int kQBytes = 8 * 2 * NT * 32 * 16;
   static constexpr int kRowsPad = NT * 8;
-  // as many page stages as fit beside the query fragments and the barriers (at most 6)
-  static constexpr int kStagesFit = (227 * 1024 - 256 - kQBytes) / kStageBytes;
-  static constexpr int kStages = kStagesFit < 6 ? kStagesFit : 6;
-  static constexpr int kRingBytes = kStages * kStageBytes;
   // rows of the output merge buffer are padded by 4 floats: the four lanes of an MMA quad
   // store rows 2t, 2t+1 of the same dims and then fall into different banks
   static constexpr int kOStride = kHeadDim + 4;
   static constexpr int kMergeBytes = kConsumerWarps * 8 * (kOStride + 2) * 4;  // 8 rows per warp
+  // Page stages: for 8 and 16 rows as many as fit beside the query fragments and the barriers
+  // (at most 6).  The 24-row shape is bound by arithmetic, not by the page stream: it takes
+  // the fewest stages that hold the merge buffer (at least 2), which measured faster (a
+  // smaller shared-memory footprint leaves more of the SM's memory to L1).
+  static constexpr int kStagesFit = (227 * 1024 - 256 - kQBytes) / kStageBytes;
+  static constexpr int kStagesMin = (kMergeBytes + kStageBytes - 1) / kStageBytes < 2
+                                        ? 2 : (kMergeBytes + kStageBytes - 1) / kStageBytes;
+  static constexpr int kStages = NT == 3 ? kStagesMin : (kStagesFit < 6 ? kStagesFit : 6);
+  static constexpr int kRingBytes = kStages * kStageBytes;
   static_assert(kMergeBytes <= kRingBytes, "merge buffer must fit in the ring");
   static constexpr int kQOffset = kRingBytes;
   static constexpr int kBarOffset = kQOffset + kQBytes;
