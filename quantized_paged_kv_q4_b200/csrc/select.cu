@@ -175,37 +175,52 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const double* 
                                                                  int32_t* __restrict__ sel_phys,
                                                                  int32_t* __restrict__ n_sel, int cap) {
   extern __shared__ __align__(16) uint8_t sm[];
-  __shared__ int hist[256];
+  // two digit histograms: pass p counts into hist[p % 2] while the other is cleared for the
+  // next pass, so a pass needs two CTA barriers; sel[p % 2] holds pass p's result
+  __shared__ int hist[2][256];
+  __shared__ int sel[2][3];  // digit, keys still needed inside its bin, keys in its bin
   __shared__ int warp_tot[kSelThreads / 32];
-  __shared__ int s_total, s_digit, s_need, s_bin;
+  __shared__ int s_total;
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the decode may set up
-  asm volatile("griddepcontrol.wait;" ::: "memory");               // the scores are complete
+  for (int b = threadIdx.x; b < 2 * 256; b += kSelThreads) (&hist[0][0])[b] = 0;
+  __syncthreads();
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the scores are complete
   const int unit = blockIdx.x;
   unsigned long long* key = reinterpret_cast<unsigned long long*>(sm);           // [n_cand]
   uint32_t* bits = reinterpret_cast<uint32_t*>(key + (n_cand > 0 ? n_cand : 1));  // [n_total / 32]
   const double* sc = scores + static_cast<long long>(unit) * n_blocks;
-  for (int i = threadIdx.x; i < n_cand; i += kSelThreads) key[i] = order_key(sc[i]);
   const int take = min(budget, n_cand);
+  const bool selecting = take > 0 && take < n_cand;
+  // the keys, with the first pass's histogram (most significant digit) counted on the way
+  for (int i = threadIdx.x; i < n_cand; i += kSelThreads) {
+    const unsigned long long k = order_key(sc[i]);
+    key[i] = k;
+    if (selecting) atomicAdd(&hist[0][static_cast<int>(k >> 56)], 1);
+  }
   unsigned long long prefix = 0ull, mask = 0ull;
   int need = take;  // how many still to take among keys matching prefix under mask
   __syncthreads();
-  if (take > 0 && take < n_cand) {
-    for (int shift = 56; shift >= 0; shift -= 8) {
-      for (int b = threadIdx.x; b < 256; b += kSelThreads) hist[b] = 0;
-      __syncthreads();
-      for (int i = threadIdx.x; i < n_cand; i += kSelThreads) {
-        const unsigned long long k = key[i];
-        if ((k & mask) == prefix) atomicAdd(&hist[static_cast<int>((k >> shift) & 255ull)], 1);
+  if (selecting) {
+    for (int shift = 56, pass = 0; shift >= 0; shift -= 8, ++pass) {
+      int* h = hist[pass & 1];
+      if (pass > 0) {
+        for (int i = threadIdx.x; i < n_cand; i += kSelThreads) {
+          const unsigned long long k = key[i];
+          if ((k & mask) == prefix) atomicAdd(&h[static_cast<int>((k >> shift) & 255ull)], 1);
+        }
+        __syncthreads();
       }
-      __syncthreads();
-      if (threadIdx.x < 32) {
+      if (threadIdx.x >= 32) {
+        // the other histogram was last read by the previous pass's scan, before its barrier
+        for (int b = threadIdx.x - 32; b < 256; b += kSelThreads - 32) hist[(pass + 1) & 1][b] = 0;
+      } else {
         // lane l owns bins 255 - 8l - e (e = 0..7), highest first; find the digit whose bin
         // holds the need-th largest remaining key
         const int lane = threadIdx.x;
         int c[8], sum = 0;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          c[e] = hist[255 - 8 * lane - e];
+          c[e] = h[255 - 8 * lane - e];
           sum += c[e];
         }
         int incl = sum;
@@ -219,21 +234,21 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const double* 
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             if (before < need && need <= before + c[e]) {
-              s_digit = 255 - 8 * lane - e;
-              s_need = need - before;
-              s_bin = c[e];
+              sel[pass & 1][0] = 255 - 8 * lane - e;
+              sel[pass & 1][1] = need - before;
+              sel[pass & 1][2] = c[e];
             }
             before += c[e];
           }
         }
       }
       __syncthreads();
-      prefix |= static_cast<unsigned long long>(s_digit) << shift;
+      // sel[pass % 2] is written again two passes on, after a barrier every thread passes
+      // only once it has read it here
+      prefix |= static_cast<unsigned long long>(sel[pass & 1][0]) << shift;
       mask |= 255ull << shift;
-      need = s_need;
-      const bool whole_bin = s_bin == s_need;
-      __syncthreads();
-      if (whole_bin) break;
+      need = sel[pass & 1][1];
+      if (sel[pass & 1][2] == need) break;
     }
   }
   // mark: keys above the threshold, and the first `need` keys equal to it in index order
