@@ -130,7 +130,6 @@ __device__ __forceinline__ unsigned long long order_key(double x) {
 
 constexpr int kSelThreads = 1024;
 constexpr int kMaxCand = 16384;
-constexpr int kMaxTotal = 65536;
 
 // Exclusive prefix sum of one int per thread over the CTA (kSelThreads threads); `warp_tot`
 // is shared scratch of kSelThreads / 32 ints.  Returns this thread's exclusive prefix and
@@ -161,6 +160,44 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* t
   return r;
 }
 
+// Exclusive prefix sums of two ints per thread over the CTA (kSelThreads threads), in one
+// pass; `warp_tot` is shared scratch of kSelThreads / 32 pairs, read again by no caller.
+// Returns this thread's exclusive prefixes and writes the CTA totals to *total (shared).
+__device__ __forceinline__ int2 block_exclusive_scan2(int a, int b, int2* warp_tot, int2* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = a, y = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int xo = __shfl_up_sync(0xffffffffu, x, o), yo = __shfl_up_sync(0xffffffffu, y, o);
+    if (lane >= o) {
+      x += xo;
+      y += yo;
+    }
+  }
+  if (lane == 31) warp_tot[warp] = make_int2(x, y);
+  __syncthreads();
+  if (warp == 0) {
+    int2 t = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int xo = __shfl_up_sync(0xffffffffu, t.x, o), yo = __shfl_up_sync(0xffffffffu, t.y, o);
+      if (lane >= o) {
+        t.x += xo;
+        t.y += yo;
+      }
+    }
+    warp_tot[lane] = t;  // inclusive over warps
+    if (lane == 31) *total = t;
+  }
+  __syncthreads();
+  int2 r = make_int2(x - a, y - b);
+  if (warp > 0) {
+    r.x += warp_tot[warp - 1].x;
+    r.y += warp_tot[warp - 1].y;
+  }
+  return r;
+}
+
 // Top-`budget` candidates by (score desc, block index asc), plus the recent window and the
 // tail, compacted into ascending logical ids.  The `take`-th largest 64-bit order key is found
 // by an 8-bit radix select, most significant digit first; candidates above it are taken, and
@@ -179,15 +216,14 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const double* 
   // next pass, so a pass needs two CTA barriers; sel[p % 2] holds pass p's result
   __shared__ int hist[2][256];
   __shared__ int sel[2][3];  // digit, keys still needed inside its bin, keys in its bin
-  __shared__ int warp_tot[kSelThreads / 32];
-  __shared__ int s_total;
+  __shared__ int2 warp_tot2[kSelThreads / 32];
+  __shared__ int2 s_tot2;  // CTA totals of (equal keys, surely taken)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the decode may set up
   for (int b = threadIdx.x; b < 2 * 256; b += kSelThreads) (&hist[0][0])[b] = 0;
   __syncthreads();
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the scores are complete
   const int unit = blockIdx.x;
-  unsigned long long* key = reinterpret_cast<unsigned long long*>(sm);           // [n_cand]
-  uint32_t* bits = reinterpret_cast<uint32_t*>(key + (n_cand > 0 ? n_cand : 1));  // [n_total / 32]
+  unsigned long long* key = reinterpret_cast<unsigned long long*>(sm);  // [n_cand]
   const double* sc = scores + static_cast<long long>(unit) * n_blocks;
   const int take = min(budget, n_cand);
   const bool selecting = take > 0 && take < n_cand;
@@ -251,67 +287,60 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const double* 
       if (sel[pass & 1][2] == need) break;
     }
   }
-  // mark: keys above the threshold, and the first `need` keys equal to it in index order
-  // (contiguous index ranges per thread, ranks of equal keys by a block scan)
-  const int words = (n_total + 31) / 32;
-  for (int w = threadIdx.x; w < words; w += kSelThreads) bits[w] = 0u;
-  __syncthreads();
-  {
-    const int per = (n_cand + kSelThreads - 1) / kSelThreads;
-    const int i0 = min(n_cand, threadIdx.x * per), i1 = min(n_cand, i0 + per);
-    int eq = 0;
-    if (take > 0 && take < n_cand)
-      for (int i = i0; i < i1; ++i) eq += (key[i] & mask) == prefix;
-    int rank = block_exclusive_scan(eq, warp_tot, &s_total);
-    for (int i = i0; i < i1; ++i) {
+  // Selection and compaction in one pass over contiguous ranges of all n_total block
+  // indices, in ascending order.  A candidate is taken when its key is above the threshold,
+  // or equal to it and among the first `need` equal keys in index order; the blocks past the
+  // candidates (the recent window and the tail) always are.  One CTA scan of (equal keys,
+  // surely taken) per thread gives the thread both the rank of its first equal key and its
+  // output position: the surely taken blocks before it plus the min(need, equal keys before
+  // it) equal ones taken among them.
+  const bool take_all = take >= n_cand;
+  const int per = (n_total + kSelThreads - 1) / kSelThreads;
+  const int i0 = min(n_total, threadIdx.x * per), i1 = min(n_total, i0 + per);
+  int eq = 0, sure = 0;
+  for (int i = i0; i < i1; ++i) {
+    if (i >= n_cand || take_all) {
+      ++sure;
+    } else if (selecting) {
+      const unsigned long long k = key[i] & mask;
+      sure += k > prefix;
+      eq += k == prefix;
+    }
+  }
+  const int2 before = block_exclusive_scan2(eq, sure, warp_tot2, &s_tot2);
+  const int32_t* pt = page_table + static_cast<long long>(unit) * n_blocks;
+  int32_t* out_l = sel_logical + static_cast<long long>(unit) * cap;
+  int32_t* out_p = sel_phys + static_cast<long long>(unit) * cap;
+  int rank = before.x;
+  int pos = before.y + max(0, min(need, before.x));
+  constexpr int kChunk = 4;  // page ids loaded up front, all independent
+  for (int c0 = i0; c0 < i1; c0 += kChunk) {
+    int32_t pg[kChunk];
+#pragma unroll
+    for (int e = 0; e < kChunk; ++e) pg[e] = c0 + e < i1 ? pt[c0 + e] : 0;
+#pragma unroll
+    for (int e = 0; e < kChunk; ++e) {
+      const int i = c0 + e;
+      if (i >= i1) break;
       bool sel;
-      if (take >= n_cand) {
+      if (i >= n_cand || take_all) {
         sel = true;
-      } else if (take <= 0) {
+      } else if (!selecting) {
         sel = false;
       } else {
         const unsigned long long k = key[i] & mask;
         sel = k > prefix || (k == prefix && rank++ < need);
       }
-      if (sel) atomicOr(&bits[i >> 5], 1u << (i & 31));
-    }
-  }
-  for (int b = n_cand + threadIdx.x; b < n_total; b += kSelThreads) atomicOr(&bits[b >> 5], 1u << (b & 31));
-  __syncthreads();
-  // compaction into ascending ids: each thread takes a contiguous range of at most kCompact
-  // block indices (their page ids are loaded up front, all independent), counts its selected
-  // ones, and writes them at the position an exclusive scan of the counts gives
-  constexpr int kCompact = 4;
-  const int32_t* pt = page_table + static_cast<long long>(unit) * n_blocks;
-  int32_t* out_l = sel_logical + static_cast<long long>(unit) * cap;
-  int32_t* out_p = sel_phys + static_cast<long long>(unit) * cap;
-  int run = 0;  // selected blocks in the ranges before this pass
-  for (int base = 0; base < n_total; base += kSelThreads * kCompact) {
-    const int i0 = base + threadIdx.x * kCompact;
-    int32_t pg[kCompact];
-    bool on[kCompact];
-    int cnt = 0;
-#pragma unroll
-    for (int e = 0; e < kCompact; ++e) {
-      const int b = i0 + e;
-      on[e] = b < n_total && ((bits[b >> 5] >> (b & 31)) & 1u);
-      pg[e] = on[e] ? pt[b] : 0;
-      cnt += on[e];
-    }
-    int pos = run + block_exclusive_scan(cnt, warp_tot, &s_total);
-    run += s_total;
-#pragma unroll
-    for (int e = 0; e < kCompact; ++e) {
-      if (on[e]) {
+      if (sel) {
         if (pos < cap) {
-          out_l[pos] = i0 + e;
+          out_l[pos] = i;
           out_p[pos] = pg[e];
         }
         ++pos;
       }
     }
   }
-  if (threadIdx.x == 0) n_sel[unit] = min(run, cap);
+  if (threadIdx.x == 0) n_sel[unit] = min(s_tot2.y + max(0, min(need, s_tot2.x)), cap);
 }
 
 cudaError_t launch_block_summaries(const kvattn_kv_desc& d, const int32_t* page_table, int n_units, int n_blocks,
@@ -326,13 +355,11 @@ cudaError_t launch_block_summaries(const kvattn_kv_desc& d, const int32_t* page_
   return cudaGetLastError();
 }
 
-size_t select_smem_bytes(int n_cand, int n_total) {
-  return static_cast<size_t>(n_cand > 0 ? n_cand : 1) * 8 + static_cast<size_t>((n_total + 31) / 32) * 4;
-}
+size_t select_smem_bytes(int n_cand) { return static_cast<size_t>(n_cand > 0 ? n_cand : 1) * 8; }
 
 cudaError_t prepare_select_kernels() {
   return cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(select_smem_bytes(kMaxCand, kMaxTotal)));
+                              static_cast<int>(select_smem_bytes(kMaxCand)));
 }
 
 cudaError_t launch_select(const float* summaries, const float* q_group, int n_units, int group, int n_blocks,
@@ -356,7 +383,7 @@ cudaError_t launch_select(const float* summaries, const float* q_group, int n_un
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(n_units);
   cfg.blockDim = dim3(kSelThreads);
-  cfg.dynamicSmemBytes = select_smem_bytes(max(n_cand, 1), n_total);
+  cfg.dynamicSmemBytes = select_smem_bytes(max(n_cand, 1));
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
